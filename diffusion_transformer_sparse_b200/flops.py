@@ -1,0 +1,46 @@
+"""Algorithmic FLOP and byte counts of the PT-DiT attention path.
+
+A multiply-add is 2 FLOP.  Attention cores count every score of every window
+(the shift mask removes no work).  Per batch item, with N tokens, M proxies,
+n tokens per TCM window and width D:
+
+  proxy SA     projections 8 M D^2        core 4 M^2 D
+  cross-attn   projections 4 N D^2 + 4 M D^2   core 4 N M D
+  WSA, SWSA    projections 8 N D^2 each   core 4 N n D each
+
+Full global self-attention over the same tokens costs 8 N D^2 + 4 N^2 D.  The
+core ratio M^2/N^2 + M/N + 2n/N is the complexity paragraph of the Qihoo-T2X
+reading note (§3 Method, "2.3% of full attention at 2048^2").
+"""
+from __future__ import annotations
+
+
+def block_flops(N: int, M: int, n: int, D: int) -> dict:
+    f = {
+        "psa_proj": 8 * M * D * D,
+        "psa_core": 4 * M * M * D,
+        "cross_proj": 4 * N * D * D + 4 * M * D * D,
+        "cross_core": 4 * N * M * D,
+        "wsa_proj": 8 * N * D * D,
+        "wsa_core": 4 * N * n * D,
+        "swsa_proj": 8 * N * D * D,
+        "swsa_core": 4 * N * n * D,
+    }
+    f["proj"] = f["psa_proj"] + f["cross_proj"] + f["wsa_proj"] + f["swsa_proj"]
+    f["core"] = f["psa_core"] + f["cross_core"] + f["wsa_core"] + f["swsa_core"]
+    f["total"] = f["proj"] + f["core"]
+    return f
+
+
+def dense_flops(N: int, D: int) -> dict:
+    return {"proj": 8 * N * D * D, "core": 4 * N * N * D, "total": 8 * N * D * D + 4 * N * N * D}
+
+
+def core_ratio(N: int, M: int, n: int) -> float:
+    """Cost of the GIIM + TCM attention cores relative to global attention (2 N^2 D)."""
+    return (M / N) ** 2 + M / N + 2 * n / N
+
+
+def average_bytes(N: int, M: int, D: int, elem: int) -> int:
+    """Window averaging: read every token once, write every proxy once."""
+    return (N + M) * D * elem

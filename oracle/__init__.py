@@ -1,0 +1,12 @@
+"""Float64 CPU oracle of the PT-DiT block-attention path.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by ``__graft_entry__.smoke()``
+and by the bench's CPU-baseline / reference leg, never by the product path.
+"""
+from .ptdit_oracle import *  # noqa: F401,F403
+from .ptdit_oracle import (  # noqa: F401
+    attention_heads, averaging, block_attn, block_attn_rows, giim, masked_self_attention,
+    multihead_attention, num_tokens, project, proxy_index, proxy_self_attention, softmax_rows,
+    tcm, token_coords, window_allow_matrix, window_region_labels, window_self_attention,
+    window_token_map,
+)

@@ -1,0 +1,402 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Each test ties one oracle function to what the pages and the mathematics fix:
+hand-derived index maps (tests/golden), torch's own multi-head attention as a
+library routine, closed forms of degenerate cases, brute force with scalar
+loops, invariants, and the pages' printed 2.3% complexity figure.  The last
+group plants plausible mistakes in the oracle and checks that a pin catches
+each one.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from diffusion_transformer_sparse_b200 import flops
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as fh:
+        return json.load(fh)
+
+
+def _weights(D, seed, k=4, scale=None):
+    rng = np.random.default_rng(seed)
+    a = math.sqrt(6.0 / (2 * D)) if scale is None else scale
+    return tuple(rng.uniform(-a, a, (D, D)) for _ in range(k))
+
+
+def torch_mha(xq, xkv, W, heads, allow=None):
+    """torch.nn.MultiheadAttention (bias-free, float64) as an independent library routine."""
+    D = xq.shape[1]
+    mha = torch.nn.MultiheadAttention(D, heads, bias=False, batch_first=True, dtype=torch.float64)
+    with torch.no_grad():
+        mha.in_proj_weight.copy_(torch.from_numpy(np.concatenate(W[:3], axis=0)))
+        mha.out_proj.weight.copy_(torch.from_numpy(W[3]))
+        mask = None if allow is None else torch.from_numpy(~allow)
+        q = torch.from_numpy(np.ascontiguousarray(xq))[None]
+        kv = torch.from_numpy(np.ascontiguousarray(xkv))[None]
+        out, _ = mha(q, kv, kv, attn_mask=mask, need_weights=False)
+    return out[0].numpy()
+
+
+def _close(a, b, tol=1e-10):
+    a, b = np.asarray(a), np.asarray(b)
+    assert a.shape == b.shape
+    assert np.all(np.isfinite(a)) and np.all(np.isfinite(b))
+    err = np.max(np.abs(a - b)) / max(1e-300, np.max(np.abs(b)))
+    assert err <= tol, f"max rel err {err:.3e} > {tol:.1e}"
+
+
+def _divisors(L):
+    return [p for p in range(1, L + 1) if L % p == 0]
+
+
+# ---------------------------------------------------------------- P1 averaging
+
+def test_proxy_index_golden():
+    for name in ("proxy_map_1x4x4_r122.json", "proxy_map_2x2x4_r212.json"):
+        g = _golden(name)
+        got = O.proxy_index(tuple(g["grid"]), tuple(g["ratio"]))
+        np.testing.assert_array_equal(got, np.array(g["proxy_of_token"]))
+
+
+@pytest.mark.parametrize("grid", [(1, 4, 4), (2, 4, 6), (4, 8, 8), (3, 6, 4)])
+def test_averaging_bruteforce(grid):
+    f, h, w = grid
+    rng = np.random.default_rng(7)
+    z = rng.standard_normal((f * h * w, 5))
+    for ratio in itertools.product(_divisors(f), _divisors(h), _divisors(w)):
+        pf, ph, pw = ratio
+        got = O.averaging(z, grid, ratio)
+        # scalar loops over each window, written from the definition
+        want = []
+        for T in range(f // pf):
+            for Y in range(h // ph):
+                for X in range(w // pw):
+                    acc = np.zeros(5)
+                    cnt = 0
+                    for t in range(T * pf, T * pf + pf):
+                        for y in range(Y * ph, Y * ph + ph):
+                            for x in range(X * pw, X * pw + pw):
+                                acc += z[(t * h + y) * w + x]
+                                cnt += 1
+                    want.append(acc / cnt)
+        _close(got, np.array(want), 1e-14)
+        # the index map groups the same tokens
+        idx = O.proxy_index(grid, ratio)
+        for m in range(got.shape[0]):
+            _close(got[m], z[idx == m].mean(axis=0), 1e-14)
+
+
+def test_averaging_rejects_non_divisible():
+    with pytest.raises(ValueError):
+        O.averaging(np.zeros((24, 2)), (1, 4, 6), (1, 4, 4))
+
+
+# ---------------------------------------------------------------- maps and masks
+
+def test_window_map_golden():
+    g = _golden("shifted_windows_1x4x4_w122_s011.json")
+    grid, window, shift = tuple(g["grid"]), tuple(g["window"]), tuple(g["shift"])
+    tok = O.window_token_map(grid, window, shift)
+    np.testing.assert_array_equal(tok, np.array(g["token_at_window_slot"]))
+    lab = O.window_region_labels(grid, window, shift)
+    for k, groups in enumerate(g["allowed_groups"]):
+        want = np.zeros((4, 4), bool)
+        for grp in groups:
+            for i in grp:
+                for j in grp:
+                    want[i, j] = True
+        np.testing.assert_array_equal(lab[k][:, None] == lab[k][None, :], want)
+
+
+@pytest.mark.parametrize("grid", [(1, 8, 8), (2, 4, 8), (4, 4, 4)])
+def test_window_maps_partition_and_match_pair_mask(grid):
+    N = O.num_tokens(grid)
+    full = O.window_allow_matrix
+    for window in itertools.product(*[_divisors(L) for L in grid]):
+        for shift in itertools.product(*[range(wd) for wd in window]):
+            tok = O.window_token_map(grid, window, shift)
+            assert sorted(tok.ravel().tolist()) == list(range(N))
+            lab = O.window_region_labels(grid, window, shift)
+            allow = np.zeros((N, N), bool)
+            for k in range(tok.shape[0]):
+                same = lab[k][:, None] == lab[k][None, :]
+                allow[np.ix_(tok[k], tok[k])] = same
+            np.testing.assert_array_equal(allow, full(grid, window, shift))
+
+
+# ---------------------------------------------------------------- P2 / cross-attn vs library
+
+def test_ratio_111_proxy_sa_is_full_self_attention():
+    grid, D, heads = (2, 4, 4), 8, 2
+    z = np.random.default_rng(1).standard_normal((32, D))
+    W = _weights(D, 2)
+    got = O.proxy_self_attention(z, grid, (1, 1, 1), W, heads)
+    _close(got, torch_mha(z, z, W, heads))
+
+
+@pytest.mark.parametrize("ratio", [(1, 2, 2), (2, 2, 1), (1, 4, 4)])
+def test_giim_matches_library_mha(ratio):
+    grid, D, heads = (2, 4, 8), 12, 3
+    z = np.random.default_rng(3).standard_normal((64, D))
+    Wp, Wc = _weights(D, 4), _weights(D, 5)
+    Pa = O.averaging(z, grid, ratio)
+    Pp = torch_mha(Pa, Pa, Wp, heads)
+    _close(O.giim(z, grid, ratio, Wp, Wc, heads, residual=False), torch_mha(z, Pp, Wc, heads))
+    _close(O.giim(z, grid, ratio, Wp, Wc, heads), z + torch_mha(z, Pp, Wc, heads))
+    _close(O.giim(z, grid, ratio, Wp, Wc, heads, proxy_residual=True, residual=False),
+           torch_mha(z, Pp + Pa, Wc, heads))
+
+
+# ---------------------------------------------------------------- P3 single window
+
+def test_single_window_broadcasts_one_vector():
+    grid, D, heads = (2, 4, 4), 8, 2
+    z = np.random.default_rng(5).standard_normal((32, D))
+    Wp, Wc = _weights(D, 6), _weights(D, 7)
+    out = O.giim(z, grid, grid, Wp, Wc, heads, residual=False)
+    Pa = z.mean(axis=0)
+    # softmax over a single key is 1: SA(P_a) = Wo Wv P_a and CS(z, P') = Wo Wv P'
+    Pp = Wp[3] @ (Wp[2] @ Pa)
+    want = Wc[3] @ (Wc[2] @ Pp)
+    for row in out:
+        _close(row, want, 1e-12)
+
+
+# ---------------------------------------------------------------- P4 special cases
+
+def test_window_equal_grid_is_full_self_attention():
+    grid, D, heads = (2, 4, 4), 8, 2
+    z = np.random.default_rng(8).standard_normal((32, D))
+    W = _weights(D, 9)
+    _close(O.window_self_attention(z, grid, grid, (0, 0, 0), W, heads), z + torch_mha(z, z, W, heads))
+
+
+def test_shift_zero_is_plain_window_attention():
+    grid, window, D, heads = (2, 4, 8), (2, 2, 4), 8, 2
+    z = np.random.default_rng(10).standard_normal((64, D))
+    W = _weights(D, 11)
+    got = O.window_self_attention(z, grid, window, (0, 0, 0), W, heads, residual=False)
+    assert np.all(O.window_region_labels(grid, window, (0, 0, 0)) == 0)
+    # each non-overlapping window attended on its own with the library routine
+    f, h, w = grid
+    for T, Y, X in itertools.product(range(0, f, 2), range(0, h, 2), range(0, w, 4)):
+        toks = [(t * h + y) * w + x for t in range(T, T + 2) for y in range(Y, Y + 2)
+                for x in range(X, X + 4)]
+        _close(got[toks], torch_mha(z[toks], z[toks], W, heads))
+
+
+# ---------------------------------------------------------------- P5, P7 two formulations
+
+@pytest.mark.parametrize("grid,window", [((1, 8, 8), (1, 4, 4)), ((4, 4, 8), (2, 2, 4)),
+                                         ((2, 6, 6), (2, 2, 2))])
+def test_half_shift_direction_does_not_matter(grid, window):
+    D, heads = 8, 2
+    shift = tuple(wd // 2 for wd in window)
+    z = np.random.default_rng(12).standard_normal((O.num_tokens(grid), D))
+    W = _weights(D, 13)
+    a = O.masked_self_attention(z, W, heads, O.window_allow_matrix(grid, window, shift))
+    b = O.masked_self_attention(z, W, heads,
+                                O.window_allow_matrix(grid, window, tuple(-s for s in shift)))
+    _close(a, b, 1e-13)
+    _close(O.window_self_attention(z, grid, window, shift, W, heads), a, 1e-12)
+
+
+@pytest.mark.parametrize("grid", [(1, 4, 8), (2, 4, 4)])
+def test_roll_formulation_matches_pair_mask_and_library(grid):
+    D, heads = 6, 2
+    z = np.random.default_rng(14).standard_normal((O.num_tokens(grid), D))
+    W = _weights(D, 15)
+    for window in itertools.product(*[[p for p in _divisors(L) if p > 1 or L == 1] for L in grid]):
+        for shift in itertools.product(*[range(wd) for wd in window]):
+            allow = O.window_allow_matrix(grid, window, shift)
+            got = O.window_self_attention(z, grid, window, shift, W, heads)
+            _close(got, O.masked_self_attention(z, W, heads, allow), 1e-12)
+            _close(got, z + torch_mha(z, z, W, heads, allow), 1e-10)
+
+
+# ---------------------------------------------------------------- P6 invariants
+
+def test_giim_permutation_equivariance():
+    grid, ratio, D, heads = (1, 4, 8), (1, 2, 2), 8, 2
+    f, h, w = grid
+    rng = np.random.default_rng(16)
+    z = rng.standard_normal((32, D))
+    Wp, Wc = _weights(D, 17), _weights(D, 18)
+    base = O.giim(z, grid, ratio, Wp, Wc, heads)
+    # swap the token blocks of proxy windows (0,0) and (1,3)
+    perm = np.arange(32)
+    for dy in range(2):
+        for dx in range(2):
+            a = (0 + dy) * w + (0 + dx)
+            b = (2 + dy) * w + (6 + dx)
+            perm[a], perm[b] = b, a
+    _close(O.giim(z[perm], grid, ratio, Wp, Wc, heads), base[perm], 1e-12)
+    # permute tokens inside every window: proxies unchanged, output permuted alike
+    perm2 = np.arange(32)
+    for Y in range(0, h, 2):
+        for X in range(0, w, 2):
+            a, b = Y * w + X, (Y + 1) * w + X + 1
+            perm2[a], perm2[b] = b, a
+    _close(O.averaging(z[perm2], grid, ratio), O.averaging(z, grid, ratio), 1e-15)
+    _close(O.giim(z[perm2], grid, ratio, Wp, Wc, heads), base[perm2], 1e-12)
+
+
+# ---------------------------------------------------------------- P8 brute force
+
+def _scalar_mha_row(zi, keys, W, heads):
+    """One query row by scalar loops: projections, per-head softmax with math.exp, output projection."""
+    Wq, Wk, Wv, Wo = W
+    D = len(zi)
+    d = D // heads
+
+    def lin(Wm, x):
+        return [sum(Wm[o][k] * x[k] for k in range(D)) for o in range(D)]
+
+    q = lin(Wq, zi)
+    ks = [lin(Wk, kj) for kj in keys]
+    vs = [lin(Wv, kj) for kj in keys]
+    o = [0.0] * D
+    for hh in range(heads):
+        c0 = hh * d
+        s = [sum(q[c0 + c] * kk[c0 + c] for c in range(d)) / math.sqrt(d) for kk in ks]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        tot = sum(e)
+        for c in range(d):
+            o[c0 + c] = sum(e[j] * vs[j][c0 + c] for j in range(len(ks))) / tot
+    return np.array(lin(Wo, o))
+
+
+def test_bruteforce_tiny_block():
+    grid, ratio, window, shift, D, heads = (2, 4, 4), (1, 2, 2), (2, 2, 2), (1, 1, 1), 4, 2
+    f, h, w = grid
+    N = 32
+    rng = np.random.default_rng(19)
+    z = rng.standard_normal((N, D))
+    Wp, Wc, Wa, Ws = (_weights(D, s) for s in (20, 21, 22, 23))
+    coords = [(t, y, x) for t in range(f) for y in range(h) for x in range(w)]
+
+    # GIIM by scalar loops
+    proxies = []
+    for T in range(0, f, ratio[0]):
+        for Y in range(0, h, ratio[1]):
+            for X in range(0, w, ratio[2]):
+                mem = [i for i, (t, y, x) in enumerate(coords)
+                       if T <= t < T + ratio[0] and Y <= y < Y + ratio[1] and X <= x < X + ratio[2]]
+                proxies.append(sum(z[i] for i in mem) / len(mem))
+    Pp = [_scalar_mha_row(p, proxies, Wp, heads) for p in proxies]
+    z1 = np.array([z[i] + _scalar_mha_row(z[i], Pp, Wc, heads) for i in range(N)])
+
+    def window_pass(zin, s):
+        # physically shift each token to its place in the rolled grid, remember
+        # along which axes the roll wrapped it, and attend among tokens that
+        # share a window and the same wrap flags
+        out = np.empty_like(zin)
+        placed = {}
+        for i, (t, y, x) in enumerate(coords):
+            pos = ((t - s[0]) % f, (y - s[1]) % h, (x - s[2]) % w)
+            wrapped = (t < s[0], y < s[1], x < s[2])
+            win = (pos[0] // window[0], pos[1] // window[1], pos[2] // window[2])
+            placed[i] = (win, wrapped)
+        Wm = Wa if s == (0, 0, 0) else Ws
+        for i in range(N):
+            keys = [zin[j] for j in range(N) if placed[j] == placed[i]]
+            out[i] = zin[i] + _scalar_mha_row(zin[i], keys, Wm, heads)
+        return out
+
+    z3 = window_pass(window_pass(z1, (0, 0, 0)), shift)
+    got = O.block_attn(z, grid, ratio, window, shift, Wp, Wc, Wa, Ws, heads)
+    _close(got, z3, 1e-12)
+
+
+def test_block_rows_closure_matches_full():
+    grid, ratio, window, shift, D, heads = (4, 8, 8), (1, 2, 4), (2, 4, 4), (1, 2, 2), 8, 2
+    rng = np.random.default_rng(24)
+    z = rng.standard_normal((256, D))
+    Ws = [_weights(D, s) for s in (25, 26, 27, 28)]
+    full = O.block_attn(z, grid, ratio, window, shift, *Ws, heads)
+    rows = np.array([0, 7, 63, 64, 130, 255, 200])
+    _close(O.block_attn_rows(z, grid, ratio, window, shift, *Ws, heads, rows), full[rows], 1e-13)
+
+
+# ---------------------------------------------------------------- P9 the pages' number
+
+def test_complexity_ratio_matches_printed_2_3_percent():
+    g = _golden("complexity_ratio_2048.json")
+    pct = 100 * flops.core_ratio(16384, 256, 64)
+    assert abs(pct - g["printed_percent"]) <= g["printed_resolution_percent"]
+    # the counter's own terms give the same ratio against its dense core
+    f = flops.block_flops(16384, 256, 64, 1152)
+    dense = flops.dense_flops(16384, 1152)
+    assert math.isclose(f["core"] / dense["core"], flops.core_ratio(16384, 256, 64))
+
+
+# ---------------------------------------------------------------- P10 invariants
+
+def test_softmax_rows_and_convex_hull():
+    rng = np.random.default_rng(29)
+    S = rng.standard_normal((7, 11)) * 5
+    S[:, 3] = -np.inf
+    Pm = O.softmax_rows(S)
+    _close(Pm.sum(axis=1), np.ones(7), 1e-15)
+    assert np.all(Pm[:, 3] == 0)
+    Q, K, V = (rng.standard_normal((9, 6)) for _ in range(3))
+    out = O.attention_heads(Q, K, V, 2)
+    for h in range(2):
+        cols = slice(3 * h, 3 * h + 3)
+        assert np.all(out[:, cols] <= V[:, cols].max(axis=0) + 1e-12)
+        assert np.all(out[:, cols] >= V[:, cols].min(axis=0) - 1e-12)
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def _pin_fails(fn):
+    try:
+        fn()
+    except AssertionError:
+        return True
+    return False
+
+
+def test_pins_catch_a_flipped_roll(monkeypatch):
+    roll = np.roll
+
+    def flipped_roll(a, shift, axis):
+        return roll(a, tuple(-s for s in shift), axis)
+
+    monkeypatch.setattr(np, "roll", flipped_roll)
+    assert _pin_fails(lambda: test_roll_formulation_matches_pair_mask_and_library((1, 4, 8)))
+
+
+def test_pins_catch_a_dropped_scale(monkeypatch):
+    monkeypatch.setattr(math, "sqrt", lambda x: 1.0)
+    assert _pin_fails(test_ratio_111_proxy_sa_is_full_self_attention)
+
+
+def test_pins_catch_a_transposed_weight(monkeypatch):
+    monkeypatch.setattr(O.ptdit_oracle, "project", lambda x, W: np.asarray(x, float) @ np.asarray(W, float))
+    assert _pin_fails(test_ratio_111_proxy_sa_is_full_self_attention)
+
+
+def test_pins_catch_a_wrong_proxy_order(monkeypatch):
+    real = O.ptdit_oracle.averaging
+
+    def col_major(z, grid, ratio):
+        f, h, w = grid
+        pf, ph, pw = ratio
+        P = real(z, grid, ratio)
+        # windows numbered column-major instead of row-major
+        return P.reshape(f // pf, h // ph, w // pw, -1).transpose(2, 1, 0, 3).reshape(P.shape)
+
+    monkeypatch.setattr(O, "averaging", col_major)
+    assert _pin_fails(lambda: test_averaging_bruteforce((1, 4, 4)))
