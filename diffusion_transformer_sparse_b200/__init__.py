@@ -1,1 +1,264 @@
-"""PT-DiT block attention (GIIM + TCM) on B200: ctypes binding over libptdit.so."""
+"""PT-DiT block attention (GIIM + TCM) on NVIDIA B200: ctypes binding over libptdit.so.
+
+Every function here only marshals arguments: torch CUDA tensors become device
+pointers, the current torch stream becomes the stream argument, and a non-zero
+status becomes a PtditError.  All arithmetic runs in the CUDA library; there is
+no CPU path.  If libptdit.so is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libptdit.so")
+
+PTDIT_F32, PTDIT_BF16 = 0, 1
+PTDIT_PROXY_RESIDUAL = 0x1
+PTDIT_NO_RESIDUAL = 0x2
+KINDS = ("average", "gemm", "attn_proxy", "attn_cross", "attn_window", "attn_dense")
+
+# Every symbol declared in include/ptdit.h.
+EXPORTS = (
+    "ptdit_proxy_average", "ptdit_workspace_bytes", "ptdit_giim", "ptdit_window_attn",
+    "ptdit_tcm", "ptdit_block_attn", "ptdit_full_attn", "ptdit_strerror", "ptdit_last_error",
+    "ptdit_debug_proxy_map", "ptdit_debug_window_map", "ptdit_timing_enable",
+    "ptdit_timing_read", "ptdit_launch_count",
+)
+
+
+class PtditError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"ptdit error {code}: {message}")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("F", ctypes.c_int), ("H", ctypes.c_int),
+                ("W", ctypes.c_int), ("D", ctypes.c_int), ("heads", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+class AttnW(ctypes.Structure):
+    _fields_ = [("wq", ctypes.c_void_p), ("wk", ctypes.c_void_p), ("wv", ctypes.c_void_p),
+                ("wo", ctypes.c_void_p)]
+
+
+_lib = None
+Int3 = ctypes.c_int * 3
+_P = ctypes.c_void_p
+_S = ctypes.POINTER(Shape)
+_W = ctypes.POINTER(AttnW)
+_I3 = ctypes.POINTER(ctypes.c_int)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libptdit.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "diffusion_transformer_sparse_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        sig = {
+            "ptdit_proxy_average": (ctypes.c_int, [_S, _I3, _P, _P, _P]),
+            "ptdit_workspace_bytes": (ctypes.c_size_t, [_S, _I3, _I3]),
+            "ptdit_giim": (ctypes.c_int, [_S, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
+                                          ctypes.c_size_t, _P]),
+            "ptdit_window_attn": (ctypes.c_int, [_S, _I3, _I3, _W, ctypes.c_uint, _P, _P, _P,
+                                                 ctypes.c_size_t, _P]),
+            "ptdit_tcm": (ctypes.c_int, [_S, _I3, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
+                                         ctypes.c_size_t, _P]),
+            "ptdit_block_attn": (ctypes.c_int, [_S, _I3, _I3, _I3, _W, _W, _W, _W, ctypes.c_uint,
+                                                _P, _P, _P, ctypes.c_size_t, _P]),
+            "ptdit_full_attn": (ctypes.c_int, [_S, _W, ctypes.c_uint, _P, _P, _P,
+                                               ctypes.c_size_t, _P]),
+            "ptdit_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+            "ptdit_last_error": (ctypes.c_char_p, []),
+            "ptdit_debug_proxy_map": (ctypes.c_int, [_I3, _I3, _P, _P]),
+            "ptdit_debug_window_map": (ctypes.c_int, [_I3, _I3, _I3, _P, _P, _P]),
+            "ptdit_timing_enable": (ctypes.c_int, [ctypes.c_int]),
+            "ptdit_timing_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
+                                                 ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
+            "ptdit_launch_count": (ctypes.c_longlong, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(code: int):
+    if code != 0:
+        raise PtditError(code, lib().ptdit_last_error().decode())
+
+
+def _i3(v) -> Int3:
+    return Int3(*[int(x) for x in v]) if v is not None else None
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return PTDIT_BF16
+    if t.dtype == torch.float32:
+        return PTDIT_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def make_shape(z, grid, heads) -> Shape:
+    """Shape of a [B, N, D] latent tensor on the (f, h, w) grid."""
+    B, N, D = z.shape
+    f, h, w = grid
+    if f * h * w != N:
+        raise ValueError(f"grid {tuple(grid)} does not hold {N} tokens")
+    return Shape(B, f, h, w, D, heads, _dtype_code(z))
+
+
+def attn_w(ws) -> AttnW:
+    """AttnW from a (Wq, Wk, Wv, Wo) tuple of [D, D] CUDA tensors."""
+    for w in ws:
+        if not w.is_contiguous():
+            raise ValueError("weights must be contiguous")
+    return AttnW(*[w.data_ptr() for w in ws])
+
+
+def _check_z(z):
+    if not z.is_cuda or not z.is_contiguous() or z.dim() != 3:
+        raise ValueError("latents must be a contiguous [B, N, D] CUDA tensor")
+
+
+def workspace_bytes(shape: Shape, ratio=None, window=None) -> int:
+    return int(lib().ptdit_workspace_bytes(ctypes.byref(shape), _i3(ratio), _i3(window)))
+
+
+def workspace(shape: Shape, ratio=None, window=None):
+    """A caller-owned workspace tensor of ptdit_workspace_bytes() bytes."""
+    import torch
+    n = workspace_bytes(shape, ratio, window)
+    if n == 0:
+        raise PtditError(2, lib().ptdit_last_error().decode())
+    return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+def ptdit_proxy_average(z, grid, ratio, proxies=None, stream=None):
+    """[B, N, D] -> [B, M, D] window means (GIIM Averaging)."""
+    import torch
+    _check_z(z)
+    shape = make_shape(z, grid, 1)
+    P = ratio[0] * ratio[1] * ratio[2]
+    if proxies is None:
+        proxies = torch.empty(z.shape[0], z.shape[1] // P, z.shape[2], dtype=z.dtype,
+                              device=z.device)
+    _check(lib().ptdit_proxy_average(ctypes.byref(shape), _i3(ratio), _ptr(z), _ptr(proxies),
+                                     _stream(stream)))
+    return proxies
+
+
+def _prep(z_in, grid, heads, z_out, ws, ratio, window):
+    import torch
+    _check_z(z_in)
+    shape = make_shape(z_in, grid, heads)
+    if z_out is None:
+        z_out = torch.empty_like(z_in)
+    if ws is None:
+        ws = workspace(shape, ratio, window)
+    return shape, z_out, ws
+
+
+def ptdit_giim(z_in, grid, ratio, psa, cross, heads, flags=0, z_out=None, ws=None,
+               stream=None):
+    shape, z_out, ws = _prep(z_in, grid, heads, z_out, ws, ratio, None)
+    wp, wc = attn_w(psa), attn_w(cross)
+    _check(lib().ptdit_giim(ctypes.byref(shape), _i3(ratio), ctypes.byref(wp), ctypes.byref(wc),
+                            flags, _ptr(z_in), _ptr(z_out), _ptr(ws), ws.numel(),
+                            _stream(stream)))
+    return z_out
+
+
+def ptdit_window_attn(z_in, grid, window, shift, w, heads, flags=0, z_out=None, ws=None,
+                      stream=None):
+    shape, z_out, ws = _prep(z_in, grid, heads, z_out, ws, None, window)
+    ww = attn_w(w)
+    _check(lib().ptdit_window_attn(ctypes.byref(shape), _i3(window), _i3(shift),
+                                   ctypes.byref(ww), flags, _ptr(z_in), _ptr(z_out), _ptr(ws),
+                                   ws.numel(), _stream(stream)))
+    return z_out
+
+
+def ptdit_tcm(z_in, grid, window, shift, wsa, swsa, heads, flags=0, z_out=None, ws=None,
+              stream=None):
+    shape, z_out, ws = _prep(z_in, grid, heads, z_out, ws, None, window)
+    wa, wb = attn_w(wsa), attn_w(swsa)
+    _check(lib().ptdit_tcm(ctypes.byref(shape), _i3(window), _i3(shift), ctypes.byref(wa),
+                           ctypes.byref(wb), flags, _ptr(z_in), _ptr(z_out), _ptr(ws),
+                           ws.numel(), _stream(stream)))
+    return z_out
+
+
+def ptdit_block_attn(z_in, grid, ratio, window, shift, psa, cross, wsa, swsa, heads, flags=0,
+                     z_out=None, ws=None, stream=None):
+    shape, z_out, ws = _prep(z_in, grid, heads, z_out, ws, ratio, window)
+    w = [attn_w(x) for x in (psa, cross, wsa, swsa)]
+    _check(lib().ptdit_block_attn(ctypes.byref(shape), _i3(ratio), _i3(window), _i3(shift),
+                                  *[ctypes.byref(x) for x in w], flags, _ptr(z_in), _ptr(z_out),
+                                  _ptr(ws), ws.numel(), _stream(stream)))
+    return z_out
+
+
+def ptdit_full_attn(z_in, grid, w, heads, flags=0, z_out=None, ws=None, stream=None):
+    shape, z_out, ws = _prep(z_in, grid, heads, z_out, ws, None, None)
+    ww = attn_w(w)
+    _check(lib().ptdit_full_attn(ctypes.byref(shape), ctypes.byref(ww), flags, _ptr(z_in),
+                                 _ptr(z_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return z_out
+
+
+def ptdit_debug_proxy_map(grid, ratio, stream=None):
+    import torch
+    N = grid[0] * grid[1] * grid[2]
+    out = torch.empty(N, dtype=torch.int32, device="cuda")
+    _check(lib().ptdit_debug_proxy_map(_i3(grid), _i3(ratio), _ptr(out), _stream(stream)))
+    return out
+
+
+def ptdit_debug_window_map(grid, window, shift, with_mask=True, stream=None):
+    import torch
+    N = grid[0] * grid[1] * grid[2]
+    n = window[0] * window[1] * window[2]
+    tok = torch.empty(N, dtype=torch.int32, device="cuda")
+    allowed = torch.empty((N // n) * n * n, dtype=torch.uint8, device="cuda") if with_mask else None
+    _check(lib().ptdit_debug_window_map(_i3(grid), _i3(window), _i3(shift), _ptr(tok),
+                                        _ptr(allowed), _stream(stream)))
+    return tok, allowed
+
+
+def ptdit_timing_enable(max_launches: int):
+    _check(lib().ptdit_timing_enable(int(max_launches)))
+
+
+def ptdit_timing_read(max_records: int = 4096):
+    """[(kind name, milliseconds)] of the launches recorded since the last read."""
+    kinds = (ctypes.c_int * max_records)()
+    ms = (ctypes.c_float * max_records)()
+    n = lib().ptdit_timing_read(kinds, ms, max_records)
+    if n < 0:
+        raise PtditError(5, lib().ptdit_last_error().decode())
+    return [(KINDS[kinds[i]], ms[i]) for i in range(n)]
+
+
+def ptdit_launch_count() -> int:
+    return int(lib().ptdit_launch_count())

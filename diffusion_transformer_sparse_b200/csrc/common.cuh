@@ -1,0 +1,133 @@
+// Shared device helpers of the PT-DiT kernels: index maps of the token grid,
+// element conversions and the internal launcher interfaces.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ptdit {
+
+// ---------------------------------------------------------------------------
+// Token grid and index maps
+//
+// Tokens are flattened row-major over the (f, h, w) grid (Qihoo-T2X reading
+// note, Fig. 2 reading).  Proxy windows and TCM windows are numbered row-major
+// over their window grid, and the tokens inside a window row-major over
+// (t, y, x).
+// ---------------------------------------------------------------------------
+
+// Proxy windows of p_f x p_h x p_w tokens (§3 Method, Eq. GIIM "Averaging").
+struct ProxyGeom {
+    int f, h, w;      // token grid
+    int pf, ph, pw;   // proxy ratio
+    int mf, mh, mw;   // windows per axis
+    int M, P;         // proxies, tokens per proxy window
+};
+
+__host__ __device__ __forceinline__ int proxy_token(const ProxyGeom &g, int m, int k) {
+    // k-th token (row-major inside the window) of proxy window m
+    int X = m % g.mw, r = m / g.mw, Y = r % g.mh, T = r / g.mh;
+    int c = k % g.pw, q = k / g.pw, b = q % g.ph, a = q / g.ph;
+    return ((T * g.pf + a) * g.h + Y * g.ph + b) * g.w + X * g.pw + c;
+}
+
+__host__ __device__ __forceinline__ int proxy_of_token(const ProxyGeom &g, int tok) {
+    int x = tok % g.w, r = tok / g.w, y = r % g.h, t = r / g.h;
+    return ((t / g.pf) * g.mh + y / g.ph) * g.mw + x / g.pw;
+}
+
+// TCM windows of w_f x w_h x w_w tokens on the grid rolled by -shift
+// (§3 Method, Eq. TCM; Swin-style cyclic shift).
+struct WinGeom {
+    int f, h, w;      // token grid
+    int wf, wh, ww;   // window
+    int sf, sh, sw;   // shift: window origin of the rolled grid is token (s_f, s_h, s_w)
+    int nwf, nwh, nww;// windows per axis
+    int n, nwin;      // tokens per window, windows per batch item
+};
+
+// Original token index held by slot `slot` of rolled-grid window `win`.
+// *wrap gets one bit per axis (t: 4, y: 2, x: 1), set where the roll carried
+// the token across the grid edge.  Two slots of one window may attend each
+// other iff their wrap bits are equal: the shift mask is this comparison.
+__host__ __device__ __forceinline__ int window_token(const WinGeom &g, int win, int slot,
+                                                     int *wrap) {
+    int wx = win % g.nww, r = win / g.nww, wy = r % g.nwh, wt = r / g.nwh;
+    int sx = slot % g.ww, q = slot / g.ww, sy = q % g.wh, st = q / g.wh;
+    int t = wt * g.wf + st + g.sf;
+    int y = wy * g.wh + sy + g.sh;
+    int x = wx * g.ww + sx + g.sw;
+    int c = 0;
+    if (t >= g.f) { t -= g.f; c |= 4; }
+    if (y >= g.h) { y -= g.h; c |= 2; }
+    if (x >= g.w) { x -= g.w; c |= 1; }
+    *wrap = c;
+    return (t * g.h + y) * g.w + x;
+}
+
+// ---------------------------------------------------------------------------
+// Element conversions
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------------------
+// Internal launcher interfaces (host side); each returns a cudaError_t.
+// ---------------------------------------------------------------------------
+enum DType { DT_F32 = 0, DT_BF16 = 1 };
+
+// out[b, m, :] = mean over window m of z[b, tok, :]
+cudaError_t launch_proxy_average(int dtype, const ProxyGeom &g, int B, int D, const void *z,
+                                 void *proxies, cudaStream_t s);
+
+// C_s[rows, nseg] = A[rows, K] * W_s[nseg, K]^T (+ R_s), s < nmat.
+// A has row stride lda; C_s and R_s share row stride ldc.  R_s may equal C_s
+// (in-place residual) or be null.
+struct GemmArgs {
+    int dtype;
+    const void *A;
+    long lda;
+    const void *W[3];
+    void *C[3];
+    const void *R[3];
+    long ldc;
+    int rows, nseg, K, nmat;
+};
+cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s);
+
+// Attention core.  Head h uses columns h*d .. h*d+d-1 of q, k, v, o.
+//   ATT_ROWS:   queries are rows [0, nq) and keys rows [0, nk) of each batch
+//               item (proxy SA, cross-attention, full SA).
+//   ATT_WINDOW: queries and keys are the tokens of one TCM window (geom),
+//               pairs with different wrap bits masked.
+enum AttnMode { ATT_ROWS = 0, ATT_WINDOW = 1 };
+struct AttnArgs {
+    int dtype, mode;
+    const void *q, *k, *v;
+    void *o;
+    long ldq, ldk, ldv, ldo;       // row strides (elements)
+    long q_bstride, k_bstride;     // rows per batch item of q/o and of k/v
+    int B, heads, d;
+    int nq, nk;                    // ATT_ROWS sizes per batch item
+    WinGeom geom;                  // ATT_WINDOW geometry
+    float scale;                   // 1/sqrt(d)
+};
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s);
+
+// Debug maps written with the kernels' own index functions.
+cudaError_t launch_debug_proxy_map(const ProxyGeom &g, int32_t *out, cudaStream_t s);
+cudaError_t launch_debug_window_map(const WinGeom &g, int32_t *tok, uint8_t *allowed,
+                                    cudaStream_t s);
+
+// Per-launch timing hooks (no-ops unless enabled by ptdit_timing_enable).
+void timing_begin(int kind, cudaStream_t s);
+void timing_end(cudaStream_t s);
+void count_launch();
+
+}  // namespace ptdit

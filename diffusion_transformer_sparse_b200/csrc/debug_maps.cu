@@ -1,0 +1,51 @@
+// Debug exports of the index maps, computed on the device with the same
+// address functions (proxy_token / proxy_of_token / window_token) that the
+// averaging and attention kernels use.
+#include "common.cuh"
+
+namespace ptdit {
+namespace {
+
+__global__ void proxy_map_kernel(ProxyGeom g, int32_t *out) {
+    const int N = g.f * g.h * g.w;
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < N; t += gridDim.x * blockDim.x) {
+        const int m = proxy_of_token(g, t);
+        // the token's slot inside its window must lead back to it through the
+        // member function the averaging kernel uses; a mismatch writes -1
+        const int x = t % g.w, y = (t / g.w) % g.h, tt = t / (g.w * g.h);
+        const int k = ((tt % g.pf) * g.ph + y % g.ph) * g.pw + x % g.pw;
+        out[t] = (proxy_token(g, m, k) == t) ? m : -1;
+    }
+}
+
+__global__ void window_map_kernel(WinGeom g, int32_t *tok, uint8_t *allowed) {
+    const long total = (long)g.nwin * g.n;
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
+         i += (long)gridDim.x * blockDim.x) {
+        const int win = (int)(i / g.n), slot = (int)(i % g.n);
+        int wi;
+        tok[i] = window_token(g, win, slot, &wi);
+        if (allowed) {
+            for (int j = 0; j < g.n; ++j) {
+                int wj;
+                window_token(g, win, j, &wj);
+                allowed[i * g.n + j] = (wi == wj) ? 1 : 0;
+            }
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_debug_proxy_map(const ProxyGeom &g, int32_t *out, cudaStream_t s) {
+    proxy_map_kernel<<<64, 256, 0, s>>>(g, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_debug_window_map(const WinGeom &g, int32_t *tok, uint8_t *allowed,
+                                    cudaStream_t s) {
+    window_map_kernel<<<64, 256, 0, s>>>(g, tok, allowed);
+    return cudaGetLastError();
+}
+
+}  // namespace ptdit

@@ -1,0 +1,142 @@
+// Window averaging: the proxy tokens of GIIM.
+//
+// Qihoo-T2X reading note, §3 Method, Eq. GIIM "Averaging" and the code
+// listing's get_proxy_token(mode="mean"): every p_f x p_h x p_w window of the
+// token grid is averaged into one proxy token.
+//
+// The kernel is a pure HBM stream: it reads every latent element once and
+// writes every proxy element once.  One CTA owns one proxy; its threads are
+// (16-byte channel chunk) x (token group).  A warp reads 512 contiguous bytes
+// of one token row per load, each thread keeps several independent 16-byte
+// loads in flight, and the token groups are summed through shared memory in
+// a fixed order, so the result is bitwise deterministic.
+#include "common.cuh"
+
+namespace ptdit {
+namespace {
+
+template <typename T, int VEC>
+struct Chunk;
+template <>
+struct Chunk<__nv_bfloat16, 8> {
+    uint4 raw;
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
+        raw = __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    __device__ __forceinline__ void add_to(float *acc) const {
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 f = __bfloat1622float2(h[i]);
+            acc[2 * i] += f.x;
+            acc[2 * i + 1] += f.y;
+        }
+    }
+    __device__ __forceinline__ static void store(__nv_bfloat16 *p, const float *v) {
+        uint4 o;
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        *reinterpret_cast<uint4 *>(p) = o;
+    }
+};
+template <>
+struct Chunk<float, 4> {
+    float4 raw;
+    __device__ __forceinline__ void load(const float *p) {
+        raw = __ldg(reinterpret_cast<const float4 *>(p));
+    }
+    __device__ __forceinline__ void add_to(float *acc) const {
+        acc[0] += raw.x; acc[1] += raw.y; acc[2] += raw.z; acc[3] += raw.w;
+    }
+    __device__ __forceinline__ static void store(float *p, const float *v) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+};
+template <typename T>
+struct Chunk<T, 1> {
+    T raw;
+    __device__ __forceinline__ void load(const T *p) { raw = p[0]; }
+    __device__ __forceinline__ void add_to(float *acc) const { acc[0] += to_f32(raw); }
+    __device__ __forceinline__ static void store(T *p, const float *v) { p[0] = from_f32<T>(v[0]); }
+};
+
+// blockIdx.x = b * M + m.  Thread t: chunk lane cl = t % CHT, token group
+// gi = t / CHT; the lanes step over the CH chunks of a row CHT at a time.
+template <typename T, int VEC>
+__global__ void __launch_bounds__(1024) proxy_average_kernel(const T *__restrict__ z,
+                                                             T *__restrict__ out, ProxyGeom g,
+                                                             int D, int CHT, int G) {
+    extern __shared__ float red[];  // [G-1][CHT][VEC]
+    const int CH = D / VEC;
+    const int m = blockIdx.x % g.M;
+    const int b = blockIdx.x / g.M;
+    const int cl = threadIdx.x % CHT;
+    const int gi = threadIdx.x / CHT;
+    const long N = (long)g.f * g.h * g.w;
+    const T *zw = z + (long)b * N * D + (long)proxy_token(g, m, 0) * D;
+
+    for (int c0 = 0; c0 < CH; c0 += CHT) {
+        const int c = c0 + cl;
+        float acc[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+        if (gi < G && c < CH) {
+            const T *zb = zw + (long)c * VEC;
+            // token k of the window sits (a*h + r)*w + q tokens after the first one
+#pragma unroll 4
+            for (int k = gi; k < g.P; k += G) {
+                int q = k % g.pw, rest = k / g.pw, r = rest % g.ph, a = rest / g.ph;
+                Chunk<T, VEC> ch;
+                ch.load(zb + ((long)(a * g.h + r) * g.w + q) * D);
+                ch.add_to(acc);
+            }
+        }
+        if (gi > 0 && gi < G) {
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) red[((gi - 1) * CHT + cl) * VEC + i] = acc[i];
+        }
+        __syncthreads();
+        if (gi == 0 && c < CH) {
+            for (int j = 1; j < G; ++j) {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) acc[i] += red[((j - 1) * CHT + cl) * VEC + i];
+            }
+            float v[VEC];
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) v[i] = acc[i] / (float)g.P;
+            Chunk<T, VEC>::store(out + ((long)b * g.M + m) * D + (long)c * VEC, v);
+        }
+        __syncthreads();
+    }
+}
+
+template <typename T, int VEC>
+cudaError_t launch_avg(const ProxyGeom &g, int B, int D, const void *z, void *out,
+                       cudaStream_t s) {
+    const int CH = D / VEC;
+    const int CHT = CH < 512 ? CH : 512;
+    int G = 512 / CHT;
+    if (G < 1) G = 1;
+    if (G > g.P) G = g.P;
+    const int threads = CHT * G;
+    const size_t smem = (size_t)(G - 1) * CHT * VEC * sizeof(float);
+    proxy_average_kernel<T, VEC><<<(unsigned)(B * g.M), threads, smem, s>>>(
+        static_cast<const T *>(z), static_cast<T *>(out), g, D, CHT, G);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_proxy_average(int dtype, const ProxyGeom &g, int B, int D, const void *z,
+                                 void *proxies, cudaStream_t s) {
+    const bool aligned = ((uintptr_t)z % 16 == 0) && ((uintptr_t)proxies % 16 == 0);
+    if (dtype == DT_BF16) {
+        if (aligned && D % 8 == 0) return launch_avg<__nv_bfloat16, 8>(g, B, D, z, proxies, s);
+        return launch_avg<__nv_bfloat16, 1>(g, B, D, z, proxies, s);
+    }
+    if (aligned && D % 4 == 0) return launch_avg<float, 4>(g, B, D, z, proxies, s);
+    return launch_avg<float, 1>(g, B, D, z, proxies, s);
+}
+
+}  // namespace ptdit

@@ -1,0 +1,626 @@
+// C ABI of the PT-DiT block-attention library: argument validation, workspace
+// layout, launch ordering on the caller's stream, error reporting and the
+// optional per-launch timing hooks.
+//
+// Launch order of ptdit_block_attn (Qihoo-T2X reading note, §3 Method and the
+// code listing of ProxyTokensTransformerBlock.forward):
+//   GIIM  1 average z -> P          2 Q,K,V = P W_psa^T     3 proxy SA core
+//         4 P' = A W_psa,o^T (+P)   5 K_c,V_c = P' W^T      6 Q_c = z W_c,q^T
+//         7 cross-attention core    8 z_out = z + O W_c,o^T
+//   TCM   9 Q,K,V = z_out W_wsa^T  10 window core (shift 0) 11 z_out += O W_wsa,o^T
+//        12 Q,K,V = z_out W_swsa^T 13 window core (shift s) 14 z_out += O W_swsa,o^T
+// The residual stream lives in z_out from step 8 on; steps 11 and 14 add in
+// place (each output element is read and written by the same thread).
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <vector>
+
+#include "common.cuh"
+#include "ptdit.h"
+
+namespace ptdit {
+cudaError_t launch_gemm_simt(const GemmArgs &a, cudaStream_t s);
+cudaError_t launch_attention_simt(const AttnArgs &a, cudaStream_t s);
+bool gemm_tc_supported(const GemmArgs &a);
+cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
+bool attention_tc_supported(const AttnArgs &a);
+cudaError_t launch_attention_tc(const AttnArgs &a, cudaStream_t s);
+
+cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s) {
+    if (gemm_tc_supported(a)) return launch_gemm_tc(a, s);
+    return launch_gemm_simt(a, s);
+}
+
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s) {
+    if (attention_tc_supported(a)) return launch_attention_tc(a, s);
+    return launch_attention_simt(a, s);
+}
+
+// ------------------------------------------------------------------ timing hooks
+namespace {
+struct TimingState {
+    int max = 0;
+    int count = 0;
+    int open_kind = -1;
+    std::vector<cudaEvent_t> ev0, ev1;
+    std::vector<int> kind;
+};
+thread_local TimingState g_timing;
+thread_local long long g_launches = 0;
+}  // namespace
+
+void timing_begin(int kind, cudaStream_t s) {
+    TimingState &t = g_timing;
+    if (t.max == 0 || t.count >= t.max) return;
+    t.open_kind = kind;
+    cudaEventRecord(t.ev0[t.count], s);
+}
+
+void timing_end(cudaStream_t s) {
+    TimingState &t = g_timing;
+    if (t.open_kind < 0) return;
+    cudaEventRecord(t.ev1[t.count], s);
+    t.kind[t.count] = t.open_kind;
+    t.open_kind = -1;
+    ++t.count;
+}
+
+void count_launch() { ++g_launches; }
+
+}  // namespace ptdit
+
+using namespace ptdit;
+
+// ------------------------------------------------------------------ errors
+namespace {
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(PTDIT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------------ validation
+struct Dims {
+    int B, f, h, w, D, heads, d, dtype;
+    long N;
+    size_t elem;
+};
+
+int check_shape(const ptdit_shape *s, Dims *o, bool attention = true) {
+    if (!s) return fail(PTDIT_ERR_NULL, "shape is NULL");
+    if (s->dtype != PTDIT_F32 && s->dtype != PTDIT_BF16)
+        return fail(PTDIT_ERR_DTYPE, "dtype %d is neither PTDIT_F32 nor PTDIT_BF16", s->dtype);
+    if (s->B < 1 || s->F < 1 || s->H < 1 || s->W < 1 || s->D < 1 || s->heads < 1)
+        return fail(PTDIT_ERR_SHAPE, "B, F, H, W, D and heads must all be positive");
+    if (s->D % s->heads)
+        return fail(PTDIT_ERR_SHAPE, "D=%d is not divisible by heads=%d", s->D, s->heads);
+    const long N = (long)s->F * s->H * s->W;
+    if (N > (1L << 30) || (long)s->B * N > (1L << 31) - 1)
+        return fail(PTDIT_ERR_SHAPE, "B*N=%ld tokens exceeds 2^31-1", (long)s->B * N);
+    if (s->D > 16384) return fail(PTDIT_ERR_SHAPE, "D=%d above 16384", s->D);
+    if (attention && s->D / s->heads > 128)
+        return fail(PTDIT_ERR_SHAPE, "head dim %d above 128", s->D / s->heads);
+    o->B = s->B; o->f = s->F; o->h = s->H; o->w = s->W; o->D = s->D;
+    o->heads = s->heads; o->d = s->D / s->heads; o->dtype = s->dtype; o->N = N;
+    o->elem = s->dtype == PTDIT_BF16 ? 2 : 4;
+    return PTDIT_OK;
+}
+
+int make_proxy(const Dims &d, const int ratio[3], ProxyGeom *g) {
+    if (!ratio) return fail(PTDIT_ERR_NULL, "ratio is NULL");
+    const int L[3] = {d.f, d.h, d.w};
+    for (int i = 0; i < 3; ++i)
+        if (ratio[i] < 1 || L[i] % ratio[i])
+            return fail(PTDIT_ERR_SHAPE, "grid axis %d (%d) is not divisible by ratio %d", i,
+                        L[i], ratio[i]);
+    g->f = d.f; g->h = d.h; g->w = d.w;
+    g->pf = ratio[0]; g->ph = ratio[1]; g->pw = ratio[2];
+    g->mf = d.f / ratio[0]; g->mh = d.h / ratio[1]; g->mw = d.w / ratio[2];
+    g->M = g->mf * g->mh * g->mw;
+    g->P = ratio[0] * ratio[1] * ratio[2];
+    return PTDIT_OK;
+}
+
+int make_window(const Dims &d, const int window[3], const int shift[3], WinGeom *g) {
+    if (!window) return fail(PTDIT_ERR_NULL, "window is NULL");
+    if (!shift) return fail(PTDIT_ERR_NULL, "shift is NULL");
+    const int L[3] = {d.f, d.h, d.w};
+    for (int i = 0; i < 3; ++i) {
+        if (window[i] < 1 || L[i] % window[i])
+            return fail(PTDIT_ERR_SHAPE, "grid axis %d (%d) is not divisible by window %d", i,
+                        L[i], window[i]);
+        if (shift[i] < 0 || shift[i] >= window[i])
+            return fail(PTDIT_ERR_SHAPE, "shift %d on axis %d is outside [0, window=%d)",
+                        shift[i], i, window[i]);
+    }
+    g->f = d.f; g->h = d.h; g->w = d.w;
+    g->wf = window[0]; g->wh = window[1]; g->ww = window[2];
+    g->sf = shift[0]; g->sh = shift[1]; g->sw = shift[2];
+    g->nwf = d.f / window[0]; g->nwh = d.h / window[1]; g->nww = d.w / window[2];
+    g->n = window[0] * window[1] * window[2];
+    g->nwin = g->nwf * g->nwh * g->nww;
+    return PTDIT_OK;
+}
+
+int check_ptr(const void *p, const char *name) {
+    if (!p) return fail(PTDIT_ERR_NULL, "%s is NULL", name);
+    if ((uintptr_t)p % 16) return fail(PTDIT_ERR_ALIGN, "%s is not 16-byte aligned", name);
+    return PTDIT_OK;
+}
+
+int check_weights(const ptdit_attn_w *w, const char *name) {
+    if (!w) return fail(PTDIT_ERR_NULL, "%s weights are NULL", name);
+    const void *p[4] = {w->wq, w->wk, w->wv, w->wo};
+    const char *nm[4] = {"wq", "wk", "wv", "wo"};
+    for (int i = 0; i < 4; ++i) {
+        if (!p[i]) return fail(PTDIT_ERR_NULL, "%s.%s is NULL", name, nm[i]);
+        if ((uintptr_t)p[i] % 16)
+            return fail(PTDIT_ERR_ALIGN, "%s.%s is not 16-byte aligned", name, nm[i]);
+    }
+    return PTDIT_OK;
+}
+
+bool overlap(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+    return x < y + nb && y < x + na;
+}
+
+// ------------------------------------------------------------------ workspace
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Ws {
+    size_t P, Qp, Kp, Vp, Ap, Pp, Kc, Vc, Q, K, V, O, total;
+};
+
+Ws ws_layout(const Dims &d, long M) {
+    Ws L;
+    size_t off = 0;
+    auto take = [&](size_t elems) {
+        const size_t o = off;
+        off += align256(elems * d.elem);
+        return o;
+    };
+    const size_t pm = (size_t)d.B * M * d.D, tn = (size_t)d.B * d.N * d.D;
+    L.P = take(pm); L.Qp = take(pm); L.Kp = take(pm); L.Vp = take(pm);
+    L.Ap = take(pm); L.Pp = take(pm); L.Kc = take(pm); L.Vc = take(pm);
+    L.Q = take(tn); L.K = take(tn); L.V = take(tn); L.O = take(tn);
+    L.total = off;
+    return L;
+}
+
+int check_ws(const Dims &d, long M, const void *ws, size_t ws_bytes, Ws *L) {
+    *L = ws_layout(d, M);
+    if (!ws) return fail(PTDIT_ERR_NULL, "workspace is NULL");
+    if ((uintptr_t)ws % 256) return fail(PTDIT_ERR_ALIGN, "workspace is not 256-byte aligned");
+    if (ws_bytes < L->total)
+        return fail(PTDIT_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L->total);
+    return PTDIT_OK;
+}
+
+// ------------------------------------------------------------------ launch helpers
+struct Run {
+    const Dims &d;
+    cudaStream_t s;
+    char *ws;
+    const Ws &L;
+    char *at(size_t off) const { return ws + off; }
+};
+
+int gemm(const Run &r, int kind, const void *A, long rows, int nmat, const void *const W[3],
+         void *const C[3], const void *const R[3], const char *what) {
+    GemmArgs g;
+    memset(&g, 0, sizeof g);
+    g.dtype = r.d.dtype;
+    g.A = A;
+    g.lda = r.d.D;
+    for (int i = 0; i < nmat; ++i) {
+        g.W[i] = W[i];
+        g.C[i] = C[i];
+        g.R[i] = R ? R[i] : nullptr;
+    }
+    g.ldc = r.d.D;
+    g.rows = (int)rows;
+    g.nseg = r.d.D;
+    g.K = r.d.D;
+    g.nmat = nmat;
+    timing_begin(kind, r.s);
+    cudaError_t e = launch_gemm(g, r.s);
+    timing_end(r.s);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
+}
+
+int attention(const Run &r, int kind, AttnArgs a, const char *what) {
+    a.dtype = r.d.dtype;
+    a.heads = r.d.heads;
+    a.d = r.d.d;
+    a.B = r.d.B;
+    a.ldq = a.ldk = a.ldv = a.ldo = r.d.D;
+    a.scale = 1.0f / sqrtf((float)r.d.d);
+    timing_begin(kind, r.s);
+    cudaError_t e = launch_attention(a, r.s);
+    timing_end(r.s);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
+}
+
+#define TRY(x)                         \
+    do {                               \
+        int _rc = (x);                 \
+        if (_rc != PTDIT_OK) return _rc; \
+    } while (0)
+
+// GIIM: z_out = (z_in +) CS(z_in, SA(Average(z_in)) (+ P_a)).
+int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
+             const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z_out) {
+    const Dims &d = r.d;
+    const long BM = (long)d.B * pg.M, BN = (long)d.B * d.N;
+    timing_begin(PTDIT_K_AVERAGE, r.s);
+    cudaError_t e = launch_proxy_average(d.dtype, pg, d.B, d.D, z_in, r.at(r.L.P), r.s);
+    timing_end(r.s);
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, "proxy average");
+    {
+        const void *W[3] = {psa->wq, psa->wk, psa->wv};
+        void *C[3] = {r.at(r.L.Qp), r.at(r.L.Kp), r.at(r.L.Vp)};
+        TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.P), BM, 3, W, C, nullptr, "proxy QKV projection"));
+    }
+    {
+        AttnArgs a;
+        memset(&a, 0, sizeof a);
+        a.mode = ATT_ROWS;
+        a.q = r.at(r.L.Qp); a.k = r.at(r.L.Kp); a.v = r.at(r.L.Vp); a.o = r.at(r.L.Ap);
+        a.q_bstride = a.k_bstride = pg.M;
+        a.nq = a.nk = pg.M;
+        TRY(attention(r, PTDIT_K_ATTN_PROXY, a, "proxy self-attention"));
+    }
+    {
+        const void *W[3] = {psa->wo, nullptr, nullptr};
+        void *C[3] = {r.at(r.L.Pp), nullptr, nullptr};
+        const void *R[3] = {(flags & PTDIT_PROXY_RESIDUAL) ? r.at(r.L.P) : nullptr, nullptr,
+                            nullptr};
+        TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.Ap), BM, 1, W, C, R, "proxy output projection"));
+    }
+    {
+        const void *W[3] = {cross->wk, cross->wv, nullptr};
+        void *C[3] = {r.at(r.L.Kc), r.at(r.L.Vc), nullptr};
+        TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.Pp), BM, 2, W, C, nullptr, "proxy K/V projection"));
+    }
+    {
+        const void *W[3] = {cross->wq, nullptr, nullptr};
+        void *C[3] = {r.at(r.L.Q), nullptr, nullptr};
+        TRY(gemm(r, PTDIT_K_GEMM, z_in, BN, 1, W, C, nullptr, "latent Q projection"));
+    }
+    {
+        AttnArgs a;
+        memset(&a, 0, sizeof a);
+        a.mode = ATT_ROWS;
+        a.q = r.at(r.L.Q); a.k = r.at(r.L.Kc); a.v = r.at(r.L.Vc); a.o = r.at(r.L.O);
+        a.q_bstride = d.N;
+        a.k_bstride = pg.M;
+        a.nq = (int)d.N;
+        a.nk = pg.M;
+        TRY(attention(r, PTDIT_K_ATTN_CROSS, a, "cross-attention"));
+    }
+    {
+        const void *W[3] = {cross->wo, nullptr, nullptr};
+        void *C[3] = {z_out, nullptr, nullptr};
+        const void *R[3] = {(flags & PTDIT_NO_RESIDUAL) ? nullptr : z_in, nullptr, nullptr};
+        TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.O), BN, 1, W, C, R, "cross output projection"));
+    }
+    return PTDIT_OK;
+}
+
+// One TCM branch: x_out = (x_in +) WSA_or_SWSA(x_in).  x_out may equal x_in.
+int run_window(const Run &r, const WinGeom &wg, const ptdit_attn_w *w, unsigned flags,
+               const void *x_in, void *x_out) {
+    const Dims &d = r.d;
+    const long BN = (long)d.B * d.N;
+    {
+        const void *W[3] = {w->wq, w->wk, w->wv};
+        void *C[3] = {r.at(r.L.Q), r.at(r.L.K), r.at(r.L.V)};
+        TRY(gemm(r, PTDIT_K_GEMM, x_in, BN, 3, W, C, nullptr, "window QKV projection"));
+    }
+    {
+        AttnArgs a;
+        memset(&a, 0, sizeof a);
+        a.mode = ATT_WINDOW;
+        a.q = r.at(r.L.Q); a.k = r.at(r.L.K); a.v = r.at(r.L.V); a.o = r.at(r.L.O);
+        a.q_bstride = a.k_bstride = d.N;
+        a.geom = wg;
+        TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "window attention"));
+    }
+    {
+        const void *W[3] = {w->wo, nullptr, nullptr};
+        void *C[3] = {x_out, nullptr, nullptr};
+        const void *R[3] = {(flags & PTDIT_NO_RESIDUAL) ? nullptr : x_in, nullptr, nullptr};
+        TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.O), BN, 1, W, C, R, "window output projection"));
+    }
+    return PTDIT_OK;
+}
+
+int check_io(const Dims &d, const void *z_in, const void *z_out, const void *ws, size_t ws_bytes) {
+    TRY(check_ptr(z_in, "z_in"));
+    TRY(check_ptr(z_out, "z_out"));
+    const size_t zb = (size_t)d.B * d.N * d.D * d.elem;
+    if (overlap(z_in, zb, z_out, zb)) return fail(PTDIT_ERR_ALIAS, "z_out overlaps z_in");
+    if (ws && overlap(ws, ws_bytes, z_out, zb))
+        return fail(PTDIT_ERR_ALIAS, "z_out overlaps the workspace");
+    if (ws && overlap(ws, ws_bytes, z_in, zb))
+        return fail(PTDIT_ERR_ALIAS, "z_in overlaps the workspace");
+    return PTDIT_OK;
+}
+
+int check_w_alias(const Dims &d, const ptdit_attn_w *w, const void *z_out) {
+    const size_t wb = (size_t)d.D * d.D * d.elem, zb = (size_t)d.B * d.N * d.D * d.elem;
+    const void *p[4] = {w->wq, w->wk, w->wv, w->wo};
+    for (int i = 0; i < 4; ++i)
+        if (overlap(p[i], wb, z_out, zb)) return fail(PTDIT_ERR_ALIAS, "z_out overlaps a weight");
+    return PTDIT_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ exported API
+extern "C" {
+
+const char *ptdit_strerror(int status) {
+    switch (status) {
+        case PTDIT_OK: return "ok";
+        case PTDIT_ERR_NULL: return "a required pointer is NULL";
+        case PTDIT_ERR_SHAPE: return "invalid sizes, ratio, window or shift";
+        case PTDIT_ERR_DTYPE: return "unknown dtype";
+        case PTDIT_ERR_WORKSPACE: return "workspace too small";
+        case PTDIT_ERR_CUDA: return "CUDA error";
+        case PTDIT_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case PTDIT_ERR_ALIGN: return "pointer not aligned";
+        case PTDIT_ERR_ALIAS: return "output overlaps an input";
+        default: return "unknown status";
+    }
+}
+
+const char *ptdit_last_error(void) { return g_err; }
+
+long long ptdit_launch_count(void) { return g_launches; }
+
+int ptdit_timing_enable(int max_launches) {
+    TimingState &t = g_timing;
+    for (auto e : t.ev0) cudaEventDestroy(e);
+    for (auto e : t.ev1) cudaEventDestroy(e);
+    t.ev0.clear(); t.ev1.clear(); t.kind.clear();
+    t.max = t.count = 0;
+    t.open_kind = -1;
+    if (max_launches <= 0) return PTDIT_OK;
+    t.ev0.resize(max_launches);
+    t.ev1.resize(max_launches);
+    t.kind.resize(max_launches);
+    for (int i = 0; i < max_launches; ++i) {
+        cudaError_t e = cudaEventCreate(&t.ev0[i]);
+        if (e == cudaSuccess) e = cudaEventCreate(&t.ev1[i]);
+        if (e != cudaSuccess) {
+            t.ev0.resize(i); t.ev1.resize(i);
+            ptdit_timing_enable(0);
+            return cuda_fail(e, "cudaEventCreate");
+        }
+    }
+    t.max = max_launches;
+    return PTDIT_OK;
+}
+
+int ptdit_timing_read(int *kind, float *ms, int max) {
+    TimingState &t = g_timing;
+    const int n = t.count < max ? t.count : max;
+    if (t.count > 0) {
+        cudaError_t e = cudaEventSynchronize(t.ev1[t.count - 1]);
+        if (e != cudaSuccess) {
+            cuda_fail(e, "cudaEventSynchronize");
+            return -1;
+        }
+    }
+    for (int i = 0; i < n; ++i) {
+        float v = 0.f;
+        if (cudaEventElapsedTime(&v, t.ev0[i], t.ev1[i]) != cudaSuccess) {
+            fail(PTDIT_ERR_CUDA, "cudaEventElapsedTime failed");
+            return -1;
+        }
+        kind[i] = t.kind[i];
+        ms[i] = v;
+    }
+    t.count = 0;
+    return n;
+}
+
+size_t ptdit_workspace_bytes(const ptdit_shape *shape, const int ratio[3], const int window[3]) {
+    Dims d;
+    if (check_shape(shape, &d) != PTDIT_OK) return 0;
+    long M = 0;
+    if (ratio) {
+        ProxyGeom pg;
+        if (make_proxy(d, ratio, &pg) != PTDIT_OK) return 0;
+        M = pg.M;
+    }
+    if (window) {
+        const int zero[3] = {0, 0, 0};
+        WinGeom wg;
+        if (make_window(d, window, zero, &wg) != PTDIT_OK) return 0;
+    }
+    return ws_layout(d, M).total;
+}
+
+int ptdit_proxy_average(const ptdit_shape *shape, const int ratio[3], const void *z,
+                        void *proxies, ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    TRY(check_shape(shape, &d, false));
+    TRY(make_proxy(d, ratio, &pg));
+    TRY(check_ptr(z, "z"));
+    TRY(check_ptr(proxies, "proxies"));
+    if (overlap(z, (size_t)d.B * d.N * d.D * d.elem, proxies, (size_t)d.B * pg.M * d.D * d.elem))
+        return fail(PTDIT_ERR_ALIAS, "proxies overlap z");
+    cudaStream_t s = (cudaStream_t)stream;
+    timing_begin(PTDIT_K_AVERAGE, s);
+    cudaError_t e = launch_proxy_average(d.dtype, pg, d.B, d.D, z, proxies, s);
+    timing_end(s);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "proxy average");
+}
+
+int ptdit_giim(const ptdit_shape *shape, const int ratio[3], const ptdit_attn_w *psa,
+               const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z_out,
+               void *ws, size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    Ws L;
+    TRY(check_shape(shape, &d));
+    TRY(make_proxy(d, ratio, &pg));
+    TRY(check_weights(psa, "psa"));
+    TRY(check_weights(cross, "cross"));
+    TRY(check_io(d, z_in, z_out, ws, ws_bytes));
+    TRY(check_w_alias(d, psa, z_out));
+    TRY(check_w_alias(d, cross, z_out));
+    TRY(check_ws(d, pg.M, ws, ws_bytes, &L));
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    return run_giim(r, pg, psa, cross, flags, z_in, z_out);
+}
+
+int ptdit_window_attn(const ptdit_shape *shape, const int window[3], const int shift[3],
+                      const ptdit_attn_w *w, unsigned flags, const void *z_in, void *z_out,
+                      void *ws, size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    WinGeom wg;
+    Ws L;
+    TRY(check_shape(shape, &d));
+    TRY(make_window(d, window, shift, &wg));
+    TRY(check_weights(w, "w"));
+    TRY(check_io(d, z_in, z_out, ws, ws_bytes));
+    TRY(check_w_alias(d, w, z_out));
+    TRY(check_ws(d, 0, ws, ws_bytes, &L));
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    return run_window(r, wg, w, flags, z_in, z_out);
+}
+
+int ptdit_tcm(const ptdit_shape *shape, const int window[3], const int shift[3],
+              const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
+              const void *z_in, void *z_out, void *ws, size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    WinGeom wg0, wg1;
+    Ws L;
+    const int zero[3] = {0, 0, 0};
+    TRY(check_shape(shape, &d));
+    TRY(make_window(d, window, shift, &wg1));
+    TRY(make_window(d, window, zero, &wg0));
+    TRY(check_weights(wsa, "wsa"));
+    TRY(check_weights(swsa, "swsa"));
+    TRY(check_io(d, z_in, z_out, ws, ws_bytes));
+    TRY(check_w_alias(d, wsa, z_out));
+    TRY(check_w_alias(d, swsa, z_out));
+    TRY(check_ws(d, 0, ws, ws_bytes, &L));
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    TRY(run_window(r, wg0, wsa, flags, z_in, z_out));
+    return run_window(r, wg1, swsa, flags, z_out, z_out);
+}
+
+int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                     const int shift[3], const ptdit_attn_w *psa, const ptdit_attn_w *cross,
+                     const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
+                     const void *z_in, void *z_out, void *ws, size_t ws_bytes,
+                     ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    WinGeom wg0, wg1;
+    Ws L;
+    const int zero[3] = {0, 0, 0};
+    TRY(check_shape(shape, &d));
+    TRY(make_proxy(d, ratio, &pg));
+    TRY(make_window(d, window, shift, &wg1));
+    TRY(make_window(d, window, zero, &wg0));
+    TRY(check_weights(psa, "psa"));
+    TRY(check_weights(cross, "cross"));
+    TRY(check_weights(wsa, "wsa"));
+    TRY(check_weights(swsa, "swsa"));
+    TRY(check_io(d, z_in, z_out, ws, ws_bytes));
+    TRY(check_w_alias(d, psa, z_out));
+    TRY(check_w_alias(d, cross, z_out));
+    TRY(check_w_alias(d, wsa, z_out));
+    TRY(check_w_alias(d, swsa, z_out));
+    TRY(check_ws(d, pg.M, ws, ws_bytes, &L));
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    TRY(run_giim(r, pg, psa, cross, flags, z_in, z_out));
+    TRY(run_window(r, wg0, wsa, flags, z_out, z_out));
+    return run_window(r, wg1, swsa, flags, z_out, z_out);
+}
+
+int ptdit_full_attn(const ptdit_shape *shape, const ptdit_attn_w *w, unsigned flags,
+                    const void *z_in, void *z_out, void *ws, size_t ws_bytes,
+                    ptdit_stream_t stream) {
+    Dims d;
+    Ws L;
+    TRY(check_shape(shape, &d));
+    TRY(check_weights(w, "w"));
+    TRY(check_io(d, z_in, z_out, ws, ws_bytes));
+    TRY(check_w_alias(d, w, z_out));
+    TRY(check_ws(d, 0, ws, ws_bytes, &L));
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    const long BN = (long)d.B * d.N;
+    {
+        const void *W[3] = {w->wq, w->wk, w->wv};
+        void *C[3] = {r.at(L.Q), r.at(L.K), r.at(L.V)};
+        TRY(gemm(r, PTDIT_K_GEMM, z_in, BN, 3, W, C, nullptr, "QKV projection"));
+    }
+    {
+        AttnArgs a;
+        memset(&a, 0, sizeof a);
+        a.mode = ATT_ROWS;
+        a.q = r.at(L.Q); a.k = r.at(L.K); a.v = r.at(L.V); a.o = r.at(L.O);
+        a.q_bstride = a.k_bstride = d.N;
+        a.nq = a.nk = (int)d.N;
+        TRY(attention(r, PTDIT_K_ATTN_DENSE, a, "full self-attention"));
+    }
+    {
+        const void *W[3] = {w->wo, nullptr, nullptr};
+        void *C[3] = {z_out, nullptr, nullptr};
+        const void *R[3] = {(flags & PTDIT_NO_RESIDUAL) ? nullptr : z_in, nullptr, nullptr};
+        TRY(gemm(r, PTDIT_K_GEMM, r.at(L.O), BN, 1, W, C, R, "output projection"));
+    }
+    return PTDIT_OK;
+}
+
+int ptdit_debug_proxy_map(const int grid[3], const int ratio[3], int32_t *proxy_of_token,
+                          ptdit_stream_t stream) {
+    if (!grid) return fail(PTDIT_ERR_NULL, "grid is NULL");
+    ptdit_shape sh = {1, grid[0], grid[1], grid[2], 1, 1, PTDIT_F32};
+    Dims d;
+    ProxyGeom pg;
+    TRY(check_shape(&sh, &d));
+    TRY(make_proxy(d, ratio, &pg));
+    if (!proxy_of_token) return fail(PTDIT_ERR_NULL, "proxy_of_token is NULL");
+    cudaError_t e = launch_debug_proxy_map(pg, proxy_of_token, (cudaStream_t)stream);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "proxy map");
+}
+
+int ptdit_debug_window_map(const int grid[3], const int window[3], const int shift[3],
+                           int32_t *token_at_slot, uint8_t *allowed, ptdit_stream_t stream) {
+    if (!grid) return fail(PTDIT_ERR_NULL, "grid is NULL");
+    ptdit_shape sh = {1, grid[0], grid[1], grid[2], 1, 1, PTDIT_F32};
+    Dims d;
+    WinGeom wg;
+    TRY(check_shape(&sh, &d));
+    TRY(make_window(d, window, shift, &wg));
+    if (!token_at_slot) return fail(PTDIT_ERR_NULL, "token_at_slot is NULL");
+    cudaError_t e = launch_debug_window_map(wg, token_at_slot, allowed, (cudaStream_t)stream);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "window map");
+}
+
+}  // extern "C"

@@ -1,0 +1,197 @@
+/*
+ * ptdit.h -- PT-DiT block attention (GIIM + TCM) for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the attention half of a PT-Block of the Proxy-Tokenized
+ * Diffusion Transformer, as stated in "Qihoo-T2X -- Proxy-Tokenized DiT for
+ * Text-to-Any-Task", §3 Method:
+ *
+ *   GIIM (Eq. GIIM)  z_s <- z_s + CS(z_s, SA(Averaging(z_s)))
+ *       Averaging: the mean of z_s over each p_f x p_h x p_w window gives the
+ *       proxy tokens P_a; SA: multi-head self-attention among the proxies;
+ *       CS: multi-head cross-attention, every latent token the query, the
+ *       proxies keys and values.
+ *   TCM  (Eq. TCM)   z^ = WSA(z_s) + z_s ;  z_w = SWSA(z^) + z^
+ *       WSA: self-attention inside non-overlapping windows; SWSA: the same
+ *       after a Swin-style cyclic roll of the grid by -s, with the pairs that
+ *       the roll wrapped masked out, followed by the roll back by +s.
+ *
+ * Conventions shared by every entry point
+ *   - Latents are [B, N, D], contiguous, N = F*H*W flattened row-major over
+ *     the (f, h, w) token grid (t slowest, x fastest).  Proxies are [B, M, D],
+ *     M = N / (p_f p_h p_w), numbered row-major over the grid of windows.
+ *   - A module's weights are four [D][D] row-major matrices, applied as
+ *     y = x W^T (PyTorch Linear layout), with no bias.  Head h owns columns
+ *     h*d .. h*d+d-1 of Q, K, V, d = D / heads.  The softmax scale is
+ *     1/sqrt(d).  The zero-initialised linear after the cross-attention of
+ *     the official code is folded into the cross-attention's W_o.
+ *   - dtype PTDIT_BF16: bf16 storage, bf16 tensor-core inputs, fp32
+ *     accumulation and softmax.  dtype PTDIT_F32: fp32 storage and fp32 FMA
+ *     arithmetic throughout (no TF32).
+ *   - Every data pointer is a DEVICE pointer owned by the caller; the
+ *     library never allocates device memory and keeps no pointer after the
+ *     call returns.  Pointers must be 16-byte aligned.  z_out must not
+ *     overlap z_in, the weights or the workspace.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default
+ *     stream).  Arguments are validated on the host first; on any error
+ *     nothing is launched and a PTDIT_ERR_* code is returned.
+ *     ptdit_last_error() gives a one-line description (per host thread).
+ *   - Every grid extent must be divisible by its proxy ratio and by its TCM
+ *     window, and 0 <= shift < window on every axis (else PTDIT_ERR_SHAPE).
+ */
+#ifndef PTDIT_H
+#define PTDIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *ptdit_stream_t; /* a cudaStream_t */
+
+enum { PTDIT_F32 = 0, PTDIT_BF16 = 1 };
+
+typedef struct {
+    int B;          /* batch items (independent) */
+    int F, H, W;    /* token grid f x h x w; N = F*H*W */
+    int D;          /* model width */
+    int heads;      /* attention heads; d = D / heads */
+    int dtype;      /* PTDIT_F32 or PTDIT_BF16 */
+} ptdit_shape;
+
+/* One attention module's projections: Q = x Wq^T, K = x Wk^T, V = x Wv^T,
+ * out = A Wo^T, each W a [D][D] row-major device array of the call's dtype. */
+typedef struct {
+    const void *wq, *wk, *wv, *wo;
+} ptdit_attn_w;
+
+/* Status codes. */
+#define PTDIT_OK            0
+#define PTDIT_ERR_NULL      1  /* a required pointer is NULL */
+#define PTDIT_ERR_SHAPE     2  /* sizes, ratios, windows or shifts are invalid */
+#define PTDIT_ERR_DTYPE     3  /* unknown dtype */
+#define PTDIT_ERR_WORKSPACE 4  /* workspace smaller than ptdit_workspace_bytes() */
+#define PTDIT_ERR_CUDA      5  /* a CUDA call or launch failed */
+#define PTDIT_ERR_TIMEOUT   6  /* a bounded device-side wait gave up */
+#define PTDIT_ERR_ALIGN     7  /* a pointer is not 16-byte aligned */
+#define PTDIT_ERR_ALIAS     8  /* z_out overlaps an input or the workspace */
+
+/* Flags. */
+#define PTDIT_PROXY_RESIDUAL 0x1u /* proxy SA adds its input: P' = SA(P_a) + P_a
+                                     (the official code listing); default P' = SA(P_a) (Eq. GIIM) */
+#define PTDIT_NO_RESIDUAL    0x2u /* drop every residual add on the latent stream:
+                                     each module returns only its attention branch */
+
+/*
+ * ptdit_proxy_average -- GIIM "Averaging" (Eq. GIIM; get_proxy_token mode "mean").
+ *   proxies[b, m, :] = mean of z[b, t, :] over the tokens t of window m.
+ *   ratio = {p_f, p_h, p_w}.  z: [B, N, D] (in), proxies: [B, M, D] (out).
+ *   Sums in fp32 in a fixed order (bitwise deterministic), one rounding.
+ */
+int ptdit_proxy_average(const ptdit_shape *shape, const int ratio[3], const void *z,
+                        void *proxies, ptdit_stream_t stream);
+
+/*
+ * ptdit_workspace_bytes -- device scratch that every call below needs for
+ * this shape (the maximum over them), or 0 for an invalid shape.  The
+ * workspace must be 256-byte aligned; its contents need no initialisation
+ * and are garbage after a call.
+ */
+size_t ptdit_workspace_bytes(const ptdit_shape *shape, const int ratio[3], const int window[3]);
+
+/*
+ * ptdit_giim -- Eq. GIIM: z_out = z_in + CS(z_in, SA(Averaging(z_in))).
+ *   psa:   the proxy self-attention's weights; cross: the cross-attention's.
+ *   flags: PTDIT_PROXY_RESIDUAL, PTDIT_NO_RESIDUAL (z_out = CS(...) only).
+ */
+int ptdit_giim(const ptdit_shape *shape, const int ratio[3], const ptdit_attn_w *psa,
+               const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z_out,
+               void *ws, size_t ws_bytes, ptdit_stream_t stream);
+
+/*
+ * ptdit_window_attn -- one TCM branch (Eq. TCM): z_out = z_in + WSA(z_in)
+ *   for shift {0,0,0}, else SWSA: Swin-style roll by -shift, attention
+ *   inside each window of window[] tokens with wrapped pairs masked out,
+ *   roll back.  flags: PTDIT_NO_RESIDUAL.
+ */
+int ptdit_window_attn(const ptdit_shape *shape, const int window[3], const int shift[3],
+                      const ptdit_attn_w *w, unsigned flags, const void *z_in, void *z_out,
+                      void *ws, size_t ws_bytes, ptdit_stream_t stream);
+
+/*
+ * ptdit_tcm -- Eq. TCM: WSA with weights wsa, then SWSA with weights swsa
+ *   and the given shift, each with its residual (unless PTDIT_NO_RESIDUAL).
+ */
+int ptdit_tcm(const ptdit_shape *shape, const int window[3], const int shift[3],
+              const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
+              const void *z_in, void *z_out, void *ws, size_t ws_bytes, ptdit_stream_t stream);
+
+/*
+ * ptdit_block_attn -- the PT-Block attention path: GIIM then TCM
+ *   (ProxyTokensTransformerBlock.forward steps 1-4 of the code listing).
+ */
+int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                     const int shift[3], const ptdit_attn_w *psa, const ptdit_attn_w *cross,
+                     const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
+                     const void *z_in, void *z_out, void *ws, size_t ws_bytes,
+                     ptdit_stream_t stream);
+
+/*
+ * ptdit_full_attn -- the dense comparator the pages measure against
+ *   (§3 complexity: full self-attention, 2 N^2 D): z_out = z_in + MHA(z_in)
+ *   over all N tokens of each batch item.  Needs ptdit_workspace_bytes().
+ */
+int ptdit_full_attn(const ptdit_shape *shape, const ptdit_attn_w *w, unsigned flags,
+                    const void *z_in, void *z_out, void *ws, size_t ws_bytes,
+                    ptdit_stream_t stream);
+
+/* ptdit_strerror -- static text for a status code. */
+const char *ptdit_strerror(int status);
+
+/* ptdit_last_error -- description of this host thread's last failed call. */
+const char *ptdit_last_error(void);
+
+/*
+ * Debug index maps, computed on the device by the same address functions the
+ * kernels use (for bit-exact comparison with an independent derivation).
+ *   ptdit_debug_proxy_map: proxy_of_token[N] (device int32).
+ *   ptdit_debug_window_map: token_at_slot[nW * n] (device int32), the
+ *     original token index at each (window, slot) of the rolled grid, windows
+ *     and slots row-major; allowed[nW * n * n] (device uint8, may be NULL),
+ *     1 where slot i may attend slot j of the same window.
+ */
+int ptdit_debug_proxy_map(const int grid[3], const int ratio[3], int32_t *proxy_of_token,
+                          ptdit_stream_t stream);
+int ptdit_debug_window_map(const int grid[3], const int window[3], const int shift[3],
+                           int32_t *token_at_slot, uint8_t *allowed, ptdit_stream_t stream);
+
+/*
+ * Kernel timing for measurement.  ptdit_timing_enable(n) makes the calling
+ * host thread's later calls record a CUDA event pair around each kernel
+ * launch on the launching stream, up to n launches (0 turns it off and
+ * frees the events).  ptdit_timing_read() synchronises on the recorded
+ * events, writes up to `max` (kind, milliseconds) pairs and clears the list;
+ * it returns the count, or -1 on error.  Kinds are PTDIT_K_*.
+ */
+enum {
+    PTDIT_K_AVERAGE = 0,   /* window averaging */
+    PTDIT_K_GEMM = 1,      /* QKV / O projections */
+    PTDIT_K_ATTN_PROXY = 2,/* proxy self-attention core */
+    PTDIT_K_ATTN_CROSS = 3,/* latent -> proxy cross-attention core */
+    PTDIT_K_ATTN_WINDOW = 4,/* window / shifted-window attention core */
+    PTDIT_K_ATTN_DENSE = 5,/* full self-attention core */
+    PTDIT_K_COUNT = 6
+};
+int ptdit_timing_enable(int max_launches);
+int ptdit_timing_read(int *kind, float *ms, int max);
+
+/* ptdit_launch_count -- kernels this host thread has launched through the library. */
+long long ptdit_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PTDIT_H */

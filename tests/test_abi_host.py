@@ -1,0 +1,135 @@
+"""Host-side tests of the C ABI: runs without a GPU.
+
+The library must load, export every function include/ptdit.h declares, size
+its workspace, and reject invalid arguments with a status code before it
+touches CUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import diffusion_transformer_sparse_b200 as pt
+from diffusion_transformer_sparse_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return pt.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "ptdit.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ptdit_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 14
+    assert set(names) == set(pt.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+    # nm agrees: the symbols are real dynamic exports with C linkage
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", pt.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    for n in names:
+        assert re.search(rf"\bT {n}$", out, re.M), n
+
+
+def test_strerror(L):
+    for code in range(9):
+        assert L.ptdit_strerror(code)
+    assert L.ptdit_strerror(0) == b"ok"
+
+
+def _shape(**kw):
+    d = dict(B=1, F=1, H=16, W=16, D=64, heads=2, dtype=pt.PTDIT_F32)
+    d.update(kw)
+    return pt.Shape(**d)
+
+
+def _bytes(L, shape, ratio, window):
+    return L.ptdit_workspace_bytes(ctypes.byref(shape), pt._i3(ratio), pt._i3(window))
+
+
+def test_workspace_bytes(L):
+    s = _shape(B=4, H=64, W=64, D=1152, heads=16, dtype=pt.PTDIT_BF16)
+    N, M, D, e = 4096, 256, 1152, 2
+
+    def a(x):
+        return (x + 255) // 256 * 256
+
+    want = 8 * a(4 * M * D * e) + 4 * a(4 * N * D * e)
+    assert _bytes(L, s, (1, 4, 4), (1, 8, 8)) == want
+    assert _bytes(L, s, None, (1, 8, 8)) == 4 * a(4 * N * D * e)
+    assert _bytes(L, s, (1, 3, 4), (1, 8, 8)) == 0      # 64 not divisible by 3
+    assert _bytes(L, s, (1, 4, 4), (1, 8, 7)) == 0
+    assert _bytes(L, _shape(D=63, heads=2), None, None) == 0
+
+
+FAKE = 1 << 20  # an aligned non-null address that is never dereferenced: validation fails first
+
+
+def _w(p=FAKE):
+    return pt.AttnW(p, p + 4096, p + 8192, p + 12288)
+
+
+def _block(L, shape, ratio=(1, 2, 2), window=(1, 4, 4), shift=(0, 2, 2), w=None, flags=0,
+           z_in=FAKE, z_out=FAKE * 64, ws=FAKE * 128, ws_bytes=1 << 40):
+    w = w or _w()
+    return L.ptdit_block_attn(ctypes.byref(shape) if shape is not None else None,
+                              pt._i3(ratio), pt._i3(window), pt._i3(shift), ctypes.byref(w),
+                              ctypes.byref(w), ctypes.byref(w), ctypes.byref(w), flags, z_in,
+                              z_out, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(shape=None), 1),
+    (dict(ratio=None), 1),
+    (dict(shift=None), 1),
+    (dict(ratio=(1, 3, 2)), 2),
+    (dict(window=(1, 5, 4)), 2),
+    (dict(shift=(0, 4, 2)), 2),
+    (dict(shift=(0, -1, 2)), 2),
+    (dict(z_in=0), 1),
+    (dict(z_out=FAKE + 8), 7),
+    (dict(ws_bytes=1024), 4),
+    (dict(z_out=FAKE + 4096), 8),
+    (dict(ws=FAKE * 64 + 256), 8),
+    (dict(w=pt.AttnW(FAKE, 0, FAKE, FAKE)), 1),
+])
+def test_block_attn_rejects(L, kw, code):
+    shape = kw.pop("shape", _shape())
+    assert _block(L, shape, **kw) == code
+    assert L.ptdit_last_error()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=7), 3),
+    (dict(D=65, heads=2), 2),
+    (dict(D=1024, heads=4), 2),   # head dim 256
+    (dict(B=0), 2),
+    (dict(H=0), 2),
+])
+def test_shape_rejects(L, kw, code):
+    assert _block(L, _shape(**kw)) == code
+
+
+def test_debug_maps_reject(L):
+    out = FAKE
+    assert L.ptdit_debug_window_map(pt._i3((1, 4, 4)), pt._i3((1, 3, 2)), pt._i3((0, 0, 0)),
+                                    out, None, None) == 2
+    assert L.ptdit_debug_proxy_map(pt._i3((1, 4, 4)), pt._i3((1, 2, 2)), None, None) == 1
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(pt, "_lib", None)
+    monkeypatch.setattr(pt, "LIB_PATH", "/nonexistent/libptdit.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        pt.lib()

@@ -1,0 +1,237 @@
+"""GPU parity: the CUDA library against the float64 oracle, element by element.
+
+Small cases span several tiles and ragged tails and are compared in full;
+the five workloads at full size are compared on sampled rows computed by the
+oracle's dependency closure, in the same launch configuration the bench times.
+Index maps are compared bit-exact.  Tolerance: max|gpu - oracle| / max|oracle|
+<= 1e-4 (fp32) or 2e-2 (bf16) per output tensor, with the residual on and off.
+"""
+import numpy as np
+import pytest
+import torch
+
+import diffusion_transformer_sparse_b200 as pt
+import oracle as O
+from diffusion_transformer_sparse_b200 import build
+from diffusion_transformer_sparse_b200.configs import WORKLOADS
+from tests.helpers import TOL, Case, rel_err, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    pt.lib()
+
+
+# ---------------------------------------------------------------- index maps (bit-exact)
+
+@pytest.mark.parametrize("grid,ratio", [((1, 16, 16), (1, 2, 2)), ((1, 64, 64), (1, 4, 4)),
+                                        ((16, 32, 48), (1, 4, 4)), ((4, 8, 12), (2, 4, 3)),
+                                        ((32, 64, 64), (1, 16, 16)), ((3, 5, 7), (1, 1, 1)),
+                                        ((2, 4, 6), (2, 4, 6))])
+def test_proxy_map_bit_exact(grid, ratio):
+    got = pt.ptdit_debug_proxy_map(grid, ratio).cpu().numpy()
+    np.testing.assert_array_equal(got, O.proxy_index(grid, ratio))
+
+
+@pytest.mark.parametrize("grid,window,shift", [
+    ((1, 16, 16), (1, 4, 4), (0, 2, 2)), ((1, 64, 64), (1, 8, 8), (0, 4, 4)),
+    ((16, 32, 48), (2, 8, 8), (1, 4, 4)), ((4, 8, 12), (2, 4, 3), (1, 3, 1)),
+    ((2, 6, 10), (2, 3, 5), (1, 1, 4)), ((1, 16, 16), (1, 16, 16), (0, 0, 0)),
+    ((1, 4, 4), (1, 2, 2), (0, 1, 1)),
+])
+def test_window_map_bit_exact(grid, window, shift):
+    tok, allowed = pt.ptdit_debug_window_map(grid, window, shift)
+    tmap = O.window_token_map(grid, window, shift)
+    np.testing.assert_array_equal(tok.cpu().numpy().reshape(tmap.shape), tmap)
+    lab = O.window_region_labels(grid, window, shift)
+    want = lab[:, :, None] == lab[:, None, :]
+    np.testing.assert_array_equal(allowed.cpu().numpy().reshape(want.shape).astype(bool), want)
+
+
+# ---------------------------------------------------------------- averaging
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B,grid,D,ratio", [
+    (1, (1, 16, 16), 64, (1, 2, 2)), (2, (4, 8, 12), 40, (2, 4, 3)), (1, (2, 6, 10), 1152, (1, 3, 5)),
+    (4, (1, 64, 64), 1152, (1, 4, 4)), (1, (3, 8, 8), 24, (3, 8, 8)), (1, (2, 4, 4), 36, (1, 1, 1)),
+    (1, (1, 8, 8), 2100, (1, 2, 2)),
+])
+def test_proxy_average(dtype, B, grid, D, ratio):
+    c = Case(B, grid, D, 1, dtype)
+    got = c.out64(pt.ptdit_proxy_average(c.z, grid, ratio))
+    # fp32: P summands of unit size lose at most ~P * 2^-24 of the largest mean
+    # (1e-5 covers P = 192); bf16 adds one output rounding of 2^-9 relative.
+    for b in range(B):
+        err = rel_err(got[b], O.averaging(c.z64[b], grid, ratio))
+        assert err <= (1e-5 if dtype == "f32" else 4e-3), err
+
+
+def test_proxy_average_is_deterministic():
+    c = Case(1, (1, 128, 128), 1152, 1, "bf16")
+    a = pt.ptdit_proxy_average(c.z, c.grid, (1, 8, 8))
+    b = pt.ptdit_proxy_average(c.z, c.grid, (1, 8, 8))
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- modules on small grids
+
+SMALL = [
+    # B, grid, D, heads, ratio, window, shift
+    (1, (1, 16, 16), 64, 2, (1, 2, 2), (1, 4, 4), (0, 2, 2)),
+    (2, (2, 8, 8), 48, 3, (1, 4, 2), (2, 4, 4), (1, 2, 2)),
+    (1, (4, 8, 12), 96, 4, (2, 2, 3), (2, 4, 3), (1, 1, 2)),
+    (1, (1, 24, 24), 144, 2, (1, 3, 3), (1, 8, 8), (0, 4, 4)),
+    (1, (2, 16, 16), 1152, 16, (1, 4, 4), (2, 8, 8), (1, 4, 4)),
+]
+
+
+def _oracle_branch(c, b, which, window, shift, ratio, flags):
+    z = c.z64[b]
+    if which == "giim":
+        return O.giim(z, c.grid, ratio, c.w64["psa"], c.w64["cross"], c.heads,
+                      proxy_residual=bool(flags & pt.PTDIT_PROXY_RESIDUAL),
+                      residual=not flags & pt.PTDIT_NO_RESIDUAL)
+    return O.window_self_attention(z, c.grid, window, shift, c.w64["wsa"], c.heads,
+                                   residual=not flags & pt.PTDIT_NO_RESIDUAL)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", SMALL)
+@pytest.mark.parametrize("flags", [0, pt.PTDIT_NO_RESIDUAL,
+                                   pt.PTDIT_NO_RESIDUAL | pt.PTDIT_PROXY_RESIDUAL])
+def test_giim_small(dtype, case, flags):
+    B, grid, D, heads, ratio, window, shift = case
+    c = Case(B, grid, D, heads, dtype)
+    out = c.out64(pt.ptdit_giim(c.z, grid, ratio, c.w["psa"], c.w["cross"], heads, flags))
+    for b in range(B):
+        assert rel_err(out[b], _oracle_branch(c, b, "giim", None, None, ratio, flags)) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", SMALL)
+@pytest.mark.parametrize("shifted", [False, True])
+@pytest.mark.parametrize("flags", [0, pt.PTDIT_NO_RESIDUAL])
+def test_window_attn_small(dtype, case, shifted, flags):
+    B, grid, D, heads, ratio, window, shift = case
+    shift = shift if shifted else (0, 0, 0)
+    c = Case(B, grid, D, heads, dtype)
+    out = c.out64(pt.ptdit_window_attn(c.z, grid, window, shift, c.w["wsa"], heads, flags))
+    for b in range(B):
+        want = _oracle_branch(c, b, "win", window, shift, None, flags)
+        assert rel_err(out[b], want) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", SMALL[:4])
+def test_block_attn_small(dtype, case):
+    B, grid, D, heads, ratio, window, shift = case
+    c = Case(B, grid, D, heads, dtype)
+    out = c.out64(pt.ptdit_block_attn(c.z, grid, ratio, window, shift, c.w["psa"], c.w["cross"],
+                                      c.w["wsa"], c.w["swsa"], heads))
+    for b in range(B):
+        want = O.block_attn(c.z64[b], grid, ratio, window, shift, c.w64["psa"], c.w64["cross"],
+                            c.w64["wsa"], c.w64["swsa"], heads)
+        assert rel_err(out[b], want) <= TOL[dtype]
+    tcm = c.out64(pt.ptdit_tcm(c.z, grid, window, shift, c.w["wsa"], c.w["swsa"], heads,
+                               pt.PTDIT_NO_RESIDUAL))
+    for b in range(B):
+        want = O.tcm(c.z64[b], grid, window, shift, c.w64["wsa"], c.w64["swsa"], heads,
+                     residual=False)
+        assert rel_err(tcm[b], want) <= TOL[dtype]
+
+
+# ---------------------------------------------------------------- degenerate cases of the method
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_single_window_broadcasts(dtype):
+    """ratio = grid: one proxy, so every latent receives the same cross-attention vector."""
+    grid = (2, 8, 8)
+    c = Case(1, grid, 64, 2, dtype)
+    out = pt.ptdit_giim(c.z, grid, grid, c.w["psa"], c.w["cross"], 2, pt.PTDIT_NO_RESIDUAL)
+    o = c.out64(out)[0]
+    assert np.all(o == o[0:1])  # bit-identical rows
+    want = O.giim(c.z64[0], grid, grid, c.w64["psa"], c.w64["cross"], 2, residual=False)
+    assert rel_err(o, want) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_ratio_111_and_full_window(dtype):
+    grid = (1, 8, 16)
+    c = Case(1, grid, 64, 2, dtype)
+    out = c.out64(pt.ptdit_giim(c.z, grid, (1, 1, 1), c.w["psa"], c.w["cross"], 2))
+    want = O.giim(c.z64[0], grid, (1, 1, 1), c.w64["psa"], c.w64["cross"], 2)
+    assert rel_err(out[0], want) <= TOL[dtype]
+    # window = grid is full self-attention, and so is the dense comparator
+    a = c.out64(pt.ptdit_window_attn(c.z, grid, grid, (0, 0, 0), c.w["wsa"], 2))
+    f = c.out64(pt.ptdit_full_attn(c.z, grid, c.w["wsa"], 2))
+    want = O.masked_self_attention(c.z64[0], c.w64["wsa"], 2, np.ones((128, 128), bool))
+    assert rel_err(a[0], want) <= TOL[dtype]
+    assert rel_err(f[0], want) <= TOL[dtype]
+
+
+def test_block_attn_is_deterministic():
+    w = WORKLOADS["tiny_16x16_f32"].with_(dtype="bf16", D=144, heads=2)
+    c = Case(2, w.grid, w.D, w.heads, "bf16")
+    args = (w.grid, w.ratio, w.window, w.shift, c.w["psa"], c.w["cross"], c.w["wsa"],
+            c.w["swsa"], w.heads)
+    a = pt.ptdit_block_attn(c.z, *args)
+    b = pt.ptdit_block_attn(c.z, *args)
+    assert torch.equal(a, b)
+
+
+def test_rejects_invalid_on_device_tensors():
+    c = Case(1, (1, 16, 16), 64, 2, "f32")
+    with pytest.raises(pt.PtditError) as e:
+        pt.ptdit_window_attn(c.z, (1, 16, 16), (1, 5, 4), (0, 0, 0), c.w["wsa"], 2)
+    assert e.value.code == 2
+    with pytest.raises(pt.PtditError) as e:
+        pt.ptdit_window_attn(c.z, (1, 16, 16), (1, 4, 4), (0, 0, 0), c.w["wsa"], 2, z_out=c.z)
+    assert e.value.code == 8
+
+
+# ---------------------------------------------------------------- the five workloads, full size
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workload_block_attn(name):
+    w = WORKLOADS[name]
+    c = Case(w.B, w.grid, w.D, w.heads, w.dtype)
+    out = pt.ptdit_block_attn(c.z, w.grid, w.ratio, w.window, w.shift, c.w["psa"], c.w["cross"],
+                              c.w["wsa"], c.w["swsa"], w.heads)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.grid, k=4, seed=len(name))
+    for b in range(w.B):
+        got = out[b, torch.from_numpy(rows).cuda()].double().cpu().numpy()
+        if w.N <= 4096 and w.dtype == "f32":
+            want = O.block_attn(c.z64[b], w.grid, w.ratio, w.window, w.shift, c.w64["psa"],
+                                c.w64["cross"], c.w64["wsa"], c.w64["swsa"], w.heads)[rows]
+        else:
+            want = O.block_attn_rows(c.z64[b], w.grid, w.ratio, w.window, w.shift, c.w64["psa"],
+                                     c.w64["cross"], c.w64["wsa"], c.w64["swsa"], w.heads, rows)
+        assert rel_err(got, want) <= TOL[w.dtype], (name, b)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS)[1:4])
+def test_workload_branches_without_residual(name):
+    """Each branch alone at full size, so residual rounding cannot hide a small branch."""
+    w = WORKLOADS[name]
+    c = Case(1, w.grid, w.D, w.heads, w.dtype)
+    rows = sample_rows(w.grid, k=4, seed=3)
+    idx = torch.from_numpy(rows).cuda()
+    g = pt.ptdit_giim(c.z[:1], w.grid, w.ratio, c.w["psa"], c.w["cross"], w.heads,
+                      pt.PTDIT_NO_RESIDUAL)
+    want = O.giim(c.z64[0], w.grid, w.ratio, c.w64["psa"], c.w64["cross"], w.heads,
+                  residual=False, rows=rows)[rows]
+    assert rel_err(g[0, idx].double().cpu().numpy(), want) <= TOL[w.dtype]
+    for shift in [(0, 0, 0), w.shift]:
+        a = pt.ptdit_window_attn(c.z[:1], w.grid, w.window, shift, c.w["swsa"], w.heads,
+                                 pt.PTDIT_NO_RESIDUAL)
+        smap = O.window_token_map(w.grid, w.window, shift)
+        win_of = np.empty(w.N, np.int64)
+        win_of[smap.ravel()] = np.repeat(np.arange(smap.shape[0]), smap.shape[1])
+        wins = np.unique(win_of[rows])
+        want = O.window_self_attention(c.z64[0], w.grid, w.window, shift, c.w64["swsa"], w.heads,
+                                       residual=False, windows=wins)[rows]
+        assert rel_err(a[0, idx].double().cpu().numpy(), want) <= TOL[w.dtype]
