@@ -23,7 +23,7 @@ EXPORTS = (
     "ptdit_proxy_average", "ptdit_workspace_bytes", "ptdit_giim", "ptdit_window_attn",
     "ptdit_tcm", "ptdit_block_attn", "ptdit_full_attn", "ptdit_strerror", "ptdit_last_error",
     "ptdit_debug_proxy_map", "ptdit_debug_window_map", "ptdit_timing_enable",
-    "ptdit_timing_read", "ptdit_launch_count",
+    "ptdit_timing_read", "ptdit_launch_count", "ptdit_window_attn_static",
 )
 
 
@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
             "ptdit_timing_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
                                                  ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
             "ptdit_launch_count": (ctypes.c_longlong, []),
+            "ptdit_window_attn_static": (ctypes.c_int, [_S, _I3, _I3, _W, ctypes.c_uint, _P, _P,
+                                                        _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)

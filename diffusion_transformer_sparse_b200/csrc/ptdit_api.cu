@@ -371,6 +371,11 @@ int check_w_alias(const Dims &d, const ptdit_attn_w *w, const void *z_out) {
 
 }  // namespace
 
+namespace ptdit {
+// Records a failure for ptdit_last_error() from another translation unit.
+int report_error(int code, const char *text) { return fail(code, "%s", text); }
+}  // namespace ptdit
+
 // ------------------------------------------------------------------ exported API
 extern "C" {
 

@@ -121,6 +121,29 @@ int ptdit_window_attn(const ptdit_shape *shape, const int window[3], const int s
                       void *ws, size_t ws_bytes, ptdit_stream_t stream);
 
 /*
+ * ptdit_window_attn_static -- ptdit_window_attn without a workspace argument,
+ *   for callers that cannot allocate device memory: code that runs where
+ *   cudaMalloc is not allowed or must not be called (it can synchronise the
+ *   device), or that only receives input and output buffers from a host
+ *   framework whose allocator it cannot reach.  The paper has no counterpart;
+ *   this is a packaging of the same computation.
+ *   Scratch is a static device array of PTDIT_STATIC_SCRATCH_BYTES inside the
+ *   library (enough for one 64x64-token grid at D = 1152 in bf16); every GPU
+ *   that loads the library's device code holds it until the process exits.  The caller still
+ *   passes z_in and z_out.  A shape whose workspace (ptdit_workspace_bytes
+ *   with ratio NULL) exceeds the maximum returns PTDIT_ERR_WORKSPACE and
+ *   launches nothing.  Nothing is allocated: no cudaMalloc, no cudaFree.
+ *   The first call on a device looks up the array's device address with
+ *   cudaGetSymbolAddress (and may load the library's device code), so make
+ *   it before any stream capture.  All calls share the one array: calls that
+ *   overlap on the GPU (unordered streams or host threads) race.
+ */
+#define PTDIT_STATIC_SCRATCH_BYTES (40u << 20)
+int ptdit_window_attn_static(const ptdit_shape *shape, const int window[3], const int shift[3],
+                             const ptdit_attn_w *w, unsigned flags, const void *z_in,
+                             void *z_out, ptdit_stream_t stream);
+
+/*
  * ptdit_tcm -- Eq. TCM: WSA with weights wsa, then SWSA with weights swsa
  *   and the given shift, each with its residual (unless PTDIT_NO_RESIDUAL).
  */
