@@ -270,6 +270,17 @@ def run_gpu(args, w):
     value = world * args.steps * w.B * w.N / (total_ms / 1e3)
     ms_step = total_ms / args.steps
 
+    if args.kernels_only:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                              "config": config_of(w), "gpu_launches": launches,
+                              "note": "--kernels-only: timed region only, for profiling"}),
+                  flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
     # per-kernel durations: the same K steps with the library's event hooks on
     pt.ptdit_timing_enable(64 * args.steps)
     hooked = timed(args.steps, step)
@@ -353,6 +364,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernels-only", action="store_true",
+                    help="stop after the timed region (no hook, e2e or CPU passes): for ncu")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     w = configs.WORKLOADS[args.workload]
