@@ -71,9 +71,9 @@ __device__ __forceinline__ Slot slot_of(const AttnArgs &a, int b, int tile, int 
         int win, slot, wit;
         if (g.n <= BQ) {
             const int pack = BQ / g.n;
-            wit = r / g.n;
+            wit = fdiv(g.f_n, r);
             win = tile * pack + wit;
-            slot = r % g.n;
+            slot = r - wit * g.n;
             if (win >= g.nwin) return s;
         } else {
             const int per = g.n / BQ;
@@ -93,6 +93,13 @@ __device__ __forceinline__ Slot slot_of(const AttnArgs &a, int b, int tile, int 
         }
     }
     return s;
+}
+
+__device__ __forceinline__ bool wait_and_fence(uint64_t *bar, uint32_t parity,
+                                               volatile int *abort, int *status) {
+    const bool ok = mbar_wait(bar, parity, abort, status);
+    fence_before_sync();
+    return ok;
 }
 
 // 16-byte chunks [c0, c1) of one row into a chunk-major tile (zero-fill for an empty slot).
@@ -197,8 +204,9 @@ __global__ void __launch_bounds__(kThreads, 3) attn_tc_kernel(AttnArgs a, int n_
                 const uint32_t bits = __ballot_sync(0xffffffffu, k.info == v);
                 if (lane == 0) kmask[v * 4 + warp] = bits;
             }
-        // the decision to go on is the same for every thread of the CTA
-        ok = __syncthreads_and(mbar_wait(bar_s, phase, abort, status));
+        // one thread waits; the barrier hands its verdict (and the tcgen05
+        // completion it observed) to the whole CTA
+        ok = __syncthreads_and(t == 0 ? wait_and_fence(bar_s, phase, abort, status) : true);
         if (!ok) break;
         fence_after_sync();
 
@@ -284,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 3) attn_tc_kernel(AttnArgs a, int n_
                          sdesc_interleave(aV + ks * 256, 128, CHUNK), idesc, ks > 0);
             mma_commit(bar_o);
         }
-        ok = __syncthreads_and(mbar_wait(bar_o, phase, abort, status));
+        ok = __syncthreads_and(t == 0 ? wait_and_fence(bar_o, phase, abort, status) : true);
         if (!ok) break;
         fence_after_sync();
         {

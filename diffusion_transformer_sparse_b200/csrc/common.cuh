@@ -9,6 +9,32 @@
 namespace ptdit {
 
 // ---------------------------------------------------------------------------
+// Division by a runtime-invariant divisor d >= 1, for numerators below 2^31:
+// q = umulhi(2n, m) >> s with s = ceil(log2 d) and m = ceil(2^(31+s) / d)
+// (Granlund & Montgomery, "Division by Invariant Integers using
+// Multiplication", PLDI 1994).  The index maps divide by grid and window
+// extents on every row address, so this replaces ~20-instruction divides.
+// ---------------------------------------------------------------------------
+struct FastDiv {
+    uint32_t d, m, s;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t s = 0;
+    while ((1ull << s) < d) ++s;
+    const uint64_t m = ((1ull << (31 + s)) + d - 1) / d;
+    return FastDiv{d, static_cast<uint32_t>(m), s};
+}
+
+__host__ __device__ __forceinline__ uint32_t fdiv(const FastDiv &f, uint32_t n) {
+#ifdef __CUDA_ARCH__
+    return __umulhi(n << 1, f.m) >> f.s;
+#else
+    return static_cast<uint32_t>((static_cast<uint64_t>(n << 1) * f.m) >> 32) >> f.s;
+#endif
+}
+
+// ---------------------------------------------------------------------------
 // Token grid and index maps
 //
 // Tokens are flattened row-major over the (f, h, w) grid (Qihoo-T2X reading
@@ -23,12 +49,15 @@ struct ProxyGeom {
     int pf, ph, pw;   // proxy ratio
     int mf, mh, mw;   // windows per axis
     int M, P;         // proxies, tokens per proxy window
+    FastDiv f_mw, f_mh, f_pw, f_ph;
 };
 
 __host__ __device__ __forceinline__ int proxy_token(const ProxyGeom &g, int m, int k) {
     // k-th token (row-major inside the window) of proxy window m
-    int X = m % g.mw, r = m / g.mw, Y = r % g.mh, T = r / g.mh;
-    int c = k % g.pw, q = k / g.pw, b = q % g.ph, a = q / g.ph;
+    const int r = fdiv(g.f_mw, m), X = m - r * g.mw;
+    const int T = fdiv(g.f_mh, r), Y = r - T * g.mh;
+    const int q = fdiv(g.f_pw, k), c = k - q * g.pw;
+    const int a = fdiv(g.f_ph, q), b = q - a * g.ph;
     return ((T * g.pf + a) * g.h + Y * g.ph + b) * g.w + X * g.pw + c;
 }
 
@@ -45,6 +74,7 @@ struct WinGeom {
     int sf, sh, sw;   // shift: window origin of the rolled grid is token (s_f, s_h, s_w)
     int nwf, nwh, nww;// windows per axis
     int n, nwin;      // tokens per window, windows per batch item
+    FastDiv f_ww, f_wh, f_nww, f_nwh, f_n;
 };
 
 // Original token index held by slot `slot` of rolled-grid window `win`.
@@ -53,8 +83,10 @@ struct WinGeom {
 // other iff their wrap bits are equal: the shift mask is this comparison.
 __host__ __device__ __forceinline__ int window_token(const WinGeom &g, int win, int slot,
                                                      int *wrap) {
-    int wx = win % g.nww, r = win / g.nww, wy = r % g.nwh, wt = r / g.nwh;
-    int sx = slot % g.ww, q = slot / g.ww, sy = q % g.wh, st = q / g.wh;
+    const int r = fdiv(g.f_nww, win), wx = win - r * g.nww;
+    const int wt = fdiv(g.f_nwh, r), wy = r - wt * g.nwh;
+    const int q = fdiv(g.f_ww, slot), sx = slot - q * g.ww;
+    const int st = fdiv(g.f_wh, q), sy = q - st * g.wh;
     int t = wt * g.wf + st + g.sf;
     int y = wy * g.wh + sy + g.sh;
     int x = wx * g.ww + sx + g.sw;

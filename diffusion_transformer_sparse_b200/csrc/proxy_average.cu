@@ -6,10 +6,11 @@
 //
 // The kernel is a pure HBM stream: it reads every latent element once and
 // writes every proxy element once.  One CTA owns one proxy; its threads are
-// (16-byte channel chunk) x (token group).  A warp reads 512 contiguous bytes
-// of one token row per load, each thread keeps several independent 16-byte
-// loads in flight, and the token groups are summed through shared memory in
-// a fixed order, so the result is bitwise deterministic.
+// (16-byte channel chunk) x (token group), about 8 tokens per group.  A warp
+// reads 512 contiguous bytes of one token row per load, each thread issues
+// all its (up to 8) independent 16-byte loads before the first add, and the
+// token groups are summed through shared memory in a fixed order, so the
+// result is bitwise deterministic.
 #include "common.cuh"
 
 namespace ptdit {
@@ -83,13 +84,22 @@ __global__ void __launch_bounds__(1024) proxy_average_kernel(const T *__restrict
         for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
         if (gi < G && c < CH) {
             const T *zb = zw + (long)c * VEC;
-            // token k of the window sits (a*h + r)*w + q tokens after the first one
-#pragma unroll 4
-            for (int k = gi; k < g.P; k += G) {
-                int q = k % g.pw, rest = k / g.pw, r = rest % g.ph, a = rest / g.ph;
-                Chunk<T, VEC> ch;
-                ch.load(zb + ((long)(a * g.h + r) * g.w + q) * D);
-                ch.add_to(acc);
+            // token k of the window sits (a*h + r)*w + q tokens after the first one;
+            // each batch issues up to 8 independent 16-byte loads before adding
+            for (int k0 = gi; k0 < g.P; k0 += 8 * G) {
+                Chunk<T, VEC> ch[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int k = k0 + u * G;
+                    if (k < g.P) {
+                        const int rest = fdiv(g.f_pw, k), q = k - rest * g.pw;
+                        const int a = fdiv(g.f_ph, rest), r = rest - a * g.ph;
+                        ch[u].load(zb + ((long)(a * g.h + r) * g.w + q) * D);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (k0 + u * G < g.P) ch[u].add_to(acc);
             }
         }
         if (gi > 0 && gi < G) {
@@ -116,9 +126,10 @@ cudaError_t launch_avg(const ProxyGeom &g, int B, int D, const void *z, void *ou
                        cudaStream_t s) {
     const int CH = D / VEC;
     const int CHT = CH < 512 ? CH : 512;
-    int G = 512 / CHT;
+    // token groups: about 8 loads per thread, at most 1024 threads per CTA
+    int G = (g.P + 7) / 8;
+    if (G > 1024 / CHT) G = 1024 / CHT;
     if (G < 1) G = 1;
-    if (G > g.P) G = g.P;
     const int threads = CHT * G;
     const size_t smem = (size_t)(G - 1) * CHT * VEC * sizeof(float);
     proxy_average_kernel<T, VEC><<<(unsigned)(B * g.M), threads, smem, s>>>(

@@ -128,6 +128,10 @@ int make_proxy(const Dims &d, const int ratio[3], ProxyGeom *g) {
     g->mf = d.f / ratio[0]; g->mh = d.h / ratio[1]; g->mw = d.w / ratio[2];
     g->M = g->mf * g->mh * g->mw;
     g->P = ratio[0] * ratio[1] * ratio[2];
+    g->f_mw = make_fastdiv(g->mw);
+    g->f_mh = make_fastdiv(g->mh);
+    g->f_pw = make_fastdiv(g->pw);
+    g->f_ph = make_fastdiv(g->ph);
     return PTDIT_OK;
 }
 
@@ -149,6 +153,11 @@ int make_window(const Dims &d, const int window[3], const int shift[3], WinGeom 
     g->nwf = d.f / window[0]; g->nwh = d.h / window[1]; g->nww = d.w / window[2];
     g->n = window[0] * window[1] * window[2];
     g->nwin = g->nwf * g->nwh * g->nww;
+    g->f_ww = make_fastdiv(g->ww);
+    g->f_wh = make_fastdiv(g->wh);
+    g->f_nww = make_fastdiv(g->nww);
+    g->f_nwh = make_fastdiv(g->nwh);
+    g->f_n = make_fastdiv(g->n);
     return PTDIT_OK;
 }
 
