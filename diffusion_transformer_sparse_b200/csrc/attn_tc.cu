@@ -1,6 +1,7 @@
-// Attention core on the 5th-generation tensor cores: window / shifted-window
-// self-attention (TCM), proxy self-attention and latent -> proxy
-// cross-attention (GIIM), and full self-attention (the dense comparator).
+// Window attention core on the 5th-generation tensor cores: window and
+// shifted-window self-attention of TCM.  (Row-mode attention -- proxy SA,
+// cross-attention, full SA -- is the warp-specialised kernel of
+// attn_rows_tc.cu; this file dispatches to it.)
 //
 // Qihoo-T2X reading note, §3 Method: Eq. GIIM (SA among the proxies, CS with
 // every latent the query and the proxies keys/values) and Eq. TCM (WSA, and
@@ -390,7 +391,14 @@ bool attention_tc_supported(const AttnArgs &a) {
     return a.nq >= 1 && a.nk >= 1;
 }
 
+cudaError_t launch_attention_rows_tc(const AttnArgs &a, cudaStream_t s);
+
 cudaError_t launch_attention_tc(const AttnArgs &a, cudaStream_t s) {
+    if (a.mode == ATT_ROWS) {
+        const cudaError_t e = launch_attention_rows_tc(a, s);
+        if (e != cudaErrorNotSupported) return e;
+        (void)cudaGetLastError();  // tensor maps rejected: use the gather kernel below
+    }
     switch (dpad_of(a.d)) {
         case 64: return launch_dpad<64>(a, s);
         case 80: return launch_dpad<80>(a, s);

@@ -50,6 +50,21 @@ bool encode_map_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint
     return r == CUDA_SUCCESS;
 }
 
+bool encode_map_rows_heads_bf16(CUtensorMap *map, const void *base, uint64_t rows,
+                                uint64_t row_pitch_bytes, int nch, int heads, int d,
+                                uint32_t box_rows, uint32_t box_chunks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {8, rows, (cuuint64_t)nch, (cuuint64_t)heads};
+    cuuint64_t strides[3] = {row_pitch_bytes, 16, (cuuint64_t)d * 2};
+    cuuint32_t box[4] = {8, box_rows, box_chunks, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
