@@ -5,23 +5,26 @@
 // each batch item; head h is columns h*d .. h*d+d-1.
 //
 // FlashAttention-style warp specialisation, one persistent CTA per SM:
-//   warp 0       loader: one TMA load per 128-row tile -- two query tiles
-//                per unit, K and V tiles into a two-stage ring.  A 4-D tensor
-//                map (8 elements, rows, 16-byte chunks, heads) writes each tile
-//                straight into the chunk-major layout below and zero-fills the
-//                padded chunk.
-//   warp 1       MMA issuer: S0 = Q0 K^T and S1 = Q1 K^T into TMEM, then
-//                P0 V and P1 V into TMEM once each softmax has written P.
+//   warp 0       loader: TMA loads of two 128-row query tiles per unit (double
+//                buffered across units) and of K and V tiles into a two-stage
+//                ring.  A head's 72 columns arrive as a 64-column box with the
+//                128-byte swizzle plus a 16-column box with the 32-byte swizzle
+//                whose last 8 columns lie past the head and read as zeros: the
+//                zero padding of d to 80 comes for free.
+//   warp 1       MMA issuer: S_g = Q_g K^T (K-major operands) into TMEM, and
+//                once softmax g has written P_g, P_g V with P_g read straight
+//                from TMEM and V as an MN-major operand (no transpose),
+//                accumulating into O_g in TMEM.
 //   warps 4-7 and 8-11   two softmax warpgroups, one per query tile: thread r
-//                owns row r (its TMEM lane), reads S with tcgen05.ld, runs the
-//                fp32 online softmax and writes P (bf16) to shared memory; the
-//                P V products accumulate in TMEM, rescaled in place only when
-//                a row's reference max has to rise.
-// Both query tiles share every K/V tile, and while one warpgroup runs its
-// softmax the tensor core works for the other.  Shared memory layout: 16-byte
-// chunks major, byte (chunk c, row r) = c * 2048 + r * 16 (the no-swizzle
-// core-matrix layout: K-major for Q, K and P, MN-major for V); d is padded
-// with zeros to a multiple of 16.  Every wait is bounded (2 s).
+//                owns row r (its TMEM lane), reads its 128 scores with one
+//                wait, runs the fp32 online softmax and writes P (bf16, two per
+//                column) back over the first 64 columns of its scores; O is
+//                rescaled in TMEM only when a row's reference max has to rise
+//                by more than 2^8.  P never touches shared memory, which
+//                leaves room for a three-stage K/V ring.
+// Both query tiles share every K/V tile; the MMA warp issues PV_0, S_0(next),
+// PV_1, S_1(next), so each softmax gets its next scores while the other one
+// works.  Every wait is bounded (2 s).
 #include <math.h>
 
 #include "tc_util.cuh"
@@ -32,23 +35,31 @@ namespace {
 using namespace tc;
 
 constexpr int BQ = 128, BKV = 128;
-constexpr uint32_t CHUNK = BQ * 16;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;  // S0, S1, O0, O1: 128 columns each
 
+constexpr int NSTAGE = 2;  // K/V ring depth
+
 template <int DPAD>
 struct RowsLayout {
-    static constexpr int TILE = BQ * DPAD * 2;
-    static constexpr int P_BYTES = BQ * BKV * 2;
-    static constexpr int OFF_Q = 0;             // Q0, Q1
-    static constexpr int OFF_K = 2 * TILE;      // K0, K1 (stages)
-    static constexpr int OFF_V = 4 * TILE;      // V0, V1
-    static constexpr int OFF_P = 6 * TILE;      // P0, P1
-    static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-    // kv_full[2], kv_empty[2], q_full, q_empty, s_full[2], p_full[2], o_full[2], drain
-    static constexpr int NBARS = 14;
+    static constexpr bool HAS_B = DPAD > 64;            // head columns 64..79
+    static constexpr int TILE_A = BQ * 64 * 2;          // 128 rows x 128 B, 128-byte swizzle
+    static constexpr int TILE_B = HAS_B ? BQ * 16 * 2 : 0;  // 128 rows x 32 B, 32-byte swizzle
+    static constexpr int TILE = TILE_A + TILE_B;        // a Q or K tile (K-major)
+    // V is the MN-major operand of P V: one MMA per K step costs the same for
+    // N = 64 or 128, so its head columns are padded to 128 with a second
+    // 64-wide 128-byte-swizzled atom (zeros past the head) instead of being
+    // split into an N = 64 and an N = 16 MMA.
+    static constexpr int VTILE = HAS_B ? 2 * TILE_A : TILE_A;
+    static constexpr int NPV = HAS_B ? 128 : 64;        // N of the P V MMA
+    static constexpr int OFF_Q = 0;                     // [unit parity][query tile]
+    static constexpr int OFF_K = 4 * TILE;              // [stage]
+    static constexpr int OFF_V = OFF_K + NSTAGE * TILE; // [stage]
+    static constexpr int OFF_BAR = OFF_V + NSTAGE * VTILE;
+    // kv_full[NSTAGE], kv_empty[NSTAGE], q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], drain
+    static constexpr int NBARS = 2 * NSTAGE + 11;
     static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
-    static_assert(TILE % 1024 == 0 && P_BYTES % 1024 == 0, "tiles stay 1 KB aligned");
+    static_assert(TILE % 1024 == 0 && TILE_A % 1024 == 0, "swizzled tiles stay 1 KB aligned");
     static_assert(BYTES <= 232448, "shared memory budget");
 };
 
@@ -68,9 +79,10 @@ __device__ __forceinline__ void decode(const AttnArgs &a, const RowsSched &sc, i
 
 template <int DPAD>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_rows_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                     const __grid_constant__ CUtensorMap mv, AttnArgs a, RowsSched sc,
-                     int *status) {
+    attn_rows_kernel(const __grid_constant__ CUtensorMap mqa, const __grid_constant__ CUtensorMap mqb,
+                     const __grid_constant__ CUtensorMap mka, const __grid_constant__ CUtensorMap mkb,
+                     const __grid_constant__ CUtensorMap mva, const __grid_constant__ CUtensorMap mvb,
+                     AttnArgs a, RowsSched sc, int *status) {
     using L = RowsLayout<DPAD>;
     constexpr int NCH = DPAD / 8;
     extern __shared__ uint8_t sm_raw[];
@@ -78,8 +90,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
-    uint64_t *kv_full = bars, *kv_empty = bars + 2, *q_full = bars + 4, *q_empty = bars + 5;
-    uint64_t *s_full = bars + 6, *p_full = bars + 8, *o_full = bars + 10, *drain = bars + 12;
+    uint64_t *kv_full = bars, *kv_empty = bars + NSTAGE;
+    uint64_t *q_full = bars + 2 * NSTAGE, *q_empty = q_full + 2, *s_full = q_full + 4;
+    uint64_t *p_full = q_full + 6, *o_full = q_full + 8, *drain = q_full + 10;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -87,15 +100,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int d = a.d, nch = d / 8;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], BQ);
             mbar_init(&o_full[s], 1);
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
         }
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
         mbar_init(drain, 1);
         *abort = 0;
         fence_mbar_init();
@@ -112,79 +127,99 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ loader
         if (lane == 0) {
-            prefetch_tensormap(&mq);
-            prefetch_tensormap(&mk);
-            prefetch_tensormap(&mv);
+            prefetch_tensormap(&mqa);
+            prefetch_tensormap(&mka);
+            prefetch_tensormap(&mva);
+            // one 128-row tile of a head: the 64-column box, then the 16-column box
+            auto load_tile = [&](uint8_t *dst, const CUtensorMap *ma, const CUtensorMap *mb,
+                                 uint64_t *bar, int row, int h) {
+                tma_load_3d(dst, ma, bar, 0, row, h);
+                if (L::HAS_B) tma_load_3d(dst + L::TILE_A, mb, bar, 64, row, h);
+            };
             int item = 0, last_q_unit = -1;
             bool ok = true;
             for (int u = u0; u < u1 && ok; ++u) {
                 int b, h, qp;
                 decode(a, sc, u, b, h, qp);
+                const int un = u - u0;
                 for (int j = 0; j < sc.kt; ++j, ++item) {
-                    const int st = item & 1;
+                    const int st = item % NSTAGE;
                     if (j == 0) {
-                        if (!mbar_wait(q_empty, ((u - u0) & 1) ^ 1, abort, status)) { ok = false; break; }
+                        const int qb = un & 1;
+                        if (!mbar_wait(&q_empty[qb], ((un >> 1) & 1) ^ 1, abort, status)) { ok = false; break; }
                         const int row0 = (int)((long)b * a.q_bstride + qp * 2 * BQ);
-                        mbar_expect_tx(q_full, 2 * L::TILE);
-                        tma_load_4d(sm + L::OFF_Q, &mq, q_full, 0, row0, 0, h);
-                        tma_load_4d(sm + L::OFF_Q + L::TILE, &mq, q_full, 0, row0 + BQ, 0, h);
-                        last_q_unit = u - u0;
+                        mbar_expect_tx(&q_full[qb], 2 * L::TILE);
+                        for (int g = 0; g < 2; ++g)
+                            load_tile(sm + L::OFF_Q + (qb * 2 + g) * L::TILE, &mqa, &mqb, &q_full[qb],
+                                      row0 + g * BQ, h);
+                        last_q_unit = un;
                     }
-                    if (!mbar_wait(&kv_empty[st], ((item >> 1) & 1) ^ 1, abort, status)) { ok = false; break; }
+                    if (!mbar_wait(&kv_empty[st], ((item / NSTAGE) & 1) ^ 1, abort, status)) { ok = false; break; }
                     const int krow = (int)((long)b * a.k_bstride + j * BKV);
-                    mbar_expect_tx(&kv_full[st], 2 * L::TILE);
-                    tma_load_4d(sm + L::OFF_K + st * L::TILE, &mk, &kv_full[st], 0, krow, 0, h);
-                    tma_load_4d(sm + L::OFF_V + st * L::TILE, &mv, &kv_full[st], 0, krow, 0, h);
+                    mbar_expect_tx(&kv_full[st], L::TILE + L::VTILE);
+                    load_tile(sm + L::OFF_K + st * L::TILE, &mka, &mkb, &kv_full[st], krow, h);
+                    uint8_t *vdst = sm + L::OFF_V + st * L::VTILE;
+                    tma_load_3d(vdst, &mva, &kv_full[st], 0, krow, h);
+                    if (L::HAS_B) tma_load_3d(vdst + L::TILE_A, &mvb, &kv_full[st], 64, krow, h);
                 }
             }
             if (!ok) {  // let copies still in flight land before the CTA exits
                 volatile int never = 0;
-                for (int i = item - 2; i < item; ++i)
-                    if (i >= 0) mbar_wait(&kv_full[i & 1], (i >> 1) & 1, &never, status);
-                if (last_q_unit >= 0) mbar_wait(q_full, last_q_unit & 1, &never, status);
+                for (int i = item - NSTAGE; i < item; ++i)
+                    if (i >= 0) mbar_wait(&kv_full[i % NSTAGE], (i / NSTAGE) & 1, &never, status);
+                if (last_q_unit >= 0)
+                    mbar_wait(&q_full[last_q_unit & 1], (last_q_unit >> 1) & 1, &never, status);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Order per item i: PV0(i), S0(i+1), PV1(i), S1(i+1), so each softmax
+        // warpgroup gets its next S right after handing over its P, while the
+        // other warpgroup is still busy.
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(BQ, BKV);
-            constexpr uint32_t idesc_o = idesc_bf16(BQ, DPAD, true);
-            int item = 0;
+            constexpr uint32_t idesc_o = idesc_bf16(BQ, L::NPV, true);
+            const int n_items = (u1 - u0) * sc.kt;
             bool ok = true, any = false;
-            for (int u = u0; u < u1 && ok; ++u) {
-                for (int j = 0; j < sc.kt; ++j, ++item) {
-                    const int st = item & 1;
-                    const uint32_t ph = item & 1;
-                    if (!mbar_wait(&kv_full[st], (item >> 1) & 1, abort, status)) { ok = false; break; }
-                    if (j == 0 && !mbar_wait(q_full, (u - u0) & 1, abort, status)) { ok = false; break; }
+            // S_g(i) = Q_g K(i)^T; waits for the K tile (and, at a unit's first
+            // tile, for the unit's Q tiles) when g == 0
+            auto issue_s = [&](int i, int g) {
+                const int st = i % NSTAGE, j = i % sc.kt, un = i / sc.kt, qb = un & 1;
+                if (g == 0) {
+                    if (!mbar_wait(&kv_full[st], (i / NSTAGE) & 1, abort, status)) return false;
+                    if (j == 0 && !mbar_wait(&q_full[qb], (un >> 1) & 1, abort, status)) return false;
                     fence_after_sync();
-                    const uint32_t aK = smem_u32(sm + L::OFF_K + st * L::TILE);
-                    const uint32_t aV = smem_u32(sm + L::OFF_V + st * L::TILE);
-                    for (int g = 0; g < 2; ++g) {
-                        const uint32_t aQ = smem_u32(sm + L::OFF_Q + g * L::TILE);
+                }
+                const uint32_t aK = smem_u32(sm + L::OFF_K + st * L::TILE);
+                const uint32_t aQ = smem_u32(sm + L::OFF_Q + (qb * 2 + g) * L::TILE);
 #pragma unroll
-                        for (int ks = 0; ks < DPAD / 16; ++ks)
-                            mma_bf16(tmem + g * BKV, sdesc_interleave(aQ + ks * 2 * CHUNK, CHUNK, 128),
-                                     sdesc_interleave(aK + ks * 2 * CHUNK, CHUNK, 128), idesc_s,
-                                     ks > 0);
-                        mma_commit(&s_full[g]);
-                    }
-                    any = true;
-                    if (j == sc.kt - 1) mma_commit(q_empty);
-                    for (int g = 0; g < 2; ++g) {
-                        if (!mbar_wait(&p_full[g], ph, abort, status)) { ok = false; break; }
-                        fence_after_sync();
-                        const uint32_t aP = smem_u32(sm + L::OFF_P + g * L::P_BYTES);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + g * BKV, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
+                             idesc_s, kk > 0);
+                if (L::HAS_B)
+                    mma_bf16(tmem + g * BKV, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
+                             idesc_s, 1);
+                mma_commit(&s_full[g]);
+                if (g == 1 && j == sc.kt - 1) mma_commit(&q_empty[qb]);  // the unit's Q tiles are read
+                any = true;
+                return true;
+            };
+            if (n_items > 0) ok = issue_s(0, 0) && issue_s(0, 1);
+            for (int i = 0; i < n_items && ok; ++i) {
+                const int st = i % NSTAGE, j = i % sc.kt;
+                const uint32_t aV = smem_u32(sm + L::OFF_V + st * L::VTILE);
+                for (int g = 0; g < 2 && ok; ++g) {
+                    if (!mbar_wait(&p_full[g], i & 1, abort, status)) { ok = false; break; }
+                    fence_after_sync();
+                    const uint32_t tP = tmem + g * BKV;  // P_g over the first 64 columns of S_g
+                    const uint32_t tO = tmem + 256 + g * 128;
 #pragma unroll
-                        for (int ks = 0; ks < BKV / 16; ++ks)
-                            mma_bf16(tmem + 256 + g * 128,
-                                     sdesc_interleave(aP + ks * 2 * CHUNK, CHUNK, 128),
-                                     sdesc_interleave(aV + ks * 256, 128, CHUNK), idesc_o,
-                                     (j | ks) > 0);
-                        mma_commit(&o_full[g]);
-                    }
-                    if (!ok) break;
-                    mma_commit(&kv_empty[st]);
+                    for (int ks = 0; ks < BKV / 16; ++ks)
+                        mma_bf16_ts(tO, tP + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
+                                    idesc_o, (j | ks) > 0);
+                    mma_commit(&o_full[g]);
+                    if (g == 1) mma_commit(&kv_empty[st]);  // both S and both P V of item i
+                    if (i + 1 < n_items) ok = issue_s(i + 1, g);
                 }
             }
             if (any) {  // every issued MMA has finished before TMEM is released
@@ -205,7 +240,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
         const uint32_t t_s = tmem + lane_base + g * BKV;
         const uint32_t t_o = tmem + lane_base + 256 + g * 128;
-        uint8_t *sP = sm + L::OFF_P + g * L::P_BYTES;
         const float sl2 = a.scale * 1.4426950408889634f;
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
         int item = 0;
@@ -220,21 +254,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nvalid = min(BKV, a.nk - j * BKV);
                 if (!mbar_wait(&s_full[g], ph, abort, status)) { ok = false; break; }
                 fence_after_sync();
-                float tmax = -INFINITY;
-#pragma unroll 1
-                for (int c0 = 0; c0 < nvalid; c0 += 32) {
-                    uint32_t s[32];
-                    tmem_ld32(t_s + c0, s);
-                    tmem_ld_wait();
-                    if (c0 + 32 <= nvalid) {
+                // the whole row of S: four loads, one wait
+                uint32_t sv[BKV];
+                tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(sv + 0));
+                tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+                tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(sv + 64));
+                tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(sv + 96));
+                tmem_ld_wait();
+                if (nvalid < BKV) {  // ragged last key tile: masked keys score -inf
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) tmax = fmaxf(tmax, __uint_as_float(s[e]));
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (c0 + e < nvalid) tmax = fmaxf(tmax, __uint_as_float(s[e]));
-                    }
+                    for (int e = 0; e < BKV; ++e)
+                        if (e >= nvalid) sv[e] = __float_as_uint(-INFINITY);
                 }
+                // row max over 8 independent chains (short dependency chains)
+                float mx[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(sv[c]);
+#pragma unroll
+                for (int e = 8; e < BKV; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
+                float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
                 tmax *= sl2;
                 if (tmax > m_ref + 8.f) {  // raise the reference; O so far shrinks by alpha
                     const float alpha = m_ref == -INFINITY ? 0.f : ex2_approx(m_ref - tmax);
@@ -257,59 +296,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l_i *= alpha;
                     m_ref = tmax;
                 }
-                const float ref = m_ref == -INFINITY ? 0.f : m_ref;
-                float psum = 0.f;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BKV; c0 += 32) {
-                    uint4 v[4];
-                    if (c0 + 32 <= nvalid) {
-                        uint32_t s[32];
-                        tmem_ld32(t_s + c0, s);
-                        tmem_ld_wait();
+                const float ref = m_ref;
+                float ps[8];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float pv[8];
+                for (int c = 0; c < 8; ++c) ps[c] = 0.f;
+                // P as bf16 pairs, written over the first 64 columns of S
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                pv[e] = ex2_approx(fmaf(__uint_as_float(s[8 * q + e]), sl2, -ref));
-                                psum += pv[e];
-                            }
-                            v[q].x = pack_bf16(pv[0], pv[1]);
-                            v[q].y = pack_bf16(pv[2], pv[3]);
-                            v[q].z = pack_bf16(pv[4], pv[5]);
-                            v[q].w = pack_bf16(pv[6], pv[7]);
-                        }
-                    } else if (c0 < nvalid) {
-                        uint32_t s[32];
-                        tmem_ld32(t_s + c0, s);
-                        tmem_ld_wait();
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float pv[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int jj = 8 * q + e;
-                                pv[e] = c0 + jj < nvalid
-                                            ? ex2_approx(fmaf(__uint_as_float(s[jj]), sl2, -ref))
-                                            : 0.f;
-                                psum += pv[e];
-                            }
-                            v[q].x = pack_bf16(pv[0], pv[1]);
-                            v[q].y = pack_bf16(pv[2], pv[3]);
-                            v[q].z = pack_bf16(pv[4], pv[5]);
-                            v[q].w = pack_bf16(pv[6], pv[7]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) v[q] = make_uint4(0, 0, 0, 0);
+                    for (int c = 0; c < 32; ++c) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[64 * half + 2 * c]), sl2, -ref));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[64 * half + 2 * c + 1]), sl2, -ref));
+                        ps[(2 * c) & 7] += p0;
+                        ps[(2 * c + 1) & 7] += p1;
+                        pk[c] = pack_bf16(p0, p1);
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4 *>(sP + ((c0 >> 3) + q) * CHUNK + r * 16) = v[q];
+                    tmem_st32(t_s + 32 * half, pk);
                 }
+                tmem_st_wait();
+                const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 l_i += psum;
                 fence_before_sync();
-                fence_async_smem();
                 mbar_arrive(&p_full[g]);
             }
             if (!ok) break;
@@ -353,15 +361,20 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
     using L = RowsLayout<DPAD>;
     int *status = device_status_ptr();
     if (!status) return cudaErrorInvalidValue;
-    const int nch = a.d / 8;
-    CUtensorMap mq, mk, mv;
-    if (!encode_map_rows_heads_bf16(&mq, a.q, (uint64_t)a.B * a.q_bstride, a.ldq * 2, nch, a.heads,
-                                    a.d, BQ, DPAD / 8) ||
-        !encode_map_rows_heads_bf16(&mk, a.k, (uint64_t)a.B * a.k_bstride, a.ldk * 2, nch, a.heads,
-                                    a.d, BKV, DPAD / 8) ||
-        !encode_map_rows_heads_bf16(&mv, a.v, (uint64_t)a.B * a.k_bstride, a.ldv * 2, nch, a.heads,
-                                    a.d, BKV, DPAD / 8))
-        return cudaErrorNotSupported;  // the caller falls back to the gather kernel
+    CUtensorMap m[6];
+    const void *base[3] = {a.q, a.k, a.v};
+    const long ld[3] = {a.ldq, a.ldk, a.ldv};
+    const uint64_t rows[3] = {(uint64_t)a.B * a.q_bstride, (uint64_t)a.B * a.k_bstride,
+                              (uint64_t)a.B * a.k_bstride};
+    for (int t = 0; t < 3; ++t) {
+        if (!encode_map_head_tile_bf16(&m[2 * t], base[t], rows[t], ld[t] * 2, a.heads, a.d, 64,
+                                       BQ, 128))
+            return cudaErrorNotSupported;  // the caller falls back to the gather kernel
+        // second box: Q and K columns 64..79 (32-byte swizzle), V columns 64..127 (128-byte)
+        if (!encode_map_head_tile_bf16(&m[2 * t + 1], base[t], rows[t], ld[t] * 2, a.heads, a.d,
+                                       t == 2 ? 64 : 16, BQ, t == 2 ? 128 : 32))
+            m[2 * t + 1] = m[2 * t];  // only used when d > 64
+    }
     RowsSched sc;
     sc.qp = (a.nq + 2 * BQ - 1) / (2 * BQ);
     sc.kt = (a.nk + BKV - 1) / BKV;
@@ -371,7 +384,8 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<DPAD>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
-    attn_rows_kernel<DPAD><<<grid, kThreads, L::BYTES, s>>>(mq, mk, mv, a, sc, status);
+    attn_rows_kernel<DPAD><<<grid, kThreads, L::BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], a,
+                                                           sc, status);
     return cudaGetLastError();
 }
 

@@ -65,6 +65,23 @@ bool encode_map_rows_heads_bf16(CUtensorMap *map, const void *base, uint64_t row
     return r == CUDA_SUCCESS;
 }
 
+bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows,
+                               uint64_t row_pitch_bytes, int heads, int d, uint32_t box_elems,
+                               uint32_t box_rows, int swizzle_bytes) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, rows, (cuuint64_t)heads};
+    cuuint64_t strides[2] = {row_pitch_bytes, (cuuint64_t)d * 2};
+    cuuint32_t box[3] = {box_elems, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw =
+        swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;

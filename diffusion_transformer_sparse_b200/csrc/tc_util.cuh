@@ -98,6 +98,15 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -139,6 +148,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (bf16, K-major) read from tensor memory,
+// lane m = row m, two K elements per 32-bit column (even element in the low half).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -231,6 +252,30 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     return d;
 }
 
+// MN-major operand with the 128-byte swizzle: 8-row K groups 1024 B apart
+// (SBO), `atom_stride` bytes between consecutive 64-wide atoms along N (LBO).
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t atom_stride) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFF) >> 4);
+    d |= static_cast<uint64_t>((atom_stride >> 4) & 0x3FFF) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// Same for the 32-byte swizzle: rows of 16 bf16 (32 B), 8-row groups 256 B
+// apart (a K-major tile of one K step, or an MN-major tile 16 wide in N).
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFF) >> 4);
+    d |= static_cast<uint64_t>(1) << 16;
+    d |= static_cast<uint64_t>(256 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(6) << 61;
+    return d;
+}
+
 // Shared-memory matrix descriptor of an operand stored without swizzle in
 // 8-row x 16-byte core matrices: `lbo` bytes between core matrices along K,
 // `sbo` bytes between 8-row groups along M/N.
@@ -294,6 +339,14 @@ bool encode_map_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint
 bool encode_map_rows_heads_bf16(CUtensorMap *map, const void *base, uint64_t rows,
                                 uint64_t row_pitch_bytes, int nch, int heads, int d,
                                 uint32_t box_rows, uint32_t box_chunks);
+
+// Host: a 3-D map over a [rows, heads * d] bf16 matrix, dims (d elements of a
+// head, rows, heads), strides (row pitch, d * 2 B); box (box_elems, box_rows,
+// 1) with the given swizzle (128 or 32 bytes).  Elements at or past d read as
+// zeros, so a box reaching past the head's last column pads it.
+bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows,
+                               uint64_t row_pitch_bytes, int heads, int d, uint32_t box_elems,
+                               uint32_t box_rows, int swizzle_bytes);
 
 int num_sms();
 
