@@ -1,0 +1,379 @@
+// Projections y = x W^T (+ residual) on pairs of SMs: tcgen05.mma.cta_group::2.
+//
+// A cluster of two CTAs computes a 256 x BN output tile with one MMA stream:
+// each CTA loads its own 128 rows of A and its own BN/2 rows of the weight
+// tile, and the pair's tensor cores read both halves.  Per SM that is half
+// the weight traffic of a one-SM 128 x BN tile, which is what limits the
+// one-SM kernel (shared-memory operand bandwidth per MMA).
+//
+//   warp 0     producer (both CTAs): TMA loads (the .cta_group::2 form, no
+//              multicast) of the CTA's A and B halves; both CTAs' copies
+//              complete on the leader CTA's full barrier, which the leader
+//              alone arms with the byte count of the pair.
+//   warp 1     MMA issuer (leader CTA only): 4 x tcgen05.mma.cta_group::2
+//              (M = 256, K = 16) per stage; tcgen05.commit multicast frees
+//              the stage in both CTAs and hands the accumulator to both
+//              epilogues.
+//   warps 2-5  epilogue (both CTAs): each reads its own TMEM half (its 128
+//              rows), adds the residual, rounds, stores, and then tells the
+//              leader (a remote mbarrier arrive from the peer) that the
+//              accumulator is free again.
+// Two TMEM accumulators overlap the next tile's MMAs with this tile's
+// epilogue.  Every wait is bounded (2 s); a timeout records
+// PTDIT_ERR_TIMEOUT in the status word.
+#include "tc_util.cuh"
+
+namespace ptdit {
+namespace {
+
+using namespace tc;
+
+constexpr int BMC = 128, BK = 64;  // rows of A per CTA, K per stage
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+
+struct Tc2Params {
+    void *C[3];
+    const void *R[3];
+    long ldc;
+    int rows, nseg, nmat;
+    int n_tiles;  // output tiles per weight matrix
+    int tiles;    // all pair tiles
+    int kblocks;
+    int *status;
+};
+
+template <int BN, int STAGES>
+struct Layout2 {
+    static constexpr int A_BYTES = BMC * BK * 2;       // 16 KB: this CTA's rows of A
+    static constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's half of the weight tile
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+    static constexpr int NBARS = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
+    static constexpr int BYTES = BAR_OFF + NBARS * 8 + 16;
+    static constexpr int ALLOC = BYTES + 1024;
+    static constexpr uint32_t ACC_STRIDE = BN <= 128 ? 128 : 256;
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "stage tiles stay 1 KB aligned");
+    static_assert(2 * ACC_STRIDE <= kTmemCols, "two accumulators must fit in TMEM");
+    static_assert(ALLOC <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// Shared-memory address of `local`'s counterpart in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void *local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map,
+                                                 uint32_t leader_bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives once on `bar` in both CTAs of the pair when the pair's MMAs so far have completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_pair_local(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
+__device__ __forceinline__ void decode_tile2(const Tc2Params &p, int t, int &m_tile, int &seg,
+                                             int &n_tile) {
+    const int per_m = p.nmat * p.n_tiles;
+    m_tile = t / per_m;
+    const int n = t % per_m;
+    seg = n / p.n_tiles;
+    n_tile = n % p.n_tiles;
+}
+
+template <int BN, int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
+                    const __grid_constant__ CUtensorMap mB1,
+                    const __grid_constant__ CUtensorMap mB2, Tc2Params p) {
+    using L = Layout2<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x / 2, npairs = gridDim.x / 2;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 8);  // one arrive per epilogue warp of both CTAs
+        }
+        mbar_init(drain, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    cluster_sync();  // barriers of both CTAs are initialised before anyone signals them
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tensormap(&mA);
+            prefetch_tensormap(&mB0);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = pair; ok && t < p.tiles; t += npairs) {
+                int m_tile, seg, n_tile;
+                decode_tile2(p, t, m_tile, seg, n_tile);
+                const CUtensorMap *mb = seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2);
+                const int arow = m_tile * 2 * BMC + rank * BMC;
+                const int brow = n_tile * BN + rank * (BN / 2);
+                for (int kb = 0; kb < p.kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + stage * L::STAGE_BYTES;
+                    const uint32_t lbar = cluster_addr(&full[stage], 0);
+                    if (leader) mbar_expect_tx(&full[stage], 2 * L::STAGE_BYTES);
+                    tma_load_2d_pair(sa, &mA, lbar, kb * BK, arow);
+                    tma_load_2d_pair(sa + L::A_BYTES, mb, lbar, kb * BK, brow);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            const uint32_t idesc = idesc_bf16(2 * BMC, BN);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true, any = false;
+            for (int t = pair; ok && t < p.tiles; t += npairs) {
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort, p.status)) break;
+                fence_after_sync();
+                const uint32_t d = tmem + acc * L::ACC_STRIDE;
+                for (int kb = 0; kb < p.kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
+                    const uint32_t sa = smem_u32(smem + stage * L::STAGE_BYTES);
+                    const uint32_t sb = sa + L::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_bf16_pair(d, sdesc_sw128(sa + kk * 32), sdesc_sw128(sb + kk * 32), idesc,
+                                      (kb | kk) != 0);
+                    any = true;
+                    mma_commit_pair(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                mma_commit_pair(&tfull[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            if (any) {  // every issued MMA has finished before TMEM is released
+                mma_commit_pair_local(drain);
+                volatile int never = 0;
+                mbar_wait(drain, 0, &never, p.status);
+            }
+        }
+    } else {
+        const int q = warp % 4;  // TMEM lanes 32q .. 32q+31 belong to this warp
+        const int r_in_tile = rank * BMC + q * 32 + lane;
+        const uint32_t tempty_leader[2] = {cluster_addr(&tempty[0], 0), cluster_addr(&tempty[1], 0)};
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int t = pair; t < p.tiles; t += npairs) {
+            int m_tile, seg, n_tile;
+            decode_tile2(p, t, m_tile, seg, n_tile);
+            if (!mbar_wait(&tfull[acc], acc_phase, abort, p.status)) break;
+            fence_after_sync();
+            const long row = static_cast<long>(m_tile) * 2 * BMC + r_in_tile;
+            const bool live = row < p.rows;
+            __nv_bfloat16 *C = static_cast<__nv_bfloat16 *>(p.C[seg]) + row * p.ldc + n_tile * BN;
+            const __nv_bfloat16 *R = static_cast<const __nv_bfloat16 *>(p.R[seg]);
+            if (R) R += row * p.ldc + n_tile * BN;
+            const uint32_t tbase = tmem + acc * L::ACC_STRIDE + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + c0, r);
+                tmem_ld_wait();
+                if (live) {
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                    if (R) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 rv = *reinterpret_cast<const uint4 *>(R + c0 + 8 * j);
+                            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&rv);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float2 f = __bfloat1622float2(h[e]);
+                                v[8 * j + 2 * e] += f.x;
+                                v[8 * j + 2 * e + 1] += f.y;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 o;
+                        o.x = pack_bf16(v[8 * j + 0], v[8 * j + 1]);
+                        o.y = pack_bf16(v[8 * j + 2], v[8 * j + 3]);
+                        o.z = pack_bf16(v[8 * j + 4], v[8 * j + 5]);
+                        o.w = pack_bf16(v[8 * j + 6], v[8 * j + 7]);
+                        *reinterpret_cast<uint4 *>(C + c0 + 8 * j) = o;
+                    }
+                }
+            }
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    }
+    if (*abort) {
+        // give copies still in flight into this CTA a moment to land
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 100000) {
+        }
+    }
+    fence_before_sync();
+    cluster_sync();  // no CTA leaves while its peer may still signal it
+    if (warp == 0) {
+        fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
+    using L = Layout2<BN, STAGES>;
+    CUtensorMap mA, mB[3];
+    if (!encode_map_2d_bf16(&mA, a.A, a.K, a.rows, a.lda * 2, BK, BMC)) return cudaErrorInvalidValue;
+    for (int i = 0; i < 3; ++i) {
+        const void *w = i < a.nmat ? a.W[i] : a.W[0];
+        if (!encode_map_2d_bf16(&mB[i], w, a.K, a.nseg, (uint64_t)a.K * 2, BK, BN / 2))
+            return cudaErrorInvalidValue;
+    }
+    Tc2Params p;
+    for (int i = 0; i < 3; ++i) {
+        p.C[i] = i < a.nmat ? a.C[i] : nullptr;
+        p.R[i] = i < a.nmat ? a.R[i] : nullptr;
+    }
+    p.ldc = a.ldc;
+    p.rows = a.rows;
+    p.nseg = a.nseg;
+    p.nmat = a.nmat;
+    p.n_tiles = a.nseg / BN;
+    p.kblocks = a.K / BK;
+    const int m_tiles = (a.rows + 2 * BMC - 1) / (2 * BMC);
+    p.tiles = m_tiles * a.nmat * p.n_tiles;
+    p.status = device_status_ptr();
+    if (!p.status) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    // persistent grid: as many pairs as can be resident at once (pairs must
+    // share a GPC, so this can be below half the SM count)
+    static int max_pairs = 0;
+    if (!max_pairs) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * 74, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = L::ALLOC;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<BN, STAGES>, &cfg) != cudaSuccess || n < 1)
+            n = (num_sms() > 0 ? num_sms() : 148) / 2;
+        (void)cudaGetLastError();
+        max_pairs = n;
+    }
+    const int pairs = p.tiles < max_pairs ? p.tiles : max_pairs;
+    gemm_tc2_kernel<BN, STAGES><<<2 * pairs, kThreads, L::ALLOC, s>>>(mA, mB[0], mB[1], mB[2], p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc2_supported(const GemmArgs &a) {
+    if (a.dtype != DT_BF16 || a.nmat < 1 || a.nmat > 3) return false;
+    if (a.K < BK || a.K % BK || a.rows < 2 * BMC || a.lda % 8 || a.ldc % 8) return false;
+    if (a.nseg % 192) return false;
+    if ((uintptr_t)a.A % 16) return false;
+    for (int i = 0; i < a.nmat; ++i)
+        if ((uintptr_t)a.W[i] % 16 || (uintptr_t)a.C[i] % 16 || (uintptr_t)a.R[i] % 16)
+            return false;
+    return true;
+}
+
+cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) { return launch_bn2<192, 6>(a, s); }
+
+}  // namespace ptdit

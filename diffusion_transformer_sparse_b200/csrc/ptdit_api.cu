@@ -25,10 +25,13 @@ cudaError_t launch_gemm_simt(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_attention_simt(const AttnArgs &a, cudaStream_t s);
 bool gemm_tc_supported(const GemmArgs &a);
 cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
+bool gemm_tc2_supported(const GemmArgs &a);
+cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s);
 bool attention_tc_supported(const AttnArgs &a);
 cudaError_t launch_attention_tc(const AttnArgs &a, cudaStream_t s);
 
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s) {
+    if (gemm_tc2_supported(a)) return launch_gemm_tc2(a, s);
     if (gemm_tc_supported(a)) return launch_gemm_tc(a, s);
     return launch_gemm_simt(a, s);
 }
