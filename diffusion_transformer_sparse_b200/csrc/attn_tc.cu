@@ -392,12 +392,16 @@ bool attention_tc_supported(const AttnArgs &a) {
 }
 
 cudaError_t launch_attention_rows_tc(const AttnArgs &a, cudaStream_t s);
+bool attention_win_tc_supported(const AttnArgs &a);
+cudaError_t launch_attention_win_tc(const AttnArgs &a, cudaStream_t s);
 
 cudaError_t launch_attention_tc(const AttnArgs &a, cudaStream_t s) {
     if (a.mode == ATT_ROWS) {
         const cudaError_t e = launch_attention_rows_tc(a, s);
         if (e != cudaErrorNotSupported) return e;
         (void)cudaGetLastError();  // tensor maps rejected: use the gather kernel below
+    } else if (attention_win_tc_supported(a)) {
+        return launch_attention_win_tc(a, s);
     }
     switch (dpad_of(a.d)) {
         case 64: return launch_dpad<64>(a, s);

@@ -308,6 +308,8 @@ __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
+// Waits for every committed cp.async group of this thread (copies issued
+// after the last cp_async_commit() are not covered).
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
