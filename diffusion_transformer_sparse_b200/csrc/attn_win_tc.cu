@@ -5,22 +5,27 @@
 //
 // One persistent CTA per SM with two independent slots; a unit is one tile
 // (128 query rows = its own 128 key rows) of one head:
-//   warps 2, 3   gather loaders, one per slot: each lane computes the token
-//                row of its slots with the roll/wrap address function (no
-//                permuted copy exists anywhere), cp.asyncs the Q, K and V rows
-//                of the head into shared memory (16-byte chunks major: the
-//                no-swizzle core-matrix layout, K-major for Q and K, MN-major
-//                for V), builds one 128-bit key mask per mask key (window in
-//                tile, wrap bits) with ballots, waits for its copies, fences
-//                them to the async proxy and arrives on the slot's barrier.
-//   warp 1       MMA issuer: S = Q K^T into TMEM, then P V with P read from
-//                TMEM (written over S by the softmax) and V from shared memory.
-//   warps 4-7, 8-11   softmax of slot 0 / slot 1: thread r owns query row r
-//                (its TMEM lane), reads only its own window's scores, applies
-//                the key mask, runs the softmax in fp32, writes P as bf16
-//                pairs into TMEM, then scales its output row by 1/l and stores
-//                it to global memory.
-// While one slot computes, the other slot's rows stream in, so HBM stays busy.
+//   warps 2, 3   loaders, one per slot: each lane computes the token row of
+//                its slots with the roll/wrap address function (no permuted
+//                copy exists anywhere), then the warp copies the head's Q, K
+//                and V rows with 16-byte cp.async into the 128-byte-swizzled
+//                K-major layout (columns 64.. in a 32-byte-swizzled block for
+//                Q and K, a second 128-byte atom for V).  Eight lanes cover
+//                one row's 128 contiguous bytes, so an instruction touches
+//                four rows instead of 32; Q and K complete on their own
+//                barrier so S = Q K^T starts while V is still arriving.  Key
+//                masks (window in tile x wrap bits) are built with ballots.
+//                (Tile loads by TMA are not used here: a box walks the head's
+//                rows one by one, and at 144 bytes a row that rate, not HBM,
+//                bounded the loads.)
+//   warp 1       MMA issuer: S = Q K^T into TMEM, then O = P V with P read
+//                from TMEM (the softmax writes it over S) and V from shared
+//                memory, padded to 128 columns so one MMA per K step covers
+//                the head.
+//   warps 4-7, 8-11   softmax of slot 0 / slot 1: thread r owns query row r,
+//                reads only its own window's scores, masks, exponentiates in
+//                fp32, writes P as bf16 pairs into TMEM, then scales its
+//                output row by 1/l and stores it.
 // Every wait is bounded (2 s).
 #include <math.h>
 
@@ -32,22 +37,28 @@ namespace {
 using namespace tc;
 
 constexpr int BQ = 128;
-constexpr uint32_t CHUNK = BQ * 16;  // bytes between 16-byte chunk columns
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;  // per slot: S/P 128 columns, O 128 columns
 constexpr int kKeys = 16;            // mask keys per tile: 2 windows x 8 wrap codes
 
 template <int DPAD>
 struct WinLayout {
-    static constexpr int TILE = BQ * DPAD * 2;
-    static constexpr int OFF_TILES = 0;                    // [slot][Q, K, V]
-    static constexpr int OFF_INFO = 6 * TILE;              // int info[2][128]
-    static constexpr int OFF_ROW = OFF_INFO + 2 * BQ * 4;  // long row[2][128]
-    static constexpr int OFF_MASK = OFF_ROW + 2 * BQ * 8;  // uint32 kmask[2][kKeys][4]
+    static constexpr bool HAS_B = DPAD > 64;                   // head columns 64..79
+    static constexpr int TILE_A = BQ * 128;                    // columns 0..63, 128-byte swizzle
+    static constexpr int TILE_B = HAS_B ? BQ * 32 : 0;         // columns 64..79, 32-byte swizzle
+    static constexpr int TILE = TILE_A + TILE_B;               // a Q or K tile (K-major)
+    static constexpr int VTILE = HAS_B ? 2 * TILE_A : TILE_A;  // V, MN-major, padded to 128
+    static constexpr int NPV = HAS_B ? 128 : 64;
+    static constexpr int SLOT = 2 * TILE + VTILE;              // Q, K, V of one slot
+    static constexpr int OFF_INFO = 2 * SLOT;                  // int info[2][128]
+    static constexpr int OFF_ROW = OFF_INFO + 2 * BQ * 4;      // long row[2][128]
+    static constexpr int OFF_MASK = OFF_ROW + 2 * BQ * 8;      // uint32 kmask[2][kKeys][4]
     static constexpr int OFF_BAR = OFF_MASK + 2 * kKeys * 16;
-    // load_full[2], slot_free[2], s_full[2], p_full[2], o_full[2], o_free[2], drain
-    static constexpr int NBARS = 13;
-    static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16;
+    // qk_full[2], v_full[2], slot_free[2], s_full[2], p_full[2], o_full[2], o_free[2], drain
+    static constexpr int NBARS = 15;
+    static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
+    static_assert(TILE_A % 1024 == 0 && TILE % 1024 == 0 && SLOT % 1024 == 0,
+                  "swizzled tiles stay 1 KB aligned");
     static_assert(BYTES <= 232448, "shared memory budget");
 };
 
@@ -56,26 +67,34 @@ struct WinSched {
     int units;  // B x tiles x heads
 };
 
+// Byte offset of 16-byte unit c of row r (0..7) inside one 128-byte-swizzled atom.
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return r * 128 + ((c ^ r) << 4); }
+// Same for a 32-byte-swizzled atom (8 rows x 2 units).
+__device__ __forceinline__ uint32_t sw32(int r, int u) { return r * 32 + ((u ^ ((r >> 2) & 1)) << 4); }
+
 template <int DPAD>
-__global__ void __launch_bounds__(kThreads, 1) attn_win_kernel(AttnArgs a, WinSched sc, int *status) {
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_win_kernel(const __grid_constant__ AttnArgs a, WinSched sc, int *status) {
     using L = WinLayout<DPAD>;
-    constexpr int NCH = DPAD / 8;
-    extern __shared__ __align__(128) uint8_t sm[];
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     int *info = reinterpret_cast<int *>(sm + L::OFF_INFO);
     long *rowsm = reinterpret_cast<long *>(sm + L::OFF_ROW);
     uint32_t *kmask = reinterpret_cast<uint32_t *>(sm + L::OFF_MASK);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
-    uint64_t *load_full = bars, *slot_free = bars + 2, *s_full = bars + 4, *p_full = bars + 6;
-    uint64_t *o_full = bars + 8, *o_free = bars + 10, *drain = bars + 12;
+    uint64_t *qk_full = bars, *v_full = bars + 2, *slot_free = bars + 4, *s_full = bars + 6;
+    uint64_t *p_full = bars + 8, *o_full = bars + 10, *o_free = bars + 12, *drain = bars + 14;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int d = a.d, nch = d / 8, n = a.geom.n;
+    const int d = a.d, n = a.geom.n, nch = d / 8;
 
     if (threadIdx.x == 0) {
         for (int g = 0; g < 2; ++g) {
-            mbar_init(&load_full[g], 32);
+            mbar_init(&qk_full[g], 32);
+            mbar_init(&v_full[g], 32);
             mbar_init(&slot_free[g], 1);
             mbar_init(&s_full[g], 1);
             mbar_init(&p_full[g], BQ);
@@ -87,11 +106,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_win_kernel(AttnArgs a, WinSc
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tslot, kTmemCols);
-    // zero the padded chunks of the six tiles once; the loaders never touch them
-    for (int i = threadIdx.x; i < 6 * BQ * (NCH - nch); i += kThreads) {
-        const int t = i / (BQ * (NCH - nch)), rest = i % (BQ * (NCH - nch));
-        const int c = nch + rest / BQ, r = rest % BQ;
-        *reinterpret_cast<uint4 *>(sm + t * L::TILE + c * CHUNK + r * 16) = make_uint4(0, 0, 0, 0);
+    // zero, once, the padding columns no copy writes: Q and K columns d..79,
+    // V columns d..127 (their products with P and Q are then exactly 0)
+    if (L::HAS_B) {
+        for (int i = threadIdx.x; i < 2 * BQ * 8; i += kThreads) {
+            const int g = i / (BQ * 8), r = (i / 8) % BQ, c = i % 8;
+            uint8_t *slot = sm + g * L::SLOT;
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            if (8 + c >= nch) {
+                if (c < 2) {
+                    const uint32_t o = L::TILE_A + (r >> 3) * 256 + sw32(r & 7, c);
+                    *reinterpret_cast<uint4 *>(slot + o) = z;
+                    *reinterpret_cast<uint4 *>(slot + L::TILE + o) = z;
+                }
+                *reinterpret_cast<uint4 *>(slot + 2 * L::TILE + L::TILE_A + (r >> 3) * 1024 +
+                                           sw128(r & 7, c)) = z;
+            }
+        }
     }
     fence_async_smem();
     fence_before_sync();
@@ -105,15 +136,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_win_kernel(AttnArgs a, WinSc
     auto unit_of = [&](int g, int k) { return u0 + g + 2 * k; };
 
     if (warp == 2 || warp == 3) {
-        // ------------------------------------------------------------ gather loader of slot g
+        // ------------------------------------------------------------ loader of slot g
         const int g = warp - 2;
-        uint8_t *sQ = sm + (3 * g + 0) * L::TILE, *sK = sm + (3 * g + 1) * L::TILE,
-                *sV = sm + (3 * g + 2) * L::TILE;
-        const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(a.q);
-        const __nv_bfloat16 *kb = static_cast<const __nv_bfloat16 *>(a.k);
-        const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(a.v);
+        uint8_t *sQ = sm + g * L::SLOT, *sK = sQ + L::TILE, *sV = sK + L::TILE;
+        const char *gq = static_cast<const char *>(a.q);
+        const char *gk = static_cast<const char *>(a.k);
+        const char *gv = static_cast<const char *>(a.v);
+        const long ldq = a.ldq * 2, ldk = a.ldk * 2, ldv = a.ldv * 2;  // row pitches in bytes
         const WinGeom &geo = a.geom;
         const int pack = BQ / n;
+        const int c8 = lane & 7;  // 16-byte chunk (columns 8 c8 .. 8 c8 + 7) of the main copies
         for (int k = 0; unit_of(g, k) < u1; ++k) {
             const int u = unit_of(g, k);
             const int h = u % a.heads, rest = u / a.heads, tile = rest % sc.tiles,
@@ -134,17 +166,57 @@ __global__ void __launch_bounds__(kThreads, 1) attn_win_kernel(AttnArgs a, WinSc
                 inf[q] = in;
                 info[g * BQ + r] = in;
                 rowsm[g * BQ + r] = row;
+            }
+            __syncwarp();
+            const long hoff = (long)h * d * 2;
+            // columns 0..63: eight lanes per row, four rows per instruction; Q and K first
+#pragma unroll 4
+            for (int it = 0; it < BQ / 4; ++it) {
+                const int r = 4 * it + (lane >> 3);
+                const long row = rowsm[g * BQ + r];
+                const uint32_t bytes = row >= 0 ? 16u : 0u;
                 const long rr = row >= 0 ? row : 0;
-                const uint32_t bytes = row >= 0 ? 16 : 0;
-                const __nv_bfloat16 *pq = qb + rr * a.ldq + (long)h * d;
-                const __nv_bfloat16 *pk = kb + rr * a.ldk + (long)h * d;
-                const __nv_bfloat16 *pv = vb + rr * a.ldv + (long)h * d;
-                for (int c = 0; c < nch; ++c) {
-                    cp_async16(sQ + c * CHUNK + r * 16, pq + c * 8, bytes);
-                    cp_async16(sK + c * CHUNK + r * 16, pk + c * 8, bytes);
-                    cp_async16(sV + c * CHUNK + r * 16, pv + c * 8, bytes);
+                const uint32_t o = (r >> 3) * 1024 + sw128(r & 7, c8);
+                cp_async16(sQ + o, gq + rr * ldq + hoff + c8 * 16, bytes);
+                cp_async16(sK + o, gk + rr * ldk + hoff + c8 * 16, bytes);
+            }
+            if (L::HAS_B) {  // columns 64 .. d-1: one row per lane
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = q * 32 + lane;
+                    const long row = rowsm[g * BQ + r];
+                    const uint32_t bytes = row >= 0 ? 16u : 0u;
+                    const long rr = row >= 0 ? row : 0;
+                    for (int c = 8; c < nch; ++c) {
+                        const uint32_t o = L::TILE_A + (r >> 3) * 256 + sw32(r & 7, c - 8);
+                        cp_async16(sQ + o, gq + rr * ldq + hoff + c * 16, bytes);
+                        cp_async16(sK + o, gk + rr * ldk + hoff + c * 16, bytes);
+                    }
                 }
             }
+            cp_async_commit();
+#pragma unroll 4
+            for (int it = 0; it < BQ / 4; ++it) {
+                const int r = 4 * it + (lane >> 3);
+                const long row = rowsm[g * BQ + r];
+                const uint32_t bytes = row >= 0 ? 16u : 0u;
+                const long rr = row >= 0 ? row : 0;
+                cp_async16(sV + (r >> 3) * 1024 + sw128(r & 7, c8), gv + rr * ldv + hoff + c8 * 16,
+                           bytes);
+            }
+            if (L::HAS_B) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = q * 32 + lane;
+                    const long row = rowsm[g * BQ + r];
+                    const uint32_t bytes = row >= 0 ? 16u : 0u;
+                    const long rr = row >= 0 ? row : 0;
+                    for (int c = 8; c < nch; ++c)
+                        cp_async16(sV + L::TILE_A + (r >> 3) * 1024 + sw128(r & 7, c - 8),
+                                   gv + rr * ldv + hoff + c * 16, bytes);
+                }
+            }
+            cp_async_commit();
             // one 128-bit key mask per mask key: keys of the same window and wrap code
             for (int v = 0; v < kKeys; ++v)
 #pragma unroll
@@ -152,10 +224,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_win_kernel(AttnArgs a, WinSc
                     const uint32_t bits = __ballot_sync(0xffffffffu, inf[q] == v);
                     if (lane == 0) kmask[(g * kKeys + v) * 4 + q] = bits;
                 }
-            cp_async_commit();  // wait_group only covers committed copies
+            cp_async_wait_group1();  // Q and K have landed (V may still be in flight)
+            fence_async_smem();
+            mbar_arrive(&qk_full[g]);
             cp_async_wait_all();
             fence_async_smem();
-            mbar_arrive(&load_full[g]);
+            mbar_arrive(&v_full[g]);
         }
         cp_async_commit();
         cp_async_wait_all();
@@ -163,32 +237,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_win_kernel(AttnArgs a, WinSc
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(BQ, BQ);
-            constexpr uint32_t idesc_o = idesc_bf16(BQ, DPAD, true);
+            constexpr uint32_t idesc_o = idesc_bf16(BQ, L::NPV, true);
             bool ok = true, any = false;
             for (int k = 0; ok && unit_of(0, k) < u1; ++k) {
                 for (int g = 0; g < 2 && ok; ++g) {
                     if (unit_of(g, k) >= u1) continue;
-                    if (!mbar_wait(&load_full[g], k & 1, abort, status)) { ok = false; break; }
+                    if (!mbar_wait(&qk_full[g], k & 1, abort, status)) { ok = false; break; }
                     fence_after_sync();
-                    const uint32_t aQ = smem_u32(sm + (3 * g + 0) * L::TILE);
-                    const uint32_t aK = smem_u32(sm + (3 * g + 1) * L::TILE);
+                    const uint32_t aQ = smem_u32(sm + g * L::SLOT);
+                    const uint32_t aK = aQ + L::TILE;
 #pragma unroll
-                    for (int ks = 0; ks < DPAD / 16; ++ks)
-                        mma_bf16(tmem + g * 256, sdesc_interleave(aQ + ks * 2 * CHUNK, CHUNK, 128),
-                                 sdesc_interleave(aK + ks * 2 * CHUNK, CHUNK, 128), idesc_s, ks > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tmem + g * 256, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
+                                 idesc_s, kk > 0);
+                    if (L::HAS_B)
+                        mma_bf16(tmem + g * 256, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
+                                 idesc_s, 1);
                     mma_commit(&s_full[g]);
                     any = true;
                 }
                 for (int g = 0; g < 2 && ok; ++g) {
                     if (unit_of(g, k) >= u1) continue;
+                    if (!mbar_wait(&v_full[g], k & 1, abort, status)) { ok = false; break; }
                     if (!mbar_wait(&p_full[g], k & 1, abort, status)) { ok = false; break; }
                     if (!mbar_wait(&o_free[g], (k & 1) ^ 1, abort, status)) { ok = false; break; }
                     fence_after_sync();
-                    const uint32_t aV = smem_u32(sm + (3 * g + 2) * L::TILE);
+                    const uint32_t aV = smem_u32(sm + g * L::SLOT + 2 * L::TILE);
 #pragma unroll
                     for (int ks = 0; ks < BQ / 16; ++ks)
                         mma_bf16_ts(tmem + g * 256 + 128, tmem + g * 256 + ks * 8,
-                                    sdesc_interleave(aV + ks * 256, 128, CHUNK), idesc_o, ks > 0);
+                                    sdesc_sw128_mn(aV + ks * 2048, L::TILE_A), idesc_o, ks > 0);
                     mma_commit(&o_full[g]);
                     mma_commit(&slot_free[g]);  // Q, K and V of this slot are read
                 }
@@ -206,16 +284,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_win_kernel(AttnArgs a, WinSc
         const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
         const uint32_t t_s = tmem + lane_base + g * 256, t_o = t_s + 128;
         const float sl2 = a.scale * 1.4426950408889634f;
+        const int nch = d / 8;
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
         // the row's own keys: its window inside the tile
         const int c_lo = n < BQ ? (r / n) * n : 0;
         for (int k = 0; unit_of(g, k) < u1; ++k) {
             const int u = unit_of(g, k);
             const int h = u % a.heads;
-            if (!mbar_wait(&load_full[g], k & 1, abort, status)) break;  // masks and rows
+            if (!mbar_wait(&qk_full[g], k & 1, abort, status)) break;  // masks and rows
             const int qi = info[g * BQ + r];
             const long qrow = rowsm[g * BQ + r];  // queries and keys share rows in window mode
-            const bool live = rowsm[g * BQ + r] >= 0;
+            const bool live = qrow >= 0;
             uint32_t allow[4] = {0u, 0u, 0u, 0u};
             if (qi >= 0) {
                 const uint4 w4 = *reinterpret_cast<const uint4 *>(kmask + (g * kKeys + qi) * 4);
@@ -314,6 +393,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_win_kernel(AttnArgs a, WinSc
             mbar_arrive(&o_free[g]);
         }
     }
+    if (*abort) {
+        // give box loads still in flight into this CTA a moment to land
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 100000) {
+        }
+    }
     fence_before_sync();
     __syncthreads();
     if (warp == 0) {
@@ -342,15 +427,18 @@ cudaError_t launch_win(const AttnArgs &a, cudaStream_t s) {
 
 }  // namespace
 
+// Windows of 64 or 128 tokens (any shape and shift), head width 64..80.
 bool attention_win_tc_supported(const AttnArgs &a) {
-    return a.mode == ATT_WINDOW && (a.geom.n == 64 || a.geom.n == 128) && a.q_bstride == a.k_bstride;
+    if (a.dtype != DT_BF16 || a.mode != ATT_WINDOW) return false;
+    if (!(a.geom.n == 64 || a.geom.n == 128) || a.q_bstride != a.k_bstride) return false;
+    if (a.d % 8 || a.d < 64 || a.d > 80) return false;
+    if (a.ldq % 8 || a.ldk % 8 || a.ldv % 8 || a.ldo % 8) return false;
+    return true;
 }
 
 cudaError_t launch_attention_win_tc(const AttnArgs &a, cudaStream_t s) {
-    const int dp = (a.d + 15) / 16 * 16;
-    if (dp == 64) return launch_win<64>(a, s);
-    if (dp == 80) return launch_win<80>(a, s);
-    return cudaErrorInvalidValue;
+    if (a.d <= 64) return launch_win<64>(a, s);
+    return launch_win<80>(a, s);
 }
 
 }  // namespace ptdit

@@ -2,9 +2,13 @@
 //
 // A cluster of two CTAs computes a 256 x BN output tile with one MMA stream:
 // each CTA loads its own 128 rows of A and its own BN/2 rows of the weight
-// tile, and the pair's tensor cores read both halves.  Per SM that is half
-// the weight traffic of a one-SM 128 x BN tile, which is what limits the
-// one-SM kernel (shared-memory operand bandwidth per MMA).
+// tile, and the pair's tensor cores read both halves.  Every operand byte is
+// written into shared memory once (TMA) and read once (MMA), so the tile's
+// bytes per FLOP set the shared-memory traffic per MMA: a 256 x 256 pair tile
+// moves 16 KB per SM per K = 16 step of 128 tensor cycles, a 256 x 192 tile
+// 14 KB per 96 cycles.  The last tile of a matrix whose width is not a
+// multiple of BN is narrower (e.g. 1152 = 4 x 256 + 128): its MMAs run with
+// the smaller N and its weight rows are split between the CTAs by that N.
 //
 //   warp 0     producer (both CTAs): TMA loads (the .cta_group::2 form, no
 //              multicast) of the CTA's A and B halves; both CTAs' copies
@@ -14,10 +18,16 @@
 //              (M = 256, K = 16) per stage; tcgen05.commit multicast frees
 //              the stage in both CTAs and hands the accumulator to both
 //              epilogues.
-//   warps 2-5  epilogue (both CTAs): each reads its own TMEM half (its 128
-//              rows), adds the residual, rounds, stores, and then tells the
-//              leader (a remote mbarrier arrive from the peer) that the
-//              accumulator is free again.
+//   warps 2-5  epilogue (both CTAs): each warp owns 32 rows of its CTA's TMEM
+//              half.  Before it waits for a tile's accumulator it starts the
+//              TMA load of its residual rows into its own staging tile, so
+//              that load overlaps the MMAs.  It then reads the accumulator
+//              32 columns at a time, adds the residual from shared memory,
+//              rounds, writes the result back over the staging tile, tells
+//              the leader (a remote mbarrier arrive from the peer) that the
+//              accumulator is free, and writes the tile out with TMA stores:
+//              whole 64-byte row segments instead of one 16-byte piece per
+//              row and instruction.
 // Two TMEM accumulators overlap the next tile's MMAs with this tile's
 // epilogue.  Every wait is bounded (2 s); a timeout records
 // PTDIT_ERR_TIMEOUT in the status word.
@@ -32,12 +42,17 @@ constexpr int BMC = 128, BK = 64;  // rows of A per CTA, K per stage
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 
+// Output and residual maps: box of 32 columns x 32 rows, 64-byte swizzle.
+struct Tc2Maps {
+    CUtensorMap C[3], R[3];
+};
+
 struct Tc2Params {
     void *C[3];
     const void *R[3];
     long ldc;
     int rows, nseg, nmat;
-    int n_tiles;  // output tiles per weight matrix
+    int n_tiles;  // output tiles per weight matrix (the last may be narrower)
     int tiles;    // all pair tiles
     int kblocks;
     int *status;
@@ -48,8 +63,11 @@ struct Layout2 {
     static constexpr int A_BYTES = BMC * BK * 2;       // 16 KB: this CTA's rows of A
     static constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's half of the weight tile
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-    static constexpr int NBARS = 2 * STAGES + 5;  // full, empty, tfull[2], tempty[2], drain
+    static constexpr int CHUNK_BYTES = 32 * 64;          // 32 rows x 32 bf16 columns
+    static constexpr int WARP_STAGE = (BN / 32) * CHUNK_BYTES;
+    static constexpr int EPI_OFF = STAGES * STAGE_BYTES;  // 4 epilogue warps' staging tiles
+    static constexpr int BAR_OFF = EPI_OFF + 4 * WARP_STAGE;
+    static constexpr int NBARS = 2 * STAGES + 9;  // full, empty, tfull[2], tempty[2], rfull[4], drain
     static constexpr int BYTES = BAR_OFF + NBARS * 8 + 16;
     static constexpr int ALLOC = BYTES + 1024;
     static constexpr uint32_t ACC_STRIDE = BN <= 128 ? 128 : 256;
@@ -124,11 +142,19 @@ __device__ __forceinline__ void decode_tile2(const Tc2Params &p, int t, int &m_t
     n_tile = n % p.n_tiles;
 }
 
+// Output columns of tile n_tile: BN, or what is left of the matrix for the last one.
+template <int BN>
+__device__ __forceinline__ int tile_width(const Tc2Params &p, int n_tile) {
+    const int w = p.nseg - n_tile * BN;
+    return w < BN ? w : BN;
+}
+
 template <int BN, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                     const __grid_constant__ CUtensorMap mB1,
-                    const __grid_constant__ CUtensorMap mB2, Tc2Params p) {
+                    const __grid_constant__ CUtensorMap mB2, const __grid_constant__ Tc2Maps mo,
+                    const __grid_constant__ Tc2Params p) {
     using L = Layout2<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -137,7 +163,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;
     uint64_t *tempty = tfull + 2;
-    uint64_t *drain = tempty + 2;
+    uint64_t *rfull = tempty + 2;
+    uint64_t *drain = rfull + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -155,6 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], 8);  // one arrive per epilogue warp of both CTAs
         }
+        for (int w = 0; w < 4; ++w) mbar_init(&rfull[w], 1);
         mbar_init(drain, 1);
         *abort = 0;
         fence_mbar_init();
@@ -183,7 +211,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 decode_tile2(p, t, m_tile, seg, n_tile);
                 const CUtensorMap *mb = seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2);
                 const int arow = m_tile * 2 * BMC + rank * BMC;
-                const int brow = n_tile * BN + rank * (BN / 2);
+                const int brow = n_tile * BN + rank * (tile_width<BN>(p, n_tile) / 2);
                 for (int kb = 0; kb < p.kblocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort, p.status)) {
                         ok = false;
@@ -203,11 +231,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         if (leader && lane == 0) {
-            const uint32_t idesc = idesc_bf16(2 * BMC, BN);
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, any = false;
             for (int t = pair; ok && t < p.tiles; t += npairs) {
+                int m_tile, seg, n_tile;
+                decode_tile2(p, t, m_tile, seg, n_tile);
+                const uint32_t idesc = idesc_bf16(2 * BMC, tile_width<BN>(p, n_tile));
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort, p.status)) break;
                 fence_after_sync();
                 const uint32_t d = tmem + acc * L::ACC_STRIDE;
@@ -243,60 +273,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else {
         const int q = warp % 4;  // TMEM lanes 32q .. 32q+31 belong to this warp
-        const int r_in_tile = rank * BMC + q * 32 + lane;
-        const uint32_t tempty_leader[2] = {cluster_addr(&tempty[0], 0), cluster_addr(&tempty[1], 0)};
+        uint8_t *stg = smem + L::EPI_OFF + q * L::WARP_STAGE;
+        const uint32_t tempty_leader0 = cluster_addr(&tempty[0], 0);
+        const uint32_t tempty_leader1 = cluster_addr(&tempty[1], 0);
+        // 64-byte swizzle of the staging tiles: 16-byte unit j of row r sits at
+        // unit j ^ ((r >> 1) & 3), which spreads a warp's row accesses over all banks
+        const uint32_t row_off = lane * 64;
+        const uint32_t sw = (lane >> 1) & 3;
         int acc = 0;
-        uint32_t acc_phase = 0;
+        uint32_t acc_phase = 0, r_phase = 0;
         for (int t = pair; t < p.tiles; t += npairs) {
             int m_tile, seg, n_tile;
             decode_tile2(p, t, m_tile, seg, n_tile);
+            const int row0 = m_tile * 2 * BMC + rank * BMC + q * 32;
+            const int col0 = n_tile * BN;
+            const int nchunk = tile_width<BN>(p, n_tile) / 32;
+            const bool has_r = p.R[seg] != nullptr;
+            if (lane == 0) {
+                bulk_wait_read_all();  // the previous tile's stores have left the staging tile
+                if (has_r) {
+                    mbar_expect_tx(&rfull[q], nchunk * L::CHUNK_BYTES);
+#pragma unroll 1
+                    for (int c = 0; c < nchunk; ++c)
+                        tma_load_2d(stg + c * L::CHUNK_BYTES, &mo.R[seg], &rfull[q], col0 + 32 * c,
+                                    row0);
+                }
+            }
+            __syncwarp();
             if (!mbar_wait(&tfull[acc], acc_phase, abort, p.status)) break;
+            if (has_r) {
+                if (!mbar_wait(&rfull[q], r_phase, abort, p.status)) break;
+                r_phase ^= 1;
+            }
             fence_after_sync();
-            const long row = static_cast<long>(m_tile) * 2 * BMC + r_in_tile;
-            const bool live = row < p.rows;
-            __nv_bfloat16 *C = static_cast<__nv_bfloat16 *>(p.C[seg]) + row * p.ldc + n_tile * BN;
-            const __nv_bfloat16 *R = static_cast<const __nv_bfloat16 *>(p.R[seg]);
-            if (R) R += row * p.ldc + n_tile * BN;
             const uint32_t tbase = tmem + acc * L::ACC_STRIDE + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
+            for (int c = 0; c < nchunk; ++c) {
                 uint32_t r[32];
-                tmem_ld32(tbase + c0, r);
+                tmem_ld32(tbase + 32 * c, r);
                 tmem_ld_wait();
-                if (live) {
-                    float v[32];
+                uint8_t *chunk = stg + c * L::CHUNK_BYTES + row_off;
+                float v[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-                    if (R) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 rv = *reinterpret_cast<const uint4 *>(R + c0 + 8 * j);
-                            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&rv);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                float2 f = __bfloat1622float2(h[e]);
-                                v[8 * j + 2 * e] += f.x;
-                                v[8 * j + 2 * e + 1] += f.y;
-                            }
-                        }
-                    }
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                if (has_r) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        uint4 o;
-                        o.x = pack_bf16(v[8 * j + 0], v[8 * j + 1]);
-                        o.y = pack_bf16(v[8 * j + 2], v[8 * j + 3]);
-                        o.z = pack_bf16(v[8 * j + 4], v[8 * j + 5]);
-                        o.w = pack_bf16(v[8 * j + 6], v[8 * j + 7]);
-                        *reinterpret_cast<uint4 *>(C + c0 + 8 * j) = o;
+                        const uint4 rv = *reinterpret_cast<const uint4 *>(chunk + ((j ^ sw) << 4));
+                        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&rv);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(h[e]);
+                            v[8 * j + 2 * e] += f.x;
+                            v[8 * j + 2 * e + 1] += f.y;
+                        }
                     }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 o;
+                    o.x = pack_bf16(v[8 * j + 0], v[8 * j + 1]);
+                    o.y = pack_bf16(v[8 * j + 2], v[8 * j + 3]);
+                    o.z = pack_bf16(v[8 * j + 4], v[8 * j + 5]);
+                    o.w = pack_bf16(v[8 * j + 6], v[8 * j + 7]);
+                    *reinterpret_cast<uint4 *>(chunk + ((j ^ sw) << 4)) = o;
                 }
             }
             fence_before_sync();
+            fence_async_smem();  // the staging writes become visible to the TMA stores
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
+            if (lane == 0) {
+                mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+#pragma unroll 1
+                for (int c = 0; c < nchunk; ++c)
+                    tma_store_2d(&mo.C[seg], stg + c * L::CHUNK_BYTES, col0 + 32 * c, row0);
+                bulk_commit();
+            }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
+        if (lane == 0) bulk_wait_all();
     }
     if (*abort) {
         // give copies still in flight into this CTA a moment to land
@@ -325,15 +381,22 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
             return cudaErrorInvalidValue;
     }
     Tc2Params p;
+    Tc2Maps mo;
     for (int i = 0; i < 3; ++i) {
         p.C[i] = i < a.nmat ? a.C[i] : nullptr;
         p.R[i] = i < a.nmat ? a.R[i] : nullptr;
+        // unused slots get a valid map over C[0] that no tile refers to
+        const void *c = p.C[i] ? p.C[i] : a.C[0];
+        const void *r = p.R[i] ? p.R[i] : c;
+        if (!encode_map_2d_bf16_sw(&mo.C[i], c, a.nseg, a.rows, (uint64_t)a.ldc * 2, 32, 32, 64) ||
+            !encode_map_2d_bf16_sw(&mo.R[i], r, a.nseg, a.rows, (uint64_t)a.ldc * 2, 32, 32, 64))
+            return cudaErrorInvalidValue;
     }
     p.ldc = a.ldc;
     p.rows = a.rows;
     p.nseg = a.nseg;
     p.nmat = a.nmat;
-    p.n_tiles = a.nseg / BN;
+    p.n_tiles = (a.nseg + BN - 1) / BN;
     p.kblocks = a.K / BK;
     const int m_tiles = (a.rows + 2 * BMC - 1) / (2 * BMC);
     p.tiles = m_tiles * a.nmat * p.n_tiles;
@@ -357,7 +420,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
         max_pairs = n;
     }
     const int pairs = p.tiles < max_pairs ? p.tiles : max_pairs;
-    gemm_tc2_kernel<BN, STAGES><<<2 * pairs, kThreads, L::ALLOC, s>>>(mA, mB[0], mB[1], mB[2], p);
+    gemm_tc2_kernel<BN, STAGES><<<2 * pairs, kThreads, L::ALLOC, s>>>(mA, mB[0], mB[1], mB[2], mo, p);
     return cudaGetLastError();
 }
 
@@ -366,7 +429,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
 bool gemm_tc2_supported(const GemmArgs &a) {
     if (a.dtype != DT_BF16 || a.nmat < 1 || a.nmat > 3) return false;
     if (a.K < BK || a.K % BK || a.rows < 2 * BMC || a.lda % 8 || a.ldc % 8) return false;
-    if (a.nseg % 192) return false;
+    if (a.nseg % 64) return false;  // tile widths: multiples of 32 per CTA half and epilogue chunk
     if ((uintptr_t)a.A % 16) return false;
     for (int i = 0; i < a.nmat; ++i)
         if ((uintptr_t)a.W[i] % 16 || (uintptr_t)a.C[i] % 16 || (uintptr_t)a.R[i] % 16)
@@ -374,6 +437,12 @@ bool gemm_tc2_supported(const GemmArgs &a) {
     return true;
 }
 
-cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) { return launch_bn2<192, 6>(a, s); }
+cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) {
+#ifndef PTDIT_GEMM2_BN
+    return launch_bn2<256, 5>(a, s);
+#else
+    return PTDIT_GEMM2_BN == 192 ? launch_bn2<192, 6>(a, s) : launch_bn2<256, 5>(a, s);
+#endif
+}
 
 }  // namespace ptdit

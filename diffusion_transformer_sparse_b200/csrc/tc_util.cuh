@@ -107,6 +107,30 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Tile store shared -> global (bulk async group of this thread); elements
+// outside the tensor's extents are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until this thread's committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Waits until this thread's committed bulk stores have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -308,6 +332,11 @@ __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
+// Waits until at most one committed cp.async group of this thread is pending.
+__device__ __forceinline__ void cp_async_wait_group1() {
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
 // Waits for every committed cp.async group of this thread (copies issued
 // after the last cp_async_commit() are not covered).
 __device__ __forceinline__ void cp_async_wait_all() {
@@ -333,6 +362,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // 128-byte swizzle.  Returns false if the driver rejects it.
 bool encode_map_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
+// Host: the same with a chosen swizzle (32, 64 or 128 bytes; the box's inner
+// extent in bytes must not exceed it).
+bool encode_map_2d_bf16_sw(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                           uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                           int swizzle_bytes);
 
 // Host: a 4-D map over a [rows, heads * d] bf16 matrix whose boxes land in
 // shared memory as 16-byte chunks major (chunk c, row r at c * box_rows * 16

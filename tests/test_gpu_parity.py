@@ -85,6 +85,10 @@ SMALL = [
     (1, (4, 8, 12), 96, 4, (2, 2, 3), (2, 4, 3), (1, 1, 2)),
     (1, (1, 24, 24), 144, 2, (1, 3, 3), (1, 8, 8), (0, 4, 4)),
     (1, (2, 16, 16), 1152, 16, (1, 4, 4), (2, 8, 8), (1, 4, 4)),
+    # head width 64 (no columns past the first 128-byte swizzle atom)
+    (1, (1, 16, 16), 128, 2, (1, 2, 2), (1, 8, 8), (0, 4, 4)),
+    # 2 x 4 x 16 windows (rows of 16 tokens) with a shift that is not half the window
+    (1, (2, 16, 32), 144, 2, (1, 4, 4), (2, 4, 16), (1, 1, 4)),
 ]
 
 
