@@ -5,12 +5,13 @@
 // each batch item; head h is columns h*d .. h*d+d-1.
 //
 // FlashAttention-style warp specialisation, one persistent CTA per SM:
-//   warp 0       loader: TMA loads of two 128-row query tiles per unit (double
-//                buffered across units) and of K and V tiles into a two-stage
-//                ring.  A head's 72 columns arrive as a 64-column box with the
-//                128-byte swizzle plus a 16-column box with the 32-byte swizzle
-//                whose last 8 columns lie past the head and read as zeros: the
-//                zero padding of d to 80 comes for free.
+//   warp 0       loader: two 128-row query tiles per unit (double buffered
+//                across units) and K and V tiles into a two-stage ring, each
+//                one contiguous bulk copy: the projections wrote Q, K and V in
+//                tiled head layout (thl.cuh), so a (tile, head) block already
+//                is the swizzled shared-memory tile (columns 0..63 with the
+//                128-byte swizzle, 64..79 with the 32-byte swizzle, zeros past
+//                the head; V padded to 128 columns).
 //   warp 1       MMA issuer: S_g = Q_g K^T (K-major operands) into TMEM, and
 //                once softmax g has written P_g, P_g V with P_g read straight
 //                from TMEM and V as an MN-major operand (no transpose),
@@ -28,6 +29,7 @@
 #include <math.h>
 
 #include "tc_util.cuh"
+#include "thl.cuh"
 
 namespace ptdit {
 namespace {
@@ -55,9 +57,13 @@ struct RowsLayout {
     static constexpr int OFF_Q = 0;                     // [unit parity][query tile]
     static constexpr int OFF_K = 4 * TILE;              // [stage]
     static constexpr int OFF_V = OFF_K + NSTAGE * TILE; // [stage]
-    static constexpr int OFF_BAR = OFF_V + NSTAGE * VTILE;
-    // kv_full[NSTAGE], kv_empty[NSTAGE], q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], drain
-    static constexpr int NBARS = 2 * NSTAGE + 11;
+    // output staging of each softmax warpgroup: 128 rows, pitch <= 160 B
+    static constexpr int STG = BQ * 160;
+    static constexpr int OFF_STG = OFF_V + NSTAGE * VTILE;
+    static constexpr int OFF_BAR = OFF_STG + 2 * STG;
+    // kv_full[NSTAGE], kv_empty[NSTAGE], q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2],
+    // drain, stage_full[2], stage_free[2]
+    static constexpr int NBARS = 2 * NSTAGE + 15;
     static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
     static_assert(TILE % 1024 == 0 && TILE_A % 1024 == 0, "swizzled tiles stay 1 KB aligned");
     static_assert(BYTES <= 232448, "shared memory budget");
@@ -79,12 +85,8 @@ __device__ __forceinline__ void decode(const AttnArgs &a, const RowsSched &sc, i
 
 template <int DPAD>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_rows_kernel(const __grid_constant__ CUtensorMap mqa, const __grid_constant__ CUtensorMap mqb,
-                     const __grid_constant__ CUtensorMap mka, const __grid_constant__ CUtensorMap mkb,
-                     const __grid_constant__ CUtensorMap mva, const __grid_constant__ CUtensorMap mvb,
-                     AttnArgs a, RowsSched sc, int *status) {
+    attn_rows_kernel(const __grid_constant__ AttnArgs a, RowsSched sc, int *status) {
     using L = RowsLayout<DPAD>;
-    constexpr int NCH = DPAD / 8;
     extern __shared__ uint8_t sm_raw[];
     // TMA destinations: align the base to 1 KB (tile offsets are multiples of 1 KB)
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) &
@@ -93,6 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *kv_full = bars, *kv_empty = bars + NSTAGE;
     uint64_t *q_full = bars + 2 * NSTAGE, *q_empty = q_full + 2, *s_full = q_full + 4;
     uint64_t *p_full = q_full + 6, *o_full = q_full + 8, *drain = q_full + 10;
+    uint64_t *stage_full = q_full + 11, *stage_free = q_full + 13;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -112,6 +115,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&q_empty[s], 1);
         }
         mbar_init(drain, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&stage_full[s], BQ);
+            mbar_init(&stage_free[s], BQ);
+        }
         *abort = 0;
         fence_mbar_init();
     }
@@ -127,14 +134,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ loader
         if (lane == 0) {
-            prefetch_tensormap(&mqa);
-            prefetch_tensormap(&mka);
-            prefetch_tensormap(&mva);
-            // one 128-row tile of a head: the 64-column box, then the 16-column box
-            auto load_tile = [&](uint8_t *dst, const CUtensorMap *ma, const CUtensorMap *mb,
-                                 uint64_t *bar, int row, int h) {
-                tma_load_3d(dst, ma, bar, 0, row, h);
-                if (L::HAS_B) tma_load_3d(dst + L::TILE_A, mb, bar, 64, row, h);
+            const uint8_t *qg = static_cast<const uint8_t *>(a.q);
+            const uint8_t *kg = static_cast<const uint8_t *>(a.k);
+            const uint8_t *vg = static_cast<const uint8_t *>(a.v);
+            // the (tile, head) block of batch item b
+            auto block = [&](const uint8_t *base, const ThlDesc &t, int b, int tile, int h,
+                             uint32_t bytes) {
+                return base + (((long)b * t.tiles + tile) * a.heads + h) * (long)bytes;
             };
             int item = 0, last_q_unit = -1;
             bool ok = true;
@@ -147,20 +153,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (j == 0) {
                         const int qb = un & 1;
                         if (!mbar_wait(&q_empty[qb], ((un >> 1) & 1) ^ 1, abort, status)) { ok = false; break; }
-                        const int row0 = (int)((long)b * a.q_bstride + qp * 2 * BQ);
-                        mbar_expect_tx(&q_full[qb], 2 * L::TILE);
-                        for (int g = 0; g < 2; ++g)
-                            load_tile(sm + L::OFF_Q + (qb * 2 + g) * L::TILE, &mqa, &mqb, &q_full[qb],
-                                      row0 + g * BQ, h);
+                        // the unit's second query tile may lie past the last one
+                        const int nqt = 2 * qp + 1 < a.tq.tiles ? 2 : 1;
+                        mbar_expect_tx(&q_full[qb], nqt * L::TILE);
+                        for (int g = 0; g < nqt; ++g)
+                            bulk_load(sm + L::OFF_Q + (qb * 2 + g) * L::TILE,
+                                      block(qg, a.tq, b, 2 * qp + g, h, L::TILE), L::TILE, &q_full[qb]);
                         last_q_unit = un;
                     }
                     if (!mbar_wait(&kv_empty[st], ((item / NSTAGE) & 1) ^ 1, abort, status)) { ok = false; break; }
-                    const int krow = (int)((long)b * a.k_bstride + j * BKV);
                     mbar_expect_tx(&kv_full[st], L::TILE + L::VTILE);
-                    load_tile(sm + L::OFF_K + st * L::TILE, &mka, &mkb, &kv_full[st], krow, h);
-                    uint8_t *vdst = sm + L::OFF_V + st * L::VTILE;
-                    tma_load_3d(vdst, &mva, &kv_full[st], 0, krow, h);
-                    if (L::HAS_B) tma_load_3d(vdst + L::TILE_A, &mvb, &kv_full[st], 64, krow, h);
+                    bulk_load(sm + L::OFF_K + st * L::TILE, block(kg, a.tk, b, j, h, L::TILE), L::TILE,
+                              &kv_full[st]);
+                    bulk_load(sm + L::OFF_V + st * L::VTILE, block(vg, a.tv, b, j, h, L::VTILE),
+                              L::VTILE, &kv_full[st]);
                 }
             }
             if (!ok) {  // let copies still in flight land before the CTA exits
@@ -242,12 +248,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_o = tmem + lane_base + 256 + g * 128;
         const float sl2 = a.scale * 1.4426950408889634f;
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
-        int item = 0;
+        // staging row pitch: an odd number of 16-byte units where that fits
+        const int pitch = nch * 16 + (nch % 8 == 0 ? 16 : 0);
+        int item = 0, un_count = 0;
         bool ok = true;
         for (int u = u0; u < u1 && ok; ++u) {
             int b, h, qp;
             decode(a, sc, u, b, h, qp);
-            const int iq = qp * 2 * BQ + g * BQ + r;
             float m_ref = -INFINITY, l_i = 0.f;
             for (int j = 0; j < sc.kt; ++j, ++item) {
                 const uint32_t ph = item & 1;
@@ -321,31 +328,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&p_full[g]);
             }
             if (!ok) break;
-            // the unit's last P V, then O / l to global memory
+            // the unit's last P V, then O / l to global memory through the staging
+            // rows, so that consecutive lanes store consecutive 16-byte pieces of
+            // a row (a few rows per store instruction instead of 32)
             if (!mbar_wait(&o_full[g], (item - 1) & 1, abort, status)) { ok = false; break; }
+            if (!mbar_wait(&stage_free[g], (un_count & 1) ^ 1, abort, status)) { ok = false; break; }
             fence_after_sync();
             const float inv = 1.f / l_i;
-            __nv_bfloat16 *dst = og + ((long)b * a.q_bstride + iq) * a.ldo + (long)h * d;
-#pragma unroll
-            for (int c0 = 0; c0 < DPAD; c0 += 16) {
-                uint32_t ov[16];
-                tmem_ld16(t_o + c0, ov);
+            uint8_t *stg = sm + L::OFF_STG + g * L::STG;
+            {
+                uint32_t ov[DPAD];
+                tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(ov));
+                tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
+                if (DPAD > 64) tmem_ld16(t_o + 64, *reinterpret_cast<uint32_t(*)[16]>(ov + 64));
                 tmem_ld_wait();
-                if (iq < a.nq) {
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        if ((c0 >> 3) + c < nch) {
-                            uint4 v;
-                            v.x = pack_bf16(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
-                            v.y = pack_bf16(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
-                            v.z = pack_bf16(__uint_as_float(ov[8 * c + 4]) * inv, __uint_as_float(ov[8 * c + 5]) * inv);
-                            v.w = pack_bf16(__uint_as_float(ov[8 * c + 6]) * inv, __uint_as_float(ov[8 * c + 7]) * inv);
-                            *reinterpret_cast<uint4 *>(dst + c0 + 8 * c) = v;
-                        }
+                for (int u = 0; u < DPAD / 8; ++u)
+                    if (u < nch) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(ov[8 * u + 0]) * inv, __uint_as_float(ov[8 * u + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(ov[8 * u + 2]) * inv, __uint_as_float(ov[8 * u + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(ov[8 * u + 4]) * inv, __uint_as_float(ov[8 * u + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(ov[8 * u + 6]) * inv, __uint_as_float(ov[8 * u + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(stg + r * pitch + u * 16) = v;
                     }
-                }
             }
             fence_before_sync();  // O is read before the next unit's first P V overwrites it
+            mbar_arrive(&stage_full[g]);
+            if (!mbar_wait(&stage_full[g], un_count & 1, abort, status)) { ok = false; break; }
+            {
+                const int q0 = qp * 2 * BQ + g * BQ;  // query index of staging row 0
+                __nv_bfloat16 *obase = og + (long)b * a.q_bstride * a.ldo + (long)h * d;
+                for (int i = r; i < BQ * nch; i += BQ) {
+                    const int row = i / nch, u = i - row * nch;
+                    if (q0 + row < a.nq)
+                        *reinterpret_cast<uint4 *>(obase + (long)(q0 + row) * a.ldo + u * 8) =
+                            *reinterpret_cast<const uint4 *>(stg + row * pitch + u * 16);
+                }
+            }
+            mbar_arrive(&stage_free[g]);
+            ++un_count;
         }
     }
     fence_before_sync();
@@ -361,20 +383,11 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
     using L = RowsLayout<DPAD>;
     int *status = device_status_ptr();
     if (!status) return cudaErrorInvalidValue;
-    CUtensorMap m[6];
-    const void *base[3] = {a.q, a.k, a.v};
-    const long ld[3] = {a.ldq, a.ldk, a.ldv};
-    const uint64_t rows[3] = {(uint64_t)a.B * a.q_bstride, (uint64_t)a.B * a.k_bstride,
-                              (uint64_t)a.B * a.k_bstride};
-    for (int t = 0; t < 3; ++t) {
-        if (!encode_map_head_tile_bf16(&m[2 * t], base[t], rows[t], ld[t] * 2, a.heads, a.d, 64,
-                                       BQ, 128))
-            return cudaErrorNotSupported;  // the caller falls back to the gather kernel
-        // second box: Q and K columns 64..79 (32-byte swizzle), V columns 64..127 (128-byte)
-        if (!encode_map_head_tile_bf16(&m[2 * t + 1], base[t], rows[t], ld[t] * 2, a.heads, a.d,
-                                       t == 2 ? 64 : 16, BQ, t == 2 ? 128 : 32))
-            m[2 * t + 1] = m[2 * t];  // only used when d > 64
-    }
+    // the tiles are the tiled-head-layout blocks the projections wrote
+    if (a.tq.mode != THL_IDENTITY || a.tk.mode != THL_IDENTITY || a.tv.mode != THL_IDENTITY ||
+        a.tq.vpad || a.tk.vpad || !a.tv.vpad || L::TILE != (int)thl_block_bytes(a.d, 0) ||
+        L::VTILE != (int)thl_block_bytes(a.d, 1))
+        return cudaErrorInvalidValue;
     RowsSched sc;
     sc.qp = (a.nq + 2 * BQ - 1) / (2 * BQ);
     sc.kt = (a.nk + BKV - 1) / BKV;
@@ -384,8 +397,7 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<DPAD>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
-    attn_rows_kernel<DPAD><<<grid, kThreads, L::BYTES, s>>>(m[0], m[1], m[2], m[3], m[4], m[5], a,
-                                                           sc, status);
+    attn_rows_kernel<DPAD><<<grid, kThreads, L::BYTES, s>>>(a, sc, status);
     return cudaGetLastError();
 }
 

@@ -1,7 +1,8 @@
-// Window attention core on the 5th-generation tensor cores: window and
-// shifted-window self-attention of TCM.  (Row-mode attention -- proxy SA,
-// cross-attention, full SA -- is the warp-specialised kernel of
-// attn_rows_tc.cu; this file dispatches to it.)
+// Attention core on the 5th-generation tensor cores for operands in plain
+// row-major layout (head widths whose operands are not tiled, e.g. 56), and
+// the dispatch: operands in tiled head layout go to the warp-specialised
+// kernels of attn_rows_tc.cu (proxy SA, cross-attention, full SA) and
+// attn_win_tc.cu (window and shifted-window SA).
 //
 // Qihoo-T2X reading note, §3 Method: Eq. GIIM (SA among the proxies, CS with
 // every latent the query and the proxies keys/values) and Eq. TCM (WSA, and
@@ -391,19 +392,22 @@ bool attention_tc_supported(const AttnArgs &a) {
     return a.nq >= 1 && a.nk >= 1;
 }
 
+// Operands in tiled head layout (head width 64..80): the warp-specialised
+// row kernel (proxy SA, cross-attention, full SA) and window kernel.
+bool attention_thl_supported(const AttnArgs &a) {
+    if (a.dtype != DT_BF16 || a.d < 64 || a.d > 80 || a.d % 8) return false;
+    if (a.mode == ATT_WINDOW)
+        return (a.geom.n == 64 || a.geom.n == 128) && a.q_bstride == a.k_bstride;
+    return a.nq >= 1 && a.nk >= 1;
+}
+
 cudaError_t launch_attention_rows_tc(const AttnArgs &a, cudaStream_t s);
-bool attention_win_tc_supported(const AttnArgs &a);
 cudaError_t launch_attention_win_tc(const AttnArgs &a, cudaStream_t s);
 
 cudaError_t launch_attention_tc(const AttnArgs &a, cudaStream_t s) {
-    if (a.mode == ATT_ROWS) {
-        const cudaError_t e = launch_attention_rows_tc(a, s);
-        if (e != cudaErrorNotSupported) return e;
-        (void)cudaGetLastError();  // tensor maps rejected: use the gather kernel below
-    } else if (attention_win_tc_supported(a)) {
-        return launch_attention_win_tc(a, s);
-    }
-    switch (dpad_of(a.d)) {
+    if (a.tq.mode != 0)
+        return a.mode == ATT_ROWS ? launch_attention_rows_tc(a, s) : launch_attention_win_tc(a, s);
+    switch (dpad_of(a.d)) {  // row-major operands: the per-tile kernel above
         case 64: return launch_dpad<64>(a, s);
         case 80: return launch_dpad<80>(a, s);
         default: return cudaErrorInvalidValue;

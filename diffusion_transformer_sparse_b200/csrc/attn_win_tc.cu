@@ -5,23 +5,23 @@
 //
 // One persistent CTA per SM with two independent slots; a unit is one tile
 // (128 query rows = its own 128 key rows) of one head:
-//   warps 2, 3   loaders, one per slot: each lane computes the token row of
-//                its slots with the roll/wrap address function (no permuted
-//                copy exists anywhere), then the warp copies the head's Q, K
-//                and V rows with 16-byte cp.async into the 128-byte-swizzled
-//                K-major layout (columns 64.. in a 32-byte-swizzled block for
-//                Q and K, a second 128-byte atom for V).  Eight lanes cover
-//                one row's 128 contiguous bytes, so an instruction touches
-//                four rows instead of 32; Q and K complete on their own
-//                barrier so S = Q K^T starts while V is still arriving.  Key
-//                masks (window in tile x wrap bits) are built with ballots.
-//                (Tile loads by TMA are not used here: a box walks the head's
-//                rows one by one, and at 144 bytes a row that rate, not HBM,
-//                bounded the loads.)
+//   warps 2, 3   loaders, one per slot: the window projection wrote Q, K and V
+//                in tiled head layout (thl.cuh) with window tiles, so the
+//                unit's Q, K and V are three contiguous 20 KB blocks, each
+//                already the swizzled shared-memory tile (columns 0..63 with
+//                the 128-byte swizzle, 64..79 with the 32-byte swizzle, zeros
+//                past the head and in rows without a window): three bulk
+//                copies, Q and K on one barrier and V on another, so that
+//                S = Q K^T starts while V is still arriving.  Meanwhile each
+//                lane computes the token of its tile rows with the roll/wrap
+//                address function (for the key masks and the output rows) and
+//                the warp builds the key masks (window in tile x wrap bits)
+//                with ballots.
 //   warp 1       MMA issuer: S = Q K^T into TMEM, then O = P V with P read
 //                from TMEM (the softmax writes it over S) and V from shared
-//                memory, padded to 128 columns so one MMA per K step covers
-//                the head.
+//                memory as the MN-major operand: columns 0..63 in one N = 64
+//                MMA per K step (128-byte swizzle), 64..79 in one N = 16 MMA
+//                (32-byte swizzle).
 //   warps 4-7, 8-11   softmax of slot 0 / slot 1: thread r owns query row r,
 //                reads only its own window's scores, masks, exponentiates in
 //                fp32, writes P as bf16 pairs into TMEM, then scales its
@@ -30,6 +30,7 @@
 #include <math.h>
 
 #include "tc_util.cuh"
+#include "thl.cuh"
 
 namespace ptdit {
 namespace {
@@ -47,15 +48,17 @@ struct WinLayout {
     static constexpr int TILE_A = BQ * 128;                    // columns 0..63, 128-byte swizzle
     static constexpr int TILE_B = HAS_B ? BQ * 32 : 0;         // columns 64..79, 32-byte swizzle
     static constexpr int TILE = TILE_A + TILE_B;               // a Q or K tile (K-major)
-    static constexpr int VTILE = HAS_B ? 2 * TILE_A : TILE_A;  // V, MN-major, padded to 128
-    static constexpr int NPV = HAS_B ? 128 : 64;
-    static constexpr int SLOT = 2 * TILE + VTILE;              // Q, K, V of one slot
+    static constexpr int SLOT = 3 * TILE;                      // Q, K, V of one slot
     static constexpr int OFF_INFO = 2 * SLOT;                  // int info[2][128]
     static constexpr int OFF_ROW = OFF_INFO + 2 * BQ * 4;      // long row[2][128]
     static constexpr int OFF_MASK = OFF_ROW + 2 * BQ * 8;      // uint32 kmask[2][kKeys][4]
-    static constexpr int OFF_BAR = OFF_MASK + 2 * kKeys * 16;
+    // output staging of each softmax warpgroup: 128 rows (pitch <= 160 B), their token rows
+    static constexpr int STG = BQ * 160;
+    static constexpr int OFF_STG = OFF_MASK + 2 * kKeys * 16;
+    static constexpr int OFF_OROW = OFF_STG + 2 * STG;        // long orow[2][128]
+    static constexpr int OFF_BAR = OFF_OROW + 2 * BQ * 8;
     // qk_full[2], v_full[2], slot_free[2], s_full[2], p_full[2], o_full[2], o_free[2], drain
-    static constexpr int NBARS = 15;
+    static constexpr int NBARS = 19;  // + stage_full[2], stage_free[2]
     static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
     static_assert(TILE_A % 1024 == 0 && TILE % 1024 == 0 && SLOT % 1024 == 0,
                   "swizzled tiles stay 1 KB aligned");
@@ -66,11 +69,6 @@ struct WinSched {
     int tiles;  // tiles per batch item
     int units;  // B x tiles x heads
 };
-
-// Byte offset of 16-byte unit c of row r (0..7) inside one 128-byte-swizzled atom.
-__device__ __forceinline__ uint32_t sw128(int r, int c) { return r * 128 + ((c ^ r) << 4); }
-// Same for a 32-byte-swizzled atom (8 rows x 2 units).
-__device__ __forceinline__ uint32_t sw32(int r, int u) { return r * 32 + ((u ^ ((r >> 2) & 1)) << 4); }
 
 template <int DPAD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -85,16 +83,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
     uint64_t *qk_full = bars, *v_full = bars + 2, *slot_free = bars + 4, *s_full = bars + 6;
     uint64_t *p_full = bars + 8, *o_full = bars + 10, *o_free = bars + 12, *drain = bars + 14;
+    uint64_t *stage_full = bars + 15, *stage_free = bars + 17;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int d = a.d, n = a.geom.n, nch = d / 8;
+    const int d = a.d, n = a.geom.n;
 
     if (threadIdx.x == 0) {
         for (int g = 0; g < 2; ++g) {
-            mbar_init(&qk_full[g], 32);
-            mbar_init(&v_full[g], 32);
+            mbar_init(&qk_full[g], 32);  // the loader's 32 lanes (rows and masks) + Q, K bytes
+            mbar_init(&v_full[g], 1);
             mbar_init(&slot_free[g], 1);
             mbar_init(&s_full[g], 1);
             mbar_init(&p_full[g], BQ);
@@ -102,29 +101,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&o_free[g], BQ);
         }
         mbar_init(drain, 1);
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(&stage_full[g], BQ);
+            mbar_init(&stage_free[g], BQ);
+        }
         *abort = 0;
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(tslot, kTmemCols);
-    // zero, once, the padding columns no copy writes: Q and K columns d..79,
-    // V columns d..127 (their products with P and Q are then exactly 0)
-    if (L::HAS_B) {
-        for (int i = threadIdx.x; i < 2 * BQ * 8; i += kThreads) {
-            const int g = i / (BQ * 8), r = (i / 8) % BQ, c = i % 8;
-            uint8_t *slot = sm + g * L::SLOT;
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            if (8 + c >= nch) {
-                if (c < 2) {
-                    const uint32_t o = L::TILE_A + (r >> 3) * 256 + sw32(r & 7, c);
-                    *reinterpret_cast<uint4 *>(slot + o) = z;
-                    *reinterpret_cast<uint4 *>(slot + L::TILE + o) = z;
-                }
-                *reinterpret_cast<uint4 *>(slot + 2 * L::TILE + L::TILE_A + (r >> 3) * 1024 +
-                                           sw128(r & 7, c)) = z;
-            }
-        }
-    }
-    fence_async_smem();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -139,105 +123,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ loader of slot g
         const int g = warp - 2;
         uint8_t *sQ = sm + g * L::SLOT, *sK = sQ + L::TILE, *sV = sK + L::TILE;
-        const char *gq = static_cast<const char *>(a.q);
-        const char *gk = static_cast<const char *>(a.k);
-        const char *gv = static_cast<const char *>(a.v);
-        const long ldq = a.ldq * 2, ldk = a.ldk * 2, ldv = a.ldv * 2;  // row pitches in bytes
+        const uint8_t *qg = static_cast<const uint8_t *>(a.q);
+        const uint8_t *kg = static_cast<const uint8_t *>(a.k);
+        const uint8_t *vg = static_cast<const uint8_t *>(a.v);
         const WinGeom &geo = a.geom;
         const int pack = BQ / n;
-        const int c8 = lane & 7;  // 16-byte chunk (columns 8 c8 .. 8 c8 + 7) of the main copies
+        int last_rest = -1;  // (batch item, tile) whose rows and masks the slot holds
         for (int k = 0; unit_of(g, k) < u1; ++k) {
             const int u = unit_of(g, k);
             const int h = u % a.heads, rest = u / a.heads, tile = rest % sc.tiles,
                       b = rest / sc.tiles;
             if (!mbar_wait(&slot_free[g], (k & 1) ^ 1, abort, status)) break;
-            int inf[4];
+            if (lane == 0) {
+                const long blk = ((long)b * sc.tiles + tile) * a.heads + h;
+                mbar_expect_tx_only(&qk_full[g], 2 * L::TILE);
+                bulk_load(sQ, qg + blk * L::TILE, L::TILE, &qk_full[g]);
+                bulk_load(sK, kg + blk * L::TILE, L::TILE, &qk_full[g]);
+                mbar_expect_tx(&v_full[g], L::TILE);
+                bulk_load(sV, vg + blk * L::TILE, L::TILE, &v_full[g]);
+            }
+            // rows and masks depend on (batch item, tile) only: the heads of one tile
+            // follow each other in this slot, so most units reuse them
+            if (rest != last_rest) {
+                last_rest = rest;
+                int inf[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int r = q * 32 + lane;
-                const int wit = r / n, win = tile * pack + wit, slot = r - wit * n;
-                long row = -1;
-                int in = -1;
-                if (win < geo.nwin) {
-                    int wrap;
-                    row = (long)b * a.k_bstride + window_token(geo, win, slot, &wrap);
-                    in = wit * 8 + wrap;
+                for (int q = 0; q < 4; ++q) {
+                    const int r = q * 32 + lane;
+                    const int wit = r / n, win = tile * pack + wit, slot = r - wit * n;
+                    long row = -1;
+                    int in = -1;
+                    if (win < geo.nwin) {
+                        int wrap;
+                        row = (long)b * a.k_bstride + window_token(geo, win, slot, &wrap);
+                        in = wit * 8 + wrap;
+                    }
+                    inf[q] = in;
+                    info[g * BQ + r] = in;
+                    rowsm[g * BQ + r] = row;
                 }
-                inf[q] = in;
-                info[g * BQ + r] = in;
-                rowsm[g * BQ + r] = row;
+                // one 128-bit key mask per mask key: keys of the same window and wrap code
+                for (int v = 0; v < kKeys; ++v)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t bits = __ballot_sync(0xffffffffu, inf[q] == v);
+                        if (lane == 0) kmask[(g * kKeys + v) * 4 + q] = bits;
+                    }
             }
             __syncwarp();
-            const long hoff = (long)h * d * 2;
-            // columns 0..63: eight lanes per row, four rows per instruction; Q and K first
-#pragma unroll 4
-            for (int it = 0; it < BQ / 4; ++it) {
-                const int r = 4 * it + (lane >> 3);
-                const long row = rowsm[g * BQ + r];
-                const uint32_t bytes = row >= 0 ? 16u : 0u;
-                const long rr = row >= 0 ? row : 0;
-                const uint32_t o = (r >> 3) * 1024 + sw128(r & 7, c8);
-                cp_async16(sQ + o, gq + rr * ldq + hoff + c8 * 16, bytes);
-                cp_async16(sK + o, gk + rr * ldk + hoff + c8 * 16, bytes);
-            }
-            if (L::HAS_B) {  // columns 64 .. d-1: one row per lane
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = q * 32 + lane;
-                    const long row = rowsm[g * BQ + r];
-                    const uint32_t bytes = row >= 0 ? 16u : 0u;
-                    const long rr = row >= 0 ? row : 0;
-                    for (int c = 8; c < nch; ++c) {
-                        const uint32_t o = L::TILE_A + (r >> 3) * 256 + sw32(r & 7, c - 8);
-                        cp_async16(sQ + o, gq + rr * ldq + hoff + c * 16, bytes);
-                        cp_async16(sK + o, gk + rr * ldk + hoff + c * 16, bytes);
-                    }
-                }
-            }
-            cp_async_commit();
-#pragma unroll 4
-            for (int it = 0; it < BQ / 4; ++it) {
-                const int r = 4 * it + (lane >> 3);
-                const long row = rowsm[g * BQ + r];
-                const uint32_t bytes = row >= 0 ? 16u : 0u;
-                const long rr = row >= 0 ? row : 0;
-                cp_async16(sV + (r >> 3) * 1024 + sw128(r & 7, c8), gv + rr * ldv + hoff + c8 * 16,
-                           bytes);
-            }
-            if (L::HAS_B) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = q * 32 + lane;
-                    const long row = rowsm[g * BQ + r];
-                    const uint32_t bytes = row >= 0 ? 16u : 0u;
-                    const long rr = row >= 0 ? row : 0;
-                    for (int c = 8; c < nch; ++c)
-                        cp_async16(sV + L::TILE_A + (r >> 3) * 1024 + sw128(r & 7, c - 8),
-                                   gv + rr * ldv + hoff + c * 16, bytes);
-                }
-            }
-            cp_async_commit();
-            // one 128-bit key mask per mask key: keys of the same window and wrap code
-            for (int v = 0; v < kKeys; ++v)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t bits = __ballot_sync(0xffffffffu, inf[q] == v);
-                    if (lane == 0) kmask[(g * kKeys + v) * 4 + q] = bits;
-                }
-            cp_async_wait_group1();  // Q and K have landed (V may still be in flight)
-            fence_async_smem();
             mbar_arrive(&qk_full[g]);
-            cp_async_wait_all();
-            fence_async_smem();
-            mbar_arrive(&v_full[g]);
         }
-        cp_async_commit();
-        cp_async_wait_all();
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(BQ, BQ);
-            constexpr uint32_t idesc_o = idesc_bf16(BQ, L::NPV, true);
+            constexpr uint32_t idesc_o = idesc_bf16(BQ, 64, true);   // V columns 0..63
+            constexpr uint32_t idesc_ob = idesc_bf16(BQ, 16, true);  // V columns 64..79
             bool ok = true, any = false;
             for (int k = 0; ok && unit_of(0, k) < u1; ++k) {
                 for (int g = 0; g < 2 && ok; ++g) {
@@ -263,10 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!mbar_wait(&o_free[g], (k & 1) ^ 1, abort, status)) { ok = false; break; }
                     fence_after_sync();
                     const uint32_t aV = smem_u32(sm + g * L::SLOT + 2 * L::TILE);
+                    const uint32_t tO = tmem + g * 256 + 128;
 #pragma unroll
-                    for (int ks = 0; ks < BQ / 16; ++ks)
-                        mma_bf16_ts(tmem + g * 256 + 128, tmem + g * 256 + ks * 8,
-                                    sdesc_sw128_mn(aV + ks * 2048, L::TILE_A), idesc_o, ks > 0);
+                    for (int ks = 0; ks < BQ / 16; ++ks) {
+                        mma_bf16_ts(tO, tmem + g * 256 + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
+                                    idesc_o, ks > 0);
+                        if (L::HAS_B)
+                            mma_bf16_ts(tO + 64, tmem + g * 256 + ks * 8,
+                                        sdesc_sw32_mn(aV + L::TILE_A + ks * 512), idesc_ob, ks > 0);
+                    }
                     mma_commit(&o_full[g]);
                     mma_commit(&slot_free[g]);  // Q, K and V of this slot are read
                 }
@@ -285,6 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_s = tmem + lane_base + g * 256, t_o = t_s + 128;
         const float sl2 = a.scale * 1.4426950408889634f;
         const int nch = d / 8;
+        // staging row pitch: an odd number of 16-byte units where that fits
+        const int pitch = nch * 16 + (nch % 8 == 0 ? 16 : 0);
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
         // the row's own keys: its window inside the tile
         const int c_lo = n < BQ ? (r / n) * n : 0;
@@ -366,31 +314,47 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
             fence_before_sync();
             mbar_arrive(&p_full[g]);
+            // O / l to global memory through the staging rows: consecutive lanes
+            // store consecutive 16-byte pieces of one token row
             if (!mbar_wait(&o_full[g], k & 1, abort, status)) break;
+            if (!mbar_wait(&stage_free[g], (k & 1) ^ 1, abort, status)) break;
             fence_after_sync();
             const float inv = 1.f / l;
-            __nv_bfloat16 *dst = og + (live ? qrow : 0) * a.ldo + (long)h * d;
-#pragma unroll
-            for (int c0 = 0; c0 < DPAD; c0 += 16) {
-                uint32_t ov[16];
-                tmem_ld16(t_o + c0, ov);
+            uint8_t *stg = sm + L::OFF_STG + g * L::STG;
+            long *orow = reinterpret_cast<long *>(sm + L::OFF_OROW) + g * BQ;
+            {
+                uint32_t ov[DPAD];
+                tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(ov));
+                tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
+                if (DPAD > 64) tmem_ld16(t_o + 64, *reinterpret_cast<uint32_t(*)[16]>(ov + 64));
                 tmem_ld_wait();
-                if (live) {
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        if ((c0 >> 3) + c < nch) {
-                            uint4 v;
-                            v.x = pack_bf16(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
-                            v.y = pack_bf16(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
-                            v.z = pack_bf16(__uint_as_float(ov[8 * c + 4]) * inv, __uint_as_float(ov[8 * c + 5]) * inv);
-                            v.w = pack_bf16(__uint_as_float(ov[8 * c + 6]) * inv, __uint_as_float(ov[8 * c + 7]) * inv);
-                            *reinterpret_cast<uint4 *>(dst + c0 + 8 * c) = v;
-                        }
+                for (int u = 0; u < DPAD / 8; ++u)
+                    if (u < nch) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(ov[8 * u + 0]) * inv, __uint_as_float(ov[8 * u + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(ov[8 * u + 2]) * inv, __uint_as_float(ov[8 * u + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(ov[8 * u + 4]) * inv, __uint_as_float(ov[8 * u + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(ov[8 * u + 6]) * inv, __uint_as_float(ov[8 * u + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(stg + r * pitch + u * 16) = v;
                     }
-                }
+                orow[r] = live ? qrow : -1;
             }
             fence_before_sync();
-            mbar_arrive(&o_free[g]);
+            mbar_arrive(&o_free[g]);  // O is read: the slot's next P V may overwrite it
+            mbar_arrive(&stage_full[g]);
+            if (!mbar_wait(&stage_full[g], k & 1, abort, status)) break;
+            {
+                __nv_bfloat16 *obase = og + (long)h * d;
+                for (int i = r; i < BQ * nch; i += BQ) {
+                    const int row = i / nch, u = i - row * nch;
+                    const long orw = orow[row];
+                    if (orw >= 0)
+                        *reinterpret_cast<uint4 *>(obase + orw * a.ldo + u * 8) =
+                            *reinterpret_cast<const uint4 *>(stg + row * pitch + u * 16);
+                }
+            }
+            mbar_arrive(&stage_free[g]);
         }
     }
     if (*abort) {
@@ -412,6 +376,10 @@ cudaError_t launch_win(const AttnArgs &a, cudaStream_t s) {
     using L = WinLayout<DPAD>;
     int *status = device_status_ptr();
     if (!status) return cudaErrorInvalidValue;
+    // the tiles are the tiled-head-layout blocks the window projection wrote
+    if (a.tq.mode != THL_WINDOW || a.tk.mode != THL_WINDOW || a.tv.mode != THL_WINDOW ||
+        a.tq.vpad || a.tk.vpad || a.tv.vpad || L::TILE != (int)thl_block_bytes(a.d, 0))
+        return cudaErrorInvalidValue;
     WinSched sc;
     const int pack = BQ / a.geom.n;
     sc.tiles = (a.geom.nwin + pack - 1) / pack;
@@ -426,15 +394,6 @@ cudaError_t launch_win(const AttnArgs &a, cudaStream_t s) {
 }
 
 }  // namespace
-
-// Windows of 64 or 128 tokens (any shape and shift), head width 64..80.
-bool attention_win_tc_supported(const AttnArgs &a) {
-    if (a.dtype != DT_BF16 || a.mode != ATT_WINDOW) return false;
-    if (!(a.geom.n == 64 || a.geom.n == 128) || a.q_bstride != a.k_bstride) return false;
-    if (a.d % 8 || a.d < 64 || a.d > 80) return false;
-    if (a.ldq % 8 || a.ldk % 8 || a.ldv % 8 || a.ldo % 8) return false;
-    return true;
-}
 
 cudaError_t launch_attention_win_tc(const AttnArgs &a, cudaStream_t s) {
     if (a.d <= 64) return launch_win<64>(a, s);

@@ -118,9 +118,20 @@ enum DType { DT_F32 = 0, DT_BF16 = 1 };
 cudaError_t launch_proxy_average(int dtype, const ProxyGeom &g, int B, int D, const void *z,
                                  void *proxies, cudaStream_t s);
 
+// Tile geometry of an operand stored in tiled head layout (thl.cuh).
+struct ThlDesc {
+    int mode;      // 0: plain row-major; 1: identity tiles; 2: window tiles
+    int vpad;      // columns 64.. padded to 128 (the row kernel's V)
+    int tiles;     // 128-row tiles per batch item
+    long rows_pb;  // rows per batch item
+    int pack;      // windows per tile (window tiles)
+    WinGeom g;     // window tiles
+};
 // C_s[rows, nseg] = A[rows, K] * W_s[nseg, K]^T (+ R_s), s < nmat.
 // A has row stride lda; C_s and R_s share row stride ldc.  R_s may equal C_s
-// (in-place residual) or be null.
+// (in-place residual) or be null.  thl[s] (or null) asks for
+// C_s in tiled head layout instead (heads of width d, no residual); only the
+// launchers that report support for it accept one.
 struct GemmArgs {
     int dtype;
     const void *A;
@@ -130,6 +141,8 @@ struct GemmArgs {
     const void *R[3];
     long ldc;
     int rows, nseg, K, nmat;
+    const ThlDesc *thl[3];
+    int heads, d;
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s);
 
@@ -149,6 +162,7 @@ struct AttnArgs {
     int nq, nk;                    // ATT_ROWS sizes per batch item
     WinGeom geom;                  // ATT_WINDOW geometry
     float scale;                   // 1/sqrt(d)
+    ThlDesc tq, tk, tv;            // layouts of q, k, v (mode 0: row-major with ldq...)
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s);
 

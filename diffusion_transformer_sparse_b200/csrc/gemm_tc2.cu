@@ -27,11 +27,18 @@
 //              the leader (a remote mbarrier arrive from the peer) that the
 //              accumulator is free, and writes the tile out with TMA stores:
 //              whole 64-byte row segments instead of one 16-byte piece per
-//              row and instruction.
+//              row and instruction.  An output in tiled head layout (the Q,
+//              K and V operands of the attention kernels) is written
+//              instead straight from registers, 16 bytes (8 columns of one
+//              head) at a time, into its (tile, head) block at the row's
+//              place in the swizzled tile; the block's padding columns are
+//              written as zeros by the lane that writes the head's last
+//              columns.
 // Two TMEM accumulators overlap the next tile's MMAs with this tile's
 // epilogue.  Every wait is bounded (2 s); a timeout records
 // PTDIT_ERR_TIMEOUT in the status word.
 #include "tc_util.cuh"
+#include "thl.cuh"
 
 namespace ptdit {
 namespace {
@@ -50,6 +57,11 @@ struct Tc2Maps {
 struct Tc2Params {
     void *C[3];
     const void *R[3];
+    Thl thl[3];  // mode THL_OFF: row-major output through the staging tiles
+    int heads, d;     // tiled outputs: heads and head width
+    int nunits[3];    // tiled outputs: 16-byte units per block row
+    FastDiv f_d;
+    uint32_t blk[3];  // tiled outputs: bytes per (tile, head) block
     long ldc;
     int rows, nseg, nmat;
     int n_tiles;  // output tiles per weight matrix (the last may be narrower)
@@ -288,6 +300,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int row0 = m_tile * 2 * BMC + rank * BMC + q * 32;
             const int col0 = n_tile * BN;
             const int nchunk = tile_width<BN>(p, n_tile) / 32;
+            if (p.thl[seg].mode != THL_OFF) {
+                // ---- tiled head layout: this lane's row, 8 columns per store
+                const Thl &tl = p.thl[seg];
+                const int grow = row0 + lane;
+                uint8_t *rbase = nullptr;
+                int tr = 0;
+                if (grow < p.rows) {
+                    const int b = grow / static_cast<int>(tl.rows_pb);
+                    int tile;
+                    thl_locate(tl, grow - static_cast<long>(b) * tl.rows_pb, tile, tr);
+                    rbase = static_cast<uint8_t *>(p.C[seg]) +
+                            ((long)b * tl.tiles + tile) * p.heads * (long)p.blk[seg];
+                }
+                if (!mbar_wait(&tfull[acc], acc_phase, abort, p.status)) break;
+                fence_after_sync();
+                const uint32_t tbase =
+                    tmem + acc * L::ACC_STRIDE + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+                for (int c = 0; c < nchunk; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + 32 * c, r);
+                    tmem_ld_wait();
+                    if (!rbase) continue;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int col = col0 + 32 * c + 8 * j;
+                        const int h = fdiv(p.f_d, col), u = (col - h * p.d) >> 3;
+                        uint8_t *hb = rbase + (long)h * p.blk[seg];
+                        uint4 o;
+                        o.x = pack_bf16(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+                        o.y = pack_bf16(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+                        o.z = pack_bf16(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+                        o.w = pack_bf16(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+                        *reinterpret_cast<uint4 *>(hb + thl_unit(tr, u, tl.vpad)) = o;
+                        if (8 * (u + 1) == p.d)  // the head's last columns: zero the padding units
+                            for (int z = u + 1; z < p.nunits[seg]; ++z)
+                                *reinterpret_cast<uint4 *>(hb + thl_unit(tr, z, tl.vpad)) =
+                                    make_uint4(0, 0, 0, 0);
+                    }
+                }
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+                continue;
+            }
             const bool has_r = p.R[seg] != nullptr;
             if (lane == 0) {
                 bulk_wait_read_all();  // the previous tile's stores have left the staging tile
@@ -382,9 +441,18 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
     }
     Tc2Params p;
     Tc2Maps mo;
+    memset(&p, 0, sizeof p);
+    p.heads = a.heads;
+    p.d = a.d > 0 ? a.d : 1;
+    p.f_d = make_fastdiv(p.d);
     for (int i = 0; i < 3; ++i) {
         p.C[i] = i < a.nmat ? a.C[i] : nullptr;
         p.R[i] = i < a.nmat ? a.R[i] : nullptr;
+        if (i < a.nmat && a.thl[i]) {
+            p.thl[i] = *a.thl[i];
+            p.blk[i] = thl_block_bytes(a.d, a.thl[i]->vpad);
+            p.nunits[i] = thl_units(a.d, a.thl[i]->vpad);
+        }
         // unused slots get a valid map over C[0] that no tile refers to
         const void *c = p.C[i] ? p.C[i] : a.C[0];
         const void *r = p.R[i] ? p.R[i] : c;
@@ -431,18 +499,15 @@ bool gemm_tc2_supported(const GemmArgs &a) {
     if (a.K < BK || a.K % BK || a.rows < 2 * BMC || a.lda % 8 || a.ldc % 8) return false;
     if (a.nseg % 64) return false;  // tile widths: multiples of 32 per CTA half and epilogue chunk
     if ((uintptr_t)a.A % 16) return false;
-    for (int i = 0; i < a.nmat; ++i)
+    for (int i = 0; i < a.nmat; ++i) {
         if ((uintptr_t)a.W[i] % 16 || (uintptr_t)a.C[i] % 16 || (uintptr_t)a.R[i] % 16)
             return false;
+        // tiled head layout: whole 8-column units per head, no residual
+        if (a.thl[i] && (a.R[i] || a.d < 8 || a.d % 8 || a.heads * a.d != a.nseg)) return false;
+    }
     return true;
 }
 
-cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) {
-#ifndef PTDIT_GEMM2_BN
-    return launch_bn2<256, 5>(a, s);
-#else
-    return PTDIT_GEMM2_BN == 192 ? launch_bn2<192, 6>(a, s) : launch_bn2<256, 5>(a, s);
-#endif
-}
+cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) { return launch_bn2<256, 5>(a, s); }
 
 }  // namespace ptdit

@@ -11,6 +11,9 @@
 //        12 Q,K,V = z_out W_swsa^T 13 window core (shift s) 14 z_out += O W_swsa,o^T
 // The residual stream lives in z_out from step 8 on; steps 11 and 14 add in
 // place (each output element is read and written by the same thread).
+// Where the tensor-core attention kernels run (bf16, head width 64..80), the
+// projections write Q, K and V in tiled head layout (thl.cuh): one block per
+// (tile, head) in the order the attention kernel reads them.
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -19,6 +22,7 @@
 
 #include "common.cuh"
 #include "ptdit.h"
+#include "thl.cuh"
 
 namespace ptdit {
 cudaError_t launch_gemm_simt(const GemmArgs &a, cudaStream_t s);
@@ -28,10 +32,13 @@ cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
 bool gemm_tc2_supported(const GemmArgs &a);
 cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s);
 bool attention_tc_supported(const AttnArgs &a);
+bool attention_thl_supported(const AttnArgs &a);
 cudaError_t launch_attention_tc(const AttnArgs &a, cudaStream_t s);
 
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s) {
     if (gemm_tc2_supported(a)) return launch_gemm_tc2(a, s);
+    for (int i = 0; i < a.nmat; ++i)  // only the 2-SM kernel writes tiled head layout
+        if (a.thl[i]) return cudaErrorNotSupported;
     if (gemm_tc_supported(a)) return launch_gemm_tc(a, s);
     return launch_gemm_simt(a, s);
 }
@@ -194,20 +201,62 @@ struct Ws {
     size_t P, Qp, Kp, Vp, Ap, Pp, Kc, Vc, Q, K, V, O, total;
 };
 
+// Whether the attention operands of this shape go through tiled head layout.
+bool thl_shape(const Dims &d) { return d.dtype == PTDIT_BF16 && d.d >= 64 && d.d <= 80 && d.d % 8 == 0; }
+
+// Bytes of `rows_pb` rows per batch item in tiled head layout.
+size_t thl_bytes(const Dims &d, long rows_pb, int vpad) {
+    return (size_t)d.B * ((rows_pb + kThlRows - 1) / kThlRows) * d.heads *
+           thl_block_bytes(d.d, vpad);
+}
+
 Ws ws_layout(const Dims &d, long M) {
     Ws L;
     size_t off = 0;
-    auto take = [&](size_t elems) {
+    auto take = [&](size_t bytes) {
         const size_t o = off;
-        off += align256(elems * d.elem);
+        off += align256(bytes);
         return o;
     };
-    const size_t pm = (size_t)d.B * M * d.D, tn = (size_t)d.B * d.N * d.D;
-    L.P = take(pm); L.Qp = take(pm); L.Kp = take(pm); L.Vp = take(pm);
-    L.Ap = take(pm); L.Pp = take(pm); L.Kc = take(pm); L.Vc = take(pm);
-    L.Q = take(tn); L.K = take(tn); L.V = take(tn); L.O = take(tn);
+    auto mx = [](size_t a, size_t b) { return a > b ? a : b; };
+    const size_t pm = (size_t)d.B * M * d.D * d.elem, tn = (size_t)d.B * d.N * d.D * d.elem;
+    const bool t = thl_shape(d);
+    // Q and K blocks of 80 columns; V blocks padded to 128 for the row kernel
+    const size_t pq = t ? thl_bytes(d, M, 0) : 0, pv = t ? thl_bytes(d, M, 1) : 0;
+    const size_t tq = t ? thl_bytes(d, d.N, 0) : 0, tv = t ? thl_bytes(d, d.N, 1) : 0;
+    L.P = take(pm); L.Qp = take(mx(pm, pq)); L.Kp = take(mx(pm, pq)); L.Vp = take(mx(pm, pv));
+    L.Ap = take(pm); L.Pp = take(pm); L.Kc = take(mx(pm, pq)); L.Vc = take(mx(pm, pv));
+    L.Q = take(mx(tn, tq)); L.K = take(mx(tn, tq)); L.V = take(mx(tn, tv)); L.O = take(tn);
     L.total = off;
     return L;
+}
+
+ThlDesc thl_identity(long rows_pb, int vpad) {
+    ThlDesc t;
+    memset(&t, 0, sizeof t);
+    t.mode = THL_IDENTITY;
+    t.vpad = vpad;
+    t.rows_pb = rows_pb;
+    t.tiles = (int)((rows_pb + kThlRows - 1) / kThlRows);
+    t.pack = 1;
+    return t;
+}
+
+ThlDesc thl_window(const WinGeom &g, long N, int vpad) {
+    ThlDesc t;
+    memset(&t, 0, sizeof t);
+    t.mode = THL_WINDOW;
+    t.vpad = vpad;
+    t.rows_pb = N;
+    t.pack = kThlRows / g.n;
+    t.tiles = (g.nwin + t.pack - 1) / t.pack;
+    t.g = g;
+    return t;
+}
+
+// Whether some tile rows of this layout hold no token (they must read as zeros).
+bool thl_has_empty_rows(const ThlDesc &t) {
+    return t.mode == THL_IDENTITY ? t.rows_pb % kThlRows != 0 : t.g.nwin % t.pack != 0;
 }
 
 int check_ws(const Dims &d, long M, const void *ws, size_t ws_bytes, Ws *L) {
@@ -220,6 +269,12 @@ int check_ws(const Dims &d, long M, const void *ws, size_t ws_bytes, Ws *L) {
 }
 
 // ------------------------------------------------------------------ launch helpers
+#define TRY(x)                         \
+    do {                               \
+        int _rc = (x);                 \
+        if (_rc != PTDIT_OK) return _rc; \
+    } while (0)
+
 struct Run {
     const Dims &d;
     cudaStream_t s;
@@ -252,6 +307,60 @@ int gemm(const Run &r, int kind, const void *A, long rows, int nmat, const void 
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
 }
 
+// Projections whose outputs C_i are in tiled head layout where thl[i] is set:
+// one fused launch when the 2-SM kernel takes the shape, else one row-major
+// projection per output into `scratch` followed by a relayout.  Tile rows
+// that hold no token are zeroed.
+int gemm_thl(const Run &r, int kind, const void *A, long rows, int nmat, const void *const W[3],
+             void *const C[3], const ThlDesc *const thl[3], void *scratch, const char *what) {
+    GemmArgs g;
+    memset(&g, 0, sizeof g);
+    g.dtype = r.d.dtype;
+    g.A = A;
+    g.lda = r.d.D;
+    for (int i = 0; i < nmat; ++i) {
+        g.W[i] = W[i];
+        g.C[i] = C[i];
+        g.thl[i] = thl[i];
+    }
+    g.ldc = r.d.D;
+    g.rows = (int)rows;
+    g.nseg = r.d.D;
+    g.K = r.d.D;
+    g.nmat = nmat;
+    g.heads = r.d.heads;
+    g.d = r.d.d;
+    if (gemm_tc2_supported(g)) {
+        timing_begin(kind, r.s);
+        cudaError_t e = launch_gemm_tc2(g, r.s);
+        timing_end(r.s);
+        count_launch();
+        if (e != cudaSuccess) return cuda_fail(e, what);
+    } else {
+        for (int i = 0; i < nmat; ++i) {
+            const void *Wi[3] = {W[i], nullptr, nullptr};
+            void *Ci[3] = {thl[i] ? scratch : C[i], nullptr, nullptr};
+            TRY(gemm(r, kind, A, rows, 1, Wi, Ci, nullptr, what));
+            if (!thl[i]) continue;
+            timing_begin(kind, r.s);
+            cudaError_t e = launch_thl_fill(*thl[i], r.d.B, r.d.heads, r.d.d, scratch, r.d.D, C[i], r.s);
+            timing_end(r.s);
+            count_launch();
+            if (e != cudaSuccess) return cuda_fail(e, "tiled head layout");
+        }
+        return PTDIT_OK;  // the relayout wrote every tile row
+    }
+    for (int i = 0; i < nmat; ++i) {
+        if (!thl[i] || !thl_has_empty_rows(*thl[i])) continue;
+        timing_begin(kind, r.s);
+        cudaError_t e = launch_thl_fill(*thl[i], r.d.B, r.d.heads, r.d.d, nullptr, r.d.D, C[i], r.s);
+        timing_end(r.s);
+        count_launch();
+        if (e != cudaSuccess) return cuda_fail(e, "tiled head layout");
+    }
+    return PTDIT_OK;
+}
+
 int attention(const Run &r, int kind, AttnArgs a, const char *what) {
     a.dtype = r.d.dtype;
     a.heads = r.d.heads;
@@ -266,11 +375,6 @@ int attention(const Run &r, int kind, AttnArgs a, const char *what) {
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
 }
 
-#define TRY(x)                         \
-    do {                               \
-        int _rc = (x);                 \
-        if (_rc != PTDIT_OK) return _rc; \
-    } while (0)
 
 // GIIM: z_out = (z_in +) CS(z_in, SA(Average(z_in)) (+ P_a)).
 int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
@@ -282,20 +386,28 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
     timing_end(r.s);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "proxy average");
+    AttnArgs pa;  // proxy self-attention
+    memset(&pa, 0, sizeof pa);
+    pa.mode = ATT_ROWS;
+    pa.dtype = d.dtype;
+    pa.d = d.d;
+    pa.q = r.at(r.L.Qp); pa.k = r.at(r.L.Kp); pa.v = r.at(r.L.Vp); pa.o = r.at(r.L.Ap);
+    pa.q_bstride = pa.k_bstride = pg.M;
+    pa.nq = pa.nk = pg.M;
+    const bool tiled = attention_thl_supported(pa);
+    const ThlDesc tp = thl_identity(pg.M, 0), tpv = thl_identity(pg.M, 1);
+    if (tiled) {
+        pa.tq = pa.tk = tp;
+        pa.tv = tpv;
+    }
     {
         const void *W[3] = {psa->wq, psa->wk, psa->wv};
         void *C[3] = {r.at(r.L.Qp), r.at(r.L.Kp), r.at(r.L.Vp)};
-        TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.P), BM, 3, W, C, nullptr, "proxy QKV projection"));
+        const ThlDesc *T[3] = {tiled ? &tp : nullptr, tiled ? &tp : nullptr, tiled ? &tpv : nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.P), BM, 3, W, C, T, r.at(r.L.Ap),
+                     "proxy QKV projection"));
     }
-    {
-        AttnArgs a;
-        memset(&a, 0, sizeof a);
-        a.mode = ATT_ROWS;
-        a.q = r.at(r.L.Qp); a.k = r.at(r.L.Kp); a.v = r.at(r.L.Vp); a.o = r.at(r.L.Ap);
-        a.q_bstride = a.k_bstride = pg.M;
-        a.nq = a.nk = pg.M;
-        TRY(attention(r, PTDIT_K_ATTN_PROXY, a, "proxy self-attention"));
-    }
+    TRY(attention(r, PTDIT_K_ATTN_PROXY, pa, "proxy self-attention"));
     {
         const void *W[3] = {psa->wo, nullptr, nullptr};
         void *C[3] = {r.at(r.L.Pp), nullptr, nullptr};
@@ -303,27 +415,34 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
                             nullptr};
         TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.Ap), BM, 1, W, C, R, "proxy output projection"));
     }
+    AttnArgs ca;  // cross-attention: latent queries, proxy keys and values
+    memset(&ca, 0, sizeof ca);
+    ca.mode = ATT_ROWS;
+    ca.q = r.at(r.L.Q); ca.k = r.at(r.L.Kc); ca.v = r.at(r.L.Vc); ca.o = r.at(r.L.O);
+    ca.q_bstride = d.N;
+    ca.k_bstride = pg.M;
+    ca.nq = (int)d.N;
+    ca.nk = pg.M;
+    const ThlDesc tn = thl_identity(d.N, 0);
+    if (tiled) {
+        ca.tq = tn;
+        ca.tk = tp;
+        ca.tv = tpv;
+    }
     {
         const void *W[3] = {cross->wk, cross->wv, nullptr};
         void *C[3] = {r.at(r.L.Kc), r.at(r.L.Vc), nullptr};
-        TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.Pp), BM, 2, W, C, nullptr, "proxy K/V projection"));
+        const ThlDesc *T[3] = {tiled ? &tp : nullptr, tiled ? &tpv : nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.Pp), BM, 2, W, C, T, r.at(r.L.Ap),
+                     "proxy K/V projection"));
     }
     {
         const void *W[3] = {cross->wq, nullptr, nullptr};
         void *C[3] = {r.at(r.L.Q), nullptr, nullptr};
-        TRY(gemm(r, PTDIT_K_GEMM, z_in, BN, 1, W, C, nullptr, "latent Q projection"));
+        const ThlDesc *T[3] = {tiled ? &tn : nullptr, nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 1, W, C, T, r.at(r.L.O), "latent Q projection"));
     }
-    {
-        AttnArgs a;
-        memset(&a, 0, sizeof a);
-        a.mode = ATT_ROWS;
-        a.q = r.at(r.L.Q); a.k = r.at(r.L.Kc); a.v = r.at(r.L.Vc); a.o = r.at(r.L.O);
-        a.q_bstride = d.N;
-        a.k_bstride = pg.M;
-        a.nq = (int)d.N;
-        a.nk = pg.M;
-        TRY(attention(r, PTDIT_K_ATTN_CROSS, a, "cross-attention"));
-    }
+    TRY(attention(r, PTDIT_K_ATTN_CROSS, ca, "cross-attention"));
     {
         const void *W[3] = {cross->wo, nullptr, nullptr};
         void *C[3] = {z_out, nullptr, nullptr};
@@ -338,20 +457,24 @@ int run_window(const Run &r, const WinGeom &wg, const ptdit_attn_w *w, unsigned 
                const void *x_in, void *x_out) {
     const Dims &d = r.d;
     const long BN = (long)d.B * d.N;
+    AttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.mode = ATT_WINDOW;
+    a.dtype = d.dtype;
+    a.d = d.d;
+    a.q = r.at(r.L.Q); a.k = r.at(r.L.K); a.v = r.at(r.L.V); a.o = r.at(r.L.O);
+    a.q_bstride = a.k_bstride = d.N;
+    a.geom = wg;
+    const bool tiled = attention_thl_supported(a);
+    const ThlDesc tw = thl_window(wg, d.N, 0);  // V too: the window kernel splits its P V
+    if (tiled) a.tq = a.tk = a.tv = tw;
     {
         const void *W[3] = {w->wq, w->wk, w->wv};
         void *C[3] = {r.at(r.L.Q), r.at(r.L.K), r.at(r.L.V)};
-        TRY(gemm(r, PTDIT_K_GEMM, x_in, BN, 3, W, C, nullptr, "window QKV projection"));
+        const ThlDesc *T[3] = {tiled ? &tw : nullptr, tiled ? &tw : nullptr, tiled ? &tw : nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, x_in, BN, 3, W, C, T, r.at(r.L.O), "window QKV projection"));
     }
-    {
-        AttnArgs a;
-        memset(&a, 0, sizeof a);
-        a.mode = ATT_WINDOW;
-        a.q = r.at(r.L.Q); a.k = r.at(r.L.K); a.v = r.at(r.L.V); a.o = r.at(r.L.O);
-        a.q_bstride = a.k_bstride = d.N;
-        a.geom = wg;
-        TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "window attention"));
-    }
+    TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "window attention"));
     {
         const void *W[3] = {w->wo, nullptr, nullptr};
         void *C[3] = {x_out, nullptr, nullptr};
@@ -589,20 +712,27 @@ int ptdit_full_attn(const ptdit_shape *shape, const ptdit_attn_w *w, unsigned fl
     TRY(check_ws(d, 0, ws, ws_bytes, &L));
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
     const long BN = (long)d.B * d.N;
+    AttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.mode = ATT_ROWS;
+    a.dtype = d.dtype;
+    a.d = d.d;
+    a.q = r.at(L.Q); a.k = r.at(L.K); a.v = r.at(L.V); a.o = r.at(L.O);
+    a.q_bstride = a.k_bstride = d.N;
+    a.nq = a.nk = (int)d.N;
+    const bool tiled = attention_thl_supported(a);
+    const ThlDesc tn = thl_identity(d.N, 0), tnv = thl_identity(d.N, 1);
+    if (tiled) {
+        a.tq = a.tk = tn;
+        a.tv = tnv;
+    }
     {
         const void *W[3] = {w->wq, w->wk, w->wv};
         void *C[3] = {r.at(L.Q), r.at(L.K), r.at(L.V)};
-        TRY(gemm(r, PTDIT_K_GEMM, z_in, BN, 3, W, C, nullptr, "QKV projection"));
+        const ThlDesc *T[3] = {tiled ? &tn : nullptr, tiled ? &tn : nullptr, tiled ? &tnv : nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 3, W, C, T, r.at(L.O), "QKV projection"));
     }
-    {
-        AttnArgs a;
-        memset(&a, 0, sizeof a);
-        a.mode = ATT_ROWS;
-        a.q = r.at(L.Q); a.k = r.at(L.K); a.v = r.at(L.V); a.o = r.at(L.O);
-        a.q_bstride = a.k_bstride = d.N;
-        a.nq = a.nk = (int)d.N;
-        TRY(attention(r, PTDIT_K_ATTN_DENSE, a, "full self-attention"));
-    }
+    TRY(attention(r, PTDIT_K_ATTN_DENSE, a, "full self-attention"));
     {
         const void *W[3] = {w->wo, nullptr, nullptr};
         void *C[3] = {z_out, nullptr, nullptr};

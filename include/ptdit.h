@@ -138,7 +138,7 @@ int ptdit_window_attn(const ptdit_shape *shape, const int window[3], const int s
  *   it before any stream capture.  All calls share the one array: calls that
  *   overlap on the GPU (unordered streams or host threads) race.
  */
-#define PTDIT_STATIC_SCRATCH_BYTES (40u << 20)
+#define PTDIT_STATIC_SCRATCH_BYTES (48u << 20)
 int ptdit_window_attn_static(const ptdit_shape *shape, const int window[3], const int shift[3],
                              const ptdit_attn_w *w, unsigned flags, const void *z_in,
                              void *z_out, ptdit_stream_t stream);

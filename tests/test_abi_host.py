@@ -65,9 +65,19 @@ def test_workspace_bytes(L):
     def a(x):
         return (x + 255) // 256 * 256
 
-    want = 8 * a(4 * M * D * e) + 4 * a(4 * N * D * e)
-    assert _bytes(L, s, (1, 4, 4), (1, 8, 8)) == want
-    assert _bytes(L, s, None, (1, 8, 8)) == 4 * a(4 * N * D * e)
+    # bf16 with heads of 72: Q, K and V are stored as (128-row tile, head) blocks of
+    # 20 KB (columns padded to 80), V of the row kernel as 32 KB blocks (padded to 128)
+    def tiled(rows, blk):
+        return 4 * -(-rows // 128) * 16 * blk
+
+    pm, tn = 4 * M * D * e, 4 * N * D * e
+    proxy = 3 * a(pm) + 3 * a(max(pm, tiled(M, 20480))) + 2 * a(max(pm, tiled(M, 32768)))
+    token = 2 * a(max(tn, tiled(N, 20480))) + a(max(tn, tiled(N, 32768))) + a(tn)
+    assert _bytes(L, s, (1, 4, 4), (1, 8, 8)) == proxy + token
+    assert _bytes(L, s, None, (1, 8, 8)) == token
+    # fp32 keeps every operand row-major
+    f = _shape(B=4, H=64, W=64, D=1152, heads=16, dtype=pt.PTDIT_F32)
+    assert _bytes(L, f, (1, 4, 4), (1, 8, 8)) == 8 * a(4 * M * D * 4) + 4 * a(4 * N * D * 4)
     assert _bytes(L, s, (1, 3, 4), (1, 8, 8)) == 0      # 64 not divisible by 3
     assert _bytes(L, s, (1, 4, 4), (1, 8, 7)) == 0
     assert _bytes(L, _shape(D=63, heads=2), None, None) == 0
