@@ -83,7 +83,7 @@ __device__ __forceinline__ void decode(const AttnArgs &a, const RowsSched &sc, i
     b = r / a.heads;
 }
 
-template <int DPAD>
+template <int DPAD, bool SUMV>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_rows_kernel(const __grid_constant__ AttnArgs a, RowsSched sc, int *status) {
     using L = RowsLayout<DPAD>;
@@ -273,14 +273,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < BKV; ++e)
                         if (e >= nvalid) sv[e] = __float_as_uint(-INFINITY);
                 }
-                // row max over 8 independent chains (short dependency chains)
+                // row max over 8 independent chains of three-input maxima
                 float mx[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(sv[c]);
 #pragma unroll
-                for (int e = 8; e < BKV; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
-                float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                for (int e = 8; e < BKV; e += 16)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        mx[c] = e + 8 + c < BKV
+                                    ? fmax3(mx[c], __uint_as_float(sv[e + c]), __uint_as_float(sv[e + 8 + c]))
+                                    : fmaxf(mx[c], __uint_as_float(sv[e + c]));
+                float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
                 tmax *= sl2;
                 if (tmax > m_ref + 8.f) {  // raise the reference; O so far shrinks by alpha
                     const float alpha = m_ref == -INFINITY ? 0.f : ex2_approx(m_ref - tmax);
@@ -307,23 +311,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float ps[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) ps[c] = 0.f;
-                // P as bf16 pairs, written over the first 64 columns of S
+                // P as bf16 pairs, written over the first 64 columns of S.  With
+                // SUMV the row sum comes out of P V (V's ones column) instead of
+                // being added up here.
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[64 * half + 2 * c]), sl2, -ref));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[64 * half + 2 * c + 1]), sl2, -ref));
-                        ps[(2 * c) & 7] += p0;
-                        ps[(2 * c + 1) & 7] += p1;
+                        const float x0 = fmaf(__uint_as_float(sv[64 * half + 2 * c]), sl2, -ref);
+                        const float x1 = fmaf(__uint_as_float(sv[64 * half + 2 * c + 1]), sl2, -ref);
+                        const float p0 = ex2_approx(x0);
+                        const float p1 = ex2_approx(x1);
+                        if (!SUMV) {
+                            ps[(2 * c) & 7] += p0;
+                            ps[(2 * c + 1) & 7] += p1;
+                        }
                         pk[c] = pack_bf16(p0, p1);
                     }
                     tmem_st32(t_s + 32 * half, pk);
                 }
                 tmem_st_wait();
-                const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-                l_i += psum;
+                if (!SUMV)
+                    l_i += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
                 fence_before_sync();
                 mbar_arrive(&p_full[g]);
             }
@@ -334,7 +344,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&o_full[g], (item - 1) & 1, abort, status)) { ok = false; break; }
             if (!mbar_wait(&stage_free[g], (un_count & 1) ^ 1, abort, status)) { ok = false; break; }
             fence_after_sync();
-            const float inv = 1.f / l_i;
             uint8_t *stg = sm + L::OFF_STG + g * L::STG;
             {
                 uint32_t ov[DPAD];
@@ -342,6 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
                 if (DPAD > 64) tmem_ld16(t_o + 64, *reinterpret_cast<uint32_t(*)[16]>(ov + 64));
                 tmem_ld_wait();
+                // SUMV: column d = DPAD - 8 of O holds the row sum of P
+                const float inv = 1.f / (SUMV ? __uint_as_float(ov[DPAD - 8]) : l_i);
 #pragma unroll
                 for (int u = 0; u < DPAD / 8; ++u)
                     if (u < nch) {
@@ -378,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int DPAD>
+template <int DPAD, bool SUMV>
 cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
     using L = RowsLayout<DPAD>;
     int *status = device_status_ptr();
@@ -394,19 +405,21 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
     sc.units = a.B * a.heads * sc.qp;
     const int sms = num_sms() > 0 ? num_sms() : 148;
     const int grid = sc.units < sms ? sc.units : sms;
-    cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<DPAD>,
+    cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<DPAD, SUMV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
-    attn_rows_kernel<DPAD><<<grid, kThreads, L::BYTES, s>>>(a, sc, status);
+    attn_rows_kernel<DPAD, SUMV><<<grid, kThreads, L::BYTES, s>>>(a, sc, status);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention_rows_tc(const AttnArgs &a, cudaStream_t s) {
-    const int dp = (a.d + 15) / 16 * 16;
-    if (dp == 64) return launch_rows<64>(a, s);
-    if (dp == 80) return launch_rows<80>(a, s);
+    // V's ones column (row sums from P V) exists when the head is 8 columns
+    // narrower than its tile (d = 72)
+    if (a.tv.ones) return a.d == 72 ? launch_rows<80, true>(a, s) : cudaErrorInvalidValue;
+    if (a.d == 64) return launch_rows<64, false>(a, s);
+    if (a.d == 80) return launch_rows<80, false>(a, s);
     return cudaErrorInvalidValue;
 }
 

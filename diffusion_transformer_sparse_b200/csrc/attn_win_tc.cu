@@ -70,7 +70,7 @@ struct WinSched {
     int units;  // B x tiles x heads
 };
 
-template <int DPAD>
+template <int DPAD, bool SUMV>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_win_kernel(const __grid_constant__ AttnArgs a, WinSched sc, int *status) {
     using L = WinLayout<DPAD>;
@@ -262,24 +262,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_wait();
                 const uint32_t w0 = c_lo == 0 ? allow[0] : allow[2];
                 const uint32_t w1 = c_lo == 0 ? allow[1] : allow[3];
-                float mx = -INFINITY;
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
                     const bool ok = ((e < 32 ? w0 : w1) >> (e & 31)) & 1u;
                     if (!ok) sv[e] = __float_as_uint(-INFINITY);
-                    mx = fmaxf(mx, __uint_as_float(sv[e]));
                 }
-                const float ref = mx * sl2;
+#pragma unroll
+                for (int e = 0; e < 64; e += 8)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        mx[c] = fmax3(mx[c], __uint_as_float(sv[e + c]), __uint_as_float(sv[e + 4 + c]));
+                const float ref = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sl2;
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
                 uint32_t pp[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), sl2, -ref));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ref));
-                    ps[c & 3] += p0 + p1;
+                    const float x0 = fmaf(__uint_as_float(sv[2 * c]), sl2, -ref);
+                    const float x1 = fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ref);
+                    const float p0 = ex2_approx(x0);
+                    const float p1 = ex2_approx(x1);
+                    if (!SUMV) ps[c & 3] += p0 + p1;
                     pp[c] = pack_bf16(p0, p1);
                 }
-                l = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                if (!SUMV) l = (ps[0] + ps[1]) + (ps[2] + ps[3]);
                 // P columns hold key pairs: this window's 64 keys, zeros for the other window
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
@@ -292,22 +298,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < 4; ++q)
                     tmem_ld32(t_s + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * q));
                 tmem_ld_wait();
-                float mx = -INFINITY;
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int e = 0; e < 128; ++e) {
+                for (int e = 0; e < 128; ++e)
                     if (!((allow[e >> 5] >> (e & 31)) & 1u)) sv[e] = __float_as_uint(-INFINITY);
-                    mx = fmaxf(mx, __uint_as_float(sv[e]));
-                }
-                const float ref = mx * sl2;
+#pragma unroll
+                for (int e = 0; e < 128; e += 8)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        mx[c] = fmax3(mx[c], __uint_as_float(sv[e + c]), __uint_as_float(sv[e + 4 + c]));
+                const float ref = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sl2;
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), sl2, -ref));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ref));
-                    ps[c & 3] += p0 + p1;
+                    const float x0 = fmaf(__uint_as_float(sv[2 * c]), sl2, -ref);
+                    const float x1 = fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ref);
+                    const float p0 = ex2_approx(x0);
+                    const float p1 = ex2_approx(x1);
+                    if (!SUMV) ps[c & 3] += p0 + p1;
                     pk[c] = pack_bf16(p0, p1);
                 }
-                l = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                if (!SUMV) l = (ps[0] + ps[1]) + (ps[2] + ps[3]);
             }
             tmem_st32(t_s, *reinterpret_cast<uint32_t(*)[32]>(pk));
             tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
@@ -319,7 +330,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&o_full[g], k & 1, abort, status)) break;
             if (!mbar_wait(&stage_free[g], (k & 1) ^ 1, abort, status)) break;
             fence_after_sync();
-            const float inv = 1.f / l;
             uint8_t *stg = sm + L::OFF_STG + g * L::STG;
             long *orow = reinterpret_cast<long *>(sm + L::OFF_OROW) + g * BQ;
             {
@@ -328,6 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
                 if (DPAD > 64) tmem_ld16(t_o + 64, *reinterpret_cast<uint32_t(*)[16]>(ov + 64));
                 tmem_ld_wait();
+                // SUMV: column d = DPAD - 8 of O holds the row sum of P
+                const float inv = 1.f / (SUMV ? __uint_as_float(ov[DPAD - 8]) : l);
 #pragma unroll
                 for (int u = 0; u < DPAD / 8; ++u)
                     if (u < nch) {
@@ -371,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int DPAD>
+template <int DPAD, bool SUMV>
 cudaError_t launch_win(const AttnArgs &a, cudaStream_t s) {
     using L = WinLayout<DPAD>;
     int *status = device_status_ptr();
@@ -386,18 +398,22 @@ cudaError_t launch_win(const AttnArgs &a, cudaStream_t s) {
     sc.units = a.B * sc.tiles * a.heads;
     const int sms = num_sms() > 0 ? num_sms() : 148;
     const int grid = (sc.units + 1) / 2 < sms ? (sc.units + 1) / 2 : sms;
-    cudaError_t e = cudaFuncSetAttribute(attn_win_kernel<DPAD>,
+    cudaError_t e = cudaFuncSetAttribute(attn_win_kernel<DPAD, SUMV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
-    attn_win_kernel<DPAD><<<grid, kThreads, L::BYTES, s>>>(a, sc, status);
+    attn_win_kernel<DPAD, SUMV><<<grid, kThreads, L::BYTES, s>>>(a, sc, status);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention_win_tc(const AttnArgs &a, cudaStream_t s) {
-    if (a.d <= 64) return launch_win<64>(a, s);
-    return launch_win<80>(a, s);
+    // V's ones column (row sums from P V) exists when the head is 8 columns
+    // narrower than its tile (d = 72)
+    if (a.tv.ones) return a.d == 72 ? launch_win<80, true>(a, s) : cudaErrorInvalidValue;
+    if (a.d == 64) return launch_win<64, false>(a, s);
+    if (a.d == 80) return launch_win<80, false>(a, s);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace ptdit

@@ -122,6 +122,7 @@ cudaError_t launch_proxy_average(int dtype, const ProxyGeom &g, int B, int D, co
 struct ThlDesc {
     int mode;      // 0: plain row-major; 1: identity tiles; 2: window tiles
     int vpad;      // columns 64.. padded to 128 (the row kernel's V)
+    int ones;      // column d of every token row holds 1 (V: P V then also sums P)
     int tiles;     // 128-row tiles per batch item
     long rows_pb;  // rows per batch item
     int pack;      // windows per tile (window tiles)

@@ -49,3 +49,4 @@ cudaError_t launch_debug_window_map(const WinGeom &g, int32_t *tok, uint8_t *all
 }
 
 }  // namespace ptdit
+

@@ -70,13 +70,15 @@ struct Tc2Params {
     int *status;
 };
 
-template <int BN, int STAGES>
+// STAGING: the row-major epilogue's staging tiles exist (launches whose outputs
+// are all in tiled head layout leave them out and use the room for stages).
+template <int BN, int STAGES, bool STAGING>
 struct Layout2 {
     static constexpr int A_BYTES = BMC * BK * 2;       // 16 KB: this CTA's rows of A
     static constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's half of the weight tile
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int CHUNK_BYTES = 32 * 64;          // 32 rows x 32 bf16 columns
-    static constexpr int WARP_STAGE = (BN / 32) * CHUNK_BYTES;
+    static constexpr int WARP_STAGE = STAGING ? (BN / 32) * CHUNK_BYTES : 0;
     static constexpr int EPI_OFF = STAGES * STAGE_BYTES;  // 4 epilogue warps' staging tiles
     static constexpr int BAR_OFF = EPI_OFF + 4 * WARP_STAGE;
     static constexpr int NBARS = 2 * STAGES + 9;  // full, empty, tfull[2], tempty[2], rfull[4], drain
@@ -161,13 +163,13 @@ __device__ __forceinline__ int tile_width(const Tc2Params &p, int n_tile) {
     return w < BN ? w : BN;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool STAGING>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                     const __grid_constant__ CUtensorMap mB1,
                     const __grid_constant__ CUtensorMap mB2, const __grid_constant__ Tc2Maps mo,
                     const __grid_constant__ Tc2Params p) {
-    using L = Layout2<BN, STAGES>;
+    using L = Layout2<BN, STAGES, STAGING>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -334,10 +336,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         o.z = pack_bf16(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
                         o.w = pack_bf16(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
                         *reinterpret_cast<uint4 *>(hb + thl_unit(tr, u, tl.vpad)) = o;
-                        if (8 * (u + 1) == p.d)  // the head's last columns: zero the padding units
+                        if (8 * (u + 1) == p.d)  // the head's last columns: write the padding units
                             for (int z = u + 1; z < p.nunits[seg]; ++z)
                                 *reinterpret_cast<uint4 *>(hb + thl_unit(tr, z, tl.vpad)) =
-                                    make_uint4(0, 0, 0, 0);
+                                    (tl.ones && z == u + 1) ? thl_ones_unit() : make_uint4(0, 0, 0, 0);
                     }
                 }
                 fence_before_sync();
@@ -347,6 +349,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (acc == 0) acc_phase ^= 1;
                 continue;
             }
+            if (!STAGING) break;  // not launched with row-major outputs
             const bool has_r = p.R[seg] != nullptr;
             if (lane == 0) {
                 bulk_wait_read_all();  // the previous tile's stores have left the staging tile
@@ -429,9 +432,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool STAGING>
 cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
-    using L = Layout2<BN, STAGES>;
+    using L = Layout2<BN, STAGES, STAGING>;
     CUtensorMap mA, mB[3];
     if (!encode_map_2d_bf16(&mA, a.A, a.K, a.rows, a.lda * 2, BK, BMC)) return cudaErrorInvalidValue;
     for (int i = 0; i < 3; ++i) {
@@ -470,7 +473,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
     p.tiles = m_tiles * a.nmat * p.n_tiles;
     p.status = device_status_ptr();
     if (!p.status) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, STAGES>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, STAGES, STAGING>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     // persistent grid: as many pairs as can be resident at once (pairs must
@@ -482,13 +485,13 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
         cfg.blockDim = dim3(kThreads, 1, 1);
         cfg.dynamicSmemBytes = L::ALLOC;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<BN, STAGES>, &cfg) != cudaSuccess || n < 1)
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<BN, STAGES, STAGING>, &cfg) != cudaSuccess || n < 1)
             n = (num_sms() > 0 ? num_sms() : 148) / 2;
         (void)cudaGetLastError();
         max_pairs = n;
     }
     const int pairs = p.tiles < max_pairs ? p.tiles : max_pairs;
-    gemm_tc2_kernel<BN, STAGES><<<2 * pairs, kThreads, L::ALLOC, s>>>(mA, mB[0], mB[1], mB[2], mo, p);
+    gemm_tc2_kernel<BN, STAGES, STAGING><<<2 * pairs, kThreads, L::ALLOC, s>>>(mA, mB[0], mB[1], mB[2], mo, p);
     return cudaGetLastError();
 }
 
@@ -508,6 +511,11 @@ bool gemm_tc2_supported(const GemmArgs &a) {
     return true;
 }
 
-cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) { return launch_bn2<256, 5>(a, s); }
+cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) {
+    bool all_tiled = true;
+    for (int i = 0; i < a.nmat; ++i) all_tiled = all_tiled && a.thl[i] != nullptr;
+    // outputs in tiled head layout need no staging tiles: two more pipeline stages
+    return all_tiled ? launch_bn2<256, 7, false>(a, s) : launch_bn2<256, 5, true>(a, s);
+}
 
 }  // namespace ptdit

@@ -231,28 +231,34 @@ Ws ws_layout(const Dims &d, long M) {
     return L;
 }
 
-ThlDesc thl_identity(long rows_pb, int vpad) {
+ThlDesc thl_identity(long rows_pb, int vpad, int ones = 0) {
     ThlDesc t;
     memset(&t, 0, sizeof t);
     t.mode = THL_IDENTITY;
     t.vpad = vpad;
+    t.ones = ones;
     t.rows_pb = rows_pb;
     t.tiles = (int)((rows_pb + kThlRows - 1) / kThlRows);
     t.pack = 1;
     return t;
 }
 
-ThlDesc thl_window(const WinGeom &g, long N, int vpad) {
+ThlDesc thl_window(const WinGeom &g, long N, int vpad, int ones = 0) {
     ThlDesc t;
     memset(&t, 0, sizeof t);
     t.mode = THL_WINDOW;
     t.vpad = vpad;
+    t.ones = ones;
     t.rows_pb = N;
     t.pack = kThlRows / g.n;
     t.tiles = (g.nwin + t.pack - 1) / t.pack;
     t.g = g;
     return t;
 }
+
+// V operands carry a column of ones (row sums of P from the P V product) when
+// the head is narrower than its 16-column-aligned tile width.
+int v_ones(const Dims &d) { return d.d % 16 != 0; }
 
 // Whether some tile rows of this layout hold no token (they must read as zeros).
 bool thl_has_empty_rows(const ThlDesc &t) {
@@ -395,7 +401,7 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
     pa.q_bstride = pa.k_bstride = pg.M;
     pa.nq = pa.nk = pg.M;
     const bool tiled = attention_thl_supported(pa);
-    const ThlDesc tp = thl_identity(pg.M, 0), tpv = thl_identity(pg.M, 1);
+    const ThlDesc tp = thl_identity(pg.M, 0), tpv = thl_identity(pg.M, 1, v_ones(d));
     if (tiled) {
         pa.tq = pa.tk = tp;
         pa.tv = tpv;
@@ -467,11 +473,15 @@ int run_window(const Run &r, const WinGeom &wg, const ptdit_attn_w *w, unsigned 
     a.geom = wg;
     const bool tiled = attention_thl_supported(a);
     const ThlDesc tw = thl_window(wg, d.N, 0);  // V too: the window kernel splits its P V
-    if (tiled) a.tq = a.tk = a.tv = tw;
+    const ThlDesc twv = thl_window(wg, d.N, 0, v_ones(d));
+    if (tiled) {
+        a.tq = a.tk = tw;
+        a.tv = twv;
+    }
     {
         const void *W[3] = {w->wq, w->wk, w->wv};
         void *C[3] = {r.at(r.L.Q), r.at(r.L.K), r.at(r.L.V)};
-        const ThlDesc *T[3] = {tiled ? &tw : nullptr, tiled ? &tw : nullptr, tiled ? &tw : nullptr};
+        const ThlDesc *T[3] = {tiled ? &tw : nullptr, tiled ? &tw : nullptr, tiled ? &twv : nullptr};
         TRY(gemm_thl(r, PTDIT_K_GEMM, x_in, BN, 3, W, C, T, r.at(r.L.O), "window QKV projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "window attention"));
@@ -721,7 +731,7 @@ int ptdit_full_attn(const ptdit_shape *shape, const ptdit_attn_w *w, unsigned fl
     a.q_bstride = a.k_bstride = d.N;
     a.nq = a.nk = (int)d.N;
     const bool tiled = attention_thl_supported(a);
-    const ThlDesc tn = thl_identity(d.N, 0), tnv = thl_identity(d.N, 1);
+    const ThlDesc tn = thl_identity(d.N, 0), tnv = thl_identity(d.N, 1, v_ones(d));
     if (tiled) {
         a.tq = a.tk = tn;
         a.tv = tnv;

@@ -26,6 +26,8 @@ __global__ void thl_fill_kernel(Thl t, int B, int heads, int d, const uint4 *__r
     uint4 v = make_uint4(0, 0, 0, 0);
     if (src && tok >= 0 && u * 8 < d)
         v = src[(((long)b * t.rows_pb + tok) * ld + (long)h * d + u * 8) / 8];
+    else if (src && tok >= 0 && t.ones && u * 8 == d)
+        v = thl_ones_unit();
     const long blk = ((long)b * t.tiles + tile) * heads + h;
     *reinterpret_cast<uint4 *>(dst + blk * thl_block_bytes(d, t.vpad) + thl_unit(r, u, t.vpad)) = v;
 }

@@ -10,7 +10,10 @@
 //                               or, padded ("vpad", the V operand of the row
 //                               kernel, one P V MMA of N = 128), a second set of
 //                               128-byte atoms holding columns 64..127
-// Columns d..79 (or d..127) and rows that hold no token are zeros.  Loading a
+// Columns d..79 (or d..127) and rows that hold no token are zeros, except that
+// with "ones" (a V operand whose head is narrower than its tile, d = 72) column
+// d of every token row holds 1: the P V product then carries the row sums of P
+// in that column, summed in fp32 from exactly the bf16 P values that weight V.  Loading a
 // tile is then one contiguous bulk copy; reading a head's 144-byte slice out of
 // every 2304-byte token row instead keeps far fewer bytes in flight per SM.
 //
@@ -39,6 +42,9 @@ __host__ __device__ inline uint32_t thl_unit(int r, int p, int vpad) {
     if (vpad) return 16384 + (r >> 3) * 1024 + (r & 7) * 128 + (((p - 8) ^ (r & 7)) << 4);
     return 16384 + (r >> 3) * 256 + (r & 7) * 32 + (((p - 8) ^ ((r >> 2) & 1)) << 4);
 }
+
+// The 16-byte unit holding head column d when "ones" is set: 1 in its first element.
+__host__ __device__ inline uint4 thl_ones_unit() { return make_uint4(0x3F80u, 0u, 0u, 0u); }
 
 // 16-byte units per block row (head columns rounded up to the layout's width).
 __host__ __device__ inline int thl_units(int d, int vpad) { return d <= 64 ? 8 : (vpad ? 16 : 10); }

@@ -190,6 +190,7 @@ int ptdit_debug_proxy_map(const int grid[3], const int ratio[3], int32_t *proxy_
 int ptdit_debug_window_map(const int grid[3], const int window[3], const int shift[3],
                            int32_t *token_at_slot, uint8_t *allowed, ptdit_stream_t stream);
 
+
 /*
  * Kernel timing for measurement.  ptdit_timing_enable(n) makes the calling
  * host thread's later calls record a CUDA event pair around each kernel

@@ -25,7 +25,7 @@ def L():
 def _declared():
     src = open(os.path.join(ROOT, "include", "ptdit.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(ptdit_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(ptdit_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_exports_every_declared_symbol(L):
