@@ -12,6 +12,12 @@ max over ranks.  Rank 0 prints one JSON line.
 
 --impl reference times the float64 CPU oracle on the host cores instead, one
 batch item per step.
+
+Measurement options beyond the default line: --grid F,H,W and --ratio F,H,W
+override the workload's token grid and proxy ratio (the long-video ratio
+sweep); --dense times the dense comparator instead, one full global
+self-attention module (QKV projection, attention over all N tokens, output
+projection and residual) per step on the same grid.
 """
 from __future__ import annotations
 
@@ -355,6 +361,59 @@ def run_gpu(args, w):
     return 0
 
 
+def run_dense(args, w):
+    """The dense comparator: ptdit_full_attn over the workload's grid."""
+    import torch
+
+    import diffusion_transformer_sparse_b200 as pt
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    z_host, W_host = host_inputs(w)
+    z = z_host.to(dev)
+    Wd = tuple(x.to(dev) for x in W_host["wsa"])
+    shape = pt.make_shape(z, w.grid, w.heads)
+    ws = pt.workspace(shape, None, None)
+    out = torch.empty_like(z)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        pt.ptdit_full_attn(z, w.grid, Wd, w.heads, z_out=out, ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    pt.ptdit_timing_enable(8 * args.steps)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    recs = pt.ptdit_timing_read(8 * args.steps)
+    pt.ptdit_timing_enable(0)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    core_ms = sum(t for k, t in recs if k == "attn_dense") / args.steps
+    f = flops.dense_flops(w.N, w.D)
+    print(json.dumps({
+        "mode": "dense", "metric": "dense global self-attention module tokens/s", "unit": UNIT,
+        "value": w.B * w.N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,
+        "warmup": args.warmup, "config": config_of(w),
+        "tflops": w.B * f["total"] / (ms / 1e3) / 1e12,
+        "core_ms": core_ms, "core_tflops": w.B * f["core"] / (core_ms / 1e3) / 1e12,
+        "note": "timing hooks on (one event pair per launch)"}), flush=True)
+    return 0
+
+
+def parse3(text):
+    v = tuple(int(x) for x in text.split(","))
+    if len(v) != 3:
+        raise argparse.ArgumentTypeError("expected three comma-separated integers")
+    return v
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -366,11 +425,21 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernels-only", action="store_true",
                     help="stop after the timed region (no hook, e2e or CPU passes): for ncu")
+    ap.add_argument("--grid", type=parse3, help="override the token grid F,H,W")
+    ap.add_argument("--ratio", type=parse3, help="override the proxy ratio F,H,W")
+    ap.add_argument("--dense", action="store_true",
+                    help="time the dense comparator (full global self-attention) instead")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     w = configs.WORKLOADS[args.workload]
+    if args.grid or args.ratio:
+        g, r = args.grid or w.grid, args.ratio or w.ratio
+        w = w.with_(grid=g, ratio=r,
+                    name=f"{w.name}@grid{'x'.join(map(str, g))}_ratio{'x'.join(map(str, r))}")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.dense:
+        return run_dense(args, w)
     return run_gpu(args, w)
 
 

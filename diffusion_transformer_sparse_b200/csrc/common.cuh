@@ -175,6 +175,7 @@ cudaError_t launch_debug_window_map(const WinGeom &g, int32_t *tok, uint8_t *all
 // Per-launch timing hooks (no-ops unless enabled by ptdit_timing_enable).
 void timing_begin(int kind, cudaStream_t s);
 void timing_end(cudaStream_t s);
+void timing_drop();  // forget the last record (its launch did not happen)
 void count_launch();
 
 }  // namespace ptdit

@@ -436,11 +436,12 @@ template <int BN, int STAGES, bool STAGING>
 cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
     using L = Layout2<BN, STAGES, STAGING>;
     CUtensorMap mA, mB[3];
-    if (!encode_map_2d_bf16(&mA, a.A, a.K, a.rows, a.lda * 2, BK, BMC)) return cudaErrorInvalidValue;
+    // a refused tensor map sends the caller to another kernel
+    if (!encode_map_2d_bf16(&mA, a.A, a.K, a.rows, a.lda * 2, BK, BMC)) return cudaErrorNotSupported;
     for (int i = 0; i < 3; ++i) {
         const void *w = i < a.nmat ? a.W[i] : a.W[0];
         if (!encode_map_2d_bf16(&mB[i], w, a.K, a.nseg, (uint64_t)a.K * 2, BK, BN / 2))
-            return cudaErrorInvalidValue;
+            return cudaErrorNotSupported;
     }
     Tc2Params p;
     Tc2Maps mo;
@@ -461,7 +462,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
         const void *r = p.R[i] ? p.R[i] : c;
         if (!encode_map_2d_bf16_sw(&mo.C[i], c, a.nseg, a.rows, (uint64_t)a.ldc * 2, 32, 32, 64) ||
             !encode_map_2d_bf16_sw(&mo.R[i], r, a.nseg, a.rows, (uint64_t)a.ldc * 2, 32, 32, 64))
-            return cudaErrorInvalidValue;
+            return cudaErrorNotSupported;
     }
     p.ldc = a.ldc;
     p.rows = a.rows;
@@ -499,7 +500,9 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
 
 bool gemm_tc2_supported(const GemmArgs &a) {
     if (a.dtype != DT_BF16 || a.nmat < 1 || a.nmat > 3) return false;
-    if (a.K < BK || a.K % BK || a.rows < 2 * BMC || a.lda % 8 || a.ldc % 8) return false;
+    // rows past the end (a matrix shorter than a tile) read as zeros through the
+    // tensor map and are never written
+    if (a.K < BK || a.K % BK || a.rows < 1 || a.lda % 8 || a.ldc % 8) return false;
     if (a.nseg % 64) return false;  // tile widths: multiples of 32 per CTA half and epilogue chunk
     if ((uintptr_t)a.A % 16) return false;
     for (int i = 0; i < a.nmat; ++i) {

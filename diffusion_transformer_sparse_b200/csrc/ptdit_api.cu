@@ -36,7 +36,11 @@ bool attention_thl_supported(const AttnArgs &a);
 cudaError_t launch_attention_tc(const AttnArgs &a, cudaStream_t s);
 
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s) {
-    if (gemm_tc2_supported(a)) return launch_gemm_tc2(a, s);
+    if (gemm_tc2_supported(a)) {
+        const cudaError_t e = launch_gemm_tc2(a, s);
+        if (e != cudaErrorNotSupported) return e;
+        (void)cudaGetLastError();  // tensor maps refused: the kernels below
+    }
     for (int i = 0; i < a.nmat; ++i)  // only the 2-SM kernel writes tiled head layout
         if (a.thl[i]) return cudaErrorNotSupported;
     if (gemm_tc_supported(a)) return launch_gemm_tc(a, s);
@@ -75,6 +79,11 @@ void timing_end(cudaStream_t s) {
     t.kind[t.count] = t.open_kind;
     t.open_kind = -1;
     ++t.count;
+}
+
+void timing_drop() {
+    TimingState &t = g_timing;
+    if (t.count > 0 && t.open_kind < 0) --t.count;
 }
 
 void count_launch() { ++g_launches; }
@@ -336,13 +345,20 @@ int gemm_thl(const Run &r, int kind, const void *A, long rows, int nmat, const v
     g.nmat = nmat;
     g.heads = r.d.heads;
     g.d = r.d.d;
+    cudaError_t e = cudaErrorNotSupported;
     if (gemm_tc2_supported(g)) {
         timing_begin(kind, r.s);
-        cudaError_t e = launch_gemm_tc2(g, r.s);
+        e = launch_gemm_tc2(g, r.s);
         timing_end(r.s);
-        count_launch();
-        if (e != cudaSuccess) return cuda_fail(e, what);
-    } else {
+        if (e == cudaErrorNotSupported) {  // tensor maps refused: nothing was launched
+            (void)cudaGetLastError();
+            timing_drop();
+        } else {
+            count_launch();
+        }
+        if (e != cudaSuccess && e != cudaErrorNotSupported) return cuda_fail(e, what);
+    }
+    if (e == cudaErrorNotSupported) {
         for (int i = 0; i < nmat; ++i) {
             const void *Wi[3] = {W[i], nullptr, nullptr};
             void *Ci[3] = {thl[i] ? scratch : C[i], nullptr, nullptr};
