@@ -21,8 +21,11 @@
 //                wait, runs the fp32 online softmax and writes P (bf16, two per
 //                column) back over the first 64 columns of its scores; O is
 //                rescaled in TMEM only when a row's reference max has to rise
-//                by more than 2^8.  P never touches shared memory, which
-//                leaves room for a three-stage K/V ring.
+//                by more than 2^8.  P never touches shared memory (a version
+//                with P in shared memory, which lets the next S be issued as
+//                soon as the softmax has read the current one, was slower: the
+//                P writes and reads crowd shared-memory bandwidth, and the
+//                unpadded V it needed costs a second, N = 16, MMA per K step).
 // Both query tiles share every K/V tile; the MMA warp issues PV_0, S_0(next),
 // PV_1, S_1(next), so each softmax gets its next scores while the other one
 // works.  Every wait is bounded (2 s).
