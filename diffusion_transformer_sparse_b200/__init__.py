@@ -16,13 +16,16 @@ LIB_PATH = os.path.join(HERE, "libptdit.so")
 PTDIT_F32, PTDIT_BF16 = 0, 1
 PTDIT_PROXY_RESIDUAL = 0x1
 PTDIT_NO_RESIDUAL = 0x2
+# status codes (include/ptdit.h)
+(PTDIT_OK, PTDIT_ERR_NULL, PTDIT_ERR_SHAPE, PTDIT_ERR_DTYPE, PTDIT_ERR_WORKSPACE, PTDIT_ERR_CUDA,
+ PTDIT_ERR_TIMEOUT, PTDIT_ERR_ALIGN, PTDIT_ERR_ALIAS) = range(9)
 KINDS = ("average", "gemm", "attn_proxy", "attn_cross", "attn_window", "attn_dense")
 
 # Every symbol declared in include/ptdit.h.
 EXPORTS = (
     "ptdit_proxy_average", "ptdit_workspace_bytes", "ptdit_giim", "ptdit_window_attn",
     "ptdit_tcm", "ptdit_block_attn", "ptdit_full_attn", "ptdit_strerror", "ptdit_last_error",
-    "ptdit_debug_proxy_map", "ptdit_debug_window_map", "ptdit_timing_enable",
+    "ptdit_debug_proxy_map", "ptdit_debug_window_map", "ptdit_device_status", "ptdit_debug_timeout", "ptdit_timing_enable",
     "ptdit_timing_read", "ptdit_launch_count", "ptdit_window_attn_static",
 )
 
@@ -77,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "ptdit_last_error": (ctypes.c_char_p, []),
             "ptdit_debug_proxy_map": (ctypes.c_int, [_I3, _I3, _P, _P]),
             "ptdit_debug_window_map": (ctypes.c_int, [_I3, _I3, _I3, _P, _P, _P]),
+            "ptdit_device_status": (ctypes.c_int, [ctypes.c_int]),
+            "ptdit_debug_timeout": (ctypes.c_int, [ctypes.c_longlong, _P]),
             "ptdit_timing_enable": (ctypes.c_int, [ctypes.c_int]),
             "ptdit_timing_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
                                                  ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
@@ -246,6 +251,20 @@ def ptdit_debug_window_map(grid, window, shift, with_mask=True, stream=None):
     _check(lib().ptdit_debug_window_map(_i3(grid), _i3(window), _i3(shift), _ptr(tok),
                                         _ptr(allowed), _stream(stream)))
     return tok, allowed
+
+
+def ptdit_device_status(reset: bool = False) -> int:
+    """The device status word (0, or PTDIT_ERR_TIMEOUT after a bounded wait gave up);
+    synchronises the device; reset clears it."""
+    v = int(lib().ptdit_device_status(1 if reset else 0))
+    if v == PTDIT_ERR_CUDA:
+        raise PtditError(v, lib().ptdit_last_error().decode())
+    return v
+
+
+def ptdit_debug_timeout(limit_ns: int, stream=None):
+    """Launch one bounded wait that nothing releases (gives up after limit_ns)."""
+    _check(lib().ptdit_debug_timeout(int(limit_ns), _stream(stream)))
 
 
 def ptdit_timing_enable(max_launches: int):

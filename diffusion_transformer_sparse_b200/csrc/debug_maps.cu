@@ -50,3 +50,46 @@ cudaError_t launch_debug_window_map(const WinGeom &g, int32_t *tok, uint8_t *all
 
 }  // namespace ptdit
 
+
+// ------------------------------------------------------------------ status word and timeout
+#include "ptdit.h"
+#include "tc_util.cuh"
+
+namespace ptdit {
+int report_error(int code, const char *text);
+namespace {
+// One thread waits on a barrier that nothing arrives on; the bounded wait gives
+// up after limit_ns and records PTDIT_ERR_TIMEOUT, as a stalled kernel would.
+__global__ void debug_timeout_kernel(int *status, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort;
+    tc::mbar_init(&bar, 1);
+    abort = 0;
+    tc::fence_mbar_init();
+    (void)tc::mbar_wait(&bar, 0, &abort, status, limit_ns);
+}
+}  // namespace
+}  // namespace ptdit
+
+extern "C" int ptdit_device_status(int reset) {
+    int *word = ptdit::device_status_ptr();
+    if (!word) return ptdit::report_error(PTDIT_ERR_CUDA, "status word unavailable");
+    int v = 0;
+    cudaError_t e = cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && reset) e = cudaMemset(word, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return ptdit::report_error(PTDIT_ERR_CUDA, cudaGetErrorString(e));
+    return v;
+}
+
+extern "C" int ptdit_debug_timeout(long long limit_ns, ptdit_stream_t stream) {
+    if (limit_ns <= 0 || limit_ns > 10000000000LL)
+        return ptdit::report_error(PTDIT_ERR_SHAPE, "limit_ns must be in (0, 10 s]");
+    int *word = ptdit::device_status_ptr();
+    if (!word) return ptdit::report_error(PTDIT_ERR_CUDA, "status word unavailable");
+    ptdit::debug_timeout_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(word, (unsigned long long)limit_ns);
+    ptdit::count_launch();
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return ptdit::report_error(PTDIT_ERR_CUDA, cudaGetErrorString(e));
+    return PTDIT_OK;
+}

@@ -16,6 +16,7 @@
 // (tile, head) in the order the attention kernel reads them.
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <vector>
@@ -106,6 +107,17 @@ int fail(int code, const char *fmt, ...) {
 
 int cuda_fail(cudaError_t e, const char *what) {
     return fail(PTDIT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Host-side fault injection (tests): PTDIT_FAULT=workspace or PTDIT_FAULT=launch.
+bool fault(const char *kind) {
+    const char *v = getenv("PTDIT_FAULT");
+    return v && strcmp(v, kind) == 0;
+}
+
+int launch_fault(const char *what) {
+    return fault("launch") ? fail(PTDIT_ERR_CUDA, "%s: launch refused (PTDIT_FAULT=launch)", what)
+                           : PTDIT_OK;
 }
 
 // ------------------------------------------------------------------ validation
@@ -276,6 +288,8 @@ bool thl_has_empty_rows(const ThlDesc &t) {
 
 int check_ws(const Dims &d, long M, const void *ws, size_t ws_bytes, Ws *L) {
     *L = ws_layout(d, M);
+    if (fault("workspace"))
+        return fail(PTDIT_ERR_WORKSPACE, "workspace refused (PTDIT_FAULT=workspace)");
     if (!ws) return fail(PTDIT_ERR_NULL, "workspace is NULL");
     if ((uintptr_t)ws % 256) return fail(PTDIT_ERR_ALIGN, "workspace is not 256-byte aligned");
     if (ws_bytes < L->total)
@@ -315,6 +329,7 @@ int gemm(const Run &r, int kind, const void *A, long rows, int nmat, const void 
     g.nseg = r.d.D;
     g.K = r.d.D;
     g.nmat = nmat;
+    TRY(launch_fault(what));
     timing_begin(kind, r.s);
     cudaError_t e = launch_gemm(g, r.s);
     timing_end(r.s);
@@ -345,6 +360,7 @@ int gemm_thl(const Run &r, int kind, const void *A, long rows, int nmat, const v
     g.nmat = nmat;
     g.heads = r.d.heads;
     g.d = r.d.d;
+    TRY(launch_fault(what));
     cudaError_t e = cudaErrorNotSupported;
     if (gemm_tc2_supported(g)) {
         timing_begin(kind, r.s);
@@ -390,6 +406,7 @@ int attention(const Run &r, int kind, AttnArgs a, const char *what) {
     a.B = r.d.B;
     a.ldq = a.ldk = a.ldv = a.ldo = r.d.D;
     a.scale = 1.0f / sqrtf((float)r.d.d);
+    TRY(launch_fault(what));
     timing_begin(kind, r.s);
     cudaError_t e = launch_attention(a, r.s);
     timing_end(r.s);
@@ -403,6 +420,7 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
              const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z_out) {
     const Dims &d = r.d;
     const long BM = (long)d.B * pg.M, BN = (long)d.B * d.N;
+    TRY(launch_fault("proxy average"));
     timing_begin(PTDIT_K_AVERAGE, r.s);
     cudaError_t e = launch_proxy_average(d.dtype, pg, d.B, d.D, z_in, r.at(r.L.P), r.s);
     timing_end(r.s);
@@ -633,6 +651,7 @@ int ptdit_proxy_average(const ptdit_shape *shape, const int ratio[3], const void
     TRY(check_ptr(proxies, "proxies"));
     if (overlap(z, (size_t)d.B * d.N * d.D * d.elem, proxies, (size_t)d.B * pg.M * d.D * d.elem))
         return fail(PTDIT_ERR_ALIAS, "proxies overlap z");
+    TRY(launch_fault("proxy average"));
     cudaStream_t s = (cudaStream_t)stream;
     timing_begin(PTDIT_K_AVERAGE, s);
     cudaError_t e = launch_proxy_average(d.dtype, pg, d.B, d.D, z, proxies, s);

@@ -214,6 +214,34 @@ int ptdit_timing_read(int *kind, float *ms, int max);
 /* ptdit_launch_count -- kernels this host thread has launched through the library. */
 long long ptdit_launch_count(void);
 
+/*
+ * ptdit_device_status -- the library's device status word on the current
+ *   device: PTDIT_OK, or PTDIT_ERR_TIMEOUT once a bounded device-side wait
+ *   (2 s in the kernels) has given up since the last reset; such a kernel
+ *   stops issuing work and returns instead of hanging, so its outputs are
+ *   incomplete.  Synchronises the device.  reset != 0 clears the word after
+ *   reading it.  Returns the word, or PTDIT_ERR_CUDA if it cannot be read.
+ */
+int ptdit_device_status(int reset);
+
+/*
+ * ptdit_debug_timeout -- launches one thread whose bounded wait, on a barrier
+ *   nothing arrives on, gives up after limit_ns nanoseconds and records
+ *   PTDIT_ERR_TIMEOUT in the device status word, exactly as a stalled kernel
+ *   would (no trap, no fault; the context stays usable).  The paper has no
+ *   counterpart: it lets tests exercise the timeout path.  Asynchronous on
+ *   `stream`.  Errors: PTDIT_ERR_SHAPE (limit_ns <= 0 or above 10 s),
+ *   PTDIT_ERR_CUDA.
+ */
+int ptdit_debug_timeout(long long limit_ns, ptdit_stream_t stream);
+
+/*
+ * Host-side fault injection for tests: with the environment variable
+ * PTDIT_FAULT set to "workspace", every call that takes a workspace reports
+ * PTDIT_ERR_WORKSPACE; set to "launch", every kernel launch is refused with
+ * PTDIT_ERR_CUDA before anything reaches the device.  Read on each call.
+ */
+
 #ifdef __cplusplus
 }
 #endif
