@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tslot;
+    pdl_wait();  // the projections that wrote Q, K and V have completed
+    pdl_trigger();
 
     const int u0 = (int)((long)blockIdx.x * sc.units / gridDim.x);
     const int u1 = (int)((long)(blockIdx.x + 1) * sc.units / gridDim.x);
@@ -411,8 +413,8 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(attn_rows_kernel<DPAD, SUMV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
-    attn_rows_kernel<DPAD, SUMV><<<grid, kThreads, L::BYTES, s>>>(a, sc, status);
-    return cudaGetLastError();
+    return launch_pdl(attn_rows_kernel<DPAD, SUMV>, dim3(grid), dim3(kThreads), L::BYTES, s, a, sc,
+                      status);
 }
 
 }  // namespace

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace ptdit {
 
 // ---------------------------------------------------------------------------
@@ -96,6 +98,35 @@ __host__ __device__ __forceinline__ int window_token(const WinGeom &g, int win, 
     if (x >= g.w) { x -= g.w; c |= 1; }
     *wrap = c;
     return (t * g.h + y) * g.w + x;
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  pdl_wait: block until the grids this one
+// depends on (the previous kernel in the stream, when launched with
+// launch_pdl) have completed and their writes are visible; a no-op otherwise.
+// pdl_trigger: let the next kernel of the stream be scheduled (its CTAs run
+// their prologue on SMs this grid has left, then wait in pdl_wait).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launches `kernel` with programmatic stream serialization: it may start while
+// the previous kernel of the stream finishes, and must call pdl_wait() before
+// it reads or writes anything that kernel (or an earlier one) touches.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------------------

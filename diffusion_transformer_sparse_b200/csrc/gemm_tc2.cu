@@ -212,6 +212,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     cluster_sync();  // barriers of both CTAs are initialised before anyone signals them
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // everything above touched only this CTA: from here on, the previous
+    // kernel's outputs (A, the residual) must be complete
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -492,8 +496,8 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
         max_pairs = n;
     }
     const int pairs = p.tiles < max_pairs ? p.tiles : max_pairs;
-    gemm_tc2_kernel<BN, STAGES, STAGING><<<2 * pairs, kThreads, L::ALLOC, s>>>(mA, mB[0], mB[1], mB[2], mo, p);
-    return cudaGetLastError();
+    return launch_pdl(gemm_tc2_kernel<BN, STAGES, STAGING>, dim3(2 * pairs), dim3(kThreads), L::ALLOC, s,
+                      mA, mB[0], mB[1], mB[2], mo, p);
 }
 
 }  // namespace

@@ -69,6 +69,8 @@ __global__ void __launch_bounds__(1024) proxy_average_kernel(const T *__restrict
                                                              T *__restrict__ out, ProxyGeom g,
                                                              int D, int CHT, int G) {
     extern __shared__ float red[];  // [G-1][CHT][VEC]
+    pdl_wait();  // z is complete
+    pdl_trigger();
     const int CH = D / VEC;
     const int m = blockIdx.x % g.M;
     const int b = blockIdx.x / g.M;
@@ -132,9 +134,8 @@ cudaError_t launch_avg(const ProxyGeom &g, int B, int D, const void *z, void *ou
     if (G < 1) G = 1;
     const int threads = CHT * G;
     const size_t smem = (size_t)(G - 1) * CHT * VEC * sizeof(float);
-    proxy_average_kernel<T, VEC><<<(unsigned)(B * g.M), threads, smem, s>>>(
-        static_cast<const T *>(z), static_cast<T *>(out), g, D, CHT, G);
-    return cudaGetLastError();
+    return launch_pdl(proxy_average_kernel<T, VEC>, dim3((unsigned)(B * g.M)), dim3(threads), smem, s,
+                      static_cast<const T *>(z), static_cast<T *>(out), g, D, CHT, G);
 }
 
 }  // namespace

@@ -424,6 +424,8 @@ bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows
 
 int num_sms();
 
+
+
 // Device address of the library's status word on the current device (0 while
 // no bounded wait has given up); nullptr if it cannot be obtained.
 int *device_status_ptr();

@@ -9,6 +9,8 @@ namespace {
 
 __global__ void thl_fill_kernel(Thl t, int B, int heads, int d, const uint4 *__restrict__ src,
                                 long ld, uint8_t *__restrict__ dst, int tile0, long items) {
+    pdl_wait();  // the projection output (or the blocks being completed) is complete
+    pdl_trigger();
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= items) return;
     const int U = thl_units(d, t.vpad);
@@ -42,10 +44,8 @@ cudaError_t launch_thl_fill(const Thl &t, int B, int heads, int d, const void *s
     if (items <= 0) return cudaSuccess;
     const int threads = 256;
     const long blocks = (items + threads - 1) / threads;
-    thl_fill_kernel<<<(unsigned)blocks, threads, 0, s>>>(t, B, heads, d,
-                                                         static_cast<const uint4 *>(src), ld,
-                                                         static_cast<uint8_t *>(dst), tile0, items);
-    return cudaGetLastError();
+    return launch_pdl(thl_fill_kernel, dim3((unsigned)blocks), dim3(threads), 0, s, t, B, heads, d,
+                      static_cast<const uint4 *>(src), ld, static_cast<uint8_t *>(dst), tile0, items);
 }
 
 }  // namespace ptdit
