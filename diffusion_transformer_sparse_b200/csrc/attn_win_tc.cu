@@ -3,29 +3,37 @@
 // packed two per 128-row tile) or 128 tokens (3D, one per tile) of the grid
 // rolled by -shift, pairs that the roll wrapped masked out.
 //
-// One persistent CTA per SM with two independent slots; a unit is one tile
-// (128 query rows = its own 128 key rows) of one head:
-//   warps 2, 3   loaders, one per slot: the window projection wrote Q, K and V
-//                in tiled head layout (thl.cuh) with window tiles, so the
-//                unit's Q, K and V are three contiguous 20 KB blocks, each
-//                already the swizzled shared-memory tile (columns 0..63 with
-//                the 128-byte swizzle, 64..79 with the 32-byte swizzle, zeros
-//                past the head and in rows without a window): three bulk
-//                copies, Q and K on one barrier and V on another, so that
-//                S = Q K^T starts while V is still arriving.  Meanwhile each
-//                lane computes the token of its tile rows with the roll/wrap
-//                address function (for the key masks and the output rows) and
-//                the warp builds the key masks (window in tile x wrap bits)
-//                with ballots.
-//   warp 1       MMA issuer: S = Q K^T into TMEM, then O = P V with P read
-//                from TMEM (the softmax writes it over S) and V from shared
-//                memory as the MN-major operand: columns 0..63 in one N = 64
-//                MMA per K step (128-byte swizzle), 64..79 in one N = 16 MMA
-//                (32-byte swizzle).
-//   warps 4-7, 8-11   softmax of slot 0 / slot 1: thread r owns query row r,
-//                reads only its own window's scores, masks, exponentiates in
-//                fp32, writes P as bf16 pairs into TMEM, then scales its
-//                output row by 1/l and stores it.
+// One persistent CTA per SM; a unit is one tile (128 query rows = its own 128
+// key rows) of one head.  Three load buffers keep up to three units' operands
+// in flight while two TMEM slots (S/P and O) alternate between the units:
+//   warp 2       loader: the window projection wrote Q, K and V in tiled head
+//                layout (thl.cuh) with window tiles, so a unit's Q, K and V
+//                are three contiguous 20 KB blocks, each already the swizzled
+//                shared-memory tile (columns 0..63 with the 128-byte swizzle,
+//                64..79 with the 32-byte swizzle, zeros past the head and in
+//                rows without a window, V's column d = 1 when d = 72): three
+//                bulk copies into the unit's buffer, Q and K on one barrier and
+//                V on another.  It also computes the token of each tile row
+//                with the roll/wrap address function (for the key masks and the
+//                output rows) and builds the key masks (window in tile x wrap
+//                bits) with ballots, once per (batch item, tile) and buffer:
+//                the heads of one tile follow each other.
+//   warp 1       MMA issuer: S = Q K^T into the unit's TMEM slot, then O = P V
+//                with P read from TMEM (the softmax writes it over S) and V
+//                from shared memory as the MN-major operand: columns 0..63 in
+//                one N = 64 MMA per K step (128-byte swizzle), 64..79 in one
+//                N = 16 MMA (32-byte swizzle).  Order: S(0), S(1), then per
+//                unit k: P V(k), S(k + 2).
+//   warps 4-7, 8-11   softmax of TMEM slot 0 / 1 (units k = 0, 2, ... /
+//                1, 3, ...): thread r owns query row r, reads only its own
+//                window's scores, masks, exponentiates in fp32 and writes P as
+//                bf16 pairs into TMEM.  Then each warp reads its 32 output rows
+//                from TMEM, scales them by 1/l, stages them in the unit's Q/K
+//                area (the tensor cores are done with it) and stores them with
+//                consecutive lanes on consecutive 16-byte pieces of a token
+//                row; when its four warps are done the buffer goes back to the
+//                loader.
+// With SUMV the row sums of P come out of P V through V's ones column.
 // Every wait is bounded (2 s).
 #include <math.h>
 
@@ -41,6 +49,7 @@ constexpr int BQ = 128;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;  // per slot: S/P 128 columns, O 128 columns
 constexpr int kKeys = 16;            // mask keys per tile: 2 windows x 8 wrap codes
+constexpr int NBUF = 3;              // load buffers: units whose operands are in flight
 
 template <int DPAD>
 struct WinLayout {
@@ -48,19 +57,19 @@ struct WinLayout {
     static constexpr int TILE_A = BQ * 128;                    // columns 0..63, 128-byte swizzle
     static constexpr int TILE_B = HAS_B ? BQ * 32 : 0;         // columns 64..79, 32-byte swizzle
     static constexpr int TILE = TILE_A + TILE_B;               // a Q or K tile (K-major)
-    static constexpr int SLOT = 3 * TILE;                      // Q, K, V of one slot
-    static constexpr int OFF_INFO = 2 * SLOT;                  // int info[2][128]
-    static constexpr int OFF_ROW = OFF_INFO + 2 * BQ * 4;      // long row[2][128]
-    static constexpr int OFF_MASK = OFF_ROW + 2 * BQ * 8;      // uint32 kmask[2][kKeys][4]
-    // output staging of each softmax warpgroup: 128 rows (pitch <= 160 B), their token rows
-    static constexpr int STG = BQ * 160;
-    static constexpr int OFF_STG = OFF_MASK + 2 * kKeys * 16;
-    static constexpr int OFF_OROW = OFF_STG + 2 * STG;        // long orow[2][128]
-    static constexpr int OFF_BAR = OFF_OROW + 2 * BQ * 8;
-    // qk_full[2], v_full[2], slot_free[2], s_full[2], p_full[2], o_full[2], o_free[2], drain
-    static constexpr int NBARS = 19;  // + stage_full[2], stage_free[2]
+    static constexpr int BUF = 3 * TILE;                       // Q, K, V of one unit
+    static constexpr int OFF_INFO = NBUF * BUF;                // int info[NBUF][128]
+    static constexpr int OFF_ROW = OFF_INFO + NBUF * BQ * 4;   // int row[NBUF][128] (token rows)
+    static constexpr int OFF_MASK = OFF_ROW + NBUF * BQ * 4;   // uint32 kmask[NBUF][kKeys][4]
+    // output staging: 32 rows (pitch <= 160 B) per softmax warp
+    static constexpr int WSTG = 32 * 160;
+    static constexpr int OFF_STG = OFF_MASK + NBUF * kKeys * 16;
+    static constexpr int OFF_OROW = OFF_STG + 8 * WSTG;       // int orow[8][32]: rows being stored
+    static constexpr int OFF_BAR = OFF_OROW + 8 * 32 * 4;
+    // qk_full[NBUF], v_full[NBUF], buf_free[NBUF], s_full[2], p_full[2], o_full[2], o_free[2], drain
+    static constexpr int NBARS = 3 * NBUF + 9;
     static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
-    static_assert(TILE_A % 1024 == 0 && TILE % 1024 == 0 && SLOT % 1024 == 0,
+    static_assert(TILE_A % 1024 == 0 && TILE % 1024 == 0 && BUF % 1024 == 0,
                   "swizzled tiles stay 1 KB aligned");
     static_assert(BYTES <= 232448, "shared memory budget");
 };
@@ -78,12 +87,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     int *info = reinterpret_cast<int *>(sm + L::OFF_INFO);
-    long *rowsm = reinterpret_cast<long *>(sm + L::OFF_ROW);
+    int *rowsm = reinterpret_cast<int *>(sm + L::OFF_ROW);  // B * N < 2^31 (checked by the API)
     uint32_t *kmask = reinterpret_cast<uint32_t *>(sm + L::OFF_MASK);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
-    uint64_t *qk_full = bars, *v_full = bars + 2, *slot_free = bars + 4, *s_full = bars + 6;
-    uint64_t *p_full = bars + 8, *o_full = bars + 10, *o_free = bars + 12, *drain = bars + 14;
-    uint64_t *stage_full = bars + 15, *stage_free = bars + 17;
+    uint64_t *qk_full = bars, *v_full = bars + NBUF, *buf_free = bars + 2 * NBUF;
+    uint64_t *s_full = bars + 3 * NBUF, *p_full = s_full + 2, *o_full = s_full + 4;
+    uint64_t *o_free = s_full + 6, *drain = s_full + 8;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -91,20 +100,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int d = a.d, n = a.geom.n;
 
     if (threadIdx.x == 0) {
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&qk_full[b], 32);  // the loader's 32 lanes (rows and masks) + Q, K bytes
+            mbar_init(&v_full[b], 1);
+            mbar_init(&buf_free[b], 1);  // the unit's P V has read its operands
+        }
         for (int g = 0; g < 2; ++g) {
-            mbar_init(&qk_full[g], 32);  // the loader's 32 lanes (rows and masks) + Q, K bytes
-            mbar_init(&v_full[g], 1);
-            mbar_init(&slot_free[g], 1);
             mbar_init(&s_full[g], 1);
             mbar_init(&p_full[g], BQ);
             mbar_init(&o_full[g], 1);
             mbar_init(&o_free[g], BQ);
         }
         mbar_init(drain, 1);
-        for (int g = 0; g < 2; ++g) {
-            mbar_init(&stage_full[g], BQ);
-            mbar_init(&stage_free[g], BQ);
-        }
         *abort = 0;
         fence_mbar_init();
     }
@@ -118,62 +125,60 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int u0 = (int)((long)blockIdx.x * sc.units / gridDim.x);
     const int u1 = (int)((long)(blockIdx.x + 1) * sc.units / gridDim.x);
-    // slot g takes units u0 + g, u0 + g + 2, ...: k-th unit of slot g
-    auto unit_of = [&](int g, int k) { return u0 + g + 2 * k; };
+    const int nunits = u1 - u0;  // local unit k: buffer k % NBUF, TMEM slot k % 2
 
-    if (warp == 2 || warp == 3) {
-        // ------------------------------------------------------------ loader of slot g
-        const int g = warp - 2;
-        uint8_t *sQ = sm + g * L::SLOT, *sK = sQ + L::TILE, *sV = sK + L::TILE;
+    if (warp == 2) {
+        // ------------------------------------------------------------ loader
         const uint8_t *qg = static_cast<const uint8_t *>(a.q);
         const uint8_t *kg = static_cast<const uint8_t *>(a.k);
         const uint8_t *vg = static_cast<const uint8_t *>(a.v);
         const WinGeom &geo = a.geom;
         const int pack = BQ / n;
-        int last_rest = -1;  // (batch item, tile) whose rows and masks the slot holds
-        for (int k = 0; unit_of(g, k) < u1; ++k) {
-            const int u = unit_of(g, k);
+        int held0 = -1, held1 = -1, held2 = -1;  // (batch item, tile) whose rows each buffer holds
+        for (int k = 0; k < nunits; ++k) {
+            const int u = u0 + k, bf = k % NBUF;
             const int h = u % a.heads, rest = u / a.heads, tile = rest % sc.tiles,
                       b = rest / sc.tiles;
-            if (!mbar_wait(&slot_free[g], (k & 1) ^ 1, abort, status)) break;
+            if (!mbar_wait(&buf_free[bf], ((k / NBUF) & 1) ^ 1, abort, status)) break;
+            uint8_t *sQ = sm + bf * L::BUF, *sK = sQ + L::TILE, *sV = sK + L::TILE;
             if (lane == 0) {
                 const long blk = ((long)b * sc.tiles + tile) * a.heads + h;
-                mbar_expect_tx_only(&qk_full[g], 2 * L::TILE);
-                bulk_load(sQ, qg + blk * L::TILE, L::TILE, &qk_full[g]);
-                bulk_load(sK, kg + blk * L::TILE, L::TILE, &qk_full[g]);
-                mbar_expect_tx(&v_full[g], L::TILE);
-                bulk_load(sV, vg + blk * L::TILE, L::TILE, &v_full[g]);
+                mbar_expect_tx_only(&qk_full[bf], 2 * L::TILE);
+                bulk_load(sQ, qg + blk * L::TILE, L::TILE, &qk_full[bf]);
+                bulk_load(sK, kg + blk * L::TILE, L::TILE, &qk_full[bf]);
+                mbar_expect_tx(&v_full[bf], L::TILE);
+                bulk_load(sV, vg + blk * L::TILE, L::TILE, &v_full[bf]);
             }
             // rows and masks depend on (batch item, tile) only: the heads of one tile
-            // follow each other in this slot, so most units reuse them
-            if (rest != last_rest) {
-                last_rest = rest;
+            // follow each other, so most units find them in their buffer already
+            int &held = bf == 0 ? held0 : (bf == 1 ? held1 : held2);
+            if (rest != held) {
+                held = rest;
                 int inf[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int r = q * 32 + lane;
                     const int wit = r / n, win = tile * pack + wit, slot = r - wit * n;
-                    long row = -1;
-                    int in = -1;
+                    int row = -1, in = -1;
                     if (win < geo.nwin) {
                         int wrap;
-                        row = (long)b * a.k_bstride + window_token(geo, win, slot, &wrap);
+                        row = static_cast<int>(b * a.k_bstride) + window_token(geo, win, slot, &wrap);
                         in = wit * 8 + wrap;
                     }
                     inf[q] = in;
-                    info[g * BQ + r] = in;
-                    rowsm[g * BQ + r] = row;
+                    info[bf * BQ + r] = in;
+                    rowsm[bf * BQ + r] = row;
                 }
                 // one 128-bit key mask per mask key: keys of the same window and wrap code
                 for (int v = 0; v < kKeys; ++v)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const uint32_t bits = __ballot_sync(0xffffffffu, inf[q] == v);
-                        if (lane == 0) kmask[(g * kKeys + v) * 4 + q] = bits;
+                        if (lane == 0) kmask[(bf * kKeys + v) * 4 + q] = bits;
                     }
             }
             __syncwarp();
-            mbar_arrive(&qk_full[g]);
+            mbar_arrive(&qk_full[bf]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -182,42 +187,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc_o = idesc_bf16(BQ, 64, true);   // V columns 0..63
             constexpr uint32_t idesc_ob = idesc_bf16(BQ, 16, true);  // V columns 64..79
             bool ok = true, any = false;
-            for (int k = 0; ok && unit_of(0, k) < u1; ++k) {
-                for (int g = 0; g < 2 && ok; ++g) {
-                    if (unit_of(g, k) >= u1) continue;
-                    if (!mbar_wait(&qk_full[g], k & 1, abort, status)) { ok = false; break; }
-                    fence_after_sync();
-                    const uint32_t aQ = smem_u32(sm + g * L::SLOT);
-                    const uint32_t aK = aQ + L::TILE;
+            // S(k) into TMEM slot k % 2 (after P V(k - 2), issued earlier, has read P(k - 2))
+            auto issue_s = [&](int k) {
+                const int bf = k % NBUF, g = k & 1;
+                if (!mbar_wait(&qk_full[bf], (k / NBUF) & 1, abort, status)) return false;
+                fence_after_sync();
+                const uint32_t aQ = smem_u32(sm + bf * L::BUF);
+                const uint32_t aK = aQ + L::TILE;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + g * 256, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
-                                 idesc_s, kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + g * 256, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
+                             idesc_s, kk > 0);
+                if (L::HAS_B)
+                    mma_bf16(tmem + g * 256, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
+                             idesc_s, 1);
+                mma_commit(&s_full[g]);
+                any = true;
+                return true;
+            };
+            // O(k) = P(k) V(k), once the softmax has written P(k) and the output of
+            // unit k - 2 has been read out of the slot's O columns
+            auto issue_pv = [&](int k) {
+                const int bf = k % NBUF, g = k & 1;
+                if (!mbar_wait(&p_full[g], (k >> 1) & 1, abort, status)) return false;
+                if (!mbar_wait(&o_free[g], ((k >> 1) & 1) ^ 1, abort, status)) return false;
+                if (!mbar_wait(&v_full[bf], (k / NBUF) & 1, abort, status)) return false;
+                fence_after_sync();
+                const uint32_t aV = smem_u32(sm + bf * L::BUF + 2 * L::TILE);
+                const uint32_t tO = tmem + g * 256 + 128;
+#pragma unroll
+                for (int ks = 0; ks < BQ / 16; ++ks) {
+                    mma_bf16_ts(tO, tmem + g * 256 + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
+                                idesc_o, ks > 0);
                     if (L::HAS_B)
-                        mma_bf16(tmem + g * 256, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
-                                 idesc_s, 1);
-                    mma_commit(&s_full[g]);
-                    any = true;
+                        mma_bf16_ts(tO + 64, tmem + g * 256 + ks * 8,
+                                    sdesc_sw32_mn(aV + L::TILE_A + ks * 512), idesc_ob, ks > 0);
                 }
-                for (int g = 0; g < 2 && ok; ++g) {
-                    if (unit_of(g, k) >= u1) continue;
-                    if (!mbar_wait(&v_full[g], k & 1, abort, status)) { ok = false; break; }
-                    if (!mbar_wait(&p_full[g], k & 1, abort, status)) { ok = false; break; }
-                    if (!mbar_wait(&o_free[g], (k & 1) ^ 1, abort, status)) { ok = false; break; }
-                    fence_after_sync();
-                    const uint32_t aV = smem_u32(sm + g * L::SLOT + 2 * L::TILE);
-                    const uint32_t tO = tmem + g * 256 + 128;
-#pragma unroll
-                    for (int ks = 0; ks < BQ / 16; ++ks) {
-                        mma_bf16_ts(tO, tmem + g * 256 + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
-                                    idesc_o, ks > 0);
-                        if (L::HAS_B)
-                            mma_bf16_ts(tO + 64, tmem + g * 256 + ks * 8,
-                                        sdesc_sw32_mn(aV + L::TILE_A + ks * 512), idesc_ob, ks > 0);
-                    }
-                    mma_commit(&o_full[g]);
-                    mma_commit(&slot_free[g]);  // Q, K and V of this slot are read
-                }
+                mma_commit(&o_full[g]);
+                mma_commit(&buf_free[bf]);  // S and P V have read the unit's Q, K and V
+                return true;
+            };
+            if (nunits > 0) ok = issue_s(0);
+            if (ok && nunits > 1) ok = issue_s(1);
+            for (int k = 0; k < nunits && ok; ++k) {
+                ok = issue_pv(k);
+                if (ok && k + 2 < nunits) ok = issue_s(k + 2);
             }
             if (any) {  // every issued MMA has finished before TMEM is released
                 mma_commit(drain);
@@ -238,22 +252,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
         // the row's own keys: its window inside the tile
         const int c_lo = n < BQ ? (r / n) * n : 0;
-        for (int k = 0; unit_of(g, k) < u1; ++k) {
-            const int u = unit_of(g, k);
+        for (int k = g; k < nunits; k += 2) {
+            const int u = u0 + k, bf = k % NBUF;
+            const uint32_t ph = (k >> 1) & 1;  // phase of this slot's barriers
             const int h = u % a.heads;
-            if (!mbar_wait(&qk_full[g], k & 1, abort, status)) break;  // masks and rows
-            const int qi = info[g * BQ + r];
-            const long qrow = rowsm[g * BQ + r];  // queries and keys share rows in window mode
-            const bool live = qrow >= 0;
+            if (!mbar_wait(&qk_full[bf], (k / NBUF) & 1, abort, status)) break;  // masks and rows
+            const int qi = info[bf * BQ + r];
+            // this row's token: the buffer's rows may be rewritten once P V has read it
+            const int qrow = rowsm[bf * BQ + r];
             uint32_t allow[4] = {0u, 0u, 0u, 0u};
             if (qi >= 0) {
-                const uint4 w4 = *reinterpret_cast<const uint4 *>(kmask + (g * kKeys + qi) * 4);
+                const uint4 w4 = *reinterpret_cast<const uint4 *>(kmask + (bf * kKeys + qi) * 4);
                 allow[0] = w4.x;
                 allow[1] = w4.y;
                 allow[2] = w4.z;
                 allow[3] = w4.w;
             }
-            if (!mbar_wait(&s_full[g], k & 1, abort, status)) break;
+            if (!mbar_wait(&s_full[g], ph, abort, status)) break;
             fence_after_sync();
             float l = 0.f;
             uint32_t pk[64];
@@ -327,52 +342,62 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
             fence_before_sync();
             mbar_arrive(&p_full[g]);
-            // O / l to global memory through the staging rows: consecutive lanes
-            // store consecutive 16-byte pieces of one token row
-            if (!mbar_wait(&o_full[g], k & 1, abort, status)) break;
-            if (!mbar_wait(&stage_free[g], (k & 1) ^ 1, abort, status)) break;
+            // O / l to global memory: each warp stages its 32 rows and stores them
+            // with consecutive lanes on consecutive 16-byte pieces of a token row;
+            // the token rows come from the unit's buffer, whose next load waits
+            // for that buffer's release by P V and is two units away
+            if (!mbar_wait(&o_full[g], ph, abort, status)) break;
             fence_after_sync();
-            uint8_t *stg = sm + L::OFF_STG + g * L::STG;
-            long *orow = reinterpret_cast<long *>(sm + L::OFF_OROW) + g * BQ;
+            uint8_t *stg = sm + L::OFF_STG + (warp - 4) * L::WSTG - (warp % 4) * 32 * pitch;
+            int *orow = reinterpret_cast<int *>(sm + L::OFF_OROW) + (warp - 4) * 32;
+            orow[lane] = qrow;
             {
                 uint32_t ov[DPAD];
                 tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(ov));
                 tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
                 if (DPAD > 64) tmem_ld16(t_o + 64, *reinterpret_cast<uint32_t(*)[16]>(ov + 64));
                 tmem_ld_wait();
+                fence_before_sync();
+                mbar_arrive(&o_free[g]);  // O is read: the slot's next P V may overwrite it
                 // SUMV: column d = DPAD - 8 of O holds the row sum of P
                 const float inv = 1.f / (SUMV ? __uint_as_float(ov[DPAD - 8]) : l);
 #pragma unroll
-                for (int u = 0; u < DPAD / 8; ++u)
-                    if (u < nch) {
+                for (int uu = 0; uu < DPAD / 8; ++uu)
+                    if (uu < nch) {
                         uint4 v;
-                        v.x = pack_bf16(__uint_as_float(ov[8 * u + 0]) * inv, __uint_as_float(ov[8 * u + 1]) * inv);
-                        v.y = pack_bf16(__uint_as_float(ov[8 * u + 2]) * inv, __uint_as_float(ov[8 * u + 3]) * inv);
-                        v.z = pack_bf16(__uint_as_float(ov[8 * u + 4]) * inv, __uint_as_float(ov[8 * u + 5]) * inv);
-                        v.w = pack_bf16(__uint_as_float(ov[8 * u + 6]) * inv, __uint_as_float(ov[8 * u + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(stg + r * pitch + u * 16) = v;
+                        v.x = pack_bf16(__uint_as_float(ov[8 * uu + 0]) * inv, __uint_as_float(ov[8 * uu + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(ov[8 * uu + 2]) * inv, __uint_as_float(ov[8 * uu + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(ov[8 * uu + 4]) * inv, __uint_as_float(ov[8 * uu + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(ov[8 * uu + 6]) * inv, __uint_as_float(ov[8 * uu + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(stg + r * pitch + uu * 16) = v;
                     }
-                orow[r] = live ? qrow : -1;
             }
-            fence_before_sync();
-            mbar_arrive(&o_free[g]);  // O is read: the slot's next P V may overwrite it
-            mbar_arrive(&stage_full[g]);
-            if (!mbar_wait(&stage_full[g], k & 1, abort, status)) break;
+            __syncwarp();
             {
+                // unit i of the warp's 32 x nch pieces: row r0 + i / nch, piece i % nch,
+                // walked incrementally (i advances by 32 per step)
+                const int r0 = (warp % 4) * 32;
+                const int drow = 32 / nch, dpc = 32 % nch;
+                int row = r0 + lane / nch, pc = lane % nch;
                 __nv_bfloat16 *obase = og + (long)h * d;
-                for (int i = r; i < BQ * nch; i += BQ) {
-                    const int row = i / nch, u = i - row * nch;
-                    const long orw = orow[row];
+                for (int i = lane; i < 32 * nch; i += 32) {
+                    const int orw = orow[row - r0];
                     if (orw >= 0)
-                        *reinterpret_cast<uint4 *>(obase + orw * a.ldo + u * 8) =
-                            *reinterpret_cast<const uint4 *>(stg + row * pitch + u * 16);
+                        *reinterpret_cast<uint4 *>(obase + (long)orw * a.ldo + pc * 8) =
+                            *reinterpret_cast<const uint4 *>(stg + row * pitch + pc * 16);
+                    row += drow;
+                    pc += dpc;
+                    if (pc >= nch) {
+                        pc -= nch;
+                        ++row;
+                    }
                 }
             }
-            mbar_arrive(&stage_free[g]);
+            __syncwarp();  // the staging rows are free for the warp's next unit
         }
     }
     if (*abort) {
-        // give box loads still in flight into this CTA a moment to land
+        // a wait gave up: let bulk copies still in flight into this CTA land
         const uint64_t t0 = globaltimer();
         while (globaltimer() - t0 < 100000) {
         }
