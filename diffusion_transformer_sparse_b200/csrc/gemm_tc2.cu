@@ -37,6 +37,13 @@
 // Two TMEM accumulators overlap the next tile's MMAs with this tile's
 // epilogue.  Every wait is bounded (2 s); a timeout records
 // PTDIT_ERR_TIMEOUT in the status word.
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
+
 #include "tc_util.cuh"
 #include "thl.cuh"
 
@@ -54,6 +61,9 @@ struct Tc2Maps {
     CUtensorMap C[3], R[3];
 };
 
+constexpr int kMaxPairs = 128;   // pairs a schedule can describe
+constexpr int kMaxSched = 4096;  // tiles a schedule can describe (larger launches: round robin)
+
 struct Tc2Params {
     void *C[3];
     const void *R[3];
@@ -68,6 +78,11 @@ struct Tc2Params {
     int tiles;    // all pair tiles
     int kblocks;
     int *status;
+    // Tile schedule: pair q runs tiles sched[first[q]] .. sched[first[q + 1] - 1] in
+    // that order; nsched == 0 means round robin (tile t to pair t % pairs).
+    int nsched;
+    uint16_t first[kMaxPairs + 1];
+    uint16_t sched[kMaxSched];
 };
 
 // STAGING: the row-major epilogue's staging tiles exist (launches whose outputs
@@ -156,6 +171,16 @@ __device__ __forceinline__ void decode_tile2(const Tc2Params &p, int t, int &m_t
     n_tile = n % p.n_tiles;
 }
 
+// The k-th tile of pair `pair` (-1 when it has no more).
+__device__ __forceinline__ int pair_tile(const Tc2Params &p, int pair, int npairs, int k) {
+    if (p.nsched) {
+        const int i = p.first[pair] + k;
+        return i < p.first[pair + 1] ? p.sched[i] : -1;
+    }
+    const int t = pair + k * npairs;
+    return t < p.tiles ? t : -1;
+}
+
 // Output columns of tile n_tile: BN, or what is left of the matrix for the last one.
 template <int BN>
 __device__ __forceinline__ int tile_width(const Tc2Params &p, int n_tile) {
@@ -224,7 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int t = pair; ok && t < p.tiles; t += npairs) {
+            for (int kt = 0, t; ok && (t = pair_tile(p, pair, npairs, kt)) >= 0; ++kt) {
                 int m_tile, seg, n_tile;
                 decode_tile2(p, t, m_tile, seg, n_tile);
                 const CUtensorMap *mb = seg == 0 ? &mB0 : (seg == 1 ? &mB1 : &mB2);
@@ -252,7 +277,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, any = false;
-            for (int t = pair; ok && t < p.tiles; t += npairs) {
+            for (int kt = 0, t; ok && (t = pair_tile(p, pair, npairs, kt)) >= 0; ++kt) {
                 int m_tile, seg, n_tile;
                 decode_tile2(p, t, m_tile, seg, n_tile);
                 const uint32_t idesc = idesc_bf16(2 * BMC, tile_width<BN>(p, n_tile));
@@ -300,7 +325,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t sw = (lane >> 1) & 3;
         int acc = 0;
         uint32_t acc_phase = 0, r_phase = 0;
-        for (int t = pair; t < p.tiles; t += npairs) {
+        for (int kt = 0, t; (t = pair_tile(p, pair, npairs, kt)) >= 0; ++kt) {
             int m_tile, seg, n_tile;
             decode_tile2(p, t, m_tile, seg, n_tile);
             const int row0 = m_tile * 2 * BMC + rank * BMC + q * 32;
@@ -436,6 +461,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
 }
 
+// Longest-processing-time schedule of the pair tiles: tiles by decreasing
+// width (the work of a tile is proportional to its columns), each to the pair
+// with the least work so far; each pair then runs its tiles in index order
+// (row blocks of A in sequence, as the pairs together sweep A).  Cached per
+// launch shape; only for launches of at most kMaxSched tiles, where the
+// round robin's imbalance (a few tiles per pair, some of half width) costs.
+struct SchedKey {
+    int tiles, per_m, n_tiles, nseg, bn, pairs;
+    bool operator<(const SchedKey &o) const {
+        return std::tie(tiles, per_m, n_tiles, nseg, bn, pairs) <
+               std::tie(o.tiles, o.per_m, o.n_tiles, o.nseg, o.bn, o.pairs);
+    }
+};
+struct SchedVal {
+    std::vector<uint16_t> first, tile;
+};
+
+const SchedVal *tile_schedule(const SchedKey &k) {
+    static std::mutex mu;
+    static std::map<SchedKey, SchedVal> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(k);
+    if (it != cache.end()) return &it->second;
+    std::vector<int> order(k.tiles), width(k.tiles);
+    for (int t = 0; t < k.tiles; ++t) {
+        const int n_tile = (t % k.per_m) % k.n_tiles;
+        const int w = k.nseg - n_tile * k.bn;
+        width[t] = w < k.bn ? w : k.bn;
+        order[t] = t;
+    }
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int a, int b) { return width[a] > width[b]; });
+    std::vector<std::vector<int>> lists(k.pairs);
+    std::priority_queue<std::pair<long, int>, std::vector<std::pair<long, int>>,
+                        std::greater<std::pair<long, int>>>
+        load;
+    for (int q = 0; q < k.pairs; ++q) load.push({0L, q});
+    for (int t : order) {
+        auto top = load.top();
+        load.pop();
+        lists[top.second].push_back(t);
+        load.push({top.first + width[t], top.second});
+    }
+    SchedVal v;
+    v.first.push_back(0);
+    for (auto &l : lists) {
+        std::sort(l.begin(), l.end());
+        for (int t : l) v.tile.push_back(static_cast<uint16_t>(t));
+        v.first.push_back(static_cast<uint16_t>(v.tile.size()));
+    }
+    return &cache.emplace(k, std::move(v)).first->second;
+}
+
 template <int BN, int STAGES, bool STAGING>
 cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
     using L = Layout2<BN, STAGES, STAGING>;
@@ -496,6 +574,14 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
         max_pairs = n;
     }
     const int pairs = p.tiles < max_pairs ? p.tiles : max_pairs;
+    p.nsched = 0;
+    if (p.tiles <= kMaxSched && pairs <= kMaxPairs && a.nseg % BN != 0) {
+        const SchedVal *sv =
+            tile_schedule(SchedKey{p.tiles, p.nmat * p.n_tiles, p.n_tiles, p.nseg, BN, pairs});
+        memcpy(p.first, sv->first.data(), sv->first.size() * sizeof(uint16_t));
+        memcpy(p.sched, sv->tile.data(), sv->tile.size() * sizeof(uint16_t));
+        p.nsched = p.tiles;
+    }
     return launch_pdl(gemm_tc2_kernel<BN, STAGES, STAGING>, dim3(2 * pairs), dim3(kThreads), L::ALLOC, s,
                       mA, mB[0], mB[1], mB[2], mo, p);
 }
