@@ -158,12 +158,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (j == 0) {
                         const int qb = un & 1;
                         if (!mbar_wait(&q_empty[qb], ((un >> 1) & 1) ^ 1, abort, status)) { ok = false; break; }
-                        // the unit's second query tile may lie past the last one
-                        const int nqt = 2 * qp + 1 < a.tq.tiles ? 2 : 1;
-                        mbar_expect_tx(&q_full[qb], nqt * L::TILE);
-                        for (int g = 0; g < nqt; ++g)
+                        // the unit's second query tile may lie past the last one: the
+                        // last tile is loaded twice then (its second results are
+                        // not stored), so no row scores uninitialised memory
+                        mbar_expect_tx(&q_full[qb], 2 * L::TILE);
+                        for (int g = 0; g < 2; ++g)
                             bulk_load(sm + L::OFF_Q + (qb * 2 + g) * L::TILE,
-                                      block(qg, a.tq, b, 2 * qp + g, h, L::TILE), L::TILE, &q_full[qb]);
+                                      block(qg, a.tq, b, min(2 * qp + g, a.tq.tiles - 1), h, L::TILE),
+                                      L::TILE, &q_full[qb]);
                         last_q_unit = un;
                     }
                     if (!mbar_wait(&kv_empty[st], ((item / NSTAGE) & 1) ^ 1, abort, status)) { ok = false; break; }
@@ -245,8 +247,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // exponentiated against a per-row reference max that is only raised
         // when a tile's max exceeds it by more than 2^8 (weights then stay
         // below 256, harmless in fp32); raising it rescales the row of O in
-        // TMEM, after the previous P V has landed.
+        // TMEM, after the previous P V has landed.  TMEM loads and stores are
+        // warp-collective, so every decision in front of one is taken by the
+        // whole warp: wait results are combined over the warp, and a rescale
+        // runs when any row of the warp needs it (the others scale by 1).
         const int g = (warp - 4) / 4;
+        auto wait_all = [&](uint64_t *bar, uint32_t par) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, par, abort, status));
+        };
         const int r = (warp % 4) * 32 + lane;  // query row of the tile = TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
         const uint32_t t_s = tmem + lane_base + g * BKV;
@@ -264,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < sc.kt; ++j, ++item) {
                 const uint32_t ph = item & 1;
                 const int nvalid = min(BKV, a.nk - j * BKV);
-                if (!mbar_wait(&s_full[g], ph, abort, status)) { ok = false; break; }
+                if (!wait_all(&s_full[g], ph)) { ok = false; break; }
                 fence_after_sync();
                 // the whole row of S: four loads, one wait
                 uint32_t sv[BKV];
@@ -291,11 +299,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     : fmaxf(mx[c], __uint_as_float(sv[e + c]));
                 float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
                 tmax *= sl2;
-                if (tmax > m_ref + 8.f) {  // raise the reference; O so far shrinks by alpha
-                    const float alpha = m_ref == -INFINITY ? 0.f : ex2_approx(m_ref - tmax);
+                const bool raise = tmax > m_ref + 8.f;  // raise the reference; O so far shrinks by alpha
+                if (__any_sync(0xffffffffu, raise)) {
+                    const float alpha = !raise ? 1.f : (m_ref == -INFINITY ? 0.f : ex2_approx(m_ref - tmax));
                     if (j > 0) {
                         // O holds P V up to tile j-1 once that MMA has landed
-                        if (!mbar_wait(&o_full[g], ph ^ 1, abort, status)) { ok = false; break; }
+                        if (!wait_all(&o_full[g], ph ^ 1)) { ok = false; break; }
                         fence_after_sync();
 #pragma unroll
                         for (int c0 = 0; c0 < DPAD; c0 += 16) {
@@ -310,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st_wait();
                     }
                     l_i *= alpha;
-                    m_ref = tmax;
+                    if (raise) m_ref = tmax;
                 }
                 const float ref = m_ref;
                 float ps[8];
@@ -346,8 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the unit's last P V, then O / l to global memory through the staging
             // rows, so that consecutive lanes store consecutive 16-byte pieces of
             // a row (a few rows per store instruction instead of 32)
-            if (!mbar_wait(&o_full[g], (item - 1) & 1, abort, status)) { ok = false; break; }
-            if (!mbar_wait(&stage_free[g], (un_count & 1) ^ 1, abort, status)) { ok = false; break; }
+            if (!wait_all(&o_full[g], (item - 1) & 1)) { ok = false; break; }
+            if (!wait_all(&stage_free[g], (un_count & 1) ^ 1)) { ok = false; break; }
             fence_after_sync();
             uint8_t *stg = sm + L::OFF_STG + g * L::STG;
             {
@@ -371,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_before_sync();  // O is read before the next unit's first P V overwrites it
             mbar_arrive(&stage_full[g]);
-            if (!mbar_wait(&stage_full[g], un_count & 1, abort, status)) { ok = false; break; }
+            if (!wait_all(&stage_full[g], un_count & 1)) { ok = false; break; }
             {
                 const int q0 = qp * 2 * BQ + g * BQ;  // query index of staging row 0
                 __nv_bfloat16 *obase = og + (long)b * a.q_bstride * a.ldo + (long)h * d;

@@ -89,6 +89,9 @@ SMALL = [
     (1, (1, 16, 16), 128, 2, (1, 2, 2), (1, 8, 8), (0, 4, 4)),
     # 2 x 4 x 16 windows (rows of 16 tokens) with a shift that is not half the window
     (1, (2, 16, 32), 144, 2, (1, 4, 4), (2, 4, 16), (1, 1, 4)),
+    # 200 and 100 proxies: key tiles whose second 64-key half is partly filled
+    (1, (1, 20, 40), 144, 2, (1, 2, 2), (1, 4, 8), (0, 2, 4)),
+    (1, (1, 20, 20), 144, 2, (1, 2, 2), (1, 4, 4), (0, 2, 2)),
 ]
 
 
