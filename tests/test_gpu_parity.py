@@ -179,6 +179,39 @@ def test_ratio_111_and_full_window(dtype):
     assert rel_err(f[0], want) <= TOL[dtype]
 
 
+def test_rescale_on_part_of_a_warp():
+    """Dense attention over two 128-key tiles where, inside every 32-row warp of the
+    first query tile, rows 0-15 score about 17 (in log2 units) against the second key
+    tile and about 0 against the first, and rows 16-31 score about 0 everywhere: half
+    of each warp raises its softmax reference (rescaling O) at the second tile and
+    half does not.  Both halves must match the oracle."""
+    grid, D, heads, a = (1, 16, 16), 144, 2, 10.0
+    N, d = 256, D // heads
+    rng = np.random.default_rng(77)
+    z = rng.normal(0.0, 0.1, (N, D))
+    rows = np.arange(N)
+    for h in range(heads):
+        e1, e2 = h * d, h * d + 1
+        z[(rows < 128) & (rows % 32 < 16), e1] += a   # queries that jump at key tile 1
+        z[rows >= 128, e2] += a                        # key tile 1
+    eye = np.eye(D)
+    wk = eye.copy()
+    for h in range(heads):  # K swaps each head's first two columns
+        e1, e2 = h * d, h * d + 1
+        wk[[e1, e2]] = wk[[e2, e1]]
+    zt = torch.tensor(z, dtype=torch.bfloat16)
+    W = tuple(torch.tensor(m, dtype=torch.bfloat16) for m in (eye, wk, eye, eye))
+    out = pt.ptdit_full_attn(zt[None].cuda(), grid, tuple(x.cuda() for x in W), heads)
+    torch.cuda.synchronize()
+    got = out[0].to("cpu", torch.float64).numpy()
+    z64 = zt.to(torch.float64).numpy()
+    W64 = tuple(x.to(torch.float64).numpy() for x in W)
+    want = O.masked_self_attention(z64, W64, heads, np.ones((N, N), bool))
+    # the jumping rows do attend to key tile 1 (the set-up does what it says)
+    assert np.allclose(want[0, 1] - z64[0, 1], a, atol=0.5)
+    assert rel_err(got, want) <= TOL["bf16"]
+
+
 def test_block_attn_is_deterministic():
     w = WORKLOADS["tiny_16x16_f32"].with_(dtype="bf16", D=144, heads=2)
     c = Case(2, w.grid, w.D, w.heads, "bf16")
