@@ -27,6 +27,7 @@ EXPORTS = (
     "ptdit_tcm", "ptdit_block_attn", "ptdit_full_attn", "ptdit_strerror", "ptdit_last_error",
     "ptdit_debug_proxy_map", "ptdit_debug_window_map", "ptdit_device_status", "ptdit_debug_timeout", "ptdit_timing_enable",
     "ptdit_timing_read", "ptdit_launch_count", "ptdit_window_attn_static",
+    "ptdit_debug_thl_map", "ptdit_debug_thl_units", "ptdit_debug_gemm_schedule",
 )
 
 
@@ -53,6 +54,7 @@ _P = ctypes.c_void_p
 _S = ctypes.POINTER(Shape)
 _W = ctypes.POINTER(AttnW)
 _I3 = ctypes.POINTER(ctypes.c_int)
+_IP = ctypes.POINTER(ctypes.c_int)  # an int the call writes
 
 
 def lib() -> ctypes.CDLL:
@@ -88,6 +90,10 @@ def lib() -> ctypes.CDLL:
             "ptdit_launch_count": (ctypes.c_longlong, []),
             "ptdit_window_attn_static": (ctypes.c_int, [_S, _I3, _I3, _W, ctypes.c_uint, _P, _P,
                                                         _P]),
+            "ptdit_debug_thl_map": (ctypes.c_int, [_I3, _I3, _I3, ctypes.c_int, _P, _P, _IP]),
+            "ptdit_debug_thl_units": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _P, _IP, _IP]),
+            "ptdit_debug_gemm_schedule": (ctypes.c_int, [ctypes.c_long, ctypes.c_int, ctypes.c_int,
+                                                         ctypes.c_int, _P, _P, _IP, _IP]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -251,6 +257,55 @@ def ptdit_debug_window_map(grid, window, shift, with_mask=True, stream=None):
     _check(lib().ptdit_debug_window_map(_i3(grid), _i3(window), _i3(shift), _ptr(tok),
                                         _ptr(allowed), _stream(stream)))
     return tok, allowed
+
+
+def ptdit_debug_thl_map(grid, window=None, shift=None):
+    """Tiled head layout of one batch item (host only): (row_of_token[N],
+    token_of_row[tiles * 128]) as int32 arrays, rows numbered tile * 128 + row and
+    -1 for rows that hold no token.  Identity tiles without `window`; with it, the
+    window tiles of the grid rolled by -shift."""
+    import numpy as np
+    N = grid[0] * grid[1] * grid[2]
+    windowed = 1 if window is not None else 0
+    w3 = _i3(window) if windowed else None
+    s3 = _i3(shift if shift is not None else (0, 0, 0)) if windowed else None
+    tiles = ctypes.c_int(0)
+    _check(lib().ptdit_debug_thl_map(_i3(grid), w3, s3, windowed, None, None, ctypes.byref(tiles)))
+    row = np.empty(N, np.int32)
+    tok = np.empty(tiles.value * 128, np.int32)
+    _check(lib().ptdit_debug_thl_map(_i3(grid), w3, s3, windowed, row.ctypes.data, tok.ctypes.data,
+                                     ctypes.byref(tiles)))
+    return row, tok
+
+
+def ptdit_debug_thl_units(d: int, vpad: bool = False):
+    """(offset[128, units] uint32, block_bytes): byte offset, inside one (tile, head)
+    block, of the 16-byte unit p of tile row r (host only)."""
+    import numpy as np
+    units, block = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().ptdit_debug_thl_units(int(d), int(vpad), None, ctypes.byref(units),
+                                       ctypes.byref(block)))
+    off = np.empty((128, units.value), np.uint32)
+    _check(lib().ptdit_debug_thl_units(int(d), int(vpad), off.ctypes.data, ctypes.byref(units),
+                                       ctypes.byref(block)))
+    return off, block.value
+
+
+def ptdit_debug_gemm_schedule(rows: int, nseg: int, nmat: int, pairs: int):
+    """Tile order of the 2-SM projection GEMM (host only): (tiles, None) when the
+    launch runs round robin, else (tiles, per-pair lists of tile indices)."""
+    import numpy as np
+    tiles, sched = ctypes.c_int(0), ctypes.c_int(0)
+    args = (int(rows), int(nseg), int(nmat), int(pairs))
+    _check(lib().ptdit_debug_gemm_schedule(*args, None, None, ctypes.byref(tiles),
+                                           ctypes.byref(sched)))
+    if not sched.value:
+        return tiles.value, None
+    first = np.empty(pairs + 1, np.int32)
+    tile = np.empty(tiles.value, np.int32)
+    _check(lib().ptdit_debug_gemm_schedule(*args, first.ctypes.data, tile.ctypes.data,
+                                           ctypes.byref(tiles), ctypes.byref(sched)))
+    return tiles.value, [tile[first[q]:first[q + 1]].tolist() for q in range(pairs)]
 
 
 def ptdit_device_status(reset: bool = False) -> int:

@@ -177,6 +177,13 @@ struct GemmArgs {
     int heads, d;
 };
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s);
+// The 2-SM projection GEMM's tile order for rows x nseg outputs of nmat
+// matrices on `pairs` CTA pairs (host only): *tiles, and *scheduled = 1 with
+// pair q taking tile[first[q]] .. tile[first[q+1] - 1] when the launch runs a
+// schedule (first and tile may be NULL to ask only), 0 for round robin.
+// Returns -1 for arguments no launch takes.
+int gemm_tc2_schedule(long rows, int nseg, int nmat, int pairs, int32_t *first, int32_t *tile,
+                      int *tiles, int *scheduled);
 
 // Attention core.  Head h uses columns h*d .. h*d+d-1 of q, k, v, o.
 //   ATT_ROWS:   queries are rows [0, nq) and keys rows [0, nk) of each batch

@@ -478,6 +478,11 @@ struct SchedVal {
     std::vector<uint16_t> first, tile;
 };
 
+// Whether a launch of `tiles` tiles on `pairs` pairs runs a schedule (else round robin).
+bool takes_schedule(int tiles, int pairs, int nseg, int bn) {
+    return tiles <= kMaxSched && pairs <= kMaxPairs && nseg % bn != 0;
+}
+
 const SchedVal *tile_schedule(const SchedKey &k) {
     static std::mutex mu;
     static std::map<SchedKey, SchedVal> cache;
@@ -575,7 +580,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
     }
     const int pairs = p.tiles < max_pairs ? p.tiles : max_pairs;
     p.nsched = 0;
-    if (p.tiles <= kMaxSched && pairs <= kMaxPairs && a.nseg % BN != 0) {
+    if (takes_schedule(p.tiles, pairs, a.nseg, BN)) {
         const SchedVal *sv =
             tile_schedule(SchedKey{p.tiles, p.nmat * p.n_tiles, p.n_tiles, p.nseg, BN, pairs});
         memcpy(p.first, sv->first.data(), sv->first.size() * sizeof(uint16_t));
@@ -602,6 +607,23 @@ bool gemm_tc2_supported(const GemmArgs &a) {
         if (a.thl[i] && (a.R[i] || a.d < 8 || a.d % 8 || a.heads * a.d != a.nseg)) return false;
     }
     return true;
+}
+
+int gemm_tc2_schedule(long rows, int nseg, int nmat, int pairs, int32_t *first, int32_t *tile,
+                      int *tiles, int *scheduled) {
+    constexpr int BN = 256;  // the tile width both launch variants use
+    if (rows < 1 || nseg < 64 || nseg % 64 || nmat < 1 || nmat > 3 || pairs < 1) return -1;
+    const long n_tiles = (nseg + BN - 1) / BN;
+    const long all = (rows + 2 * BMC - 1) / (2 * BMC) * nmat * n_tiles;
+    if (all > (1L << 30)) return -1;
+    *tiles = static_cast<int>(all);
+    *scheduled = takes_schedule(*tiles, pairs, nseg, BN) ? 1 : 0;
+    if (!*scheduled || !first || !tile) return 0;
+    const SchedVal *sv = tile_schedule(
+        SchedKey{*tiles, nmat * static_cast<int>(n_tiles), static_cast<int>(n_tiles), nseg, BN, pairs});
+    for (size_t i = 0; i < sv->first.size(); ++i) first[i] = sv->first[i];
+    for (size_t i = 0; i < sv->tile.size(); ++i) tile[i] = sv->tile[i];
+    return 0;
 }
 
 cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) {

@@ -815,4 +815,58 @@ int ptdit_debug_window_map(const int grid[3], const int window[3], const int shi
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "window map");
 }
 
+int ptdit_debug_thl_map(const int grid[3], const int window[3], const int shift[3], int windowed,
+                        int32_t *row_of_token, int32_t *token_of_row, int *tiles) {
+    if (!grid) return fail(PTDIT_ERR_NULL, "grid is NULL");
+    if (!tiles) return fail(PTDIT_ERR_NULL, "tiles is NULL");
+    ptdit_shape sh = {1, grid[0], grid[1], grid[2], 1, 1, PTDIT_F32};
+    Dims d;
+    TRY(check_shape(&sh, &d));
+    ThlDesc t;
+    if (windowed) {
+        WinGeom wg;
+        TRY(make_window(d, window, shift, &wg));
+        if (wg.n > kThlRows || kThlRows % wg.n)
+            return fail(PTDIT_ERR_SHAPE, "windows of %d tokens do not pack into %d-row tiles", wg.n,
+                        kThlRows);
+        t = thl_window(wg, d.N, 0);
+    } else {
+        t = thl_identity(d.N, 0);
+    }
+    *tiles = t.tiles;
+    if (row_of_token)
+        for (long tok = 0; tok < d.N; ++tok) {
+            int tile, r;
+            thl_locate(t, tok, tile, r);
+            row_of_token[tok] = tile * kThlRows + r;
+        }
+    if (token_of_row)
+        for (int tile = 0; tile < t.tiles; ++tile)
+            for (int r = 0; r < kThlRows; ++r)
+                token_of_row[tile * kThlRows + r] = static_cast<int32_t>(thl_token(t, tile, r));
+    return PTDIT_OK;
+}
+
+int ptdit_debug_thl_units(int d, int vpad, uint32_t *offset, int *units, int *block_bytes) {
+    if (!units || !block_bytes) return fail(PTDIT_ERR_NULL, "units or block_bytes is NULL");
+    if (d < 8 || d > 80 || d % 8)
+        return fail(PTDIT_ERR_SHAPE, "head width %d: the tiled layout holds 8 .. 80, multiples of 8", d);
+    const int vp = vpad && d > 64;
+    *units = thl_units(d, vp);
+    *block_bytes = static_cast<int>(thl_block_bytes(d, vp));
+    if (offset)
+        for (int r = 0; r < kThlRows; ++r)
+            for (int p = 0; p < *units; ++p) offset[r * *units + p] = thl_unit(r, p, vp);
+    return PTDIT_OK;
+}
+
+int ptdit_debug_gemm_schedule(long rows, int nseg, int nmat, int pairs, int32_t *first,
+                              int32_t *tile, int *tiles, int *scheduled) {
+    if (!tiles || !scheduled) return fail(PTDIT_ERR_NULL, "tiles or scheduled is NULL");
+    if (gemm_tc2_schedule(rows, nseg, nmat, pairs, first, tile, tiles, scheduled) != 0)
+        return fail(PTDIT_ERR_SHAPE, "no projection launch takes rows %ld, nseg %d, nmat %d, %d pairs",
+                    rows, nseg, nmat, pairs);
+    return PTDIT_OK;
+}
+
 }  // extern "C"

@@ -152,8 +152,9 @@ int ptdit_tcm(const ptdit_shape *shape, const int window[3], const int shift[3],
               const void *z_in, void *z_out, void *ws, size_t ws_bytes, ptdit_stream_t stream);
 
 /*
- * ptdit_block_attn -- the PT-Block attention path: GIIM then TCM
- *   (ProxyTokensTransformerBlock.forward steps 1-4 of the code listing).
+ * ptdit_block_attn -- the PT-Block attention path: GIIM then TCM, in the
+ *   order the block's forward pass runs them (Qihoo-T2X reading note, §3
+ *   Method, Eq. GIIM and Eq. TCM).
  */
 int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int window[3],
                      const int shift[3], const ptdit_attn_w *psa, const ptdit_attn_w *cross,
@@ -189,6 +190,45 @@ int ptdit_debug_proxy_map(const int grid[3], const int ratio[3], int32_t *proxy_
                           ptdit_stream_t stream);
 int ptdit_debug_window_map(const int grid[3], const int window[3], const int shift[3],
                            int32_t *token_at_slot, uint8_t *allowed, ptdit_stream_t stream);
+
+/*
+ * Host-only views of the data layout and the projection schedule, computed by
+ * the same host functions the launches use (no GPU, no CUDA call; for tests).
+ * All arrays are host memory owned by the caller; a NULL array skips that
+ * output, so a first call with NULL arrays returns the sizes.  Errors:
+ * PTDIT_ERR_NULL for a NULL count pointer, PTDIT_ERR_SHAPE for arguments no
+ * launch takes; nothing is written then.
+ *
+ *   ptdit_debug_thl_map -- the tiled head layout (THL) of the Q, K and V
+ *     operands of one batch item of the grid: one block per (128-row tile,
+ *     head), each the shared-memory tile the attention kernels read.
+ *     windowed = 0: identity tiles (tile t holds tokens 128 t .. 128 t + 127,
+ *     the layout of the proxy self-attention and cross-attention operands);
+ *     windowed = 1: window tiles of the grid rolled by -shift (window and shift
+ *     as in ptdit_window_attn; the window size must divide 128): 128 / n
+ *     windows per tile in window order, slots row-major inside a window.
+ *     Writes *tiles, row_of_token[N] = tile * 128 + row, and
+ *     token_of_row[*tiles * 128] = the token held by each tile row, or -1.
+ *   ptdit_debug_thl_units -- byte offset, inside one (tile, head) block of
+ *     head width d (8 .. 80, a multiple of 8; vpad: the V operand of the row
+ *     kernel, columns padded to 128), of the 16-byte unit p (head columns
+ *     8 p .. 8 p + 7) of tile row r: offset[r * units + p] for r < 128 and
+ *     p < units.  Writes *units and *block_bytes.
+ *   ptdit_debug_gemm_schedule -- the order in which the 2-SM projection GEMM
+ *     (256 x 256 output tiles; a matrix's last tile narrower when nseg is not a
+ *     multiple of 256) hands its rows x nseg outputs of nmat matrices to
+ *     `pairs` CTA pairs.  Writes *tiles and *scheduled: 1 when the launch runs
+ *     a longest-processing-time schedule, pair q taking tile[first[q]] ..
+ *     tile[first[q + 1] - 1] (first[pairs + 1], tile[*tiles]); 0 when it runs
+ *     round robin (tile t on pair t mod pairs; first and tile untouched).
+ *     Tile t covers row block t / (nmat * n_tiles), matrix (t / n_tiles) mod
+ *     nmat and column block t mod n_tiles, n_tiles = ceil(nseg / 256).
+ */
+int ptdit_debug_thl_map(const int grid[3], const int window[3], const int shift[3], int windowed,
+                        int32_t *row_of_token, int32_t *token_of_row, int *tiles);
+int ptdit_debug_thl_units(int d, int vpad, uint32_t *offset, int *units, int *block_bytes);
+int ptdit_debug_gemm_schedule(long rows, int nseg, int nmat, int pairs, int32_t *first,
+                              int32_t *tile, int *tiles, int *scheduled);
 
 
 /*
