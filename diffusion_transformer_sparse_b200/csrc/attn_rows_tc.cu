@@ -28,7 +28,10 @@
 //                unpadded V it needed costs a second, N = 16, MMA per K step).
 // Both query tiles share every K/V tile; the MMA warp issues PV_0, S_0(next),
 // PV_1, S_1(next), so each softmax gets its next scores while the other one
-// works.  Every wait is bounded (2 s).
+// works.  Splitting each tile's scores into two 64-key slots (so that the next
+// half's scores are ready when the softmax of a half ends) was slower: it
+// doubles the softmax -> P V -> S round trips, each about as long as before.
+// Every wait is bounded (2 s).
 #include <math.h>
 
 #include "tc_util.cuh"
