@@ -45,6 +45,8 @@ against closed forms, library routines, brute force or hand-derived fixtures.
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -52,6 +54,20 @@ import numpy as np
 # very long sequence stays small.  Rows are independent, so chunking changes
 # no arithmetic.
 _ROW_CHUNK = 4096
+
+# Heads are independent: above this many scores per head they run on a pool
+# of host threads (numpy releases the GIL in its matrix products and
+# element-wise passes).  Each head's arithmetic is the same either way and
+# writes its own columns of the result, so the output is bit-identical.
+_PARALLEL_SCORES = 1 << 22
+_POOL = None
+
+
+def _pool():
+    global _POOL
+    if _POOL is None:
+        _POOL = ThreadPoolExecutor(max_workers=max(1, min(16, os.cpu_count() or 1)))
+    return _POOL
 
 
 def _f64(a) -> np.ndarray:
@@ -108,6 +124,41 @@ def averaging(z, grid, ratio) -> np.ndarray:
     return blocks.mean(axis=(1, 3, 5)).reshape(-1, D)
 
 
+def window_members(grid, ratio) -> np.ndarray:
+    """[M, P]: the tokens of each proxy window, windows row-major over the window
+    grid, members row-major (t, y, x) inside the window."""
+    _check_divisible(grid, ratio, "ratio")
+    f, h, w = grid
+    pf, ph, pw = ratio
+    idx = np.arange(num_tokens(grid)).reshape(f // pf, pf, h // ph, ph, w // pw, pw)
+    return idx.transpose(0, 2, 4, 1, 3, 5).reshape(-1, pf * ph * pw)
+
+
+def proxy_tokens(z, grid, ratio, mode="mean", slots=None) -> np.ndarray:
+    """The proxy tokens of each window under the three extraction modes that the
+    pages compare  [T2X code-comparison section, get_proxy_token(mode=...); §3
+    Method ablation notes: Average / Top-Left / Random].
+
+    mean:   the window mean (Eq. GIIM, the method's choice);
+    first:  the window's first member in (t, y, x) order, i.e. its top-left
+            token in its first frame;
+    random: member slots[m] of window m; the random draw itself is an input
+            (slots, an int array [M] with 0 <= slots[m] < p_f p_h p_w).
+    """
+    if mode == "mean":
+        return averaging(z, grid, ratio)
+    z = _f64(z)
+    members = window_members(grid, ratio)
+    if mode == "first":
+        return z[members[:, 0]]
+    if mode == "random":
+        slots = np.asarray(slots)
+        if slots.shape != (members.shape[0],) or np.any(slots < 0) or np.any(slots >= members.shape[1]):
+            raise ValueError("slots must hold one member index per window")
+        return z[members[np.arange(members.shape[0]), slots]]
+    raise ValueError(f"unknown proxy mode {mode!r}")
+
+
 # --------------------------------------------------------------------------
 # Multi-head attention (the SA / CS / WSA / SWSA operator of Eq. GIIM, Eq. TCM)
 # --------------------------------------------------------------------------
@@ -137,14 +188,25 @@ def attention_heads(Q, K, V, heads, allow=None) -> np.ndarray:
     d = D // heads
     scale = 1.0 / math.sqrt(d)
     out = np.empty((Nq, D))
-    for h in range(heads):
+
+    parallel = heads > 1 and Nq * K.shape[0] >= _PARALLEL_SCORES
+    # concurrent heads each hold one chunk of scores: keep a chunk near 16 M entries
+    chunk = max(64, min(_ROW_CHUNK, (1 << 24) // max(1, K.shape[0]))) if parallel else _ROW_CHUNK
+
+    def head(h):
         cols = slice(h * d, (h + 1) * d)
-        for q0 in range(0, Nq, _ROW_CHUNK):
-            q1 = min(Nq, q0 + _ROW_CHUNK)
+        for q0 in range(0, Nq, chunk):
+            q1 = min(Nq, q0 + chunk)
             S = (Q[q0:q1, cols] @ K[:, cols].T) * scale
             if allow is not None:
                 S = np.where(allow[q0:q1], S, -np.inf)
             out[q0:q1, cols] = softmax_rows(S) @ V[:, cols]
+
+    if parallel:
+        list(_pool().map(head, range(heads)))
+    else:
+        for h in range(heads):
+            head(h)
     return out
 
 
@@ -159,15 +221,17 @@ def multihead_attention(x_q, x_kv, W, heads, allow=None) -> np.ndarray:
 # GIIM  [T2X §3 Eq. GIIM: z_s = CS(z_s, SA(Averaging(z_s))); code listing steps 1-2]
 # --------------------------------------------------------------------------
 
-def proxy_self_attention(z, grid, ratio, W_psa, heads, proxy_residual=False) -> np.ndarray:
-    """P' = SA(Averaging(z_s)) (+ P_a when proxy_residual)."""
-    Pa = averaging(z, grid, ratio)
+def proxy_self_attention(z, grid, ratio, W_psa, heads, proxy_residual=False, proxy_mode="mean",
+                         slots=None) -> np.ndarray:
+    """P' = SA(Averaging(z_s)) (+ P_a when proxy_residual); proxy_mode and slots
+    select another extraction (proxy_tokens)."""
+    Pa = proxy_tokens(z, grid, ratio, proxy_mode, slots)
     Pp = multihead_attention(Pa, Pa, W_psa, heads)
     return Pp + Pa if proxy_residual else Pp
 
 
 def giim(z, grid, ratio, W_psa, W_cross, heads, *, proxy_residual=False, residual=True,
-         rows=None) -> np.ndarray:
+         rows=None, proxy_mode="mean", slots=None) -> np.ndarray:
     """GIIM of one batch item.  z [N, D] -> [N, D].
 
     Cross-attention CS takes every latent token as the query and the proxies
@@ -175,7 +239,7 @@ def giim(z, grid, ratio, W_psa, W_cross, heads, *, proxy_residual=False, residua
     ``rows`` given, only those output rows are computed and the others are NaN.
     """
     z = _f64(z)
-    Pp = proxy_self_attention(z, grid, ratio, W_psa, heads, proxy_residual)
+    Pp = proxy_self_attention(z, grid, ratio, W_psa, heads, proxy_residual, proxy_mode, slots)
     if rows is None:
         cs = multihead_attention(z, Pp, W_cross, heads)
         return z + cs if residual else cs

@@ -400,3 +400,80 @@ def test_pins_catch_a_wrong_proxy_order(monkeypatch):
 
     monkeypatch.setattr(O, "averaging", col_major)
     assert _pin_fails(lambda: test_averaging_bruteforce((1, 4, 4)))
+
+
+# ---------------------------------------------------------------- proxy extraction modes
+
+def test_proxy_first_and_members_golden():
+    g = _golden("proxy_first_2x4x4.json")
+    grid = tuple(g["grid"])
+    z = np.arange(O.num_tokens(grid), dtype=np.float64)[:, None] * np.ones((1, 3))
+    for case in g["cases"]:
+        got = O.proxy_tokens(z, grid, tuple(case["ratio"]), "first")
+        np.testing.assert_array_equal(got[:, 0], case["first_token"])
+    np.testing.assert_array_equal(O.window_members(grid, (1, 2, 2))[3],
+                                  g["members_ratio_122_window_3"])
+
+
+@pytest.mark.parametrize("grid,ratio", [((2, 4, 6), (1, 2, 3)), ((4, 4, 4), (2, 2, 1)),
+                                        ((3, 2, 5), (3, 1, 5)), ((2, 6, 4), (1, 1, 1))])
+def test_proxy_random_bruteforce(grid, ratio):
+    """Scalar loops: member k of window m is the k-th smallest token index whose
+    window (from coordinates) is m."""
+    rng = np.random.default_rng(3)
+    f, h, w = grid
+    pf, ph, pw = ratio
+    N, P = f * h * w, pf * ph * pw
+    M = N // P
+    z = rng.normal(size=(N, 5))
+    slots = rng.integers(0, P, M)
+    got = O.proxy_tokens(z, grid, ratio, "random", slots)
+    for m in range(M):
+        members = []
+        for t in range(N):
+            tt, y, x = t // (h * w), (t // w) % h, t % w
+            if ((tt // pf) * (h // ph) + y // ph) * (w // pw) + x // pw == m:
+                members.append(t)
+        assert len(members) == P
+        assert np.array_equal(got[m], z[members[slots[m]]])
+    # slot 0 everywhere is the 'first' mode
+    assert np.array_equal(O.proxy_tokens(z, grid, ratio, "random", np.zeros(M, int)),
+                          O.proxy_tokens(z, grid, ratio, "first"))
+
+
+def test_mean_of_all_single_token_proxies_is_the_average():
+    """Averaging the 'random' extraction over every slot gives the window mean."""
+    grid, ratio = (2, 8, 6), (2, 4, 3)
+    rng = np.random.default_rng(8)
+    z = rng.normal(size=(O.num_tokens(grid), 7))
+    P = 24
+    M = O.num_tokens(grid) // P
+    acc = sum(O.proxy_tokens(z, grid, ratio, "random", np.full(M, k)) for k in range(P)) / P
+    _close(acc, O.proxy_tokens(z, grid, ratio, "mean"), 1e-13)
+
+
+def test_giim_with_first_proxies_matches_library_mha():
+    grid, ratio, D, heads = (2, 4, 4), (1, 2, 2), 12, 3
+    rng = np.random.default_rng(21)
+    z = rng.normal(size=(O.num_tokens(grid), D))
+    Wp, Wc = _weights(D, 1), _weights(D, 2)
+    Pa = z[[0, 2, 8, 10, 16, 18, 24, 26]]  # golden first tokens
+    Pp = torch_mha(Pa, Pa, Wp, heads)
+    want = z + torch_mha(z, Pp, Wc, heads)
+    _close(O.giim(z, grid, ratio, Wp, Wc, heads, proxy_mode="first"), want, 1e-10)
+
+
+def test_proxy_modes_reject_bad_input():
+    z = np.zeros((16, 2))
+    with pytest.raises(ValueError):
+        O.proxy_tokens(z, (1, 4, 4), (1, 2, 2), "random", np.array([0, 1, 2, 4]))
+    with pytest.raises(ValueError):
+        O.proxy_tokens(z, (1, 4, 4), (1, 2, 2), "median")
+
+
+def test_pins_catch_a_last_token_proxy(monkeypatch):
+    """A 'first' mode that took each window's last member is caught by the golden."""
+    real = O.window_members
+    monkeypatch.setattr(O.ptdit_oracle, "window_members", lambda g, r: real(g, r)[:, ::-1])
+    with pytest.raises(AssertionError):
+        test_proxy_first_and_members_golden()
