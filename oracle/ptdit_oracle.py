@@ -404,3 +404,64 @@ def masked_self_attention(z, W, heads, allow, *, residual=True) -> np.ndarray:
     z = _f64(z)
     y = multihead_attention(z, z, W, heads, allow)
     return z + y if residual else y
+
+
+# --------------------------------------------------------------------------
+# The complete PT-Block  [T2X §3 Method: "PT-Block (GIIM + TCM + text
+# cross-attn + MLP)", the block diagram; code-comparison section,
+# ProxyTokensTransformerBlock.forward steps 1-4]
+#
+# Readings (the pages name the sub-layers and their order but not the norms'
+# form, the MLP's width or activation, nor where each norm sits):
+#   * every sub-layer is pre-norm with a residual: x <- x + F(LN(x)); the proxy
+#     self-attention normalises the proxies (proxy_norm1) and adds them back,
+#     as the listing's step 1 does;
+#   * LN is a LayerNorm over D with a per-channel scale and shift and
+#     epsilon eps; its variance is the population (biased) variance;
+#   * the text cross-attention takes the normalised latents as queries and the
+#     text tokens (already projected to width D outside the block) as keys and
+#     values;
+#   * the MLP is fc1 (D -> Dh, bias) -> GELU, tanh form -> fc2 (Dh -> D, bias),
+#     the feed-forward of the DiT / PixArt-alpha blocks PT-DiT is compared with;
+#   * attention projections have no bias (as in the rest of this path).
+# --------------------------------------------------------------------------
+
+def layer_norm(x, gamma, beta, eps=1e-6) -> np.ndarray:
+    """Per row: (x - mean) / sqrt(var + eps) * gamma + beta, var the mean squared deviation."""
+    x = _f64(x)
+    mu = x.mean(axis=1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * _f64(gamma) + _f64(beta)
+
+
+def gelu_tanh(x) -> np.ndarray:
+    """GELU in its tanh form: x/2 (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
+    x = _f64(x)
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def mlp(x, W1, b1, W2, b2) -> np.ndarray:
+    """fc2(GELU(fc1(x))): W1 [Dh][D], b1 [Dh], W2 [D][Dh], b2 [D]."""
+    return project(gelu_tanh(project(x, W1) + _f64(b1)), W2) + _f64(b2)
+
+
+def pt_block(z, grid, ratio, window, shift, W, norms, mlp_w, text, heads, *, eps=1e-6,
+             proxy_mode="mean", slots=None) -> np.ndarray:
+    """One complete PT-Block on one batch item.  z [N, D] -> [N, D].
+
+    W: {"psa", "cross", "wsa", "swsa", "text"} -> (Wq, Wk, Wv, Wo);
+    norms: {"proxy", "cross", "wsa", "swsa", "text", "mlp"} -> (gamma, beta);
+    mlp_w: (W1, b1, W2, b2); text: [L, D] text tokens.
+    """
+    z = _f64(z)
+    ln = {k: (lambda x, g=g, b=b: layer_norm(x, g, b, eps)) for k, (g, b) in norms.items()}
+    Pa = proxy_tokens(z, grid, ratio, proxy_mode, slots)
+    Pn = ln["proxy"](Pa)
+    Pp = Pa + multihead_attention(Pn, Pn, W["psa"], heads)
+    z1 = z + multihead_attention(ln["cross"](z), Pp, W["cross"], heads)
+    z2 = z1 + window_self_attention(ln["wsa"](z1), grid, window, (0, 0, 0), W["wsa"], heads,
+                                    residual=False)
+    z3 = z2 + window_self_attention(ln["swsa"](z2), grid, window, shift, W["swsa"], heads,
+                                    residual=False)
+    z4 = z3 + multihead_attention(ln["text"](z3), _f64(text), W["text"], heads)
+    return z4 + mlp(ln["mlp"](z4), *mlp_w)

@@ -477,3 +477,116 @@ def test_pins_catch_a_last_token_proxy(monkeypatch):
     monkeypatch.setattr(O.ptdit_oracle, "window_members", lambda g, r: real(g, r)[:, ::-1])
     with pytest.raises(AssertionError):
         test_proxy_first_and_members_golden()
+
+
+# ---------------------------------------------------------------- the complete PT-Block
+
+def _norm_params(D, rng):
+    return (1.0 + 0.1 * rng.normal(size=D), 0.1 * rng.normal(size=D))
+
+
+def test_layer_norm_matches_library():
+    rng = np.random.default_rng(5)
+    x = rng.normal(size=(37, 24)) * 3 + 1
+    g, b = _norm_params(24, rng)
+    ln = torch.nn.LayerNorm(24, eps=1e-6, dtype=torch.float64)
+    with torch.no_grad():
+        ln.weight.copy_(torch.from_numpy(g))
+        ln.bias.copy_(torch.from_numpy(b))
+        want = ln(torch.from_numpy(x)).numpy()
+    _close(O.layer_norm(x, g, b, 1e-6), want, 1e-12)
+    # unit scale, zero shift: every row has mean 0 and mean square var / (var + eps)
+    y = O.layer_norm(x, np.ones(24), np.zeros(24), 1e-6)
+    assert np.allclose(y.mean(axis=1), 0, atol=1e-12)
+    var = x.var(axis=1)
+    assert np.allclose((y ** 2).mean(axis=1), var / (var + 1e-6), rtol=1e-12)
+
+
+def test_gelu_tanh_matches_library_and_closed_forms():
+    x = np.linspace(-9, 9, 1001)
+    want = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    _close(O.gelu_tanh(x), want, 1e-14)
+    assert O.gelu_tanh(np.array([0.0]))[0] == 0.0
+    assert np.allclose(O.gelu_tanh(x) - O.gelu_tanh(-x), x, atol=1e-14)  # gelu(x) - gelu(-x) = x
+
+
+def test_mlp_matches_library():
+    rng = np.random.default_rng(6)
+    D, Dh = 12, 48
+    x = rng.normal(size=(9, D))
+    W1, W2 = rng.normal(size=(Dh, D)) / 4, rng.normal(size=(D, Dh)) / 7
+    b1, b2 = rng.normal(size=Dh), rng.normal(size=D)
+    net = torch.nn.Sequential(torch.nn.Linear(D, Dh, dtype=torch.float64),
+                              torch.nn.GELU(approximate="tanh"),
+                              torch.nn.Linear(Dh, D, dtype=torch.float64))
+    with torch.no_grad():
+        for lin, W, b in ((net[0], W1, b1), (net[2], W2, b2)):
+            lin.weight.copy_(torch.from_numpy(W))
+            lin.bias.copy_(torch.from_numpy(b))
+        want = net(torch.from_numpy(x)).numpy()
+    _close(O.mlp(x, W1, b1, W2, b2), want, 1e-12)
+
+
+def _block_inputs(D, heads, N, L, seed):
+    rng = np.random.default_rng(seed)
+    W = {m: _weights(D, 30 + i) for i, m in enumerate(("psa", "cross", "wsa", "swsa", "text"))}
+    norms = {k: _norm_params(D, rng) for k in ("proxy", "cross", "wsa", "swsa", "text", "mlp")}
+    Dh = 4 * D
+    mlp_w = (rng.normal(size=(Dh, D)) / math.sqrt(D), 0.1 * rng.normal(size=Dh),
+             rng.normal(size=(D, Dh)) / math.sqrt(Dh), 0.1 * rng.normal(size=D))
+    return rng.normal(size=(N, D)), W, norms, mlp_w, rng.normal(size=(L, D))
+
+
+def test_pt_block_matches_library_composition():
+    """The block wired from torch's LayerNorm, MultiheadAttention (window branches
+    as full attention under the pinned pair mask) and an nn.Sequential MLP."""
+    grid, ratio, window, shift, D, heads = (2, 4, 4), (1, 2, 2), (2, 2, 2), (1, 1, 1), 12, 2
+    N = O.num_tokens(grid)
+    z, W, norms, mlp_w, text = _block_inputs(D, heads, N, 5, 40)
+
+    def tln(x, key):
+        ln = torch.nn.LayerNorm(D, eps=1e-6, dtype=torch.float64)
+        with torch.no_grad():
+            ln.weight.copy_(torch.from_numpy(norms[key][0]))
+            ln.bias.copy_(torch.from_numpy(norms[key][1]))
+            return ln(torch.from_numpy(x)).numpy()
+
+    Pa = O.averaging(z, grid, ratio)
+    Pp = Pa + torch_mha(tln(Pa, "proxy"), tln(Pa, "proxy"), W["psa"], heads)
+    z1 = z + torch_mha(tln(z, "cross"), Pp, W["cross"], heads)
+    a0 = O.window_allow_matrix(grid, window, (0, 0, 0))
+    a1 = O.window_allow_matrix(grid, window, shift)
+    z2 = z1 + torch_mha(tln(z1, "wsa"), tln(z1, "wsa"), W["wsa"], heads, a0)
+    z3 = z2 + torch_mha(tln(z2, "swsa"), tln(z2, "swsa"), W["swsa"], heads, a1)
+    z4 = z3 + torch_mha(tln(z3, "text"), text, W["text"], heads)
+    net = torch.nn.Sequential(torch.nn.Linear(D, 4 * D, dtype=torch.float64),
+                              torch.nn.GELU(approximate="tanh"),
+                              torch.nn.Linear(4 * D, D, dtype=torch.float64))
+    with torch.no_grad():
+        net[0].weight.copy_(torch.from_numpy(mlp_w[0]))
+        net[0].bias.copy_(torch.from_numpy(mlp_w[1]))
+        net[2].weight.copy_(torch.from_numpy(mlp_w[2]))
+        net[2].bias.copy_(torch.from_numpy(mlp_w[3]))
+        want = z4 + net(torch.from_numpy(tln(z4, "mlp"))).numpy()
+    got = O.pt_block(z, grid, ratio, window, shift, W, norms, mlp_w, text, heads)
+    _close(got, want, 1e-10)
+
+
+def test_pins_catch_an_unbiased_variance(monkeypatch):
+    real = O.ptdit_oracle.layer_norm
+
+    def wrong(x, g, b, eps=1e-6):
+        x = np.asarray(x, dtype=np.float64)
+        return (x - x.mean(1, keepdims=True)) / np.sqrt(x.var(1, ddof=1, keepdims=True) + eps) * g + b
+
+    monkeypatch.setattr(O, "layer_norm", wrong)
+    with pytest.raises(AssertionError):
+        test_layer_norm_matches_library()
+    monkeypatch.setattr(O, "layer_norm", real)
+
+
+def test_pins_catch_a_wrong_mlp_term(monkeypatch):
+    real = O.ptdit_oracle.mlp
+    monkeypatch.setattr(O.ptdit_oracle, "mlp", lambda x, *w: real(x, *w) - x)
+    with pytest.raises(AssertionError):
+        test_pt_block_matches_library_composition()
