@@ -3,15 +3,18 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 A step is one ptdit_block_attn call over one batch of the workload (default:
-the 1024px text-to-image grid, 4 x 64 x 64 tokens, D = 1152, 16 heads, bf16),
-inputs resident in HBM.  L2 is flushed (a 256 MiB write) before every timed
+the long high-resolution video, 32 x 64 x 64 = 131072 tokens, D = 1152, 16
+heads, bf16, proxy ratio (1,16,16), TCM window 2 x 8 x 8), inputs resident in
+HBM.  L2 is flushed (a 256 MiB write) before every timed
 step and each step is timed alone with CUDA events on the launching stream.
 Under torchrun every rank runs its own replica of the workload (batch items
 are independent, so there is no data-path collective); the job time is the
 max over ranks.  Rank 0 prints one JSON line.
 
---impl reference times the float64 CPU oracle on the host cores instead, one
-batch item per step.
+--impl reference times the float64 CPU oracle on the host cores instead: each
+step runs the oracle's stages on a bounded sample of one batch item (all
+proxies, a sample of latent rows for the cross-attention and a sample of
+windows for each TCM branch) and extrapolates the whole item's time from it.
 
 Measurement options beyond the default line: --grid F,H,W and --ratio F,H,W
 override the workload's token grid and proxy ratio (the long-video ratio
@@ -39,8 +42,10 @@ METRIC = "PT-Block attention tokens/s and TFLOP/s (bf16, 1 B200) vs tensor/HBM r
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 
-# DRAM bytes per launch of the dominant kernel from one ncu capture of the
-# current kernel source (None when the kernel changed since the capture).
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernel, averaged over the launches of one step, from one ncu capture
+# of the current kernel source, per workload.  Absent when the kernel changed
+# since the capture.
 TRAFFIC = {}
 
 
@@ -186,31 +191,79 @@ def cpu_baseline(w, z, W, min_seconds=10.0, max_items=16):
                       f"block_attn in float64, {dt:.1f} s"}
 
 
+_FIXED = {}
+
+
+def oracle_sample_step(w, z64, W64, rng, rows=2048, windows=16):
+    """One reference step: the oracle's stages on a bounded sample of one batch
+    item, and the whole item's time extrapolated from it.
+
+    Every stage runs the oracle as it stands.  Averaging and proxy self-attention
+    run in full (their cost does not grow with the sample); the cross-attention
+    runs for `rows` random latent rows and each TCM branch for `windows` random
+    windows, and their per-row and per-window times are scaled to the whole
+    grid.  A branch's fixed cost (the roll and window partition of the whole
+    grid) is timed separately, with no window, and added once.
+    Returns (extrapolated seconds per item, seconds spent)."""
+    import numpy as np
+
+    import oracle as O
+    t_start = time.perf_counter()
+    z = z64[0]
+    t0 = time.perf_counter()
+    Pp = O.proxy_self_attention(z, w.grid, w.ratio, W64["psa"], w.heads)
+    t_proxy = time.perf_counter() - t0
+    r = rng.choice(w.N, size=min(rows, w.N), replace=False)
+    t0 = time.perf_counter()
+    _ = z[r] + O.multihead_attention(z[r], Pp, W64["cross"], w.heads)
+    t_cross = (time.perf_counter() - t0) * w.N / len(r)
+    nwin = w.N // w.n
+    t_tcm = 0.0
+    for shift, m in (((0, 0, 0), "wsa"), (w.shift, "swsa")):
+        if (w.name, shift) not in _FIXED:
+            t0 = time.perf_counter()
+            O.window_self_attention(z, w.grid, w.window, shift, W64[m], w.heads, windows=[])
+            _FIXED[(w.name, shift)] = time.perf_counter() - t0
+        fixed = _FIXED[(w.name, shift)]
+        k = rng.choice(nwin, size=min(windows, nwin), replace=False)
+        t0 = time.perf_counter()
+        O.window_self_attention(z, w.grid, w.window, shift, W64[m], w.heads, windows=k)
+        part = time.perf_counter() - t0
+        t_tcm += fixed + max(0.0, part - fixed) * nwin / len(k)
+    return t_proxy + t_cross + t_tcm, time.perf_counter() - t_start
+
+
 def run_reference(args, w):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
+    import numpy as np
     z, W = host_inputs(w)
     from diffusion_transformer_sparse_b200 import synth
     z64 = [synth.as_f64(z[0])]
     W64 = {m: tuple(synth.as_f64(x) for x in ws) for m, ws in W.items()}
+    rng = np.random.default_rng(2024)
     for _ in range(args.warmup):
-        oracle_step(w, z64, W64, 0)
-    times = []
+        oracle_sample_step(w, z64, W64, rng)
+    est, spent = [], 0.0
     for _ in range(args.steps):
-        t0 = time.perf_counter()
-        oracle_step(w, z64, W64, 0)
-        times.append(time.perf_counter() - t0)
-    total = sum(times)
+        t, dt = oracle_sample_step(w, z64, W64, rng)
+        est.append(t)
+        spent += dt
+    total = sum(est)
     value = args.steps * w.N / total
+    sample = (f"per step: one of {w.B} batch items of {w.name}; averaging and proxy SA in "
+              f"full, cross-attention on 2048 random latent rows, each TCM branch on 16 "
+              f"random windows plus its whole-grid roll, scaled to all {w.N} rows and "
+              f"{w.N // w.n} windows (extrapolated); {spent / args.steps:.2f} s of CPU work "
+              f"per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                         "sample": f"one of {w.B} batch items of {w.name} per step, full "
-                                   "block_attn in float64"},
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -224,6 +277,24 @@ def config_of(w):
 
 
 # ------------------------------------------------------------------ GPU arm
+def kernel_work(w):
+    """Algorithmic work per step of each kernel kind (library timing-hook names):
+    (amount, unit, bound).  Averaging and the window cores are HBM-bound and
+    count bytes: averaging reads N and writes M rows of D elements; a window
+    core reads Q, K and V and writes O, 4 N D elements per launch.  The others
+    count FLOP (a multiply-add is 2)."""
+    e = 2 if w.dtype == "bf16" else 4
+    f = flops.block_flops(w.N, w.M, w.n, w.D)
+    B = w.B
+    return {
+        "average": (B * flops.average_bytes(w.N, w.M, w.D, e), "bytes", "hbm"),
+        "gemm": (B * f["proj"], "flop", "tensor"),
+        "attn_proxy": (B * f["psa_core"], "flop", "tensor"),
+        "attn_cross": (B * f["cross_core"], "flop", "tensor"),
+        "attn_window": (B * 2 * 4 * w.N * w.D * e, "bytes", "hbm"),
+    }
+
+
 def run_gpu(args, w):
     import torch
 
@@ -243,9 +314,9 @@ def run_gpu(args, w):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(zin=z, zout=out):
+    def step(zin=z, zout=out, s=stream):
         pt.ptdit_block_attn(zin, w.grid, w.ratio, w.window, w.shift, W["psa"], W["cross"],
-                            W["wsa"], W["swsa"], w.heads, z_out=zout, ws=ws, stream=stream)
+                            W["wsa"], W["swsa"], w.heads, z_out=zout, ws=ws, stream=s)
 
     def timed(K, fn):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -287,7 +358,11 @@ def run_gpu(args, w):
             dist.destroy_process_group()
         return 0
 
-    # per-kernel durations: the same K steps with the library's event hooks on
+    # per-kernel durations: the same K steps with the library's event hooks on.
+    # An event pair around every launch also keeps each kernel from starting its
+    # prologue under the previous one's tail (programmatic dependent launch), so
+    # the hooked steps run slower than the timed ones (timing_hook_overhead); the
+    # per-kernel times are those of kernels that run alone.
     pt.ptdit_timing_enable(64 * args.steps)
     hooked = timed(args.steps, step)
     recs = pt.ptdit_timing_read(64 * args.steps)
@@ -297,43 +372,55 @@ def run_gpu(args, w):
         d = per_kind.setdefault(k, [0, 0.0])
         d[0] += 1
         d[1] += t
-    f = flops.block_flops(w.N, w.M, w.n, w.D)
     peaks = load_peaks()
+    f = flops.block_flops(w.N, w.M, w.n, w.D)
     step_flops = w.B * f["total"]
-    gemm_ms = per_kind.get("gemm", [0, 0.0])[1] / args.steps
-    gemm_launches = per_kind.get("gemm", [0, 0.0])[0] / args.steps
+    work = kernel_work(w)
+    kernels = {}
+    hooked_kernel_ms = sum(v[1] for v in per_kind.values()) / args.steps
+    for k, (n, t) in sorted(per_kind.items()):
+        kms = t / args.steps
+        ent = {"launches_per_step": n / args.steps, "ms_per_step": kms,
+               "share": kms / max(1e-9, hooked_kernel_ms)}
+        if k in work and kms > 0:
+            amount, unit, bound = work[k]
+            if unit == "bytes":
+                ach = amount / (kms / 1e3) / 1e9
+                ent.update({"bound": "hbm", "algorithmic_bytes_per_step": amount,
+                            "achieved": ach, "unit": "GB/s", "peak": peaks["hbm"],
+                            "frac": ach / peaks["hbm"]})
+            else:
+                ach = amount / (kms / 1e3) / 1e12
+                ent.update({"bound": "tensor", "algorithmic_flop_per_step": amount,
+                            "achieved": ach, "unit": "TFLOP/s", "peak": peaks["bf16"],
+                            "frac": ach / peaks["bf16"]})
+        kernels[k] = ent
+    gemm_n, gemm_t = per_kind.get("gemm", [0, 0.0])
+    gemm_ms = gemm_t / args.steps
     proj_flops = w.B * f["proj"]
     achieved = proj_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    peak_note = "measured" if peaks["source"] == "measured" else "fallback"
+    traffic = TRAFFIC.get(w.name)
     roofline = {
-        "kernel": "gemm (QKV and O projections)", "bound": "tensor",
-        "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-        "frac": achieved / peaks["bf16_sustained"] if achieved else None,
-        "traffic": TRAFFIC.get("gemm"),
-        "peak_kind": f"bf16 sustained, {peaks['source']}",
-        "launches_per_step": gemm_launches,
+        "kernel": "gemm_tc2 (QKV and O projections)", "bound": "tensor",
+        "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
+        "frac": achieved / peaks["bf16"] if achieved else None,
+        "traffic": traffic,
+        "peak_kind": f"bf16 dense burst, of {peak_note} (each launch is timed alone, "
+                     f"well under a second)",
+        "frac_of_sustained": achieved / peaks["bf16_sustained"] if achieved else None,
+        "launches_per_step": gemm_n / args.steps,
+        "flops_per_launch": proj_flops / max(1, gemm_n / args.steps),
         "flops_per_step": proj_flops,
     }
-    kernels = {k: {"launches_per_step": v[0] / args.steps, "ms_per_step": v[1] / args.steps,
-                   "share": v[1] / max(1e-9, sum(x[1] for x in per_kind.values()))}
-               for k, v in sorted(per_kind.items())}
     hook_overhead = sum(hooked) / max(1e-9, sum(ms))
 
-    # end to end through the public call with pinned host buffers
-    z_pin = z_host.pin_memory()
-    out_pin = torch.empty_like(z_host).pin_memory()
-
-    def e2e_step():
-        z.copy_(z_pin, non_blocking=True)
-        step()
-        out_pin.copy_(out, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    barrier(dist, dev)
-    e2e_ms = max_over_ranks(sum(timed(args.steps, e2e_step)), dist, dev)
-    zbytes = z.numel() * z.element_size()
-    e2e = {"value": world * args.steps * w.B * w.N / (e2e_ms / 1e3), "unit": UNIT,
-           "h2d_bytes_per_step": zbytes, "d2h_bytes_per_step": zbytes}
+    # end to end through the public call: every step copies its input from pinned
+    # host memory and its result back.  Step k's input copy runs on its own
+    # stream during step k - 1 and step k's output copy during step k + 1
+    # (double-buffered device tensors, ordered by events), so PCIe and the
+    # computation overlap the way a serving loop would run them.
+    e2e = e2e_pipelined(args.steps, w, z_host, step, dev, stream, dist)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -359,6 +446,59 @@ def run_gpu(args, w):
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def e2e_pipelined(K, w, z_host, step, dev, stream, dist):
+    """Tokens/s of K steps, each copying its input host -> device and its output
+    device -> host, with the copies overlapped with neighbouring steps."""
+    import torch
+    z_pin = z_host.pin_memory()
+    h_out = [torch.empty_like(z_host).pin_memory() for _ in range(2)]
+    d_in = [torch.empty(z_host.shape, dtype=z_host.dtype, device=dev) for _ in range(2)]
+    d_out = [torch.empty_like(d_in[0]) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def run(K):
+        ev = lambda: torch.cuda.Event()
+        h2d, comp, d2h = [ev() for _ in range(K)], [ev() for _ in range(K)], [ev() for _ in range(K)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        s_in.wait_event(t0)
+
+        def copy_in(k):
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(comp[k - 2])  # step k - 2 has read d_in[k % 2]
+                d_in[k % 2].copy_(z_pin, non_blocking=True)
+                h2d[k].record(s_in)
+
+        copy_in(0)
+        for k in range(K):
+            if k + 1 < K:
+                copy_in(k + 1)
+            stream.wait_event(h2d[k])
+            if k >= 2:
+                stream.wait_event(d2h[k - 2])  # d_out[k % 2] has been copied out
+            step(d_in[k % 2], d_out[k % 2], stream)
+            comp[k].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp[k])
+                h_out[k % 2].copy_(d_out[k % 2], non_blocking=True)
+                d2h[k].record(s_out)
+        stream.wait_event(d2h[K - 1])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        return t0.elapsed_time(t1)
+
+    run(2)
+    barrier(dist, dev)
+    e2e_ms = max_over_ranks(run(K), dist, dev)
+    world = dist.get_world_size() if dist is not None else 1
+    zbytes = z_host.numel() * z_host.element_size()
+    return {"value": world * K * w.B * w.N / (e2e_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": zbytes, "d2h_bytes_per_step": zbytes,
+            "ms_per_step": e2e_ms / K,
+            "note": "input and output copies double-buffered on their own streams"}
 
 
 def run_dense(args, w):
@@ -407,6 +547,66 @@ def run_dense(args, w):
     return 0
 
 
+def run_block(args, w, L=120):
+    """The complete PT-Block (ptdit_pt_block): GIIM, TCM, text cross-attention over
+    L text tokens and the MLP (D -> 4 D -> D), pre-norm residual sub-layers."""
+    import torch
+
+    import diffusion_transformer_sparse_b200 as pt
+    from diffusion_transformer_sparse_b200 import synth
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    z_host, W_host = host_inputs(w)
+    z = z_host.to(dev)
+    Dh = 4 * w.D
+    bp = synth.block_params(w.D, Dh, w.dtype)
+    attn = {m: tuple(x.to(dev) for x in ws) for m, ws in W_host.items()}
+    attn["text"] = tuple(x.to(dev) for x in bp["text"])
+    norms = {k: tuple(x.to(dev) for x in v) for k, v in bp["norms"].items()}
+    mlp_w = tuple(x.to(dev) for x in bp["mlp"])
+    text = synth.text_tokens(w.B, L, w.D, w.dtype).to(dev)
+    shape = pt.make_shape(z, w.grid, w.heads)
+    ws = pt.pt_block_workspace(shape, w.ratio, L, Dh)
+    out = torch.empty_like(z)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        pt.ptdit_pt_block(z, w.grid, w.ratio, w.window, w.shift, attn, norms, mlp_w, text,
+                          w.heads, z_out=out, ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    pt.ptdit_timing_enable(64 * args.steps)
+    for _ in range(args.steps):
+        flush.zero_()
+        step()
+    recs = pt.ptdit_timing_read(64 * args.steps)
+    pt.ptdit_timing_enable(0)
+    per = {}
+    for k, t in recs:
+        per[k] = per.get(k, 0.0) + t / args.steps
+    f = flops.pt_block_flops(w.N, w.M, w.n, w.D, L, Dh)
+    print(json.dumps({
+        "mode": "pt_block", "metric": "complete PT-Block tokens/s", "unit": UNIT,
+        "value": w.B * w.N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,
+        "warmup": args.warmup, "config": dict(config_of(w), text_len=L, mlp_hidden=Dh),
+        "tflops": w.B * f["total"] / (ms / 1e3) / 1e12,
+        "kernels_ms_per_step": per, "note": "per-kernel times from a second pass with hooks"}),
+        flush=True)
+    return 0
+
+
 def parse3(text):
     v = tuple(int(x) for x in text.split(","))
     if len(v) != 3:
@@ -429,6 +629,8 @@ def main(argv=None):
     ap.add_argument("--ratio", type=parse3, help="override the proxy ratio F,H,W")
     ap.add_argument("--dense", action="store_true",
                     help="time the dense comparator (full global self-attention) instead")
+    ap.add_argument("--block", action="store_true",
+                    help="time the complete PT-Block (norms, text cross-attention, MLP) instead")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     w = configs.WORKLOADS[args.workload]
@@ -440,6 +642,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.dense:
         return run_dense(args, w)
+    if args.block:
+        return run_block(args, w)
     return run_gpu(args, w)
 
 

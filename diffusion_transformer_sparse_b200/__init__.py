@@ -16,10 +16,13 @@ LIB_PATH = os.path.join(HERE, "libptdit.so")
 PTDIT_F32, PTDIT_BF16 = 0, 1
 PTDIT_PROXY_RESIDUAL = 0x1
 PTDIT_NO_RESIDUAL = 0x2
+PTDIT_PROXY_MEAN, PTDIT_PROXY_FIRST, PTDIT_PROXY_RANDOM = 0, 1, 2
+PROXY_MODES = {"mean": PTDIT_PROXY_MEAN, "first": PTDIT_PROXY_FIRST, "random": PTDIT_PROXY_RANDOM}
 # status codes (include/ptdit.h)
 (PTDIT_OK, PTDIT_ERR_NULL, PTDIT_ERR_SHAPE, PTDIT_ERR_DTYPE, PTDIT_ERR_WORKSPACE, PTDIT_ERR_CUDA,
  PTDIT_ERR_TIMEOUT, PTDIT_ERR_ALIGN, PTDIT_ERR_ALIAS) = range(9)
-KINDS = ("average", "gemm", "attn_proxy", "attn_cross", "attn_window", "attn_dense")
+KINDS = ("average", "gemm", "attn_proxy", "attn_cross", "attn_window", "attn_dense", "norm",
+         "attn_text")
 
 # Every symbol declared in include/ptdit.h.
 EXPORTS = (
@@ -28,6 +31,8 @@ EXPORTS = (
     "ptdit_debug_proxy_map", "ptdit_debug_window_map", "ptdit_device_status", "ptdit_debug_timeout", "ptdit_timing_enable",
     "ptdit_timing_read", "ptdit_launch_count", "ptdit_window_attn_static",
     "ptdit_debug_thl_map", "ptdit_debug_thl_units", "ptdit_debug_gemm_schedule",
+    "ptdit_proxy_extract", "ptdit_giim_ex", "ptdit_pt_block", "ptdit_pt_block_workspace_bytes",
+    "ptdit_debug_wait_limit",
 )
 
 
@@ -46,6 +51,17 @@ class Shape(ctypes.Structure):
 class AttnW(ctypes.Structure):
     _fields_ = [("wq", ctypes.c_void_p), ("wk", ctypes.c_void_p), ("wv", ctypes.c_void_p),
                 ("wo", ctypes.c_void_p)]
+
+
+class NormW(ctypes.Structure):
+    _fields_ = [("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p)]
+
+
+class BlockW(ctypes.Structure):
+    _fields_ = ([(m, AttnW) for m in ("psa", "cross", "wsa", "swsa", "text")] +
+                [("norm_" + k, NormW) for k in ("proxy", "cross", "wsa", "swsa", "text", "mlp")] +
+                [("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("w2", ctypes.c_void_p),
+                 ("b2", ctypes.c_void_p), ("mlp_hidden", ctypes.c_int), ("eps", ctypes.c_float)])
 
 
 _lib = None
@@ -68,6 +84,14 @@ def lib() -> ctypes.CDLL:
         sig = {
             "ptdit_proxy_average": (ctypes.c_int, [_S, _I3, _P, _P, _P]),
             "ptdit_workspace_bytes": (ctypes.c_size_t, [_S, _I3, _I3]),
+            "ptdit_proxy_extract": (ctypes.c_int, [_S, _I3, ctypes.c_int, _P, _P, _P, _P]),
+            "ptdit_pt_block_workspace_bytes": (ctypes.c_size_t, [_S, _I3, ctypes.c_int,
+                                                                 ctypes.c_int]),
+            "ptdit_pt_block": (ctypes.c_int, [_S, _I3, _I3, _I3, ctypes.POINTER(BlockW), _P,
+                                              ctypes.c_int, ctypes.c_int, _P, _P, _P, _P,
+                                              ctypes.c_size_t, _P]),
+            "ptdit_giim_ex": (ctypes.c_int, [_S, _I3, ctypes.c_int, _P, _W, _W, ctypes.c_uint, _P,
+                                             _P, _P, ctypes.c_size_t, _P]),
             "ptdit_giim": (ctypes.c_int, [_S, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
                                           ctypes.c_size_t, _P]),
             "ptdit_window_attn": (ctypes.c_int, [_S, _I3, _I3, _W, ctypes.c_uint, _P, _P, _P,
@@ -84,6 +108,7 @@ def lib() -> ctypes.CDLL:
             "ptdit_debug_window_map": (ctypes.c_int, [_I3, _I3, _I3, _P, _P, _P]),
             "ptdit_device_status": (ctypes.c_int, [ctypes.c_int]),
             "ptdit_debug_timeout": (ctypes.c_int, [ctypes.c_longlong, _P]),
+            "ptdit_debug_wait_limit": (ctypes.c_int, [ctypes.c_longlong]),
             "ptdit_timing_enable": (ctypes.c_int, [ctypes.c_int]),
             "ptdit_timing_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
                                                  ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
@@ -181,6 +206,33 @@ def ptdit_proxy_average(z, grid, ratio, proxies=None, stream=None):
     return proxies
 
 
+def _slots(mode, slots, B, M):
+    """Device int32 slot array for PTDIT_PROXY_RANDOM (None otherwise)."""
+    if PROXY_MODES[mode] != PTDIT_PROXY_RANDOM:
+        return None
+    if slots is None or not slots.is_cuda or slots.dtype.is_floating_point:
+        raise ValueError("mode 'random' needs a CUDA int32 slots tensor of B * M entries")
+    if slots.numel() != B * M:
+        raise ValueError(f"slots holds {slots.numel()} entries, expected {B * M}")
+    return slots.contiguous()
+
+
+def ptdit_proxy_extract(z, grid, ratio, mode="mean", slots=None, proxies=None, stream=None):
+    """[B, N, D] -> [B, M, D] proxy tokens: window mean, first token or the slot-th
+    member of each window (slots: CUDA int32 [B, M])."""
+    import torch
+    _check_z(z)
+    shape = make_shape(z, grid, 1)
+    P = ratio[0] * ratio[1] * ratio[2]
+    M = z.shape[1] // P
+    if proxies is None:
+        proxies = torch.empty(z.shape[0], M, z.shape[2], dtype=z.dtype, device=z.device)
+    sl = _slots(mode, slots, z.shape[0], M)
+    _check(lib().ptdit_proxy_extract(ctypes.byref(shape), _i3(ratio), PROXY_MODES[mode],
+                                     _ptr(sl), _ptr(z), _ptr(proxies), _stream(stream)))
+    return proxies
+
+
 def _prep(z_in, grid, heads, z_out, ws, ratio, window):
     import torch
     _check_z(z_in)
@@ -199,6 +251,69 @@ def ptdit_giim(z_in, grid, ratio, psa, cross, heads, flags=0, z_out=None, ws=Non
     _check(lib().ptdit_giim(ctypes.byref(shape), _i3(ratio), ctypes.byref(wp), ctypes.byref(wc),
                             flags, _ptr(z_in), _ptr(z_out), _ptr(ws), ws.numel(),
                             _stream(stream)))
+    return z_out
+
+
+def ptdit_giim_ex(z_in, grid, ratio, mode, slots, psa, cross, heads, flags=0, z_out=None,
+                  ws=None, stream=None):
+    shape, z_out, ws = _prep(z_in, grid, heads, z_out, ws, ratio, None)
+    P = ratio[0] * ratio[1] * ratio[2]
+    sl = _slots(mode, slots, z_in.shape[0], z_in.shape[1] // P)
+    wp, wc = attn_w(psa), attn_w(cross)
+    _check(lib().ptdit_giim_ex(ctypes.byref(shape), _i3(ratio), PROXY_MODES[mode], _ptr(sl),
+                               ctypes.byref(wp), ctypes.byref(wc), flags, _ptr(z_in), _ptr(z_out),
+                               _ptr(ws), ws.numel(), _stream(stream)))
+    return z_out
+
+
+def block_w(attn: dict, norms: dict, mlp, eps: float = 1e-6) -> BlockW:
+    """BlockW from {"psa", "cross", "wsa", "swsa", "text"} -> (Wq, Wk, Wv, Wo), {norm name}
+    -> (gamma, beta) and (W1, b1, W2, b2), all contiguous CUDA tensors."""
+    bw = BlockW()
+    for m in ("psa", "cross", "wsa", "swsa", "text"):
+        setattr(bw, m, attn_w(attn[m]))
+    for k in ("proxy", "cross", "wsa", "swsa", "text", "mlp"):
+        g, b = norms[k]
+        setattr(bw, "norm_" + k, NormW(g.data_ptr(), b.data_ptr()))
+    W1, b1, W2, b2 = mlp
+    for t in (W1, b1, W2, b2):
+        if not t.is_contiguous():
+            raise ValueError("MLP parameters must be contiguous")
+    bw.w1, bw.b1, bw.w2, bw.b2 = W1.data_ptr(), b1.data_ptr(), W2.data_ptr(), b2.data_ptr()
+    bw.mlp_hidden = int(W1.shape[0])
+    bw.eps = float(eps)
+    return bw
+
+
+def pt_block_workspace(shape: Shape, ratio, text_len: int, mlp_hidden: int):
+    import torch
+    n = int(lib().ptdit_pt_block_workspace_bytes(ctypes.byref(shape), _i3(ratio), int(text_len),
+                                                 int(mlp_hidden)))
+    if n == 0:
+        raise PtditError(2, "invalid arguments for the block workspace")
+    return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+def ptdit_pt_block(z_in, grid, ratio, window, shift, attn: dict, norms: dict, mlp, text, heads,
+                   eps=1e-6, mode="mean", slots=None, z_out=None, ws=None, stream=None):
+    """One complete PT-Block (GIIM, TCM, text cross-attention, MLP; pre-norm residual
+    sub-layers).  text: [B, L, D] CUDA tensor of text tokens at the model width."""
+    import torch
+    _check_z(z_in)
+    shape = make_shape(z_in, grid, heads)
+    if not text.is_cuda or not text.is_contiguous() or text.dim() != 3:
+        raise ValueError("text must be a contiguous [B, L, D] CUDA tensor")
+    bw = block_w(attn, norms, mlp, eps)
+    if z_out is None:
+        z_out = torch.empty_like(z_in)
+    if ws is None:
+        ws = pt_block_workspace(shape, ratio, text.shape[1], bw.mlp_hidden)
+    P = ratio[0] * ratio[1] * ratio[2]
+    sl = _slots(mode, slots, z_in.shape[0], z_in.shape[1] // P)
+    _check(lib().ptdit_pt_block(ctypes.byref(shape), _i3(ratio), _i3(window), _i3(shift),
+                                ctypes.byref(bw), _ptr(text), int(text.shape[1]),
+                                PROXY_MODES[mode], _ptr(sl), _ptr(z_in), _ptr(z_out), _ptr(ws),
+                                ws.numel(), _stream(stream)))
     return z_out
 
 
@@ -320,6 +435,11 @@ def ptdit_device_status(reset: bool = False) -> int:
 def ptdit_debug_timeout(limit_ns: int, stream=None):
     """Launch one bounded wait that nothing releases (gives up after limit_ns)."""
     _check(lib().ptdit_debug_timeout(int(limit_ns), _stream(stream)))
+
+
+def ptdit_debug_wait_limit(limit_ns: int):
+    """Limit of the window kernel's waits for work on this thread (0: the default 2 s)."""
+    _check(lib().ptdit_debug_wait_limit(int(limit_ns)))
 
 
 def ptdit_timing_enable(max_launches: int):

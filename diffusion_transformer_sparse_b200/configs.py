@@ -51,10 +51,20 @@ WORKLOADS = {
         Workload("t2i_2048px_128x128", 1, (1, 128, 128), 1152, 16, "bf16", (1, 8, 8), (1, 8, 8), (0, 4, 4)),
         Workload("t2v_16x32x48", 1, (16, 32, 48), 1152, 16, "bf16", (1, 4, 4), (2, 8, 8), (1, 4, 4)),
         Workload("video_32x64x64", 1, (32, 64, 64), 1152, 16, "bf16", (1, 16, 16), (2, 8, 8), (1, 4, 4)),
+        # the pages' own video setting: temporal compression p_f = 4 (§3 Method,
+        # compression-ratio paragraph) on the T2V clip and on the long video
+        Workload("t2v_pf4_16x32x48", 1, (16, 32, 48), 1152, 16, "bf16", (4, 4, 4), (2, 8, 8), (1, 4, 4)),
+        Workload("video_pf4_32x64x64", 1, (32, 64, 64), 1152, 16, "bf16", (4, 8, 8), (2, 8, 8), (1, 4, 4)),
+        # text-to-multiview: 24 views of one object treated as the frames of a
+        # video (T2MV section), 512 px views -> 32 x 32 tokens, p_f = 4
+        Workload("t2mv_24x32x32", 1, (24, 32, 32), 1152, 16, "bf16", (4, 4, 4), (2, 8, 8), (1, 4, 4)),
     ]
 }
 ORDER = list(WORKLOADS)
-# The headline bench workload: the 1024px text-to-image grid, batch 4.
-HEADLINE = "t2i_1024px_64x64_b4"
+# The five workloads of the scope (the others are the pages' video / multiview settings).
+CORE = ORDER[:5]
+# The headline bench workload: the largest grid, the long high-resolution video
+# (32 x 64 x 64 tokens).
+HEADLINE = "video_32x64x64"
 # Ratio sweep on the long video grid.
 RATIO_SWEEP = [(1, 2, 2), (1, 4, 4), (1, 8, 8), (1, 16, 16)]

@@ -432,12 +432,11 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_attention_rows_tc(const AttnArgs &a, cudaStream_t s) {
-    // V's ones column (row sums from P V) exists when the head is 8 columns
-    // narrower than its tile (d = 72)
-    if (a.tv.ones) return a.d == 72 ? launch_rows<80, true>(a, s) : cudaErrorInvalidValue;
-    if (a.d == 64) return launch_rows<64, false>(a, s);
-    if (a.d == 80) return launch_rows<80, false>(a, s);
-    return cudaErrorInvalidValue;
+    // d = 72: the row sums come out of P V through V's ones column (column 72);
+    // other widths (8 .. 80, multiples of 8) sum P in the softmax
+    if (a.d < 8 || a.d > 80 || a.d % 8) return cudaErrorInvalidValue;
+    if (a.d == 72 && a.tv.ones) return launch_rows<80, true>(a, s);
+    return a.d <= 64 ? launch_rows<64, false>(a, s) : launch_rows<80, false>(a, s);
 }
 
 }  // namespace ptdit

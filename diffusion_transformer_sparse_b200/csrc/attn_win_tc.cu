@@ -34,7 +34,8 @@
 //                row; when its four warps are done the buffer goes back to the
 //                loader.
 // With SUMV the row sums of P come out of P V through V's ones column.
-// Every wait is bounded (2 s).
+// Every wait is bounded (2 s, or the limit ptdit_debug_wait_limit sets); the
+// loader and softmax warps decide to give up per warp, never per lane.
 #include <math.h>
 
 #include "tc_util.cuh"
@@ -48,7 +49,11 @@ using namespace tc;
 constexpr int BQ = 128;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;  // per slot: S/P 128 columns, O 128 columns
-constexpr int kKeys = 16;            // mask keys per tile: 2 windows x 8 wrap codes
+// Key masks of a tile: one per (window in tile, wrap code).  Windows of 16, 32
+// or 64 tokens (8, 4 or 2 per tile, each inside one 64-key half of the tile)
+// keep 64 bits per mask, the bits of their half: up to 64 masks.  A window of
+// 128 tokens keeps 128 bits per mask: 8 masks.  512 bytes per buffer either way.
+constexpr int kMaskWords = 128;
 constexpr int NBUF = 3;              // load buffers: units whose operands are in flight
 
 template <int DPAD>
@@ -60,10 +65,10 @@ struct WinLayout {
     static constexpr int BUF = 3 * TILE;                       // Q, K, V of one unit
     static constexpr int OFF_INFO = NBUF * BUF;                // int info[NBUF][128]
     static constexpr int OFF_ROW = OFF_INFO + NBUF * BQ * 4;   // int row[NBUF][128] (token rows)
-    static constexpr int OFF_MASK = OFF_ROW + NBUF * BQ * 4;   // uint32 kmask[NBUF][kKeys][4]
+    static constexpr int OFF_MASK = OFF_ROW + NBUF * BQ * 4;   // uint32 kmask[NBUF][kMaskWords]
     // output staging: 32 rows (pitch <= 160 B) per softmax warp
     static constexpr int WSTG = 32 * 160;
-    static constexpr int OFF_STG = OFF_MASK + NBUF * kKeys * 16;
+    static constexpr int OFF_STG = OFF_MASK + NBUF * kMaskWords * 4;
     static constexpr int OFF_OROW = OFF_STG + 8 * WSTG;       // int orow[8][32]: rows being stored
     static constexpr int OFF_BAR = OFF_OROW + 8 * 32 * 4;
     // qk_full[NBUF], v_full[NBUF], buf_free[NBUF], s_full[2], p_full[2], o_full[2], o_free[2], drain
@@ -77,6 +82,7 @@ struct WinLayout {
 struct WinSched {
     int tiles;  // tiles per batch item
     int units;  // B x tiles x heads
+    unsigned long long wait_ns;  // limit of every wait for work (the final drain keeps 2 s)
 };
 
 template <int DPAD, bool SUMV>
@@ -139,7 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int u = u0 + k, bf = k % NBUF;
             const int h = u % a.heads, rest = u / a.heads, tile = rest % sc.tiles,
                       b = rest / sc.tiles;
-            if (!mbar_wait(&buf_free[bf], ((k / NBUF) & 1) ^ 1, abort, status)) break;
+            if (!mbar_wait_warp(&buf_free[bf], ((k / NBUF) & 1) ^ 1, abort, status, sc.wait_ns))
+                break;
             uint8_t *sQ = sm + bf * L::BUF, *sK = sQ + L::TILE, *sV = sK + L::TILE;
             if (lane == 0) {
                 const long blk = ((long)b * sc.tiles + tile) * a.heads + h;
@@ -169,13 +176,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     info[bf * BQ + r] = in;
                     rowsm[bf * BQ + r] = row;
                 }
-                // one 128-bit key mask per mask key: keys of the same window and wrap code
-                for (int v = 0; v < kKeys; ++v)
+                // one key mask per mask key (window in tile, wrap code): the keys of
+                // the same window and wrap code, over the window's 64-key half of
+                // the tile (windows of up to 64 tokens) or over all 128 keys
+                const int nkeys = n < BQ ? (BQ / n) * 8 : 8;
+                for (int v = 0; v < nkeys; ++v) {
+                    const int half = n < BQ ? ((v >> 3) * n) >> 6 : 0;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const uint32_t bits = __ballot_sync(0xffffffffu, inf[q] == v);
-                        if (lane == 0) kmask[(bf * kKeys + v) * 4 + q] = bits;
+                        if (lane == 0) {
+                            if (n >= BQ)
+                                kmask[bf * kMaskWords + v * 4 + q] = bits;
+                            else if ((q >> 1) == half)
+                                kmask[bf * kMaskWords + v * 2 + (q & 1)] = bits;
+                        }
                     }
+                }
             }
             __syncwarp();
             mbar_arrive(&qk_full[bf]);
@@ -190,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // S(k) into TMEM slot k % 2 (after P V(k - 2), issued earlier, has read P(k - 2))
             auto issue_s = [&](int k) {
                 const int bf = k % NBUF, g = k & 1;
-                if (!mbar_wait(&qk_full[bf], (k / NBUF) & 1, abort, status)) return false;
+                if (!mbar_wait(&qk_full[bf], (k / NBUF) & 1, abort, status, sc.wait_ns)) return false;
                 fence_after_sync();
                 const uint32_t aQ = smem_u32(sm + bf * L::BUF);
                 const uint32_t aK = aQ + L::TILE;
@@ -209,9 +226,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // unit k - 2 has been read out of the slot's O columns
             auto issue_pv = [&](int k) {
                 const int bf = k % NBUF, g = k & 1;
-                if (!mbar_wait(&p_full[g], (k >> 1) & 1, abort, status)) return false;
-                if (!mbar_wait(&o_free[g], ((k >> 1) & 1) ^ 1, abort, status)) return false;
-                if (!mbar_wait(&v_full[bf], (k / NBUF) & 1, abort, status)) return false;
+                if (!mbar_wait(&p_full[g], (k >> 1) & 1, abort, status, sc.wait_ns)) return false;
+                if (!mbar_wait(&o_free[g], ((k >> 1) & 1) ^ 1, abort, status, sc.wait_ns))
+                    return false;
+                if (!mbar_wait(&v_full[bf], (k / NBUF) & 1, abort, status, sc.wait_ns)) return false;
                 fence_after_sync();
                 const uint32_t aV = smem_u32(sm + bf * L::BUF + 2 * L::TILE);
                 const uint32_t tO = tmem + g * 256 + 128;
@@ -251,24 +269,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pitch = nch * 16 + (nch % 8 == 0 ? 16 : 0);
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
         // the row's own keys: its window inside the tile
-        const int c_lo = n < BQ ? (r / n) * n : 0;
+        // (windows of up to 64 tokens lie inside one 64-key half of the tile)
+        const int c_lo = n < BQ ? (r >> 6) << 6 : 0;
         for (int k = g; k < nunits; k += 2) {
             const int u = u0 + k, bf = k % NBUF;
             const uint32_t ph = (k >> 1) & 1;  // phase of this slot's barriers
             const int h = u % a.heads;
-            if (!mbar_wait(&qk_full[bf], (k / NBUF) & 1, abort, status)) break;  // masks and rows
+            // every wait of these warps is decided by the whole warp (a TMEM load or
+            // store, which all 32 lanes must reach, follows each of them)
+            if (!mbar_wait_warp(&qk_full[bf], (k / NBUF) & 1, abort, status, sc.wait_ns))
+                break;  // masks and rows
             const int qi = info[bf * BQ + r];
             // this row's token: the buffer's rows may be rewritten once P V has read it
             const int qrow = rowsm[bf * BQ + r];
             uint32_t allow[4] = {0u, 0u, 0u, 0u};
             if (qi >= 0) {
-                const uint4 w4 = *reinterpret_cast<const uint4 *>(kmask + (bf * kKeys + qi) * 4);
-                allow[0] = w4.x;
-                allow[1] = w4.y;
-                allow[2] = w4.z;
-                allow[3] = w4.w;
+                if (n < BQ) {  // the 64 bits of the row's half
+                    const uint2 w2 =
+                        *reinterpret_cast<const uint2 *>(kmask + bf * kMaskWords + qi * 2);
+                    allow[0] = w2.x;
+                    allow[1] = w2.y;
+                } else {
+                    const uint4 w4 =
+                        *reinterpret_cast<const uint4 *>(kmask + bf * kMaskWords + qi * 4);
+                    allow[0] = w4.x;
+                    allow[1] = w4.y;
+                    allow[2] = w4.z;
+                    allow[3] = w4.w;
+                }
             }
-            if (!mbar_wait(&s_full[g], ph, abort, status)) break;
+            if (!mbar_wait_warp(&s_full[g], ph, abort, status, sc.wait_ns)) break;
             fence_after_sync();
             float l = 0.f;
             uint32_t pk[64];
@@ -277,8 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(t_s + c_lo, *reinterpret_cast<uint32_t(*)[32]>(sv));
                 tmem_ld32(t_s + c_lo + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
                 tmem_ld_wait();
-                const uint32_t w0 = c_lo == 0 ? allow[0] : allow[2];
-                const uint32_t w1 = c_lo == 0 ? allow[1] : allow[3];
+                const uint32_t w0 = allow[0], w1 = allow[1];
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
@@ -346,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // with consecutive lanes on consecutive 16-byte pieces of a token row;
             // the token rows come from the unit's buffer, whose next load waits
             // for that buffer's release by P V and is two units away
-            if (!mbar_wait(&o_full[g], ph, abort, status)) break;
+            if (!mbar_wait_warp(&o_full[g], ph, abort, status, sc.wait_ns)) break;
             fence_after_sync();
             uint8_t *stg = sm + L::OFF_STG + (warp - 4) * L::WSTG - (warp % 4) * 32 * pitch;
             int *orow = reinterpret_cast<int *>(sm + L::OFF_OROW) + (warp - 4) * 32;
@@ -423,6 +452,7 @@ cudaError_t launch_win(const AttnArgs &a, cudaStream_t s) {
     const int pack = BQ / a.geom.n;
     sc.tiles = (a.geom.nwin + pack - 1) / pack;
     sc.units = a.B * sc.tiles * a.heads;
+    sc.wait_ns = debug_wait_limit_ns();
     const int sms = num_sms() > 0 ? num_sms() : 148;
     const int grid = (sc.units + 1) / 2 < sms ? (sc.units + 1) / 2 : sms;
     cudaError_t e = cudaFuncSetAttribute(attn_win_kernel<DPAD, SUMV>,
@@ -435,12 +465,13 @@ cudaError_t launch_win(const AttnArgs &a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_attention_win_tc(const AttnArgs &a, cudaStream_t s) {
-    // V's ones column (row sums from P V) exists when the head is 8 columns
-    // narrower than its tile (d = 72)
-    if (a.tv.ones) return a.d == 72 ? launch_win<80, true>(a, s) : cudaErrorInvalidValue;
-    if (a.d == 64) return launch_win<64, false>(a, s);
-    if (a.d == 80) return launch_win<80, false>(a, s);
-    return cudaErrorInvalidValue;
+    if (a.d < 8 || a.d > 80 || a.d % 8) return cudaErrorInvalidValue;
+    const int n = a.geom.n;
+    if (n != 16 && n != 32 && n != 64 && n != 128) return cudaErrorInvalidValue;
+    // d = 72: the row sums come out of P V through V's ones column (column 72);
+    // other widths sum P in the softmax (a ones column, if any, goes unread)
+    if (a.d == 72 && a.tv.ones) return launch_win<80, true>(a, s);
+    return a.d <= 64 ? launch_win<64, false>(a, s) : launch_win<80, false>(a, s);
 }
 
 }  // namespace ptdit

@@ -149,6 +149,15 @@ enum DType { DT_F32 = 0, DT_BF16 = 1 };
 cudaError_t launch_proxy_average(int dtype, const ProxyGeom &g, int B, int D, const void *z,
                                  void *proxies, cudaStream_t s);
 
+// out[b, m, :] = z[b, member slots[b * M + m] of window m, :] (member 0, the
+// window's first token, when slots is null); a slot outside [0, P) leaves the
+// row zero and sets *status to PTDIT_ERR_SHAPE.
+cudaError_t launch_proxy_select(int dtype, const ProxyGeom &g, int B, int D, const void *z,
+                                void *proxies, const int32_t *slots, int *status, cudaStream_t s);
+
+// Device address of the library's status word on the current device.
+int *device_status_ptr();
+
 // Tile geometry of an operand stored in tiled head layout (thl.cuh).
 struct ThlDesc {
     int mode;      // 0: plain row-major; 1: identity tiles; 2: window tiles
@@ -164,6 +173,10 @@ struct ThlDesc {
 // (in-place residual) or be null.  thl[s] (or null) asks for
 // C_s in tiled head layout instead (heads of width d, no residual); only the
 // launchers that report support for it accept one.
+// bias[s] (or null), a vector of nseg values of the call's dtype, is added to
+// C_s before the activation `act` and before the residual:
+// C_s = act(A W_s^T + bias_s) + R_s.
+enum GemmAct { ACT_NONE = 0, ACT_GELU_TANH = 1 };
 struct GemmArgs {
     int dtype;
     const void *A;
@@ -175,7 +188,29 @@ struct GemmArgs {
     int rows, nseg, K, nmat;
     const ThlDesc *thl[3];
     int heads, d;
+    const void *bias[3];
+    int act;
 };
+
+// GELU, tanh form: x/2 (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).  The fp32
+// path calls tanhf; the bf16 paths, whose result is rounded to bf16 (relative
+// step 2^-8) right after, use the hardware tanh approximation (relative error
+// about 2^-11).
+__device__ __forceinline__ float gelu_tanh_arg(float x) {
+    return 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
+}
+__device__ __forceinline__ float gelu_tanh_exact(float x) {
+    return 0.5f * x * (1.f + tanhf(gelu_tanh_arg(x)));
+}
+__device__ __forceinline__ float gelu_tanh_fast(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(gelu_tanh_arg(x)));
+    return 0.5f * x * (1.f + t);
+}
+
+// y[r, :] = LayerNorm(x[r, :]) * gamma + beta over D columns (rows x D, contiguous).
+cudaError_t launch_layer_norm(int dtype, long rows, int D, const void *x, const void *gamma,
+                              const void *beta, float eps, void *y, cudaStream_t s);
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s);
 // The 2-SM projection GEMM's tile order for rows x nseg outputs of nmat
 // matrices on `pairs` CTA pairs (host only): *tiles, and *scheduled = 1 with

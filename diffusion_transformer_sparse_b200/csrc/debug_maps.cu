@@ -57,6 +57,7 @@ cudaError_t launch_debug_window_map(const WinGeom &g, int32_t *tok, uint8_t *all
 
 namespace ptdit {
 int report_error(int code, const char *text);
+void set_debug_wait_limit_ns(unsigned long long ns);
 namespace {
 // One thread waits on a barrier that nothing arrives on; the bounded wait gives
 // up after limit_ns and records PTDIT_ERR_TIMEOUT, as a stalled kernel would.
@@ -91,5 +92,12 @@ extern "C" int ptdit_debug_timeout(long long limit_ns, ptdit_stream_t stream) {
     ptdit::count_launch();
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return ptdit::report_error(PTDIT_ERR_CUDA, cudaGetErrorString(e));
+    return PTDIT_OK;
+}
+
+extern "C" int ptdit_debug_wait_limit(long long limit_ns) {
+    if (limit_ns < 0 || limit_ns > 10000000000LL)
+        return ptdit::report_error(PTDIT_ERR_SHAPE, "limit_ns must be in [0, 10 s]");
+    ptdit::set_debug_wait_limit_ns((unsigned long long)limit_ns);
     return PTDIT_OK;
 }

@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
     const T *__restrict__ W = static_cast<const T *>(a.W[s]);
     T *C = static_cast<T *>(a.C[s]);
     const T *R = static_cast<const T *>(a.R[s]);
+    const T *bias = static_cast<const T *>(a.bias[s]);
     const int row0 = blockIdx.y * BM, col0 = blockIdx.x * BN;
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
     const int lr = tid / 4, lk = (tid % 4) * 4;  // loader: row (or weight row), 4 consecutive k
@@ -64,6 +65,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
             const int c = col0 + tx * 4 + j;
             if (c >= a.nseg) continue;
             float v = acc[i][j];
+            if (bias) v += to_f32(bias[c]);
+            if (a.act == ACT_GELU_TANH) v = gelu_tanh_exact(v);
             if (R) v += to_f32(R[(long)r * a.ldc + c]);
             C[(long)r * a.ldc + c] = from_f32<T>(v);
         }

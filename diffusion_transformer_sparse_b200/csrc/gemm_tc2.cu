@@ -67,6 +67,8 @@ constexpr int kMaxSched = 4096;  // tiles a schedule can describe (larger launch
 struct Tc2Params {
     void *C[3];
     const void *R[3];
+    const void *bias[3];  // row-major outputs: bias added before act and the residual
+    int act;              // GemmAct
     Thl thl[3];  // mode THL_OFF: row-major output through the staging tiles
     int heads, d;     // tiled outputs: heads and head width
     int nunits[3];    // tiled outputs: 16-byte units per block row
@@ -330,7 +332,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             decode_tile2(p, t, m_tile, seg, n_tile);
             const int row0 = m_tile * 2 * BMC + rank * BMC + q * 32;
             const int col0 = n_tile * BN;
-            const int nchunk = tile_width<BN>(p, n_tile) / 32;
+            // 32-column chunks; a tile whose width is 16 past a multiple of 32 ends in a
+            // half chunk (its other 16 columns are outside the matrix: not stored)
+            const int cend = col0 + tile_width<BN>(p, n_tile);
+            const int nchunk = (tile_width<BN>(p, n_tile) + 31) / 32;
             if (p.thl[seg].mode != THL_OFF) {
                 // ---- tiled head layout: this lane's row, 8 columns per store
                 const Thl &tl = p.thl[seg];
@@ -357,6 +362,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int col = col0 + 32 * c + 8 * j;
+                        if (col >= cend) break;
                         const int h = fdiv(p.f_d, col), u = (col - h * p.d) >> 3;
                         uint8_t *hb = rbase + (long)h * p.blk[seg];
                         uint4 o;
@@ -407,6 +413,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                if (p.bias[seg]) {  // the 32 columns of this chunk: the same for every lane
+                    const uint4 *bp = reinterpret_cast<const uint4 *>(
+                        static_cast<const __nv_bfloat16 *>(p.bias[seg]) + col0 + 32 * c);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (col0 + 32 * c + 8 * j >= cend) break;
+                        const uint4 bv = __ldg(bp + j);
+                        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&bv);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(h[e]);
+                            v[8 * j + 2 * e] += f.x;
+                            v[8 * j + 2 * e + 1] += f.y;
+                        }
+                    }
+                }
+                if (p.act == ACT_GELU_TANH) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_fast(v[i]);
+                }
                 if (has_r) {
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -539,6 +565,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
     for (int i = 0; i < 3; ++i) {
         p.C[i] = i < a.nmat ? a.C[i] : nullptr;
         p.R[i] = i < a.nmat ? a.R[i] : nullptr;
+        p.bias[i] = i < a.nmat ? a.bias[i] : nullptr;
         if (i < a.nmat && a.thl[i]) {
             p.thl[i] = *a.thl[i];
             p.blk[i] = thl_block_bytes(a.d, a.thl[i]->vpad);
@@ -551,12 +578,13 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
             !encode_map_2d_bf16_sw(&mo.R[i], r, a.nseg, a.rows, (uint64_t)a.ldc * 2, 32, 32, 64))
             return cudaErrorNotSupported;
     }
+    p.act = a.act;
     p.ldc = a.ldc;
     p.rows = a.rows;
     p.nseg = a.nseg;
     p.nmat = a.nmat;
     p.n_tiles = (a.nseg + BN - 1) / BN;
-    p.kblocks = a.K / BK;
+    p.kblocks = (a.K + BK - 1) / BK;  // a last partial K block reads zeros past K
     const int m_tiles = (a.rows + 2 * BMC - 1) / (2 * BMC);
     p.tiles = m_tiles * a.nmat * p.n_tiles;
     p.status = device_status_ptr();
@@ -597,14 +625,19 @@ bool gemm_tc2_supported(const GemmArgs &a) {
     if (a.dtype != DT_BF16 || a.nmat < 1 || a.nmat > 3) return false;
     // rows past the end (a matrix shorter than a tile) read as zeros through the
     // tensor map and are never written
-    if (a.K < BK || a.K % BK || a.rows < 1 || a.lda % 8 || a.ldc % 8) return false;
-    if (a.nseg % 64) return false;  // tile widths: multiples of 32 per CTA half and epilogue chunk
+    // K: whole 16-byte rows for the tensor maps (a last partial K block reads
+    // zeros); nseg: tile widths N with N % 16 == 0 (N / 2 weight rows per CTA)
+    if (a.K < 8 || a.K % 8 || a.rows < 1 || a.lda % 8 || a.ldc % 8) return false;
+    if (a.nseg < 16 || a.nseg % 16) return false;
     if ((uintptr_t)a.A % 16) return false;
     for (int i = 0; i < a.nmat; ++i) {
-        if ((uintptr_t)a.W[i] % 16 || (uintptr_t)a.C[i] % 16 || (uintptr_t)a.R[i] % 16)
+        if ((uintptr_t)a.W[i] % 16 || (uintptr_t)a.C[i] % 16 || (uintptr_t)a.R[i] % 16 ||
+            (uintptr_t)a.bias[i] % 16)
             return false;
-        // tiled head layout: whole 8-column units per head, no residual
-        if (a.thl[i] && (a.R[i] || a.d < 8 || a.d % 8 || a.heads * a.d != a.nseg)) return false;
+        // tiled head layout: whole 8-column units per head, no residual, bias or activation
+        if (a.thl[i] && (a.R[i] || a.bias[i] || a.act != ACT_NONE || a.d < 8 || a.d % 8 ||
+                         a.heads * a.d != a.nseg))
+            return false;
     }
     return true;
 }
@@ -612,7 +645,7 @@ bool gemm_tc2_supported(const GemmArgs &a) {
 int gemm_tc2_schedule(long rows, int nseg, int nmat, int pairs, int32_t *first, int32_t *tile,
                       int *tiles, int *scheduled) {
     constexpr int BN = 256;  // the tile width both launch variants use
-    if (rows < 1 || nseg < 64 || nseg % 64 || nmat < 1 || nmat > 3 || pairs < 1) return -1;
+    if (rows < 1 || nseg < 16 || nseg % 16 || nmat < 1 || nmat > 3 || pairs < 1) return -1;
     const long n_tiles = (nseg + BN - 1) / BN;
     const long all = (rows + 2 * BMC - 1) / (2 * BMC) * nmat * n_tiles;
     if (all > (1L << 30)) return -1;

@@ -6,10 +6,14 @@
 // Host code cannot use the array's name as a device address (on the host it
 // names a stand-in object), so the first call on each device, with that device
 // current, asks the runtime for the array's device address with
-// cudaGetSymbolAddress and keeps it; later calls on that device reuse it.
-// That first call may load this file's device code, so make it before any
-// stream capture begins.  Nothing here allocates: the call hands the array to
+// cudaGetSymbolAddress and keeps it, together with the context that was
+// current; later calls on that device reuse it while the same context is
+// current, and look it up again in a new one (after cudaDeviceReset the
+// module, and with it the array, may sit at another address).  That first
+// call may load this file's device code, so make it before any stream capture
+// begins.  Nothing here allocates: the call hands the array to
 // ptdit_window_attn as its workspace.
+#include <cuda.h>
 #include <mutex>
 #include <stdio.h>
 
@@ -33,6 +37,26 @@ __device__ __align__(256) unsigned char g_scratch[PTDIT_STATIC_SCRATCH_BYTES];
 
 std::mutex g_mu;
 void *g_addr[kMaxDevices] = {};
+CUcontext g_ctx[kMaxDevices] = {};
+
+// The driver's cuCtxGetCurrent, reached through the runtime (no -lcuda).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CUcontext current_context() {
+    static CtxGetCurrentFn fn = nullptr;
+    static bool looked = false;
+    if (!looked) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        looked = true;
+    }
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
 
 int scratch_address(void **out) {
     int dev = 0;
@@ -45,7 +69,8 @@ int scratch_address(void **out) {
     if (dev < 0 || dev >= kMaxDevices)
         return ptdit::report_error(PTDIT_ERR_CUDA, "device ordinal above 63");
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
+    const CUcontext ctx = current_context();
+    if (!g_addr[dev] || !ctx || ctx != g_ctx[dev]) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_scratch);
         if (e != cudaSuccess || !p) {
@@ -55,6 +80,7 @@ int scratch_address(void **out) {
             return ptdit::report_error(PTDIT_ERR_CUDA, msg);
         }
         g_addr[dev] = p;
+        g_ctx[dev] = ctx;
     }
     *out = g_addr[dev];
     return PTDIT_OK;

@@ -138,7 +138,72 @@ cudaError_t launch_avg(const ProxyGeom &g, int B, int D, const void *z, void *ou
                       static_cast<const T *>(z), static_cast<T *>(out), g, D, CHT, G);
 }
 
+template <typename T, int VEC>
+struct Vec {
+    using type = T;
+};
+template <>
+struct Vec<__nv_bfloat16, 8> {
+    using type = uint4;
+};
+template <>
+struct Vec<float, 4> {
+    using type = float4;
+};
+
+// Single-token proxies: out[b, m] = z[b, member slot(b, m) of window m], with
+// slot 0 (the window's first token in (t, y, x) order: its top-left token in
+// its first frame) when `slots` is null.  One warp per proxy row, 16-byte
+// copies; a slot outside [0, P) leaves the row zero and records
+// PTDIT_ERR_SHAPE in the status word.
+template <typename T, int VEC>
+__global__ void __launch_bounds__(256) proxy_select_kernel(const T *__restrict__ z,
+                                                           T *__restrict__ out, ProxyGeom g,
+                                                           int B, int D,
+                                                           const int32_t *__restrict__ slots,
+                                                           int *status) {
+    pdl_wait();
+    pdl_trigger();
+    const long row = (long)blockIdx.x * 8 + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= (long)B * g.M) return;
+    const int m = static_cast<int>(row % g.M);
+    const long b = row / g.M;
+    const int slot = slots ? slots[row] : 0;
+    const bool ok = slot >= 0 && slot < g.P;
+    if (!ok && lane == 0) atomicExch(status, 2 /* PTDIT_ERR_SHAPE */);
+    const long N = (long)g.f * g.h * g.w;
+    const T *src = z + (b * N + (ok ? proxy_token(g, m, slot) : 0)) * D;
+    T *dst = out + row * D;
+    using V = typename Vec<T, VEC>::type;
+    const V *vs = reinterpret_cast<const V *>(src);
+    V *vd = reinterpret_cast<V *>(dst);
+    const int CH = D / VEC;
+    for (int c = lane; c < CH; c += 32) vd[c] = ok ? vs[c] : V{};
+}
+
+template <typename T, int VEC>
+cudaError_t launch_select(const ProxyGeom &g, int B, int D, const void *z, void *out,
+                          const int32_t *slots, int *status, cudaStream_t s) {
+    const long rows = (long)B * g.M;
+    return launch_pdl(proxy_select_kernel<T, VEC>, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, s,
+                      static_cast<const T *>(z), static_cast<T *>(out), g, B, D, slots, status);
+}
+
 }  // namespace
+
+cudaError_t launch_proxy_select(int dtype, const ProxyGeom &g, int B, int D, const void *z,
+                                void *proxies, const int32_t *slots, int *status,
+                                cudaStream_t s) {
+    const bool aligned = ((uintptr_t)z % 16 == 0) && ((uintptr_t)proxies % 16 == 0);
+    if (dtype == DT_BF16) {
+        if (aligned && D % 8 == 0)
+            return launch_select<__nv_bfloat16, 8>(g, B, D, z, proxies, slots, status, s);
+        return launch_select<__nv_bfloat16, 1>(g, B, D, z, proxies, slots, status, s);
+    }
+    if (aligned && D % 4 == 0) return launch_select<float, 4>(g, B, D, z, proxies, slots, status, s);
+    return launch_select<float, 1>(g, B, D, z, proxies, slots, status, s);
+}
 
 cudaError_t launch_proxy_average(int dtype, const ProxyGeom &g, int B, int D, const void *z,
                                  void *proxies, cudaStream_t s) {

@@ -28,28 +28,29 @@
 namespace ptdit {
 cudaError_t launch_gemm_simt(const GemmArgs &a, cudaStream_t s);
 cudaError_t launch_attention_simt(const AttnArgs &a, cudaStream_t s);
-bool gemm_tc_supported(const GemmArgs &a);
-cudaError_t launch_gemm_tc(const GemmArgs &a, cudaStream_t s);
 bool gemm_tc2_supported(const GemmArgs &a);
 cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s);
 bool attention_tc_supported(const AttnArgs &a);
 bool attention_thl_supported(const AttnArgs &a);
 cudaError_t launch_attention_tc(const AttnArgs &a, cudaStream_t s);
 
+// bf16 projections run on the tensor cores (2-SM kernel); fp32 projections are
+// the CUDA-core FMA path.  A bf16 shape the tensor-core kernel does not take
+// is refused by the API before anything is launched.
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s) {
-    if (gemm_tc2_supported(a)) {
-        const cudaError_t e = launch_gemm_tc2(a, s);
-        if (e != cudaErrorNotSupported) return e;
-        (void)cudaGetLastError();  // tensor maps refused: the kernels below
-    }
+    if (a.dtype == DT_BF16)
+        return gemm_tc2_supported(a) ? launch_gemm_tc2(a, s) : cudaErrorNotSupported;
     for (int i = 0; i < a.nmat; ++i)  // only the 2-SM kernel writes tiled head layout
         if (a.thl[i]) return cudaErrorNotSupported;
-    if (gemm_tc_supported(a)) return launch_gemm_tc(a, s);
     return launch_gemm_simt(a, s);
 }
 
+// bf16 attention runs on the tensor cores (operands in tiled head layout);
+// fp32 attention is the CUDA-core FMA path.  A bf16 shape without a
+// tensor-core kernel is refused by the API before anything is launched.
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s) {
-    if (attention_tc_supported(a)) return launch_attention_tc(a, s);
+    if (a.dtype == DT_BF16)
+        return attention_tc_supported(a) ? launch_attention_tc(a, s) : cudaErrorNotSupported;
     return launch_attention_simt(a, s);
 }
 
@@ -219,11 +220,33 @@ bool overlap(const void *a, size_t na, const void *b, size_t nb) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Ws {
-    size_t P, Qp, Kp, Vp, Ap, Pp, Kc, Vc, Q, K, V, O, total;
+    size_t P, Qp, Kp, Vp, Ap, Pp, Kc, Vc, Q, K, V, O;
+    size_t Xn, H, Kt, Vt;  // the complete block only: norm output, MLP hidden, text K and V
+    size_t total;
 };
 
 // Whether the attention operands of this shape go through tiled head layout.
-bool thl_shape(const Dims &d) { return d.dtype == PTDIT_BF16 && d.d >= 64 && d.d <= 80 && d.d % 8 == 0; }
+bool thl_shape(const Dims &d) { return d.dtype == PTDIT_BF16 && d.d >= 8 && d.d <= 80 && d.d % 8 == 0; }
+
+// bf16 attention has tensor-core kernels for head widths 8 .. 80 in steps of 8
+// and windows of 16, 32, 64 or 128 tokens; other bf16 shapes are refused.
+int check_bf16_attention(const Dims &d, const WinGeom *wg = nullptr) {
+    if (d.dtype != PTDIT_BF16) return PTDIT_OK;
+    if (d.D % 16)
+        return fail(PTDIT_ERR_SHAPE,
+                    "bf16 projections take widths D that are multiples of 16 (tensor cores); "
+                    "D=%d has no bf16 kernel (PTDIT_F32 takes any width)", d.D);
+    if (!thl_shape(d))
+        return fail(PTDIT_ERR_SHAPE,
+                    "bf16 attention takes head widths 8..80 in steps of 8 (tensor cores); "
+                    "head width %d has no bf16 kernel (PTDIT_F32 takes any width)", d.d);
+    if (wg && wg->n != 16 && wg->n != 32 && wg->n != 64 && wg->n != 128)
+        return fail(PTDIT_ERR_SHAPE,
+                    "bf16 window attention takes windows of 16, 32, 64 or 128 tokens "
+                    "(tensor cores); a window of %d tokens has no bf16 kernel "
+                    "(PTDIT_F32 takes any window)", wg->n);
+    return PTDIT_OK;
+}
 
 // Bytes of `rows_pb` rows per batch item in tiled head layout.
 size_t thl_bytes(const Dims &d, long rows_pb, int vpad) {
@@ -231,7 +254,8 @@ size_t thl_bytes(const Dims &d, long rows_pb, int vpad) {
            thl_block_bytes(d.d, vpad);
 }
 
-Ws ws_layout(const Dims &d, long M) {
+// L, Dh: text tokens and MLP width of the complete block (0 for the attention path).
+Ws ws_layout(const Dims &d, long M, long Lt = 0, long Dh = 0) {
     Ws L;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -248,6 +272,14 @@ Ws ws_layout(const Dims &d, long M) {
     L.P = take(pm); L.Qp = take(mx(pm, pq)); L.Kp = take(mx(pm, pq)); L.Vp = take(mx(pm, pv));
     L.Ap = take(pm); L.Pp = take(pm); L.Kc = take(mx(pm, pq)); L.Vc = take(mx(pm, pv));
     L.Q = take(mx(tn, tq)); L.K = take(mx(tn, tq)); L.V = take(mx(tn, tv)); L.O = take(tn);
+    L.Xn = L.H = L.Kt = L.Vt = 0;
+    if (Dh > 0) {
+        const size_t tl = (size_t)d.B * Lt * d.D * d.elem;
+        L.Xn = take(mx(tn, pm));
+        L.H = take((size_t)d.B * d.N * Dh * d.elem);
+        L.Kt = take(mx(tl, t ? thl_bytes(d, Lt, 0) : 0));
+        L.Vt = take(mx(tl, t ? thl_bytes(d, Lt, 1) : 0));
+    }
     L.total = off;
     return L;
 }
@@ -286,8 +318,9 @@ bool thl_has_empty_rows(const ThlDesc &t) {
     return t.mode == THL_IDENTITY ? t.rows_pb % kThlRows != 0 : t.g.nwin % t.pack != 0;
 }
 
-int check_ws(const Dims &d, long M, const void *ws, size_t ws_bytes, Ws *L) {
-    *L = ws_layout(d, M);
+int check_ws(const Dims &d, long M, const void *ws, size_t ws_bytes, Ws *L, long Lt = 0,
+             long Dh = 0) {
+    *L = ws_layout(d, M, Lt, Dh);
     if (fault("workspace"))
         return fail(PTDIT_ERR_WORKSPACE, "workspace refused (PTDIT_FAULT=workspace)");
     if (!ws) return fail(PTDIT_ERR_NULL, "workspace is NULL");
@@ -311,6 +344,33 @@ struct Run {
     const Ws &L;
     char *at(size_t off) const { return ws + off; }
 };
+
+// C = act(A W^T + bias) + R for one weight matrix of nseg x K (row stride K);
+// A has row stride lda = K, C and R row stride ldc = nseg.
+int gemm_ex(const Run &r, int kind, const void *A, long rows, int K, int nseg, const void *W,
+            void *C, const void *R, const void *bias, int act, const char *what) {
+    GemmArgs g;
+    memset(&g, 0, sizeof g);
+    g.dtype = r.d.dtype;
+    g.A = A;
+    g.lda = K;
+    g.W[0] = W;
+    g.C[0] = C;
+    g.R[0] = R;
+    g.bias[0] = bias;
+    g.act = act;
+    g.ldc = nseg;
+    g.rows = (int)rows;
+    g.nseg = nseg;
+    g.K = K;
+    g.nmat = 1;
+    TRY(launch_fault(what));
+    timing_begin(kind, r.s);
+    cudaError_t e = launch_gemm(g, r.s);
+    timing_end(r.s);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
+}
 
 int gemm(const Run &r, int kind, const void *A, long rows, int nmat, const void *const W[3],
          void *const C[3], const void *const R[3], const char *what) {
@@ -414,18 +474,69 @@ int attention(const Run &r, int kind, AttnArgs a, const char *what) {
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
 }
 
+// The pre-norms of the complete block (null members: the attention path, no norm).
+struct NormSet {
+    const ptdit_norm_w *proxy, *cross, *wsa, *swsa, *text, *mlp;
+    float eps;
+};
 
-// GIIM: z_out = (z_in +) CS(z_in, SA(Average(z_in)) (+ P_a)).
-int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
-             const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z_out) {
-    const Dims &d = r.d;
-    const long BM = (long)d.B * pg.M, BN = (long)d.B * d.N;
-    TRY(launch_fault("proxy average"));
-    timing_begin(PTDIT_K_AVERAGE, r.s);
-    cudaError_t e = launch_proxy_average(d.dtype, pg, d.B, d.D, z_in, r.at(r.L.P), r.s);
+// y = LayerNorm(x) * gamma + beta over the model width, rows x D.
+int layer_norm(const Run &r, const ptdit_norm_w *nw, float eps, const void *x, long rows, void *y,
+               const char *what) {
+    TRY(launch_fault(what));
+    timing_begin(PTDIT_K_NORM, r.s);
+    cudaError_t e = launch_layer_norm(r.d.dtype, rows, r.d.D, x, nw->gamma, nw->beta, eps, y, r.s);
     timing_end(r.s);
     count_launch();
-    if (e != cudaSuccess) return cuda_fail(e, "proxy average");
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
+}
+
+
+// GIIM: z_out = (z_in +) CS(z_in, SA(Average(z_in)) (+ P_a)).
+// The proxy tokens P_a of every window: the mean (the method), or one member
+// of the window (the pages' Top-Left and Random ablation variants).
+int extract_proxies(const Dims &d, const ProxyGeom &pg, int mode, const int32_t *slots,
+                    const void *z, void *proxies, cudaStream_t s) {
+    TRY(launch_fault("proxy extraction"));
+    cudaError_t e;
+    timing_begin(PTDIT_K_AVERAGE, s);
+    if (mode == PTDIT_PROXY_MEAN) {
+        e = launch_proxy_average(d.dtype, pg, d.B, d.D, z, proxies, s);
+    } else {
+        int *status = device_status_ptr();
+        e = status ? launch_proxy_select(d.dtype, pg, d.B, d.D, z, proxies,
+                                         mode == PTDIT_PROXY_RANDOM ? slots : nullptr, status, s)
+                   : cudaErrorInvalidValue;
+    }
+    timing_end(s);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "proxy extraction");
+}
+
+int check_proxy_mode(int mode, const int32_t *slots) {
+    if (mode != PTDIT_PROXY_MEAN && mode != PTDIT_PROXY_FIRST && mode != PTDIT_PROXY_RANDOM)
+        return fail(PTDIT_ERR_SHAPE, "proxy mode %d is not MEAN, FIRST or RANDOM", mode);
+    if (mode == PTDIT_PROXY_RANDOM) {
+        if (!slots) return fail(PTDIT_ERR_NULL, "PTDIT_PROXY_RANDOM needs a slots array");
+        if ((uintptr_t)slots % 4) return fail(PTDIT_ERR_ALIGN, "slots is not 4-byte aligned");
+    }
+    return PTDIT_OK;
+}
+
+// With norms (the complete block): the proxy self-attention reads LN(P_a) and
+// adds P_a; the cross-attention's queries come from LN(z_in).
+int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
+             const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z_out,
+             int mode = PTDIT_PROXY_MEAN, const int32_t *slots = nullptr,
+             const NormSet *nm = nullptr) {
+    const Dims &d = r.d;
+    const long BM = (long)d.B * pg.M, BN = (long)d.B * d.N;
+    TRY(extract_proxies(d, pg, mode, slots, z_in, r.at(r.L.P), r.s));
+    const void *pin = r.at(r.L.P), *zq = z_in;
+    if (nm) {
+        TRY(layer_norm(r, nm->proxy, nm->eps, r.at(r.L.P), BM, r.at(r.L.Xn), "proxy norm"));
+        pin = r.at(r.L.Xn);
+    }
     AttnArgs pa;  // proxy self-attention
     memset(&pa, 0, sizeof pa);
     pa.mode = ATT_ROWS;
@@ -444,15 +555,15 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
         const void *W[3] = {psa->wq, psa->wk, psa->wv};
         void *C[3] = {r.at(r.L.Qp), r.at(r.L.Kp), r.at(r.L.Vp)};
         const ThlDesc *T[3] = {tiled ? &tp : nullptr, tiled ? &tp : nullptr, tiled ? &tpv : nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.P), BM, 3, W, C, T, r.at(r.L.Ap),
+        TRY(gemm_thl(r, PTDIT_K_GEMM, pin, BM, 3, W, C, T, r.at(r.L.Ap),
                      "proxy QKV projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_PROXY, pa, "proxy self-attention"));
     {
         const void *W[3] = {psa->wo, nullptr, nullptr};
         void *C[3] = {r.at(r.L.Pp), nullptr, nullptr};
-        const void *R[3] = {(flags & PTDIT_PROXY_RESIDUAL) ? r.at(r.L.P) : nullptr, nullptr,
-                            nullptr};
+        const void *R[3] = {(nm || (flags & PTDIT_PROXY_RESIDUAL)) ? r.at(r.L.P) : nullptr,
+                            nullptr, nullptr};
         TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.Ap), BM, 1, W, C, R, "proxy output projection"));
     }
     AttnArgs ca;  // cross-attention: latent queries, proxy keys and values
@@ -476,11 +587,15 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
         TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.Pp), BM, 2, W, C, T, r.at(r.L.Ap),
                      "proxy K/V projection"));
     }
+    if (nm) {
+        TRY(layer_norm(r, nm->cross, nm->eps, z_in, BN, r.at(r.L.Xn), "cross-attention norm"));
+        zq = r.at(r.L.Xn);
+    }
     {
         const void *W[3] = {cross->wq, nullptr, nullptr};
         void *C[3] = {r.at(r.L.Q), nullptr, nullptr};
         const ThlDesc *T[3] = {tiled ? &tn : nullptr, nullptr, nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 1, W, C, T, r.at(r.L.O), "latent Q projection"));
+        TRY(gemm_thl(r, PTDIT_K_GEMM, zq, BN, 1, W, C, T, r.at(r.L.O), "latent Q projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_CROSS, ca, "cross-attention"));
     {
@@ -492,11 +607,17 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
     return PTDIT_OK;
 }
 
-// One TCM branch: x_out = (x_in +) WSA_or_SWSA(x_in).  x_out may equal x_in.
+// One TCM branch: x_out = (x_in +) WSA_or_SWSA(x_in), or, with a norm (the
+// complete block), x_out = x_in + WSA_or_SWSA(LN(x_in)).  x_out may equal x_in.
 int run_window(const Run &r, const WinGeom &wg, const ptdit_attn_w *w, unsigned flags,
-               const void *x_in, void *x_out) {
+               const void *x_in, void *x_out, const ptdit_norm_w *nw = nullptr, float eps = 0.f) {
     const Dims &d = r.d;
     const long BN = (long)d.B * d.N;
+    const void *xa = x_in;
+    if (nw) {
+        TRY(layer_norm(r, nw, eps, x_in, BN, r.at(r.L.Xn), "window norm"));
+        xa = r.at(r.L.Xn);
+    }
     AttnArgs a;
     memset(&a, 0, sizeof a);
     a.mode = ATT_WINDOW;
@@ -516,7 +637,7 @@ int run_window(const Run &r, const WinGeom &wg, const ptdit_attn_w *w, unsigned 
         const void *W[3] = {w->wq, w->wk, w->wv};
         void *C[3] = {r.at(r.L.Q), r.at(r.L.K), r.at(r.L.V)};
         const ThlDesc *T[3] = {tiled ? &tw : nullptr, tiled ? &tw : nullptr, tiled ? &twv : nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, x_in, BN, 3, W, C, T, r.at(r.L.O), "window QKV projection"));
+        TRY(gemm_thl(r, PTDIT_K_GEMM, xa, BN, 3, W, C, T, r.at(r.L.O), "window QKV projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "window attention"));
     {
@@ -526,6 +647,60 @@ int run_window(const Run &r, const WinGeom &wg, const ptdit_attn_w *w, unsigned 
         TRY(gemm(r, PTDIT_K_GEMM, r.at(r.L.O), BN, 1, W, C, R, "window output projection"));
     }
     return PTDIT_OK;
+}
+
+// Text cross-attention of the complete block, in place on z:
+// z += MHA(LN(z) as queries, text tokens [B, Lt, D] as keys and values).
+int run_text(const Run &r, const ptdit_attn_w *w, const ptdit_norm_w *nw, float eps,
+             const void *text, int Lt, void *z) {
+    const Dims &d = r.d;
+    const long BN = (long)d.B * d.N, BL = (long)d.B * Lt;
+    TRY(layer_norm(r, nw, eps, z, BN, r.at(r.L.Xn), "text-attention norm"));
+    AttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.mode = ATT_ROWS;
+    a.dtype = d.dtype;
+    a.d = d.d;
+    a.q = r.at(r.L.Q); a.k = r.at(r.L.Kt); a.v = r.at(r.L.Vt); a.o = r.at(r.L.O);
+    a.q_bstride = d.N;
+    a.k_bstride = Lt;
+    a.nq = (int)d.N;
+    a.nk = Lt;
+    const bool tiled = attention_thl_supported(a);
+    const ThlDesc tn = thl_identity(d.N, 0), tt = thl_identity(Lt, 0),
+                  ttv = thl_identity(Lt, 1, v_ones(d));
+    if (tiled) {
+        a.tq = tn;
+        a.tk = tt;
+        a.tv = ttv;
+    }
+    {
+        const void *W[3] = {w->wk, w->wv, nullptr};
+        void *C[3] = {r.at(r.L.Kt), r.at(r.L.Vt), nullptr};
+        const ThlDesc *T[3] = {tiled ? &tt : nullptr, tiled ? &ttv : nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, text, BL, 2, W, C, T, r.at(r.L.O), "text K/V projection"));
+    }
+    {
+        const void *W[3] = {w->wq, nullptr, nullptr};
+        void *C[3] = {r.at(r.L.Q), nullptr, nullptr};
+        const ThlDesc *T[3] = {tiled ? &tn : nullptr, nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.Xn), BN, 1, W, C, T, r.at(r.L.O),
+                     "text-attention Q projection"));
+    }
+    TRY(attention(r, PTDIT_K_ATTN_TEXT, a, "text cross-attention"));
+    return gemm_ex(r, PTDIT_K_GEMM, r.at(r.L.O), BN, d.D, d.D, w->wo, z, z, nullptr, ACT_NONE,
+                   "text-attention output projection");
+}
+
+// MLP of the complete block, in place on z: z += fc2(GELU(fc1(LN(z)) + b1)) + b2.
+int run_mlp(const Run &r, const ptdit_block_w *w, float eps, void *z) {
+    const Dims &d = r.d;
+    const long BN = (long)d.B * d.N;
+    TRY(layer_norm(r, &w->norm_mlp, eps, z, BN, r.at(r.L.Xn), "MLP norm"));
+    TRY(gemm_ex(r, PTDIT_K_GEMM, r.at(r.L.Xn), BN, d.D, w->mlp_hidden, w->w1, r.at(r.L.H),
+                nullptr, w->b1, ACT_GELU_TANH, "MLP fc1"));
+    return gemm_ex(r, PTDIT_K_GEMM, r.at(r.L.H), BN, w->mlp_hidden, d.D, w->w2, z, z, w->b2,
+                   ACT_NONE, "MLP fc2");
 }
 
 int check_io(const Dims &d, const void *z_in, const void *z_out, const void *ws, size_t ws_bytes) {
@@ -660,6 +835,42 @@ int ptdit_proxy_average(const ptdit_shape *shape, const int ratio[3], const void
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "proxy average");
 }
 
+int ptdit_proxy_extract(const ptdit_shape *shape, const int ratio[3], int mode,
+                        const int32_t *slots, const void *z, void *proxies,
+                        ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    TRY(check_shape(shape, &d, false));
+    TRY(make_proxy(d, ratio, &pg));
+    TRY(check_proxy_mode(mode, slots));
+    TRY(check_ptr(z, "z"));
+    TRY(check_ptr(proxies, "proxies"));
+    if (overlap(z, (size_t)d.B * d.N * d.D * d.elem, proxies, (size_t)d.B * pg.M * d.D * d.elem))
+        return fail(PTDIT_ERR_ALIAS, "proxies overlap z");
+    return extract_proxies(d, pg, mode, slots, z, proxies, (cudaStream_t)stream);
+}
+
+int ptdit_giim_ex(const ptdit_shape *shape, const int ratio[3], int mode, const int32_t *slots,
+                  const ptdit_attn_w *psa, const ptdit_attn_w *cross, unsigned flags,
+                  const void *z_in, void *z_out, void *ws, size_t ws_bytes,
+                  ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    Ws L;
+    TRY(check_shape(shape, &d));
+    TRY(check_bf16_attention(d));
+    TRY(make_proxy(d, ratio, &pg));
+    TRY(check_proxy_mode(mode, slots));
+    TRY(check_weights(psa, "psa"));
+    TRY(check_weights(cross, "cross"));
+    TRY(check_io(d, z_in, z_out, ws, ws_bytes));
+    TRY(check_w_alias(d, psa, z_out));
+    TRY(check_w_alias(d, cross, z_out));
+    TRY(check_ws(d, pg.M, ws, ws_bytes, &L));
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    return run_giim(r, pg, psa, cross, flags, z_in, z_out, mode, slots);
+}
+
 int ptdit_giim(const ptdit_shape *shape, const int ratio[3], const ptdit_attn_w *psa,
                const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z_out,
                void *ws, size_t ws_bytes, ptdit_stream_t stream) {
@@ -667,6 +878,7 @@ int ptdit_giim(const ptdit_shape *shape, const int ratio[3], const ptdit_attn_w 
     ProxyGeom pg;
     Ws L;
     TRY(check_shape(shape, &d));
+    TRY(check_bf16_attention(d));
     TRY(make_proxy(d, ratio, &pg));
     TRY(check_weights(psa, "psa"));
     TRY(check_weights(cross, "cross"));
@@ -686,6 +898,7 @@ int ptdit_window_attn(const ptdit_shape *shape, const int window[3], const int s
     Ws L;
     TRY(check_shape(shape, &d));
     TRY(make_window(d, window, shift, &wg));
+    TRY(check_bf16_attention(d, &wg));
     TRY(check_weights(w, "w"));
     TRY(check_io(d, z_in, z_out, ws, ws_bytes));
     TRY(check_w_alias(d, w, z_out));
@@ -704,6 +917,7 @@ int ptdit_tcm(const ptdit_shape *shape, const int window[3], const int shift[3],
     TRY(check_shape(shape, &d));
     TRY(make_window(d, window, shift, &wg1));
     TRY(make_window(d, window, zero, &wg0));
+    TRY(check_bf16_attention(d, &wg0));
     TRY(check_weights(wsa, "wsa"));
     TRY(check_weights(swsa, "swsa"));
     TRY(check_io(d, z_in, z_out, ws, ws_bytes));
@@ -729,6 +943,7 @@ int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int win
     TRY(make_proxy(d, ratio, &pg));
     TRY(make_window(d, window, shift, &wg1));
     TRY(make_window(d, window, zero, &wg0));
+    TRY(check_bf16_attention(d, &wg0));
     TRY(check_weights(psa, "psa"));
     TRY(check_weights(cross, "cross"));
     TRY(check_weights(wsa, "wsa"));
@@ -745,12 +960,84 @@ int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int win
     return run_window(r, wg1, swsa, flags, z_out, z_out);
 }
 
+size_t ptdit_pt_block_workspace_bytes(const ptdit_shape *shape, const int ratio[3],
+                                      int text_len, int mlp_hidden) {
+    Dims d;
+    ProxyGeom pg;
+    if (check_shape(shape, &d) != PTDIT_OK || text_len < 1 || mlp_hidden < 1) return 0;
+    if (make_proxy(d, ratio, &pg) != PTDIT_OK) return 0;
+    return ws_layout(d, pg.M, text_len, mlp_hidden).total;
+}
+
+int ptdit_pt_block(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                   const int shift[3], const ptdit_block_w *w, const void *text, int text_len,
+                   int proxy_mode, const int32_t *slots, const void *z_in, void *z_out, void *ws,
+                   size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    WinGeom wg0, wg1;
+    Ws L;
+    const int zero[3] = {0, 0, 0};
+    TRY(check_shape(shape, &d));
+    TRY(make_proxy(d, ratio, &pg));
+    TRY(make_window(d, window, shift, &wg1));
+    TRY(make_window(d, window, zero, &wg0));
+    TRY(check_bf16_attention(d, &wg0));
+    TRY(check_proxy_mode(proxy_mode, slots));
+    if (!w) return fail(PTDIT_ERR_NULL, "block weights are NULL");
+    const ptdit_attn_w *mods[5] = {&w->psa, &w->cross, &w->wsa, &w->swsa, &w->text};
+    const char *names[5] = {"psa", "cross", "wsa", "swsa", "text"};
+    for (int i = 0; i < 5; ++i) {
+        TRY(check_weights(mods[i], names[i]));
+        TRY(check_w_alias(d, mods[i], z_out));
+    }
+    const ptdit_norm_w *norms[6] = {&w->norm_proxy, &w->norm_cross, &w->norm_wsa,
+                                    &w->norm_swsa, &w->norm_text, &w->norm_mlp};
+    const size_t zb = (size_t)d.B * d.N * d.D * d.elem, vb = (size_t)d.D * d.elem;
+    for (int i = 0; i < 6; ++i) {
+        TRY(check_ptr(norms[i]->gamma, "norm gamma"));
+        TRY(check_ptr(norms[i]->beta, "norm beta"));
+        if (overlap(norms[i]->gamma, vb, z_out, zb) || overlap(norms[i]->beta, vb, z_out, zb))
+            return fail(PTDIT_ERR_ALIAS, "z_out overlaps a norm parameter");
+    }
+    if (w->mlp_hidden < 1) return fail(PTDIT_ERR_SHAPE, "mlp_hidden %d < 1", w->mlp_hidden);
+    if (d.dtype == PTDIT_BF16 && w->mlp_hidden % 16)
+        return fail(PTDIT_ERR_SHAPE, "bf16 MLP widths must be multiples of 16 (mlp_hidden=%d)",
+                    w->mlp_hidden);
+    if (!(w->eps > 0.f) || w->eps > 1.f)
+        return fail(PTDIT_ERR_SHAPE, "eps must be in (0, 1]");
+    const size_t hb = (size_t)w->mlp_hidden * d.D * d.elem, bh = (size_t)w->mlp_hidden * d.elem;
+    TRY(check_ptr(w->w1, "w1"));
+    TRY(check_ptr(w->b1, "b1"));
+    TRY(check_ptr(w->w2, "w2"));
+    TRY(check_ptr(w->b2, "b2"));
+    if (overlap(w->w1, hb, z_out, zb) || overlap(w->w2, hb, z_out, zb) ||
+        overlap(w->b1, bh, z_out, zb) || overlap(w->b2, vb, z_out, zb))
+        return fail(PTDIT_ERR_ALIAS, "z_out overlaps an MLP weight");
+    if (text_len < 1) return fail(PTDIT_ERR_SHAPE, "text_len %d < 1", text_len);
+    TRY(check_ptr(text, "text"));
+    if (overlap(text, (size_t)d.B * text_len * d.D * d.elem, z_out, zb))
+        return fail(PTDIT_ERR_ALIAS, "z_out overlaps the text tokens");
+    TRY(check_io(d, z_in, z_out, ws, ws_bytes));
+    TRY(check_ws(d, pg.M, ws, ws_bytes, &L, text_len, w->mlp_hidden));
+    if (ws && overlap(ws, ws_bytes, text, (size_t)d.B * text_len * d.D * d.elem))
+        return fail(PTDIT_ERR_ALIAS, "the text tokens overlap the workspace");
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    const NormSet nm{norms[0], norms[1], norms[2], norms[3], norms[4], norms[5], w->eps};
+    TRY(run_giim(r, pg, &w->psa, &w->cross, 0, z_in, z_out, proxy_mode, slots, &nm));
+    TRY(run_window(r, wg0, &w->wsa, 0, z_out, z_out, nm.wsa, nm.eps));
+    TRY(run_window(r, wg1, &w->swsa, 0, z_out, z_out, nm.swsa, nm.eps));
+    TRY(run_text(r, &w->text, nm.text, nm.eps, text, text_len, z_out));
+    return run_mlp(r, w, nm.eps, z_out);
+}
+
 int ptdit_full_attn(const ptdit_shape *shape, const ptdit_attn_w *w, unsigned flags,
                     const void *z_in, void *z_out, void *ws, size_t ws_bytes,
                     ptdit_stream_t stream) {
     Dims d;
     Ws L;
     TRY(check_shape(shape, &d));
+    TRY(check_bf16_attention(d));
     TRY(check_weights(w, "w"));
     TRY(check_io(d, z_in, z_out, ws, ws_bytes));
     TRY(check_w_alias(d, w, z_out));

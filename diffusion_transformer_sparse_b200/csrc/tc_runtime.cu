@@ -92,6 +92,16 @@ bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows
     return r == CUDA_SUCCESS;
 }
 
+namespace {
+thread_local unsigned long long g_wait_limit_ns = 0;
+}
+
+unsigned long long debug_wait_limit_ns() {
+    return g_wait_limit_ns ? g_wait_limit_ns : tc::kWaitLimitNs;
+}
+
+void set_debug_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns = ns; }
+
 int num_sms() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;

@@ -85,6 +85,36 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// mbar_wait for code where all 32 lanes of the warp wait together and a
+// warp-collective instruction (tcgen05.ld/st .sync.aligned, a ballot) follows:
+// the decision to give up is taken by the whole warp, so no lane can leave
+// while another keeps waiting.  The first try is a plain try_wait (a complete
+// phase stays complete until this warp itself arrives on the barrier, so lanes
+// that see it late see it on their next try); only the slow path votes.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                               int *status, uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned active = __activemask();
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        bool got = false;
+#pragma unroll 1
+        for (int i = 0; i < 32 && !got; ++i) got = mbar_try_wait(bar, parity);
+        const unsigned seen = __ballot_sync(active, got);
+        if (seen == active) return true;
+        if (seen != 0) continue;  // the phase is complete: the other lanes see it next time
+        const bool quit = *abort || globaltimer() - t0 > limit_ns;
+        if (__any_sync(active, quit)) {
+            if ((active & -active) == (1u << (threadIdx.x & 31)) && !*abort) {
+                *abort = 1;
+                atomicExch(status, 6 /* PTDIT_ERR_TIMEOUT */);
+            }
+            __syncwarp(active);
+            return false;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
                                             int x, int y) {
@@ -423,6 +453,10 @@ bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows
                                uint32_t box_rows, int swizzle_bytes);
 
 int num_sms();
+
+// Limit of the window kernel's waits for work on this host thread: kWaitLimitNs
+// unless ptdit_debug_wait_limit set a shorter one.
+unsigned long long debug_wait_limit_ns();
 
 
 

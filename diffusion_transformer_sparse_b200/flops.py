@@ -44,3 +44,17 @@ def core_ratio(N: int, M: int, n: int) -> float:
 def average_bytes(N: int, M: int, D: int, elem: int) -> int:
     """Window averaging: read every token once, write every proxy once."""
     return (N + M) * D * elem
+
+
+def pt_block_flops(N: int, M: int, n: int, D: int, L: int, Dh: int) -> dict:
+    """The complete PT-Block: the attention path plus the text cross-attention
+    (projections 4 N D^2 + 4 L D^2, core 4 N L D) and the MLP (4 N D Dh).
+    Norms, bias adds and the GELU are not counted."""
+    f = block_flops(N, M, n, D)
+    f["text_proj"] = 4 * N * D * D + 4 * L * D * D
+    f["text_core"] = 4 * N * L * D
+    f["mlp"] = 4 * N * D * Dh
+    f["proj"] += f["text_proj"] + f["mlp"]
+    f["core"] += f["text_core"]
+    f["total"] = f["proj"] + f["core"]
+    return f

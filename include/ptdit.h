@@ -94,6 +94,36 @@ int ptdit_proxy_average(const ptdit_shape *shape, const int ratio[3], const void
                         void *proxies, ptdit_stream_t stream);
 
 /*
+ * Proxy extraction modes (Qihoo-T2X reading note, code-comparison section,
+ * get_proxy_token(mode=...), and the proxy-extraction ablation of §3 Method:
+ * Average / Top-Left / Random).
+ *   PTDIT_PROXY_MEAN    the window mean (Eq. GIIM; the method's choice)
+ *   PTDIT_PROXY_FIRST   the window's first token in (t, y, x) order: its
+ *                       top-left token in its first frame
+ *   PTDIT_PROXY_RANDOM  the window member the caller's slots array names:
+ *                       slots is a DEVICE int32 array [B * M] (batch item
+ *                       major), slots[b*M + m] in [0, p_f p_h p_w) counting
+ *                       the window's members row-major over (t, y, x).  The
+ *                       random draw is the caller's; a slot outside the range
+ *                       leaves that proxy zero and records PTDIT_ERR_SHAPE in
+ *                       the device status word (ptdit_device_status).
+ */
+#define PTDIT_PROXY_MEAN   0
+#define PTDIT_PROXY_FIRST  1
+#define PTDIT_PROXY_RANDOM 2
+
+/*
+ * ptdit_proxy_extract -- the proxy tokens under any of the three modes.
+ *   mode PTDIT_PROXY_MEAN is ptdit_proxy_average.  Single-token modes copy
+ *   their token bit for bit.  slots: see PTDIT_PROXY_RANDOM (NULL otherwise;
+ *   ignored).  Errors as ptdit_proxy_average, plus PTDIT_ERR_SHAPE for an
+ *   unknown mode and PTDIT_ERR_NULL for RANDOM without slots.
+ */
+int ptdit_proxy_extract(const ptdit_shape *shape, const int ratio[3], int mode,
+                        const int32_t *slots, const void *z, void *proxies,
+                        ptdit_stream_t stream);
+
+/*
  * ptdit_workspace_bytes -- device scratch that every call below needs for
  * this shape (the maximum over them), or 0 for an invalid shape.  The
  * workspace must be 256-byte aligned; its contents need no initialisation
@@ -109,6 +139,15 @@ size_t ptdit_workspace_bytes(const ptdit_shape *shape, const int ratio[3], const
 int ptdit_giim(const ptdit_shape *shape, const int ratio[3], const ptdit_attn_w *psa,
                const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z_out,
                void *ws, size_t ws_bytes, ptdit_stream_t stream);
+
+/*
+ * ptdit_giim_ex -- ptdit_giim with the proxy tokens extracted by `mode`
+ *   (and `slots`, for PTDIT_PROXY_RANDOM) instead of the window mean.
+ */
+int ptdit_giim_ex(const ptdit_shape *shape, const int ratio[3], int mode, const int32_t *slots,
+                  const ptdit_attn_w *psa, const ptdit_attn_w *cross, unsigned flags,
+                  const void *z_in, void *z_out, void *ws, size_t ws_bytes,
+                  ptdit_stream_t stream);
 
 /*
  * ptdit_window_attn -- one TCM branch (Eq. TCM): z_out = z_in + WSA(z_in)
@@ -161,6 +200,57 @@ int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int win
                      const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
                      const void *z_in, void *z_out, void *ws, size_t ws_bytes,
                      ptdit_stream_t stream);
+
+/*
+ * The complete PT-Block (Qihoo-T2X reading note, §3 Method: "PT-Block (GIIM +
+ * TCM + text cross-attn + MLP)" and the block diagram; code-comparison
+ * section, ProxyTokensTransformerBlock.forward).  Every sub-layer is pre-norm
+ * with a residual (the pages name the sub-layers and their order; the norm
+ * form, the MLP's activation and the position of each norm are this library's
+ * reading, stated here):
+ *   P_a = proxies of z (proxy_mode)      P' = P_a + SA(LN_proxy(P_a))
+ *   z1 = z  + CS(LN_cross(z), P')        z2 = z1 + WSA(LN_wsa(z1))
+ *   z3 = z2 + SWSA(LN_swsa(z2))          z4 = z3 + MHA(LN_text(z3), text)
+ *   z_out = z4 + fc2(GELU(fc1(LN_mlp(z4))))
+ * LN(x) = (x - mean) / sqrt(var + eps) * gamma + beta over the D channels of
+ * a token (var: mean squared deviation); GELU in its tanh form; fc1 = x W1^T
+ * + b1 (W1 [mlp_hidden][D]), fc2 = h W2^T + b2 (W2 [D][mlp_hidden]).  The
+ * attention projections have no bias.  The text tokens are [B, text_len, D]
+ * (already projected to the model width), keys and values of the text
+ * cross-attention.  All parameters are DEVICE arrays of the call's dtype,
+ * 16-byte aligned.
+ */
+typedef struct {
+    const void *gamma, *beta;  /* [D] each */
+} ptdit_norm_w;
+
+typedef struct {
+    ptdit_attn_w psa, cross, wsa, swsa, text;
+    ptdit_norm_w norm_proxy, norm_cross, norm_wsa, norm_swsa, norm_text, norm_mlp;
+    const void *w1, *b1;  /* [mlp_hidden][D], [mlp_hidden] */
+    const void *w2, *b2;  /* [D][mlp_hidden], [D] */
+    int mlp_hidden;       /* width of the MLP's hidden layer (4 D in DiT-style blocks) */
+    float eps;            /* LayerNorm epsilon, in (0, 1] (1e-6 in DiT-style blocks) */
+} ptdit_block_w;
+
+/*
+ * ptdit_pt_block_workspace_bytes -- workspace of ptdit_pt_block for this
+ *   shape, ratio, text length and MLP width (0 for invalid arguments).
+ */
+size_t ptdit_pt_block_workspace_bytes(const ptdit_shape *shape, const int ratio[3],
+                                      int text_len, int mlp_hidden);
+
+/*
+ * ptdit_pt_block -- one complete PT-Block (above).  proxy_mode / slots as in
+ *   ptdit_giim_ex (PTDIT_PROXY_MEAN is the method).  z_out must not overlap
+ *   z_in, any parameter, the text tokens or the workspace.  Errors as
+ *   ptdit_block_attn, plus PTDIT_ERR_SHAPE for text_len < 1, mlp_hidden < 1
+ *   or eps outside (0, 1].
+ */
+int ptdit_pt_block(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                   const int shift[3], const ptdit_block_w *w, const void *text, int text_len,
+                   int proxy_mode, const int32_t *slots, const void *z_in, void *z_out, void *ws,
+                   size_t ws_bytes, ptdit_stream_t stream);
 
 /*
  * ptdit_full_attn -- the dense comparator the pages measure against
@@ -246,7 +336,9 @@ enum {
     PTDIT_K_ATTN_CROSS = 3,/* latent -> proxy cross-attention core */
     PTDIT_K_ATTN_WINDOW = 4,/* window / shifted-window attention core */
     PTDIT_K_ATTN_DENSE = 5,/* full self-attention core */
-    PTDIT_K_COUNT = 6
+    PTDIT_K_NORM = 6,      /* LayerNorm of the complete block */
+    PTDIT_K_ATTN_TEXT = 7, /* text cross-attention core of the complete block */
+    PTDIT_K_COUNT = 8
 };
 int ptdit_timing_enable(int max_launches);
 int ptdit_timing_read(int *kind, float *ms, int max);
@@ -274,6 +366,20 @@ int ptdit_device_status(int reset);
  *   PTDIT_ERR_CUDA.
  */
 int ptdit_debug_timeout(long long limit_ns, ptdit_stream_t stream);
+
+/*
+ * ptdit_debug_wait_limit -- sets, for this host thread's later launches of
+ *   the window-attention kernel (ptdit_window_attn, ptdit_tcm,
+ *   ptdit_block_attn and ptdit_window_attn_static), the limit of every
+ *   device-side wait for work to limit_ns nanoseconds; 0 restores the default
+ *   (2 s).  A limit shorter than the work makes those waits give up: the
+ *   kernel records PTDIT_ERR_TIMEOUT in the device status word, waits (2 s at
+ *   most) for the tensor-core work it issued, and returns with its output
+ *   incomplete; the context stays usable.  The paper has no counterpart: it
+ *   lets tests exercise the give-up path of a real kernel.  Errors:
+ *   PTDIT_ERR_SHAPE (limit_ns < 0 or above 10 s).
+ */
+int ptdit_debug_wait_limit(long long limit_ns);
 
 /*
  * Host-side fault injection for tests: with the environment variable

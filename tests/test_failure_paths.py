@@ -72,6 +72,33 @@ def test_bounded_wait_gives_up_and_reports_timeout():
 
 
 @pytest.mark.gpu
+def test_window_kernel_gives_up_as_whole_warps():
+    """The window-attention kernel with a 1 ns limit on its waits for work: the
+    waits give up (the loader and softmax warps decide per warp, so no lane is
+    left behind at a warp-collective TMEM access), the kernel records
+    PTDIT_ERR_TIMEOUT and returns, and the next regular call matches the oracle."""
+    import torch
+    import oracle as O
+    from tests.helpers import Case, rel_err, TOL
+    pt.lib()
+    grid, window, shift = (1, 64, 64), (1, 8, 8), (0, 4, 4)
+    c = Case(1, grid, 1152, 16, "bf16")
+    pt.ptdit_device_status(reset=True)
+    pt.ptdit_debug_wait_limit(1)
+    try:
+        pt.ptdit_window_attn(c.z, grid, window, shift, c.w["swsa"], 16)
+        torch.cuda.synchronize()
+    finally:
+        pt.ptdit_debug_wait_limit(0)
+    assert pt.ptdit_device_status(reset=True) == pt.PTDIT_ERR_TIMEOUT
+    assert pt.ptdit_device_status() == pt.PTDIT_OK
+    out = c.out64(pt.ptdit_window_attn(c.z, grid, window, shift, c.w["swsa"], 16))
+    want = O.window_self_attention(c.z64[0], grid, window, shift, c.w64["swsa"], 16)
+    assert rel_err(out[0], want) <= TOL["bf16"]
+    assert pt.ptdit_device_status() == pt.PTDIT_OK
+
+
+@pytest.mark.gpu
 def test_injected_launch_fault_launches_nothing():
     code = """
         import torch
@@ -95,3 +122,6 @@ def test_timeout_limit_is_validated():
     pt.lib()
     assert pt.lib().ptdit_debug_timeout(0, None) == pt.PTDIT_ERR_SHAPE
     assert pt.lib().ptdit_debug_timeout(20_000_000_000, None) == pt.PTDIT_ERR_SHAPE
+    assert pt.lib().ptdit_debug_wait_limit(-1) == pt.PTDIT_ERR_SHAPE
+    assert pt.lib().ptdit_debug_wait_limit(20_000_000_000) == pt.PTDIT_ERR_SHAPE
+    assert pt.lib().ptdit_debug_wait_limit(0) == pt.PTDIT_OK
