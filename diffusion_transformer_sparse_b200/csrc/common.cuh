@@ -158,6 +158,9 @@ cudaError_t launch_proxy_select(int dtype, const ProxyGeom &g, int B, int D, con
 // Device address of the library's status word on the current device.
 int *device_status_ptr();
 
+// SMs of the current device (0 if it cannot be read).
+int num_sms();
+
 // Tile geometry of an operand stored in tiled head layout (thl.cuh).
 struct ThlDesc {
     int mode;      // 0: plain row-major; 1: identity tiles; 2: window tiles

@@ -37,6 +37,8 @@
 // Two TMEM accumulators overlap the next tile's MMAs with this tile's
 // epilogue.  Every wait is bounded (2 s); a timeout records
 // PTDIT_ERR_TIMEOUT in the status word.
+#include <stdlib.h>
+
 #include <algorithm>
 #include <map>
 #include <mutex>
@@ -89,13 +91,13 @@ struct Tc2Params {
 
 // STAGING: the row-major epilogue's staging tiles exist (launches whose outputs
 // are all in tiled head layout leave them out and use the room for stages).
-template <int BN, int STAGES, bool STAGING>
+template <int BN, int STAGES, bool STAGING, int SCH>
 struct Layout2 {
     static constexpr int A_BYTES = BMC * BK * 2;       // 16 KB: this CTA's rows of A
     static constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's half of the weight tile
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int CHUNK_BYTES = 32 * 64;          // 32 rows x 32 bf16 columns
-    static constexpr int WARP_STAGE = STAGING ? (BN / 32) * CHUNK_BYTES : 0;
+    static constexpr int WARP_STAGE = STAGING ? SCH * CHUNK_BYTES : 0;  // SCH chunks per pass
     static constexpr int EPI_OFF = STAGES * STAGE_BYTES;  // 4 epilogue warps' staging tiles
     static constexpr int BAR_OFF = EPI_OFF + 4 * WARP_STAGE;
     static constexpr int NBARS = 2 * STAGES + 9;  // full, empty, tfull[2], tempty[2], rfull[4], drain
@@ -190,13 +192,13 @@ __device__ __forceinline__ int tile_width(const Tc2Params &p, int n_tile) {
     return w < BN ? w : BN;
 }
 
-template <int BN, int STAGES, bool STAGING>
+template <int BN, int STAGES, bool STAGING, int SCH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB0,
                     const __grid_constant__ CUtensorMap mB1,
                     const __grid_constant__ CUtensorMap mB2, const __grid_constant__ Tc2Maps mo,
                     const __grid_constant__ Tc2Params p) {
-    using L = Layout2<BN, STAGES, STAGING>;
+    using L = Layout2<BN, STAGES, STAGING, SCH>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -386,86 +388,94 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             if (!STAGING) break;  // not launched with row-major outputs
             const bool has_r = p.R[seg] != nullptr;
-            if (lane == 0) {
-                bulk_wait_read_all();  // the previous tile's stores have left the staging tile
-                if (has_r) {
-                    mbar_expect_tx(&rfull[q], nchunk * L::CHUNK_BYTES);
-#pragma unroll 1
-                    for (int c = 0; c < nchunk; ++c)
-                        tma_load_2d(stg + c * L::CHUNK_BYTES, &mo.R[seg], &rfull[q], col0 + 32 * c,
-                                    row0);
-                }
-            }
-            __syncwarp();
-            if (!mbar_wait(&tfull[acc], acc_phase, abort, p.status)) break;
-            if (has_r) {
-                if (!mbar_wait(&rfull[q], r_phase, abort, p.status)) break;
-                r_phase ^= 1;
-            }
-            fence_after_sync();
             const uint32_t tbase = tmem + acc * L::ACC_STRIDE + (static_cast<uint32_t>(q * 32) << 16);
+            bool ok = true;
+            // the tile's chunks in passes of SCH through the warp's staging tiles
 #pragma unroll 1
-            for (int c = 0; c < nchunk; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tbase + 32 * c, r);
-                tmem_ld_wait();
-                uint8_t *chunk = stg + c * L::CHUNK_BYTES + row_off;
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-                if (p.bias[seg]) {  // the 32 columns of this chunk: the same for every lane
-                    const uint4 *bp = reinterpret_cast<const uint4 *>(
-                        static_cast<const __nv_bfloat16 *>(p.bias[seg]) + col0 + 32 * c);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (col0 + 32 * c + 8 * j >= cend) break;
-                        const uint4 bv = __ldg(bp + j);
-                        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&bv);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(h[e]);
-                            v[8 * j + 2 * e] += f.x;
-                            v[8 * j + 2 * e + 1] += f.y;
-                        }
+            for (int c0 = 0; c0 < nchunk && ok; c0 += SCH) {
+                const int c1 = c0 + SCH < nchunk ? c0 + SCH : nchunk;
+                if (lane == 0) {
+                    bulk_wait_read_all();  // the previous pass's stores have left the staging tiles
+                    if (has_r) {
+                        mbar_expect_tx(&rfull[q], (c1 - c0) * L::CHUNK_BYTES);
+#pragma unroll 1
+                        for (int c = c0; c < c1; ++c)
+                            tma_load_2d(stg + (c - c0) * L::CHUNK_BYTES, &mo.R[seg], &rfull[q],
+                                        col0 + 32 * c, row0);
                     }
                 }
-                if (p.act == ACT_GELU_TANH) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_fast(v[i]);
-                }
+                __syncwarp();
+                if (c0 == 0 && !mbar_wait(&tfull[acc], acc_phase, abort, p.status)) { ok = false; break; }
                 if (has_r) {
+                    if (!mbar_wait(&rfull[q], r_phase, abort, p.status)) { ok = false; break; }
+                    r_phase ^= 1;
+                }
+                fence_after_sync();
+#pragma unroll 1
+                for (int c = c0; c < c1; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + 32 * c, r);
+                    tmem_ld_wait();
+                    uint8_t *chunk = stg + (c - c0) * L::CHUNK_BYTES + row_off;
+                    float v[32];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint4 rv = *reinterpret_cast<const uint4 *>(chunk + ((j ^ sw) << 4));
-                        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&rv);
+                    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                    if (p.bias[seg]) {  // the 32 columns of this chunk: the same for every lane
+                        const uint4 *bp = reinterpret_cast<const uint4 *>(
+                            static_cast<const __nv_bfloat16 *>(p.bias[seg]) + col0 + 32 * c);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(h[e]);
-                            v[8 * j + 2 * e] += f.x;
-                            v[8 * j + 2 * e + 1] += f.y;
+                        for (int j = 0; j < 4; ++j) {
+                            if (col0 + 32 * c + 8 * j >= cend) break;
+                            const uint4 bv = __ldg(bp + j);
+                            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&bv);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = __bfloat1622float2(h[e]);
+                                v[8 * j + 2 * e] += f.x;
+                                v[8 * j + 2 * e + 1] += f.y;
+                            }
                         }
                     }
-                }
+                    if (p.act == ACT_GELU_TANH) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint4 o;
-                    o.x = pack_bf16(v[8 * j + 0], v[8 * j + 1]);
-                    o.y = pack_bf16(v[8 * j + 2], v[8 * j + 3]);
-                    o.z = pack_bf16(v[8 * j + 4], v[8 * j + 5]);
-                    o.w = pack_bf16(v[8 * j + 6], v[8 * j + 7]);
-                    *reinterpret_cast<uint4 *>(chunk + ((j ^ sw) << 4)) = o;
+                        for (int i = 0; i < 32; ++i) v[i] = gelu_tanh_fast(v[i]);
+                    }
+                    if (has_r) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint4 rv = *reinterpret_cast<const uint4 *>(chunk + ((j ^ sw) << 4));
+                            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&rv);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = __bfloat1622float2(h[e]);
+                                v[8 * j + 2 * e] += f.x;
+                                v[8 * j + 2 * e + 1] += f.y;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 o;
+                        o.x = pack_bf16(v[8 * j + 0], v[8 * j + 1]);
+                        o.y = pack_bf16(v[8 * j + 2], v[8 * j + 3]);
+                        o.z = pack_bf16(v[8 * j + 4], v[8 * j + 5]);
+                        o.w = pack_bf16(v[8 * j + 6], v[8 * j + 7]);
+                        *reinterpret_cast<uint4 *>(chunk + ((j ^ sw) << 4)) = o;
+                    }
+                }
+                fence_before_sync();
+                fence_async_smem();  // the staging writes become visible to the TMA stores
+                __syncwarp();
+                if (lane == 0) {
+                    if (c1 == nchunk)  // the accumulator is read: the next tile may overwrite it
+                        mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+#pragma unroll 1
+                    for (int c = c0; c < c1; ++c)
+                        tma_store_2d(&mo.C[seg], stg + (c - c0) * L::CHUNK_BYTES, col0 + 32 * c, row0);
+                    bulk_commit();
                 }
             }
-            fence_before_sync();
-            fence_async_smem();  // the staging writes become visible to the TMA stores
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-#pragma unroll 1
-                for (int c = 0; c < nchunk; ++c)
-                    tma_store_2d(&mo.C[seg], stg + c * L::CHUNK_BYTES, col0 + 32 * c, row0);
-                bulk_commit();
-            }
+            if (!ok) break;
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
@@ -545,9 +555,9 @@ const SchedVal *tile_schedule(const SchedKey &k) {
     return &cache.emplace(k, std::move(v)).first->second;
 }
 
-template <int BN, int STAGES, bool STAGING>
+template <int BN, int STAGES, bool STAGING, int SCH>
 cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
-    using L = Layout2<BN, STAGES, STAGING>;
+    using L = Layout2<BN, STAGES, STAGING, SCH>;
     CUtensorMap mA, mB[3];
     // a refused tensor map sends the caller to another kernel
     if (!encode_map_2d_bf16(&mA, a.A, a.K, a.rows, a.lda * 2, BK, BMC)) return cudaErrorNotSupported;
@@ -589,7 +599,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
     p.tiles = m_tiles * a.nmat * p.n_tiles;
     p.status = device_status_ptr();
     if (!p.status) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, STAGES, STAGING>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, STAGES, STAGING, SCH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     // persistent grid: as many pairs as can be resident at once (pairs must
@@ -601,7 +611,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
         cfg.blockDim = dim3(kThreads, 1, 1);
         cfg.dynamicSmemBytes = L::ALLOC;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<BN, STAGES, STAGING>, &cfg) != cudaSuccess || n < 1)
+        if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<BN, STAGES, STAGING, SCH>, &cfg) != cudaSuccess || n < 1)
             n = (num_sms() > 0 ? num_sms() : 148) / 2;
         (void)cudaGetLastError();
         max_pairs = n;
@@ -615,7 +625,7 @@ cudaError_t launch_bn2(const GemmArgs &a, cudaStream_t s) {
         memcpy(p.sched, sv->tile.data(), sv->tile.size() * sizeof(uint16_t));
         p.nsched = p.tiles;
     }
-    return launch_pdl(gemm_tc2_kernel<BN, STAGES, STAGING>, dim3(2 * pairs), dim3(kThreads), L::ALLOC, s,
+    return launch_pdl(gemm_tc2_kernel<BN, STAGES, STAGING, SCH>, dim3(2 * pairs), dim3(kThreads), L::ALLOC, s,
                       mA, mB[0], mB[1], mB[2], mo, p);
 }
 
@@ -663,7 +673,12 @@ cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) {
     bool all_tiled = true;
     for (int i = 0; i < a.nmat; ++i) all_tiled = all_tiled && a.thl[i] != nullptr;
     // outputs in tiled head layout need no staging tiles: two more pipeline stages
-    return all_tiled ? launch_bn2<256, 7, false>(a, s) : launch_bn2<256, 5, true>(a, s);
+    if (all_tiled) return launch_bn2<256, 7, false, 8>(a, s);
+    // row-major outputs: half a tile's columns staged per pass leaves room for a
+    // sixth pipeline stage
+    const char *v = getenv("PTDIT_GEMM_EPI");
+    if (v && v[0] == '8') return launch_bn2<256, 5, true, 8>(a, s);
+    return launch_bn2<256, 6, true, 4>(a, s);
 }
 
 }  // namespace ptdit

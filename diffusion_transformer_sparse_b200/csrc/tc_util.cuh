@@ -64,18 +64,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of the phase (try_wait may suspend the thread for a while
+// before it answers; test_wait answers at once).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// A wait with a limit below kWaitLimitNs (ptdit_debug_wait_limit) polls with
+// test_wait, so that the limit bites even where try_wait's own suspension would
+// outlast it; regular waits use try_wait.
+__device__ __forceinline__ bool mbar_poll(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    return limit_ns < kWaitLimitNs ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity);
+}
+
 // Waits for the phase of `bar` with the given parity.  Returns false if the
 // wait ran past kWaitLimitNs (then *status gets PTDIT_ERR_TIMEOUT and *abort
 // is raised for the rest of the CTA) or another role already raised *abort;
 // the caller then stops issuing work.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int *status, uint64_t limit_ns = kWaitLimitNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_poll(bar, parity, limit_ns)) return true;
     const uint64_t t0 = globaltimer();
     for (;;) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+            if (mbar_poll(bar, parity, limit_ns)) return true;
         if (*abort) return false;
         if (globaltimer() - t0 > limit_ns) {
             *abort = 1;
@@ -93,13 +114,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 // that see it late see it on their next try); only the slow path votes.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
                                                int *status, uint64_t limit_ns = kWaitLimitNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_poll(bar, parity, limit_ns)) return true;
     const unsigned active = __activemask();
     const uint64_t t0 = globaltimer();
     for (;;) {
         bool got = false;
 #pragma unroll 1
-        for (int i = 0; i < 32 && !got; ++i) got = mbar_try_wait(bar, parity);
+        for (int i = 0; i < 32 && !got; ++i) got = mbar_poll(bar, parity, limit_ns);
         const unsigned seen = __ballot_sync(active, got);
         if (seen == active) return true;
         if (seen != 0) continue;  // the phase is complete: the other lanes see it next time
