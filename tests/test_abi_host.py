@@ -143,3 +143,88 @@ def test_python_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(pt, "LIB_PATH", "/nonexistent/libptdit.so")
     with pytest.raises(RuntimeError, match="missing"):
         pt.lib()
+
+
+# ---------------------------------------------------------------- bf16 tensor-core shapes
+
+@pytest.mark.parametrize("kw,window,msg", [
+    (dict(D=176, heads=2, dtype=pt.PTDIT_BF16), (1, 4, 4), b"head width 88"),
+    (dict(D=120, heads=2, dtype=pt.PTDIT_BF16), (1, 4, 4), b"multiples of 16"),
+    (dict(F=4, H=8, W=12, D=96, heads=4, dtype=pt.PTDIT_BF16), (2, 4, 3), b"24 tokens"),
+    (dict(F=2, H=16, W=16, D=64, heads=2, dtype=pt.PTDIT_BF16), (2, 16, 16), b"512 tokens"),
+])
+def test_bf16_shapes_without_tensor_core_kernel_are_refused(L, kw, window, msg):
+    s = _shape(**kw)
+    assert _block(L, s, ratio=(1, 2, 2), window=window, shift=(0, 0, 0)) == 2
+    assert msg in L.ptdit_last_error()
+
+
+def test_fp32_takes_the_shapes_bf16_refuses(L):
+    # same shape in fp32 passes validation and only fails on the (fake) workspace size
+    s = _shape(F=4, H=8, W=12, D=96, heads=4, dtype=pt.PTDIT_F32)
+    assert _block(L, s, ratio=(1, 2, 2), window=(2, 4, 3), shift=(0, 0, 0), ws_bytes=16) == 4
+
+
+# ---------------------------------------------------------------- proxy modes and the complete block
+
+def test_proxy_extract_rejects(L):
+    s = _shape()
+    r = pt._i3((1, 2, 2))
+    assert L.ptdit_proxy_extract(ctypes.byref(s), r, 3, None, FAKE, FAKE * 64, None) == 2
+    assert L.ptdit_proxy_extract(ctypes.byref(s), r, pt.PTDIT_PROXY_RANDOM, None, FAKE,
+                                 FAKE * 64, None) == 1
+    assert L.ptdit_proxy_extract(ctypes.byref(s), r, pt.PTDIT_PROXY_RANDOM, FAKE + 2, FAKE,
+                                 FAKE * 64, None) == 7
+    assert L.ptdit_proxy_extract(ctypes.byref(s), pt._i3((1, 3, 2)), 1, None, FAKE, FAKE * 64,
+                                 None) == 2
+
+
+def _bw(**kw):
+    bw = pt.BlockW()
+    for i, m in enumerate(("psa", "cross", "wsa", "swsa", "text")):
+        setattr(bw, m, _w(FAKE * (2 + i)))
+    for i, k in enumerate(("proxy", "cross", "wsa", "swsa", "text", "mlp")):
+        setattr(bw, "norm_" + k, pt.NormW(FAKE * 8 + i * 4096, FAKE * 9 + i * 4096))
+    bw.w1, bw.b1, bw.w2, bw.b2 = FAKE * 10, FAKE * 11, FAKE * 12, FAKE * 13
+    bw.mlp_hidden, bw.eps = 256, 1e-6
+    for k, v in kw.items():
+        setattr(bw, k, v)
+    return bw
+
+
+def _pt_block(L, shape, bw, text=FAKE * 14, text_len=7, mode=0, slots=None, ws_bytes=1 << 40):
+    return L.ptdit_pt_block(ctypes.byref(shape), pt._i3((1, 2, 2)), pt._i3((1, 4, 4)),
+                            pt._i3((0, 2, 2)), ctypes.byref(bw), text, text_len, mode, slots,
+                            FAKE * 32, FAKE * 64, FAKE * 128, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(text_len=0), 2),
+    (dict(text=0), 1),
+    (dict(bw=dict(mlp_hidden=0)), 2),
+    (dict(bw=dict(eps=0.0)), 2),
+    (dict(bw=dict(eps=2.0)), 2),
+    (dict(bw=dict(w1=0)), 1),
+    (dict(bw=dict(b2=FAKE * 13 + 4)), 7),
+    (dict(mode=2), 1),
+    (dict(ws_bytes=4096), 4),
+])
+def test_pt_block_rejects(L, kw, code):
+    bw = _bw(**kw.pop("bw", {}))
+    assert _pt_block(L, _shape(), bw, **kw) == code
+    assert L.ptdit_last_error()
+
+
+def test_pt_block_rejects_bf16_mlp_width_not_multiple_of_16(L):
+    s = _shape(D=64, heads=2, dtype=pt.PTDIT_BF16)
+    assert _pt_block(L, s, _bw(mlp_hidden=200)) == 2
+    assert b"multiples of 16" in L.ptdit_last_error()
+
+
+def test_pt_block_workspace_covers_the_attention_path(L):
+    s = _shape(B=2, F=2, H=16, W=16, D=1152, heads=16, dtype=pt.PTDIT_BF16)
+    attn = _bytes(L, s, (1, 4, 4), (2, 8, 8))
+    n = L.ptdit_pt_block_workspace_bytes(ctypes.byref(s), pt._i3((1, 4, 4)), 120, 4608)
+    # plus the norm output, the MLP hidden layer and the text K / V blocks
+    assert n >= attn + 2 * 512 * 4608 * 2 + 2 * 512 * 1152 * 2
+    assert L.ptdit_pt_block_workspace_bytes(ctypes.byref(s), pt._i3((1, 4, 4)), 0, 4608) == 0
