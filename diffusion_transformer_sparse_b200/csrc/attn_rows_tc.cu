@@ -1,39 +1,37 @@
 // Row-mode attention core on the tensor cores: proxy self-attention and
 // latent -> proxy cross-attention of GIIM (Qihoo-T2X reading note, §3
-// Method, Eq. GIIM), the text cross-attention of the complete PT-Block, and
-// full self-attention (the dense comparator of the complexity paragraph).
-// Queries are rows [0, nq) and keys rows [0, nk) of each batch item; head h
-// is columns h*d .. h*d+d-1.
+// Method, Eq. GIIM), and full self-attention (the dense comparator of the
+// complexity paragraph).  Queries are rows [0, nq) and keys rows [0, nk) of
+// each batch item; head h is columns h*d .. h*d+d-1.
 //
-// One persistent CTA per SM; a unit is two 128-row query tiles (A, B) of one
-// (batch item, head).  The unit's work is a sequence of items, one per
-// (key tile j, query tile t) in the order (0,A), (0,B), (1,A), (1,B), ...,
-// so both query tiles use each K/V tile while it is in shared memory.
-//   warp 0       loader: the unit's two Q tiles (double buffered across
-//                units) and each key tile's K and V into a two-stage ring,
-//                each one contiguous bulk copy: the projections wrote Q, K and
-//                V in tiled head layout (thl.cuh), so a (tile, head) block is
-//                already the swizzled shared-memory tile (V padded to 128
-//                columns for d > 64: one P V MMA per K step).
-//   warp 1       MMA issuer: S(i) = Q_t K_j^T into score buffer i % 2 of TMEM,
-//                and, once the softmax has written P(i) over it, O_t += P(i) V_j
-//                with P read from TMEM; then S(i + 2).  The scores of the next
-//                item are computed while the softmax of this one runs, and a
-//                P V never waits for the next item's scores.
-//   warps 4-7, 8-11   softmax: both warpgroups work on every item, thread r of
-//                warpgroup g owning keys 64 g .. 64 g + 63 of query row r (its
-//                TMEM lane).  The two threads of a row exchange their maxima
-//                through shared memory (an mbarrier per warp pair and item
-//                parity), keep one reference max per query tile that only rises
-//                by more than 2^8 (rescaling that tile's O in TMEM after its
-//                previous P V has landed), exponentiate 64 scores each with
-//                ex2.approx and write their half of P as bf16 pairs.  After a
-//                unit's last item they read O_A and O_B, divide by the row sum
-//                (V's ones column when d = 72, else the two halves' sums) and
-//                store each warp's 32 rows through its own staging rows, with
-//                consecutive lanes on consecutive 16-byte pieces of a row.
-// TMEM: score buffers at columns 0 and 128, O_A at 256, O_B at 384.
-// Every wait is bounded (2 s); the softmax warps decide per warp.
+// FlashAttention-style warp specialisation, one persistent CTA per SM:
+//   warp 0       loader: two 128-row query tiles per unit (double buffered
+//                across units) and K and V tiles into a two-stage ring, each
+//                one contiguous bulk copy: the projections wrote Q, K and V in
+//                tiled head layout (thl.cuh), so a (tile, head) block already
+//                is the swizzled shared-memory tile (columns 0..63 with the
+//                128-byte swizzle, 64..79 with the 32-byte swizzle, zeros past
+//                the head; V padded to 128 columns).
+//   warp 1       MMA issuer: S_g = Q_g K^T (K-major operands) into TMEM, and
+//                once softmax g has written P_g, P_g V with P_g read straight
+//                from TMEM and V as an MN-major operand (no transpose),
+//                accumulating into O_g in TMEM.
+//   warps 4-7 and 8-11   two softmax warpgroups, one per query tile: thread r
+//                owns row r (its TMEM lane), reads its 128 scores with one
+//                wait, runs the fp32 online softmax and writes P (bf16, two per
+//                column) back over the first 64 columns of its scores; O is
+//                rescaled in TMEM only when a row's reference max has to rise
+//                by more than 2^8.  P never touches shared memory (a version
+//                with P in shared memory, which lets the next S be issued as
+//                soon as the softmax has read the current one, was slower: the
+//                P writes and reads crowd shared-memory bandwidth, and the
+//                unpadded V it needed costs a second, N = 16, MMA per K step).
+// Both query tiles share every K/V tile; the MMA warp issues PV_0, S_0(next),
+// PV_1, S_1(next), so each softmax gets its next scores while the other one
+// works.  Splitting each tile's scores into two 64-key slots (so that the next
+// half's scores are ready when the softmax of a half ends) was slower: it
+// doubles the softmax -> P V -> S round trips, each about as long as before.
+// Every wait is bounded (2 s).
 #include <math.h>
 
 #include "tc_util.cuh"
@@ -46,31 +44,32 @@ using namespace tc;
 
 constexpr int BQ = 128, BKV = 128;
 constexpr int kThreads = 384;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 512;  // S0, S1, O0, O1: 128 columns each
+
 constexpr int NSTAGE = 2;  // K/V ring depth
 
 template <int DPAD>
 struct RowsLayout {
-    static constexpr bool HAS_B = DPAD > 64;             // head columns 64..79
-    static constexpr int TILE_A = BQ * 64 * 2;           // 128 rows x 128 B, 128-byte swizzle
+    static constexpr bool HAS_B = DPAD > 64;            // head columns 64..79
+    static constexpr int TILE_A = BQ * 64 * 2;          // 128 rows x 128 B, 128-byte swizzle
     static constexpr int TILE_B = HAS_B ? BQ * 16 * 2 : 0;  // 128 rows x 32 B, 32-byte swizzle
-    static constexpr int TILE = TILE_A + TILE_B;         // a Q or K tile (K-major)
-    // V is the MN-major operand of P V, padded to 128 columns for d > 64 (one
-    // N = 128 MMA per K step costs what an N = 64 one does)
+    static constexpr int TILE = TILE_A + TILE_B;        // a Q or K tile (K-major)
+    // V is the MN-major operand of P V: one MMA per K step costs the same for
+    // N = 64 or 128, so its head columns are padded to 128 with a second
+    // 64-wide 128-byte-swizzled atom (zeros past the head) instead of being
+    // split into an N = 64 and an N = 16 MMA.
     static constexpr int VTILE = HAS_B ? 2 * TILE_A : TILE_A;
-    static constexpr int NPV = HAS_B ? 128 : 64;         // N of the P V MMA
-    static constexpr int OFF_Q = 0;                      // [unit parity][query tile]
-    static constexpr int OFF_K = 4 * TILE;               // [stage]
-    static constexpr int OFF_V = OFF_K + NSTAGE * TILE;  // [stage]
-    static constexpr int OFF_XM = OFF_V + NSTAGE * VTILE;  // float [item parity][half][128]
-    static constexpr int OFF_XL = OFF_XM + 2 * 2 * BQ * 4;  // float [query tile][half][128]
-    // output staging: 32 rows of at most 6 16-byte units per softmax warp
-    static constexpr int WSTG = 32 * 96;
-    static constexpr int OFF_STG = OFF_XL + 2 * 2 * BQ * 4;
-    static constexpr int OFF_BAR = OFF_STG + 8 * WSTG;
-    // q_full[2], q_empty[2], kv_full[2], kv_empty[2], s_full[2], p_full[2],
-    // pv_done[2], o_full[2], xbar[4][2], lbar[4], drain
-    static constexpr int NBARS = 16 + 8 + 4 + 1;
+    static constexpr int NPV = HAS_B ? 128 : 64;        // N of the P V MMA
+    static constexpr int OFF_Q = 0;                     // [unit parity][query tile]
+    static constexpr int OFF_K = 4 * TILE;              // [stage]
+    static constexpr int OFF_V = OFF_K + NSTAGE * TILE; // [stage]
+    // output staging of each softmax warpgroup: 128 rows, pitch <= 160 B
+    static constexpr int STG = BQ * 160;
+    static constexpr int OFF_STG = OFF_V + NSTAGE * VTILE;
+    static constexpr int OFF_BAR = OFF_STG + 2 * STG;
+    // kv_full[NSTAGE], kv_empty[NSTAGE], q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2],
+    // drain, stage_full[2], stage_free[2]
+    static constexpr int NBARS = 2 * NSTAGE + 15;
     static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
     static_assert(TILE % 1024 == 0 && TILE_A % 1024 == 0, "swizzled tiles stay 1 KB aligned");
     static_assert(BYTES <= 232448, "shared memory budget");
@@ -99,11 +98,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
-    uint64_t *q_full = bars, *q_empty = bars + 2, *kv_full = bars + 4, *kv_empty = bars + 6;
-    uint64_t *s_full = bars + 8, *p_full = bars + 10, *pv_done = bars + 12, *o_full = bars + 14;
-    uint64_t *xbar = bars + 16;  // [warp pair][item parity]
-    uint64_t *lbar = bars + 24;  // [warp pair]
-    uint64_t *drain = bars + 28;
+    uint64_t *kv_full = bars, *kv_empty = bars + NSTAGE;
+    uint64_t *q_full = bars + 2 * NSTAGE, *q_empty = q_full + 2, *s_full = q_full + 4;
+    uint64_t *p_full = q_full + 6, *o_full = q_full + 8, *drain = q_full + 10;
+    uint64_t *stage_full = q_full + 11, *stage_free = q_full + 13;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -111,22 +109,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int d = a.d, nch = d / 8;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&q_full[s], 1);
-            mbar_init(&q_empty[s], 1);
+        for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
-            mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], 2 * BQ);  // both threads of every row
-            mbar_init(&pv_done[s], 1);
-            mbar_init(&o_full[s], 1);
         }
-        for (int w = 0; w < 4; ++w) {
-            mbar_init(&xbar[2 * w], 64);
-            mbar_init(&xbar[2 * w + 1], 64);
-            mbar_init(&lbar[w], 64);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], BQ);
+            mbar_init(&o_full[s], 1);
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
         }
         mbar_init(drain, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&stage_full[s], BQ);
+            mbar_init(&stage_free[s], BQ);
+        }
         *abort = 0;
         fence_mbar_init();
     }
@@ -140,7 +138,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int u0 = (int)((long)blockIdx.x * sc.units / gridDim.x);
     const int u1 = (int)((long)(blockIdx.x + 1) * sc.units / gridDim.x);
-    const int kt = sc.kt;
 
     if (warp == 0) {
         // ------------------------------------------------------------ loader
@@ -153,24 +150,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                              uint32_t bytes) {
                 return base + (((long)b * t.tiles + tile) * a.heads + h) * (long)bytes;
             };
-            int kc = 0, last_q_unit = -1;
+            int item = 0, last_q_unit = -1;
             bool ok = true;
             for (int u = u0; u < u1 && ok; ++u) {
                 int b, h, qp;
                 decode(a, sc, u, b, h, qp);
-                const int un = u - u0, qb = un & 1;
-                if (!mbar_wait(&q_empty[qb], ((un >> 1) & 1) ^ 1, abort, status)) { ok = false; break; }
-                // the unit's second query tile may lie past the last one: the last
-                // tile is loaded twice then (its second results are not stored)
-                mbar_expect_tx(&q_full[qb], 2 * L::TILE);
-                for (int g = 0; g < 2; ++g)
-                    bulk_load(sm + L::OFF_Q + (qb * 2 + g) * L::TILE,
-                              block(qg, a.tq, b, min(2 * qp + g, a.tq.tiles - 1), h, L::TILE),
-                              L::TILE, &q_full[qb]);
-                last_q_unit = un;
-                for (int j = 0; j < kt; ++j, ++kc) {
-                    const int st = kc % NSTAGE;
-                    if (!mbar_wait(&kv_empty[st], ((kc / NSTAGE) & 1) ^ 1, abort, status)) { ok = false; break; }
+                const int un = u - u0;
+                for (int j = 0; j < sc.kt; ++j, ++item) {
+                    const int st = item % NSTAGE;
+                    if (j == 0) {
+                        const int qb = un & 1;
+                        if (!mbar_wait(&q_empty[qb], ((un >> 1) & 1) ^ 1, abort, status)) { ok = false; break; }
+                        // the unit's second query tile may lie past the last one: the
+                        // last tile is loaded twice then (its second results are
+                        // not stored), so no row scores uninitialised memory
+                        mbar_expect_tx(&q_full[qb], 2 * L::TILE);
+                        for (int g = 0; g < 2; ++g)
+                            bulk_load(sm + L::OFF_Q + (qb * 2 + g) * L::TILE,
+                                      block(qg, a.tq, b, min(2 * qp + g, a.tq.tiles - 1), h, L::TILE),
+                                      L::TILE, &q_full[qb]);
+                        last_q_unit = un;
+                    }
+                    if (!mbar_wait(&kv_empty[st], ((item / NSTAGE) & 1) ^ 1, abort, status)) { ok = false; break; }
                     mbar_expect_tx(&kv_full[st], L::TILE + L::VTILE);
                     bulk_load(sm + L::OFF_K + st * L::TILE, block(kg, a.tk, b, j, h, L::TILE), L::TILE,
                               &kv_full[st]);
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) {  // let copies still in flight land before the CTA exits
                 volatile int never = 0;
-                for (int i = kc - NSTAGE; i < kc; ++i)
+                for (int i = item - NSTAGE; i < item; ++i)
                     if (i >= 0) mbar_wait(&kv_full[i % NSTAGE], (i / NSTAGE) & 1, &never, status);
                 if (last_q_unit >= 0)
                     mbar_wait(&q_full[last_q_unit & 1], (last_q_unit >> 1) & 1, &never, status);
@@ -188,55 +189,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Order per item i: PV0(i), S0(i+1), PV1(i), S1(i+1), so each softmax
+        // warpgroup gets its next S right after handing over its P, while the
+        // other warpgroup is still busy.
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(BQ, BKV);
             constexpr uint32_t idesc_o = idesc_bf16(BQ, L::NPV, true);
-            const int per_unit = 2 * kt;
-            const int n_items = (u1 - u0) * per_unit;
+            const int n_items = (u1 - u0) * sc.kt;
             bool ok = true, any = false;
-            // S(i) = Q_t K_j^T into score buffer i % 2 (after P V(i - 2), issued
-            // before it, has read P(i - 2) out of that buffer: tcgen05.mma
-            // instructions of one thread run in issue order)
-            auto issue_s = [&](int i) {
-                const int un = i / per_unit, il = i % per_unit, j = il >> 1, t = il & 1;
-                const int kc = un * kt + j, st = kc % NSTAGE, qb = un & 1;
-                if (t == 0) {
-                    if (!mbar_wait(&kv_full[st], (kc / NSTAGE) & 1, abort, status)) return false;
+            // S_g(i) = Q_g K(i)^T; waits for the K tile (and, at a unit's first
+            // tile, for the unit's Q tiles) when g == 0
+            auto issue_s = [&](int i, int g) {
+                const int st = i % NSTAGE, j = i % sc.kt, un = i / sc.kt, qb = un & 1;
+                if (g == 0) {
+                    if (!mbar_wait(&kv_full[st], (i / NSTAGE) & 1, abort, status)) return false;
                     if (j == 0 && !mbar_wait(&q_full[qb], (un >> 1) & 1, abort, status)) return false;
                     fence_after_sync();
                 }
                 const uint32_t aK = smem_u32(sm + L::OFF_K + st * L::TILE);
-                const uint32_t aQ = smem_u32(sm + L::OFF_Q + (qb * 2 + t) * L::TILE);
-                const uint32_t tS = tmem + (i & 1) * BKV;
+                const uint32_t aQ = smem_u32(sm + L::OFF_Q + (qb * 2 + g) * L::TILE);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tS, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32), idesc_s,
-                             kk > 0);
+                    mma_bf16(tmem + g * BKV, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
+                             idesc_s, kk > 0);
                 if (L::HAS_B)
-                    mma_bf16(tS, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A), idesc_s, 1);
-                mma_commit(&s_full[i & 1]);
-                if (t == 1 && j == kt - 1) mma_commit(&q_empty[qb]);  // the unit's Q tiles are read
+                    mma_bf16(tmem + g * BKV, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
+                             idesc_s, 1);
+                mma_commit(&s_full[g]);
+                if (g == 1 && j == sc.kt - 1) mma_commit(&q_empty[qb]);  // the unit's Q tiles are read
                 any = true;
                 return true;
             };
-            if (n_items > 0) ok = issue_s(0);
-            if (ok && n_items > 1) ok = issue_s(1);
+            if (n_items > 0) ok = issue_s(0, 0) && issue_s(0, 1);
             for (int i = 0; i < n_items && ok; ++i) {
-                const int un = i / per_unit, il = i % per_unit, j = il >> 1, t = il & 1;
-                const int kc = un * kt + j, st = kc % NSTAGE;
-                if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, abort, status)) { ok = false; break; }
-                fence_after_sync();
+                const int st = i % NSTAGE, j = i % sc.kt;
                 const uint32_t aV = smem_u32(sm + L::OFF_V + st * L::VTILE);
-                const uint32_t tP = tmem + (i & 1) * BKV;  // P over the first 64 columns
-                const uint32_t tO = tmem + 256 + t * 128;
+                for (int g = 0; g < 2 && ok; ++g) {
+                    if (!mbar_wait(&p_full[g], i & 1, abort, status)) { ok = false; break; }
+                    fence_after_sync();
+                    const uint32_t tP = tmem + g * BKV;  // P_g over the first 64 columns of S_g
+                    const uint32_t tO = tmem + 256 + g * 128;
 #pragma unroll
-                for (int ks = 0; ks < BKV / 16; ++ks)
-                    mma_bf16_ts(tO, tP + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A), idesc_o,
-                                (j | ks) > 0);
-                mma_commit(&pv_done[t]);
-                if (t == 1) mma_commit(&kv_empty[st]);  // both S and both P V of key tile j
-                if (j == kt - 1) mma_commit(&o_full[t]);
-                if (i + 2 < n_items) ok = issue_s(i + 2);
+                    for (int ks = 0; ks < BKV / 16; ++ks)
+                        mma_bf16_ts(tO, tP + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
+                                    idesc_o, (j | ks) > 0);
+                    mma_commit(&o_full[g]);
+                    if (g == 1) mma_commit(&kv_empty[st]);  // both S and both P V of item i
+                    if (i + 1 < n_items) ok = issue_s(i + 1, g);
+                }
             }
             if (any) {  // every issued MMA has finished before TMEM is released
                 mma_commit(drain);
@@ -245,163 +245,157 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp >= 4) {
-        // ------------------------------------------------------------ softmax
-        // TMEM loads and stores are warp-collective: every decision in front of
-        // one is taken by the whole warp (bounded waits per warp; a rescale runs
-        // when any row of the warp needs it, the others scale by 1).
-        const int hf = (warp - 4) / 4, w = warp % 4;
-        const int r = w * 32 + lane;  // query row of the tile = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>(w * 32) << 16;
-        float *xm = reinterpret_cast<float *>(sm + L::OFF_XM);  // [item parity][half][row]
-        float *xl = reinterpret_cast<float *>(sm + L::OFF_XL);  // [query tile][half][row]
+        // ------------------------------------------------------------ softmax warpgroups
+        // The output accumulates in TMEM (each P V adds onto it).  Scores are
+        // exponentiated against a per-row reference max that is only raised
+        // when a tile's max exceeds it by more than 2^8 (weights then stay
+        // below 256, harmless in fp32); raising it rescales the row of O in
+        // TMEM, after the previous P V has landed.  TMEM loads and stores are
+        // warp-collective, so every decision in front of one is taken by the
+        // whole warp: wait results are combined over the warp, and a rescale
+        // runs when any row of the warp needs it (the others scale by 1).
+        const int g = (warp - 4) / 4;
+        auto wait_all = [&](uint64_t *bar, uint32_t par) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, par, abort, status));
+        };
+        const int r = (warp % 4) * 32 + lane;  // query row of the tile = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + g * BKV;
+        const uint32_t t_o = tmem + lane_base + 256 + g * 128;
         const float sl2 = a.scale * 1.4426950408889634f;
         __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
-        // output units (8 columns) of this thread: half 0 the first ceil(nch / 2)
-        const int nu0 = (nch + 1) / 2, ub = hf ? nu0 : 0, nu = hf ? nch - nu0 : nu0;
-        const int pitch = nu * 16 + (nu % 2 == 0 ? 16 : 0);  // an odd number of 16-byte units
-        uint8_t *stg = sm + L::OFF_STG + (warp - 4) * L::WSTG;
-        // O columns this thread rescales: half 0 [0, 64), half 1 [64, DPAD)
-        const int oc0 = hf ? 64 : 0, oc1 = hf ? DPAD : (DPAD < 64 ? DPAD : 64);
-        int it = 0, un_count = 0;
+        // staging row pitch: an odd number of 16-byte units where that fits
+        const int pitch = nch * 16 + (nch % 8 == 0 ? 16 : 0);
+        int item = 0, un_count = 0;
         bool ok = true;
-        for (int u = u0; u < u1 && ok; ++u, ++un_count) {
+        for (int u = u0; u < u1 && ok; ++u) {
             int b, h, qp;
             decode(a, sc, u, b, h, qp);
-            float m_ref[2] = {-INFINITY, -INFINITY}, l_i[2] = {0.f, 0.f};
-            for (int j = 0; j < kt && ok; ++j) {
+            float m_ref = -INFINITY, l_i = 0.f;
+            for (int j = 0; j < sc.kt; ++j, ++item) {
+                const uint32_t ph = item & 1;
                 const int nvalid = min(BKV, a.nk - j * BKV);
+                if (!wait_all(&s_full[g], ph)) { ok = false; break; }
+                fence_after_sync();
+                // the whole row of S: four loads, one wait
+                uint32_t sv[BKV];
+                tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(sv + 0));
+                tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+                tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(sv + 64));
+                tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(sv + 96));
+                tmem_ld_wait();
+                if (nvalid < BKV) {  // ragged last key tile: masked keys score -inf
 #pragma unroll
-                for (int t = 0; t < 2; ++t, ++it) {
-                    if (!mbar_wait_warp(&s_full[it & 1], (it >> 1) & 1, abort, status)) { ok = false; break; }
-                    fence_after_sync();
-                    const uint32_t t_s = tmem + lane_base + (it & 1) * BKV;
-                    uint32_t sv[64];
-                    tmem_ld32(t_s + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(sv));
-                    tmem_ld32(t_s + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-                    tmem_ld_wait();
-                    if (nvalid < BKV) {  // ragged last key tile: absent keys score -inf
+                    for (int e = 0; e < BKV; ++e)
+                        if (e >= nvalid) sv[e] = __float_as_uint(-INFINITY);
+                }
+                // row max over 8 independent chains of three-input maxima
+                float mx[8];
 #pragma unroll
-                        for (int e = 0; e < 64; ++e)
-                            if (64 * hf + e >= nvalid) sv[e] = __float_as_uint(-INFINITY);
-                    }
-                    float mx[4];
+                for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(sv[c]);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) mx[c] = __uint_as_float(sv[c]);
+                for (int e = 8; e < BKV; e += 16)
 #pragma unroll
-                    for (int e = 4; e < 64; e += 8)
+                    for (int c = 0; c < 8; ++c)
+                        mx[c] = e + 8 + c < BKV
+                                    ? fmax3(mx[c], __uint_as_float(sv[e + c]), __uint_as_float(sv[e + 8 + c]))
+                                    : fmaxf(mx[c], __uint_as_float(sv[e + c]));
+                float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+                tmax *= sl2;
+                const bool raise = tmax > m_ref + 8.f;  // raise the reference; O so far shrinks by alpha
+                if (__any_sync(0xffffffffu, raise)) {
+                    const float alpha = !raise ? 1.f : (m_ref == -INFINITY ? 0.f : ex2_approx(m_ref - tmax));
+                    if (j > 0) {
+                        // O holds P V up to tile j-1 once that MMA has landed
+                        if (!wait_all(&o_full[g], ph ^ 1)) { ok = false; break; }
+                        fence_after_sync();
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            mx[c] = e + 4 + c < 64
-                                        ? fmax3(mx[c], __uint_as_float(sv[e + c]), __uint_as_float(sv[e + 4 + c]))
-                                        : fmaxf(mx[c], __uint_as_float(sv[e + c]));
-                    const float mine = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-                    // the row's other half, through shared memory: both threads of the
-                    // row arrive on the warp pair's barrier of this item parity (and
-                    // have both read their scores before either writes P over them)
-                    float *xs = xm + (it & 1) * 2 * BQ;
-                    xs[hf * BQ + r] = mine;
-                    mbar_arrive(&xbar[2 * w + (it & 1)]);
-                    if (!mbar_wait_warp(&xbar[2 * w + (it & 1)], (it >> 1) & 1, abort, status)) { ok = false; break; }
-                    const float tmax = fmaxf(mine, xs[(1 - hf) * BQ + r]) * sl2;
-                    const bool raise = tmax > m_ref[t] + 8.f;  // O so far shrinks by alpha
-                    if (__any_sync(0xffffffffu, raise)) {
-                        const float alpha =
-                            !raise ? 1.f : (m_ref[t] == -INFINITY ? 0.f : ex2_approx(m_ref[t] - tmax));
-                        if (j > 0 && oc0 < oc1) {
-                            // O_t holds P V up to key tile j - 1 once that MMA has landed
-                            // (pv_done[t] completes once per P V of query tile t)
-                            const int pvc = un_count * kt + j - 1;
-                            if (!mbar_wait_warp(&pv_done[t], pvc & 1, abort, status)) { ok = false; break; }
-                            fence_after_sync();
-                            const uint32_t t_o = tmem + lane_base + 256 + t * 128;
+                        for (int c0 = 0; c0 < DPAD; c0 += 16) {
+                            uint32_t ov[16];
+                            tmem_ld16(t_o + c0, ov);
+                            tmem_ld_wait();
 #pragma unroll
-                            for (int c0 = 0; c0 < 64; c0 += 16) {
-                                if (oc0 + c0 >= oc1) break;
-                                uint32_t ov[16];
-                                tmem_ld16(t_o + oc0 + c0, ov);
-                                tmem_ld_wait();
-#pragma unroll
-                                for (int e = 0; e < 16; ++e)
-                                    ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                                tmem_st16(t_o + oc0 + c0, ov);
-                            }
-                            tmem_st_wait();
+                            for (int e = 0; e < 16; ++e)
+                                ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                            tmem_st16(t_o + c0, ov);
                         }
-                        l_i[t] *= alpha;
-                        if (raise) m_ref[t] = tmax;
+                        tmem_st_wait();
                     }
-                    const float ref = m_ref[t];
-                    float ps[4] = {0.f, 0.f, 0.f, 0.f};
+                    l_i *= alpha;
+                    if (raise) m_ref = tmax;
+                }
+                const float ref = m_ref;
+                float ps[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) ps[c] = 0.f;
+                // P as bf16 pairs, written over the first 64 columns of S.  With
+                // SUMV the row sum comes out of P V (V's ones column) instead of
+                // being added up here.
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), sl2, -ref));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ref));
-                        if (!SUMV) ps[c & 3] += p0 + p1;
+                        const float x0 = fmaf(__uint_as_float(sv[64 * half + 2 * c]), sl2, -ref);
+                        const float x1 = fmaf(__uint_as_float(sv[64 * half + 2 * c + 1]), sl2, -ref);
+                        const float p0 = ex2_approx(x0);
+                        const float p1 = ex2_approx(x1);
+                        if (!SUMV) {
+                            ps[(2 * c) & 7] += p0;
+                            ps[(2 * c + 1) & 7] += p1;
+                        }
                         pk[c] = pack_bf16(p0, p1);
                     }
-                    // keys 64 hf .. 64 hf + 63 as bf16 pairs: columns 32 hf .. 32 hf + 31
-                    tmem_st32(t_s + 32 * hf, pk);
-                    tmem_st_wait();
-                    if (!SUMV) l_i[t] += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-                    fence_before_sync();
-                    mbar_arrive(&p_full[it & 1]);
+                    tmem_st32(t_s + 32 * half, pk);
                 }
+                tmem_st_wait();
+                if (!SUMV)
+                    l_i += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+                fence_before_sync();
+                mbar_arrive(&p_full[g]);
             }
             if (!ok) break;
-            // ---- the unit's outputs: O_A, then O_B
-#pragma unroll 1
-            for (int t = 0; t < 2; ++t) {
-                float lsum = 0.f;
-                if (!SUMV) {  // the row sum of P: both halves (lbar completes once per tile)
-                    float *xt = xl + t * 2 * BQ;
-                    xt[hf * BQ + r] = l_i[t];
-                    mbar_arrive(&lbar[w]);
-                    if (!mbar_wait_warp(&lbar[w], t, abort, status)) { ok = false; break; }
-                    lsum = l_i[t] + xt[(1 - hf) * BQ + r];
-                }
-                if (!mbar_wait_warp(&o_full[t], un_count & 1, abort, status)) { ok = false; break; }
-                fence_after_sync();
-                const uint32_t t_o = tmem + lane_base + 256 + t * 128;
-                uint32_t ov[40];
-#pragma unroll
-                for (int v = 0; v < 5; ++v)
-                    if (v < nu) tmem_ld8(t_o + 8 * (ub + v), *reinterpret_cast<uint32_t(*)[8]>(ov + 8 * v));
-                uint32_t sv8[8];
-                if (SUMV) tmem_ld8(t_o + d, sv8);  // V's ones column: the row sum of P
+            // the unit's last P V, then O / l to global memory through the staging
+            // rows, so that consecutive lanes store consecutive 16-byte pieces of
+            // a row (a few rows per store instruction instead of 32)
+            if (!wait_all(&o_full[g], (item - 1) & 1)) { ok = false; break; }
+            if (!wait_all(&stage_free[g], (un_count & 1) ^ 1)) { ok = false; break; }
+            fence_after_sync();
+            uint8_t *stg = sm + L::OFF_STG + g * L::STG;
+            {
+                uint32_t ov[DPAD];
+                tmem_ld32(t_o, *reinterpret_cast<uint32_t(*)[32]>(ov));
+                tmem_ld32(t_o + 32, *reinterpret_cast<uint32_t(*)[32]>(ov + 32));
+                if (DPAD > 64) tmem_ld16(t_o + 64, *reinterpret_cast<uint32_t(*)[16]>(ov + 64));
                 tmem_ld_wait();
-                // O is in registers: the next unit's first P V may overwrite it after
-                // this thread's next arrival on p_full
-                fence_before_sync();
-                const float inv = 1.f / (SUMV ? __uint_as_float(sv8[0]) : lsum);
+                // SUMV: column d = DPAD - 8 of O holds the row sum of P
+                const float inv = 1.f / (SUMV ? __uint_as_float(ov[DPAD - 8]) : l_i);
 #pragma unroll
-                for (int v = 0; v < 5; ++v)
-                    if (v < nu) {
-                        uint4 o;
-                        o.x = pack_bf16(__uint_as_float(ov[8 * v + 0]) * inv, __uint_as_float(ov[8 * v + 1]) * inv);
-                        o.y = pack_bf16(__uint_as_float(ov[8 * v + 2]) * inv, __uint_as_float(ov[8 * v + 3]) * inv);
-                        o.z = pack_bf16(__uint_as_float(ov[8 * v + 4]) * inv, __uint_as_float(ov[8 * v + 5]) * inv);
-                        o.w = pack_bf16(__uint_as_float(ov[8 * v + 6]) * inv, __uint_as_float(ov[8 * v + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(stg + lane * pitch + v * 16) = o;
+                for (int u = 0; u < DPAD / 8; ++u)
+                    if (u < nch) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(ov[8 * u + 0]) * inv, __uint_as_float(ov[8 * u + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(ov[8 * u + 2]) * inv, __uint_as_float(ov[8 * u + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(ov[8 * u + 4]) * inv, __uint_as_float(ov[8 * u + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(ov[8 * u + 6]) * inv, __uint_as_float(ov[8 * u + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(stg + r * pitch + u * 16) = v;
                     }
-                __syncwarp();
-                // the warp's 32 rows x nu units: consecutive lanes on consecutive units
-                const long q0 = (long)(2 * qp + t) * BQ + w * 32;  // query index of staging row 0
-                __nv_bfloat16 *obase = og + (long)b * a.q_bstride * a.ldo + (long)h * d + 8 * ub;
-                for (int i = lane; i < 32 * nu; i += 32) {
-                    const int row = i / nu, v = i - row * nu;
-                    if (q0 + row < a.nq)
-                        *reinterpret_cast<uint4 *>(obase + (q0 + row) * a.ldo + v * 8) =
-                            *reinterpret_cast<const uint4 *>(stg + row * pitch + v * 16);
-                }
-                __syncwarp();  // the staging rows are free again
             }
-        }
-    }
-    if (*abort) {
-        // a wait gave up: let bulk copies still in flight into this CTA land
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 100000) {
+            fence_before_sync();  // O is read before the next unit's first P V overwrites it
+            mbar_arrive(&stage_full[g]);
+            if (!wait_all(&stage_full[g], un_count & 1)) { ok = false; break; }
+            {
+                const int q0 = qp * 2 * BQ + g * BQ;  // query index of staging row 0
+                __nv_bfloat16 *obase = og + (long)b * a.q_bstride * a.ldo + (long)h * d;
+                for (int i = r; i < BQ * nch; i += BQ) {
+                    const int row = i / nch, u = i - row * nch;
+                    if (q0 + row < a.nq)
+                        *reinterpret_cast<uint4 *>(obase + (long)(q0 + row) * a.ldo + u * 8) =
+                            *reinterpret_cast<const uint4 *>(stg + row * pitch + u * 16);
+                }
+            }
+            mbar_arrive(&stage_free[g]);
+            ++un_count;
         }
     }
     fence_before_sync();

@@ -62,34 +62,29 @@ struct Chunk<T, 1> {
     __device__ __forceinline__ static void store(T *p, const float *v) { p[0] = from_f32<T>(v[0]); }
 };
 
-// blockIdx.x = (b * M + m) * parts + part: the CTA averages chunks
-// [part * CH / parts, (part + 1) * CH / parts) of window m (splitting the
-// channels over `parts` CTAs evens out the last wave of CTAs).  Thread t:
-// chunk lane cl = t % CHT, token group gi = t / CHT; the lanes step over the
-// CTA's chunks CHT at a time.
+// blockIdx.x = b * M + m.  Thread t: chunk lane cl = t % CHT, token group
+// gi = t / CHT; the lanes step over the CH chunks of a row CHT at a time.
 template <typename T, int VEC>
 __global__ void __launch_bounds__(1024) proxy_average_kernel(const T *__restrict__ z,
                                                              T *__restrict__ out, ProxyGeom g,
-                                                             int D, int CHT, int G, int parts) {
+                                                             int D, int CHT, int G) {
     extern __shared__ float red[];  // [G-1][CHT][VEC]
     pdl_wait();  // z is complete
     pdl_trigger();
     const int CH = D / VEC;
-    const int part = blockIdx.x % parts;
-    const int m = (blockIdx.x / parts) % g.M;
-    const int b = blockIdx.x / parts / g.M;
-    const int cbeg = part * CH / parts, cend = (part + 1) * CH / parts;
+    const int m = blockIdx.x % g.M;
+    const int b = blockIdx.x / g.M;
     const int cl = threadIdx.x % CHT;
     const int gi = threadIdx.x / CHT;
     const long N = (long)g.f * g.h * g.w;
     const T *zw = z + (long)b * N * D + (long)proxy_token(g, m, 0) * D;
 
-    for (int c0 = cbeg; c0 < cend; c0 += CHT) {
+    for (int c0 = 0; c0 < CH; c0 += CHT) {
         const int c = c0 + cl;
         float acc[VEC];
 #pragma unroll
         for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
-        if (gi < G && c < cend) {
+        if (gi < G && c < CH) {
             const T *zb = zw + (long)c * VEC;
             // token k of the window sits (a*h + r)*w + q tokens after the first one;
             // each batch issues up to 8 independent 16-byte loads before adding
@@ -114,7 +109,7 @@ __global__ void __launch_bounds__(1024) proxy_average_kernel(const T *__restrict
             for (int i = 0; i < VEC; ++i) red[((gi - 1) * CHT + cl) * VEC + i] = acc[i];
         }
         __syncthreads();
-        if (gi == 0 && c < cend) {
+        if (gi == 0 && c < CH) {
             for (int j = 1; j < G; ++j) {
 #pragma unroll
                 for (int i = 0; i < VEC; ++i) acc[i] += red[((j - 1) * CHT + cl) * VEC + i];
@@ -128,41 +123,19 @@ __global__ void __launch_bounds__(1024) proxy_average_kernel(const T *__restrict
     }
 }
 
-// Channel parts per window: the count (1..4, dividing CH) whose CTAs fill the
-// last wave best, at two CTAs per SM.
-int avg_parts(long windows, int CH) {
-    const int sms = num_sms() > 0 ? num_sms() : 148;
-    const long slots = 2L * sms;
-    int best = 1;
-    double best_fill = 0.0;
-    for (int parts = 1; parts <= 4; ++parts) {
-        if (CH % parts || CH / parts < 32) continue;
-        const long ctas = windows * parts;
-        const double fill = (double)ctas / (double)(((ctas + slots - 1) / slots) * slots);
-        if (fill > best_fill + 0.02) {
-            best = parts;
-            best_fill = fill;
-        }
-    }
-    return best;
-}
-
 template <typename T, int VEC>
 cudaError_t launch_avg(const ProxyGeom &g, int B, int D, const void *z, void *out,
                        cudaStream_t s) {
     const int CH = D / VEC;
-    const int parts = avg_parts((long)B * g.M, CH);
-    const int CHP = CH / parts;
-    const int CHT = CHP < 512 ? CHP : 512;
+    const int CHT = CH < 512 ? CH : 512;
     // token groups: about 8 loads per thread, at most 1024 threads per CTA
     int G = (g.P + 7) / 8;
     if (G > 1024 / CHT) G = 1024 / CHT;
     if (G < 1) G = 1;
     const int threads = CHT * G;
     const size_t smem = (size_t)(G - 1) * CHT * VEC * sizeof(float);
-    return launch_pdl(proxy_average_kernel<T, VEC>, dim3((unsigned)(B * g.M * parts)), dim3(threads),
-                      smem, s, static_cast<const T *>(z), static_cast<T *>(out), g, D, CHT, G,
-                      parts);
+    return launch_pdl(proxy_average_kernel<T, VEC>, dim3((unsigned)(B * g.M)), dim3(threads), smem, s,
+                      static_cast<const T *>(z), static_cast<T *>(out), g, D, CHT, G);
 }
 
 template <typename T, int VEC>
