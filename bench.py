@@ -46,7 +46,13 @@ L2_FLUSH_BYTES = 256 << 20
 # dominant kernel, averaged over the launches of one step, from one ncu capture
 # of the current kernel source, per workload.  Absent when the kernel changed
 # since the capture.
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/gemm_tc2_t2i_2048px_qkv_and_oproj.md: nine launches measured
+    "t2i_2048px_128x128": 59.4e6,
+    # the same capture scaled by rows to the long video (a lower bound: at 16384 rows
+    # part of every output is still in L2 when the kernel ends)
+    "video_32x64x64": 461e6,
+}
 
 
 def load_peaks():
