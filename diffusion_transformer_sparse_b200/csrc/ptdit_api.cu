@@ -398,11 +398,10 @@ int gemm(const Run &r, int kind, const void *A, long rows, int nmat, const void 
 }
 
 // Projections whose outputs C_i are in tiled head layout where thl[i] is set:
-// one fused launch when the 2-SM kernel takes the shape, else one row-major
-// projection per output into `scratch` followed by a relayout.  Tile rows
-// that hold no token are zeroed.
+// one fused launch of the 2-SM kernel (row-major outputs of the fp32 path: one
+// projection per output).  Tile rows that hold no token are zeroed.
 int gemm_thl(const Run &r, int kind, const void *A, long rows, int nmat, const void *const W[3],
-             void *const C[3], const ThlDesc *const thl[3], void *scratch, const char *what) {
+             void *const C[3], const ThlDesc *const thl[3], const char *what) {
     GemmArgs g;
     memset(&g, 0, sizeof g);
     g.dtype = r.d.dtype;
@@ -435,23 +434,20 @@ int gemm_thl(const Run &r, int kind, const void *A, long rows, int nmat, const v
         if (e != cudaSuccess && e != cudaErrorNotSupported) return cuda_fail(e, what);
     }
     if (e == cudaErrorNotSupported) {
+        // row-major outputs (the fp32 path): one projection per output; tiled outputs
+        // exist only where the 2-SM kernel runs (every bf16 shape the API accepts)
         for (int i = 0; i < nmat; ++i) {
+            if (thl[i]) return cuda_fail(cudaErrorNotSupported, what);
             const void *Wi[3] = {W[i], nullptr, nullptr};
-            void *Ci[3] = {thl[i] ? scratch : C[i], nullptr, nullptr};
+            void *Ci[3] = {C[i], nullptr, nullptr};
             TRY(gemm(r, kind, A, rows, 1, Wi, Ci, nullptr, what));
-            if (!thl[i]) continue;
-            timing_begin(kind, r.s);
-            cudaError_t e = launch_thl_fill(*thl[i], r.d.B, r.d.heads, r.d.d, scratch, r.d.D, C[i], r.s);
-            timing_end(r.s);
-            count_launch();
-            if (e != cudaSuccess) return cuda_fail(e, "tiled head layout");
         }
-        return PTDIT_OK;  // the relayout wrote every tile row
+        return PTDIT_OK;
     }
     for (int i = 0; i < nmat; ++i) {
         if (!thl[i] || !thl_has_empty_rows(*thl[i])) continue;
         timing_begin(kind, r.s);
-        cudaError_t e = launch_thl_fill(*thl[i], r.d.B, r.d.heads, r.d.d, nullptr, r.d.D, C[i], r.s);
+        cudaError_t e = launch_thl_zero_rows(*thl[i], r.d.B, r.d.heads, r.d.d, C[i], r.s);
         timing_end(r.s);
         count_launch();
         if (e != cudaSuccess) return cuda_fail(e, "tiled head layout");
@@ -555,8 +551,7 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
         const void *W[3] = {psa->wq, psa->wk, psa->wv};
         void *C[3] = {r.at(r.L.Qp), r.at(r.L.Kp), r.at(r.L.Vp)};
         const ThlDesc *T[3] = {tiled ? &tp : nullptr, tiled ? &tp : nullptr, tiled ? &tpv : nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, pin, BM, 3, W, C, T, r.at(r.L.Ap),
-                     "proxy QKV projection"));
+        TRY(gemm_thl(r, PTDIT_K_GEMM, pin, BM, 3, W, C, T, "proxy QKV projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_PROXY, pa, "proxy self-attention"));
     {
@@ -584,8 +579,7 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
         const void *W[3] = {cross->wk, cross->wv, nullptr};
         void *C[3] = {r.at(r.L.Kc), r.at(r.L.Vc), nullptr};
         const ThlDesc *T[3] = {tiled ? &tp : nullptr, tiled ? &tpv : nullptr, nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.Pp), BM, 2, W, C, T, r.at(r.L.Ap),
-                     "proxy K/V projection"));
+        TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.Pp), BM, 2, W, C, T, "proxy K/V projection"));
     }
     if (nm) {
         TRY(layer_norm(r, nm->cross, nm->eps, z_in, BN, r.at(r.L.Xn), "cross-attention norm"));
@@ -595,7 +589,7 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
         const void *W[3] = {cross->wq, nullptr, nullptr};
         void *C[3] = {r.at(r.L.Q), nullptr, nullptr};
         const ThlDesc *T[3] = {tiled ? &tn : nullptr, nullptr, nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, zq, BN, 1, W, C, T, r.at(r.L.O), "latent Q projection"));
+        TRY(gemm_thl(r, PTDIT_K_GEMM, zq, BN, 1, W, C, T, "latent Q projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_CROSS, ca, "cross-attention"));
     {
@@ -637,7 +631,7 @@ int run_window(const Run &r, const WinGeom &wg, const ptdit_attn_w *w, unsigned 
         const void *W[3] = {w->wq, w->wk, w->wv};
         void *C[3] = {r.at(r.L.Q), r.at(r.L.K), r.at(r.L.V)};
         const ThlDesc *T[3] = {tiled ? &tw : nullptr, tiled ? &tw : nullptr, tiled ? &twv : nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, xa, BN, 3, W, C, T, r.at(r.L.O), "window QKV projection"));
+        TRY(gemm_thl(r, PTDIT_K_GEMM, xa, BN, 3, W, C, T, "window QKV projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "window attention"));
     {
@@ -678,13 +672,13 @@ int run_text(const Run &r, const ptdit_attn_w *w, const ptdit_norm_w *nw, float 
         const void *W[3] = {w->wk, w->wv, nullptr};
         void *C[3] = {r.at(r.L.Kt), r.at(r.L.Vt), nullptr};
         const ThlDesc *T[3] = {tiled ? &tt : nullptr, tiled ? &ttv : nullptr, nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, text, BL, 2, W, C, T, r.at(r.L.O), "text K/V projection"));
+        TRY(gemm_thl(r, PTDIT_K_GEMM, text, BL, 2, W, C, T, "text K/V projection"));
     }
     {
         const void *W[3] = {w->wq, nullptr, nullptr};
         void *C[3] = {r.at(r.L.Q), nullptr, nullptr};
         const ThlDesc *T[3] = {tiled ? &tn : nullptr, nullptr, nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.Xn), BN, 1, W, C, T, r.at(r.L.O),
+        TRY(gemm_thl(r, PTDIT_K_GEMM, r.at(r.L.Xn), BN, 1, W, C, T,
                      "text-attention Q projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_TEXT, a, "text cross-attention"));
@@ -1062,7 +1056,7 @@ int ptdit_full_attn(const ptdit_shape *shape, const ptdit_attn_w *w, unsigned fl
         const void *W[3] = {w->wq, w->wk, w->wv};
         void *C[3] = {r.at(L.Q), r.at(L.K), r.at(L.V)};
         const ThlDesc *T[3] = {tiled ? &tn : nullptr, tiled ? &tn : nullptr, tiled ? &tnv : nullptr};
-        TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 3, W, C, T, r.at(L.O), "QKV projection"));
+        TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 3, W, C, T, "QKV projection"));
     }
     TRY(attention(r, PTDIT_K_ATTN_DENSE, a, "full self-attention"));
     {

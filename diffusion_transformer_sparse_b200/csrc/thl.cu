@@ -1,15 +1,16 @@
-// Relayout of a row-major projection output into tiled head layout blocks,
-// and the zeroing of tile rows that hold no token (see thl.cuh).  The fused
-// projection epilogue writes THL directly; this kernel serves the projection
-// paths that write row-major, and the ragged tail rows of the fused path.
+// Zeroing of the tile rows of a tiled-head-layout operand that hold no token
+// (see thl.cuh).  The projection epilogue writes every row that holds a token;
+// this kernel writes zeros over the ragged tail rows of the last tile of each
+// batch item, every unit of them (a V operand's ones column included: a row
+// without a token must contribute nothing to any sum).
 #include "thl.cuh"
 
 namespace ptdit {
 namespace {
 
-__global__ void thl_fill_kernel(Thl t, int B, int heads, int d, const uint4 *__restrict__ src,
-                                long ld, uint8_t *__restrict__ dst, int tile0, long items) {
-    pdl_wait();  // the projection output (or the blocks being completed) is complete
+__global__ void thl_zero_kernel(Thl t, int B, int heads, int d, uint8_t *__restrict__ dst,
+                                long items) {
+    pdl_wait();  // the projection writing the blocks' other rows has completed
     pdl_trigger();
     const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= items) return;
@@ -19,33 +20,24 @@ __global__ void thl_fill_kernel(Thl t, int B, int heads, int d, const uint4 *__r
     const int r = static_cast<int>(rest % kThlRows);
     rest /= kThlRows;
     const int h = static_cast<int>(rest % heads);
-    rest /= heads;
-    const int span = t.tiles - tile0;  // tiles covered per batch item
-    const int tile = tile0 + static_cast<int>(rest % span);
-    const int b = static_cast<int>(rest / span);
-    const long tok = thl_token(t, tile, r);
-    if (!src && tok >= 0) return;  // only the rows without a token
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (src && tok >= 0 && u * 8 < d)
-        v = src[(((long)b * t.rows_pb + tok) * ld + (long)h * d + u * 8) / 8];
-    else if (src && tok >= 0 && t.ones && u * 8 == d)
-        v = thl_ones_unit();
+    const int b = static_cast<int>(rest / heads);
+    const int tile = t.tiles - 1;  // only the last tile of a batch item has empty rows
+    if (thl_token(t, tile, r) >= 0) return;
     const long blk = ((long)b * t.tiles + tile) * heads + h;
-    *reinterpret_cast<uint4 *>(dst + blk * thl_block_bytes(d, t.vpad) + thl_unit(r, u, t.vpad)) = v;
+    *reinterpret_cast<uint4 *>(dst + blk * thl_block_bytes(d, t.vpad) + thl_unit(r, u, t.vpad)) =
+        make_uint4(0, 0, 0, 0);
 }
 
 }  // namespace
 
-cudaError_t launch_thl_fill(const Thl &t, int B, int heads, int d, const void *src, long ld,
-                            void *dst, cudaStream_t s) {
-    // with src == nullptr only the last tile of each batch item can hold empty rows
-    const int tile0 = src ? 0 : t.tiles - 1;
-    const long items = (long)B * (t.tiles - tile0) * heads * kThlRows * thl_units(d, t.vpad);
-    if (items <= 0) return cudaSuccess;
+cudaError_t launch_thl_zero_rows(const Thl &t, int B, int heads, int d, void *dst,
+                                 cudaStream_t s) {
+    const long items = (long)B * heads * kThlRows * thl_units(d, t.vpad);
+    if (items <= 0 || t.tiles < 1) return cudaSuccess;
     const int threads = 256;
     const long blocks = (items + threads - 1) / threads;
-    return launch_pdl(thl_fill_kernel, dim3((unsigned)blocks), dim3(threads), 0, s, t, B, heads, d,
-                      static_cast<const uint4 *>(src), ld, static_cast<uint8_t *>(dst), tile0, items);
+    return launch_pdl(thl_zero_kernel, dim3((unsigned)blocks), dim3(threads), 0, s, t, B, heads, d,
+                      static_cast<uint8_t *>(dst), items);
 }
 
 }  // namespace ptdit

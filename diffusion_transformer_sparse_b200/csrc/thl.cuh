@@ -83,9 +83,8 @@ __host__ __device__ inline long thl_token(const Thl &t, int tile, int r) {
     return window_token(t.g, win, r % t.g.n, &wrap);
 }
 
-// Writes the matrix [B * rows_pb, ld] (head h = columns h*d ..) as THL blocks
-// at dst, or, with src == nullptr, zeroes only the rows that hold no token.
-cudaError_t launch_thl_fill(const Thl &t, int B, int heads, int d, const void *src, long ld,
-                            void *dst, cudaStream_t s);
+// Writes zeros into the tile rows that hold no token (the last tile of each
+// batch item), for every head of the operand at dst.
+cudaError_t launch_thl_zero_rows(const Thl &t, int B, int heads, int d, void *dst, cudaStream_t s);
 
 }  // namespace ptdit
