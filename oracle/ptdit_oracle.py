@@ -39,8 +39,15 @@ Readings taken where the pages are silent or ambiguous:
     row-major over (t, y, x);
   * every grid extent must be divisible by its ratio and its window.
 
+Backward (training) of a TCM branch: ``window_self_attention_bwd`` returns
+dL/dz and the four weight gradients for a given dL/dout, by the chain rule
+written out per window and head (``attention_heads_bwd`` holds the softmax
+Jacobian step); roll and window partition are row permutations, so their
+adjoints are the inverse permutations.
+
 Every function here is pinned by the CPU tests (tests/test_oracle_pins.py)
-against closed forms, library routines, brute force or hand-derived fixtures.
+against closed forms, library routines, brute force, hand-derived fixtures or,
+for the gradients, central finite differences and torch autograd.
 """
 from __future__ import annotations
 
@@ -329,6 +336,76 @@ def window_self_attention(z, grid, window, shift, W, heads, *, residual=True,
         yw[k] = multihead_attention(zw[k], zw[k], W, heads, allow)
     y = np.roll(_from_windows(yw, grid, window), shift=tuple(shift), axis=(0, 1, 2)).reshape(N, D)
     return z + y if residual else y
+
+
+def attention_heads_bwd(Q, K, V, dA, heads, allow=None):
+    """Gradients of attention_heads with respect to Q, K and V, given dA = dL/dA.
+
+    Per head h, with S = c Q_h K_h^T (c = 1/sqrt(d), masked entries -inf),
+    P = softmax(S) row by row and A_h = P V_h, the chain rule gives
+        dV_h = P^T dA_h,   dP = dA_h V_h^T,
+        dS   = P * (dP - rowsum(P * dP))     (the softmax Jacobian, row by row),
+        dQ_h = c dS K_h,   dK_h = c dS^T Q_h.
+    Masked entries have P = 0, so they pass no gradient.  Returns (dQ, dK, dV).
+    """
+    Q, K, V, dA = _f64(Q), _f64(K), _f64(V), _f64(dA)
+    d = Q.shape[1] // heads
+    c = 1.0 / math.sqrt(d)
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    for h in range(heads):
+        cols = slice(h * d, (h + 1) * d)
+        S = (Q[:, cols] @ K[:, cols].T) * c
+        if allow is not None:
+            S = np.where(allow, S, -np.inf)
+        P = softmax_rows(S)
+        dV[:, cols] = P.T @ dA[:, cols]
+        dP = dA[:, cols] @ V[:, cols].T
+        dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+        dQ[:, cols] = c * (dS @ K[:, cols])
+        dK[:, cols] = c * (dS.T @ Q[:, cols])
+    return dQ, dK, dV
+
+
+def window_self_attention_bwd(z, grid, window, shift, W, heads, dout, *, residual=True):
+    """Backward of window_self_attention on one batch item (one TCM branch).
+
+    out = (z +) roll(+s)(merge(Y_k)), Y_k = MHA(Z_k, Z_k) Wo^T over each window
+    Z_k of roll(-s)(z).  Given dout = dL/dout, returns
+    (dz, (dWq, dWk, dWv, dWo)): dL/dz and the weight gradients, each [D][D] in
+    the [out][in] storage of W.  Roll and window partition are permutations of
+    the rows, so their adjoints are the inverse permutations: the gradient rows
+    are gathered into windows exactly as z was, and scattered back the same
+    way.  Per window, with X = Z_k, A = attention output, dY = the window's
+    rows of dout:
+        dWo += dY^T A,  dA = dY Wo,  (dQ, dK, dV) = attention_heads_bwd(...),
+        dWq += dQ^T X,  dWk += dK^T X,  dWv += dV^T X,
+        dX = dQ Wq + dK Wk + dV Wv.
+    """
+    f, h, w = grid
+    z, dout = _f64(z), _f64(dout)
+    Wq, Wk, Wv, Wo = (_f64(x) for x in W)
+    N, D = z.shape
+    back = tuple(-s for s in shift)
+    zw = _to_windows(np.roll(z.reshape(f, h, w, D), shift=back, axis=(0, 1, 2)), window)
+    gw = _to_windows(np.roll(dout.reshape(f, h, w, D), shift=back, axis=(0, 1, 2)), window)
+    lab = window_region_labels(grid, window, shift)
+    dWq, dWk, dWv, dWo = (np.zeros((D, D)) for _ in range(4))
+    dxw = np.empty_like(zw)
+    for k in range(zw.shape[0]):
+        allow = lab[k][:, None] == lab[k][None, :]
+        X, dY = zw[k], gw[k]
+        Q, K, V = X @ Wq.T, X @ Wk.T, X @ Wv.T
+        A = attention_heads(Q, K, V, heads, allow)
+        dWo += dY.T @ A
+        dQ, dK, dV = attention_heads_bwd(Q, K, V, dY @ Wo, heads, allow)
+        dWq += dQ.T @ X
+        dWk += dK.T @ X
+        dWv += dV.T @ X
+        dxw[k] = dQ @ Wq + dK @ Wk + dV @ Wv
+    dz = np.roll(_from_windows(dxw, grid, window), shift=tuple(shift), axis=(0, 1, 2)).reshape(N, D)
+    if residual:
+        dz = dz + dout
+    return dz, (dWq, dWk, dWv, dWo)
 
 
 def tcm(z, grid, window, shift, W_wsa, W_swsa, heads, *, residual=True) -> np.ndarray:

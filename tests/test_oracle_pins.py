@@ -590,3 +590,132 @@ def test_pins_catch_a_wrong_mlp_term(monkeypatch):
     monkeypatch.setattr(O.ptdit_oracle, "mlp", lambda x, *w: real(x, *w) - x)
     with pytest.raises(AssertionError):
         test_pt_block_matches_library_composition()
+
+
+# ---------------------------------------------------------------- backward of a TCM branch
+
+BWD_CASES = [  # grid, window, shift: 2D and 3D windows, with and without the roll's wrap masks
+    ((1, 4, 4), (1, 2, 2), (0, 0, 0)),
+    ((1, 4, 4), (1, 2, 2), (0, 1, 1)),
+    ((2, 4, 4), (2, 2, 2), (1, 1, 1)),
+    ((2, 4, 6), (2, 2, 3), (1, 1, 2)),
+]
+
+
+def _bwd_inputs(grid, D, seed):
+    rng = np.random.default_rng(seed)
+    N = O.num_tokens(grid)
+    return rng.standard_normal((N, D)), rng.standard_normal((N, D)), _weights(D, seed + 1, scale=0.5)
+
+
+@pytest.mark.parametrize("grid,window,shift", BWD_CASES)
+def test_window_bwd_matches_finite_differences(grid, window, shift):
+    """Directional derivatives of L = <dout, out> by central differences in float64,
+    along random directions of z and of each weight matrix."""
+    D, heads = 8, 2
+    z, dout, W = _bwd_inputs(grid, D, 7)
+    dz, dW = O.window_self_attention_bwd(z, grid, window, shift, W, heads, dout)
+
+    def L(zz, WW):
+        return float(np.sum(dout * O.window_self_attention(zz, grid, window, shift, WW, heads)))
+
+    rng = np.random.default_rng(11)
+    eps = 1e-5
+    U = rng.standard_normal(z.shape)
+    fd = (L(z + eps * U, W) - L(z - eps * U, W)) / (2 * eps)
+    assert abs(fd - np.sum(dz * U)) <= 1e-7 * max(1.0, abs(fd))
+    for i in range(4):
+        V = rng.standard_normal(W[i].shape)
+        Wp, Wm = list(W), list(W)
+        Wp[i], Wm[i] = W[i] + eps * V, W[i] - eps * V
+        fd = (L(z, tuple(Wp)) - L(z, tuple(Wm))) / (2 * eps)
+        assert abs(fd - np.sum(dW[i] * V)) <= 1e-7 * max(1.0, abs(fd)), ("dW", i)
+
+
+def _torch_window_branch(z, grid, window, shift, W, heads):
+    """The TCM branch in torch ops (float64): roll, window partition, masked multi-head
+    attention, merge, roll back, residual; differentiated by autograd."""
+    f, h, w = grid
+    N, D = z.shape
+    wf, wh, ww = window
+    d = D // heads
+    zr = torch.roll(z.reshape(f, h, w, D), shifts=tuple(-s for s in shift), dims=(0, 1, 2))
+    x = zr.reshape(f // wf, wf, h // wh, wh, w // ww, ww, D).permute(0, 2, 4, 1, 3, 5, 6)
+    x = x.reshape(-1, wf * wh * ww, D)
+    # a pair attends iff the roll did not wrap between them along any axis: the last
+    # s positions of each axis of the rolled grid hold the tokens that wrapped around
+    pos = np.stack(np.meshgrid(np.arange(f), np.arange(h), np.arange(w), indexing="ij"), -1)
+    side = np.stack([(pos[..., a] >= [f, h, w][a] - shift[a]) & (shift[a] > 0)
+                     for a in range(3)], -1)
+    side = torch.from_numpy(side.reshape(f // wf, wf, h // wh, wh, w // ww, ww, 3)
+                            .transpose(0, 2, 4, 1, 3, 5, 6).reshape(x.shape[0], -1, 3))
+    allow = (side[:, :, None, :] == side[:, None, :, :]).all(-1)
+    Wq, Wk, Wv, Wo = W
+
+    def split(t):
+        return t.reshape(t.shape[0], t.shape[1], heads, d).transpose(1, 2)
+
+    q, k, v = split(x @ Wq.T), split(x @ Wk.T), split(x @ Wv.T)
+    s = (q @ k.transpose(-1, -2)) / math.sqrt(d)
+    s = s.masked_fill(~allow[:, None], float("-inf"))
+    a = (torch.softmax(s, dim=-1) @ v).transpose(1, 2).reshape(x.shape[0], -1, D)
+    y = (a @ Wo.T).reshape(f // wf, h // wh, w // ww, wf, wh, ww, D).permute(0, 3, 1, 4, 2, 5, 6)
+    y = torch.roll(y.reshape(f, h, w, D), shifts=tuple(shift), dims=(0, 1, 2)).reshape(N, D)
+    return z + y
+
+
+@pytest.mark.parametrize("grid,window,shift", BWD_CASES)
+def test_window_bwd_matches_autograd(grid, window, shift):
+    D, heads = 16, 4
+    z, dout, W = _bwd_inputs(grid, D, 21)
+    dz, dW = O.window_self_attention_bwd(z, grid, window, shift, W, heads, dout)
+    zt = torch.from_numpy(z).requires_grad_()
+    Wt = tuple(torch.from_numpy(x).requires_grad_() for x in W)
+    out = _torch_window_branch(zt, grid, window, shift, Wt, heads)
+    _close(out.detach().numpy(), O.window_self_attention(z, grid, window, shift, W, heads))
+    out.backward(torch.from_numpy(dout))
+    _close(dz, zt.grad.numpy())
+    for i in range(4):
+        _close(dW[i], Wt[i].grad.numpy())
+
+
+def test_window_bwd_without_residual_drops_dout():
+    grid, window, shift = BWD_CASES[2]
+    z, dout, W = _bwd_inputs(grid, 8, 3)
+    dz, dW = O.window_self_attention_bwd(z, grid, window, shift, W, 2, dout)
+    dz0, dW0 = O.window_self_attention_bwd(z, grid, window, shift, W, 2, dout, residual=False)
+    _close(dz0 + dout, dz)
+    for a, b in zip(dW, dW0):
+        _close(a, b)
+
+
+def test_pins_catch_a_dropped_softmax_jacobian_term(monkeypatch):
+    def no_rowsum(Q, K, V, dA, heads, allow=None):
+        d = Q.shape[1] // heads
+        c = 1.0 / math.sqrt(d)
+        dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+        for h in range(heads):
+            cols = slice(h * d, (h + 1) * d)
+            S = (Q[:, cols] @ K[:, cols].T) * c
+            if allow is not None:
+                S = np.where(allow, S, -np.inf)
+            P = O.softmax_rows(S)
+            dV[:, cols] = P.T @ dA[:, cols]
+            dS = P * (dA[:, cols] @ V[:, cols].T)  # the rowsum term is missing
+            dQ[:, cols] = c * (dS @ K[:, cols])
+            dK[:, cols] = c * (dS.T @ Q[:, cols])
+        return dQ, dK, dV
+
+    monkeypatch.setattr(O.ptdit_oracle, "attention_heads_bwd", no_rowsum)
+    assert _pin_fails(lambda: test_window_bwd_matches_finite_differences(*BWD_CASES[1]))
+
+
+def test_pins_catch_swapped_query_and_key_gradients(monkeypatch):
+    real = O.ptdit_oracle.attention_heads_bwd
+
+    def swapped(*a, **k):
+        dQ, dK, dV = real(*a, **k)
+        return dK, dQ, dV
+
+    monkeypatch.setattr(O.ptdit_oracle, "attention_heads_bwd", swapped)
+    assert _pin_fails(lambda: test_window_bwd_matches_finite_differences(*BWD_CASES[2]))
