@@ -22,7 +22,7 @@ PROXY_MODES = {"mean": PTDIT_PROXY_MEAN, "first": PTDIT_PROXY_FIRST, "random": P
 (PTDIT_OK, PTDIT_ERR_NULL, PTDIT_ERR_SHAPE, PTDIT_ERR_DTYPE, PTDIT_ERR_WORKSPACE, PTDIT_ERR_CUDA,
  PTDIT_ERR_TIMEOUT, PTDIT_ERR_ALIGN, PTDIT_ERR_ALIAS) = range(9)
 KINDS = ("average", "gemm", "attn_proxy", "attn_cross", "attn_window", "attn_dense", "norm",
-         "attn_text")
+         "attn_text", "attn_window_bwd", "wgrad", "transpose")
 
 # Every symbol declared in include/ptdit.h.
 EXPORTS = (
@@ -32,7 +32,7 @@ EXPORTS = (
     "ptdit_timing_read", "ptdit_launch_count", "ptdit_window_attn_static",
     "ptdit_debug_thl_map", "ptdit_debug_thl_units", "ptdit_debug_gemm_schedule",
     "ptdit_proxy_extract", "ptdit_giim_ex", "ptdit_pt_block", "ptdit_pt_block_workspace_bytes",
-    "ptdit_debug_wait_limit",
+    "ptdit_debug_wait_limit", "ptdit_window_attn_bwd", "ptdit_window_attn_bwd_workspace_bytes",
 )
 
 
@@ -51,6 +51,11 @@ class Shape(ctypes.Structure):
 class AttnW(ctypes.Structure):
     _fields_ = [("wq", ctypes.c_void_p), ("wk", ctypes.c_void_p), ("wv", ctypes.c_void_p),
                 ("wo", ctypes.c_void_p)]
+
+
+class AttnWgrad(ctypes.Structure):
+    _fields_ = [("dwq", ctypes.c_void_p), ("dwk", ctypes.c_void_p), ("dwv", ctypes.c_void_p),
+                ("dwo", ctypes.c_void_p)]
 
 
 class NormW(ctypes.Structure):
@@ -98,6 +103,10 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.c_size_t, _P]),
             "ptdit_tcm": (ctypes.c_int, [_S, _I3, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
                                          ctypes.c_size_t, _P]),
+            "ptdit_window_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
+            "ptdit_window_attn_bwd": (ctypes.c_int, [_S, _I3, _I3, _W, ctypes.c_uint, _P, _P, _P,
+                                                     ctypes.POINTER(AttnWgrad), _P,
+                                                     ctypes.c_size_t, _P]),
             "ptdit_block_attn": (ctypes.c_int, [_S, _I3, _I3, _I3, _W, _W, _W, _W, ctypes.c_uint,
                                                 _P, _P, _P, ctypes.c_size_t, _P]),
             "ptdit_full_attn": (ctypes.c_int, [_S, _W, ctypes.c_uint, _P, _P, _P,
@@ -325,6 +334,39 @@ def ptdit_window_attn(z_in, grid, window, shift, w, heads, flags=0, z_out=None, 
                                    ctypes.byref(ww), flags, _ptr(z_in), _ptr(z_out), _ptr(ws),
                                    ws.numel(), _stream(stream)))
     return z_out
+
+
+def window_attn_bwd_workspace(shape: Shape, window):
+    """A uint8 device buffer of ptdit_window_attn_bwd_workspace_bytes()."""
+    import torch
+    n = lib().ptdit_window_attn_bwd_workspace_bytes(ctypes.byref(shape), _i3(window))
+    if n == 0:
+        raise PtditError(PTDIT_ERR_SHAPE, "invalid shape or window")
+    return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+def ptdit_window_attn_bwd(z_in, dz_out, grid, window, shift, w, heads, flags=0, dz_in=None,
+                          dw=None, ws=None, stream=None):
+    """Backward of ptdit_window_attn: returns (dz_in, (dWq, dWk, dWv, dWo)), the weight
+    gradients fp32 [D, D]."""
+    import torch
+    _check_z(z_in)
+    _check_z(dz_out)
+    shape = make_shape(z_in, grid, heads)
+    if dz_in is None:
+        dz_in = torch.empty_like(z_in)
+    if dw is None:
+        dw = tuple(torch.empty(z_in.shape[-1], z_in.shape[-1], dtype=torch.float32,
+                               device=z_in.device) for _ in range(4))
+    if ws is None:
+        ws = window_attn_bwd_workspace(shape, window)
+    ww = attn_w(w)
+    g = AttnWgrad(*[_ptr(x) for x in dw])
+    _check(lib().ptdit_window_attn_bwd(ctypes.byref(shape), _i3(window), _i3(shift),
+                                       ctypes.byref(ww), flags, _ptr(z_in), _ptr(dz_out),
+                                       _ptr(dz_in), ctypes.byref(g), _ptr(ws), ws.numel(),
+                                       _stream(stream)))
+    return dz_in, tuple(dw)
 
 
 def ptdit_tcm(z_in, grid, window, shift, wsa, swsa, heads, flags=0, z_out=None, ws=None,

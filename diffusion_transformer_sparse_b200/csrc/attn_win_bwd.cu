@@ -1,0 +1,501 @@
+// Backward of window and shifted-window self-attention (one TCM branch of the
+// Qihoo-T2X reading note, §3 Method, Eq. TCM) on the tensor cores: given the
+// window tiles of Q, K, V and of dO = dL/d(attention output), it writes dQ, dK
+// and dV.  Per head, with S = c Q K^T (c = 1/sqrt(d), masked pairs -inf) and P
+// its row softmax:
+//   dV = P^T dO,   dP = dO V^T,   dS = P * (dP - rowsum(P * dP)),
+//   dQ = c dS K,   dK = c dS^T Q.
+// A window lies inside one 128-row tile (one window of 128 tokens, or two of
+// 64, four of 32, eight of 16 packed side by side), so every sum above stays
+// inside the tile: a unit (tile, head) needs nothing from any other unit.
+//
+// One persistent CTA per SM, units in the forward kernel's order (the heads
+// of one tile follow each other).  Two load buffers (Q, K, V, dO blocks of the
+// tiled head layout, thl.cuh) keep the next unit's loads in flight:
+//   warp 0       loader: four bulk copies per unit; the tile rows' key masks
+//                (window in tile x wrap bits, built with ballots as in the
+//                forward kernel) once per (batch item, tile) and buffer
+//   warp 1       MMA issuer: S = Q K^T and dP = dO V^T into TMEM (K-major
+//                operands); once the softmax warpgroup has written P and dS to
+//                shared memory: dV = P^T dO, dK = dS^T Q (P and dS read as
+//                MN-major A operands) and dQ = dS K (dS as K-major A), with
+//                dO, Q, K as MN-major B operands (head columns 0..63 with the
+//                128-byte swizzle, 64..79 with the 32-byte swizzle: an N = 64
+//                and an N = 16 MMA per K step).  dQ accumulates in dP's
+//                columns (the softmax has read dP by then), so the next unit's
+//                S is issued as soon as this unit's softmax has read S and dP,
+//                its dP once the epilogue has read dQ.
+//   warps 4-7    softmax warpgroup, thread r = query row r: the row max and
+//                sum over its window's keys, then P (normalised) and
+//                rowsum(P * dP), then dS (c folded in), written as bf16 rows of
+//                a 128 x 128 tile with the 128-byte swizzle; zeros for keys of
+//                other windows and for rows without a token.
+//   warps 8-11   epilogue, thread r = tile row r: dQ, dK, dV of row r (its
+//                token is both a query and a key of the window) to the
+//                row-major [B N, 3 D] gradient buffer (dQ, dK, dV column blocks,
+//                head h at columns h d .. h d + d - 1 of each).
+// TMEM (every accumulator and load starts on a 64-column boundary): S 0-127,
+// dP and then dQ 128-255, dV 256-383, dK 384-511 (head columns 0..63 at the
+// base, 64..79 at base + 64).  Every wait is bounded (2 s).
+#include "tc_util.cuh"
+#include "thl.cuh"
+
+namespace ptdit {
+namespace {
+
+using namespace tc;
+
+constexpr int BQ = 128;
+constexpr int kThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 128, T_DV = 256, T_DK = 384;
+constexpr int kMaskWords = 128;  // key masks per buffer, as in the forward kernel
+constexpr int NBUF = 2;
+
+template <int DPAD>
+struct BwdLayout {
+    static constexpr bool HAS_B = DPAD > 64;            // head columns 64..79
+    static constexpr int TILE_A = BQ * 128;             // columns 0..63, 128-byte swizzle
+    static constexpr int TILE_B = HAS_B ? BQ * 32 : 0;  // columns 64..79, 32-byte swizzle
+    static constexpr int TILE = TILE_A + TILE_B;
+    static constexpr int BUF = 4 * TILE;                // Q, K, V, dO of one unit
+    static constexpr int OFF_P = NBUF * BUF;            // P: 2 key halves x 128 rows x 128 B
+    static constexpr int OFF_DS = OFF_P + 2 * TILE_A;   // dS: same layout
+    static constexpr int OFF_INFO = OFF_DS + 2 * TILE_A;  // int8 info[NBUF][128]
+    static constexpr int OFF_MASK = OFF_INFO + NBUF * BQ; // uint32 kmask[NBUF][kMaskWords]
+    static constexpr int OFF_BAR = OFF_MASK + NBUF * kMaskWords * 4;
+    // ld_full[NBUF], buf_free[NBUF], s_full, dp_full, sp_free, pds_full, pds_free, acc_full,
+    // dq_free, acc_free, drain
+    static constexpr int NBARS = 2 * NBUF + 9;
+    static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
+    static_assert(TILE_A % 1024 == 0 && TILE % 1024 == 0, "swizzled tiles stay 1 KB aligned");
+    static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+struct BwdSched {
+    int tiles;  // tiles per batch item
+    int units;  // B x tiles x heads
+};
+
+// Byte offset of 16-byte chunk c (keys 8c .. 8c + 7) of row r in a 128 x 128
+// bf16 tile stored as two 64-key halves with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t pds_chunk(int r, int c) {
+    return (c >> 3) * (BQ * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+}
+
+template <int DPAD>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_win_bwd_kernel(const __grid_constant__ AttnArgs a, const void *__restrict__ dout,
+                        __nv_bfloat16 *__restrict__ dqkv, long ldg, BwdSched sc, int *status) {
+    using L = BwdLayout<DPAD>;
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    int8_t *info = reinterpret_cast<int8_t *>(sm + L::OFF_INFO);
+    uint32_t *kmask = reinterpret_cast<uint32_t *>(sm + L::OFF_MASK);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
+    uint64_t *ld_full = bars, *buf_free = bars + NBUF;
+    uint64_t *s_full = bars + 2 * NBUF, *dp_full = s_full + 1, *sp_free = s_full + 2;
+    uint64_t *pds_full = s_full + 3, *pds_free = s_full + 4, *acc_full = s_full + 5;
+    uint64_t *dq_free = s_full + 6, *acc_free = s_full + 7, *drain = s_full + 8;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
+    volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int d = a.d, n = a.geom.n, D = a.heads * a.d;
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&ld_full[b], 32);  // the loader's 32 lanes (masks) + the four blocks' bytes
+            mbar_init(&buf_free[b], 1);  // the unit's last MMA has read its blocks
+        }
+        mbar_init(s_full, 1);
+        mbar_init(dp_full, 1);
+        mbar_init(sp_free, BQ);
+        mbar_init(pds_full, BQ);
+        mbar_init(pds_free, 1);
+        mbar_init(acc_full, 1);
+        mbar_init(dq_free, BQ);
+        mbar_init(acc_free, BQ);
+        mbar_init(drain, 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(tslot, kTmemCols);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tslot;
+    pdl_wait();  // the projections that wrote Q, K, V and dO have completed
+    pdl_trigger();
+
+    const int u0 = (int)((long)blockIdx.x * sc.units / gridDim.x);
+    const int u1 = (int)((long)(blockIdx.x + 1) * sc.units / gridDim.x);
+    const int nunits = u1 - u0;  // local unit k: buffer k % NBUF
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ loader
+        const uint8_t *src[4] = {static_cast<const uint8_t *>(a.q), static_cast<const uint8_t *>(a.k),
+                                 static_cast<const uint8_t *>(a.v),
+                                 static_cast<const uint8_t *>(dout)};
+        const WinGeom &geo = a.geom;
+        const int pack = BQ / n;
+        int held0 = -1, held1 = -1;  // (batch item, tile) whose masks each buffer holds
+        for (int k = 0; k < nunits; ++k) {
+            const int u = u0 + k, bf = k % NBUF;
+            const int h = u % a.heads, rest = u / a.heads, tile = rest % sc.tiles,
+                      b = rest / sc.tiles;
+            if (!mbar_wait_warp(&buf_free[bf], ((k / NBUF) & 1) ^ 1, abort, status)) break;
+            if (lane == 0) {
+                const long blk = ((long)b * sc.tiles + tile) * a.heads + h;
+                mbar_expect_tx_only(&ld_full[bf], 4 * L::TILE);
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    bulk_load(sm + bf * L::BUF + m * L::TILE, src[m] + blk * L::TILE, L::TILE,
+                              &ld_full[bf]);
+            }
+            const int held = bf == 0 ? held0 : held1;
+            if (rest != held) {
+                if (bf == 0) held0 = rest; else held1 = rest;
+                int inf[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = q * 32 + lane;
+                    const int wit = r / n, win = tile * pack + wit, slot = r - wit * n;
+                    int in = -1;
+                    if (win < geo.nwin) {
+                        int wrap;
+                        (void)window_token(geo, win, slot, &wrap);
+                        in = wit * 8 + wrap;
+                    }
+                    inf[q] = in;
+                    info[bf * BQ + r] = static_cast<int8_t>(in);
+                }
+                const int nkeys = n < BQ ? (BQ / n) * 8 : 8;
+                for (int v = 0; v < nkeys; ++v) {
+                    const int half = n < BQ ? ((v >> 3) * n) >> 6 : 0;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t bits = __ballot_sync(0xffffffffu, inf[q] == v);
+                        if (lane == 0) {
+                            if (n >= BQ)
+                                kmask[bf * kMaskWords + v * 4 + q] = bits;
+                            else if ((q >> 1) == half)
+                                kmask[bf * kMaskWords + v * 2 + (q & 1)] = bits;
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            mbar_arrive(&ld_full[bf]);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(BQ, BQ);                 // K-major A and B
+            constexpr uint32_t id_mm64 = idesc_bf16(BQ, 64, true, true);  // MN-major A and B
+            constexpr uint32_t id_mm16 = idesc_bf16(BQ, 16, true, true);
+            constexpr uint32_t id_km64 = idesc_bf16(BQ, 64, true, false); // K-major A, MN-major B
+            constexpr uint32_t id_km16 = idesc_bf16(BQ, 16, true, false);
+            const uint32_t aP = smem_u32(sm + L::OFF_P), aDS = smem_u32(sm + L::OFF_DS);
+            bool ok = true, any = false;
+            // X (rows x head columns) times Y^T into TMEM column d_col
+            auto scores = [&](uint32_t d_col, uint32_t aX, uint32_t aY) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + d_col, sdesc_sw128(aX + kk * 32), sdesc_sw128(aY + kk * 32), id_s,
+                             kk > 0);
+                if (L::HAS_B)
+                    mma_bf16(tmem + d_col, sdesc_sw32(aX + L::TILE_A), sdesc_sw32(aY + L::TILE_A),
+                             id_s, 1);
+            };
+            // S = Q K^T of unit k (waits for its blocks)
+            auto issue_s = [&](int k) {
+                const int bf = k % NBUF;
+                if (!mbar_wait(&ld_full[bf], (k / NBUF) & 1, abort, status)) return false;
+                fence_after_sync();
+                const uint32_t aQ = smem_u32(sm + bf * L::BUF);
+                scores(T_S, aQ, aQ + L::TILE);
+                mma_commit(s_full);
+                any = true;
+                return true;
+            };
+            // dP = dO V^T of unit k (its blocks are in, S(k) waited for them)
+            auto issue_dp = [&](int k) {
+                const uint32_t aQ = smem_u32(sm + (k % NBUF) * L::BUF);
+                scores(T_DP, aQ + 3 * L::TILE, aQ + 2 * L::TILE);
+                mma_commit(dp_full);
+            };
+            // D (rows of the reduction: K steps of 16) += A^T-or-A times the head
+            // columns of the MN-major B operand at aB (N = 64, then N = 16)
+            auto grad = [&](uint32_t d_col, uint64_t a_desc, uint32_t aB, int ks, bool a_mn) {
+                mma_bf16(tmem + d_col, a_desc, sdesc_sw128_mn(aB + ks * 2048, L::TILE_A),
+                         a_mn ? id_mm64 : id_km64, ks > 0);
+                if (L::HAS_B)
+                    mma_bf16(tmem + d_col + 64, a_desc, sdesc_sw32_mn(aB + L::TILE_A + ks * 512),
+                             a_mn ? id_mm16 : id_km16, ks > 0);
+            };
+            auto issue_grads = [&](int k) {
+                const int bf = k % NBUF;
+                if (!mbar_wait(pds_full, k & 1, abort, status)) return false;
+                if (k > 0 && !mbar_wait(acc_free, (k - 1) & 1, abort, status)) return false;
+                fence_after_sync();
+                const uint32_t aQ = smem_u32(sm + bf * L::BUF), aK = aQ + L::TILE,
+                               aO = aQ + 3 * L::TILE;
+#pragma unroll
+                for (int ks = 0; ks < BQ / 16; ++ks) {
+                    // A = P^T / dS^T: the 16 query rows ks of the tile, MN-major (keys contiguous)
+                    const uint64_t pT = sdesc_sw128_mn(aP + ks * 2048, L::TILE_A);
+                    const uint64_t sT = sdesc_sw128_mn(aDS + ks * 2048, L::TILE_A);
+                    // A = dS: keys 16 ks .. 16 ks + 15 of every query row, K-major
+                    const uint64_t sK = sdesc_sw128(aDS + (ks >> 2) * L::TILE_A + (ks & 3) * 32);
+                    grad(T_DV, pT, aO, ks, true);   // dV += P^T dO
+                    grad(T_DK, sT, aQ, ks, true);   // dK += dS^T Q
+                    grad(T_DQ, sK, aK, ks, false);  // dQ += dS K
+                }
+                mma_commit(acc_full);
+                mma_commit(pds_free);
+                mma_commit(&buf_free[bf]);
+                return true;
+            };
+            if (nunits > 0) {
+                ok = issue_s(0);
+                if (ok) issue_dp(0);
+            }
+            for (int k = 0; k < nunits && ok; ++k) {
+                // the softmax has read this unit's S and dP: the next S may overwrite S,
+                // and the gradients (dQ in dP's columns) may start
+                if (!mbar_wait(sp_free, k & 1, abort, status)) break;
+                if (k + 1 < nunits) ok = issue_s(k + 1);
+                if (ok) ok = issue_grads(k);
+                if (ok && k + 1 < nunits) {
+                    // the epilogue has read dQ(k) out of dP's columns
+                    if (!mbar_wait(dq_free, k & 1, abort, status)) break;
+                    fence_after_sync();
+                    issue_dp(k + 1);
+                }
+            }
+            if (any) {  // every issued MMA has finished before TMEM is released
+                mma_commit(drain);
+                volatile int never = 0;
+                mbar_wait(drain, 0, &never, status);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ softmax warpgroup
+        const int r = (warp % 4) * 32 + lane;  // query row of the tile = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + T_S, t_dp = tmem + lane_base + T_DP;
+        const float c = a.scale, sl2 = a.scale * 1.4426950408889634f;
+        uint8_t *sP = sm + L::OFF_P, *sDS = sm + L::OFF_DS;
+        // this row's keys: its window's 64-key half of the tile (windows of up to 64
+        // tokens lie inside one half), or all 128 keys
+        const int c_lo = n < BQ ? (r >> 6) << 6 : 0, nk = n < BQ ? 64 : 128;
+        for (int k = 0; k < nunits; ++k) {
+            const int bf = k % NBUF;
+            if (!mbar_wait_warp(&ld_full[bf], (k / NBUF) & 1, abort, status)) break;
+            const int qi = info[bf * BQ + r];
+            uint32_t allow[4] = {0u, 0u, 0u, 0u};
+            if (qi >= 0) {
+                if (n < BQ) {
+                    allow[0] = kmask[bf * kMaskWords + qi * 2];
+                    allow[1] = kmask[bf * kMaskWords + qi * 2 + 1];
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) allow[q] = kmask[bf * kMaskWords + qi * 4 + q];
+                }
+            }
+            if (!mbar_wait_warp(s_full, k & 1, abort, status)) break;
+            fence_after_sync();
+            // pass 1: row max over the allowed keys; pass 2: the row sum
+            float m = -INFINITY;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                if (jj * 32 >= nk) break;
+                uint32_t sv[32];
+                tmem_ld32(t_s + c_lo + jj * 32, sv);
+                tmem_ld_wait();
+                const uint32_t w = allow[jj];
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if ((w >> e) & 1u) m = fmaxf(m, __uint_as_float(sv[e]));
+            }
+            const float ms = m * sl2;
+            float l = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                if (jj * 32 >= nk) break;
+                uint32_t sv[32];
+                tmem_ld32(t_s + c_lo + jj * 32, sv);
+                tmem_ld_wait();
+                const uint32_t w = allow[jj];
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if ((w >> e) & 1u) l += ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -ms));
+            }
+            // P = 2^(s sl2 - ms - log2 l); a row without a token has no allowed key
+            const float off = qi >= 0 ? ms + __log2f(l) : 0.f;
+            // the previous unit's MMAs have read P and dS; this unit's dP is in
+            if (!mbar_wait_warp(pds_free, (k & 1) ^ 1, abort, status)) break;
+            if (!mbar_wait_warp(dp_full, k & 1, abort, status)) break;
+            fence_after_sync();
+            // pass 3: P to shared memory and delta = rowsum(P * dP)
+            float delta = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                if (jj * 32 >= nk) break;
+                const int j = jj * 32;
+                uint32_t sv[32], dv[32];
+                tmem_ld32(t_s + c_lo + j, sv);
+                tmem_ld32(t_dp + c_lo + j, dv);
+                tmem_ld_wait();
+                const uint32_t w = allow[jj];
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = ((w >> e) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -off)) : 0.f;
+                    const float p1 = ((w >> (e + 1)) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -off)) : 0.f;
+                    pk[e / 2] = pack_bf16(p0, p1);
+                    // delta from the bf16 weights the MMAs use
+                    const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e / 2]));
+                    delta = fmaf(pr.x, __uint_as_float(dv[e]), delta);
+                    delta = fmaf(pr.y, __uint_as_float(dv[e + 1]), delta);
+                }
+                const int c0 = (c_lo + j) >> 3;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(sP + pds_chunk(r, c0 + q)) =
+                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            }
+            // pass 4: dS = c P (dP - delta)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                if (jj * 32 >= nk) break;
+                const int j = jj * 32;
+                uint32_t dv[32];
+                tmem_ld32(t_dp + c_lo + j, dv);
+                tmem_ld_wait();
+                const int c0 = (c_lo + j) >> 3;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 p4 = *reinterpret_cast<const uint4 *>(sP + pds_chunk(r, c0 + q));
+                    const uint32_t pw[4] = {p4.x, p4.y, p4.z, p4.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[t]));
+                        const int e = 8 * q + 2 * t;
+                        o[t] = pack_bf16(c * pr.x * (__uint_as_float(dv[e]) - delta),
+                                         c * pr.y * (__uint_as_float(dv[e + 1]) - delta));
+                    }
+                    *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, c0 + q)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+            fence_before_sync();
+            mbar_arrive(sp_free);  // S and dP are read
+            // the keys of the other windows of the tile: zero weights and gradients
+            if (n < BQ) {
+                const int o0 = (64 - c_lo) >> 3;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    *reinterpret_cast<uint4 *>(sP + pds_chunk(r, o0 + q)) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, o0 + q)) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_async_smem();  // the tensor cores read what these threads wrote
+            mbar_arrive(pds_full);
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ epilogue
+        const int r = (warp % 4) * 32 + lane;  // tile row = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
+        const WinGeom &geo = a.geom;
+        const int pack = BQ / n, nch = d / 8;
+        for (int k = 0; k < nunits; ++k) {
+            const int u = u0 + k;
+            const int h = u % a.heads, rest = u / a.heads, tile = rest % sc.tiles,
+                      b = rest / sc.tiles;
+            const int wit = r / n, win = tile * pack + wit, slot = r - wit * n;
+            long row = -1;
+            if (win < geo.nwin) {
+                int wrap;
+                row = (long)b * a.k_bstride + window_token(geo, win, slot, &wrap);
+            }
+            if (!mbar_wait_warp(acc_full, k & 1, abort, status)) break;
+            fence_after_sync();
+            __nv_bfloat16 *dst = row >= 0 ? dqkv + row * ldg + (long)h * d : nullptr;
+#pragma unroll
+            for (int m = 0; m < 3; ++m) {
+                uint32_t v[DPAD];
+                const uint32_t t = tmem + lane_base + (m == 0 ? T_DQ : (m == 1 ? T_DK : T_DV));
+                tmem_ld32(t, *reinterpret_cast<uint32_t(*)[32]>(v));
+                tmem_ld32(t + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                if (DPAD > 64) tmem_ld16(t + 64, *reinterpret_cast<uint32_t(*)[16]>(v + 64));
+                tmem_ld_wait();
+                if (m == 0) {  // dQ is out of dP's columns: the next dP may go there
+                    fence_before_sync();
+                    mbar_arrive(dq_free);
+                }
+                if (row >= 0) {
+#pragma unroll
+                    for (int uu = 0; uu < DPAD / 8; ++uu)
+                        if (uu < nch) {
+                            uint4 o;
+                            o.x = pack_bf16(__uint_as_float(v[8 * uu + 0]), __uint_as_float(v[8 * uu + 1]));
+                            o.y = pack_bf16(__uint_as_float(v[8 * uu + 2]), __uint_as_float(v[8 * uu + 3]));
+                            o.z = pack_bf16(__uint_as_float(v[8 * uu + 4]), __uint_as_float(v[8 * uu + 5]));
+                            o.w = pack_bf16(__uint_as_float(v[8 * uu + 6]), __uint_as_float(v[8 * uu + 7]));
+                            *reinterpret_cast<uint4 *>(dst + (long)m * D + 8 * uu) = o;
+                        }
+                }
+            }
+            fence_before_sync();
+            mbar_arrive(acc_free);  // the next unit's gradient MMAs may overwrite TMEM
+        }
+    }
+    if (*abort) {
+        // a wait gave up: let bulk copies still in flight into this CTA land
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 100000) {
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int DPAD>
+cudaError_t launch_bwd(const AttnArgs &a, const void *dout, void *dqkv, long ldg, cudaStream_t s) {
+    using L = BwdLayout<DPAD>;
+    int *status = device_status_ptr();
+    if (!status) return cudaErrorInvalidValue;
+    if (a.tq.mode != THL_WINDOW || a.tk.mode != THL_WINDOW || a.tv.mode != THL_WINDOW ||
+        a.tq.vpad || a.tk.vpad || a.tv.vpad || L::TILE != (int)thl_block_bytes(a.d, 0))
+        return cudaErrorInvalidValue;
+    BwdSched sc;
+    const int pack = BQ / a.geom.n;
+    sc.tiles = (a.geom.nwin + pack - 1) / pack;
+    sc.units = a.B * sc.tiles * a.heads;
+    const int sms = num_sms() > 0 ? num_sms() : 148;
+    const int grid = sc.units < sms ? sc.units : sms;
+    cudaError_t e = cudaFuncSetAttribute(attn_win_bwd_kernel<DPAD>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(attn_win_bwd_kernel<DPAD>, dim3(grid), dim3(kThreads), L::BYTES, s, a, dout,
+                      static_cast<__nv_bfloat16 *>(dqkv), ldg, sc, status);
+}
+
+}  // namespace
+
+cudaError_t launch_attention_win_bwd(const AttnArgs &a, const void *dout, void *dqkv, long ldg,
+                                     cudaStream_t s) {
+    if (a.d < 8 || a.d > 80 || a.d % 8) return cudaErrorInvalidValue;
+    const int n = a.geom.n;
+    if (n != 16 && n != 32 && n != 64 && n != 128) return cudaErrorInvalidValue;
+    return a.d <= 64 ? launch_bwd<64>(a, dout, dqkv, ldg, s) : launch_bwd<80>(a, dout, dqkv, ldg, s);
+}
+
+}  // namespace ptdit

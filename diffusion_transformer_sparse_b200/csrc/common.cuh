@@ -215,6 +215,29 @@ __device__ __forceinline__ float gelu_tanh_fast(float x) {
 cudaError_t launch_layer_norm(int dtype, long rows, int D, const void *x, const void *gamma,
                               const void *beta, float eps, void *y, cudaStream_t s);
 cudaError_t launch_gemm(const GemmArgs &a, cudaStream_t s);
+
+// Weight gradients dW_i = G_i^T X_i (fp32 [M][N], added into zeroed outputs):
+// G_i is columns gcol[i] .. gcol[i] + M - 1 of the row-major gradient buffer
+// G[src[i]] (ldg columns), X_i the first N columns of X[src[i]] (ldx columns),
+// both over `rows` token rows (the reduction).
+constexpr int kWgradMax = 4;
+struct WgradArgs {
+    const void *G[2];
+    int ldg[2];
+    const void *X[2];
+    int ldx[2];
+    int nmat;
+    int src[kWgradMax], gcol[kWgradMax];
+    float *dW[kWgradMax];
+    int M, N, rows;
+};
+bool wgrad_supported(const WgradArgs &a);
+cudaError_t launch_wgrad(const WgradArgs &a, cudaStream_t s);
+
+// dst[c][r] = src[r][c] for a row-major bf16 [rows][cols] matrix (dst has
+// row stride ldd >= rows, so several transposes can fill one wider matrix).
+cudaError_t launch_transpose_bf16(const void *src, int rows, int cols, void *dst, long ldd,
+                                  cudaStream_t s);
 // The 2-SM projection GEMM's tile order for rows x nseg outputs of nmat
 // matrices on `pairs` CTA pairs (host only): *tiles, and *scheduled = 1 with
 // pair q taking tile[first[q]] .. tile[first[q+1] - 1] when the launch runs a
@@ -242,6 +265,11 @@ struct AttnArgs {
     ThlDesc tq, tk, tv;            // layouts of q, k, v (mode 0: row-major with ldq...)
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s);
+// Backward of window attention: a holds the window tiles of Q, K, V (tiled
+// head layout), dout those of dL/dO; writes dQ, dK, dV as the column blocks
+// [0, D), [D, 2D), [2D, 3D) of the row-major [B N][ldg] buffer dqkv.
+cudaError_t launch_attention_win_bwd(const AttnArgs &a, const void *dout, void *dqkv, long ldg,
+                                     cudaStream_t s);
 
 // Debug maps written with the kernels' own index functions.
 cudaError_t launch_debug_proxy_map(const ProxyGeom &g, int32_t *out, cudaStream_t s);

@@ -717,6 +717,131 @@ int check_w_alias(const Dims &d, const ptdit_attn_w *w, const void *z_out) {
     return PTDIT_OK;
 }
 
+// ------------------------------------------------------------------ backward of a TCM branch
+struct WsBwd {
+    size_t Q, K, V, dO, A, G, WoT, WqkvT, total;
+};
+
+// Q, K, V and dO window tiles, the recomputed attention output A, the
+// gradient rows [dQ dK dV] (B N x 3 D) and the transposed weights.
+WsBwd ws_layout_bwd(const Dims &d) {
+    WsBwd L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    const size_t tq = thl_bytes(d, d.N, 0), tn = (size_t)d.B * d.N * d.D * d.elem;
+    L.Q = take(tq); L.K = take(tq); L.V = take(tq); L.dO = take(tq);
+    L.A = take(tn); L.G = take(3 * tn);
+    L.WoT = take((size_t)d.D * d.D * d.elem);
+    L.WqkvT = take((size_t)3 * d.D * d.D * d.elem);
+    L.total = off;
+    return L;
+}
+
+int check_bwd_shape(const Dims &d, const WinGeom &wg) {
+    if (d.dtype != PTDIT_BF16)
+        return fail(PTDIT_ERR_DTYPE, "the backward runs in bf16 only (tensor cores)");
+    TRY(check_bf16_attention(d, &wg));
+    if (d.D % 128)
+        return fail(PTDIT_ERR_SHAPE,
+                    "the backward's weight-gradient kernel takes D a multiple of 128; D=%d", d.D);
+    return PTDIT_OK;
+}
+
+int transpose(const Run &r, const void *src, int rows, int cols, void *dst, long ldd) {
+    TRY(launch_fault("weight transpose"));
+    timing_begin(PTDIT_K_TRANSPOSE, r.s);
+    cudaError_t e = launch_transpose_bf16(src, rows, cols, dst, ldd, r.s);
+    timing_end(r.s);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "weight transpose");
+}
+
+int run_window_bwd(const Run &r, const WsBwd &Lb, const WinGeom &wg, const ptdit_attn_w *w,
+                   unsigned flags, const void *z_in, const void *dz_out, void *dz_in,
+                   const ptdit_attn_wgrad *dw) {
+    const Dims &d = r.d;
+    const long BN = (long)d.B * d.N;
+    void *Q = r.at(Lb.Q), *K = r.at(Lb.K), *V = r.at(Lb.V), *dO = r.at(Lb.dO);
+    void *A = r.at(Lb.A), *G = r.at(Lb.G), *WoT = r.at(Lb.WoT), *WqkvT = r.at(Lb.WqkvT);
+    AttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.mode = ATT_WINDOW;
+    a.dtype = d.dtype;
+    a.d = d.d;
+    a.q = Q; a.k = K; a.v = V; a.o = A;
+    a.q_bstride = a.k_bstride = d.N;
+    a.geom = wg;
+    const ThlDesc tw = thl_window(wg, d.N, 0);
+    const ThlDesc twv = thl_window(wg, d.N, 0, v_ones(d));
+    a.tq = a.tk = tw;
+    a.tv = twv;
+    // the branch recomputed from its input: Q, K, V and the attention output A
+    {
+        const void *W[3] = {w->wq, w->wk, w->wv};
+        void *C[3] = {Q, K, V};
+        const ThlDesc *T[3] = {&tw, &tw, &twv};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 3, W, C, T, "backward: QKV projection"));
+    }
+    TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "backward: window attention"));
+    // W^T for the input gradients: dA = dz_out Wo, dx = [dQ dK dV] [Wq; Wk; Wv]
+    TRY(transpose(r, w->wo, d.D, d.D, WoT, d.D));
+    const void *Wi[3] = {w->wq, w->wk, w->wv};
+    for (int i = 0; i < 3; ++i)
+        TRY(transpose(r, Wi[i], d.D, d.D, static_cast<char *>(WqkvT) + (size_t)i * d.D * d.elem,
+                      3L * d.D));
+    {
+        const void *W[3] = {WoT, nullptr, nullptr};
+        void *C[3] = {dO, nullptr, nullptr};
+        const ThlDesc *T[3] = {&tw, nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, dz_out, BN, 1, W, C, T, "backward: dA = dz_out Wo"));
+    }
+    // dQ, dK, dV per window and head
+    a.heads = d.heads;
+    a.B = d.B;
+    a.ldq = a.ldk = a.ldv = a.ldo = d.D;
+    a.scale = 1.0f / sqrtf((float)d.d);
+    TRY(launch_fault("window attention backward"));
+    timing_begin(PTDIT_K_ATTN_WINDOW_BWD, r.s);
+    cudaError_t e = launch_attention_win_bwd(a, dO, G, 3L * d.D, r.s);
+    timing_end(r.s);
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, "window attention backward");
+    // dz_in = (dz_out +) [dQ dK dV] [Wq; Wk; Wv]
+    TRY(gemm_ex(r, PTDIT_K_GEMM, G, BN, 3 * d.D, d.D, WqkvT, dz_in,
+                (flags & PTDIT_NO_RESIDUAL) ? nullptr : dz_out, nullptr, ACT_NONE,
+                "backward: input gradient"));
+    // weight gradients: dW{q,k,v} = [dQ dK dV]^T z_in, dWo = dz_out^T A
+    float *outs[4] = {dw->dwq, dw->dwk, dw->dwv, dw->dwo};
+    for (int i = 0; i < 4; ++i) {
+        cudaError_t em = cudaMemsetAsync(outs[i], 0, (size_t)d.D * d.D * sizeof(float), r.s);
+        if (em != cudaSuccess) return cuda_fail(em, "zeroing the weight gradients");
+    }
+    WgradArgs g;
+    memset(&g, 0, sizeof g);
+    g.G[0] = G; g.ldg[0] = 3 * d.D; g.X[0] = z_in; g.ldx[0] = d.D;
+    g.G[1] = dz_out; g.ldg[1] = d.D; g.X[1] = A; g.ldx[1] = d.D;
+    g.nmat = 4;
+    const int src[4] = {0, 0, 0, 1}, col[4] = {0, d.D, 2 * d.D, 0};
+    for (int i = 0; i < 4; ++i) {
+        g.src[i] = src[i];
+        g.gcol[i] = col[i];
+        g.dW[i] = outs[i];
+    }
+    g.M = g.N = d.D;
+    g.rows = (int)BN;
+    if (!wgrad_supported(g)) return cuda_fail(cudaErrorNotSupported, "weight gradients");
+    TRY(launch_fault("weight gradients"));
+    timing_begin(PTDIT_K_WGRAD, r.s);
+    e = launch_wgrad(g, r.s);
+    timing_end(r.s);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "weight gradients");
+}
+
 }  // namespace
 
 namespace ptdit {
@@ -899,6 +1024,56 @@ int ptdit_window_attn(const ptdit_shape *shape, const int window[3], const int s
     TRY(check_ws(d, 0, ws, ws_bytes, &L));
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
     return run_window(r, wg, w, flags, z_in, z_out);
+}
+
+size_t ptdit_window_attn_bwd_workspace_bytes(const ptdit_shape *shape, const int window[3]) {
+    Dims d;
+    if (check_shape(shape, &d) != PTDIT_OK) return 0;
+    const int zero[3] = {0, 0, 0};
+    WinGeom wg;
+    if (make_window(d, window, zero, &wg) != PTDIT_OK) return 0;
+    return ws_layout_bwd(d).total;
+}
+
+int ptdit_window_attn_bwd(const ptdit_shape *shape, const int window[3], const int shift[3],
+                          const ptdit_attn_w *w, unsigned flags, const void *z_in,
+                          const void *dz_out, void *dz_in, const ptdit_attn_wgrad *dw, void *ws,
+                          size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    WinGeom wg;
+    TRY(check_shape(shape, &d));
+    TRY(make_window(d, window, shift, &wg));
+    TRY(check_bwd_shape(d, wg));
+    TRY(check_weights(w, "w"));
+    TRY(check_io(d, z_in, dz_in, ws, ws_bytes));
+    TRY(check_ptr(dz_out, "dz_out"));
+    TRY(check_w_alias(d, w, dz_in));
+    if (!dw) return fail(PTDIT_ERR_NULL, "dw is NULL");
+    const size_t zb = (size_t)d.B * d.N * d.D * d.elem, gb = (size_t)d.D * d.D * sizeof(float);
+    if (overlap(dz_out, zb, dz_in, zb)) return fail(PTDIT_ERR_ALIAS, "dz_in overlaps dz_out");
+    if (ws && overlap(ws, ws_bytes, dz_out, zb))
+        return fail(PTDIT_ERR_ALIAS, "dz_out overlaps the workspace");
+    float *outs[4] = {dw->dwq, dw->dwk, dw->dwv, dw->dwo};
+    const char *nm[4] = {"dw.dwq", "dw.dwk", "dw.dwv", "dw.dwo"};
+    for (int i = 0; i < 4; ++i) {
+        TRY(check_ptr(outs[i], nm[i]));
+        if (overlap(outs[i], gb, dz_in, zb) || overlap(outs[i], gb, z_in, zb) ||
+            overlap(outs[i], gb, dz_out, zb) || (ws && overlap(outs[i], gb, ws, ws_bytes)))
+            return fail(PTDIT_ERR_ALIAS, "%s overlaps another argument or the workspace", nm[i]);
+        for (int j = 0; j < i; ++j)
+            if (overlap(outs[i], gb, outs[j], gb))
+                return fail(PTDIT_ERR_ALIAS, "%s overlaps %s", nm[i], nm[j]);
+    }
+    const WsBwd Lb = ws_layout_bwd(d);
+    if (fault("workspace"))
+        return fail(PTDIT_ERR_WORKSPACE, "workspace refused (PTDIT_FAULT=workspace)");
+    if (!ws) return fail(PTDIT_ERR_NULL, "workspace is NULL");
+    if ((uintptr_t)ws % 256) return fail(PTDIT_ERR_ALIGN, "workspace is not 256-byte aligned");
+    if (ws_bytes < Lb.total)
+        return fail(PTDIT_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, Lb.total);
+    const Ws none{};
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), none};
+    return run_window_bwd(r, Lb, wg, w, flags, z_in, dz_out, dz_in, dw);
 }
 
 int ptdit_tcm(const ptdit_shape *shape, const int window[3], const int shift[3],

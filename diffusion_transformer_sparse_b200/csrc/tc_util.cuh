@@ -395,10 +395,13 @@ __device__ __forceinline__ uint64_t sdesc_interleave(uint32_t saddr, uint32_t lb
 
 // Instruction descriptor of tcgen05.mma.kind::f16: fp32 accumulator (bits
 // 4-5 = 1), A and B bf16 (bits 7-9 and 10-12 = 1), both K-major unless
-// b_mn_major, N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major = false) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+// a_mn_major (bit 15) or b_mn_major (bit 16), N >> 3 in bits 17-22, M >> 4 in
+// bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major = false,
+                                                  bool a_mn_major = false) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // 16-byte asynchronous global -> shared copy through L2; src_bytes < 16

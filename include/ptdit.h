@@ -183,6 +183,37 @@ int ptdit_window_attn_static(const ptdit_shape *shape, const int window[3], cons
                              void *z_out, ptdit_stream_t stream);
 
 /*
+ * ptdit_window_attn_bwd -- backward (training) of ptdit_window_attn: given the
+ *   branch input z_in and dz_out = dL/dz_out, writes dz_in = dL/dz_in and the
+ *   four weight gradients dL/dWq, dL/dWk, dL/dWv, dL/dWo.  With
+ *   PTDIT_NO_RESIDUAL the branch had no residual (dz_in then omits dz_out).
+ *   The branch is recomputed from z_in (Q, K, V and the attention output);
+ *   per window and head the chain rule is the standard one for softmax
+ *   attention: dV = P^T dA, dP = dA V^T, dS = P * (dP - rowsum(P * dP)),
+ *   dQ = c dS K, dK = c dS^T Q (c = 1/sqrt(d), dA = dz_out Wo), then
+ *   dz_in = (dz_out +) roll back of [dQ dK dV] [Wq; Wk; Wv] and
+ *   dW = (gradient)^T (input) summed over all B N tokens.
+ *   Arguments: z_in, dz_out [B, N, D] bf16; dz_in [B, N, D] bf16 (must not
+ *   overlap any other argument); dw: four fp32 [D][D] row-major arrays in
+ *   the weights' [out][in] layout, overwritten (zeroed on `stream`, then the
+ *   token slices' contributions are added with atomic vector reductions, so
+ *   the summation order varies from run to run at fp32 rounding level).
+ *   Workspace: ptdit_window_attn_bwd_workspace_bytes(shape, window) bytes,
+ *   256-byte aligned, contents garbage after the call.
+ *   Supported: dtype PTDIT_BF16 only, D a multiple of 128, head widths 8..80
+ *   in steps of 8, windows of 16, 32, 64 or 128 tokens; anything else returns
+ *   PTDIT_ERR_SHAPE (PTDIT_ERR_DTYPE for PTDIT_F32) and launches nothing.
+ */
+typedef struct {
+    float *dwq, *dwk, *dwv, *dwo;
+} ptdit_attn_wgrad;
+size_t ptdit_window_attn_bwd_workspace_bytes(const ptdit_shape *shape, const int window[3]);
+int ptdit_window_attn_bwd(const ptdit_shape *shape, const int window[3], const int shift[3],
+                          const ptdit_attn_w *w, unsigned flags, const void *z_in,
+                          const void *dz_out, void *dz_in, const ptdit_attn_wgrad *dw, void *ws,
+                          size_t ws_bytes, ptdit_stream_t stream);
+
+/*
  * ptdit_tcm -- Eq. TCM: WSA with weights wsa, then SWSA with weights swsa
  *   and the given shift, each with its residual (unless PTDIT_NO_RESIDUAL).
  */
@@ -338,7 +369,10 @@ enum {
     PTDIT_K_ATTN_DENSE = 5,/* full self-attention core */
     PTDIT_K_NORM = 6,      /* LayerNorm of the complete block */
     PTDIT_K_ATTN_TEXT = 7, /* text cross-attention core of the complete block */
-    PTDIT_K_COUNT = 8
+    PTDIT_K_ATTN_WINDOW_BWD = 8, /* window attention core, backward */
+    PTDIT_K_WGRAD = 9,     /* weight gradients of the projections */
+    PTDIT_K_TRANSPOSE = 10,/* weight transposes of the backward */
+    PTDIT_K_COUNT = 11
 };
 int ptdit_timing_enable(int max_launches);
 int ptdit_timing_read(int *kind, float *ms, int max);

@@ -1,0 +1,94 @@
+"""Backward of one TCM branch (ptdit_window_attn_bwd) on the GPU against the
+float64 oracle's hand-derived gradients (pinned on the CPU by finite
+differences and autograd): dL/dz and the four weight gradients, whole tensors,
+at shapes that reach every window size, head width, the roll's wrap masks and a
+ragged last tile, and at a full-size workload in the bench's launch
+configuration (persistent kernels with many units per CTA, split-K weight
+gradients over all tokens)."""
+import numpy as np
+import pytest
+import torch
+
+import diffusion_transformer_sparse_b200 as pt
+import oracle as O
+from diffusion_transformer_sparse_b200 import build, synth
+from tests.helpers import TOL, Case, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    pt.lib()
+
+
+def _dout(B, N, D, seed=500):
+    return torch.stack([synth.latent(N, D, seed + b, "bf16") for b in range(B)])
+
+
+def _check(c, window, shift, flags=0):
+    dout_cpu = _dout(c.B, c.N, c.D)
+    dz, dw = pt.ptdit_window_attn_bwd(c.z, dout_cpu.cuda(), c.grid, window, shift, c.w["wsa"],
+                                      c.heads, flags)
+    dz = c.out64(dz)
+    dw = [c.out64(x) for x in dw]
+    g64 = synth.as_f64(dout_cpu)
+    want_w = [np.zeros((c.D, c.D)) for _ in range(4)]
+    for b in range(c.B):
+        wdz, wdw = O.window_self_attention_bwd(c.z64[b], c.grid, window, shift, c.w64["wsa"],
+                                               c.heads, g64[b], residual=not flags)
+        assert rel_err(dz[b], wdz) <= TOL["bf16"], ("dz", b)
+        for i in range(4):
+            want_w[i] += wdw[i]
+    for i, name in enumerate(("dWq", "dWk", "dWv", "dWo")):
+        assert rel_err(dw[i], want_w[i]) <= TOL["bf16"], name
+
+
+CASES = [  # grid, D, heads, window, shift
+    ((1, 16, 16), 128, 2, (1, 8, 8), (0, 0, 0)),    # 2D windows of 64, two per tile, d = 64
+    ((1, 16, 16), 128, 2, (1, 8, 8), (0, 4, 4)),    # the same shifted: wrap masks
+    ((2, 16, 16), 256, 4, (2, 8, 8), (1, 4, 4)),    # 3D windows of 128 tokens
+    ((2, 8, 16), 1152, 16, (2, 8, 8), (1, 4, 4)),   # d = 72: V's ones column
+    ((1, 24, 8), 1152, 16, (1, 8, 8), (0, 4, 4)),   # 3 windows: the last tile half empty
+    ((1, 16, 16), 128, 4, (1, 4, 4), (0, 2, 2)),    # windows of 16 (eight per tile), d = 32
+    ((1, 16, 32), 128, 2, (1, 4, 8), (0, 2, 4)),    # windows of 32 (four per tile)
+    ((2, 16, 16), 640, 8, (2, 8, 8), (1, 4, 4)),    # d = 80
+]
+
+
+@pytest.mark.parametrize("grid,D,heads,window,shift", CASES)
+def test_window_bwd_small(grid, D, heads, window, shift):
+    c = Case(1, grid, D, heads, "bf16")
+    _check(c, window, shift)
+
+
+def test_window_bwd_without_residual():
+    c = Case(1, (2, 16, 16), 256, 4, "bf16")
+    _check(c, (2, 8, 8), (1, 4, 4), pt.PTDIT_NO_RESIDUAL)
+
+
+def test_window_bwd_full_size_1024px():
+    """t2i 1024 px: B = 4 items of 64 x 64 tokens, D = 1152, 16 heads, windows of 8 x 8,
+    shifted by half a window; 2048 units over 148 CTAs, weight gradients over 16384 tokens."""
+    c = Case(4, (1, 64, 64), 1152, 16, "bf16")
+    _check(c, (1, 8, 8), (0, 4, 4))
+
+
+def test_window_bwd_full_size_t2v():
+    """t2v: 16 x 32 x 48 tokens, 3D windows of 2 x 8 x 8 = 128 tokens, shifted."""
+    c = Case(1, (16, 32, 48), 1152, 16, "bf16")
+    _check(c, (2, 8, 8), (1, 4, 4))
+
+
+def test_window_bwd_refuses_what_it_does_not_run():
+    z = torch.zeros(1, 256, 64, dtype=torch.bfloat16, device="cuda")
+    w = tuple(torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    with pytest.raises(pt.PtditError) as e:  # D not a multiple of 128
+        pt.ptdit_window_attn_bwd(z, z.clone(), (1, 16, 16), (1, 8, 8), (0, 0, 0), w, 1)
+    assert e.value.code == pt.PTDIT_ERR_SHAPE
+    z32 = torch.zeros(1, 256, 128, dtype=torch.float32, device="cuda")
+    w32 = tuple(torch.zeros(128, 128, dtype=torch.float32, device="cuda") for _ in range(4))
+    with pytest.raises(pt.PtditError) as e:  # fp32
+        pt.ptdit_window_attn_bwd(z32, z32.clone(), (1, 16, 16), (1, 8, 8), (0, 0, 0), w32, 2)
+    assert e.value.code == pt.PTDIT_ERR_DTYPE
