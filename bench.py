@@ -628,6 +628,70 @@ def run_block(args, w, L=120):
     return 0
 
 
+def run_bwd(args, w):
+    """Backward of the shifted-window TCM branch (ptdit_window_attn_bwd): dL/dz and the four
+    weight gradients for a synthetic upstream gradient, per step."""
+    import torch
+
+    import diffusion_transformer_sparse_b200 as pt
+    from diffusion_transformer_sparse_b200 import synth
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    z_host, W_host = host_inputs(w)
+    z = z_host.to(dev)
+    dout = torch.stack([synth.latent(w.N, w.D, 500 + b, w.dtype) for b in range(w.B)]).to(dev)
+    W = tuple(x.to(dev) for x in W_host["swsa"])
+    shape = pt.make_shape(z, w.grid, w.heads)
+    ws = pt.window_attn_bwd_workspace(shape, w.window)
+    dz = torch.empty_like(z)
+    dw = tuple(torch.empty(w.D, w.D, dtype=torch.float32, device=dev) for _ in range(4))
+    do_flush = l2_policy(w)[0]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        pt.ptdit_window_attn_bwd(z, dout, w.grid, w.window, w.shift, W, w.heads, dz_in=dz, dw=dw,
+                                 ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        if do_flush:
+            flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    pt.ptdit_timing_enable(64 * args.steps)
+    for _ in range(args.steps):
+        if do_flush:
+            flush.zero_()
+        step()
+    recs = pt.ptdit_timing_read(64 * args.steps)
+    pt.ptdit_timing_enable(0)
+    per = {}
+    for k, t in recs:
+        per[k] = per.get(k, 0.0) + t / args.steps
+    f = flops.window_bwd_flops(w.N, w.n, w.D)
+    rate = {
+        "gemm (recompute Q/K/V, dA, dx)": w.B * f["gemm"] / (per.get("gemm", 0) / 1e3) / 1e12,
+        "wgrad": w.B * f["wgrad"] / (per.get("wgrad", 0) / 1e3) / 1e12,
+        "attn_window_bwd": w.B * f["core_bwd"] / (per.get("attn_window_bwd", 0) / 1e3) / 1e12,
+    } if all(per.get(k) for k in ("gemm", "wgrad", "attn_window_bwd")) else {}
+    print(json.dumps({
+        "mode": "window_bwd", "metric": "backward of one TCM branch, tokens/s", "unit": UNIT,
+        "value": w.B * w.N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,
+        "warmup": args.warmup, "config": dict(config_of(w), l2=l2_policy(w)[1]),
+        "tflops": w.B * f["total"] / (ms / 1e3) / 1e12, "flops_per_step": w.B * f["total"],
+        "kernels_ms_per_step": per, "kernels_tflops": rate,
+        "note": "per-kernel times from a second pass with hooks"}), flush=True)
+    return 0
+
+
 def parse3(text):
     v = tuple(int(x) for x in text.split(","))
     if len(v) != 3:
@@ -650,6 +714,8 @@ def main(argv=None):
     ap.add_argument("--ratio", type=parse3, help="override the proxy ratio F,H,W")
     ap.add_argument("--dense", action="store_true",
                     help="time the dense comparator (full global self-attention) instead")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward of the shifted-window TCM branch instead")
     ap.add_argument("--block", action="store_true",
                     help="time the complete PT-Block (norms, text cross-attention, MLP) instead")
     args = ap.parse_args(argv)
@@ -663,6 +729,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.dense:
         return run_dense(args, w)
+    if args.bwd:
+        return run_bwd(args, w)
     if args.block:
         return run_block(args, w)
     return run_gpu(args, w)

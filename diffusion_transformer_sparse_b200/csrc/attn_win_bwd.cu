@@ -12,10 +12,10 @@
 // One persistent CTA per SM, units in the forward kernel's order (the heads
 // of one tile follow each other).  Two load buffers (Q, K, V, dO blocks of the
 // tiled head layout, thl.cuh) keep the next unit's loads in flight:
-//   warp 0       loader: four bulk copies per unit; the tile rows' key masks
+//   warp 8       loader: four bulk copies per unit; the tile rows' key masks
 //                (window in tile x wrap bits, built with ballots as in the
 //                forward kernel) once per (batch item, tile) and buffer
-//   warp 1       MMA issuer: S = Q K^T and dP = dO V^T into TMEM (K-major
+//   warp 9       MMA issuer (warps 10 and 11 only pad the CTA to whole warpgroups): S = Q K^T and dP = dO V^T into TMEM (K-major
 //                operands); once the softmax warpgroup has written P and dS to
 //                shared memory: dV = P^T dO, dK = dS^T Q (P and dS read as
 //                MN-major A operands) and dQ = dS K (dS as K-major A), with
@@ -25,18 +25,21 @@
 //                columns (the softmax has read dP by then), so the next unit's
 //                S is issued as soon as this unit's softmax has read S and dP,
 //                its dP once the epilogue has read dQ.
-//   warps 4-7    softmax warpgroup, thread r = query row r: the row max and
-//                sum over its window's keys, then P (normalised) and
-//                rowsum(P * dP), then dS (c folded in), written as bf16 rows of
-//                a 128 x 128 tile with the 128-byte swizzle; zeros for keys of
-//                other windows and for rows without a token.
-//   warps 8-11   epilogue, thread r = tile row r: dQ, dK, dV of row r (its
+//   warps 0-3    softmax warpgroup, thread r = query row r: reads its
+//                window's scores once (max, exponentials, sum), keeps P
+//                normalised as bf16 pairs in registers, then rowsum(P * dP) and
+//                dS (c folded in) from two reads of dP, and writes P and dS as
+//                bf16 rows of 128 x 128 tiles with the 128-byte swizzle; zeros
+//                for keys of other windows and for rows without a token.
+//   warps 4-7    epilogue, thread r = tile row r: dQ, dK, dV of row r (its
 //                token is both a query and a key of the window) to the
 //                row-major [B N, 3 D] gradient buffer (dQ, dK, dV column blocks,
 //                head h at columns h d .. h d + d - 1 of each).
 // TMEM (every accumulator and load starts on a 64-column boundary): S 0-127,
 // dP and then dQ 128-255, dV 256-383, dK 384-511 (head columns 0..63 at the
 // base, 64..79 at base + 64).  Every wait is bounded (2 s).
+#include <type_traits>
+
 #include "tc_util.cuh"
 #include "thl.cuh"
 
@@ -133,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int u1 = (int)((long)(blockIdx.x + 1) * sc.units / gridDim.x);
     const int nunits = u1 - u0;  // local unit k: buffer k % NBUF
 
-    if (warp == 0) {
+    if (warp == 8) {
         // ------------------------------------------------------------ loader
         const uint8_t *src[4] = {static_cast<const uint8_t *>(a.q), static_cast<const uint8_t *>(a.k),
                                  static_cast<const uint8_t *>(a.v),
@@ -189,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             mbar_arrive(&ld_full[bf]);
         }
-    } else if (warp == 1) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_bf16(BQ, BQ);                 // K-major A and B
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_wait(drain, 0, &never, status);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp < 4) {
         // ------------------------------------------------------------ softmax warpgroup
         const int r = (warp % 4) * 32 + lane;  // query row of the tile = TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
@@ -290,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *sP = sm + L::OFF_P, *sDS = sm + L::OFF_DS;
         // this row's keys: its window's 64-key half of the tile (windows of up to 64
         // tokens lie inside one half), or all 128 keys
-        const int c_lo = n < BQ ? (r >> 6) << 6 : 0, nk = n < BQ ? 64 : 128;
+        const int c_lo = n < BQ ? (r >> 6) << 6 : 0;
         for (int k = 0; k < nunits; ++k) {
             const int bf = k % NBUF;
             if (!mbar_wait_warp(&ld_full[bf], (k / NBUF) & 1, abort, status)) break;
@@ -307,90 +310,129 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!mbar_wait_warp(s_full, k & 1, abort, status)) break;
             fence_after_sync();
-            // pass 1: row max over the allowed keys; pass 2: the row sum
-            float m = -INFINITY;
+            // S of this row's keys, read once: the row max and sum, then P normalised and
+            // packed as bf16 pairs in registers until the previous unit's MMAs are done
+            // with the shared-memory P and dS tiles
+            bool okw = true;
+            auto row = [&](auto NKc) {
+                constexpr int NK = decltype(NKc)::value;  // the row's window span of keys
+                // 64 keys per read of S: the row max over every half first, then the
+                // exponentials, packed as bf16 pairs as soon as they are computed
+                // (eight independent chains for every sum and max: one warp per SM
+                // sub-partition runs this code, so nothing else hides their latency)
+                float mx[8];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                if (jj * 32 >= nk) break;
-                uint32_t sv[32];
-                tmem_ld32(t_s + c_lo + jj * 32, sv);
-                tmem_ld_wait();
-                const uint32_t w = allow[jj];
+                for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if ((w >> e) & 1u) m = fmaxf(m, __uint_as_float(sv[e]));
-            }
-            const float ms = m * sl2;
-            float l = 0.f;
+                for (int hh = 0; hh < NK / 64; ++hh) {
+                    uint32_t sv[64];
+                    tmem_ld32(t_s + c_lo + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                    tmem_ld32(t_s + c_lo + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+                    tmem_ld_wait();
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                if (jj * 32 >= nk) break;
-                uint32_t sv[32];
-                tmem_ld32(t_s + c_lo + jj * 32, sv);
-                tmem_ld_wait();
-                const uint32_t w = allow[jj];
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if ((w >> e) & 1u) l += ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -ms));
-            }
-            // P = 2^(s sl2 - ms - log2 l); a row without a token has no allowed key
-            const float off = qi >= 0 ? ms + __log2f(l) : 0.f;
-            // the previous unit's MMAs have read P and dS; this unit's dP is in
-            if (!mbar_wait_warp(pds_free, (k & 1) ^ 1, abort, status)) break;
-            if (!mbar_wait_warp(dp_full, k & 1, abort, status)) break;
-            fence_after_sync();
-            // pass 3: P to shared memory and delta = rowsum(P * dP)
-            float delta = 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                if (jj * 32 >= nk) break;
-                const int j = jj * 32;
-                uint32_t sv[32], dv[32];
-                tmem_ld32(t_s + c_lo + j, sv);
-                tmem_ld32(t_dp + c_lo + j, dv);
-                tmem_ld_wait();
-                const uint32_t w = allow[jj];
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float p0 = ((w >> e) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -off)) : 0.f;
-                    const float p1 = ((w >> (e + 1)) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -off)) : 0.f;
-                    pk[e / 2] = pack_bf16(p0, p1);
-                    // delta from the bf16 weights the MMAs use
-                    const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e / 2]));
-                    delta = fmaf(pr.x, __uint_as_float(dv[e]), delta);
-                    delta = fmaf(pr.y, __uint_as_float(dv[e + 1]), delta);
+                    for (int e = 0; e < 64; ++e)
+                        if ((allow[2 * hh + (e >> 5)] >> (e & 31)) & 1u)
+                            mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
                 }
-                const int c0 = (c_lo + j) >> 3;
+                const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                const float ms = m * sl2;
+                float ls[8];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(sP + pds_chunk(r, c0 + q)) =
-                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-            }
-            // pass 4: dS = c P (dP - delta)
+                for (int i = 0; i < 8; ++i) ls[i] = 0.f;
+                uint32_t pk[NK / 2];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                if (jj * 32 >= nk) break;
-                const int j = jj * 32;
-                uint32_t dv[32];
-                tmem_ld32(t_dp + c_lo + j, dv);
-                tmem_ld_wait();
-                const int c0 = (c_lo + j) >> 3;
+                for (int hh = 0; hh < NK / 64; ++hh) {
+                    uint32_t sv[64];
+                    tmem_ld32(t_s + c_lo + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sv));
+                    tmem_ld32(t_s + c_lo + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+                    tmem_ld_wait();
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 p4 = *reinterpret_cast<const uint4 *>(sP + pds_chunk(r, c0 + q));
-                    const uint32_t pw[4] = {p4.x, p4.y, p4.z, p4.w};
-                    uint32_t o[4];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[t]));
-                        const int e = 8 * q + 2 * t;
-                        o[t] = pack_bf16(c * pr.x * (__uint_as_float(dv[e]) - delta),
-                                         c * pr.y * (__uint_as_float(dv[e + 1]) - delta));
+                    for (int e = 0; e < 64; e += 2) {
+                        const uint32_t w = allow[2 * hh + (e >> 5)];
+                        const float p0 = ((w >> (e & 31)) & 1u)
+                                             ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -ms))
+                                             : 0.f;
+                        const float p1 = ((w >> ((e + 1) & 31)) & 1u)
+                                             ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -ms))
+                                             : 0.f;
+                        ls[(e >> 1) & 7] += p0 + p1;
+                        pk[32 * hh + e / 2] = pack_bf16(p0, p1);
                     }
-                    *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, c0 + q)) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
-            }
+                const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                // a row without a token has no allowed key: P = 0
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+                for (int e = 0; e < NK / 2; ++e) {
+                    const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e]));
+                    pk[e] = pack_bf16(pr.x * inv, pr.y * inv);
+                }
+                // the previous unit's MMAs have read P and dS; this unit's dP is in
+                if (!mbar_wait_warp(pds_free, (k & 1) ^ 1, abort, status) ||
+                    !mbar_wait_warp(dp_full, k & 1, abort, status)) {
+                    okw = false;
+                    return;
+                }
+                fence_after_sync();
+#pragma unroll
+                for (int q = 0; q < NK / 8; ++q)
+                    *reinterpret_cast<uint4 *>(sP + pds_chunk(r, (c_lo >> 3) + q)) =
+                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                // delta = rowsum(P * dP) from the bf16 weights the MMAs use, read back from
+                // this row of the shared-memory P tile (so that they need no registers);
+                // dP in halves of 64 keys
+                float dl[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dl[i] = 0.f;
+#pragma unroll
+                for (int hh = 0; hh < NK / 64; ++hh) {
+                    uint32_t dv[64];
+                    tmem_ld32(t_dp + c_lo + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(dv));
+                    tmem_ld32(t_dp + c_lo + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 p4 = *reinterpret_cast<const uint4 *>(sP + pds_chunk(r, ((c_lo + 64 * hh) >> 3) + q));
+                        const uint32_t pw[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[t]));
+                            dl[2 * t] = fmaf(pr.x, __uint_as_float(dv[8 * q + 2 * t]), dl[2 * t]);
+                            dl[2 * t + 1] = fmaf(pr.y, __uint_as_float(dv[8 * q + 2 * t + 1]), dl[2 * t + 1]);
+                        }
+                    }
+                }
+                const float delta = ((dl[0] + dl[1]) + (dl[2] + dl[3])) + ((dl[4] + dl[5]) + (dl[6] + dl[7]));
+                // dS = c P (dP - delta), 16 bytes (8 keys) per store
+#pragma unroll
+                for (int hh = 0; hh < NK / 64; ++hh) {
+                    uint32_t dv[64];
+                    tmem_ld32(t_dp + c_lo + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(dv));
+                    tmem_ld32(t_dp + c_lo + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t off = pds_chunk(r, ((c_lo + 64 * hh) >> 3) + q);
+                        const uint4 p4 = *reinterpret_cast<const uint4 *>(sP + off);
+                        const uint32_t pw[4] = {p4.x, p4.y, p4.z, p4.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const int e = 8 * q + 2 * t;
+                            const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[t]));
+                            o[t] = pack_bf16(c * pr.x * (__uint_as_float(dv[e]) - delta),
+                                             c * pr.y * (__uint_as_float(dv[e + 1]) - delta));
+                        }
+                        *reinterpret_cast<uint4 *>(sDS + off) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+            };
+            if (n < BQ)
+                row(std::integral_constant<int, 64>{});
+            else
+                row(std::integral_constant<int, 128>{});
+            if (!okw) break;
             fence_before_sync();
             mbar_arrive(sp_free);  // S and dP are read
             // the keys of the other windows of the tile: zero weights and gradients
@@ -405,8 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_async_smem();  // the tensor cores read what these threads wrote
             mbar_arrive(pds_full);
         }
-    } else if (warp >= 8) {
-        // ------------------------------------------------------------ epilogue
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ epilogue (warps 4-7)
         const int r = (warp % 4) * 32 + lane;  // tile row = TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
         const WinGeom &geo = a.geom;

@@ -58,3 +58,21 @@ def pt_block_flops(N: int, M: int, n: int, D: int, L: int, Dh: int) -> dict:
     f["core"] += f["text_core"]
     f["total"] = f["proj"] + f["core"]
     return f
+
+
+def window_bwd_flops(N: int, n: int, D: int) -> dict:
+    """Backward of one TCM branch as ptdit_window_attn_bwd runs it, per batch item:
+    the recomputed forward (Q/K/V projections 6 N D^2, attention 4 N n D), dA = dout Wo
+    (2 N D^2), the attention backward (S, dP, dV, dK, dQ: 10 N n D), the input gradient
+    [dQ dK dV][Wq; Wk; Wv] (6 N D^2) and the weight gradients (8 N D^2)."""
+    f = {
+        "recompute_proj": 6 * N * D * D,
+        "recompute_core": 4 * N * n * D,
+        "dA": 2 * N * D * D,
+        "core_bwd": 10 * N * n * D,
+        "dx": 6 * N * D * D,
+        "wgrad": 8 * N * D * D,
+    }
+    f["gemm"] = f["recompute_proj"] + f["dA"] + f["dx"]
+    f["total"] = sum(v for k, v in f.items() if k != "gemm")
+    return f
