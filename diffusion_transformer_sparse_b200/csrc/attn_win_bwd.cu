@@ -52,7 +52,6 @@ constexpr int BQ = 128;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 128, T_DV = 256, T_DK = 384;
-constexpr int kMaskWords = 128;  // key masks per buffer, as in the forward kernel
 constexpr int NBUF = 2;
 
 template <int DPAD>
@@ -65,12 +64,14 @@ struct BwdLayout {
     static constexpr int OFF_P = NBUF * BUF;            // P: 2 key halves x 128 rows x 128 B
     static constexpr int OFF_DS = OFF_P + 2 * TILE_A;   // dS: same layout
     static constexpr int OFF_INFO = OFF_DS + 2 * TILE_A;  // int8 info[NBUF][128]
-    static constexpr int OFF_MASK = OFF_INFO + NBUF * BQ; // uint32 kmask[NBUF][kMaskWords]
-    static constexpr int OFF_BAR = OFF_MASK + NBUF * kMaskWords * 4;
+    // float exchange[warpgroup][2][BQ]: (max, sum), then rowsum(P dP) in the sum's place
+    static constexpr int OFF_X = OFF_INFO + NBUF * BQ;
+    static constexpr int OFF_BAR = OFF_X + 2 * 2 * BQ * 4;
     // ld_full[NBUF], buf_free[NBUF], s_full, dp_full, sp_free, pds_full, pds_free, acc_full,
-    // dq_free, acc_free, drain
-    static constexpr int NBARS = 2 * NBUF + 9;
-    static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
+    // dq_free, acc_free, drain, x_full[2], x_read, stg_done
+    static constexpr int NBARS = 2 * NBUF + 13;
+    // no alignment slack: the kernel checks that the base is 1 KB aligned
+    static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16;
     static_assert(TILE_A % 1024 == 0 && TILE % 1024 == 0, "swizzled tiles stay 1 KB aligned");
     static_assert(BYTES <= 232448, "shared memory budget");
 };
@@ -92,15 +93,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __nv_bfloat16 *__restrict__ dqkv, long ldg, BwdSched sc, int *status) {
     using L = BwdLayout<DPAD>;
     extern __shared__ uint8_t sm_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // the swizzled tiles need a 1 KB aligned base; the allocation has no slack, so a
+    // base that is not aligned is reported instead of used
+    if (smem_u32(sm_raw) & 1023u) {
+        if (threadIdx.x == 0) atomicExch(status, 5 /* PTDIT_ERR_CUDA */);
+        return;
+    }
+    uint8_t *sm = sm_raw;
     int8_t *info = reinterpret_cast<int8_t *>(sm + L::OFF_INFO);
-    uint32_t *kmask = reinterpret_cast<uint32_t *>(sm + L::OFF_MASK);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
     uint64_t *ld_full = bars, *buf_free = bars + NBUF;
     uint64_t *s_full = bars + 2 * NBUF, *dp_full = s_full + 1, *sp_free = s_full + 2;
     uint64_t *pds_full = s_full + 3, *pds_free = s_full + 4, *acc_full = s_full + 5;
     uint64_t *dq_free = s_full + 6, *acc_free = s_full + 7, *drain = s_full + 8;
+    uint64_t *x_full = s_full + 9;  // the warpgroups' exchanges of a unit: max and sum, rowsum
+    uint64_t *x_read = s_full + 11; // each warpgroup has read the other's max and sum
+    uint64_t *stg_done = s_full + 12;  // both warpgroups have staged a unit's gradients
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -114,12 +122,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(sp_free, BQ);
-        mbar_init(pds_full, BQ);
+        mbar_init(sp_free, 2 * BQ);   // both warpgroups
+        mbar_init(pds_full, 2 * BQ);
         mbar_init(pds_free, 1);
         mbar_init(acc_full, 1);
-        mbar_init(dq_free, BQ);
-        mbar_init(acc_free, BQ);
+        mbar_init(dq_free, BQ);       // warpgroup 0 reads dQ
+        mbar_init(acc_free, 2 * BQ);
+        mbar_init(&x_full[0], 2 * BQ);
+        mbar_init(&x_full[1], 2 * BQ);
+        mbar_init(x_read, 2 * BQ);
+        mbar_init(stg_done, 2 * BQ);
         mbar_init(drain, 1);
         *abort = 0;
         fence_mbar_init();
@@ -157,10 +169,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_load(sm + bf * L::BUF + m * L::TILE, src[m] + blk * L::TILE, L::TILE,
                               &ld_full[bf]);
             }
+            // window in tile and wrap bits of every tile row (rows of one tile attend each
+            // other iff these agree): once per (batch item, tile) and buffer
             const int held = bf == 0 ? held0 : held1;
             if (rest != held) {
                 if (bf == 0) held0 = rest; else held1 = rest;
-                int inf[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const int r = q * 32 + lane;
@@ -171,22 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (void)window_token(geo, win, slot, &wrap);
                         in = wit * 8 + wrap;
                     }
-                    inf[q] = in;
                     info[bf * BQ + r] = static_cast<int8_t>(in);
-                }
-                const int nkeys = n < BQ ? (BQ / n) * 8 : 8;
-                for (int v = 0; v < nkeys; ++v) {
-                    const int half = n < BQ ? ((v >> 3) * n) >> 6 : 0;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t bits = __ballot_sync(0xffffffffu, inf[q] == v);
-                        if (lane == 0) {
-                            if (n >= BQ)
-                                kmask[bf * kMaskWords + v * 4 + q] = bits;
-                            else if ((q >> 1) == half)
-                                kmask[bf * kMaskWords + v * 2 + (q & 1)] = bits;
-                        }
-                    }
                 }
             }
             __syncwarp();
@@ -284,177 +282,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_wait(drain, 0, &never, status);
             }
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ softmax warpgroup
-        const int r = (warp % 4) * 32 + lane;  // query row of the tile = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
-        const uint32_t t_s = tmem + lane_base + T_S, t_dp = tmem + lane_base + T_DP;
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ softmax + epilogue
+        // Warpgroup g = warp / 4 takes half of every row's keys (thread r: query row r,
+        // its TMEM lane): keys 64 g .. 64 g + 63 of a 128-token window, or 32 of the
+        // 64 keys of a smaller window's half of the tile.  The halves' maxima and sums
+        // are combined once per unit (each half exponentiates against its own max;
+        // the shared scale is 2^(m_g - m) / l), and rowsum(P * dP) once more.
+        const int g = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const float c = a.scale, sl2 = a.scale * 1.4426950408889634f;
         uint8_t *sP = sm + L::OFF_P, *sDS = sm + L::OFF_DS;
-        // this row's keys: its window's 64-key half of the tile (windows of up to 64
-        // tokens lie inside one half), or all 128 keys
-        const int c_lo = n < BQ ? (r >> 6) << 6 : 0;
-        for (int k = 0; k < nunits; ++k) {
-            const int bf = k % NBUF;
-            if (!mbar_wait_warp(&ld_full[bf], (k / NBUF) & 1, abort, status)) break;
-            const int qi = info[bf * BQ + r];
-            uint32_t allow[4] = {0u, 0u, 0u, 0u};
-            if (qi >= 0) {
-                if (n < BQ) {
-                    allow[0] = kmask[bf * kMaskWords + qi * 2];
-                    allow[1] = kmask[bf * kMaskWords + qi * 2 + 1];
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) allow[q] = kmask[bf * kMaskWords + qi * 4 + q];
-                }
-            }
-            if (!mbar_wait_warp(s_full, k & 1, abort, status)) break;
-            fence_after_sync();
-            // S of this row's keys, read once: the row max and sum, then P normalised and
-            // packed as bf16 pairs in registers until the previous unit's MMAs are done
-            // with the shared-memory P and dS tiles
-            bool okw = true;
-            auto row = [&](auto NKc) {
-                constexpr int NK = decltype(NKc)::value;  // the row's window span of keys
-                // 64 keys per read of S: the row max over every half first, then the
-                // exponentials, packed as bf16 pairs as soon as they are computed
-                // (eight independent chains for every sum and max: one warp per SM
-                // sub-partition runs this code, so nothing else hides their latency)
-                float mx[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-#pragma unroll
-                for (int hh = 0; hh < NK / 64; ++hh) {
-                    uint32_t sv[64];
-                    tmem_ld32(t_s + c_lo + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sv));
-                    tmem_ld32(t_s + c_lo + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        if ((allow[2 * hh + (e >> 5)] >> (e & 31)) & 1u)
-                            mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
-                }
-                const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                const float ms = m * sl2;
-                float ls[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) ls[i] = 0.f;
-                uint32_t pk[NK / 2];
-#pragma unroll
-                for (int hh = 0; hh < NK / 64; ++hh) {
-                    uint32_t sv[64];
-                    tmem_ld32(t_s + c_lo + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sv));
-                    tmem_ld32(t_s + c_lo + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 64; e += 2) {
-                        const uint32_t w = allow[2 * hh + (e >> 5)];
-                        const float p0 = ((w >> (e & 31)) & 1u)
-                                             ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -ms))
-                                             : 0.f;
-                        const float p1 = ((w >> ((e + 1) & 31)) & 1u)
-                                             ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -ms))
-                                             : 0.f;
-                        ls[(e >> 1) & 7] += p0 + p1;
-                        pk[32 * hh + e / 2] = pack_bf16(p0, p1);
-                    }
-                }
-                const float l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-                // a row without a token has no allowed key: P = 0
-                const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-                for (int e = 0; e < NK / 2; ++e) {
-                    const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e]));
-                    pk[e] = pack_bf16(pr.x * inv, pr.y * inv);
-                }
-                // the previous unit's MMAs have read P and dS; this unit's dP is in
-                if (!mbar_wait_warp(pds_free, (k & 1) ^ 1, abort, status) ||
-                    !mbar_wait_warp(dp_full, k & 1, abort, status)) {
-                    okw = false;
-                    return;
-                }
-                fence_after_sync();
-#pragma unroll
-                for (int q = 0; q < NK / 8; ++q)
-                    *reinterpret_cast<uint4 *>(sP + pds_chunk(r, (c_lo >> 3) + q)) =
-                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                // delta = rowsum(P * dP) from the bf16 weights the MMAs use, read back from
-                // this row of the shared-memory P tile (so that they need no registers);
-                // dP in halves of 64 keys
-                float dl[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) dl[i] = 0.f;
-#pragma unroll
-                for (int hh = 0; hh < NK / 64; ++hh) {
-                    uint32_t dv[64];
-                    tmem_ld32(t_dp + c_lo + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(dv));
-                    tmem_ld32(t_dp + c_lo + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 p4 = *reinterpret_cast<const uint4 *>(sP + pds_chunk(r, ((c_lo + 64 * hh) >> 3) + q));
-                        const uint32_t pw[4] = {p4.x, p4.y, p4.z, p4.w};
-#pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[t]));
-                            dl[2 * t] = fmaf(pr.x, __uint_as_float(dv[8 * q + 2 * t]), dl[2 * t]);
-                            dl[2 * t + 1] = fmaf(pr.y, __uint_as_float(dv[8 * q + 2 * t + 1]), dl[2 * t + 1]);
-                        }
-                    }
-                }
-                const float delta = ((dl[0] + dl[1]) + (dl[2] + dl[3])) + ((dl[4] + dl[5]) + (dl[6] + dl[7]));
-                // dS = c P (dP - delta), 16 bytes (8 keys) per store
-#pragma unroll
-                for (int hh = 0; hh < NK / 64; ++hh) {
-                    uint32_t dv[64];
-                    tmem_ld32(t_dp + c_lo + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(dv));
-                    tmem_ld32(t_dp + c_lo + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint32_t off = pds_chunk(r, ((c_lo + 64 * hh) >> 3) + q);
-                        const uint4 p4 = *reinterpret_cast<const uint4 *>(sP + off);
-                        const uint32_t pw[4] = {p4.x, p4.y, p4.z, p4.w};
-                        uint32_t o[4];
-#pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            const int e = 8 * q + 2 * t;
-                            const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[t]));
-                            o[t] = pack_bf16(c * pr.x * (__uint_as_float(dv[e]) - delta),
-                                             c * pr.y * (__uint_as_float(dv[e + 1]) - delta));
-                        }
-                        *reinterpret_cast<uint4 *>(sDS + off) = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                }
-            };
-            if (n < BQ)
-                row(std::integral_constant<int, 64>{});
-            else
-                row(std::integral_constant<int, 128>{});
-            if (!okw) break;
-            fence_before_sync();
-            mbar_arrive(sp_free);  // S and dP are read
-            // the keys of the other windows of the tile: zero weights and gradients
-            if (n < BQ) {
-                const int o0 = (64 - c_lo) >> 3;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    *reinterpret_cast<uint4 *>(sP + pds_chunk(r, o0 + q)) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, o0 + q)) = make_uint4(0, 0, 0, 0);
-                }
-            }
-            fence_async_smem();  // the tensor cores read what these threads wrote
-            mbar_arrive(pds_full);
-        }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ epilogue (warps 4-7)
-        const int r = (warp % 4) * 32 + lane;  // tile row = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>((warp % 4) * 32) << 16;
+        float *xch = reinterpret_cast<float *>(sm + L::OFF_X);  // [g][2][BQ]
+        const int c_lo = n < BQ ? (r >> 6) << 6 : 0;            // the row's 64-key half
+        const int kofs = n < BQ ? c_lo + 32 * g : 64 * g;       // first key of this warpgroup
+        const uint32_t t_s = tmem + lane_base + T_S + kofs, t_dp = tmem + lane_base + T_DP + kofs;
         const WinGeom &geo = a.geom;
         const int pack = BQ / n, nch = d / 8;
-        for (int k = 0; k < nunits; ++k) {
-            const int u = u0 + k;
+        // gradients of unit kk out of TMEM: dQ and dV by warpgroup 0, dK by warpgroup 1
+        auto epilogue = [&](int kk) {
+            if (!mbar_wait_warp(acc_full, kk & 1, abort, status)) return false;
+            fence_after_sync();
+            const int u = u0 + kk;
             const int h = u % a.heads, rest = u / a.heads, tile = rest % sc.tiles,
                       b = rest / sc.tiles;
             const int wit = r / n, win = tile * pack + wit, slot = r - wit * n;
@@ -463,11 +313,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int wrap;
                 row = (long)b * a.k_bstride + window_token(geo, win, slot, &wrap);
             }
-            if (!mbar_wait_warp(acc_full, k & 1, abort, status)) break;
-            fence_after_sync();
-            __nv_bfloat16 *dst = row >= 0 ? dqkv + row * ldg + (long)h * d : nullptr;
+            // staging: this warp's 8 KB of the P / dS tiles (the unit's MMAs are done with
+            // them; the next P is written only after both warpgroups are through here)
+            uint8_t *stg = sm + L::OFF_P + warp * 8192;
+            const int pitch = nch * 16 + (nch % 8 == 0 ? 16 : 0);  // an odd number of 16 B units
+            // warpgroup 0 writes dQ and dV, warpgroup 1 dK
 #pragma unroll
-            for (int m = 0; m < 3; ++m) {
+            for (int i = 0; i < 2; ++i) {
+                if (g == 1 && i == 1) break;
+                const int m = g == 1 ? 1 : (i == 0 ? 0 : 2);  // column block: dQ 0, dK 1, dV 2
                 uint32_t v[DPAD];
                 const uint32_t t = tmem + lane_base + (m == 0 ? T_DQ : (m == 1 ? T_DK : T_DV));
                 tmem_ld32(t, *reinterpret_cast<uint32_t(*)[32]>(v));
@@ -478,22 +332,191 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_before_sync();
                     mbar_arrive(dq_free);
                 }
-                if (row >= 0) {
+                if (m != 0 && (g == 1 || i == 1)) {  // this warpgroup's last TMEM read
+                    fence_before_sync();
+                    mbar_arrive(acc_free);  // the next unit's gradient MMAs may overwrite TMEM
+                }
 #pragma unroll
-                    for (int uu = 0; uu < DPAD / 8; ++uu)
-                        if (uu < nch) {
-                            uint4 o;
-                            o.x = pack_bf16(__uint_as_float(v[8 * uu + 0]), __uint_as_float(v[8 * uu + 1]));
-                            o.y = pack_bf16(__uint_as_float(v[8 * uu + 2]), __uint_as_float(v[8 * uu + 3]));
-                            o.z = pack_bf16(__uint_as_float(v[8 * uu + 4]), __uint_as_float(v[8 * uu + 5]));
-                            o.w = pack_bf16(__uint_as_float(v[8 * uu + 6]), __uint_as_float(v[8 * uu + 7]));
-                            *reinterpret_cast<uint4 *>(dst + (long)m * D + 8 * uu) = o;
-                        }
+                for (int uu = 0; uu < DPAD / 8; ++uu)
+                    if (uu < nch) {
+                        uint4 o;
+                        o.x = pack_bf16(__uint_as_float(v[8 * uu + 0]), __uint_as_float(v[8 * uu + 1]));
+                        o.y = pack_bf16(__uint_as_float(v[8 * uu + 2]), __uint_as_float(v[8 * uu + 3]));
+                        o.z = pack_bf16(__uint_as_float(v[8 * uu + 4]), __uint_as_float(v[8 * uu + 5]));
+                        o.w = pack_bf16(__uint_as_float(v[8 * uu + 6]), __uint_as_float(v[8 * uu + 7]));
+                        *reinterpret_cast<uint4 *>(stg + lane * pitch + uu * 16) = o;
+                    }
+                __syncwarp();
+                // consecutive lanes on consecutive 16-byte pieces of a token row: item j of
+                // the warp's 32 x nch pieces is piece j % nch of staging row j / nch, walked
+                // incrementally (j advances by 32 per step)
+                const int drow = 32 / nch, dpc = 32 % nch;
+                int rr = lane / nch, cc = lane % nch;
+                __nv_bfloat16 *colbase = dqkv + (long)m * D + (long)h * d;
+#pragma unroll 1
+                for (int j = lane; j < 32 * nch; j += 32) {
+                    const long trow = __shfl_sync(0xffffffffu, row, rr);  // that row's token
+                    if (trow >= 0)
+                        *reinterpret_cast<uint4 *>(colbase + trow * ldg + 8 * cc) =
+                            *reinterpret_cast<const uint4 *>(stg + rr * pitch + cc * 16);
+                    rr += drow;
+                    cc += dpc;
+                    if (cc >= nch) {
+                        cc -= nch;
+                        ++rr;
+                    }
+                }
+                __syncwarp();  // the staging rows are free for the next block
+            }
+            return true;
+        };
+        bool okw = true;
+        auto unit = [&](int k, auto NKc) {
+            constexpr int NK = decltype(NKc)::value;  // this warpgroup's keys of the row
+            const int bf = k % NBUF;
+            if (!mbar_wait_warp(&ld_full[bf], (k / NBUF) & 1, abort, status)) { okw = false; return; }
+            // key e of this half is allowed iff its window-in-tile and wrap bits equal the
+            // row's (a row without a token, qi < 0, allows none)
+            const int qi = info[bf * BQ + r];
+            uint32_t aw[2] = {0u, 0u};
+            {
+                const uint32_t *ik = reinterpret_cast<const uint32_t *>(info + bf * BQ + kofs);
+#pragma unroll
+                for (int i = 0; i < NK / 4; ++i) {
+                    const uint32_t wv = ik[i];  // the same word in every lane: a broadcast
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (qi >= 0 && static_cast<int8_t>(wv >> (8 * j)) == qi)
+                            aw[(4 * i + j) >> 5] |= 1u << ((4 * i + j) & 31);
                 }
             }
+            if (!mbar_wait_warp(s_full, k & 1, abort, status)) { okw = false; return; }
+            fence_after_sync();
+            // this half's scores, read once: its max, its exponentials (bf16 pairs), its sum
+            uint32_t pk[NK / 2];
+            float ms_g, l_g;
+            {
+                uint32_t sv[NK];
+#pragma unroll
+                for (int q = 0; q < NK / 32; ++q)
+                    tmem_ld32(t_s + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * q));
+                tmem_ld_wait();
+                float mx[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < NK; ++e)
+                    if ((aw[e >> 5] >> (e & 31)) & 1u) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
+                ms_g = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+                float ls[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ls[i] = 0.f;
+#pragma unroll
+                for (int e = 0; e < NK; e += 2) {
+                    const uint32_t w = aw[e >> 5];
+                    const float p0 = ((w >> (e & 31)) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -ms_g)) : 0.f;
+                    const float p1 = ((w >> ((e + 1) & 31)) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -ms_g)) : 0.f;
+                    ls[(e >> 1) & 7] += p0 + p1;
+                    pk[e / 2] = pack_bf16(p0, p1);
+                }
+                l_g = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+            }
+            // combine the halves: m = max(m_0, m_1), l = sum of l_g 2^(m_g - m)
+            // (the slots are rewritten only after the other warpgroup has read them: the
+            // sum's slot carries rowsum(P dP) once x_read shows it read, and the next
+            // unit's values follow sp_free, which needs both warpgroups)
+            float *xm = xch + g * 2 * BQ;
+            const float *xo = xch + (g ^ 1) * 2 * BQ;
+            xm[r] = ms_g;
+            xm[BQ + r] = l_g;
+            mbar_arrive(&x_full[0]);
+            if (!mbar_wait_warp(&x_full[0], k & 1, abort, status)) { okw = false; return; }
+            const float ms_o = xo[r], l_o = xo[BQ + r];
+            mbar_arrive(x_read);
+            const float msx = fmaxf(ms_g, ms_o);
+            const float f_g = ms_g == -INFINITY ? 0.f : ex2_approx(ms_g - msx);
+            const float f_o = ms_o == -INFINITY ? 0.f : ex2_approx(ms_o - msx);
+            const float lsum = l_g * f_g + l_o * f_o;
+            const float scale = lsum > 0.f ? f_g / lsum : 0.f;  // no allowed key: P = 0
+#pragma unroll
+            for (int e = 0; e < NK / 2; ++e) {
+                const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e]));
+                pk[e] = pack_bf16(pr.x * scale, pr.y * scale);
+            }
+            // the previous unit's gradients out of TMEM (their dQ read lets this unit's
+            // dP go into dP's columns)
+            if (k > 0) {
+                if (!epilogue(k - 1)) { okw = false; return; }
+                // the other warpgroup's staging (in the P / dS tiles) is done too
+                mbar_arrive(stg_done);
+                if (!mbar_wait_warp(stg_done, (k - 1) & 1, abort, status)) { okw = false; return; }
+            }
+            // the previous unit's MMAs have read P and dS; this unit's dP is in
+            if (!mbar_wait_warp(pds_free, (k & 1) ^ 1, abort, status) ||
+                !mbar_wait_warp(dp_full, k & 1, abort, status)) {
+                okw = false;
+                return;
+            }
+            fence_after_sync();
+#pragma unroll
+            for (int q = 0; q < NK / 8; ++q)
+                *reinterpret_cast<uint4 *>(sP + pds_chunk(r, (kofs >> 3) + q)) =
+                    make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            // this half of dP, read once: rowsum(P * dP) over both halves, then dS
+            uint32_t dv[NK];
+#pragma unroll
+            for (int q = 0; q < NK / 32; ++q)
+                tmem_ld32(t_dp + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(dv + 32 * q));
+            tmem_ld_wait();
+            float dl[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dl[i] = 0.f;
+#pragma unroll
+            for (int e = 0; e < NK; e += 2) {
+                const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e / 2]));
+                dl[e & 7] = fmaf(pr.x, __uint_as_float(dv[e]), dl[e & 7]);
+                dl[(e & 7) + 1] = fmaf(pr.y, __uint_as_float(dv[e + 1]), dl[(e & 7) + 1]);
+            }
+            const float d_g = ((dl[0] + dl[1]) + (dl[2] + dl[3])) + ((dl[4] + dl[5]) + (dl[6] + dl[7]));
+            if (!mbar_wait_warp(x_read, k & 1, abort, status)) { okw = false; return; }
+            xm[BQ + r] = d_g;
+            mbar_arrive(&x_full[1]);
+            if (!mbar_wait_warp(&x_full[1], k & 1, abort, status)) { okw = false; return; }
+            const float delta = d_g + xo[BQ + r];
+#pragma unroll
+            for (int q = 0; q < NK / 8; ++q) {
+                uint32_t o[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int e = 8 * q + 2 * t;
+                    const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e / 2]));
+                    o[t] = pack_bf16(c * pr.x * (__uint_as_float(dv[e]) - delta),
+                                     c * pr.y * (__uint_as_float(dv[e + 1]) - delta));
+                }
+                *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, (kofs >> 3) + q)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
             fence_before_sync();
-            mbar_arrive(acc_free);  // the next unit's gradient MMAs may overwrite TMEM
+            mbar_arrive(sp_free);  // S and dP are read
+            // the keys of the tile's other window half: zero weights and gradients
+            if (n < BQ) {
+                const int o0 = ((64 - c_lo) >> 3) + 4 * g;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    *reinterpret_cast<uint4 *>(sP + pds_chunk(r, o0 + q)) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, o0 + q)) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_async_smem();  // the tensor cores read what these threads wrote
+            mbar_arrive(pds_full);
+        };
+        for (int k = 0; k < nunits && okw; ++k) {
+            if (n < BQ)
+                unit(k, std::integral_constant<int, 32>{});
+            else
+                unit(k, std::integral_constant<int, 64>{});
         }
+        if (okw && nunits > 0) epilogue(nunits - 1);
     }
     if (*abort) {
         // a wait gave up: let bulk copies still in flight into this CTA land
