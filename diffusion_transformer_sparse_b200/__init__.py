@@ -33,6 +33,7 @@ EXPORTS = (
     "ptdit_debug_thl_map", "ptdit_debug_thl_units", "ptdit_debug_gemm_schedule",
     "ptdit_proxy_extract", "ptdit_giim_ex", "ptdit_pt_block", "ptdit_pt_block_workspace_bytes",
     "ptdit_debug_wait_limit", "ptdit_window_attn_bwd", "ptdit_window_attn_bwd_workspace_bytes",
+    "ptdit_tcm_bwd", "ptdit_tcm_bwd_workspace_bytes",
 )
 
 
@@ -104,6 +105,10 @@ def lib() -> ctypes.CDLL:
             "ptdit_tcm": (ctypes.c_int, [_S, _I3, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
                                          ctypes.c_size_t, _P]),
             "ptdit_window_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
+            "ptdit_tcm_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
+            "ptdit_tcm_bwd": (ctypes.c_int, [_S, _I3, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
+                                             ctypes.POINTER(AttnWgrad), ctypes.POINTER(AttnWgrad),
+                                             _P, ctypes.c_size_t, _P]),
             "ptdit_window_attn_bwd": (ctypes.c_int, [_S, _I3, _I3, _W, ctypes.c_uint, _P, _P, _P,
                                                      ctypes.POINTER(AttnWgrad), _P,
                                                      ctypes.c_size_t, _P]),
@@ -367,6 +372,32 @@ def ptdit_window_attn_bwd(z_in, dz_out, grid, window, shift, w, heads, flags=0, 
                                        _ptr(dz_in), ctypes.byref(g), _ptr(ws), ws.numel(),
                                        _stream(stream)))
     return dz_in, tuple(dw)
+
+
+def ptdit_tcm_bwd(z_in, dz_out, grid, window, shift, wsa, swsa, heads, flags=0, dz_in=None,
+                  ws=None, stream=None):
+    """Backward of ptdit_tcm: returns (dz_in, dW_wsa, dW_swsa), each dW four fp32 [D, D]."""
+    import torch
+    _check_z(z_in)
+    _check_z(dz_out)
+    shape = make_shape(z_in, grid, heads)
+    if dz_in is None:
+        dz_in = torch.empty_like(z_in)
+    D = z_in.shape[-1]
+    dwa = tuple(torch.empty(D, D, dtype=torch.float32, device=z_in.device) for _ in range(4))
+    dwb = tuple(torch.empty(D, D, dtype=torch.float32, device=z_in.device) for _ in range(4))
+    if ws is None:
+        n = lib().ptdit_tcm_bwd_workspace_bytes(ctypes.byref(shape), _i3(window))
+        if n == 0:
+            raise PtditError(PTDIT_ERR_SHAPE, "invalid shape or window")
+        ws = torch.empty(n, dtype=torch.uint8, device=z_in.device)
+    wa, wb = attn_w(wsa), attn_w(swsa)
+    ga, gb = AttnWgrad(*[_ptr(x) for x in dwa]), AttnWgrad(*[_ptr(x) for x in dwb])
+    _check(lib().ptdit_tcm_bwd(ctypes.byref(shape), _i3(window), _i3(shift), ctypes.byref(wa),
+                               ctypes.byref(wb), flags, _ptr(z_in), _ptr(dz_out), _ptr(dz_in),
+                               ctypes.byref(ga), ctypes.byref(gb), _ptr(ws), ws.numel(),
+                               _stream(stream)))
+    return dz_in, dwa, dwb
 
 
 def ptdit_tcm(z_in, grid, window, shift, wsa, swsa, heads, flags=0, z_out=None, ws=None,

@@ -842,6 +842,64 @@ int run_window_bwd(const Run &r, const WsBwd &Lb, const WinGeom &wg, const ptdit
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "weight gradients");
 }
 
+// The TCM backward's workspace: the branch backward's, then z^ and dL/dz^.
+struct TcmBwd {
+    WsBwd bwd;
+    size_t zh, dzh, total;
+};
+TcmBwd tcm_bwd_layout(const Dims &d) {
+    TcmBwd T;
+    T.bwd = ws_layout_bwd(d);
+    const size_t tn = align256((size_t)d.B * d.N * d.D * d.elem);
+    T.zh = T.bwd.total;
+    T.dzh = T.zh + tn;
+    T.total = T.dzh + tn;
+    return T;
+}
+
+int check_bwd_io(const Dims &d, const ptdit_attn_w *w, const void *z_in, const void *dz_out,
+                 void *dz_in, const void *ws, size_t ws_bytes) {
+    TRY(check_io(d, z_in, dz_in, ws, ws_bytes));
+    TRY(check_ptr(dz_out, "dz_out"));
+    TRY(check_w_alias(d, w, dz_in));
+    const size_t zb = (size_t)d.B * d.N * d.D * d.elem;
+    if (overlap(dz_out, zb, dz_in, zb)) return fail(PTDIT_ERR_ALIAS, "dz_in overlaps dz_out");
+    if (ws && overlap(ws, ws_bytes, dz_out, zb))
+        return fail(PTDIT_ERR_ALIAS, "dz_out overlaps the workspace");
+    return PTDIT_OK;
+}
+
+int check_wgrad(const Dims &d, const ptdit_attn_wgrad *dw, const char *name, const void *z_in,
+                const void *dz_out, const void *dz_in, const void *ws, size_t ws_bytes) {
+    if (!dw) return fail(PTDIT_ERR_NULL, "%s is NULL", name);
+    const size_t zb = (size_t)d.B * d.N * d.D * d.elem, gb = (size_t)d.D * d.D * sizeof(float);
+    const float *outs[4] = {dw->dwq, dw->dwk, dw->dwv, dw->dwo};
+    const char *nm[4] = {"dwq", "dwk", "dwv", "dwo"};
+    for (int i = 0; i < 4; ++i) {
+        if (!outs[i]) return fail(PTDIT_ERR_NULL, "%s.%s is NULL", name, nm[i]);
+        if ((uintptr_t)outs[i] % 16)
+            return fail(PTDIT_ERR_ALIGN, "%s.%s is not 16-byte aligned", name, nm[i]);
+        if (overlap(outs[i], gb, dz_in, zb) || overlap(outs[i], gb, z_in, zb) ||
+            overlap(outs[i], gb, dz_out, zb) || (ws && overlap(outs[i], gb, ws, ws_bytes)))
+            return fail(PTDIT_ERR_ALIAS, "%s.%s overlaps another argument or the workspace",
+                        name, nm[i]);
+        for (int j = 0; j < i; ++j)
+            if (overlap(outs[i], gb, outs[j], gb))
+                return fail(PTDIT_ERR_ALIAS, "%s.%s overlaps %s.%s", name, nm[i], name, nm[j]);
+    }
+    return PTDIT_OK;
+}
+
+int check_bwd_ws(const void *ws, size_t ws_bytes, size_t need) {
+    if (fault("workspace"))
+        return fail(PTDIT_ERR_WORKSPACE, "workspace refused (PTDIT_FAULT=workspace)");
+    if (!ws) return fail(PTDIT_ERR_NULL, "workspace is NULL");
+    if ((uintptr_t)ws % 256) return fail(PTDIT_ERR_ALIGN, "workspace is not 256-byte aligned");
+    if (ws_bytes < need)
+        return fail(PTDIT_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+    return PTDIT_OK;
+}
+
 }  // namespace
 
 namespace ptdit {
@@ -1045,35 +1103,63 @@ int ptdit_window_attn_bwd(const ptdit_shape *shape, const int window[3], const i
     TRY(make_window(d, window, shift, &wg));
     TRY(check_bwd_shape(d, wg));
     TRY(check_weights(w, "w"));
-    TRY(check_io(d, z_in, dz_in, ws, ws_bytes));
-    TRY(check_ptr(dz_out, "dz_out"));
-    TRY(check_w_alias(d, w, dz_in));
-    if (!dw) return fail(PTDIT_ERR_NULL, "dw is NULL");
-    const size_t zb = (size_t)d.B * d.N * d.D * d.elem, gb = (size_t)d.D * d.D * sizeof(float);
-    if (overlap(dz_out, zb, dz_in, zb)) return fail(PTDIT_ERR_ALIAS, "dz_in overlaps dz_out");
-    if (ws && overlap(ws, ws_bytes, dz_out, zb))
-        return fail(PTDIT_ERR_ALIAS, "dz_out overlaps the workspace");
-    float *outs[4] = {dw->dwq, dw->dwk, dw->dwv, dw->dwo};
-    const char *nm[4] = {"dw.dwq", "dw.dwk", "dw.dwv", "dw.dwo"};
-    for (int i = 0; i < 4; ++i) {
-        TRY(check_ptr(outs[i], nm[i]));
-        if (overlap(outs[i], gb, dz_in, zb) || overlap(outs[i], gb, z_in, zb) ||
-            overlap(outs[i], gb, dz_out, zb) || (ws && overlap(outs[i], gb, ws, ws_bytes)))
-            return fail(PTDIT_ERR_ALIAS, "%s overlaps another argument or the workspace", nm[i]);
-        for (int j = 0; j < i; ++j)
-            if (overlap(outs[i], gb, outs[j], gb))
-                return fail(PTDIT_ERR_ALIAS, "%s overlaps %s", nm[i], nm[j]);
-    }
+    TRY(check_bwd_io(d, w, z_in, dz_out, dz_in, ws, ws_bytes));
+    TRY(check_wgrad(d, dw, "dw", z_in, dz_out, dz_in, ws, ws_bytes));
     const WsBwd Lb = ws_layout_bwd(d);
-    if (fault("workspace"))
-        return fail(PTDIT_ERR_WORKSPACE, "workspace refused (PTDIT_FAULT=workspace)");
-    if (!ws) return fail(PTDIT_ERR_NULL, "workspace is NULL");
-    if ((uintptr_t)ws % 256) return fail(PTDIT_ERR_ALIGN, "workspace is not 256-byte aligned");
-    if (ws_bytes < Lb.total)
-        return fail(PTDIT_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, Lb.total);
+    TRY(check_bwd_ws(ws, ws_bytes, Lb.total));
     const Ws none{};
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), none};
     return run_window_bwd(r, Lb, wg, w, flags, z_in, dz_out, dz_in, dw);
+}
+
+size_t ptdit_tcm_bwd_workspace_bytes(const ptdit_shape *shape, const int window[3]) {
+    Dims d;
+    if (check_shape(shape, &d) != PTDIT_OK) return 0;
+    const int zero[3] = {0, 0, 0};
+    WinGeom wg;
+    if (make_window(d, window, zero, &wg) != PTDIT_OK) return 0;
+    return tcm_bwd_layout(d).total;
+}
+
+int ptdit_tcm_bwd(const ptdit_shape *shape, const int window[3], const int shift[3],
+                  const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
+                  const void *z_in, const void *dz_out, void *dz_in,
+                  const ptdit_attn_wgrad *dw_wsa, const ptdit_attn_wgrad *dw_swsa, void *ws,
+                  size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    WinGeom wg0, wg1;
+    const int zero[3] = {0, 0, 0};
+    TRY(check_shape(shape, &d));
+    TRY(make_window(d, window, shift, &wg1));
+    TRY(make_window(d, window, zero, &wg0));
+    TRY(check_bwd_shape(d, wg0));
+    TRY(check_weights(wsa, "wsa"));
+    TRY(check_weights(swsa, "swsa"));
+    TRY(check_bwd_io(d, wsa, z_in, dz_out, dz_in, ws, ws_bytes));
+    TRY(check_bwd_io(d, swsa, z_in, dz_out, dz_in, ws, ws_bytes));
+    TRY(check_wgrad(d, dw_wsa, "dw_wsa", z_in, dz_out, dz_in, ws, ws_bytes));
+    TRY(check_wgrad(d, dw_swsa, "dw_swsa", z_in, dz_out, dz_in, ws, ws_bytes));
+    {
+        const size_t gb = (size_t)d.D * d.D * sizeof(float);
+        const float *a[4] = {dw_wsa->dwq, dw_wsa->dwk, dw_wsa->dwv, dw_wsa->dwo};
+        const float *b[4] = {dw_swsa->dwq, dw_swsa->dwk, dw_swsa->dwv, dw_swsa->dwo};
+        for (int i = 0; i < 4; ++i)
+            for (int j = 0; j < 4; ++j)
+                if (overlap(a[i], gb, b[j], gb))
+                    return fail(PTDIT_ERR_ALIAS, "dw_wsa and dw_swsa overlap");
+    }
+    const TcmBwd T = tcm_bwd_layout(d);
+    TRY(check_bwd_ws(ws, ws_bytes, T.total));
+    // z^ = WSA(z_in) (+ z_in), with the forward's workspace laid over the backward's
+    Ws Lf{};
+    Lf.Q = T.bwd.Q; Lf.K = T.bwd.K; Lf.V = T.bwd.V; Lf.O = T.bwd.A;
+    Run rf{d, (cudaStream_t)stream, static_cast<char *>(ws), Lf};
+    void *zh = rf.at(T.zh), *dzh = rf.at(T.dzh);
+    TRY(run_window(rf, wg0, wsa, flags, z_in, zh));
+    const Ws none{};
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), none};
+    TRY(run_window_bwd(r, T.bwd, wg1, swsa, flags, zh, dz_out, dzh, dw_swsa));
+    return run_window_bwd(r, T.bwd, wg0, wsa, flags, z_in, dzh, dz_in, dw_wsa);
 }
 
 int ptdit_tcm(const ptdit_shape *shape, const int window[3], const int shift[3],

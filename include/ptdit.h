@@ -214,6 +214,21 @@ int ptdit_window_attn_bwd(const ptdit_shape *shape, const int window[3], const i
                           size_t ws_bytes, ptdit_stream_t stream);
 
 /*
+ * ptdit_tcm_bwd -- backward of ptdit_tcm: z^ = WSA(z_in) (+ z_in) is recomputed,
+ *   then the SWSA branch's backward at z^ and the WSA branch's backward at
+ *   z_in (each as ptdit_window_attn_bwd).  dw_wsa and dw_swsa receive the two
+ *   modules' weight gradients (fp32, overwritten).  Workspace:
+ *   ptdit_tcm_bwd_workspace_bytes(shape, window).  Restrictions and errors as
+ *   ptdit_window_attn_bwd.
+ */
+size_t ptdit_tcm_bwd_workspace_bytes(const ptdit_shape *shape, const int window[3]);
+int ptdit_tcm_bwd(const ptdit_shape *shape, const int window[3], const int shift[3],
+                  const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
+                  const void *z_in, const void *dz_out, void *dz_in,
+                  const ptdit_attn_wgrad *dw_wsa, const ptdit_attn_wgrad *dw_swsa, void *ws,
+                  size_t ws_bytes, ptdit_stream_t stream);
+
+/*
  * ptdit_tcm -- Eq. TCM: WSA with weights wsa, then SWSA with weights swsa
  *   and the given shift, each with its residual (unless PTDIT_NO_RESIDUAL).
  */

@@ -408,6 +408,18 @@ def window_self_attention_bwd(z, grid, window, shift, W, heads, dout, *, residua
     return dz, (dWq, dWk, dWv, dWo)
 
 
+def tcm_bwd(z, grid, window, shift, W_wsa, W_swsa, heads, dout, *, residual=True):
+    """Backward of tcm: the chain rule through its two branches.  z^ = WSA(z) (+ z) is
+    recomputed; SWSA's backward at z^ gives dL/dz^ and SWSA's weight gradients, WSA's
+    backward at z with dL/dz^ gives dL/dz and WSA's.  Returns (dz, dW_wsa, dW_swsa)."""
+    zh = window_self_attention(z, grid, window, (0, 0, 0), W_wsa, heads, residual=residual)
+    dzh, dW_swsa = window_self_attention_bwd(zh, grid, window, shift, W_swsa, heads, dout,
+                                             residual=residual)
+    dz, dW_wsa = window_self_attention_bwd(z, grid, window, (0, 0, 0), W_wsa, heads, dzh,
+                                           residual=residual)
+    return dz, dW_wsa, dW_swsa
+
+
 def tcm(z, grid, window, shift, W_wsa, W_swsa, heads, *, residual=True) -> np.ndarray:
     """ẑ = WSA(z) + z;  z_w = SWSA(ẑ) + ẑ   [T2X §3 Eq. TCM]."""
     zh = window_self_attention(z, grid, window, (0, 0, 0), W_wsa, heads, residual=residual)

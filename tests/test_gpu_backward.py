@@ -92,3 +92,29 @@ def test_window_bwd_refuses_what_it_does_not_run():
     with pytest.raises(pt.PtditError) as e:  # fp32
         pt.ptdit_window_attn_bwd(z32, z32.clone(), (1, 16, 16), (1, 8, 8), (0, 0, 0), w32, 2)
     assert e.value.code == pt.PTDIT_ERR_DTYPE
+
+
+@pytest.mark.parametrize("grid,D,heads,window,shift,B", [
+    ((2, 16, 16), 256, 4, (2, 8, 8), (1, 4, 4), 1),
+    ((1, 64, 64), 1152, 16, (1, 8, 8), (0, 4, 4), 2),
+])
+def test_tcm_bwd(grid, D, heads, window, shift, B):
+    """Both TCM branches: dL/dz and each module's weight gradients."""
+    c = Case(B, grid, D, heads, "bf16")
+    dout_cpu = _dout(c.B, c.N, c.D)
+    dz, dwa, dwb = pt.ptdit_tcm_bwd(c.z, dout_cpu.cuda(), c.grid, window, shift, c.w["wsa"],
+                                    c.w["swsa"], c.heads)
+    dz = c.out64(dz)
+    g64 = synth.as_f64(dout_cpu)
+    want_a = [np.zeros((c.D, c.D)) for _ in range(4)]
+    want_b = [np.zeros((c.D, c.D)) for _ in range(4)]
+    for b in range(c.B):
+        wdz, wa, wb = O.tcm_bwd(c.z64[b], c.grid, window, shift, c.w64["wsa"], c.w64["swsa"],
+                                c.heads, g64[b])
+        assert rel_err(dz[b], wdz) <= TOL["bf16"], ("dz", b)
+        for i in range(4):
+            want_a[i] += wa[i]
+            want_b[i] += wb[i]
+    for i in range(4):
+        assert rel_err(c.out64(dwa[i]), want_a[i]) <= TOL["bf16"], ("wsa", i)
+        assert rel_err(c.out64(dwb[i]), want_b[i]) <= TOL["bf16"], ("swsa", i)

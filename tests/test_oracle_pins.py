@@ -719,3 +719,30 @@ def test_pins_catch_swapped_query_and_key_gradients(monkeypatch):
 
     monkeypatch.setattr(O.ptdit_oracle, "attention_heads_bwd", swapped)
     assert _pin_fails(lambda: test_window_bwd_matches_finite_differences(*BWD_CASES[2]))
+
+
+def test_tcm_bwd_matches_finite_differences():
+    """The two-branch composition: directional derivatives of <dout, tcm(z)> in z and in
+    one weight of each module."""
+    grid, window, shift = (2, 4, 4), (2, 2, 2), (1, 1, 1)
+    D, heads = 8, 2
+    z, dout, Wa = _bwd_inputs(grid, D, 31)
+    Wb = _weights(D, 77, scale=0.5)
+    dz, dWa, dWb = O.tcm_bwd(z, grid, window, shift, Wa, Wb, heads, dout)
+
+    def L(zz, A, Bw):
+        return float(np.sum(dout * O.tcm(zz, grid, window, shift, A, Bw, heads)))
+
+    rng = np.random.default_rng(5)
+    eps = 1e-5
+    U = rng.standard_normal(z.shape)
+    fd = (L(z + eps * U, Wa, Wb) - L(z - eps * U, Wa, Wb)) / (2 * eps)
+    assert abs(fd - np.sum(dz * U)) <= 1e-7 * max(1.0, abs(fd))
+    for which, grads in ((0, dWa), (1, dWb)):
+        for i in (0, 3):
+            V = rng.standard_normal((D, D))
+            P, M = [list(Wa), list(Wb)], [list(Wa), list(Wb)]
+            P[which][i] = P[which][i] + eps * V
+            M[which][i] = M[which][i] - eps * V
+            fd = (L(z, tuple(P[0]), tuple(P[1])) - L(z, tuple(M[0]), tuple(M[1]))) / (2 * eps)
+            assert abs(fd - np.sum(grads[i] * V)) <= 1e-7 * max(1.0, abs(fd)), (which, i)
