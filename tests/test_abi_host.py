@@ -228,3 +228,75 @@ def test_pt_block_workspace_covers_the_attention_path(L):
     # plus the norm output, the MLP hidden layer and the text K / V blocks
     assert n >= attn + 2 * 512 * 4608 * 2 + 2 * 512 * 1152 * 2
     assert L.ptdit_pt_block_workspace_bytes(ctypes.byref(s), pt._i3((1, 4, 4)), 0, 4608) == 0
+
+
+# ---------------------------------------------------------------- backward entry points (host checks)
+
+def _bshape(**kw):
+    d = dict(B=1, F=1, H=16, W=16, D=128, heads=2, dtype=pt.PTDIT_BF16)
+    d.update(kw)
+    return pt.Shape(**d)
+
+
+def _wg(base):
+    return pt.AttnWgrad(base, base + 0x100000, base + 0x200000, base + 0x300000)
+
+
+def _bwd(L, shape, dw, window=(1, 8, 8), z_in=FAKE * 20, dz_out=FAKE * 21, dz_in=FAKE * 22,
+         ws_bytes=1 << 40):
+    g = None if dw is None else ctypes.byref(dw)
+    return L.ptdit_window_attn_bwd(ctypes.byref(shape), pt._i3(window), pt._i3((0, 4, 4)),
+                                   ctypes.byref(_w(FAKE * 2)), 0, z_in, dz_out, dz_in, g,
+                                   FAKE * 128, ws_bytes, None)
+
+
+def test_window_bwd_workspace_bytes(L):
+    s = _bshape(B=4, H=64, W=64, D=1152, heads=16)
+    n = L.ptdit_window_attn_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 8, 8)))
+    tq = 4 * 32 * 16 * 20480          # Q, K, V, dA window tiles (32 tiles per item)
+    tn = 4 * 4096 * 1152 * 2
+    assert n == 4 * tq + tn + 3 * tn + 1152 * 1152 * 2 + 3 * 1152 * 1152 * 2
+    t = L.ptdit_tcm_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 8, 8)))
+    assert t == n + 2 * tn  # plus z^ and dL/dz^
+    assert L.ptdit_window_attn_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 3, 8))) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(shape=dict(dtype=pt.PTDIT_F32)), 3),          # bf16 only
+    (dict(shape=dict(D=64, heads=1)), 2),                # D a multiple of 128
+    (dict(shape=dict(D=128, heads=1)), 2),               # head width 128: no bf16 kernel
+    (dict(window=(1, 4, 2)), 2),                         # a window of 8 tokens
+    (dict(dw=None), 1),
+    (dict(dw="null_dwk"), 1),
+    (dict(dw="misaligned_dwv"), 7),
+    (dict(dw="dwq_on_dz_in"), 8),
+    (dict(dz_in=FAKE * 21), 8),                          # dz_in is dz_out
+    (dict(dz_out=0), 1),
+    (dict(ws_bytes=4096), 4),
+])
+def test_window_bwd_rejects(L, kw, code):
+    """Every case fails validation on the host: nothing is launched."""
+    s = _bshape(**kw.pop("shape", {}))
+    dw = _wg(FAKE * 40)
+    special = kw.pop("dw", dw)
+    if special == "null_dwk":
+        dw.dwk = 0
+    elif special == "misaligned_dwv":
+        dw.dwv = FAKE * 40 + 0x200004
+    elif special == "dwq_on_dz_in":
+        dw.dwq = FAKE * 22
+    elif special is None:
+        dw = None
+    assert _bwd(L, s, dw, **kw) == code
+    assert L.ptdit_last_error()
+
+
+def test_tcm_bwd_rejects_overlapping_gradients(L):
+    s = _bshape()
+    a, b = _wg(FAKE * 40), _wg(FAKE * 40 + 0x300000)  # b.dwq is a.dwo
+    rc = L.ptdit_tcm_bwd(ctypes.byref(s), pt._i3((1, 8, 8)), pt._i3((0, 4, 4)),
+                         ctypes.byref(_w(FAKE * 2)), ctypes.byref(_w(FAKE * 3)), 0, FAKE * 20,
+                         FAKE * 21, FAKE * 22, ctypes.byref(a), ctypes.byref(b), FAKE * 128,
+                         1 << 40, None)
+    assert rc == 8
+    assert b"overlap" in L.ptdit_last_error()
