@@ -39,7 +39,8 @@ Readings taken where the pages are silent or ambiguous:
     row-major over (t, y, x);
   * every grid extent must be divisible by its ratio and its window.
 
-Backward (training) of a TCM branch: ``window_self_attention_bwd`` returns
+Backward (training) of GIIM: ``giim_bwd`` (``averaging_bwd`` is the averaging's
+adjoint).  Backward of a TCM branch: ``window_self_attention_bwd`` returns
 dL/dz and the four weight gradients for a given dL/dout, by the chain rule
 written out per window and head (``attention_heads_bwd`` holds the softmax
 Jacobian step); roll and window partition are row permutations, so their
@@ -260,6 +261,56 @@ def giim(z, grid, ratio, W_psa, W_cross, heads, *, proxy_residual=False, residua
 # --------------------------------------------------------------------------
 # TCM  [T2X §3 Eq. TCM; window_shift / window_Ishift; NEWS Technical Principles]
 # --------------------------------------------------------------------------
+
+def averaging_bwd(dP, grid, ratio) -> np.ndarray:
+    """Adjoint of averaging: every token of window m receives dP[m] / (p_f p_h p_w).
+    dP [M, D] -> [N, D]."""
+    _check_divisible(grid, ratio, "ratio")
+    f, h, w = grid
+    pf, ph, pw = ratio
+    dP = _f64(dP)
+    D = dP.shape[1]
+    g = dP.reshape(f // pf, 1, h // ph, 1, w // pw, 1, D) / (pf * ph * pw)
+    return np.broadcast_to(g, (f // pf, pf, h // ph, ph, w // pw, pw, D)).reshape(-1, D).copy()
+
+
+def giim_bwd(z, grid, ratio, W_psa, W_cross, heads, dout, *, proxy_residual=False,
+             residual=True):
+    """Backward of giim (window-mean proxies) on one batch item: the chain rule through
+    the cross-attention (queries from z, keys and values from P'), the proxy
+    self-attention and the averaging.  Returns (dz, dW_psa, dW_cross), the weight
+    gradients in the weights' [out][in] storage.
+        out = z + Ac Wco^T,  Ac = MHA core(z Wcq^T, P' Wck^T, P' Wcv^T)
+        P'  = Ap Wpo^T (+ P_a),  Ap = MHA core(P_a Wpq^T, P_a Wpk^T, P_a Wpv^T)
+        P_a = averaging(z)
+    """
+    z, dout = _f64(z), _f64(dout)
+    Wpq, Wpk, Wpv, Wpo = (_f64(x) for x in W_psa)
+    Wcq, Wck, Wcv, Wco = (_f64(x) for x in W_cross)
+    # forward, keeping what the backward reads
+    Pa = averaging(z, grid, ratio)
+    Pq, Pk, Pv = Pa @ Wpq.T, Pa @ Wpk.T, Pa @ Wpv.T
+    Ap = attention_heads(Pq, Pk, Pv, heads)
+    Pp = Ap @ Wpo.T + (Pa if proxy_residual else 0.0)
+    Cq, Ck, Cv = z @ Wcq.T, Pp @ Wck.T, Pp @ Wcv.T
+    Ac = attention_heads(Cq, Ck, Cv, heads)
+    # cross-attention and its projections
+    dWco = dout.T @ Ac
+    dCq, dCk, dCv = attention_heads_bwd(Cq, Ck, Cv, dout @ Wco, heads)
+    dz = dCq @ Wcq
+    dWcq, dWck, dWcv = dCq.T @ z, dCk.T @ Pp, dCv.T @ Pp
+    dPp = dCk @ Wck + dCv @ Wcv
+    # proxy self-attention and its projections
+    dWpo = dPp.T @ Ap
+    dPq, dPk, dPv = attention_heads_bwd(Pq, Pk, Pv, dPp @ Wpo, heads)
+    dPa = dPq @ Wpq + dPk @ Wpk + dPv @ Wpv + (dPp if proxy_residual else 0.0)
+    dWpq, dWpk, dWpv = dPq.T @ Pa, dPk.T @ Pa, dPv.T @ Pa
+    # the averaging
+    dz = dz + averaging_bwd(dPa, grid, ratio)
+    if residual:
+        dz = dz + dout
+    return dz, (dWpq, dWpk, dWpv, dWpo), (dWcq, dWck, dWcv, dWco)
+
 
 def _to_windows(g, window) -> np.ndarray:
     """[f, h, w, ...] -> [num_windows, n, ...]: windows row-major, slots row-major (t, y, x)."""

@@ -746,3 +746,55 @@ def test_tcm_bwd_matches_finite_differences():
             M[which][i] = M[which][i] - eps * V
             fd = (L(z, tuple(P[0]), tuple(P[1])) - L(z, tuple(M[0]), tuple(M[1]))) / (2 * eps)
             assert abs(fd - np.sum(grads[i] * V)) <= 1e-7 * max(1.0, abs(fd)), (which, i)
+
+
+
+# ---------------------------------------------------------------- backward of GIIM
+
+@pytest.mark.parametrize("proxy_residual", [False, True])
+def test_giim_bwd_matches_finite_differences(proxy_residual):
+    """Directional derivatives of <dout, giim(z)> in z and in every weight of both modules."""
+    grid, ratio, D, heads = (2, 4, 4), (1, 2, 2), 8, 2
+    rng = np.random.default_rng(9)
+    N = O.num_tokens(grid)
+    z, dout = rng.standard_normal((N, D)), rng.standard_normal((N, D))
+    Wp, Wc = _weights(D, 41, scale=0.5), _weights(D, 42, scale=0.5)
+    dz, dWp, dWc = O.giim_bwd(z, grid, ratio, Wp, Wc, heads, dout, proxy_residual=proxy_residual)
+
+    def L(zz, A, C):
+        return float(np.sum(dout * O.giim(zz, grid, ratio, A, C, heads,
+                                          proxy_residual=proxy_residual)))
+
+    eps = 1e-5
+    U = rng.standard_normal(z.shape)
+    fd = (L(z + eps * U, Wp, Wc) - L(z - eps * U, Wp, Wc)) / (2 * eps)
+    assert abs(fd - np.sum(dz * U)) <= 1e-7 * max(1.0, abs(fd))
+    for which, grads in ((0, dWp), (1, dWc)):
+        for i in range(4):
+            V = rng.standard_normal((D, D))
+            P, M = [list(Wp), list(Wc)], [list(Wp), list(Wc)]
+            P[which][i] = P[which][i] + eps * V
+            M[which][i] = M[which][i] - eps * V
+            fd = (L(z, tuple(P[0]), tuple(P[1])) - L(z, tuple(M[0]), tuple(M[1]))) / (2 * eps)
+            assert abs(fd - np.sum(grads[i] * V)) <= 1e-7 * max(1.0, abs(fd)), (which, i)
+
+
+def test_averaging_bwd_is_the_adjoint():
+    """<averaging(z), dP> = <z, averaging_bwd(dP)> for random z, dP."""
+    grid, ratio = (4, 6, 4), (2, 3, 2)
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((O.num_tokens(grid), 5))
+    dP = rng.standard_normal((O.averaging(z, grid, ratio).shape[0], 5))
+    lhs = np.sum(O.averaging(z, grid, ratio) * dP)
+    rhs = np.sum(z * O.averaging_bwd(dP, grid, ratio))
+    assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs))
+
+
+def test_pins_catch_an_averaging_adjoint_without_the_divisor(monkeypatch):
+    real = O.ptdit_oracle.averaging_bwd
+
+    def no_divisor(dP, grid, ratio):
+        return real(dP, grid, ratio) * (ratio[0] * ratio[1] * ratio[2])
+
+    monkeypatch.setattr(O.ptdit_oracle, "averaging_bwd", no_divisor)
+    assert _pin_fails(lambda: test_giim_bwd_matches_finite_differences(False))
