@@ -22,7 +22,7 @@ PROXY_MODES = {"mean": PTDIT_PROXY_MEAN, "first": PTDIT_PROXY_FIRST, "random": P
 (PTDIT_OK, PTDIT_ERR_NULL, PTDIT_ERR_SHAPE, PTDIT_ERR_DTYPE, PTDIT_ERR_WORKSPACE, PTDIT_ERR_CUDA,
  PTDIT_ERR_TIMEOUT, PTDIT_ERR_ALIGN, PTDIT_ERR_ALIAS) = range(9)
 KINDS = ("average", "gemm", "attn_proxy", "attn_cross", "attn_window", "attn_dense", "norm",
-         "attn_text", "attn_window_bwd", "wgrad", "transpose")
+         "attn_text", "attn_window_bwd", "wgrad", "transpose", "attn_rows_bwd")
 
 # Every symbol declared in include/ptdit.h.
 EXPORTS = (
@@ -33,7 +33,8 @@ EXPORTS = (
     "ptdit_debug_thl_map", "ptdit_debug_thl_units", "ptdit_debug_gemm_schedule",
     "ptdit_proxy_extract", "ptdit_giim_ex", "ptdit_pt_block", "ptdit_pt_block_workspace_bytes",
     "ptdit_debug_wait_limit", "ptdit_window_attn_bwd", "ptdit_window_attn_bwd_workspace_bytes",
-    "ptdit_tcm_bwd", "ptdit_tcm_bwd_workspace_bytes",
+    "ptdit_tcm_bwd", "ptdit_tcm_bwd_workspace_bytes", "ptdit_giim_bwd",
+    "ptdit_giim_bwd_workspace_bytes",
 )
 
 
@@ -106,6 +107,10 @@ def lib() -> ctypes.CDLL:
                                          ctypes.c_size_t, _P]),
             "ptdit_window_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
             "ptdit_tcm_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
+            "ptdit_giim_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
+            "ptdit_giim_bwd": (ctypes.c_int, [_S, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
+                                              ctypes.POINTER(AttnWgrad), ctypes.POINTER(AttnWgrad),
+                                              _P, ctypes.c_size_t, _P]),
             "ptdit_tcm_bwd": (ctypes.c_int, [_S, _I3, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
                                              ctypes.POINTER(AttnWgrad), ctypes.POINTER(AttnWgrad),
                                              _P, ctypes.c_size_t, _P]),
@@ -372,6 +377,33 @@ def ptdit_window_attn_bwd(z_in, dz_out, grid, window, shift, w, heads, flags=0, 
                                        _ptr(dz_in), ctypes.byref(g), _ptr(ws), ws.numel(),
                                        _stream(stream)))
     return dz_in, tuple(dw)
+
+
+def ptdit_giim_bwd(z_in, dz_out, grid, ratio, psa, cross, heads, flags=0, dz_in=None, ws=None,
+                   stream=None):
+    """Backward of ptdit_giim (window-mean proxies): returns (dz_in, dW_psa, dW_cross), each
+    dW four fp32 [D, D]."""
+    import torch
+    _check_z(z_in)
+    _check_z(dz_out)
+    shape = make_shape(z_in, grid, heads)
+    if dz_in is None:
+        dz_in = torch.empty_like(z_in)
+    D = z_in.shape[-1]
+    dwp = tuple(torch.empty(D, D, dtype=torch.float32, device=z_in.device) for _ in range(4))
+    dwc = tuple(torch.empty(D, D, dtype=torch.float32, device=z_in.device) for _ in range(4))
+    if ws is None:
+        n = lib().ptdit_giim_bwd_workspace_bytes(ctypes.byref(shape), _i3(ratio))
+        if n == 0:
+            raise PtditError(PTDIT_ERR_SHAPE, "invalid shape or ratio")
+        ws = torch.empty(n, dtype=torch.uint8, device=z_in.device)
+    wp, wc = attn_w(psa), attn_w(cross)
+    gp, gc = AttnWgrad(*[_ptr(x) for x in dwp]), AttnWgrad(*[_ptr(x) for x in dwc])
+    _check(lib().ptdit_giim_bwd(ctypes.byref(shape), _i3(ratio), ctypes.byref(wp),
+                                ctypes.byref(wc), flags, _ptr(z_in), _ptr(dz_out), _ptr(dz_in),
+                                ctypes.byref(gp), ctypes.byref(gc), _ptr(ws), ws.numel(),
+                                _stream(stream)))
+    return dz_in, dwp, dwc
 
 
 def ptdit_tcm_bwd(z_in, dz_out, grid, window, shift, wsa, swsa, heads, flags=0, dz_in=None,

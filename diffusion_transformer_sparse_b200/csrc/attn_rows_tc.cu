@@ -369,7 +369,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (DPAD > 64) tmem_ld16(t_o + 64, *reinterpret_cast<uint32_t(*)[16]>(ov + 64));
                 tmem_ld_wait();
                 // SUMV: column d = DPAD - 8 of O holds the row sum of P
-                const float inv = 1.f / (SUMV ? __uint_as_float(ov[DPAD - 8]) : l_i);
+                const float lrow = SUMV ? __uint_as_float(ov[DPAD - 8]) : l_i;
+                const float inv = 1.f / lrow;
+                // the row's log-sum-exp of the scaled scores, base 2 (for a backward pass)
+                if (a.lse) {
+                    const int q = qp * 2 * BQ + g * BQ + r;
+                    if (q < a.nq) a.lse[((long)b * a.heads + h) * a.nq + q] = m_ref + __log2f(lrow);
+                }
 #pragma unroll
                 for (int u = 0; u < DPAD / 8; ++u)
                     if (u < nch) {

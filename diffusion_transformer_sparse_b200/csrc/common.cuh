@@ -234,6 +234,14 @@ struct WgradArgs {
 bool wgrad_supported(const WgradArgs &a);
 cudaError_t launch_wgrad(const WgradArgs &a, cudaStream_t s);
 
+// GIIM backward's element-wise steps (bf16): delta[b][h][q] = dO . O over head h's
+// columns of row q of item b (dO in tiled head layout, identity tiles without
+// padding; O row-major with row stride ld); dz = (dout +) dPa[proxy] / P.
+cudaError_t launch_row_delta(const void *dO_tiles, const void *O, int B, int nq, int heads,
+                             int d, long ld, float *delta, cudaStream_t s);
+cudaError_t launch_proxy_broadcast(const ProxyGeom &g, int B, int D, const void *dPa,
+                                   const void *dout, void *dz, cudaStream_t s);
+
 // dst[c][r] = src[r][c] for a row-major bf16 [rows][cols] matrix (dst has
 // row stride ldd >= rows, so several transposes can fill one wider matrix).
 cudaError_t launch_transpose_bf16(const void *src, int rows, int cols, void *dst, long ldd,
@@ -263,6 +271,9 @@ struct AttnArgs {
     WinGeom geom;                  // ATT_WINDOW geometry
     float scale;                   // 1/sqrt(d)
     ThlDesc tq, tk, tv;            // layouts of q, k, v (mode 0: row-major with ldq...)
+    // ATT_ROWS on the tensor cores, when set: each query row's log2-sum-exp2 of its
+    // scaled scores, [B][heads][nq] (the backward recomputes P from it)
+    float *lse;
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s);
 // Backward of window attention: a holds the window tiles of Q, K, V (tiled
@@ -270,6 +281,29 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s);
 // [0, D), [D, 2D), [2D, 3D) of the row-major [B N][ldg] buffer dqkv.
 cudaError_t launch_attention_win_bwd(const AttnArgs &a, const void *dout, void *dqkv, long ldg,
                                      cudaStream_t s);
+// Backward of row attention: a holds identity tiles of Q (nq rows), K and V (nk
+// rows, V without padding), dout those of dL/dO; lse and delta are [B][heads][nq].
+// Writes dQ of key tile j into columns [j D, (j + 1) D) of the bf16 [B nq][ldq]
+// buffer dq and adds dK, dV into the zeroed fp32 [B nk][D] buffers dk, dv.
+// kmean (fp32 [B][D], the mean of each item's key rows, or NULL): dQ of every key
+// tile is taken against the keys less kmean (each row of the exact dS sums to
+// zero, so dS K = dS (K - kmean); with the rounded dS, the second form keeps the
+// keys' common component out of dQ).
+cudaError_t launch_attention_rows_bwd(const AttnArgs &a, const void *dout, const float *lse,
+                                      const float *delta, const float *kmean, void *dq, long ldq,
+                                      float *dk, float *dv, cudaStream_t s);
+// mean[b][h d + c] = the mean over the nk key rows of item b of column c of head h,
+// K in tiled head layout (identity tiles, no padding).
+cudaError_t launch_key_mean(const void *K_tiles, int B, int nk, int heads, int d, float *mean,
+                            cudaStream_t s);
+// dst[b M + r][c] = bf16(src[b M + r][c] - mean over r' of src[b M + r'][c]) for the
+// fp32 row-major [B M][cols] src; dst has row stride ldd.
+cudaError_t launch_center_to_bf16(const float *src, int B, int M, int cols, void *dst, long ldd,
+                                  cudaStream_t s);
+// fp32 -> bf16, n elements (a multiple of 8), into a strided destination: element
+// i of row i / cols goes to dst[(i / cols) ldd + i % cols].
+cudaError_t launch_to_bf16(const float *src, long rows, int cols, void *dst, long ldd,
+                           cudaStream_t s);
 
 // Debug maps written with the kernels' own index functions.
 cudaError_t launch_debug_proxy_map(const ProxyGeom &g, int32_t *out, cudaStream_t s);

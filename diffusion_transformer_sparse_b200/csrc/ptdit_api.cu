@@ -900,6 +900,248 @@ int check_bwd_ws(const void *ws, size_t ws_bytes, size_t need) {
     return PTDIT_OK;
 }
 
+// ------------------------------------------------------------------ backward of GIIM
+struct WsGB {
+    size_t Pa, Pq, Pk, Pvf, Pvb, Ap, Pp, Ck, Cvf, Cvb, dAp, dPp, dKVc, Gp, dPa;
+    size_t dKc, dVc, dKp, dVp, lse_p, del_p, km_p;
+    size_t Cq, Ac, dAc, Gc, lse_c, del_c, km_c;
+    size_t WcoT, WcqT, WckvT, WpoT, WpT;
+    int ktc, ktp;
+    size_t total;
+};
+
+WsGB ws_layout_giim_bwd(const Dims &d, long M) {
+    WsGB L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    const size_t e = d.elem, BM = (size_t)d.B * M, BN = (size_t)d.B * d.N, D = d.D;
+    const size_t tp = thl_bytes(d, M, 0), tpv = thl_bytes(d, M, 1), tn = thl_bytes(d, d.N, 0);
+    L.ktc = L.ktp = (int)((M + kThlRows - 1) / kThlRows);
+    L.Pa = take(BM * D * e); L.Pq = take(tp); L.Pk = take(tp); L.Pvf = take(tpv); L.Pvb = take(tp);
+    L.Ap = take(BM * D * e); L.Pp = take(BM * D * e);
+    L.Ck = take(tp); L.Cvf = take(tpv); L.Cvb = take(tp);
+    L.dAp = take(tp); L.dPp = take(BM * D * e); L.dKVc = take(BM * 2 * D * e);
+    L.Gp = take(BM * (L.ktp + 2) * D * e); L.dPa = take(BM * D * e);
+    L.dKc = take(BM * D * 4); L.dVc = take(BM * D * 4); L.dKp = take(BM * D * 4);
+    L.dVp = take(BM * D * 4);
+    L.lse_p = take(BM * d.heads * 4); L.del_p = take(BM * d.heads * 4);
+    L.km_p = take((size_t)d.B * D * 4); L.km_c = take((size_t)d.B * D * 4);
+    L.Cq = take(tn); L.Ac = take(BN * D * e); L.dAc = take(tn); L.Gc = take(BN * L.ktc * D * e);
+    L.lse_c = take(BN * d.heads * 4); L.del_c = take(BN * d.heads * 4);
+    L.WcoT = take(D * D * e); L.WcqT = take(D * L.ktc * D * e); L.WckvT = take(D * 2 * D * e);
+    L.WpoT = take(D * D * e); L.WpT = take(D * (L.ktp + 2) * D * e);
+    L.total = off;
+    return L;
+}
+
+// dW[i] (+)= G^T X over `rows` rows for column blocks gcol[i] of G: launches of up to
+// kWgradMax matrices (several blocks may add into one dW).
+int wgrad_blocks(const Run &r, const void *G, int ldg, const int *gcol, float *const *dW, int n,
+                 const void *X, long rows, const char *what) {
+    for (int i0 = 0; i0 < n; i0 += kWgradMax) {
+        WgradArgs g;
+        memset(&g, 0, sizeof g);
+        g.G[0] = G; g.ldg[0] = ldg; g.X[0] = X; g.ldx[0] = r.d.D;
+        g.nmat = n - i0 < kWgradMax ? n - i0 : kWgradMax;
+        for (int i = 0; i < g.nmat; ++i) {
+            g.src[i] = 0;
+            g.gcol[i] = gcol[i0 + i];
+            g.dW[i] = dW[i0 + i];
+        }
+        g.M = g.N = r.d.D;
+        g.rows = (int)rows;
+        if (!wgrad_supported(g)) return cuda_fail(cudaErrorNotSupported, what);
+        TRY(launch_fault(what));
+        timing_begin(PTDIT_K_WGRAD, r.s);
+        cudaError_t e = launch_wgrad(g, r.s);
+        timing_end(r.s);
+        count_launch();
+        if (e != cudaSuccess) return cuda_fail(e, what);
+    }
+    return PTDIT_OK;
+}
+
+// Row-attention backward with the keys' mean (kmean, fp32 [B][D]) taken first.
+int rows_bwd(const Run &r, AttnArgs a, const void *dO, const float *lse, const float *del,
+             float *kmean, void *dq, long ldq, float *dk, float *dv, const char *what) {
+    a.dtype = r.d.dtype;
+    a.heads = r.d.heads;
+    a.d = r.d.d;
+    a.B = r.d.B;
+    a.scale = 1.0f / sqrtf((float)r.d.d);
+    for (float *p : {dk, dv}) {
+        cudaError_t em = cudaMemsetAsync(p, 0, (size_t)r.d.B * a.nk * r.d.D * sizeof(float), r.s);
+        if (em != cudaSuccess) return cuda_fail(em, "zeroing the key and value gradients");
+    }
+    cudaError_t em = launch_key_mean(a.k, a.B, a.nk, a.heads, a.d, kmean, r.s);
+    count_launch();
+    if (em != cudaSuccess) return cuda_fail(em, "backward: key mean");
+    TRY(launch_fault(what));
+    timing_begin(PTDIT_K_ATTN_ROWS_BWD, r.s);
+    cudaError_t e = launch_attention_rows_bwd(a, dO, lse, del, kmean, dq, ldq, dk, dv, r.s);
+    timing_end(r.s);
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
+}
+
+int elementwise(const Run &r, cudaError_t e, const char *what) {
+    count_launch();
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
+}
+
+int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_attn_w *psa,
+                 const ptdit_attn_w *cross, unsigned flags, const void *z_in, const void *dz_out,
+                 void *dz_in, const ptdit_attn_wgrad *dwp, const ptdit_attn_wgrad *dwc) {
+    const Dims &d = r.d;
+    const int M = pg.M, D = d.D, ktc = Lb.ktc, ktp = Lb.ktp;
+    const long BM = (long)d.B * M, BN = (long)d.B * d.N;
+    auto P = [&](size_t o) { return r.at(o); };
+    auto F = [&](size_t o) { return reinterpret_cast<float *>(r.at(o)); };
+    const ThlDesc tp = thl_identity(M, 0), tpv = thl_identity(M, 1, v_ones(d));
+    const ThlDesc tn = thl_identity(d.N, 0);
+    // ---- the forward, recomputed, keeping what the backward reads
+    TRY(extract_proxies(d, pg, PTDIT_PROXY_MEAN, nullptr, z_in, P(Lb.Pa), r.s));
+    {
+        const void *W[3] = {psa->wq, psa->wk, psa->wv};
+        void *C[3] = {P(Lb.Pq), P(Lb.Pk), P(Lb.Pvf)};
+        const ThlDesc *T[3] = {&tp, &tp, &tpv};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, P(Lb.Pa), BM, 3, W, C, T, "backward: proxy QKV"));
+        const void *Wv[3] = {psa->wv, nullptr, nullptr};
+        void *Cv[3] = {P(Lb.Pvb), nullptr, nullptr};
+        const ThlDesc *Tv[3] = {&tp, nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, P(Lb.Pa), BM, 1, Wv, Cv, Tv, "backward: proxy V"));
+    }
+    AttnArgs pa;
+    memset(&pa, 0, sizeof pa);
+    pa.mode = ATT_ROWS;
+    pa.q = P(Lb.Pq); pa.k = P(Lb.Pk); pa.v = P(Lb.Pvf); pa.o = P(Lb.Ap);
+    pa.q_bstride = pa.k_bstride = M;
+    pa.nq = pa.nk = M;
+    pa.tq = pa.tk = tp;
+    pa.tv = tpv;
+    pa.lse = F(Lb.lse_p);
+    TRY(attention(r, PTDIT_K_ATTN_PROXY, pa, "backward: proxy self-attention"));
+    {
+        const void *W[3] = {psa->wo, nullptr, nullptr};
+        void *C[3] = {P(Lb.Pp), nullptr, nullptr};
+        const void *R[3] = {(flags & PTDIT_PROXY_RESIDUAL) ? P(Lb.Pa) : nullptr, nullptr, nullptr};
+        TRY(gemm(r, PTDIT_K_GEMM, P(Lb.Ap), BM, 1, W, C, R, "backward: proxy output"));
+    }
+    {
+        const void *W[3] = {cross->wk, cross->wv, cross->wv};
+        void *C[3] = {P(Lb.Ck), P(Lb.Cvf), P(Lb.Cvb)};
+        const ThlDesc *T[3] = {&tp, &tpv, &tp};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, P(Lb.Pp), BM, 3, W, C, T, "backward: proxy K/V"));
+        const void *Wq[3] = {cross->wq, nullptr, nullptr};
+        void *Cq[3] = {P(Lb.Cq), nullptr, nullptr};
+        const ThlDesc *Tq[3] = {&tn, nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 1, Wq, Cq, Tq, "backward: latent Q"));
+    }
+    AttnArgs ca;
+    memset(&ca, 0, sizeof ca);
+    ca.mode = ATT_ROWS;
+    ca.q = P(Lb.Cq); ca.k = P(Lb.Ck); ca.v = P(Lb.Cvf); ca.o = P(Lb.Ac);
+    ca.q_bstride = d.N;
+    ca.k_bstride = M;
+    ca.nq = (int)d.N;
+    ca.nk = M;
+    ca.tq = tn;
+    ca.tk = tp;
+    ca.tv = tpv;
+    ca.lse = F(Lb.lse_c);
+    TRY(attention(r, PTDIT_K_ATTN_CROSS, ca, "backward: cross-attention"));
+    // ---- transposed weights for the input gradients
+    TRY(transpose(r, cross->wo, D, D, P(Lb.WcoT), D));
+    for (int j = 0; j < ktc; ++j)
+        TRY(transpose(r, cross->wq, D, D, P(Lb.WcqT) + (size_t)j * D * d.elem, (long)ktc * D));
+    TRY(transpose(r, cross->wk, D, D, P(Lb.WckvT), 2L * D));
+    TRY(transpose(r, cross->wv, D, D, P(Lb.WckvT) + (size_t)D * d.elem, 2L * D));
+    TRY(transpose(r, psa->wo, D, D, P(Lb.WpoT), D));
+    const long ldp = (long)(ktp + 2) * D;
+    for (int j = 0; j < ktp; ++j)
+        TRY(transpose(r, psa->wq, D, D, P(Lb.WpT) + (size_t)j * D * d.elem, ldp));
+    TRY(transpose(r, psa->wk, D, D, P(Lb.WpT) + (size_t)ktp * D * d.elem, ldp));
+    TRY(transpose(r, psa->wv, D, D, P(Lb.WpT) + (size_t)(ktp + 1) * D * d.elem, ldp));
+    // ---- cross-attention backward
+    {
+        const void *W[3] = {P(Lb.WcoT), nullptr, nullptr};
+        void *C[3] = {P(Lb.dAc), nullptr, nullptr};
+        const ThlDesc *T[3] = {&tn, nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, dz_out, BN, 1, W, C, T, "backward: dA = dz_out Wo"));
+    }
+    TRY(elementwise(r, launch_row_delta(P(Lb.dAc), P(Lb.Ac), d.B, (int)d.N, d.heads, d.d, D,
+                                        F(Lb.del_c), r.s), "backward: rowsum(dO O)"));
+    AttnArgs cb = ca;
+    cb.v = P(Lb.Cvb);
+    cb.tv = tp;
+    TRY(rows_bwd(r, cb, P(Lb.dAc), F(Lb.lse_c), F(Lb.del_c), F(Lb.km_c), P(Lb.Gc), (long)ktc * D,
+                 F(Lb.dKc), F(Lb.dVc), "cross-attention backward"));
+    TRY(elementwise(r, launch_center_to_bf16(F(Lb.dKc), d.B, M, D, P(Lb.dKVc), 2L * D, r.s),
+                    "backward: dK"));
+    TRY(elementwise(r, launch_to_bf16(F(Lb.dVc), BM, D, P(Lb.dKVc) + (size_t)D * d.elem, 2L * D, r.s),
+                    "backward: dV"));
+    TRY(gemm_ex(r, PTDIT_K_GEMM, P(Lb.dKVc), BM, 2 * D, D, P(Lb.WckvT), P(Lb.dPp), nullptr, nullptr,
+                ACT_NONE, "backward: dP' = dK Wk + dV Wv"));
+    // ---- proxy self-attention backward
+    {
+        const void *W[3] = {P(Lb.WpoT), nullptr, nullptr};
+        void *C[3] = {P(Lb.dAp), nullptr, nullptr};
+        const ThlDesc *T[3] = {&tp, nullptr, nullptr};
+        TRY(gemm_thl(r, PTDIT_K_GEMM, P(Lb.dPp), BM, 1, W, C, T, "backward: dAp = dP' Wo"));
+    }
+    TRY(elementwise(r, launch_row_delta(P(Lb.dAp), P(Lb.Ap), d.B, M, d.heads, d.d, D, F(Lb.del_p),
+                                        r.s), "backward: proxy rowsum(dO O)"));
+    AttnArgs pb = pa;
+    pb.v = P(Lb.Pvb);
+    pb.tv = tp;
+    TRY(rows_bwd(r, pb, P(Lb.dAp), F(Lb.lse_p), F(Lb.del_p), F(Lb.km_p), P(Lb.Gp), ldp, F(Lb.dKp),
+                 F(Lb.dVp), "proxy self-attention backward"));
+    TRY(elementwise(r, launch_center_to_bf16(F(Lb.dKp), d.B, M, D, P(Lb.Gp) + (size_t)ktp * D * d.elem,
+                                             ldp, r.s), "backward: proxy dK"));
+    TRY(elementwise(r, launch_to_bf16(F(Lb.dVp), BM, D, P(Lb.Gp) + (size_t)(ktp + 1) * D * d.elem,
+                                      ldp, r.s), "backward: proxy dV"));
+    TRY(gemm_ex(r, PTDIT_K_GEMM, P(Lb.Gp), BM, (int)ldp, D, P(Lb.WpT), P(Lb.dPa),
+                (flags & PTDIT_PROXY_RESIDUAL) ? P(Lb.dPp) : nullptr, nullptr, ACT_NONE,
+                "backward: dP_a"));
+    // ---- dz_in = (dz_out +) averaging^T(dP_a) + sum over key tiles of dQ_j Wq
+    TRY(elementwise(r, launch_proxy_broadcast(pg, d.B, D, P(Lb.dPa),
+                                              (flags & PTDIT_NO_RESIDUAL) ? nullptr : dz_out, dz_in, r.s),
+                    "backward: averaging adjoint"));
+    TRY(gemm_ex(r, PTDIT_K_GEMM, P(Lb.Gc), BN, ktc * D, D, P(Lb.WcqT), dz_in, dz_in, nullptr,
+                ACT_NONE, "backward: input gradient"));
+    // ---- weight gradients
+    float *outs[8] = {dwp->dwq, dwp->dwk, dwp->dwv, dwp->dwo, dwc->dwq, dwc->dwk, dwc->dwv, dwc->dwo};
+    for (float *o : outs) {
+        cudaError_t em = cudaMemsetAsync(o, 0, (size_t)D * D * sizeof(float), r.s);
+        if (em != cudaSuccess) return cuda_fail(em, "zeroing the weight gradients");
+    }
+    {
+        const int c0[1] = {0};
+        float *o1[1] = {dwc->dwo};
+        TRY(wgrad_blocks(r, dz_out, D, c0, o1, 1, P(Lb.Ac), BN, "backward: dWo (cross)"));
+        int cq[64];
+        float *oq[64];
+        for (int j = 0; j < ktc && j < 64; ++j) { cq[j] = j * D; oq[j] = dwc->dwq; }
+        TRY(wgrad_blocks(r, P(Lb.Gc), ktc * D, cq, oq, ktc, z_in, BN, "backward: dWq (cross)"));
+        const int ckv[2] = {0, D};
+        float *okv[2] = {dwc->dwk, dwc->dwv};
+        TRY(wgrad_blocks(r, P(Lb.dKVc), 2 * D, ckv, okv, 2, P(Lb.Pp), BM, "backward: dWk, dWv (cross)"));
+        TRY(wgrad_blocks(r, P(Lb.dPp), D, c0, &outs[3], 1, P(Lb.Ap), BM, "backward: dWo (proxy)"));
+        int cp[66];
+        float *op[66];
+        int n = 0;
+        for (int j = 0; j < ktp && n < 64; ++j, ++n) { cp[n] = j * D; op[n] = dwp->dwq; }
+        cp[n] = ktp * D; op[n++] = dwp->dwk;
+        cp[n] = (ktp + 1) * D; op[n++] = dwp->dwv;
+        TRY(wgrad_blocks(r, P(Lb.Gp), (int)ldp, cp, op, n, P(Lb.Pa), BM, "backward: dWq, dWk, dWv (proxy)"));
+    }
+    return PTDIT_OK;
+}
+
 }  // namespace
 
 namespace ptdit {
@@ -1110,6 +1352,51 @@ int ptdit_window_attn_bwd(const ptdit_shape *shape, const int window[3], const i
     const Ws none{};
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), none};
     return run_window_bwd(r, Lb, wg, w, flags, z_in, dz_out, dz_in, dw);
+}
+
+size_t ptdit_giim_bwd_workspace_bytes(const ptdit_shape *shape, const int ratio[3]) {
+    Dims d;
+    ProxyGeom pg;
+    if (check_shape(shape, &d) != PTDIT_OK || make_proxy(d, ratio, &pg) != PTDIT_OK) return 0;
+    return ws_layout_giim_bwd(d, pg.M).total;
+}
+
+int ptdit_giim_bwd(const ptdit_shape *shape, const int ratio[3], const ptdit_attn_w *psa,
+                   const ptdit_attn_w *cross, unsigned flags, const void *z_in, const void *dz_out,
+                   void *dz_in, const ptdit_attn_wgrad *dw_psa, const ptdit_attn_wgrad *dw_cross,
+                   void *ws, size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    TRY(check_shape(shape, &d));
+    TRY(make_proxy(d, ratio, &pg));
+    if (d.dtype != PTDIT_BF16)
+        return fail(PTDIT_ERR_DTYPE, "the backward runs in bf16 only (tensor cores)");
+    TRY(check_bf16_attention(d));
+    if (d.D % 128)
+        return fail(PTDIT_ERR_SHAPE,
+                    "the backward's weight-gradient kernel takes D a multiple of 128; D=%d", d.D);
+    if ((pg.M + kThlRows - 1) / kThlRows > 64)
+        return fail(PTDIT_ERR_SHAPE, "the backward takes at most 8192 proxies; M=%d", pg.M);
+    TRY(check_weights(psa, "psa"));
+    TRY(check_weights(cross, "cross"));
+    TRY(check_bwd_io(d, psa, z_in, dz_out, dz_in, ws, ws_bytes));
+    TRY(check_bwd_io(d, cross, z_in, dz_out, dz_in, ws, ws_bytes));
+    TRY(check_wgrad(d, dw_psa, "dw_psa", z_in, dz_out, dz_in, ws, ws_bytes));
+    TRY(check_wgrad(d, dw_cross, "dw_cross", z_in, dz_out, dz_in, ws, ws_bytes));
+    {
+        const size_t gb = (size_t)d.D * d.D * sizeof(float);
+        const float *a[4] = {dw_psa->dwq, dw_psa->dwk, dw_psa->dwv, dw_psa->dwo};
+        const float *b[4] = {dw_cross->dwq, dw_cross->dwk, dw_cross->dwv, dw_cross->dwo};
+        for (int i = 0; i < 4; ++i)
+            for (int j = 0; j < 4; ++j)
+                if (overlap(a[i], gb, b[j], gb))
+                    return fail(PTDIT_ERR_ALIAS, "dw_psa and dw_cross overlap");
+    }
+    const WsGB Lb = ws_layout_giim_bwd(d, pg.M);
+    TRY(check_bwd_ws(ws, ws_bytes, Lb.total));
+    const Ws none{};
+    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), none};
+    return run_giim_bwd(r, Lb, pg, psa, cross, flags, z_in, dz_out, dz_in, dw_psa, dw_cross);
 }
 
 size_t ptdit_tcm_bwd_workspace_bytes(const ptdit_shape *shape, const int window[3]) {

@@ -214,6 +214,26 @@ int ptdit_window_attn_bwd(const ptdit_shape *shape, const int window[3], const i
                           size_t ws_bytes, ptdit_stream_t stream);
 
 /*
+ * ptdit_giim_bwd -- backward (training) of ptdit_giim with window-mean proxies:
+ *   given z_in and dz_out = dL/dz_out, writes dz_in = dL/dz_in and both modules'
+ *   weight gradients (fp32 [D][D], overwritten).  The forward is recomputed
+ *   (keeping each query row's log-sum-exp); per head the attention backward is
+ *   the softmax chain rule with delta = rowsum(dO * O); dK and dV of each
+ *   128-key tile are summed over all queries, dQ over the key tiles through a
+ *   projection over the stacked weights; the averaging's adjoint hands every
+ *   token dP_a[window] / P.  flags: PTDIT_PROXY_RESIDUAL, PTDIT_NO_RESIDUAL.
+ *   Workspace: ptdit_giim_bwd_workspace_bytes(shape, ratio).  Supported: bf16,
+ *   D a multiple of 128, head widths 8..80 in steps of 8, at most 8192
+ *   proxies; else PTDIT_ERR_SHAPE / PTDIT_ERR_DTYPE, nothing launched.
+ */
+size_t ptdit_giim_bwd_workspace_bytes(const ptdit_shape *shape, const int ratio[3]);
+int ptdit_giim_bwd(const ptdit_shape *shape, const int ratio[3], const ptdit_attn_w *psa,
+                   const ptdit_attn_w *cross, unsigned flags, const void *z_in,
+                   const void *dz_out, void *dz_in, const ptdit_attn_wgrad *dw_psa,
+                   const ptdit_attn_wgrad *dw_cross, void *ws, size_t ws_bytes,
+                   ptdit_stream_t stream);
+
+/*
  * ptdit_tcm_bwd -- backward of ptdit_tcm: z^ = WSA(z_in) (+ z_in) is recomputed,
  *   then the SWSA branch's backward at z^ and the WSA branch's backward at
  *   z_in (each as ptdit_window_attn_bwd).  dw_wsa and dw_swsa receive the two
@@ -387,7 +407,8 @@ enum {
     PTDIT_K_ATTN_WINDOW_BWD = 8, /* window attention core, backward */
     PTDIT_K_WGRAD = 9,     /* weight gradients of the projections */
     PTDIT_K_TRANSPOSE = 10,/* weight transposes of the backward */
-    PTDIT_K_COUNT = 11
+    PTDIT_K_ATTN_ROWS_BWD = 11, /* cross / proxy attention core, backward */
+    PTDIT_K_COUNT = 12
 };
 int ptdit_timing_enable(int max_launches);
 int ptdit_timing_read(int *kind, float *ms, int max);

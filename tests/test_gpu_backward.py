@@ -118,3 +118,73 @@ def test_tcm_bwd(grid, D, heads, window, shift, B):
     for i in range(4):
         assert rel_err(c.out64(dwa[i]), want_a[i]) <= TOL["bf16"], ("wsa", i)
         assert rel_err(c.out64(dwb[i]), want_b[i]) <= TOL["bf16"], ("swsa", i)
+
+
+
+# ---------------------------------------------------------------- GIIM
+
+def _proxy_kappa(z64, grid, ratio, Wp, heads, proxy_residual):
+    """max |column mean| / max |deviation| of the PSA output P' (the cross keys' source).
+
+    P' stores in bf16 within 2^-8 of each element, i.e. within 2^-8 |mean| absolute,
+    while dWq and dWk of the cross-attention depend only on the proxies' deviations
+    from their mean (the softmax ignores a shift common to all keys): their error
+    relative to their size is of order 2^-8 kappa."""
+    Pa = O.averaging(z64, grid, ratio)
+    Pp = O.attention_heads(Pa @ Wp[0].T, Pa @ Wp[1].T, Pa @ Wp[2].T, heads) @ Wp[3].T
+    if proxy_residual:
+        Pp = Pp + Pa
+    m = Pp.mean(axis=0)
+    return float(np.abs(m).max() / np.abs(Pp - m).max())
+
+
+def _check_giim(c, ratio, flags=0):
+    dout_cpu = _dout(c.B, c.N, c.D)
+    dz, dwp, dwc = pt.ptdit_giim_bwd(c.z, dout_cpu.cuda(), c.grid, ratio, c.w["psa"], c.w["cross"],
+                                     c.heads, flags)
+    dz = c.out64(dz)
+    g64 = synth.as_f64(dout_cpu)
+    want_p = [np.zeros((c.D, c.D)) for _ in range(4)]
+    want_c = [np.zeros((c.D, c.D)) for _ in range(4)]
+    kappa = 0.0
+    for b in range(c.B):
+        kappa = max(kappa, _proxy_kappa(c.z64[b], c.grid, ratio, c.w64["psa"], c.heads,
+                                        bool(flags & pt.PTDIT_PROXY_RESIDUAL)))
+        wdz, wp, wc = O.giim_bwd(c.z64[b], c.grid, ratio, c.w64["psa"], c.w64["cross"], c.heads,
+                                 g64[b], proxy_residual=bool(flags & pt.PTDIT_PROXY_RESIDUAL),
+                                 residual=not flags & pt.PTDIT_NO_RESIDUAL)
+        assert rel_err(dz[b], wdz) <= TOL["bf16"], ("dz", b)
+        for i in range(4):
+            want_p[i] += wp[i]
+            want_c[i] += wc[i]
+    # the cross dWq, dWk: the bf16 tolerance plus twice the storage bound 2^-8 kappa
+    tol_qk = TOL["bf16"] + 2 * 2.0 ** -8 * kappa
+    for i, name in enumerate(("dWq", "dWk", "dWv", "dWo")):
+        assert rel_err(c.out64(dwp[i]), want_p[i]) <= TOL["bf16"], ("psa", name)
+        tol = tol_qk if i < 2 else TOL["bf16"]
+        assert rel_err(c.out64(dwc[i]), want_c[i]) <= tol, ("cross", name, kappa)
+
+
+GIIM_CASES = [  # grid, D, heads, ratio
+    ((1, 16, 16), 128, 2, (1, 4, 4)),     # 16 proxies: one ragged key tile, d = 64
+    ((2, 16, 16), 256, 4, (1, 2, 2)),     # 128 proxies: one full key tile
+    ((2, 16, 32), 1152, 16, (1, 2, 2)),   # 256 proxies: two key tiles, d = 72
+    ((1, 24, 40), 640, 8, (1, 2, 2)),     # 240 proxies, 960 latents: ragged tiles, d = 80
+    ((1, 16, 16), 128, 4, (1, 1, 1)),     # every token a proxy (256 x 256), d = 32
+]
+
+
+@pytest.mark.parametrize("grid,D,heads,ratio", GIIM_CASES)
+def test_giim_bwd_small(grid, D, heads, ratio):
+    _check_giim(Case(1, grid, D, heads, "bf16"), ratio)
+
+
+@pytest.mark.parametrize("flags", ["proxy_residual", "no_residual"])
+def test_giim_bwd_flags(flags):
+    f = pt.PTDIT_PROXY_RESIDUAL if flags == "proxy_residual" else pt.PTDIT_NO_RESIDUAL
+    _check_giim(Case(1, (2, 16, 32), 1152, 16, "bf16"), (1, 2, 2), f)
+
+
+def test_giim_bwd_full_size_1024px():
+    """t2i 1024 px: B = 4 items of 64 x 64 latents, 256 proxies each, D = 1152."""
+    _check_giim(Case(4, (1, 64, 64), 1152, 16, "bf16"), (1, 4, 4))

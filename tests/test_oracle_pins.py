@@ -798,3 +798,26 @@ def test_pins_catch_an_averaging_adjoint_without_the_divisor(monkeypatch):
 
     monkeypatch.setattr(O.ptdit_oracle, "averaging_bwd", no_divisor)
     assert _pin_fails(lambda: test_giim_bwd_matches_finite_differences(False))
+
+
+def test_attention_bwd_ignores_a_common_key_shift():
+    """Adding one vector m to every key adds c Q_h m_h to each score row, which the
+    row softmax removes: P, A and so dQ, dK, dV are unchanged, and the key
+    gradients of every head sum to zero over the keys (each row of dS does).  The
+    row-attention backward relies on both: it takes dQ against the keys less their
+    mean and centres dK over the keys."""
+    rng = np.random.default_rng(11)
+    nq, nk, D, heads = 9, 7, 8, 2
+    Q, K, V, dA = (rng.standard_normal((n, D)) for n in (nq, nk, nk, nq))
+    m = 3.0 + rng.standard_normal(D)
+    dQ, dK, dV = O.attention_heads_bwd(Q, K, V, dA, heads)
+    dQs, dKs, dVs = O.attention_heads_bwd(Q, K + m, V, dA, heads)
+    for got, want in ((dQs, dQ), (dKs, dK), (dVs, dV)):
+        assert np.allclose(got, want, rtol=0, atol=1e-12)
+    assert np.abs(dK.sum(axis=0)).max() <= 1e-12 * np.abs(dK).max()
+    # not a property of any key gradient: a dK without the rowsum term fails it
+    d = D // heads
+    S = (Q[:, :d] @ K[:, :d].T) / np.sqrt(d)
+    P = O.softmax_rows(S)
+    wrong = (P * (dA[:, :d] @ V[:, :d].T)).T @ Q[:, :d]
+    assert np.abs(wrong.sum(axis=0)).max() > 1e-3
