@@ -485,6 +485,21 @@ def block_attn(z, grid, ratio, window, shift, W_psa, W_cross, W_wsa, W_swsa, hea
     return tcm(z1, grid, window, shift, W_wsa, W_swsa, heads, residual=residual)
 
 
+def block_attn_bwd(z, grid, ratio, window, shift, W_psa, W_cross, W_wsa, W_swsa, heads, dout,
+                   *, proxy_residual=False, residual=True):
+    """Backward of block_attn on one batch item: z1 = giim(z) is recomputed, TCM's
+    backward at z1 gives dL/dz1 and both window modules' weight gradients, GIIM's
+    backward at z with dL/dz1 gives dL/dz and the proxy and cross modules'.
+    Returns (dz, dW_psa, dW_cross, dW_wsa, dW_swsa)."""
+    z1 = giim(z, grid, ratio, W_psa, W_cross, heads, proxy_residual=proxy_residual,
+              residual=residual)
+    dz1, dW_wsa, dW_swsa = tcm_bwd(z1, grid, window, shift, W_wsa, W_swsa, heads, dout,
+                                   residual=residual)
+    dz, dW_psa, dW_cross = giim_bwd(z, grid, ratio, W_psa, W_cross, heads, dz1,
+                                    proxy_residual=proxy_residual, residual=residual)
+    return dz, dW_psa, dW_cross, dW_wsa, dW_swsa
+
+
 def block_attn_rows(z, grid, ratio, window, shift, W_psa, W_cross, W_wsa, W_swsa, heads, rows,
                     *, proxy_residual=False, residual=True) -> np.ndarray:
     """block_attn at the listed token rows only, from the full input z.

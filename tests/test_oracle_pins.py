@@ -821,3 +821,30 @@ def test_attention_bwd_ignores_a_common_key_shift():
     P = O.softmax_rows(S)
     wrong = (P * (dA[:, :d] @ V[:, :d].T)).T @ Q[:, :d]
     assert np.abs(wrong.sum(axis=0)).max() > 1e-3
+
+
+def test_block_attn_bwd_matches_finite_differences():
+    """The whole path, GIIM then TCM: directional derivatives of <dout, block_attn(z)>
+    in z and in one weight of each of the four modules."""
+    grid, ratio, window, shift = (2, 4, 4), (1, 2, 2), (2, 2, 2), (1, 1, 1)
+    D, heads = 8, 2
+    rng = np.random.default_rng(13)
+    N = O.num_tokens(grid)
+    z, dout = rng.standard_normal((N, D)), rng.standard_normal((N, D))
+    W = [_weights(D, 50 + i, scale=0.5) for i in range(4)]
+    dz, *dW = O.block_attn_bwd(z, grid, ratio, window, shift, *W, heads, dout)
+
+    def L(zz, Ws):
+        return float(np.sum(dout * O.block_attn(zz, grid, ratio, window, shift, *Ws, heads)))
+
+    eps = 1e-5
+    U = rng.standard_normal(z.shape)
+    fd = (L(z + eps * U, W) - L(z - eps * U, W)) / (2 * eps)
+    assert abs(fd - np.sum(dz * U)) <= 1e-7 * max(1.0, abs(fd))
+    for m, i in ((0, 1), (1, 0), (2, 2), (3, 3)):
+        V = rng.standard_normal((D, D))
+        P, M = [list(w) for w in W], [list(w) for w in W]
+        P[m][i] = P[m][i] + eps * V
+        M[m][i] = M[m][i] - eps * V
+        fd = (L(z, [tuple(w) for w in P]) - L(z, [tuple(w) for w in M])) / (2 * eps)
+        assert abs(fd - np.sum(dW[m][i] * V)) <= 1e-7 * max(1.0, abs(fd)), (m, i)
