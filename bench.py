@@ -27,6 +27,7 @@ projection and residual) per step on the same grid.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -628,9 +629,11 @@ def run_block(args, w, L=120):
     return 0
 
 
-def run_bwd(args, w):
-    """Backward of the shifted-window TCM branch (ptdit_window_attn_bwd): dL/dz and the four
-    weight gradients for a synthetic upstream gradient, per step."""
+def run_bwd(args, w, branch=False):
+    """Backward of the block-attention path (ptdit_block_attn_bwd: GIIM recomputed, TCM's
+    backward, GIIM's backward), or with branch=True of the shifted-window TCM branch
+    alone (ptdit_window_attn_bwd): dL/dz and the weight gradients for a synthetic
+    upstream gradient, per step."""
     import torch
 
     import diffusion_transformer_sparse_b200 as pt
@@ -640,24 +643,42 @@ def run_bwd(args, w):
     z_host, W_host = host_inputs(w)
     z = z_host.to(dev)
     dout = torch.stack([synth.latent(w.N, w.D, 500 + b, w.dtype) for b in range(w.B)]).to(dev)
-    W = tuple(x.to(dev) for x in W_host["swsa"])
+    W = {m: tuple(x.to(dev) for x in W_host[m]) for m in ("psa", "cross", "wsa", "swsa")}
     shape = pt.make_shape(z, w.grid, w.heads)
-    ws = pt.window_attn_bwd_workspace(shape, w.window)
     dz = torch.empty_like(z)
-    dw = tuple(torch.empty(w.D, w.D, dtype=torch.float32, device=dev) for _ in range(4))
+    nmod = 1 if branch else 4
+    dw = [tuple(torch.empty(w.D, w.D, dtype=torch.float32, device=dev) for _ in range(4))
+          for _ in range(nmod)]
+    if branch:
+        ws = pt.window_attn_bwd_workspace(shape, w.window)
+    else:
+        n = pt.lib().ptdit_block_attn_bwd_workspace_bytes(ctypes.byref(shape), pt._i3(w.ratio),
+                                                         pt._i3(w.window))
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
     do_flush = l2_policy(w)[0]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    wg = [pt.AttnWgrad(*[x.data_ptr() for x in g]) for g in dw]
+    wa = [pt.attn_w(W[m]) for m in ("psa", "cross", "wsa", "swsa")]
 
     def step():
-        pt.ptdit_window_attn_bwd(z, dout, w.grid, w.window, w.shift, W, w.heads, dz_in=dz, dw=dw,
-                                 ws=ws, stream=stream)
+        if branch:
+            pt.ptdit_window_attn_bwd(z, dout, w.grid, w.window, w.shift, W["swsa"], w.heads,
+                                     dz_in=dz, dw=dw[0], ws=ws, stream=stream)
+            return
+        rc = pt.lib().ptdit_block_attn_bwd(
+            ctypes.byref(shape), pt._i3(w.ratio), pt._i3(w.window), pt._i3(w.shift),
+            *[ctypes.byref(x) for x in wa], 0, z.data_ptr(), dout.data_ptr(), dz.data_ptr(),
+            *[ctypes.byref(x) for x in wg], ws.data_ptr(), ws.numel(), stream.cuda_stream)
+        if rc != 0:
+            raise pt.PtditError(rc, pt.lib().ptdit_last_error().decode())
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    n0 = pt.ptdit_launch_count()
     for e0, e1 in evs:
         if do_flush:
             flush.zero_()
@@ -665,29 +686,34 @@ def run_bwd(args, w):
         step()
         e1.record(stream)
     torch.cuda.synchronize(dev)
+    launches = (pt.ptdit_launch_count() - n0) // args.steps
     ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
-    pt.ptdit_timing_enable(64 * args.steps)
+    pt.ptdit_timing_enable(128 * args.steps)
     for _ in range(args.steps):
         if do_flush:
             flush.zero_()
         step()
-    recs = pt.ptdit_timing_read(64 * args.steps)
+    recs = pt.ptdit_timing_read(128 * args.steps)
     pt.ptdit_timing_enable(0)
     per = {}
     for k, t in recs:
         per[k] = per.get(k, 0.0) + t / args.steps
-    f = flops.window_bwd_flops(w.N, w.n, w.D)
-    rate = {
-        "gemm (recompute Q/K/V, dA, dx)": w.B * f["gemm"] / (per.get("gemm", 0) / 1e3) / 1e12,
-        "wgrad": w.B * f["wgrad"] / (per.get("wgrad", 0) / 1e3) / 1e12,
-        "attn_window_bwd": w.B * f["core_bwd"] / (per.get("attn_window_bwd", 0) / 1e3) / 1e12,
-    } if all(per.get(k) for k in ("gemm", "wgrad", "attn_window_bwd")) else {}
+    if branch:
+        f = flops.window_bwd_flops(w.N, w.n, w.D)
+        metric, mode = "backward of one TCM branch, tokens/s", "window_bwd"
+        cores = {"attn_window_bwd": w.B * f["core_bwd"]}
+    else:
+        f = flops.block_bwd_flops(w.N, w.M, w.n, w.D)
+        metric, mode = "backward of the block-attention path (GIIM + TCM), tokens/s", "block_bwd"
+        cores = {"attn_window_bwd": w.B * f["window_core_bwd"],
+                 "attn_rows_bwd": w.B * f["rows_core_bwd"]}
+    rate = {k: v / (per[k] / 1e3) / 1e12 for k, v in cores.items() if per.get(k)}
     print(json.dumps({
-        "mode": "window_bwd", "metric": "backward of one TCM branch, tokens/s", "unit": UNIT,
+        "mode": mode, "metric": metric, "unit": UNIT,
         "value": w.B * w.N / (ms / 1e3), "ms_per_step": ms, "steps": args.steps,
         "warmup": args.warmup, "config": dict(config_of(w), l2=l2_policy(w)[1]),
         "tflops": w.B * f["total"] / (ms / 1e3) / 1e12, "flops_per_step": w.B * f["total"],
-        "kernels_ms_per_step": per, "kernels_tflops": rate,
+        "gpu_launches": launches, "kernels_ms_per_step": per, "kernels_tflops": rate,
         "note": "per-kernel times from a second pass with hooks"}), flush=True)
     return 0
 
@@ -715,7 +741,9 @@ def main(argv=None):
     ap.add_argument("--dense", action="store_true",
                     help="time the dense comparator (full global self-attention) instead")
     ap.add_argument("--bwd", action="store_true",
-                    help="time the backward of the shifted-window TCM branch instead")
+                    help="time the backward of the block-attention path instead")
+    ap.add_argument("--bwd-branch", action="store_true",
+                    help="time the backward of the shifted-window TCM branch alone instead")
     ap.add_argument("--block", action="store_true",
                     help="time the complete PT-Block (norms, text cross-attention, MLP) instead")
     args = ap.parse_args(argv)
@@ -729,8 +757,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.dense:
         return run_dense(args, w)
-    if args.bwd:
-        return run_bwd(args, w)
+    if args.bwd or args.bwd_branch:
+        return run_bwd(args, w, branch=args.bwd_branch)
     if args.block:
         return run_block(args, w)
     return run_gpu(args, w)

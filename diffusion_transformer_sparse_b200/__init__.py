@@ -34,7 +34,8 @@ EXPORTS = (
     "ptdit_proxy_extract", "ptdit_giim_ex", "ptdit_pt_block", "ptdit_pt_block_workspace_bytes",
     "ptdit_debug_wait_limit", "ptdit_window_attn_bwd", "ptdit_window_attn_bwd_workspace_bytes",
     "ptdit_tcm_bwd", "ptdit_tcm_bwd_workspace_bytes", "ptdit_giim_bwd",
-    "ptdit_giim_bwd_workspace_bytes",
+    "ptdit_giim_bwd_workspace_bytes", "ptdit_block_attn_bwd",
+    "ptdit_block_attn_bwd_workspace_bytes",
 )
 
 
@@ -108,6 +109,11 @@ def lib() -> ctypes.CDLL:
             "ptdit_window_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
             "ptdit_tcm_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
             "ptdit_giim_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
+            "ptdit_block_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3, _I3]),
+            "ptdit_block_attn_bwd": (ctypes.c_int, [_S, _I3, _I3, _I3, _W, _W, _W, _W,
+                                                    ctypes.c_uint, _P, _P, _P]
+                                     + [ctypes.POINTER(AttnWgrad)] * 4
+                                     + [_P, ctypes.c_size_t, _P]),
             "ptdit_giim_bwd": (ctypes.c_int, [_S, _I3, _W, _W, ctypes.c_uint, _P, _P, _P,
                                               ctypes.POINTER(AttnWgrad), ctypes.POINTER(AttnWgrad),
                                               _P, ctypes.c_size_t, _P]),
@@ -430,6 +436,34 @@ def ptdit_tcm_bwd(z_in, dz_out, grid, window, shift, wsa, swsa, heads, flags=0, 
                                ctypes.byref(ga), ctypes.byref(gb), _ptr(ws), ws.numel(),
                                _stream(stream)))
     return dz_in, dwa, dwb
+
+
+def ptdit_block_attn_bwd(z_in, dz_out, grid, ratio, window, shift, psa, cross, wsa, swsa, heads,
+                         flags=0, dz_in=None, ws=None, stream=None):
+    """Backward of ptdit_block_attn: returns (dz_in, dW_psa, dW_cross, dW_wsa, dW_swsa),
+    each dW four fp32 [D, D]."""
+    import torch
+    _check_z(z_in)
+    _check_z(dz_out)
+    shape = make_shape(z_in, grid, heads)
+    if dz_in is None:
+        dz_in = torch.empty_like(z_in)
+    D = z_in.shape[-1]
+    dws = [tuple(torch.empty(D, D, dtype=torch.float32, device=z_in.device) for _ in range(4))
+           for _ in range(4)]
+    if ws is None:
+        n = lib().ptdit_block_attn_bwd_workspace_bytes(ctypes.byref(shape), _i3(ratio),
+                                                      _i3(window))
+        if n == 0:
+            raise PtditError(PTDIT_ERR_SHAPE, "invalid shape, ratio or window")
+        ws = torch.empty(n, dtype=torch.uint8, device=z_in.device)
+    w = [attn_w(x) for x in (psa, cross, wsa, swsa)]
+    g = [AttnWgrad(*[_ptr(x) for x in dw]) for dw in dws]
+    _check(lib().ptdit_block_attn_bwd(ctypes.byref(shape), _i3(ratio), _i3(window), _i3(shift),
+                                      *[ctypes.byref(x) for x in w], flags, _ptr(z_in),
+                                      _ptr(dz_out), _ptr(dz_in), *[ctypes.byref(x) for x in g],
+                                      _ptr(ws), ws.numel(), _stream(stream)))
+    return (dz_in, *dws)
 
 
 def ptdit_tcm(z_in, grid, window, shift, wsa, swsa, heads, flags=0, z_out=None, ws=None,

@@ -292,6 +292,10 @@ cudaError_t launch_attention_win_bwd(const AttnArgs &a, const void *dout, void *
 cudaError_t launch_attention_rows_bwd(const AttnArgs &a, const void *dout, const float *lse,
                                       const float *delta, const float *kmean, void *dq, long ldq,
                                       float *dk, float *dv, cudaStream_t s);
+// dst[r][c] = sum over j < nblk of src[r][j D + c], bf16 in and out (fp32 sums); src
+// has row stride lds, dst ldd.
+cudaError_t launch_sum_blocks_bf16(const void *src, long rows, int nblk, int D, long lds,
+                                  void *dst, long ldd, cudaStream_t s);
 // mean[b][h d + c] = the mean over the nk key rows of item b of column c of head h,
 // K in tiled head layout (identity tiles, no padding).
 cudaError_t launch_key_mean(const void *K_tiles, int B, int nk, int heads, int d, float *mean,

@@ -8,6 +8,8 @@
 //   to_bf16          the fp32 key and value gradients to bf16 operands
 //   key_mean         per (batch item, head) the mean of the valid key rows (fp32),
 //                    read from the tiled head layout
+//   sum_blocks       dQ summed over the key tiles: dst = sum over j of the column
+//                    blocks [j D, (j + 1) D) of src (bf16, fp32 sums)
 //   center_to_bf16   the fp32 key gradient less its mean over each batch item's keys,
 //                    as bf16 (the projection of the softmax backward onto its
 //                    exact constraint: every row of dS sums to zero, so the exact
@@ -92,6 +94,33 @@ __global__ void to_bf16_kernel(const float *__restrict__ src, long rows, int col
     *reinterpret_cast<uint4 *>(dst + r * ldd + c) = *reinterpret_cast<const uint4 *>(o);
 }
 
+// One thread per 8 columns of one row: the nblk blocks' 16-byte pieces summed in fp32.
+__global__ void sum_blocks_kernel(const __nv_bfloat16 *__restrict__ src, long rows, int nblk,
+                                  int D, long lds, __nv_bfloat16 *__restrict__ dst, long ldd) {
+    pdl_wait();
+    pdl_trigger();
+    const int pieces = D / 8;
+    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= rows * pieces) return;
+    const long r = idx / pieces;
+    const int c = static_cast<int>(idx - r * pieces) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const __nv_bfloat16 *p = src + r * lds + c;
+    for (int j = 0; j < nblk; ++j) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(p + (long)j * D);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[t]));
+            acc[2 * t] += f.x;
+            acc[2 * t + 1] += f.y;
+        }
+    }
+    __nv_bfloat162 o[4] = {__floats2bfloat162_rn(acc[0], acc[1]), __floats2bfloat162_rn(acc[2], acc[3]),
+                           __floats2bfloat162_rn(acc[4], acc[5]), __floats2bfloat162_rn(acc[6], acc[7])};
+    *reinterpret_cast<uint4 *>(dst + r * ldd + c) = *reinterpret_cast<const uint4 *>(o);
+}
+
 // One CTA per (batch item, head): thread (row lane, 16-byte unit) sums its unit over
 // the rows of its lane; the lanes meet in shared memory.
 __global__ void key_mean_kernel(const uint8_t *__restrict__ K, int nk, int heads, int d,
@@ -154,6 +183,16 @@ __global__ void center_to_bf16_kernel(const float *__restrict__ src, int M, int 
 }
 
 }  // namespace
+
+cudaError_t launch_sum_blocks_bf16(const void *src, long rows, int nblk, int D, long lds,
+                                  void *dst, long ldd, cudaStream_t s) {
+    if (rows < 1 || nblk < 1 || D % 8 || lds % 8 || ldd % 8) return cudaErrorInvalidValue;
+    const long n = rows * (D / 8);
+    const int threads = 256;
+    return launch_pdl(sum_blocks_kernel, dim3((unsigned)((n + threads - 1) / threads)),
+                      dim3(threads), 0, s, static_cast<const __nv_bfloat16 *>(src), rows, nblk, D,
+                      lds, static_cast<__nv_bfloat16 *>(dst), ldd);
+}
 
 cudaError_t launch_key_mean(const void *K_tiles, int B, int nk, int heads, int d, float *mean,
                             cudaStream_t s) {

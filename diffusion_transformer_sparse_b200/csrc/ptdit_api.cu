@@ -857,6 +857,25 @@ TcmBwd tcm_bwd_layout(const Dims &d) {
     return T;
 }
 
+// TCM's backward in the workspace at ws (tcm_bwd_layout): z^ = WSA(z_in) (+ z_in) with
+// the forward's buffers laid over the backward's, then SWSA's backward at z^ and
+// WSA's at z_in.
+int run_tcm_bwd(const Dims &d, cudaStream_t s, char *ws, const WinGeom &wg0, const WinGeom &wg1,
+                const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
+                const void *z_in, const void *dz_out, void *dz_in, const ptdit_attn_wgrad *dw_wsa,
+                const ptdit_attn_wgrad *dw_swsa) {
+    const TcmBwd T = tcm_bwd_layout(d);
+    Ws Lf{};
+    Lf.Q = T.bwd.Q; Lf.K = T.bwd.K; Lf.V = T.bwd.V; Lf.O = T.bwd.A;
+    Run rf{d, s, ws, Lf};
+    void *zh = rf.at(T.zh), *dzh = rf.at(T.dzh);
+    TRY(run_window(rf, wg0, wsa, flags, z_in, zh));
+    const Ws none{};
+    Run r{d, s, ws, none};
+    TRY(run_window_bwd(r, T.bwd, wg1, swsa, flags, zh, dz_out, dzh, dw_swsa));
+    return run_window_bwd(r, T.bwd, wg0, wsa, flags, z_in, dzh, dz_in, dw_wsa);
+}
+
 int check_bwd_io(const Dims &d, const ptdit_attn_w *w, const void *z_in, const void *dz_out,
                  void *dz_in, const void *ws, size_t ws_bytes) {
     TRY(check_io(d, z_in, dz_in, ws, ws_bytes));
@@ -901,10 +920,12 @@ int check_bwd_ws(const void *ws, size_t ws_bytes, size_t need) {
 }
 
 // ------------------------------------------------------------------ backward of GIIM
+// Gc / Gq: dQ of each key tile as column blocks (only with more than one key tile),
+// summed into dQc / the first block of Gp = [dQ | dK | dV] of the proxies.
 struct WsGB {
-    size_t Pa, Pq, Pk, Pvf, Pvb, Ap, Pp, Ck, Cvf, Cvb, dAp, dPp, dKVc, Gp, dPa;
+    size_t Pa, Pq, Pk, Pvf, Pvb, Ap, Pp, Ck, Cvf, Cvb, dAp, dPp, dKVc, Gq, Gp, dPa;
     size_t dKc, dVc, dKp, dVp, lse_p, del_p, km_p;
-    size_t Cq, Ac, dAc, Gc, lse_c, del_c, km_c;
+    size_t Cq, Ac, dAc, Gc, dQc, lse_c, del_c, km_c;
     size_t WcoT, WcqT, WckvT, WpoT, WpT;
     int ktc, ktp;
     size_t total;
@@ -925,15 +946,17 @@ WsGB ws_layout_giim_bwd(const Dims &d, long M) {
     L.Ap = take(BM * D * e); L.Pp = take(BM * D * e);
     L.Ck = take(tp); L.Cvf = take(tpv); L.Cvb = take(tp);
     L.dAp = take(tp); L.dPp = take(BM * D * e); L.dKVc = take(BM * 2 * D * e);
-    L.Gp = take(BM * (L.ktp + 2) * D * e); L.dPa = take(BM * D * e);
+    L.Gq = take(L.ktp > 1 ? BM * L.ktp * D * e : 0); L.Gp = take(BM * 3 * D * e);
+    L.dPa = take(BM * D * e);
     L.dKc = take(BM * D * 4); L.dVc = take(BM * D * 4); L.dKp = take(BM * D * 4);
     L.dVp = take(BM * D * 4);
     L.lse_p = take(BM * d.heads * 4); L.del_p = take(BM * d.heads * 4);
     L.km_p = take((size_t)d.B * D * 4); L.km_c = take((size_t)d.B * D * 4);
-    L.Cq = take(tn); L.Ac = take(BN * D * e); L.dAc = take(tn); L.Gc = take(BN * L.ktc * D * e);
+    L.Cq = take(tn); L.Ac = take(BN * D * e); L.dAc = take(tn);
+    L.Gc = take(L.ktc > 1 ? BN * L.ktc * D * e : 0); L.dQc = take(BN * D * e);
     L.lse_c = take(BN * d.heads * 4); L.del_c = take(BN * d.heads * 4);
-    L.WcoT = take(D * D * e); L.WcqT = take(D * L.ktc * D * e); L.WckvT = take(D * 2 * D * e);
-    L.WpoT = take(D * D * e); L.WpT = take(D * (L.ktp + 2) * D * e);
+    L.WcoT = take(D * D * e); L.WcqT = take(D * D * e); L.WckvT = take(D * 2 * D * e);
+    L.WpoT = take(D * D * e); L.WpT = take(D * 3 * D * e);
     L.total = off;
     return L;
 }
@@ -1056,16 +1079,14 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
     TRY(attention(r, PTDIT_K_ATTN_CROSS, ca, "backward: cross-attention"));
     // ---- transposed weights for the input gradients
     TRY(transpose(r, cross->wo, D, D, P(Lb.WcoT), D));
-    for (int j = 0; j < ktc; ++j)
-        TRY(transpose(r, cross->wq, D, D, P(Lb.WcqT) + (size_t)j * D * d.elem, (long)ktc * D));
+    TRY(transpose(r, cross->wq, D, D, P(Lb.WcqT), D));
     TRY(transpose(r, cross->wk, D, D, P(Lb.WckvT), 2L * D));
     TRY(transpose(r, cross->wv, D, D, P(Lb.WckvT) + (size_t)D * d.elem, 2L * D));
     TRY(transpose(r, psa->wo, D, D, P(Lb.WpoT), D));
-    const long ldp = (long)(ktp + 2) * D;
-    for (int j = 0; j < ktp; ++j)
-        TRY(transpose(r, psa->wq, D, D, P(Lb.WpT) + (size_t)j * D * d.elem, ldp));
-    TRY(transpose(r, psa->wk, D, D, P(Lb.WpT) + (size_t)ktp * D * d.elem, ldp));
-    TRY(transpose(r, psa->wv, D, D, P(Lb.WpT) + (size_t)(ktp + 1) * D * d.elem, ldp));
+    const long ldp = 3L * D;
+    TRY(transpose(r, psa->wq, D, D, P(Lb.WpT), ldp));
+    TRY(transpose(r, psa->wk, D, D, P(Lb.WpT) + (size_t)D * d.elem, ldp));
+    TRY(transpose(r, psa->wv, D, D, P(Lb.WpT) + (size_t)2 * D * d.elem, ldp));
     // ---- cross-attention backward
     {
         const void *W[3] = {P(Lb.WcoT), nullptr, nullptr};
@@ -1078,8 +1099,13 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
     AttnArgs cb = ca;
     cb.v = P(Lb.Cvb);
     cb.tv = tp;
-    TRY(rows_bwd(r, cb, P(Lb.dAc), F(Lb.lse_c), F(Lb.del_c), F(Lb.km_c), P(Lb.Gc), (long)ktc * D,
-                 F(Lb.dKc), F(Lb.dVc), "cross-attention backward"));
+    // dQ straight into dQc with one key tile, else per key tile, then summed
+    TRY(rows_bwd(r, cb, P(Lb.dAc), F(Lb.lse_c), F(Lb.del_c), F(Lb.km_c),
+                 ktc > 1 ? P(Lb.Gc) : P(Lb.dQc), ktc > 1 ? (long)ktc * D : (long)D, F(Lb.dKc),
+                 F(Lb.dVc), "cross-attention backward"));
+    if (ktc > 1)
+        TRY(elementwise(r, launch_sum_blocks_bf16(P(Lb.Gc), BN, ktc, D, (long)ktc * D, P(Lb.dQc), D,
+                                                  r.s), "backward: dQ over the key tiles"));
     TRY(elementwise(r, launch_center_to_bf16(F(Lb.dKc), d.B, M, D, P(Lb.dKVc), 2L * D, r.s),
                     "backward: dK"));
     TRY(elementwise(r, launch_to_bf16(F(Lb.dVc), BM, D, P(Lb.dKVc) + (size_t)D * d.elem, 2L * D, r.s),
@@ -1098,20 +1124,24 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
     AttnArgs pb = pa;
     pb.v = P(Lb.Pvb);
     pb.tv = tp;
-    TRY(rows_bwd(r, pb, P(Lb.dAp), F(Lb.lse_p), F(Lb.del_p), F(Lb.km_p), P(Lb.Gp), ldp, F(Lb.dKp),
+    TRY(rows_bwd(r, pb, P(Lb.dAp), F(Lb.lse_p), F(Lb.del_p), F(Lb.km_p),
+                 ktp > 1 ? P(Lb.Gq) : P(Lb.Gp), ktp > 1 ? (long)ktp * D : ldp, F(Lb.dKp),
                  F(Lb.dVp), "proxy self-attention backward"));
-    TRY(elementwise(r, launch_center_to_bf16(F(Lb.dKp), d.B, M, D, P(Lb.Gp) + (size_t)ktp * D * d.elem,
+    if (ktp > 1)
+        TRY(elementwise(r, launch_sum_blocks_bf16(P(Lb.Gq), BM, ktp, D, (long)ktp * D, P(Lb.Gp), ldp,
+                                                  r.s), "backward: proxy dQ over the key tiles"));
+    TRY(elementwise(r, launch_center_to_bf16(F(Lb.dKp), d.B, M, D, P(Lb.Gp) + (size_t)D * d.elem,
                                              ldp, r.s), "backward: proxy dK"));
-    TRY(elementwise(r, launch_to_bf16(F(Lb.dVp), BM, D, P(Lb.Gp) + (size_t)(ktp + 1) * D * d.elem,
-                                      ldp, r.s), "backward: proxy dV"));
+    TRY(elementwise(r, launch_to_bf16(F(Lb.dVp), BM, D, P(Lb.Gp) + (size_t)2 * D * d.elem, ldp, r.s),
+                    "backward: proxy dV"));
     TRY(gemm_ex(r, PTDIT_K_GEMM, P(Lb.Gp), BM, (int)ldp, D, P(Lb.WpT), P(Lb.dPa),
                 (flags & PTDIT_PROXY_RESIDUAL) ? P(Lb.dPp) : nullptr, nullptr, ACT_NONE,
                 "backward: dP_a"));
-    // ---- dz_in = (dz_out +) averaging^T(dP_a) + sum over key tiles of dQ_j Wq
+    // ---- dz_in = (dz_out +) averaging^T(dP_a) + dQ Wq
     TRY(elementwise(r, launch_proxy_broadcast(pg, d.B, D, P(Lb.dPa),
                                               (flags & PTDIT_NO_RESIDUAL) ? nullptr : dz_out, dz_in, r.s),
                     "backward: averaging adjoint"));
-    TRY(gemm_ex(r, PTDIT_K_GEMM, P(Lb.Gc), BN, ktc * D, D, P(Lb.WcqT), dz_in, dz_in, nullptr,
+    TRY(gemm_ex(r, PTDIT_K_GEMM, P(Lb.dQc), BN, D, D, P(Lb.WcqT), dz_in, dz_in, nullptr,
                 ACT_NONE, "backward: input gradient"));
     // ---- weight gradients
     float *outs[8] = {dwp->dwq, dwp->dwk, dwp->dwv, dwp->dwo, dwc->dwq, dwc->dwk, dwc->dwv, dwc->dwo};
@@ -1123,21 +1153,14 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
         const int c0[1] = {0};
         float *o1[1] = {dwc->dwo};
         TRY(wgrad_blocks(r, dz_out, D, c0, o1, 1, P(Lb.Ac), BN, "backward: dWo (cross)"));
-        int cq[64];
-        float *oq[64];
-        for (int j = 0; j < ktc && j < 64; ++j) { cq[j] = j * D; oq[j] = dwc->dwq; }
-        TRY(wgrad_blocks(r, P(Lb.Gc), ktc * D, cq, oq, ktc, z_in, BN, "backward: dWq (cross)"));
+        TRY(wgrad_blocks(r, P(Lb.dQc), D, c0, &outs[4], 1, z_in, BN, "backward: dWq (cross)"));
         const int ckv[2] = {0, D};
         float *okv[2] = {dwc->dwk, dwc->dwv};
         TRY(wgrad_blocks(r, P(Lb.dKVc), 2 * D, ckv, okv, 2, P(Lb.Pp), BM, "backward: dWk, dWv (cross)"));
         TRY(wgrad_blocks(r, P(Lb.dPp), D, c0, &outs[3], 1, P(Lb.Ap), BM, "backward: dWo (proxy)"));
-        int cp[66];
-        float *op[66];
-        int n = 0;
-        for (int j = 0; j < ktp && n < 64; ++j, ++n) { cp[n] = j * D; op[n] = dwp->dwq; }
-        cp[n] = ktp * D; op[n++] = dwp->dwk;
-        cp[n] = (ktp + 1) * D; op[n++] = dwp->dwv;
-        TRY(wgrad_blocks(r, P(Lb.Gp), (int)ldp, cp, op, n, P(Lb.Pa), BM, "backward: dWq, dWk, dWv (proxy)"));
+        const int cp[3] = {0, D, 2 * D};
+        TRY(wgrad_blocks(r, P(Lb.Gp), (int)ldp, cp, &outs[0], 3, P(Lb.Pa), BM,
+                         "backward: dWq, dWk, dWv (proxy)"));
     }
     return PTDIT_OK;
 }
@@ -1435,18 +1458,9 @@ int ptdit_tcm_bwd(const ptdit_shape *shape, const int window[3], const int shift
                 if (overlap(a[i], gb, b[j], gb))
                     return fail(PTDIT_ERR_ALIAS, "dw_wsa and dw_swsa overlap");
     }
-    const TcmBwd T = tcm_bwd_layout(d);
-    TRY(check_bwd_ws(ws, ws_bytes, T.total));
-    // z^ = WSA(z_in) (+ z_in), with the forward's workspace laid over the backward's
-    Ws Lf{};
-    Lf.Q = T.bwd.Q; Lf.K = T.bwd.K; Lf.V = T.bwd.V; Lf.O = T.bwd.A;
-    Run rf{d, (cudaStream_t)stream, static_cast<char *>(ws), Lf};
-    void *zh = rf.at(T.zh), *dzh = rf.at(T.dzh);
-    TRY(run_window(rf, wg0, wsa, flags, z_in, zh));
-    const Ws none{};
-    Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), none};
-    TRY(run_window_bwd(r, T.bwd, wg1, swsa, flags, zh, dz_out, dzh, dw_swsa));
-    return run_window_bwd(r, T.bwd, wg0, wsa, flags, z_in, dzh, dz_in, dw_wsa);
+    TRY(check_bwd_ws(ws, ws_bytes, tcm_bwd_layout(d).total));
+    return run_tcm_bwd(d, (cudaStream_t)stream, static_cast<char *>(ws), wg0, wg1, wsa, swsa, flags,
+                       z_in, dz_out, dz_in, dw_wsa, dw_swsa);
 }
 
 int ptdit_tcm(const ptdit_shape *shape, const int window[3], const int shift[3],
@@ -1500,6 +1514,94 @@ int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int win
     TRY(run_giim(r, pg, psa, cross, flags, z_in, z_out));
     TRY(run_window(r, wg0, wsa, flags, z_out, z_out));
     return run_window(r, wg1, swsa, flags, z_out, z_out);
+}
+
+// ------------------------------------------------------------------ backward of the path
+// z1 and dL/dz1, then one area that the three stages (GIIM's forward, TCM's backward,
+// GIIM's backward) take in turn.
+struct BlockBwd {
+    size_t z1, dz1, area, total;
+};
+BlockBwd block_bwd_layout(const Dims &d, long M) {
+    BlockBwd L;
+    const size_t tn = align256((size_t)d.B * d.N * d.D * d.elem);
+    L.z1 = 0;
+    L.dz1 = tn;
+    L.area = 2 * tn;
+    size_t need = ws_layout(d, M).total;
+    const size_t t = tcm_bwd_layout(d).total, g = ws_layout_giim_bwd(d, M).total;
+    need = need > t ? need : t;
+    need = need > g ? need : g;
+    L.total = L.area + need;
+    return L;
+}
+
+size_t ptdit_block_attn_bwd_workspace_bytes(const ptdit_shape *shape, const int ratio[3],
+                                            const int window[3]) {
+    Dims d;
+    ProxyGeom pg;
+    WinGeom wg;
+    const int zero[3] = {0, 0, 0};
+    if (check_shape(shape, &d) != PTDIT_OK || make_proxy(d, ratio, &pg) != PTDIT_OK ||
+        make_window(d, window, zero, &wg) != PTDIT_OK)
+        return 0;
+    return block_bwd_layout(d, pg.M).total;
+}
+
+int ptdit_block_attn_bwd(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                         const int shift[3], const ptdit_attn_w *psa, const ptdit_attn_w *cross,
+                         const ptdit_attn_w *wsa, const ptdit_attn_w *swsa, unsigned flags,
+                         const void *z_in, const void *dz_out, void *dz_in,
+                         const ptdit_attn_wgrad *dw_psa, const ptdit_attn_wgrad *dw_cross,
+                         const ptdit_attn_wgrad *dw_wsa, const ptdit_attn_wgrad *dw_swsa, void *ws,
+                         size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    WinGeom wg0, wg1;
+    const int zero[3] = {0, 0, 0};
+    TRY(check_shape(shape, &d));
+    TRY(make_proxy(d, ratio, &pg));
+    TRY(make_window(d, window, shift, &wg1));
+    TRY(make_window(d, window, zero, &wg0));
+    TRY(check_bwd_shape(d, wg0));
+    if ((pg.M + kThlRows - 1) / kThlRows > 64)
+        return fail(PTDIT_ERR_SHAPE, "the backward takes at most 8192 proxies; M=%d", pg.M);
+    const ptdit_attn_w *W[4] = {psa, cross, wsa, swsa};
+    const ptdit_attn_wgrad *G[4] = {dw_psa, dw_cross, dw_wsa, dw_swsa};
+    const char *wn[4] = {"psa", "cross", "wsa", "swsa"};
+    const char *gn[4] = {"dw_psa", "dw_cross", "dw_wsa", "dw_swsa"};
+    for (int m = 0; m < 4; ++m) {
+        TRY(check_weights(W[m], wn[m]));
+        TRY(check_bwd_io(d, W[m], z_in, dz_out, dz_in, ws, ws_bytes));
+    }
+    for (int m = 0; m < 4; ++m) TRY(check_wgrad(d, G[m], gn[m], z_in, dz_out, dz_in, ws, ws_bytes));
+    {
+        const size_t gb = (size_t)d.D * d.D * sizeof(float);
+        for (int m = 0; m < 4; ++m)
+            for (int n = 0; n < m; ++n) {
+                const float *a[4] = {G[m]->dwq, G[m]->dwk, G[m]->dwv, G[m]->dwo};
+                const float *b[4] = {G[n]->dwq, G[n]->dwk, G[n]->dwv, G[n]->dwo};
+                for (int i = 0; i < 4; ++i)
+                    for (int j = 0; j < 4; ++j)
+                        if (overlap(a[i], gb, b[j], gb))
+                            return fail(PTDIT_ERR_ALIAS, "%s and %s overlap", gn[m], gn[n]);
+            }
+    }
+    const BlockBwd L = block_bwd_layout(d, pg.M);
+    TRY(check_bwd_ws(ws, ws_bytes, L.total));
+    const cudaStream_t s = (cudaStream_t)stream;
+    char *base = static_cast<char *>(ws), *area = base + L.area;
+    void *z1 = base + L.z1, *dz1 = base + L.dz1;
+    {
+        const Ws Lf = ws_layout(d, pg.M);
+        Run rf{d, s, area, Lf};
+        TRY(run_giim(rf, pg, psa, cross, flags, z_in, z1));
+    }
+    TRY(run_tcm_bwd(d, s, area, wg0, wg1, wsa, swsa, flags, z1, dz_out, dz1, dw_wsa, dw_swsa));
+    const Ws none{};
+    Run r{d, s, area, none};
+    return run_giim_bwd(r, ws_layout_giim_bwd(d, pg.M), pg, psa, cross, flags, z_in, dz1, dz_in,
+                        dw_psa, dw_cross);
 }
 
 size_t ptdit_pt_block_workspace_bytes(const ptdit_shape *shape, const int ratio[3],

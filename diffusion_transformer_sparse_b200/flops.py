@@ -76,3 +76,41 @@ def window_bwd_flops(N: int, n: int, D: int) -> dict:
     f["gemm"] = f["recompute_proj"] + f["dA"] + f["dx"]
     f["total"] = sum(v for k, v in f.items() if k != "gemm")
     return f
+
+
+def giim_bwd_flops(N: int, M: int, D: int) -> dict:
+    """Backward of GIIM as ptdit_giim_bwd runs it, per batch item: the forward
+    recomputed without the output projection, dA = dout Wo (2 N D^2), the cross
+    core's backward (S, dP, dV, dK, dQ: 10 N M D), dP' = [dK dV][Wk; Wv] (4 M D^2),
+    dA_p = dP' Wo (2 M D^2), the proxy core's backward (10 M^2 D), dP_a =
+    [dQ dK dV][Wq; Wk; Wv] (6 M D^2), dz = dQ Wq (2 N D^2) and the weight gradients
+    (cross 4 N D^2 + 4 M D^2, proxy 8 M D^2)."""
+    fwd = block_flops(N, M, 0, D)
+    f = {
+        "recompute": fwd["psa_proj"] + fwd["psa_core"] + fwd["cross_proj"] - 2 * N * D * D
+        + fwd["cross_core"],
+        "rows_core_bwd": 10 * N * M * D + 10 * M * M * D,
+        "dx": 2 * N * D * D + 4 * M * D * D + 2 * M * D * D + 6 * M * D * D + 2 * N * D * D,
+        "wgrad": 4 * N * D * D + 4 * M * D * D + 8 * M * D * D,
+    }
+    f["total"] = sum(f.values())
+    return f
+
+
+def block_bwd_flops(N: int, M: int, n: int, D: int) -> dict:
+    """Backward of the block-attention path as ptdit_block_attn_bwd runs it, per batch
+    item: GIIM's forward for z1, TCM's backward (the WSA forward for z^ and both
+    branches' backward) and GIIM's backward."""
+    fwd = block_flops(N, M, n, D)
+    w = window_bwd_flops(N, n, D)
+    g = giim_bwd_flops(N, M, D)
+    f = {
+        "giim_forward": fwd["psa_proj"] + fwd["psa_core"] + fwd["cross_proj"] + fwd["cross_core"],
+        "tcm_recompute": fwd["wsa_proj"] + fwd["wsa_core"],
+        "tcm_bwd": 2 * w["total"],
+        "giim_bwd": g["total"],
+    }
+    f["total"] = sum(f.values())
+    f["window_core_bwd"] = 2 * w["core_bwd"]
+    f["rows_core_bwd"] = g["rows_core_bwd"]
+    return f

@@ -300,3 +300,70 @@ def test_tcm_bwd_rejects_overlapping_gradients(L):
                          1 << 40, None)
     assert rc == 8
     assert b"overlap" in L.ptdit_last_error()
+
+
+def _giim_bwd(L, shape, dwp, dwc, ratio=(1, 2, 2), z_in=FAKE * 20, dz_out=FAKE * 21,
+              dz_in=FAKE * 22, ws_bytes=1 << 40):
+    gp = None if dwp is None else ctypes.byref(dwp)
+    return L.ptdit_giim_bwd(ctypes.byref(shape), pt._i3(ratio), ctypes.byref(_w(FAKE * 2)),
+                            ctypes.byref(_w(FAKE * 3)), 0, z_in, dz_out, dz_in, gp,
+                            ctypes.byref(dwc), FAKE * 128, ws_bytes, None)
+
+
+def test_giim_and_block_bwd_workspace_bytes(L):
+    s = _bshape(B=4, H=64, W=64, D=1152, heads=16)
+    g = L.ptdit_giim_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 4, 4)))
+    t = L.ptdit_tcm_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 8, 8)))
+    f = _bytes(L, s, (1, 4, 4), (1, 8, 8))
+    tn = 4 * 4096 * 1152 * 2
+    # at least the proxies' Q/K/V blocks, the latents' Q and dA blocks and the
+    # stacked dQ blocks (two key tiles of 128 proxies: 256 proxies per item)
+    assert g >= 2 * 4 * 32 * 16 * 20480 + 4 * 4096 * 2 * 1152 * 2
+    n = L.ptdit_block_attn_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 4, 4)),
+                                               pt._i3((1, 8, 8)))
+    assert n == 2 * tn + max(f, t, g)  # z1, dL/dz1, then the largest stage
+    assert L.ptdit_giim_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 3, 4))) == 0
+    assert L.ptdit_block_attn_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 4, 4)),
+                                                  pt._i3((1, 3, 8))) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(shape=dict(dtype=pt.PTDIT_F32)), 3),          # bf16 only
+    (dict(shape=dict(D=64, heads=1)), 2),                # D a multiple of 128
+    (dict(ratio=(1, 3, 2)), 2),                          # ratio does not divide the grid
+    (dict(shape=dict(H=512, W=512), ratio=(1, 1, 2)), 2),  # 131072 proxies: above 8192
+    (dict(dwp=None), 1),
+    (dict(dwp="on_dw_cross"), 8),
+    (dict(dz_in=FAKE * 21), 8),                          # dz_in is dz_out
+    (dict(z_in=0), 1),
+    (dict(ws_bytes=4096), 4),
+])
+def test_giim_bwd_rejects(L, kw, code):
+    """Every case fails validation on the host: nothing is launched."""
+    s = _bshape(**kw.pop("shape", {}))
+    dwp, dwc = _wg(FAKE * 40), _wg(FAKE * 80)
+    special = kw.pop("dwp", dwp)
+    if special == "on_dw_cross":
+        dwp = _wg(FAKE * 80 + 0x100000)  # dwp.dwq is dwc.dwk
+    elif special is None:
+        dwp = None
+    assert _giim_bwd(L, s, dwp, dwc, **kw) == code
+    assert L.ptdit_last_error()
+
+
+def test_block_attn_bwd_rejects(L):
+    s = _bshape()
+    g = [_wg(FAKE * (40 + 8 * i)) for i in range(4)]
+
+    def call(shape=s, grads=g, window=(1, 8, 8), ws_bytes=1 << 40):
+        return L.ptdit_block_attn_bwd(
+            ctypes.byref(shape), pt._i3((1, 2, 2)), pt._i3(window), pt._i3((0, 4, 4)),
+            *[ctypes.byref(_w(FAKE * (2 + i))) for i in range(4)], 0, FAKE * 20, FAKE * 21,
+            FAKE * 22, *[ctypes.byref(x) for x in grads], FAKE * 128, ws_bytes, None)
+
+    assert call(shape=_bshape(dtype=pt.PTDIT_F32)) == 3
+    assert call(window=(1, 4, 2)) == 2                   # a window of 8 tokens
+    assert call(ws_bytes=4096) == 4
+    clash = [g[0], g[1], g[2], _wg(FAKE * 40 + 0x200000)]  # dw_swsa.dwq is dw_psa.dwv
+    assert call(grads=clash) == 8
+    assert b"dw_swsa and dw_psa overlap" in L.ptdit_last_error()

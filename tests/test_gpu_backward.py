@@ -188,3 +188,36 @@ def test_giim_bwd_flags(flags):
 def test_giim_bwd_full_size_1024px():
     """t2i 1024 px: B = 4 items of 64 x 64 latents, 256 proxies each, D = 1152."""
     _check_giim(Case(4, (1, 64, 64), 1152, 16, "bf16"), (1, 4, 4))
+
+
+# ---------------------------------------------------------------- the whole path
+
+@pytest.mark.parametrize("grid,D,heads,ratio,window,shift,B", [
+    ((2, 16, 32), 1152, 16, (1, 2, 2), (2, 8, 8), (1, 4, 4), 1),
+    # t2i 1024 px (two of its four items): 64 x 64 latents, 256 proxies, 8 x 8 windows
+    ((1, 64, 64), 1152, 16, (1, 4, 4), (1, 8, 8), (0, 4, 4), 2),
+])
+def test_block_attn_bwd(grid, D, heads, ratio, window, shift, B):
+    """GIIM then TCM: dL/dz and the four modules' weight gradients."""
+    c = Case(B, grid, D, heads, "bf16")
+    dout_cpu = _dout(c.B, c.N, c.D)
+    dz, *dw = pt.ptdit_block_attn_bwd(c.z, dout_cpu.cuda(), c.grid, ratio, window, shift,
+                                      c.w["psa"], c.w["cross"], c.w["wsa"], c.w["swsa"], c.heads)
+    dz = c.out64(dz)
+    g64 = synth.as_f64(dout_cpu)
+    mods = ("psa", "cross", "wsa", "swsa")
+    want = [[np.zeros((c.D, c.D)) for _ in range(4)] for _ in mods]
+    kappa = 0.0
+    for b in range(c.B):
+        wdz, *ww = O.block_attn_bwd(c.z64[b], c.grid, ratio, window, shift,
+                                    *[c.w64[m] for m in mods], c.heads, g64[b])
+        assert rel_err(dz[b], wdz) <= TOL["bf16"], ("dz", b)
+        for m in range(4):
+            for i in range(4):
+                want[m][i] += ww[m][i]
+        kappa = max(kappa, _proxy_kappa(c.z64[b], c.grid, ratio, c.w64["psa"], c.heads, False))
+    tol_qk = TOL["bf16"] + 2 * 2.0 ** -8 * kappa
+    for m, name in enumerate(mods):
+        for i in range(4):
+            tol = tol_qk if (name == "cross" and i < 2) else TOL["bf16"]
+            assert rel_err(c.out64(dw[m][i]), want[m][i]) <= tol, (name, i, kappa)
