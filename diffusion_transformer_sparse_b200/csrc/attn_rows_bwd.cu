@@ -10,11 +10,11 @@
 // outputs once (vector reductions), and writes dQ of each (query tile, key tile)
 // into its own column block of a bf16 [B nq, KT D] buffer (the caller sums the KT
 // blocks: the input-gradient projection takes K = KT D with the weights stacked).
-// Given the keys' mean m (kmean), dQ of each key tile is written as
-// c dS (K - m) = c dS K - rho m, rho = the row sums of the bf16 dS the MMA used: the
-// exact dS rows sum to zero, so this is the same gradient, but the rounding of dS
-// no longer multiplies the keys' common component (proxy keys are averages and
-// share most of their value).
+// The caller passes keys less their mean over each item's keys (the softmax
+// ignores a shift common to all keys, so the forward's output is the same and
+// its log-sum-exp is taken with the same keys): dQ = c dS (K - m) is then the
+// exact gradient, and the rounding of the bf16 dS no longer multiplies the keys'
+// common component (proxy keys are averages and share most of their value).
 //
 // One persistent CTA per SM, 384 threads:
 //   warp 8       loader: the item's K and V blocks (tiled head layout,
@@ -27,8 +27,7 @@
 //                r): P from lse, dS from delta (no exchange between them), the
 //                previous query tile's dQ through their own staging rows with
 //                coalesced stores, and at an item's end the key tile's dK (warp-
-//                group 1) and dV (warpgroup 0); the row sums of dS meet in
-//                shared memory (two buffers, one barrier each)
+//                group 1) and dV (warpgroup 0)
 // TMEM (64-column aligned): S 0-127, dP then dQ 128-255, dV 256-383, dK 384-511.
 // Every wait is bounded (2 s).
 #include <type_traits>
@@ -58,11 +57,10 @@ struct RbLayout {
     static constexpr int OFF_P = OFF_Q + NQB * 2 * TILE; // P, dS: 2 key halves x 128 rows x 128 B
     static constexpr int OFF_DS = OFF_P + 2 * TILE_A;
     static constexpr int OFF_STG = OFF_DS + 2 * TILE_A;  // [8 warps][32 rows][96 B] dQ staging
-    static constexpr int OFF_RHO = OFF_STG + 8 * 32 * 96;  // [2 tiles][2 warpgroups][BQ] fp32
-    static constexpr int OFF_BAR = OFF_RHO + 2 * 2 * BQ * 4;
+    static constexpr int OFF_BAR = OFF_STG + 8 * 32 * 96;
     // kv_full, kv_free, q_full[NQB], q_free[NQB], s_full, dp_full, sp_free, pds_full,
-    // pds_free, dq_full, dq_free, kvacc_full, kvacc_free, drain, rho_full[2]
-    static constexpr int NBARS = 2 * NQB + 14;
+    // pds_free, dq_full, dq_free, kvacc_full, kvacc_free, drain
+    static constexpr int NBARS = 2 * NQB + 12;
     static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16;  // the kernel checks 1 KB alignment
     static_assert(TILE_A % 1024 == 0 && TILE % 1024 == 0, "swizzled tiles stay 1 KB aligned");
     static_assert(BYTES <= 232448, "shared memory budget");
@@ -101,7 +99,7 @@ template <int DPAD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_rows_bwd_kernel(const __grid_constant__ AttnArgs a, const void *__restrict__ dout,
                          const float *__restrict__ lse, const float *__restrict__ delta,
-                         const float *__restrict__ kmean, __nv_bfloat16 *__restrict__ dq, long ldq, float *__restrict__ dk,
+                         __nv_bfloat16 *__restrict__ dq, long ldq, float *__restrict__ dk,
                          float *__restrict__ dv, RbSched sc, int *status) {
     using L = RbLayout<DPAD>;
     extern __shared__ uint8_t sm_raw[];
@@ -115,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *s_full = q_free + NQB, *dp_full = s_full + 1, *sp_free = s_full + 2;
     uint64_t *pds_full = s_full + 3, *pds_free = s_full + 4, *dq_full = s_full + 5;
     uint64_t *dq_free = s_full + 6, *kvacc_full = s_full + 7, *kvacc_free = s_full + 8;
-    uint64_t *drain = s_full + 9, *rho_full = s_full + 10;
+    uint64_t *drain = s_full + 9;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tslot + 1);
 
@@ -139,8 +137,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(kvacc_full, 1);
         mbar_init(kvacc_free, 2 * BQ);
         mbar_init(drain, 1);
-        mbar_init(&rho_full[0], 2 * BQ);
-        mbar_init(&rho_full[1], 2 * BQ);
         *abort = 0;
         fence_mbar_init();
     }
@@ -302,43 +298,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float c = a.scale, sl2 = a.scale * 1.4426950408889634f;
         uint8_t *sP = sm + L::OFF_P, *sDS = sm + L::OFF_DS;
         uint8_t *stg = sm + L::OFF_STG + warp * 32 * 96;
-        float *rho = reinterpret_cast<float *>(sm + L::OFF_RHO);
         const int kofs = 64 * g;
         // dQ of tile tt (query tile qi of item (b, h, j)) out of TMEM: warpgroup 0 writes
         // the head's pieces 0-3, warpgroup 1 pieces 4..
         auto dq_epilogue = [&](int tt, int b, int h, int j, int qi) {
             if (!mbar_wait_warp(dq_full, tt & 1, abort, status)) return false;
-            if (!mbar_wait_warp(&rho_full[tt & 1], (tt >> 1) & 1, abort, status)) return false;
             fence_after_sync();
             uint32_t v[48];
             const uint32_t t = tmem + lane_base + T_DQ + 32 * g;
             tmem_ld32(t, *reinterpret_cast<uint32_t(*)[32]>(v));
             if (g == 1 && DPAD > 64) tmem_ld16(t + 32, *reinterpret_cast<uint32_t(*)[16]>(v + 32));
-            const float rs = rho[(tt & 1) * 2 * BQ + r] + rho[(tt & 1) * 2 * BQ + BQ + r];
             tmem_ld_wait();
             fence_before_sync();
-            mbar_arrive(dq_free);  // dQ and the row sums are read: the next dP may go here
+            mbar_arrive(dq_free);  // dQ is read: the next dP may go to these columns
             const int u0 = g == 0 ? 0 : 4, nu = g == 0 ? min(4, nch) : max(0, nch - 4);
-            const float *km = kmean ? kmean + (long)b * D + (long)h * d + 8 * u0 : nullptr;
 #pragma unroll
             for (int uu = 0; uu < 6; ++uu)
                 if (uu < nu) {
-                    float x[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(v[8 * uu + e]);
-                    if (km) {
-                        const float4 m0 = *reinterpret_cast<const float4 *>(km + 8 * uu);
-                        const float4 m1 = *reinterpret_cast<const float4 *>(km + 8 * uu + 4);
-                        x[0] = fmaf(-rs, m0.x, x[0]); x[1] = fmaf(-rs, m0.y, x[1]);
-                        x[2] = fmaf(-rs, m0.z, x[2]); x[3] = fmaf(-rs, m0.w, x[3]);
-                        x[4] = fmaf(-rs, m1.x, x[4]); x[5] = fmaf(-rs, m1.y, x[5]);
-                        x[6] = fmaf(-rs, m1.z, x[6]); x[7] = fmaf(-rs, m1.w, x[7]);
-                    }
                     uint4 o;
-                    o.x = pack_bf16(x[0], x[1]);
-                    o.y = pack_bf16(x[2], x[3]);
-                    o.z = pack_bf16(x[4], x[5]);
-                    o.w = pack_bf16(x[6], x[7]);
+                    o.x = pack_bf16(__uint_as_float(v[8 * uu + 0]), __uint_as_float(v[8 * uu + 1]));
+                    o.y = pack_bf16(__uint_as_float(v[8 * uu + 2]), __uint_as_float(v[8 * uu + 3]));
+                    o.z = pack_bf16(__uint_as_float(v[8 * uu + 4]), __uint_as_float(v[8 * uu + 5]));
+                    o.w = pack_bf16(__uint_as_float(v[8 * uu + 6]), __uint_as_float(v[8 * uu + 7]));
                     *reinterpret_cast<uint4 *>(stg + lane * 96 + 16 * uu) = o;
                 }
             __syncwarp();
@@ -412,12 +393,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(tmem + lane_base + T_S + kofs, *reinterpret_cast<uint32_t(*)[32]>(sv));
                     tmem_ld32(tmem + lane_base + T_S + kofs + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
                     tmem_ld_wait();
+                    if (qv && key0 + 64 <= a.nk) {  // every key of the half is valid
 #pragma unroll
-                    for (int e = 0; e < 64; e += 2) {
-                        const bool v0 = qv && key0 + e < a.nk, v1 = qv && key0 + e + 1 < a.nk;
-                        const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -l2)) : 0.f;
-                        const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -l2)) : 0.f;
-                        pk[e / 2] = pack_bf16(p0, p1);
+                        for (int e = 0; e < 64; e += 2)
+                            pk[e / 2] = pack_bf16(ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -l2)),
+                                                  ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -l2)));
+                    } else {
+                        const int nv = qv ? (int)max(0L, min(64L, (long)a.nk - key0)) : 0;
+#pragma unroll
+                        for (int e = 0; e < 64; e += 2) {
+                            const float p0 = e < nv ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -l2)) : 0.f;
+                            const float p1 = e + 1 < nv ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -l2)) : 0.f;
+                            pk[e / 2] = pack_bf16(p0, p1);
+                        }
                     }
                 }
                 // the previous tile's dQ (and its item's dK, dV when it closed one)
@@ -435,7 +423,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int qq = 0; qq < 8; ++qq)
                     *reinterpret_cast<uint4 *>(sP + pds_chunk(r, (kofs >> 3) + qq)) =
                         make_uint4(pk[4 * qq], pk[4 * qq + 1], pk[4 * qq + 2], pk[4 * qq + 3]);
-                float rsum = 0.f;  // this warpgroup's part of the row sum of the bf16 dS
                 {
                     uint32_t dvv[64];
                     tmem_ld32(tmem + lane_base + T_DP + kofs, *reinterpret_cast<uint32_t(*)[32]>(dvv));
@@ -450,19 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e / 2]));
                             o[u] = pack_bf16(c * pr.x * (__uint_as_float(dvv[e]) - dl),
                                              c * pr.y * (__uint_as_float(dvv[e + 1]) - dl));
-                            const float2 ds = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&o[u]));
-                            rsum += ds.x + ds.y;
                         }
                         *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, (kofs >> 3) + qq)) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
-                rho[(t & 1) * 2 * BQ + g * BQ + r] = rsum;
                 fence_before_sync();
                 mbar_arrive(sp_free);
                 fence_async_smem();
                 mbar_arrive(pds_full);
-                mbar_arrive(&rho_full[t & 1]);
                 have_prev = true;
                 pb = b; ph = h; pj = j; pqi = qi; pnix = n_item;
                 prev_last = qi + 1 == q1;
@@ -488,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int DPAD>
 cudaError_t launch_rb(const AttnArgs &a, const void *dout, const float *lse, const float *delta,
-                      const float *kmean, void *dq, long ldq, float *dk, float *dv, cudaStream_t s) {
+                      void *dq, long ldq, float *dk, float *dv, cudaStream_t s) {
     using L = RbLayout<DPAD>;
     int *status = device_status_ptr();
     if (!status) return cudaErrorInvalidValue;
@@ -510,17 +493,17 @@ cudaError_t launch_rb(const AttnArgs &a, const void *dout, const float *lse, con
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
     return launch_pdl(attn_rows_bwd_kernel<DPAD>, dim3(grid), dim3(kThreads), L::BYTES, s, a, dout,
-                      lse, delta, kmean, static_cast<__nv_bfloat16 *>(dq), ldq, dk, dv, sc, status);
+                      lse, delta, static_cast<__nv_bfloat16 *>(dq), ldq, dk, dv, sc, status);
 }
 
 }  // namespace
 
 cudaError_t launch_attention_rows_bwd(const AttnArgs &a, const void *dout, const float *lse,
-                                      const float *delta, const float *kmean, void *dq, long ldq,
-                                      float *dk, float *dv, cudaStream_t s) {
+                                      const float *delta, void *dq, long ldq, float *dk, float *dv,
+                                      cudaStream_t s) {
     if (a.d < 8 || a.d > 80 || a.d % 8 || a.nq < 1 || a.nk < 1) return cudaErrorInvalidValue;
-    return a.d <= 64 ? launch_rb<64>(a, dout, lse, delta, kmean, dq, ldq, dk, dv, s)
-                     : launch_rb<80>(a, dout, lse, delta, kmean, dq, ldq, dk, dv, s);
+    return a.d <= 64 ? launch_rb<64>(a, dout, lse, delta, dq, ldq, dk, dv, s)
+                     : launch_rb<80>(a, dout, lse, delta, dq, ldq, dk, dv, s);
 }
 
 }  // namespace ptdit

@@ -285,13 +285,9 @@ cudaError_t launch_attention_win_bwd(const AttnArgs &a, const void *dout, void *
 // rows, V without padding), dout those of dL/dO; lse and delta are [B][heads][nq].
 // Writes dQ of key tile j into columns [j D, (j + 1) D) of the bf16 [B nq][ldq]
 // buffer dq and adds dK, dV into the zeroed fp32 [B nk][D] buffers dk, dv.
-// kmean (fp32 [B][D], the mean of each item's key rows, or NULL): dQ of every key
-// tile is taken against the keys less kmean (each row of the exact dS sums to
-// zero, so dS K = dS (K - kmean); with the rounded dS, the second form keeps the
-// keys' common component out of dQ).
 cudaError_t launch_attention_rows_bwd(const AttnArgs &a, const void *dout, const float *lse,
-                                      const float *delta, const float *kmean, void *dq, long ldq,
-                                      float *dk, float *dv, cudaStream_t s);
+                                      const float *delta, void *dq, long ldq, float *dk, float *dv,
+                                      cudaStream_t s);
 // dst[r][c] = sum over j < nblk of src[r][j D + c], bf16 in and out (fp32 sums); src
 // has row stride lds, dst ldd.
 cudaError_t launch_sum_blocks_bf16(const void *src, long rows, int nblk, int D, long lds,
@@ -300,6 +296,10 @@ cudaError_t launch_sum_blocks_bf16(const void *src, long rows, int nblk, int D, 
 // K in tiled head layout (identity tiles, no padding).
 cudaError_t launch_key_mean(const void *K_tiles, int B, int nk, int heads, int d, float *mean,
                             cudaStream_t s);
+// K[b][k][h d + c] -= mean[b][h d + c] for the nk valid key rows of the tiled head
+// layout (identity tiles, no padding), in bf16 through fp32.
+cudaError_t launch_center_keys(void *K_tiles, int B, int nk, int heads, int d, const float *mean,
+                               cudaStream_t s);
 // dst[b M + r][c] = bf16(src[b M + r][c] - mean over r' of src[b M + r'][c]) for the
 // fp32 row-major [B M][cols] src; dst has row stride ldd.
 cudaError_t launch_center_to_bf16(const float *src, int B, int M, int cols, void *dst, long ldd,

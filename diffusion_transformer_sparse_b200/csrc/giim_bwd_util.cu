@@ -8,6 +8,9 @@
 //   to_bf16          the fp32 key and value gradients to bf16 operands
 //   key_mean         per (batch item, head) the mean of the valid key rows (fp32),
 //                    read from the tiled head layout
+//   center_keys      the key rows less that mean, in place (the backward then
+//                    takes dQ = c dS (K - mean), which is exact: every row of dS
+//                    sums to zero)
 //   sum_blocks       dQ summed over the key tiles: dst = sum over j of the column
 //                    blocks [j D, (j + 1) D) of src (bf16, fp32 sums)
 //   center_to_bf16   the fp32 key gradient less its mean over each batch item's keys,
@@ -157,6 +160,35 @@ __global__ void key_mean_kernel(const uint8_t *__restrict__ K, int nk, int heads
     }
 }
 
+// One thread per (batch item, key row, head, 16-byte unit) of the valid rows.
+__global__ void center_keys_kernel(uint8_t *__restrict__ K, int B, int nk, int heads, int d,
+                                   const float *__restrict__ mean) {
+    pdl_wait();
+    pdl_trigger();
+    const int units = d / 8;
+    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long)B * nk * heads * units) return;
+    const int u = static_cast<int>(idx % units);
+    long rest = idx / units;
+    const int h = static_cast<int>(rest % heads);
+    rest /= heads;
+    const int k = static_cast<int>(rest % nk);
+    const long b = rest / nk;
+    const int tiles = (nk + kThlRows - 1) / kThlRows, tile = k / kThlRows, tr = k % kThlRows;
+    uint4 *p = reinterpret_cast<uint4 *>(K + ((b * tiles + tile) * heads + h) * (long)thl_block_bytes(d, 0) +
+                                         thl_unit(tr, u, 0));
+    const float *m = mean + b * heads * d + (long)h * d + 8 * u;
+    const uint4 v = *p;
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[t]));
+        const __nv_bfloat162 o = __floats2bfloat162_rn(f.x - m[2 * t], f.y - m[2 * t + 1]);
+        w[t] = *reinterpret_cast<const uint32_t *>(&o);
+    }
+    *p = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // One CTA per (batch item, 32 columns): lane = column, the 8 warps stride over the
 // item's M rows, first for the column sums, then for the centred bf16 values.
 __global__ void center_to_bf16_kernel(const float *__restrict__ src, int M, int cols,
@@ -199,6 +231,15 @@ cudaError_t launch_key_mean(const void *K_tiles, int B, int nk, int heads, int d
     if (B < 1 || nk < 1 || d < 8 || d % 8 || d > 80) return cudaErrorInvalidValue;
     return launch_pdl(key_mean_kernel, dim3((unsigned)(B * heads)), dim3(256), 0, s,
                       static_cast<const uint8_t *>(K_tiles), nk, heads, d, mean);
+}
+
+cudaError_t launch_center_keys(void *K_tiles, int B, int nk, int heads, int d, const float *mean,
+                               cudaStream_t s) {
+    if (B < 1 || nk < 1 || d < 8 || d % 8 || d > 80) return cudaErrorInvalidValue;
+    const long n = (long)B * nk * heads * (d / 8);
+    const int threads = 256;
+    return launch_pdl(center_keys_kernel, dim3((unsigned)((n + threads - 1) / threads)),
+                      dim3(threads), 0, s, static_cast<uint8_t *>(K_tiles), B, nk, heads, d, mean);
 }
 
 cudaError_t launch_center_to_bf16(const float *src, int B, int M, int cols, void *dst, long ldd,

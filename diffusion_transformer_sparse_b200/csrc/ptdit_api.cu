@@ -988,9 +988,8 @@ int wgrad_blocks(const Run &r, const void *G, int ldg, const int *gcol, float *c
     return PTDIT_OK;
 }
 
-// Row-attention backward with the keys' mean (kmean, fp32 [B][D]) taken first.
 int rows_bwd(const Run &r, AttnArgs a, const void *dO, const float *lse, const float *del,
-             float *kmean, void *dq, long ldq, float *dk, float *dv, const char *what) {
+             void *dq, long ldq, float *dk, float *dv, const char *what) {
     a.dtype = r.d.dtype;
     a.heads = r.d.heads;
     a.d = r.d.d;
@@ -1000,12 +999,9 @@ int rows_bwd(const Run &r, AttnArgs a, const void *dO, const float *lse, const f
         cudaError_t em = cudaMemsetAsync(p, 0, (size_t)r.d.B * a.nk * r.d.D * sizeof(float), r.s);
         if (em != cudaSuccess) return cuda_fail(em, "zeroing the key and value gradients");
     }
-    cudaError_t em = launch_key_mean(a.k, a.B, a.nk, a.heads, a.d, kmean, r.s);
-    count_launch();
-    if (em != cudaSuccess) return cuda_fail(em, "backward: key mean");
     TRY(launch_fault(what));
     timing_begin(PTDIT_K_ATTN_ROWS_BWD, r.s);
-    cudaError_t e = launch_attention_rows_bwd(a, dO, lse, del, kmean, dq, ldq, dk, dv, r.s);
+    cudaError_t e = launch_attention_rows_bwd(a, dO, lse, del, dq, ldq, dk, dv, r.s);
     timing_end(r.s);
     count_launch();
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
@@ -1014,6 +1010,16 @@ int rows_bwd(const Run &r, AttnArgs a, const void *dO, const float *lse, const f
 int elementwise(const Run &r, cudaError_t e, const char *what) {
     count_launch();
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, what);
+}
+
+// Keys in tiled head layout less their mean over each item's nk keys, in place (the
+// attention's output is unchanged; its backward then keeps the keys' common
+// component out of dQ).
+int center_keys(const Run &r, void *K, int nk, float *mean) {
+    const Dims &d = r.d;
+    TRY(elementwise(r, launch_key_mean(K, d.B, nk, d.heads, d.d, mean, r.s), "backward: key mean"));
+    return elementwise(r, launch_center_keys(K, d.B, nk, d.heads, d.d, mean, r.s),
+                       "backward: keys less their mean");
 }
 
 int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_attn_w *psa,
@@ -1038,6 +1044,7 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
         const ThlDesc *Tv[3] = {&tp, nullptr, nullptr};
         TRY(gemm_thl(r, PTDIT_K_GEMM, P(Lb.Pa), BM, 1, Wv, Cv, Tv, "backward: proxy V"));
     }
+    TRY(center_keys(r, P(Lb.Pk), M, F(Lb.km_p)));
     AttnArgs pa;
     memset(&pa, 0, sizeof pa);
     pa.mode = ATT_ROWS;
@@ -1064,6 +1071,7 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
         const ThlDesc *Tq[3] = {&tn, nullptr, nullptr};
         TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 1, Wq, Cq, Tq, "backward: latent Q"));
     }
+    TRY(center_keys(r, P(Lb.Ck), M, F(Lb.km_c)));
     AttnArgs ca;
     memset(&ca, 0, sizeof ca);
     ca.mode = ATT_ROWS;
@@ -1100,8 +1108,7 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
     cb.v = P(Lb.Cvb);
     cb.tv = tp;
     // dQ straight into dQc with one key tile, else per key tile, then summed
-    TRY(rows_bwd(r, cb, P(Lb.dAc), F(Lb.lse_c), F(Lb.del_c), F(Lb.km_c),
-                 ktc > 1 ? P(Lb.Gc) : P(Lb.dQc), ktc > 1 ? (long)ktc * D : (long)D, F(Lb.dKc),
+    TRY(rows_bwd(r, cb, P(Lb.dAc), F(Lb.lse_c), F(Lb.del_c), ktc > 1 ? P(Lb.Gc) : P(Lb.dQc), ktc > 1 ? (long)ktc * D : (long)D, F(Lb.dKc),
                  F(Lb.dVc), "cross-attention backward"));
     if (ktc > 1)
         TRY(elementwise(r, launch_sum_blocks_bf16(P(Lb.Gc), BN, ktc, D, (long)ktc * D, P(Lb.dQc), D,
@@ -1124,8 +1131,7 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
     AttnArgs pb = pa;
     pb.v = P(Lb.Pvb);
     pb.tv = tp;
-    TRY(rows_bwd(r, pb, P(Lb.dAp), F(Lb.lse_p), F(Lb.del_p), F(Lb.km_p),
-                 ktp > 1 ? P(Lb.Gq) : P(Lb.Gp), ktp > 1 ? (long)ktp * D : ldp, F(Lb.dKp),
+    TRY(rows_bwd(r, pb, P(Lb.dAp), F(Lb.lse_p), F(Lb.del_p), ktp > 1 ? P(Lb.Gq) : P(Lb.Gp), ktp > 1 ? (long)ktp * D : ldp, F(Lb.dKp),
                  F(Lb.dVp), "proxy self-attention backward"));
     if (ktp > 1)
         TRY(elementwise(r, launch_sum_blocks_bf16(P(Lb.Gq), BM, ktp, D, (long)ktp * D, P(Lb.Gp), ldp,
