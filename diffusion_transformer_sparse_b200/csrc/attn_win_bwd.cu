@@ -404,21 +404,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float mx[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+                // every key of the half allowed (all of WSA, SWSA away from the wrap): no
+                // per-key selects
+                const bool all = aw[0] == (NK >= 32 ? 0xffffffffu : ((1u << NK) - 1u)) &&
+                                 aw[1] == (NK >= 64 ? 0xffffffffu : 0u);
+                if (all) {
 #pragma unroll
-                for (int e = 0; e < NK; ++e)
-                    if ((aw[e >> 5] >> (e & 31)) & 1u) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
+                    for (int e = 0; e < NK; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < NK; ++e)
+                        if ((aw[e >> 5] >> (e & 31)) & 1u) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sv[e]));
+                }
                 ms_g = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
                 float ls[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) ls[i] = 0.f;
+                if (all) {
 #pragma unroll
-                for (int e = 0; e < NK; e += 2) {
-                    const uint32_t w = aw[e >> 5];
-                    const float p0 = ((w >> (e & 31)) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -ms_g)) : 0.f;
-                    const float p1 = ((w >> ((e + 1) & 31)) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -ms_g)) : 0.f;
-                    ls[(e >> 1) & 7] += p0 + p1;
-                    pk[e / 2] = pack_bf16(p0, p1);
+                    for (int e = 0; e < NK; e += 2) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -ms_g));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -ms_g));
+                        ls[(e >> 1) & 7] += p0 + p1;
+                        pk[e / 2] = pack_bf16(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < NK; e += 2) {
+                        const uint32_t w = aw[e >> 5];
+                        const float p0 = ((w >> (e & 31)) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -ms_g)) : 0.f;
+                        const float p1 = ((w >> ((e + 1) & 31)) & 1u) ? ex2_approx(fmaf(__uint_as_float(sv[e + 1]), sl2, -ms_g)) : 0.f;
+                        ls[(e >> 1) & 7] += p0 + p1;
+                        pk[e / 2] = pack_bf16(p0, p1);
+                    }
                 }
                 l_g = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
             }

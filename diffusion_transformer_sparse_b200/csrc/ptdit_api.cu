@@ -1022,17 +1022,48 @@ int center_keys(const Run &r, void *K, int nk, float *mean) {
                        "backward: keys less their mean");
 }
 
-int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_attn_w *psa,
-                 const ptdit_attn_w *cross, unsigned flags, const void *z_in, const void *dz_out,
-                 void *dz_in, const ptdit_attn_wgrad *dwp, const ptdit_attn_wgrad *dwc) {
+// The attention arguments of GIIM's two cores over the backward's workspace.
+AttnArgs giim_bwd_proxy_args(const Run &r, const WsGB &Lb, int M) {
+    AttnArgs pa;
+    memset(&pa, 0, sizeof pa);
+    pa.mode = ATT_ROWS;
+    pa.q = r.at(Lb.Pq); pa.k = r.at(Lb.Pk); pa.v = r.at(Lb.Pvf); pa.o = r.at(Lb.Ap);
+    pa.q_bstride = pa.k_bstride = M;
+    pa.nq = pa.nk = M;
+    pa.tq = pa.tk = thl_identity(M, 0);
+    pa.tv = thl_identity(M, 1, v_ones(r.d));
+    pa.lse = reinterpret_cast<float *>(r.at(Lb.lse_p));
+    return pa;
+}
+
+AttnArgs giim_bwd_cross_args(const Run &r, const WsGB &Lb, int M) {
+    AttnArgs ca;
+    memset(&ca, 0, sizeof ca);
+    ca.mode = ATT_ROWS;
+    ca.q = r.at(Lb.Cq); ca.k = r.at(Lb.Ck); ca.v = r.at(Lb.Cvf); ca.o = r.at(Lb.Ac);
+    ca.q_bstride = r.d.N;
+    ca.k_bstride = M;
+    ca.nq = (int)r.d.N;
+    ca.nk = M;
+    ca.tq = thl_identity(r.d.N, 0);
+    ca.tk = thl_identity(M, 0);
+    ca.tv = thl_identity(M, 1, v_ones(r.d));
+    ca.lse = reinterpret_cast<float *>(r.at(Lb.lse_c));
+    return ca;
+}
+
+// GIIM's forward recomputed into the backward's workspace, keeping what the backward
+// reads (proxies, projections with centred keys, both cores' outputs and log-sum-exp);
+// with z1 set, also the module's output z1 = (z_in +) A_c Wo^T.
+int giim_recompute(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_attn_w *psa,
+                   const ptdit_attn_w *cross, unsigned flags, const void *z_in, void *z1) {
     const Dims &d = r.d;
-    const int M = pg.M, D = d.D, ktc = Lb.ktc, ktp = Lb.ktp;
+    const int M = pg.M;
     const long BM = (long)d.B * M, BN = (long)d.B * d.N;
     auto P = [&](size_t o) { return r.at(o); };
     auto F = [&](size_t o) { return reinterpret_cast<float *>(r.at(o)); };
     const ThlDesc tp = thl_identity(M, 0), tpv = thl_identity(M, 1, v_ones(d));
     const ThlDesc tn = thl_identity(d.N, 0);
-    // ---- the forward, recomputed, keeping what the backward reads
     TRY(extract_proxies(d, pg, PTDIT_PROXY_MEAN, nullptr, z_in, P(Lb.Pa), r.s));
     {
         const void *W[3] = {psa->wq, psa->wk, psa->wv};
@@ -1045,16 +1076,8 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
         TRY(gemm_thl(r, PTDIT_K_GEMM, P(Lb.Pa), BM, 1, Wv, Cv, Tv, "backward: proxy V"));
     }
     TRY(center_keys(r, P(Lb.Pk), M, F(Lb.km_p)));
-    AttnArgs pa;
-    memset(&pa, 0, sizeof pa);
-    pa.mode = ATT_ROWS;
-    pa.q = P(Lb.Pq); pa.k = P(Lb.Pk); pa.v = P(Lb.Pvf); pa.o = P(Lb.Ap);
-    pa.q_bstride = pa.k_bstride = M;
-    pa.nq = pa.nk = M;
-    pa.tq = pa.tk = tp;
-    pa.tv = tpv;
-    pa.lse = F(Lb.lse_p);
-    TRY(attention(r, PTDIT_K_ATTN_PROXY, pa, "backward: proxy self-attention"));
+    TRY(attention(r, PTDIT_K_ATTN_PROXY, giim_bwd_proxy_args(r, Lb, M),
+                  "backward: proxy self-attention"));
     {
         const void *W[3] = {psa->wo, nullptr, nullptr};
         void *C[3] = {P(Lb.Pp), nullptr, nullptr};
@@ -1072,19 +1095,27 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
         TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 1, Wq, Cq, Tq, "backward: latent Q"));
     }
     TRY(center_keys(r, P(Lb.Ck), M, F(Lb.km_c)));
-    AttnArgs ca;
-    memset(&ca, 0, sizeof ca);
-    ca.mode = ATT_ROWS;
-    ca.q = P(Lb.Cq); ca.k = P(Lb.Ck); ca.v = P(Lb.Cvf); ca.o = P(Lb.Ac);
-    ca.q_bstride = d.N;
-    ca.k_bstride = M;
-    ca.nq = (int)d.N;
-    ca.nk = M;
-    ca.tq = tn;
-    ca.tk = tp;
-    ca.tv = tpv;
-    ca.lse = F(Lb.lse_c);
-    TRY(attention(r, PTDIT_K_ATTN_CROSS, ca, "backward: cross-attention"));
+    TRY(attention(r, PTDIT_K_ATTN_CROSS, giim_bwd_cross_args(r, Lb, M), "backward: cross-attention"));
+    if (z1) {
+        const void *W[3] = {cross->wo, nullptr, nullptr};
+        void *C[3] = {z1, nullptr, nullptr};
+        const void *R[3] = {(flags & PTDIT_NO_RESIDUAL) ? nullptr : z_in, nullptr, nullptr};
+        TRY(gemm(r, PTDIT_K_GEMM, P(Lb.Ac), BN, 1, W, C, R, "backward: cross output projection"));
+    }
+    return PTDIT_OK;
+}
+
+// GIIM's backward once giim_recompute has filled the workspace.
+int giim_backward(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_attn_w *psa,
+                  const ptdit_attn_w *cross, unsigned flags, const void *z_in, const void *dz_out,
+                  void *dz_in, const ptdit_attn_wgrad *dwp, const ptdit_attn_wgrad *dwc) {
+    const Dims &d = r.d;
+    const int M = pg.M, D = d.D, ktc = Lb.ktc, ktp = Lb.ktp;
+    const long BM = (long)d.B * M, BN = (long)d.B * d.N;
+    auto P = [&](size_t o) { return r.at(o); };
+    auto F = [&](size_t o) { return reinterpret_cast<float *>(r.at(o)); };
+    const ThlDesc tp = thl_identity(M, 0), tn = thl_identity(d.N, 0);
+    const AttnArgs pa = giim_bwd_proxy_args(r, Lb, M), ca = giim_bwd_cross_args(r, Lb, M);
     // ---- transposed weights for the input gradients
     TRY(transpose(r, cross->wo, D, D, P(Lb.WcoT), D));
     TRY(transpose(r, cross->wq, D, D, P(Lb.WcqT), D));
@@ -1169,6 +1200,13 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
                          "backward: dWq, dWk, dWv (proxy)"));
     }
     return PTDIT_OK;
+}
+
+int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_attn_w *psa,
+                 const ptdit_attn_w *cross, unsigned flags, const void *z_in, const void *dz_out,
+                 void *dz_in, const ptdit_attn_wgrad *dwp, const ptdit_attn_wgrad *dwc) {
+    TRY(giim_recompute(r, Lb, pg, psa, cross, flags, z_in, nullptr));
+    return giim_backward(r, Lb, pg, psa, cross, flags, z_in, dz_out, dz_in, dwp, dwc);
 }
 
 }  // namespace
@@ -1523,22 +1561,19 @@ int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int win
 }
 
 // ------------------------------------------------------------------ backward of the path
-// z1 and dL/dz1, then one area that the three stages (GIIM's forward, TCM's backward,
-// GIIM's backward) take in turn.
+// z1 and dL/dz1, GIIM's backward area (its recomputed forward stays there while TCM's
+// backward runs), then TCM's backward area.
 struct BlockBwd {
-    size_t z1, dz1, area, total;
+    size_t z1, dz1, giim, tcm, total;
 };
 BlockBwd block_bwd_layout(const Dims &d, long M) {
     BlockBwd L;
     const size_t tn = align256((size_t)d.B * d.N * d.D * d.elem);
     L.z1 = 0;
     L.dz1 = tn;
-    L.area = 2 * tn;
-    size_t need = ws_layout(d, M).total;
-    const size_t t = tcm_bwd_layout(d).total, g = ws_layout_giim_bwd(d, M).total;
-    need = need > t ? need : t;
-    need = need > g ? need : g;
-    L.total = L.area + need;
+    L.giim = 2 * tn;
+    L.tcm = L.giim + ws_layout_giim_bwd(d, M).total;
+    L.total = L.tcm + tcm_bwd_layout(d).total;
     return L;
 }
 
@@ -1596,18 +1631,15 @@ int ptdit_block_attn_bwd(const ptdit_shape *shape, const int ratio[3], const int
     const BlockBwd L = block_bwd_layout(d, pg.M);
     TRY(check_bwd_ws(ws, ws_bytes, L.total));
     const cudaStream_t s = (cudaStream_t)stream;
-    char *base = static_cast<char *>(ws), *area = base + L.area;
+    char *base = static_cast<char *>(ws);
     void *z1 = base + L.z1, *dz1 = base + L.dz1;
-    {
-        const Ws Lf = ws_layout(d, pg.M);
-        Run rf{d, s, area, Lf};
-        TRY(run_giim(rf, pg, psa, cross, flags, z_in, z1));
-    }
-    TRY(run_tcm_bwd(d, s, area, wg0, wg1, wsa, swsa, flags, z1, dz_out, dz1, dw_wsa, dw_swsa));
     const Ws none{};
-    Run r{d, s, area, none};
-    return run_giim_bwd(r, ws_layout_giim_bwd(d, pg.M), pg, psa, cross, flags, z_in, dz1, dz_in,
-                        dw_psa, dw_cross);
+    const WsGB Lg = ws_layout_giim_bwd(d, pg.M);
+    Run rg{d, s, base + L.giim, none};
+    TRY(giim_recompute(rg, Lg, pg, psa, cross, flags, z_in, z1));
+    TRY(run_tcm_bwd(d, s, base + L.tcm, wg0, wg1, wsa, swsa, flags, z1, dz_out, dz1, dw_wsa,
+                    dw_swsa));
+    return giim_backward(rg, Lg, pg, psa, cross, flags, z_in, dz1, dz_in, dw_psa, dw_cross);
 }
 
 size_t ptdit_pt_block_workspace_bytes(const ptdit_shape *shape, const int ratio[3],

@@ -249,16 +249,16 @@ int ptdit_tcm_bwd(const ptdit_shape *shape, const int window[3], const int shift
                   size_t ws_bytes, ptdit_stream_t stream);
 
 /*
- * ptdit_block_attn_bwd -- backward (training) of ptdit_block_attn: z1 = GIIM(z_in)
- *   is recomputed, then ptdit_tcm_bwd's steps at z1 give dL/dz1 and the WSA and
- *   SWSA weight gradients, then ptdit_giim_bwd's steps at z_in with dL/dz1 give
- *   dz_in and the proxy and cross modules' weight gradients (Qihoo-T2X reading
- *   note, §3 Method, Eq. GIIM and Eq. TCM: the chain rule through the block's
- *   forward order).  The 16 weight gradients (fp32 [D][D], overwritten) must not
- *   overlap one another or any other argument.  Workspace:
- *   ptdit_block_attn_bwd_workspace_bytes(shape, ratio, window) (z1, dL/dz1 and one
- *   area the three stages share).  Restrictions and errors: those of
- *   ptdit_giim_bwd and ptdit_tcm_bwd together.
+ * ptdit_block_attn_bwd -- backward (training) of ptdit_block_attn: GIIM's forward
+ *   is recomputed once (z1 = GIIM(z_in) and what GIIM's backward reads), then
+ *   ptdit_tcm_bwd's steps at z1 give dL/dz1 and the WSA and SWSA weight
+ *   gradients, then GIIM's backward with dL/dz1 gives dz_in and the proxy and
+ *   cross modules' weight gradients (Qihoo-T2X reading note, §3 Method, Eq. GIIM
+ *   and Eq. TCM: the chain rule through the block's forward order).  The 16 weight
+ *   gradients (fp32 [D][D], overwritten) must not overlap one another or any
+ *   other argument.  Workspace: ptdit_block_attn_bwd_workspace_bytes(shape,
+ *   ratio, window): z1, dL/dz1, ptdit_giim_bwd's workspace and ptdit_tcm_bwd's.
+ *   Restrictions and errors: those of ptdit_giim_bwd and ptdit_tcm_bwd together.
  */
 size_t ptdit_block_attn_bwd_workspace_bytes(const ptdit_shape *shape, const int ratio[3],
                                             const int window[3]);
