@@ -760,9 +760,10 @@ int transpose(const Run &r, const void *src, int rows, int cols, void *dst, long
     return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "weight transpose");
 }
 
+// recompute = false: Q, K, V and A already hold the branch's forward at z_in.
 int run_window_bwd(const Run &r, const WsBwd &Lb, const WinGeom &wg, const ptdit_attn_w *w,
                    unsigned flags, const void *z_in, const void *dz_out, void *dz_in,
-                   const ptdit_attn_wgrad *dw) {
+                   const ptdit_attn_wgrad *dw, bool recompute = true) {
     const Dims &d = r.d;
     const long BN = (long)d.B * d.N;
     void *Q = r.at(Lb.Q), *K = r.at(Lb.K), *V = r.at(Lb.V), *dO = r.at(Lb.dO);
@@ -780,13 +781,13 @@ int run_window_bwd(const Run &r, const WsBwd &Lb, const WinGeom &wg, const ptdit
     a.tq = a.tk = tw;
     a.tv = twv;
     // the branch recomputed from its input: Q, K, V and the attention output A
-    {
+    if (recompute) {
         const void *W[3] = {w->wq, w->wk, w->wv};
         void *C[3] = {Q, K, V};
         const ThlDesc *T[3] = {&tw, &tw, &twv};
         TRY(gemm_thl(r, PTDIT_K_GEMM, z_in, BN, 3, W, C, T, "backward: QKV projection"));
+        TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "backward: window attention"));
     }
-    TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "backward: window attention"));
     // W^T for the input gradients: dA = dz_out Wo, dx = [dQ dK dV] [Wq; Wk; Wv]
     TRY(transpose(r, w->wo, d.D, d.D, WoT, d.D));
     const void *Wi[3] = {w->wq, w->wk, w->wv};
@@ -843,17 +844,23 @@ int run_window_bwd(const Run &r, const WsBwd &Lb, const WinGeom &wg, const ptdit
 }
 
 // The TCM backward's workspace: the branch backward's, then z^ and dL/dz^.
+// The SWSA branch's backward buffers, z^ and dL/dz^, and WSA's forward at z_in (its Q,
+// K, V window tiles and attention output, which WSA's backward then reuses).
 struct TcmBwd {
     WsBwd bwd;
-    size_t zh, dzh, total;
+    size_t zh, dzh, wq, wk, wv, wa, total;
 };
 TcmBwd tcm_bwd_layout(const Dims &d) {
     TcmBwd T;
     T.bwd = ws_layout_bwd(d);
-    const size_t tn = align256((size_t)d.B * d.N * d.D * d.elem);
+    const size_t tn = align256((size_t)d.B * d.N * d.D * d.elem), tq = align256(thl_bytes(d, d.N, 0));
     T.zh = T.bwd.total;
     T.dzh = T.zh + tn;
-    T.total = T.dzh + tn;
+    T.wq = T.dzh + tn;
+    T.wk = T.wq + tq;
+    T.wv = T.wk + tq;
+    T.wa = T.wv + tq;
+    T.total = T.wa + tn;
     return T;
 }
 
@@ -866,14 +873,16 @@ int run_tcm_bwd(const Dims &d, cudaStream_t s, char *ws, const WinGeom &wg0, con
                 const ptdit_attn_wgrad *dw_swsa) {
     const TcmBwd T = tcm_bwd_layout(d);
     Ws Lf{};
-    Lf.Q = T.bwd.Q; Lf.K = T.bwd.K; Lf.V = T.bwd.V; Lf.O = T.bwd.A;
+    Lf.Q = T.wq; Lf.K = T.wk; Lf.V = T.wv; Lf.O = T.wa;
     Run rf{d, s, ws, Lf};
     void *zh = rf.at(T.zh), *dzh = rf.at(T.dzh);
     TRY(run_window(rf, wg0, wsa, flags, z_in, zh));
     const Ws none{};
     Run r{d, s, ws, none};
     TRY(run_window_bwd(r, T.bwd, wg1, swsa, flags, zh, dz_out, dzh, dw_swsa));
-    return run_window_bwd(r, T.bwd, wg0, wsa, flags, z_in, dzh, dz_in, dw_wsa);
+    WsBwd Lw = T.bwd;  // WSA's backward on the forward kept above
+    Lw.Q = T.wq; Lw.K = T.wk; Lw.V = T.wv; Lw.A = T.wa;
+    return run_window_bwd(r, Lw, wg0, wsa, flags, z_in, dzh, dz_in, dw_wsa, false);
 }
 
 int check_bwd_io(const Dims &d, const ptdit_attn_w *w, const void *z_in, const void *dz_out,

@@ -99,15 +99,15 @@ def giim_bwd_flops(N: int, M: int, D: int) -> dict:
 
 def block_bwd_flops(N: int, M: int, n: int, D: int) -> dict:
     """Backward of the block-attention path as ptdit_block_attn_bwd runs it, per batch
-    item: GIIM's forward for z1, TCM's backward (the WSA forward for z^ and both
-    branches' backward) and GIIM's backward."""
+    item: GIIM's forward for z1, TCM's backward (the WSA forward for z^, then both
+    branches' backward, WSA's on the forward kept from z^) and GIIM's backward."""
     fwd = block_flops(N, M, n, D)
     w = window_bwd_flops(N, n, D)
     g = giim_bwd_flops(N, M, D)
     f = {
         "giim_forward": fwd["psa_proj"] + fwd["psa_core"] + fwd["cross_proj"] + fwd["cross_core"],
         "tcm_recompute": fwd["wsa_proj"] + fwd["wsa_core"],
-        "tcm_bwd": 2 * w["total"],
+        "tcm_bwd": 2 * w["total"] - w["recompute_proj"] - w["recompute_core"],
         "giim_bwd": g["total"],
     }
     f["total"] = sum(f.values())

@@ -234,9 +234,10 @@ int ptdit_giim_bwd(const ptdit_shape *shape, const int ratio[3], const ptdit_att
                    ptdit_stream_t stream);
 
 /*
- * ptdit_tcm_bwd -- backward of ptdit_tcm: z^ = WSA(z_in) (+ z_in) is recomputed,
- *   then the SWSA branch's backward at z^ and the WSA branch's backward at
- *   z_in (each as ptdit_window_attn_bwd).  dw_wsa and dw_swsa receive the two
+ * ptdit_tcm_bwd -- backward of ptdit_tcm: z^ = WSA(z_in) (+ z_in) is recomputed
+ *   (WSA's Q, K, V and attention output kept in the workspace), then the SWSA
+ *   branch's backward at z^ and the WSA branch's backward at z_in (each as
+ *   ptdit_window_attn_bwd; WSA's reuses the kept forward).  dw_wsa and dw_swsa receive the two
  *   modules' weight gradients (fp32, overwritten).  Workspace:
  *   ptdit_tcm_bwd_workspace_bytes(shape, window).  Restrictions and errors as
  *   ptdit_window_attn_bwd.

@@ -257,7 +257,7 @@ def test_window_bwd_workspace_bytes(L):
     tn = 4 * 4096 * 1152 * 2
     assert n == 4 * tq + tn + 3 * tn + 1152 * 1152 * 2 + 3 * 1152 * 1152 * 2
     t = L.ptdit_tcm_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 8, 8)))
-    assert t == n + 2 * tn  # plus z^ and dL/dz^
+    assert t == n + 2 * tn + 3 * tq + tn  # plus z^, dL/dz^ and WSA's kept Q, K, V and A
     assert L.ptdit_window_attn_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 3, 8))) == 0
 
 
