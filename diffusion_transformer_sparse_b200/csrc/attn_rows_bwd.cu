@@ -20,15 +20,20 @@
 //   warp 8       loader: the item's K and V blocks (tiled head layout,
 //                thl.cuh, no V padding), and each query tile's Q and dO blocks
 //                (two buffers)
-//   warp 9       MMA issuer: S = Q K^T and dP = dO V^T into TMEM; once P and dS
-//                are in shared memory: dV += P^T dO, dK += dS^T Q (accumulated
-//                over the item's query tiles) and dQ = dS K (dP's columns)
+//   warp 9       MMA issuer: S = Q K^T into TMEM, dP = dO V^T into S's columns
+//                once S is read; once P and dS are in shared memory: dV += P^T dO,
+//                dK += dS^T Q (accumulated over the item's query tiles) and dQ =
+//                dS K.  Within an item a tile's work is issued as S(t+1), dV(t),
+//                dK(t), dP(t+1), dQ(t): the warpgroups compute P(t+1) while dV(t)
+//                and dK(t) run; P is released after dV, dS after dQ.  An item's
+//                last tile issues its gradients first (the next item's K and V
+//                load once dQ has read K).
 //   warps 0-7    two warpgroups, 64 keys of every row each (thread r: query row
-//                r): P from lse, dS from delta (no exchange between them), the
-//                previous query tile's dQ through their own staging rows with
+//                r): P from lse, dS from delta (no exchange between them), then
+//                the previous query tile's dQ through their own staging rows with
 //                coalesced stores, and at an item's end the key tile's dK (warp-
 //                group 1) and dV (warpgroup 0)
-// TMEM (64-column aligned): S 0-127, dP then dQ 128-255, dV 256-383, dK 384-511.
+// TMEM (64-column aligned): S then dP 0-127, dQ 128-255, dV 256-383, dK 384-511.
 // Every wait is bounded (2 s).
 #include <type_traits>
 
@@ -43,7 +48,7 @@ using namespace tc;
 constexpr int BQ = 128;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 128, T_DV = 256, T_DK = 384;
+constexpr uint32_t T_S = 0, T_DP = 0, T_DQ = 128, T_DV = 256, T_DK = 384;
 constexpr int NQB = 2;  // query-tile buffers
 
 template <int DPAD>
@@ -58,8 +63,8 @@ struct RbLayout {
     static constexpr int OFF_DS = OFF_P + 2 * TILE_A;
     static constexpr int OFF_STG = OFF_DS + 2 * TILE_A;  // [8 warps][32 rows][96 B] dQ staging
     static constexpr int OFF_BAR = OFF_STG + 8 * 32 * 96;
-    // kv_full, kv_free, q_full[NQB], q_free[NQB], s_full, dp_full, sp_free, pds_full,
-    // pds_free, dq_full, dq_free, kvacc_full, kvacc_free, drain
+    // kv_full, kv_free, q_full[NQB], q_free[NQB], s_full, dp_full, s_read, pds_full,
+    // p_free, dq_full, dq_free, kvacc_full, kvacc_free, drain
     static constexpr int NBARS = 2 * NQB + 12;
     static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16;  // the kernel checks 1 KB alignment
     static_assert(TILE_A % 1024 == 0 && TILE % 1024 == 0, "swizzled tiles stay 1 KB aligned");
@@ -110,8 +115,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sm = sm_raw;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
     uint64_t *kv_full = bars, *kv_free = bars + 1, *q_full = bars + 2, *q_free = q_full + NQB;
-    uint64_t *s_full = q_free + NQB, *dp_full = s_full + 1, *sp_free = s_full + 2;
-    uint64_t *pds_full = s_full + 3, *pds_free = s_full + 4, *dq_full = s_full + 5;
+    uint64_t *s_full = q_free + NQB, *dp_full = s_full + 1, *s_read = s_full + 2;
+    uint64_t *pds_full = s_full + 3, *p_free = s_full + 4, *dq_full = s_full + 5;
     uint64_t *dq_free = s_full + 6, *kvacc_full = s_full + 7, *kvacc_free = s_full + 8;
     uint64_t *drain = s_full + 9;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
@@ -129,9 +134,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(sp_free, 2 * BQ);
+        mbar_init(s_read, 2 * BQ);
         mbar_init(pds_full, 2 * BQ);
-        mbar_init(pds_free, 1);
+        mbar_init(p_free, 1);
         mbar_init(dq_full, 1);
         mbar_init(dq_free, 2 * BQ);
         mbar_init(kvacc_full, 1);
@@ -195,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t id_km16 = idesc_bf16(BQ, 16, true, false);
             const uint32_t aP = smem_u32(sm + L::OFF_P), aDS = smem_u32(sm + L::OFF_DS);
             const uint32_t aK = smem_u32(sm + L::OFF_K), aV = smem_u32(sm + L::OFF_V);
+            auto qbuf = [&](int t) { return smem_u32(sm + L::OFF_Q + (t % NQB) * 2 * L::TILE); };
             auto scores = [&](uint32_t d_col, uint32_t aX, uint32_t aY) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
@@ -218,7 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true, any = false;
             int it = i0, n_item = 0, pos = 0;  // item of tile t, its ordinal, t's place in it
             while (it < i1 && item_tiles(it) == 0) ++it;
-            // the tiles' items: (first tile of an item?, last tile of an item?)
             auto advance = [&](int &itx, int &nix, int &posx) {
                 if (++posx == item_tiles(itx)) {
                     posx = 0;
@@ -226,59 +231,73 @@ __global__ void __launch_bounds__(kThreads, 1)
                     do { ++itx; } while (itx < i1 && item_tiles(itx) == 0);
                 }
             };
+            // S(t) into columns 0-127 (K of item nix when t opens it)
             auto issue_s = [&](int t, bool new_item, int nix) {
                 if (new_item && !mbar_wait(kv_full, nix & 1, abort, status)) return false;
                 if (!mbar_wait(&q_full[t % NQB], (t / NQB) & 1, abort, status)) return false;
                 fence_after_sync();
-                scores(T_S, smem_u32(sm + L::OFF_Q + (t % NQB) * 2 * L::TILE), aK);
+                scores(T_S, qbuf(t), aK);
                 mma_commit(s_full);
                 any = true;
                 return true;
             };
+            // dP(t) into the same columns once the warpgroups have read S(t)
             auto issue_dp = [&](int t) {
-                scores(T_DP, smem_u32(sm + L::OFF_Q + (t % NQB) * 2 * L::TILE + L::TILE), aV);
+                if (!mbar_wait(s_read, t & 1, abort, status)) return false;
+                fence_after_sync();
+                scores(T_DP, qbuf(t) + L::TILE, aV);
                 mma_commit(dp_full);
+                return true;
             };
-            if (T > 0) {
-                ok = issue_s(0, true, 0);
-                if (ok) issue_dp(0);
-            }
+            // dV += P^T dO, then dK += dS^T Q of tile t (the item's first tile overwrites)
+            auto issue_dvdk = [&](int t, bool first) {
+                const uint32_t aQ = qbuf(t), aO = aQ + L::TILE;
+#pragma unroll
+                for (int ks = 0; ks < BQ / 16; ++ks)
+                    grad(T_DV, sdesc_sw128_mn(aP + ks * 2048, L::TILE_A), aO, ks, true,
+                         !first || ks > 0);
+                mma_commit(p_free);  // P is read
+#pragma unroll
+                for (int ks = 0; ks < BQ / 16; ++ks)
+                    grad(T_DK, sdesc_sw128_mn(aDS + ks * 2048, L::TILE_A), aQ, ks, true,
+                         !first || ks > 0);
+                mma_commit(&q_free[t % NQB]);  // Q and dO are read
+            };
+            // dQ = dS K of tile t in its own columns, once the previous dQ is read
+            auto issue_dq = [&](int t) {
+                if (t > 0 && !mbar_wait(dq_free, (t - 1) & 1, abort, status)) return false;
+                fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < BQ / 16; ++ks)
+                    grad(T_DQ, sdesc_sw128(aDS + (ks >> 2) * L::TILE_A + (ks & 3) * 32), aK, ks,
+                         false, ks > 0);
+                mma_commit(dq_full);  // dQ is in TMEM and dS is read
+                return true;
+            };
+            if (T > 0) ok = issue_s(0, true, 0) && issue_dp(0);
             for (int t = 0; t < T && ok; ++t) {
                 const bool first = pos == 0, last = pos + 1 == item_tiles(it);
                 int it2 = it, n2 = n_item, pos2 = pos;
                 advance(it2, n2, pos2);  // tile t + 1
-                if (!mbar_wait(sp_free, t & 1, abort, status)) break;
-                // the next tile's scores, unless it opens a new item (its K arrives only
-                // once this tile's gradients have freed the key buffer)
-                if (t + 1 < T && !last) ok = issue_s(t + 1, false, n2);
-                if (!ok) break;
+                // P(t) and dS(t) written, dP(t) read (S's columns are free)
                 if (!mbar_wait(pds_full, t & 1, abort, status)) break;
                 if (first && n_item > 0 && !mbar_wait(kvacc_free, (n_item - 1) & 1, abort, status))
                     break;
                 fence_after_sync();
-                const uint32_t aQ = smem_u32(sm + L::OFF_Q + (t % NQB) * 2 * L::TILE);
-                const uint32_t aO = aQ + L::TILE;
-#pragma unroll
-                for (int ks = 0; ks < BQ / 16; ++ks) {
-                    const uint64_t pT = sdesc_sw128_mn(aP + ks * 2048, L::TILE_A);
-                    const uint64_t sT = sdesc_sw128_mn(aDS + ks * 2048, L::TILE_A);
-                    const uint64_t sK = sdesc_sw128(aDS + (ks >> 2) * L::TILE_A + (ks & 3) * 32);
-                    grad(T_DV, pT, aO, ks, true, !first || ks > 0);  // dV += P^T dO
-                    grad(T_DK, sT, aQ, ks, true, !first || ks > 0);  // dK += dS^T Q
-                    grad(T_DQ, sK, aK, ks, false, ks > 0);           // dQ = dS K
-                }
-                mma_commit(dq_full);
-                mma_commit(pds_free);
-                mma_commit(&q_free[t % NQB]);
-                if (last) {
+                if (!last) {
+                    // within an item: the next S, this tile's dV and dK, the next dP, this
+                    // dQ, so that the warpgroups compute the next P while dV and dK run
+                    if (!issue_s(t + 1, false, n2)) break;
+                    issue_dvdk(t, first);
+                    ok = issue_dp(t + 1) && issue_dq(t);
+                } else {
+                    // the item's last tile: its gradients first (the next item's K and V
+                    // load only once dQ has read K)
+                    issue_dvdk(t, first);
+                    if (!issue_dq(t)) break;
                     mma_commit(kvacc_full);
                     mma_commit(kv_free);
-                    if (t + 1 < T) ok = issue_s(t + 1, true, n2);
-                }
-                if (ok && t + 1 < T) {
-                    if (!mbar_wait(dq_free, t & 1, abort, status)) break;
-                    fence_after_sync();
-                    issue_dp(t + 1);
+                    if (t + 1 < T) ok = issue_s(t + 1, true, n2) && issue_dp(t + 1);
                 }
                 it = it2;
                 n_item = n2;
@@ -301,8 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kofs = 64 * g;
         // dQ of tile tt (query tile qi of item (b, h, j)) out of TMEM: warpgroup 0 writes
         // the head's pieces 0-3, warpgroup 1 pieces 4..
-        auto dq_epilogue = [&](int tt, int b, int h, int j, int qi) {
-            if (!mbar_wait_warp(dq_full, tt & 1, abort, status)) return false;
+        auto dq_epilogue = [&](int tt, int b, int h, int j, int qi, bool wait) {
+            if (wait && !mbar_wait_warp(dq_full, tt & 1, abort, status)) return false;
             fence_after_sync();
             uint32_t v[48];
             const uint32_t t = tmem + lane_base + T_DQ + 32 * g;
@@ -310,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (g == 1 && DPAD > 64) tmem_ld16(t + 32, *reinterpret_cast<uint32_t(*)[16]>(v + 32));
             tmem_ld_wait();
             fence_before_sync();
-            mbar_arrive(dq_free);  // dQ is read: the next dP may go to these columns
+            mbar_arrive(dq_free);  // dQ is read: the next dQ may go to these columns
             const int u0 = g == 0 ? 0 : 4, nu = g == 0 ? min(4, nch) : max(0, nch - 4);
 #pragma unroll
             for (int uu = 0; uu < 6; ++uu)
@@ -393,6 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(tmem + lane_base + T_S + kofs, *reinterpret_cast<uint32_t(*)[32]>(sv));
                     tmem_ld32(tmem + lane_base + T_S + kofs + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
                     tmem_ld_wait();
+                    fence_before_sync();
+                    mbar_arrive(s_read);  // S is read: dP may go to its columns
                     if (qv && key0 + 64 <= a.nk) {  // every key of the half is valid
 #pragma unroll
                         for (int e = 0; e < 64; e += 2)
@@ -408,44 +429,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                // the previous tile's dQ (and its item's dK, dV when it closed one)
-                if (have_prev) {
-                    if (!dq_epilogue(t - 1, pb, ph, pj, pqi)) { okw = false; break; }
-                    if (prev_last && !kv_flush(pnix, pb, ph, pj)) { okw = false; break; }
-                }
-                if (!mbar_wait_warp(pds_free, (t & 1) ^ 1, abort, status) ||
-                    !mbar_wait_warp(dp_full, t & 1, abort, status)) {
-                    okw = false;
-                    break;
-                }
-                fence_after_sync();
+                // P into shared memory once the previous tile's dV has read it
+                if (t > 0 && !mbar_wait_warp(p_free, (t - 1) & 1, abort, status)) { okw = false; break; }
 #pragma unroll
                 for (int qq = 0; qq < 8; ++qq)
                     *reinterpret_cast<uint4 *>(sP + pds_chunk(r, (kofs >> 3) + qq)) =
                         make_uint4(pk[4 * qq], pk[4 * qq + 1], pk[4 * qq + 2], pk[4 * qq + 3]);
+                // dS = c P (dP - delta) in registers, then into shared memory once the
+                // previous tile's dK and dQ have read it
+                if (!mbar_wait_warp(dp_full, t & 1, abort, status)) { okw = false; break; }
+                fence_after_sync();
+                uint32_t ds[32];
                 {
                     uint32_t dvv[64];
                     tmem_ld32(tmem + lane_base + T_DP + kofs, *reinterpret_cast<uint32_t(*)[32]>(dvv));
                     tmem_ld32(tmem + lane_base + T_DP + kofs + 32, *reinterpret_cast<uint32_t(*)[32]>(dvv + 32));
                     tmem_ld_wait();
 #pragma unroll
-                    for (int qq = 0; qq < 8; ++qq) {
-                        uint32_t o[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int e = 8 * qq + 2 * u;
-                            const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e / 2]));
-                            o[u] = pack_bf16(c * pr.x * (__uint_as_float(dvv[e]) - dl),
-                                             c * pr.y * (__uint_as_float(dvv[e + 1]) - dl));
-                        }
-                        *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, (kofs >> 3) + qq)) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
+                    for (int e = 0; e < 64; e += 2) {
+                        const float2 pr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pk[e / 2]));
+                        ds[e / 2] = pack_bf16(c * pr.x * (__uint_as_float(dvv[e]) - dl),
+                                              c * pr.y * (__uint_as_float(dvv[e + 1]) - dl));
                     }
                 }
-                fence_before_sync();
-                mbar_arrive(sp_free);
+                if (t > 0 && !mbar_wait_warp(dq_full, (t - 1) & 1, abort, status)) { okw = false; break; }
+#pragma unroll
+                for (int qq = 0; qq < 8; ++qq)
+                    *reinterpret_cast<uint4 *>(sDS + pds_chunk(r, (kofs >> 3) + qq)) =
+                        make_uint4(ds[4 * qq], ds[4 * qq + 1], ds[4 * qq + 2], ds[4 * qq + 3]);
+                fence_before_sync();  // dP is read: the next S may go to its columns
                 fence_async_smem();
                 mbar_arrive(pds_full);
+                // the previous tile's dQ (its dq_full is complete), and its item's dK, dV
+                // when it closed one
+                if (have_prev) {
+                    if (!dq_epilogue(t - 1, pb, ph, pj, pqi, false)) { okw = false; break; }
+                    if (prev_last && !kv_flush(pnix, pb, ph, pj)) { okw = false; break; }
+                }
                 have_prev = true;
                 pb = b; ph = h; pj = j; pqi = qi; pnix = n_item;
                 prev_last = qi + 1 == q1;
@@ -453,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_item;
         }
         if (okw && have_prev) {
-            if (dq_epilogue(t - 1, pb, ph, pj, pqi) && prev_last) kv_flush(pnix, pb, ph, pj);
+            if (dq_epilogue(t - 1, pb, ph, pj, pqi, true) && prev_last) kv_flush(pnix, pb, ph, pj);
         }
     }
     if (*abort) {
