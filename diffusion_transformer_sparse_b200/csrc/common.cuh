@@ -242,10 +242,22 @@ cudaError_t launch_row_delta(const void *dO_tiles, const void *O, int B, int nq,
 cudaError_t launch_proxy_broadcast(const ProxyGeom &g, int B, int D, const void *dPa,
                                    const void *dout, void *dz, cudaStream_t s);
 
-// dst[c][r] = src[r][c] for a row-major bf16 [rows][cols] matrix (dst has
-// row stride ldd >= rows, so several transposes can fill one wider matrix).
-cudaError_t launch_transpose_bf16(const void *src, int rows, int cols, void *dst, long ldd,
-                                  cudaStream_t s);
+// dst[c][r] = src[r][c] for row-major bf16 [rows][cols] matrices (dst has row
+// stride ldd >= rows, so several transposes can fill one wider matrix), up to
+// kTransposeMax in one launch; rows, cols and ldd multiples of 8, src and dst
+// 16-byte aligned.
+constexpr int kTransposeMax = 8;
+struct TransposeJob {
+    const void *src;
+    void *dst;
+    int rows, cols;
+    long ldd;
+};
+struct TransposeBatch {
+    TransposeJob job[kTransposeMax];
+    int n;
+};
+cudaError_t launch_transpose_batch_bf16(const TransposeBatch &jb, cudaStream_t s);
 // The 2-SM projection GEMM's tile order for rows x nseg outputs of nmat
 // matrices on `pairs` CTA pairs (host only): *tiles, and *scheduled = 1 with
 // pair q taking tile[first[q]] .. tile[first[q+1] - 1] when the launch runs a

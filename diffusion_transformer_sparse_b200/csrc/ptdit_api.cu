@@ -751,13 +751,18 @@ int check_bwd_shape(const Dims &d, const WinGeom &wg) {
     return PTDIT_OK;
 }
 
-int transpose(const Run &r, const void *src, int rows, int cols, void *dst, long ldd) {
-    TRY(launch_fault("weight transpose"));
+// The D x D weights' transposes: src[i]^T into dst[i] (row stride ldd[i]), one launch.
+int transposes(const Run &r, int n, const void *const *src, void *const *dst, const long *ldd) {
+    TransposeBatch jb;
+    memset(&jb, 0, sizeof jb);
+    jb.n = n;
+    for (int i = 0; i < n; ++i) jb.job[i] = TransposeJob{src[i], dst[i], r.d.D, r.d.D, ldd[i]};
+    TRY(launch_fault("weight transposes"));
     timing_begin(PTDIT_K_TRANSPOSE, r.s);
-    cudaError_t e = launch_transpose_bf16(src, rows, cols, dst, ldd, r.s);
+    cudaError_t e = launch_transpose_batch_bf16(jb, r.s);
     timing_end(r.s);
     count_launch();
-    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "weight transpose");
+    return e == cudaSuccess ? PTDIT_OK : cuda_fail(e, "weight transposes");
 }
 
 // recompute = false: Q, K, V and A already hold the branch's forward at z_in.
@@ -789,11 +794,14 @@ int run_window_bwd(const Run &r, const WsBwd &Lb, const WinGeom &wg, const ptdit
         TRY(attention(r, PTDIT_K_ATTN_WINDOW, a, "backward: window attention"));
     }
     // W^T for the input gradients: dA = dz_out Wo, dx = [dQ dK dV] [Wq; Wk; Wv]
-    TRY(transpose(r, w->wo, d.D, d.D, WoT, d.D));
-    const void *Wi[3] = {w->wq, w->wk, w->wv};
-    for (int i = 0; i < 3; ++i)
-        TRY(transpose(r, Wi[i], d.D, d.D, static_cast<char *>(WqkvT) + (size_t)i * d.D * d.elem,
-                      3L * d.D));
+    {
+        char *qkv = static_cast<char *>(WqkvT);
+        const size_t blk = (size_t)d.D * d.elem;
+        const void *src[4] = {w->wo, w->wq, w->wk, w->wv};
+        void *dst[4] = {WoT, qkv, qkv + blk, qkv + 2 * blk};
+        const long ld[4] = {d.D, 3L * d.D, 3L * d.D, 3L * d.D};
+        TRY(transposes(r, 4, src, dst, ld));
+    }
     {
         const void *W[3] = {WoT, nullptr, nullptr};
         void *C[3] = {dO, nullptr, nullptr};
@@ -1126,15 +1134,16 @@ int giim_backward(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit
     const ThlDesc tp = thl_identity(M, 0), tn = thl_identity(d.N, 0);
     const AttnArgs pa = giim_bwd_proxy_args(r, Lb, M), ca = giim_bwd_cross_args(r, Lb, M);
     // ---- transposed weights for the input gradients
-    TRY(transpose(r, cross->wo, D, D, P(Lb.WcoT), D));
-    TRY(transpose(r, cross->wq, D, D, P(Lb.WcqT), D));
-    TRY(transpose(r, cross->wk, D, D, P(Lb.WckvT), 2L * D));
-    TRY(transpose(r, cross->wv, D, D, P(Lb.WckvT) + (size_t)D * d.elem, 2L * D));
-    TRY(transpose(r, psa->wo, D, D, P(Lb.WpoT), D));
     const long ldp = 3L * D;
-    TRY(transpose(r, psa->wq, D, D, P(Lb.WpT), ldp));
-    TRY(transpose(r, psa->wk, D, D, P(Lb.WpT) + (size_t)D * d.elem, ldp));
-    TRY(transpose(r, psa->wv, D, D, P(Lb.WpT) + (size_t)2 * D * d.elem, ldp));
+    {
+        const size_t blk = (size_t)D * d.elem;
+        const void *src[8] = {cross->wo, cross->wq, cross->wk, cross->wv,
+                              psa->wo, psa->wq, psa->wk, psa->wv};
+        void *dst[8] = {P(Lb.WcoT), P(Lb.WcqT), P(Lb.WckvT), P(Lb.WckvT) + blk,
+                        P(Lb.WpoT), P(Lb.WpT), P(Lb.WpT) + blk, P(Lb.WpT) + 2 * blk};
+        const long ld[8] = {D, D, 2L * D, 2L * D, D, ldp, ldp, ldp};
+        TRY(transposes(r, 8, src, dst, ld));
+    }
     // ---- cross-attention backward
     {
         const void *W[3] = {P(Lb.WcoT), nullptr, nullptr};
