@@ -296,22 +296,28 @@ def config_of(w):
 
 
 # ------------------------------------------------------------------ GPU arm
-def kernel_work(w):
+def kernel_work(w, fused=False):
     """Algorithmic work per step of each kernel kind (library timing-hook names):
     (amount, unit, bound).  Averaging and the window cores are HBM-bound and
     count bytes: averaging reads N and writes M rows of D elements; a window
     core reads Q, K and V and writes O, 4 N D elements per launch.  The others
-    count FLOP (a multiply-add is 2)."""
+    count FLOP (a multiply-add is 2).  With the fused window kernel, the two
+    window branches' Q/K/V projections (6 N D^2 each) and cores count there."""
     e = 2 if w.dtype == "bf16" else 4
     f = flops.block_flops(w.N, w.M, w.n, w.D)
     B = w.B
-    return {
+    work = {
         "average": (B * flops.average_bytes(w.N, w.M, w.D, e), "bytes", "hbm"),
         "gemm": (B * f["proj"], "flop", "tensor"),
         "attn_proxy": (B * f["psa_core"], "flop", "tensor"),
         "attn_cross": (B * f["cross_core"], "flop", "tensor"),
         "attn_window": (B * 2 * 4 * w.N * w.D * e, "bytes", "hbm"),
     }
+    if fused:
+        qkv = 2 * 6 * w.N * w.D * w.D
+        work["gemm"] = (B * (f["proj"] - qkv), "flop", "tensor")
+        work["attn_window_fused"] = (B * (qkv + f["wsa_core"] + f["swsa_core"]), "flop", "tensor")
+    return work
 
 
 def run_gpu(args, w):
@@ -323,6 +329,8 @@ def run_gpu(args, w):
     dev = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
     pt.lib()
+    if getattr(args, "fused_window", False):
+        pt.lib().ptdit_window_fused(1)
 
     z_host, W_host = host_inputs(w)
     z = z_host.to(dev)
@@ -397,7 +405,7 @@ def run_gpu(args, w):
     peaks = load_peaks()
     f = flops.block_flops(w.N, w.M, w.n, w.D)
     step_flops = w.B * f["total"]
-    work = kernel_work(w)
+    work = kernel_work(w, fused="attn_window_fused" in per_kind)
     kernels = {}
     hooked_kernel_ms = sum(v[1] for v in per_kind.values()) / args.steps
     for k, (n, t) in sorted(per_kind.items()):
@@ -419,7 +427,7 @@ def run_gpu(args, w):
         kernels[k] = ent
     gemm_n, gemm_t = per_kind.get("gemm", [0, 0.0])
     gemm_ms = gemm_t / args.steps
-    proj_flops = w.B * f["proj"]
+    proj_flops = work["gemm"][0]
     achieved = proj_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     peak_note = "measured" if peaks["source"] == "measured" else "fallback"
     traffic = TRAFFIC.get(w.name)
@@ -454,7 +462,8 @@ def run_gpu(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
             "data": "synthetic (seeded N(0,1) latents, Xavier-uniform weights)",
-            "config": config_of(w),
+            "config": dict(config_of(w), window_kernels="fused projection + attention"
+                           if getattr(args, "fused_window", False) else "projection, then attention"),
             "tflops": step_flops / (ms_step / 1e3) / 1e12,
             "roofline": roofline,
             "cpu_baseline": cpu,
@@ -740,6 +749,9 @@ def main(argv=None):
     ap.add_argument("--ratio", type=parse3, help="override the proxy ratio F,H,W")
     ap.add_argument("--dense", action="store_true",
                     help="time the dense comparator (full global self-attention) instead")
+    ap.add_argument("--fused-window", action="store_true",
+                    help="take the fused window Q/K/V projection + attention kernel "
+                         "(ptdit_window_fused(1)) for windows of 128 tokens")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward of the block-attention path instead")
     ap.add_argument("--bwd-branch", action="store_true",

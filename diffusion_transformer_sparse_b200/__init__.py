@@ -22,7 +22,8 @@ PROXY_MODES = {"mean": PTDIT_PROXY_MEAN, "first": PTDIT_PROXY_FIRST, "random": P
 (PTDIT_OK, PTDIT_ERR_NULL, PTDIT_ERR_SHAPE, PTDIT_ERR_DTYPE, PTDIT_ERR_WORKSPACE, PTDIT_ERR_CUDA,
  PTDIT_ERR_TIMEOUT, PTDIT_ERR_ALIGN, PTDIT_ERR_ALIAS) = range(9)
 KINDS = ("average", "gemm", "attn_proxy", "attn_cross", "attn_window", "attn_dense", "norm",
-         "attn_text", "attn_window_bwd", "wgrad", "transpose", "attn_rows_bwd")
+         "attn_text", "attn_window_bwd", "wgrad", "transpose", "attn_rows_bwd",
+         "attn_window_fused")
 
 # Every symbol declared in include/ptdit.h.
 EXPORTS = (
@@ -35,7 +36,7 @@ EXPORTS = (
     "ptdit_debug_wait_limit", "ptdit_window_attn_bwd", "ptdit_window_attn_bwd_workspace_bytes",
     "ptdit_tcm_bwd", "ptdit_tcm_bwd_workspace_bytes", "ptdit_giim_bwd",
     "ptdit_giim_bwd_workspace_bytes", "ptdit_block_attn_bwd",
-    "ptdit_block_attn_bwd_workspace_bytes",
+    "ptdit_block_attn_bwd_workspace_bytes", "ptdit_window_fused",
 )
 
 
@@ -134,6 +135,7 @@ def lib() -> ctypes.CDLL:
             "ptdit_device_status": (ctypes.c_int, [ctypes.c_int]),
             "ptdit_debug_timeout": (ctypes.c_int, [ctypes.c_longlong, _P]),
             "ptdit_debug_wait_limit": (ctypes.c_int, [ctypes.c_longlong]),
+            "ptdit_window_fused": (ctypes.c_int, [ctypes.c_int]),
             "ptdit_timing_enable": (ctypes.c_int, [ctypes.c_int]),
             "ptdit_timing_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int),
                                                  ctypes.POINTER(ctypes.c_float), ctypes.c_int]),

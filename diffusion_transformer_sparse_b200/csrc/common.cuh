@@ -321,6 +321,32 @@ cudaError_t launch_center_to_bf16(const float *src, int B, int M, int cols, void
 cudaError_t launch_to_bf16(const float *src, long rows, int cols, void *dst, long ldd,
                            cudaStream_t s);
 
+// Fused window Q/K/V projection + window attention (windows of 128 tokens):
+// win_fused_plan fills the geometry (sub-boxes a rolled window is loaded as) or
+// returns false for shapes it does not take; launch_repack_qkv writes the heads'
+// [Wq_h; Wk_h; Wv_h] rows (N per head) into win_fused_weight_bytes(p) bytes;
+// launch_win_fused writes the attention output, [B N, D] row-major with row
+// stride p.ldo, for the token grid z ([B, F, H, W, D]).
+struct WinFusedParams {
+    int B, F, H, W, D, heads, d, N;  // N: weight rows per head, 3 d rounded up to 16
+    int wt, wy, wx;                  // window
+    int st, sy, sx;                  // shift (roll by -shift)
+    int bt, by, bx;                  // sub-box of a window
+    int nb, R;                       // sub-boxes per window, rows per sub-box
+    int units;                       // B x windows (set by the launcher)
+    float scale;                     // 1/sqrt(d)
+    __nv_bfloat16 *o;
+    long ldo;
+    int *status;
+    unsigned long long wait_ns;
+};
+bool win_fused_plan(int D, int heads, int d, const int window[3], const int shift[3],
+                    WinFusedParams *p);
+size_t win_fused_weight_bytes(const WinFusedParams &p);
+cudaError_t launch_repack_qkv(const void *wq, const void *wk, const void *wv,
+                              const WinFusedParams &p, void *out, cudaStream_t s);
+cudaError_t launch_win_fused(const void *z, const void *wr, WinFusedParams p, cudaStream_t s);
+
 // Debug maps written with the kernels' own index functions.
 cudaError_t launch_debug_proxy_map(const ProxyGeom &g, int32_t *out, cudaStream_t s);
 cudaError_t launch_debug_window_map(const WinGeom &g, int32_t *tok, uint8_t *allowed,

@@ -116,6 +116,11 @@ bool fault(const char *kind) {
     return v && strcmp(v, kind) == 0;
 }
 
+// Whether this host thread's window branches may take the fused projection +
+// attention kernel (ptdit_window_fused).
+thread_local bool g_window_fused = false;
+bool fused_window_disabled() { return !g_window_fused; }
+
 int launch_fault(const char *what) {
     return fault("launch") ? fail(PTDIT_ERR_CUDA, "%s: launch refused (PTDIT_FAULT=launch)", what)
                            : PTDIT_OK;
@@ -223,6 +228,9 @@ struct Ws {
     size_t P, Qp, Kp, Vp, Ap, Pp, Kc, Vc, Q, K, V, O;
     size_t Xn, H, Kt, Vt;  // the complete block only: norm output, MLP hidden, text K and V
     size_t total;
+    // past total: the heads' repacked Q/K/V weight rows of the fused window kernel
+    // (a workspace of total_fused bytes lets windows of 128 tokens take it)
+    size_t Wr, total_fused;
 };
 
 // Whether the attention operands of this shape go through tiled head layout.
@@ -281,6 +289,12 @@ Ws ws_layout(const Dims &d, long M, long Lt = 0, long Dh = 0) {
         L.Vt = take(mx(tl, t ? thl_bytes(d, Lt, 1) : 0));
     }
     L.total = off;
+    L.Wr = off;
+    L.total_fused = off;
+    if (thl_shape(d) && d.D % 64 == 0) {  // the fused window kernel's weight rows
+        const size_t N = (size_t)(3 * d.d + 15) / 16 * 16;
+        L.total_fused += align256((size_t)d.heads * N * d.D * d.elem);
+    }
     return L;
 }
 
@@ -342,6 +356,7 @@ struct Run {
     cudaStream_t s;
     char *ws;
     const Ws &L;
+    size_t cap = 0;  // the caller's workspace bytes (0: only L.total known)
     char *at(size_t off) const { return ws + off; }
 };
 
@@ -603,14 +618,44 @@ int run_giim(const Run &r, const ProxyGeom &pg, const ptdit_attn_w *psa,
 
 // One TCM branch: x_out = (x_in +) WSA_or_SWSA(x_in), or, with a norm (the
 // complete block), x_out = x_in + WSA_or_SWSA(LN(x_in)).  x_out may equal x_in.
+// fused_ok = false: Q, K and V must come out in the workspace (a caller reuses them),
+// so the fused projection + attention kernel is not taken.
 int run_window(const Run &r, const WinGeom &wg, const ptdit_attn_w *w, unsigned flags,
-               const void *x_in, void *x_out, const ptdit_norm_w *nw = nullptr, float eps = 0.f) {
+               const void *x_in, void *x_out, const ptdit_norm_w *nw = nullptr, float eps = 0.f,
+               bool fused_ok = true) {
     const Dims &d = r.d;
     const long BN = (long)d.B * d.N;
     const void *xa = x_in;
     if (nw) {
         TRY(layer_norm(r, nw, eps, x_in, BN, r.at(r.L.Xn), "window norm"));
         xa = r.at(r.L.Xn);
+    }
+    // windows of 128 tokens in bf16, given the workspace for the heads' repacked weight
+    // rows: the projection and the attention in one kernel
+    WinFusedParams fp;
+    const int win3[3] = {wg.wf, wg.wh, wg.ww}, sh3[3] = {wg.sf, wg.sh, wg.sw};
+    if (fused_ok && d.dtype == PTDIT_BF16 && !fused_window_disabled() &&
+        win_fused_plan(d.D, d.heads, d.d, win3, sh3, &fp) && r.cap >= r.L.total_fused &&
+        r.L.Wr + win_fused_weight_bytes(fp) <= r.L.total_fused) {
+        void *wr = r.at(r.L.Wr);
+        TRY(launch_fault("weight repack"));
+        cudaError_t e = launch_repack_qkv(w->wq, w->wk, w->wv, fp, wr, r.s);
+        count_launch();
+        if (e != cudaSuccess) return cuda_fail(e, "weight repack");
+        fp.B = d.B; fp.F = d.f; fp.H = d.h; fp.W = d.w;
+        fp.scale = 1.0f / sqrtf((float)d.d);
+        fp.o = reinterpret_cast<__nv_bfloat16 *>(r.at(r.L.O));
+        fp.ldo = d.D;
+        TRY(launch_fault("fused window attention"));
+        timing_begin(PTDIT_K_ATTN_WINDOW_FUSED, r.s);
+        e = launch_win_fused(xa, wr, fp, r.s);
+        timing_end(r.s);
+        count_launch();
+        if (e != cudaSuccess) return cuda_fail(e, "fused window projection + attention");
+        const void *W[3] = {w->wo, nullptr, nullptr};
+        void *C[3] = {x_out, nullptr, nullptr};
+        const void *R[3] = {(flags & PTDIT_NO_RESIDUAL) ? nullptr : x_in, nullptr, nullptr};
+        return gemm(r, PTDIT_K_GEMM, r.at(r.L.O), BN, 1, W, C, R, "window output projection");
     }
     AttnArgs a;
     memset(&a, 0, sizeof a);
@@ -884,7 +929,7 @@ int run_tcm_bwd(const Dims &d, cudaStream_t s, char *ws, const WinGeom &wg0, con
     Lf.Q = T.wq; Lf.K = T.wk; Lf.V = T.wv; Lf.O = T.wa;
     Run rf{d, s, ws, Lf};
     void *zh = rf.at(T.zh), *dzh = rf.at(T.dzh);
-    TRY(run_window(rf, wg0, wsa, flags, z_in, zh));
+    TRY(run_window(rf, wg0, wsa, flags, z_in, zh, nullptr, 0.f, false));
     const Ws none{};
     Run r{d, s, ws, none};
     TRY(run_window_bwd(r, T.bwd, wg1, swsa, flags, zh, dz_out, dzh, dw_swsa));
@@ -1316,6 +1361,7 @@ size_t ptdit_workspace_bytes(const ptdit_shape *shape, const int ratio[3], const
         const int zero[3] = {0, 0, 0};
         WinGeom wg;
         if (make_window(d, window, zero, &wg) != PTDIT_OK) return 0;
+        if (wg.n == 128) return ws_layout(d, M).total_fused;
     }
     return ws_layout(d, M).total;
 }
@@ -1372,6 +1418,7 @@ int ptdit_giim_ex(const ptdit_shape *shape, const int ratio[3], int mode, const 
     TRY(check_w_alias(d, cross, z_out));
     TRY(check_ws(d, pg.M, ws, ws_bytes, &L));
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    r.cap = ws_bytes;
     return run_giim(r, pg, psa, cross, flags, z_in, z_out, mode, slots);
 }
 
@@ -1391,6 +1438,7 @@ int ptdit_giim(const ptdit_shape *shape, const int ratio[3], const ptdit_attn_w 
     TRY(check_w_alias(d, cross, z_out));
     TRY(check_ws(d, pg.M, ws, ws_bytes, &L));
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    r.cap = ws_bytes;
     return run_giim(r, pg, psa, cross, flags, z_in, z_out);
 }
 
@@ -1408,6 +1456,7 @@ int ptdit_window_attn(const ptdit_shape *shape, const int window[3], const int s
     TRY(check_w_alias(d, w, z_out));
     TRY(check_ws(d, 0, ws, ws_bytes, &L));
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    r.cap = ws_bytes;
     return run_window(r, wg, w, flags, z_in, z_out);
 }
 
@@ -1543,6 +1592,7 @@ int ptdit_tcm(const ptdit_shape *shape, const int window[3], const int shift[3],
     TRY(check_w_alias(d, swsa, z_out));
     TRY(check_ws(d, 0, ws, ws_bytes, &L));
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    r.cap = ws_bytes;
     TRY(run_window(r, wg0, wsa, flags, z_in, z_out));
     return run_window(r, wg1, swsa, flags, z_out, z_out);
 }
@@ -1573,6 +1623,7 @@ int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int win
     TRY(check_w_alias(d, swsa, z_out));
     TRY(check_ws(d, pg.M, ws, ws_bytes, &L));
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    r.cap = ws_bytes;
     TRY(run_giim(r, pg, psa, cross, flags, z_in, z_out));
     TRY(run_window(r, wg0, wsa, flags, z_out, z_out));
     return run_window(r, wg1, swsa, flags, z_out, z_out);
@@ -1593,6 +1644,12 @@ BlockBwd block_bwd_layout(const Dims &d, long M) {
     L.tcm = L.giim + ws_layout_giim_bwd(d, M).total;
     L.total = L.tcm + tcm_bwd_layout(d).total;
     return L;
+}
+
+int ptdit_window_fused(int enable) {
+    const int prev = g_window_fused ? 1 : 0;
+    if (enable == 0 || enable == 1) g_window_fused = enable == 1;
+    return prev;
 }
 
 size_t ptdit_block_attn_bwd_workspace_bytes(const ptdit_shape *shape, const int ratio[3],
@@ -1666,7 +1723,7 @@ size_t ptdit_pt_block_workspace_bytes(const ptdit_shape *shape, const int ratio[
     ProxyGeom pg;
     if (check_shape(shape, &d) != PTDIT_OK || text_len < 1 || mlp_hidden < 1) return 0;
     if (make_proxy(d, ratio, &pg) != PTDIT_OK) return 0;
-    return ws_layout(d, pg.M, text_len, mlp_hidden).total;
+    return ws_layout(d, pg.M, text_len, mlp_hidden).total_fused;
 }
 
 int ptdit_pt_block(const ptdit_shape *shape, const int ratio[3], const int window[3],
@@ -1723,6 +1780,7 @@ int ptdit_pt_block(const ptdit_shape *shape, const int ratio[3], const int windo
     if (ws && overlap(ws, ws_bytes, text, (size_t)d.B * text_len * d.D * d.elem))
         return fail(PTDIT_ERR_ALIAS, "the text tokens overlap the workspace");
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    r.cap = ws_bytes;
     const NormSet nm{norms[0], norms[1], norms[2], norms[3], norms[4], norms[5], w->eps};
     TRY(run_giim(r, pg, &w->psa, &w->cross, 0, z_in, z_out, proxy_mode, slots, &nm));
     TRY(run_window(r, wg0, &w->wsa, 0, z_out, z_out, nm.wsa, nm.eps));
@@ -1743,6 +1801,7 @@ int ptdit_full_attn(const ptdit_shape *shape, const ptdit_attn_w *w, unsigned fl
     TRY(check_w_alias(d, w, z_out));
     TRY(check_ws(d, 0, ws, ws_bytes, &L));
     Run r{d, (cudaStream_t)stream, static_cast<char *>(ws), L};
+    r.cap = ws_bytes;
     const long BN = (long)d.B * d.N;
     AttnArgs a;
     memset(&a, 0, sizeof a);

@@ -92,6 +92,22 @@ bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows
     return r == CUDA_SUCCESS;
 }
 
+bool encode_map_grid_bf16(CUtensorMap *map, const void *base, int B, int F, int H, int W, int D,
+                          uint32_t box_c, uint32_t box_x, uint32_t box_y, uint32_t box_t) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t e = 2;
+    cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)F, (cuuint64_t)B};
+    cuuint64_t strides[4] = {(cuuint64_t)D * e, (cuuint64_t)W * D * e, (cuuint64_t)H * W * D * e,
+                             (cuuint64_t)F * H * W * D * e};
+    cuuint32_t box[5] = {box_c, box_x, box_y, box_t, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 thread_local unsigned long long g_wait_limit_ns = 0;
 }

@@ -165,6 +165,16 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
+        "r"(c3), "r"(c4)
+        : "memory");
+}
+
 // Contiguous copy global -> shared of `bytes` (a multiple of 16; both
 // addresses 16-byte aligned), completing on `bar` (no multicast).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
@@ -475,6 +485,12 @@ bool encode_map_rows_heads_bf16(CUtensorMap *map, const void *base, uint64_t row
 bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows,
                                uint64_t row_pitch_bytes, int heads, int d, uint32_t box_elems,
                                uint32_t box_rows, int swizzle_bytes);
+
+// Host: a 5-D map over a [B, F, H, W, D] bf16 token grid, dims (D, W, H, F, B), with the
+// 128-byte swizzle; box (box_c channels, box_x, box_y, box_t tokens, 1 item): a box of
+// tokens lands as box_x * box_y * box_t rows of box_c channels, x fastest.
+bool encode_map_grid_bf16(CUtensorMap *map, const void *base, int B, int F, int H, int W, int D,
+                          uint32_t box_c, uint32_t box_x, uint32_t box_y, uint32_t box_t);
 
 int num_sms();
 

@@ -127,7 +127,11 @@ int ptdit_proxy_extract(const ptdit_shape *shape, const int ratio[3], int mode,
  * ptdit_workspace_bytes -- device scratch that every call below needs for
  * this shape (the maximum over them), or 0 for an invalid shape.  The
  * workspace must be 256-byte aligned; its contents need no initialisation
- * and are garbage after a call.
+ * and are garbage after a call.  For a window of 128 tokens in bf16 the size
+ * includes the heads' repacked Q/K/V weight rows (3 d rounded up to 16 rows of
+ * D per head) that the fused projection + window-attention kernel reads
+ * (ptdit_window_fused); a smaller workspace that holds everything else is
+ * accepted and runs the two-kernel form.
  */
 size_t ptdit_workspace_bytes(const ptdit_shape *shape, const int ratio[3], const int window[3]);
 
@@ -431,7 +435,8 @@ enum {
     PTDIT_K_WGRAD = 9,     /* weight gradients of the projections */
     PTDIT_K_TRANSPOSE = 10,/* weight transposes of the backward */
     PTDIT_K_ATTN_ROWS_BWD = 11, /* cross / proxy attention core, backward */
-    PTDIT_K_COUNT = 12
+    PTDIT_K_ATTN_WINDOW_FUSED = 12, /* window Q/K/V projection + window attention, fused */
+    PTDIT_K_COUNT = 13
 };
 int ptdit_timing_enable(int max_launches);
 int ptdit_timing_read(int *kind, float *ms, int max);
@@ -459,6 +464,22 @@ int ptdit_device_status(int reset);
  *   PTDIT_ERR_CUDA.
  */
 int ptdit_debug_timeout(long long limit_ns, ptdit_stream_t stream);
+
+/*
+ * ptdit_window_fused -- selects, for this host thread's later calls, how a TCM
+ *   branch with windows of 128 tokens runs in bf16 (Qihoo-T2X reading note, §3
+ *   Method, Eq. TCM): enable = 1 takes one kernel per branch for the window Q/K/V
+ *   projection and the window attention (Q, K and V stay on chip; the heads'
+ *   weight rows are repacked into the workspace first), 0 (the default) the
+ *   projection kernel then the window-attention kernel (Q, K and V through the
+ *   workspace), which is the faster form on B200: the fused kernel streams a
+ *   head's weight rows for every window.  Both give the same result up to
+ *   rounding order.  Other window
+ *   sizes, fp32, and the forward that ptdit_tcm_bwd recomputes (whose Q, K and V
+ *   its backward reuses) always take the second form.  Any other value of enable
+ *   only reads the setting.  Returns the previous setting (0 or 1).
+ */
+int ptdit_window_fused(int enable);
 
 /*
  * ptdit_debug_wait_limit -- sets, for this host thread's later launches of

@@ -83,6 +83,16 @@ def test_workspace_bytes(L):
     assert _bytes(L, _shape(D=63, heads=2), None, None) == 0
 
 
+def test_workspace_bytes_with_128_token_windows(L):
+    """Windows of 128 tokens in bf16: the size adds the fused kernel's repacked weight
+    rows, 16 heads x 224 rows (3 x 72 rounded up to 16) x 1152 columns."""
+    s = _shape(B=1, F=2, H=16, W=16, D=1152, heads=16, dtype=pt.PTDIT_BF16)
+    plain = _bytes(L, s, None, (1, 8, 8))
+    assert _bytes(L, s, None, (2, 8, 8)) == plain + 16 * 224 * 1152 * 2
+    f = _shape(B=1, F=2, H=16, W=16, D=1152, heads=16, dtype=pt.PTDIT_F32)
+    assert _bytes(L, f, None, (2, 8, 8)) == _bytes(L, f, None, (1, 8, 8))
+
+
 FAKE = 1 << 20  # an aligned non-null address that is never dereferenced: validation fails first
 
 
