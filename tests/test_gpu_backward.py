@@ -196,6 +196,8 @@ def test_giim_bwd_full_size_1024px():
     ((2, 16, 32), 1152, 16, (1, 2, 2), (2, 8, 8), (1, 4, 4), 1),
     # t2i 1024 px (two of its four items): 64 x 64 latents, 256 proxies, 8 x 8 windows
     ((1, 64, 64), 1152, 16, (1, 4, 4), (1, 8, 8), (0, 4, 4), 2),
+    # t2v in full: 16 x 32 x 48 latents, 1536 proxies (12 key tiles summed), 3D windows
+    ((16, 32, 48), 1152, 16, (1, 4, 4), (2, 8, 8), (1, 4, 4), 1),
 ])
 def test_block_attn_bwd(grid, D, heads, ratio, window, shift, B):
     """GIIM then TCM: dL/dz and the four modules' weight gradients."""
