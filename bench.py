@@ -638,7 +638,7 @@ def run_block(args, w, L=120):
     return 0
 
 
-def run_bwd(args, w, branch=False):
+def run_bwd(args, w, branch=False, train=False):
     """Backward of the block-attention path (ptdit_block_attn_bwd: GIIM recomputed, TCM's
     backward, GIIM's backward), or with branch=True of the shifted-window TCM branch
     alone (ptdit_window_attn_bwd): dL/dz and the weight gradients for a synthetic
@@ -660,6 +660,9 @@ def run_bwd(args, w, branch=False):
           for _ in range(nmod)]
     if branch:
         ws = pt.window_attn_bwd_workspace(shape, w.window)
+    elif train:
+        ws = pt.train_workspace(z, w.grid, w.ratio, w.window, w.heads)
+        zout = torch.empty_like(z)
     else:
         n = pt.lib().ptdit_block_attn_bwd_workspace_bytes(ctypes.byref(shape), pt._i3(w.ratio),
                                                          pt._i3(w.window))
@@ -674,6 +677,18 @@ def run_bwd(args, w, branch=False):
         if branch:
             pt.ptdit_window_attn_bwd(z, dout, w.grid, w.window, w.shift, W["swsa"], w.heads,
                                      dz_in=dz, dw=dw[0], ws=ws, stream=stream)
+            return
+        if train:
+            args3 = (ctypes.byref(shape), pt._i3(w.ratio), pt._i3(w.window), pt._i3(w.shift),
+                     *[ctypes.byref(x) for x in wa], 0, z.data_ptr())
+            rc = pt.lib().ptdit_block_attn_fwd_train(*args3, zout.data_ptr(), ws.data_ptr(),
+                                                     ws.numel(), stream.cuda_stream)
+            if rc == 0:
+                rc = pt.lib().ptdit_block_attn_bwd_saved(
+                    *args3, dout.data_ptr(), dz.data_ptr(), *[ctypes.byref(x) for x in wg],
+                    ws.data_ptr(), ws.numel(), stream.cuda_stream)
+            if rc != 0:
+                raise pt.PtditError(rc, pt.lib().ptdit_last_error().decode())
             return
         rc = pt.lib().ptdit_block_attn_bwd(
             ctypes.byref(shape), pt._i3(w.ratio), pt._i3(w.window), pt._i3(w.shift),
@@ -711,6 +726,12 @@ def run_bwd(args, w, branch=False):
         f = flops.window_bwd_flops(w.N, w.n, w.D)
         metric, mode = "backward of one TCM branch, tokens/s", "window_bwd"
         cores = {"attn_window_bwd": w.B * f["core_bwd"]}
+    elif train:
+        f = flops.train_step_flops(w.N, w.M, w.n, w.D)
+        metric = "training step of the block-attention path (forward keeping its activations, then backward), tokens/s"
+        mode = "train_step"
+        cores = {"attn_window_bwd": w.B * f["window_core_bwd"],
+                 "attn_rows_bwd": w.B * f["rows_core_bwd"]}
     else:
         f = flops.block_bwd_flops(w.N, w.M, w.n, w.D)
         metric, mode = "backward of the block-attention path (GIIM + TCM), tokens/s", "block_bwd"
@@ -754,6 +775,9 @@ def main(argv=None):
                          "(ptdit_window_fused(1)) for windows of 128 tokens")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward of the block-attention path instead")
+    ap.add_argument("--train", action="store_true",
+                    help="time a training step of the block-attention path: the forward that "
+                         "keeps its activations, then the backward from them")
     ap.add_argument("--bwd-branch", action="store_true",
                     help="time the backward of the shifted-window TCM branch alone instead")
     ap.add_argument("--block", action="store_true",
@@ -769,8 +793,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.dense:
         return run_dense(args, w)
-    if args.bwd or args.bwd_branch:
-        return run_bwd(args, w, branch=args.bwd_branch)
+    if args.bwd or args.bwd_branch or args.train:
+        return run_bwd(args, w, branch=args.bwd_branch, train=args.train)
     if args.block:
         return run_block(args, w)
     return run_gpu(args, w)

@@ -37,6 +37,8 @@ EXPORTS = (
     "ptdit_tcm_bwd", "ptdit_tcm_bwd_workspace_bytes", "ptdit_giim_bwd",
     "ptdit_giim_bwd_workspace_bytes", "ptdit_block_attn_bwd",
     "ptdit_block_attn_bwd_workspace_bytes", "ptdit_window_fused",
+    "ptdit_block_attn_train_workspace_bytes", "ptdit_block_attn_fwd_train",
+    "ptdit_block_attn_bwd_saved",
 )
 
 
@@ -111,6 +113,14 @@ def lib() -> ctypes.CDLL:
             "ptdit_tcm_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
             "ptdit_giim_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3]),
             "ptdit_block_attn_bwd_workspace_bytes": (ctypes.c_size_t, [_S, _I3, _I3]),
+            "ptdit_block_attn_train_workspace_bytes": (ctypes.c_size_t, [_S, _I3, _I3]),
+            "ptdit_block_attn_fwd_train": (ctypes.c_int, [_S, _I3, _I3, _I3, _W, _W, _W, _W,
+                                                          ctypes.c_uint, _P, _P, _P,
+                                                          ctypes.c_size_t, _P]),
+            "ptdit_block_attn_bwd_saved": (ctypes.c_int, [_S, _I3, _I3, _I3, _W, _W, _W, _W,
+                                                          ctypes.c_uint, _P, _P, _P]
+                                           + [ctypes.POINTER(AttnWgrad)] * 4
+                                           + [_P, ctypes.c_size_t, _P]),
             "ptdit_block_attn_bwd": (ctypes.c_int, [_S, _I3, _I3, _I3, _W, _W, _W, _W,
                                                     ctypes.c_uint, _P, _P, _P]
                                      + [ctypes.POINTER(AttnWgrad)] * 4
@@ -465,6 +475,56 @@ def ptdit_block_attn_bwd(z_in, dz_out, grid, ratio, window, shift, psa, cross, w
                                       *[ctypes.byref(x) for x in w], flags, _ptr(z_in),
                                       _ptr(dz_out), _ptr(dz_in), *[ctypes.byref(x) for x in g],
                                       _ptr(ws), ws.numel(), _stream(stream)))
+    return (dz_in, *dws)
+
+
+def train_workspace(z_in, grid, ratio, window, heads):
+    """A uint8 device buffer of ptdit_block_attn_train_workspace_bytes()."""
+    import torch
+    shape = make_shape(z_in, grid, heads)
+    n = lib().ptdit_block_attn_train_workspace_bytes(ctypes.byref(shape), _i3(ratio), _i3(window))
+    if n == 0:
+        raise PtditError(PTDIT_ERR_SHAPE, "invalid shape, ratio or window")
+    return torch.empty(n, dtype=torch.uint8, device=z_in.device)
+
+
+def ptdit_block_attn_fwd_train(z_in, grid, ratio, window, shift, psa, cross, wsa, swsa, heads, ws,
+                               flags=0, z_out=None, stream=None):
+    """The block-attention forward that keeps its activations in ws (train_workspace) for
+    ptdit_block_attn_bwd_saved; returns z_out."""
+    import torch
+    _check_z(z_in)
+    shape = make_shape(z_in, grid, heads)
+    if z_out is None:
+        z_out = torch.empty_like(z_in)
+    w = [attn_w(x) for x in (psa, cross, wsa, swsa)]
+    _check(lib().ptdit_block_attn_fwd_train(ctypes.byref(shape), _i3(ratio), _i3(window),
+                                            _i3(shift), *[ctypes.byref(x) for x in w], flags,
+                                            _ptr(z_in), _ptr(z_out), _ptr(ws), ws.numel(),
+                                            _stream(stream)))
+    return z_out
+
+
+def ptdit_block_attn_bwd_saved(z_in, dz_out, grid, ratio, window, shift, psa, cross, wsa, swsa,
+                               heads, ws, flags=0, dz_in=None, stream=None):
+    """The block-attention backward from the activations ptdit_block_attn_fwd_train kept in
+    ws: returns (dz_in, dW_psa, dW_cross, dW_wsa, dW_swsa), each dW four fp32 [D, D]."""
+    import torch
+    _check_z(z_in)
+    _check_z(dz_out)
+    shape = make_shape(z_in, grid, heads)
+    if dz_in is None:
+        dz_in = torch.empty_like(z_in)
+    D = z_in.shape[-1]
+    dws = [tuple(torch.empty(D, D, dtype=torch.float32, device=z_in.device) for _ in range(4))
+           for _ in range(4)]
+    w = [attn_w(x) for x in (psa, cross, wsa, swsa)]
+    g = [AttnWgrad(*[_ptr(x) for x in dw]) for dw in dws]
+    _check(lib().ptdit_block_attn_bwd_saved(ctypes.byref(shape), _i3(ratio), _i3(window),
+                                            _i3(shift), *[ctypes.byref(x) for x in w], flags,
+                                            _ptr(z_in), _ptr(dz_out), _ptr(dz_in),
+                                            *[ctypes.byref(x) for x in g], _ptr(ws), ws.numel(),
+                                            _stream(stream)))
     return (dz_in, *dws)
 
 

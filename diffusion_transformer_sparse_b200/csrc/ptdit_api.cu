@@ -1272,6 +1272,81 @@ int run_giim_bwd(const Run &r, const WsGB &Lb, const ProxyGeom &pg, const ptdit_
     return giim_backward(r, Lb, pg, psa, cross, flags, z_in, dz_out, dz_in, dwp, dwc);
 }
 
+// ------------------------------------------------------------------ backward of the path
+// z1 and dL/dz1, GIIM's backward area (its recomputed forward stays there while TCM's
+// backward runs), then TCM's backward area.
+struct BlockBwd {
+    size_t z1, dz1, giim, tcm, total;
+};
+BlockBwd block_bwd_layout(const Dims &d, long M) {
+    BlockBwd L;
+    const size_t tn = align256((size_t)d.B * d.N * d.D * d.elem);
+    L.z1 = 0;
+    L.dz1 = tn;
+    L.giim = 2 * tn;
+    L.tcm = L.giim + ws_layout_giim_bwd(d, M).total;
+    L.total = L.tcm + tcm_bwd_layout(d).total;
+    return L;
+}
+
+// The block path's geometry for the backward entry points: shape, proxies, both
+// windows, the backward's restrictions.
+int path_geometry(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                  const int shift[3], Dims *d, ProxyGeom *pg, WinGeom *wg0, WinGeom *wg1) {
+    const int zero[3] = {0, 0, 0};
+    TRY(check_shape(shape, d));
+    TRY(make_proxy(*d, ratio, pg));
+    TRY(make_window(*d, window, shift, wg1));
+    TRY(make_window(*d, window, zero, wg0));
+    TRY(check_bwd_shape(*d, *wg0));
+    if ((pg->M + kThlRows - 1) / kThlRows > 64)
+        return fail(PTDIT_ERR_SHAPE, "the backward takes at most 8192 proxies; M=%d", pg->M);
+    return PTDIT_OK;
+}
+
+// The four modules' weights and weight gradients against each other and the I/O.
+int check_path_grads(const Dims &d, const ptdit_attn_w *const *W, const ptdit_attn_wgrad *const *G,
+                     const void *z_in, const void *dz_out, const void *dz_in, const void *ws,
+                     size_t ws_bytes) {
+    const char *wn[4] = {"psa", "cross", "wsa", "swsa"};
+    const char *gn[4] = {"dw_psa", "dw_cross", "dw_wsa", "dw_swsa"};
+    for (int m = 0; m < 4; ++m) {
+        TRY(check_weights(W[m], wn[m]));
+        TRY(check_bwd_io(d, W[m], z_in, dz_out, const_cast<void *>(dz_in), ws, ws_bytes));
+    }
+    for (int m = 0; m < 4; ++m) TRY(check_wgrad(d, G[m], gn[m], z_in, dz_out, dz_in, ws, ws_bytes));
+    const size_t gb = (size_t)d.D * d.D * sizeof(float);
+    for (int m = 0; m < 4; ++m)
+        for (int n = 0; n < m; ++n) {
+            const float *a[4] = {G[m]->dwq, G[m]->dwk, G[m]->dwv, G[m]->dwo};
+            const float *b[4] = {G[n]->dwq, G[n]->dwk, G[n]->dwv, G[n]->dwo};
+            for (int i = 0; i < 4; ++i)
+                for (int j = 0; j < 4; ++j)
+                    if (overlap(a[i], gb, b[j], gb))
+                        return fail(PTDIT_ERR_ALIAS, "%s and %s overlap", gn[m], gn[n]);
+        }
+    return PTDIT_OK;
+}
+
+// The training pair's workspace: the whole-path backward's areas (z1, dL/dz1, GIIM's
+// area, TCM's area with z^ and WSA's kept forward), then SWSA's kept Q, K, V window
+// tiles and attention output.
+struct TrainLayout {
+    BlockBwd b;
+    size_t sq, sk, sv, sa, total;
+};
+TrainLayout train_layout(const Dims &d, long M) {
+    TrainLayout T;
+    T.b = block_bwd_layout(d, M);
+    const size_t tq = align256(thl_bytes(d, d.N, 0));
+    T.sq = T.b.total;
+    T.sk = T.sq + tq;
+    T.sv = T.sk + tq;
+    T.sa = T.sv + tq;
+    T.total = T.sa + align256((size_t)d.B * d.N * d.D * d.elem);
+    return T;
+}
+
 }  // namespace
 
 namespace ptdit {
@@ -1629,23 +1704,6 @@ int ptdit_block_attn(const ptdit_shape *shape, const int ratio[3], const int win
     return run_window(r, wg1, swsa, flags, z_out, z_out);
 }
 
-// ------------------------------------------------------------------ backward of the path
-// z1 and dL/dz1, GIIM's backward area (its recomputed forward stays there while TCM's
-// backward runs), then TCM's backward area.
-struct BlockBwd {
-    size_t z1, dz1, giim, tcm, total;
-};
-BlockBwd block_bwd_layout(const Dims &d, long M) {
-    BlockBwd L;
-    const size_t tn = align256((size_t)d.B * d.N * d.D * d.elem);
-    L.z1 = 0;
-    L.dz1 = tn;
-    L.giim = 2 * tn;
-    L.tcm = L.giim + ws_layout_giim_bwd(d, M).total;
-    L.total = L.tcm + tcm_bwd_layout(d).total;
-    return L;
-}
-
 int ptdit_window_fused(int enable) {
     const int prev = g_window_fused ? 1 : 0;
     if (enable == 0 || enable == 1) g_window_fused = enable == 1;
@@ -1674,35 +1732,10 @@ int ptdit_block_attn_bwd(const ptdit_shape *shape, const int ratio[3], const int
     Dims d;
     ProxyGeom pg;
     WinGeom wg0, wg1;
-    const int zero[3] = {0, 0, 0};
-    TRY(check_shape(shape, &d));
-    TRY(make_proxy(d, ratio, &pg));
-    TRY(make_window(d, window, shift, &wg1));
-    TRY(make_window(d, window, zero, &wg0));
-    TRY(check_bwd_shape(d, wg0));
-    if ((pg.M + kThlRows - 1) / kThlRows > 64)
-        return fail(PTDIT_ERR_SHAPE, "the backward takes at most 8192 proxies; M=%d", pg.M);
+    TRY(path_geometry(shape, ratio, window, shift, &d, &pg, &wg0, &wg1));
     const ptdit_attn_w *W[4] = {psa, cross, wsa, swsa};
     const ptdit_attn_wgrad *G[4] = {dw_psa, dw_cross, dw_wsa, dw_swsa};
-    const char *wn[4] = {"psa", "cross", "wsa", "swsa"};
-    const char *gn[4] = {"dw_psa", "dw_cross", "dw_wsa", "dw_swsa"};
-    for (int m = 0; m < 4; ++m) {
-        TRY(check_weights(W[m], wn[m]));
-        TRY(check_bwd_io(d, W[m], z_in, dz_out, dz_in, ws, ws_bytes));
-    }
-    for (int m = 0; m < 4; ++m) TRY(check_wgrad(d, G[m], gn[m], z_in, dz_out, dz_in, ws, ws_bytes));
-    {
-        const size_t gb = (size_t)d.D * d.D * sizeof(float);
-        for (int m = 0; m < 4; ++m)
-            for (int n = 0; n < m; ++n) {
-                const float *a[4] = {G[m]->dwq, G[m]->dwk, G[m]->dwv, G[m]->dwo};
-                const float *b[4] = {G[n]->dwq, G[n]->dwk, G[n]->dwv, G[n]->dwo};
-                for (int i = 0; i < 4; ++i)
-                    for (int j = 0; j < 4; ++j)
-                        if (overlap(a[i], gb, b[j], gb))
-                            return fail(PTDIT_ERR_ALIAS, "%s and %s overlap", gn[m], gn[n]);
-            }
-    }
+    TRY(check_path_grads(d, W, G, z_in, dz_out, dz_in, ws, ws_bytes));
     const BlockBwd L = block_bwd_layout(d, pg.M);
     TRY(check_bwd_ws(ws, ws_bytes, L.total));
     const cudaStream_t s = (cudaStream_t)stream;
@@ -1714,6 +1747,88 @@ int ptdit_block_attn_bwd(const ptdit_shape *shape, const int ratio[3], const int
     TRY(giim_recompute(rg, Lg, pg, psa, cross, flags, z_in, z1));
     TRY(run_tcm_bwd(d, s, base + L.tcm, wg0, wg1, wsa, swsa, flags, z1, dz_out, dz1, dw_wsa,
                     dw_swsa));
+    return giim_backward(rg, Lg, pg, psa, cross, flags, z_in, dz1, dz_in, dw_psa, dw_cross);
+}
+
+size_t ptdit_block_attn_train_workspace_bytes(const ptdit_shape *shape, const int ratio[3],
+                                              const int window[3]) {
+    Dims d;
+    ProxyGeom pg;
+    WinGeom wg;
+    const int zero[3] = {0, 0, 0};
+    if (check_shape(shape, &d) != PTDIT_OK || make_proxy(d, ratio, &pg) != PTDIT_OK ||
+        make_window(d, window, zero, &wg) != PTDIT_OK)
+        return 0;
+    return train_layout(d, pg.M).total;
+}
+
+int ptdit_block_attn_fwd_train(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                               const int shift[3], const ptdit_attn_w *psa,
+                               const ptdit_attn_w *cross, const ptdit_attn_w *wsa,
+                               const ptdit_attn_w *swsa, unsigned flags, const void *z_in,
+                               void *z_out, void *ws, size_t ws_bytes, ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    WinGeom wg0, wg1;
+    TRY(path_geometry(shape, ratio, window, shift, &d, &pg, &wg0, &wg1));
+    const ptdit_attn_w *W[4] = {psa, cross, wsa, swsa};
+    const char *wn[4] = {"psa", "cross", "wsa", "swsa"};
+    for (int m = 0; m < 4; ++m) TRY(check_weights(W[m], wn[m]));
+    TRY(check_io(d, z_in, z_out, ws, ws_bytes));
+    for (int m = 0; m < 4; ++m) TRY(check_w_alias(d, W[m], z_out));
+    const TrainLayout T = train_layout(d, pg.M);
+    TRY(check_bwd_ws(ws, ws_bytes, T.total));
+    const cudaStream_t s = (cudaStream_t)stream;
+    char *base = static_cast<char *>(ws), *tcm = base + T.b.tcm;
+    const Ws none{};
+    const WsGB Lg = ws_layout_giim_bwd(d, pg.M);
+    Run rg{d, s, base + T.b.giim, none};
+    void *z1 = base + T.b.z1;
+    TRY(giim_recompute(rg, Lg, pg, psa, cross, flags, z_in, z1));
+    const TcmBwd Tc = tcm_bwd_layout(d);
+    void *zh = tcm + Tc.zh;
+    Ws Lw{};  // WSA's Q, K, V and attention output stay where its backward reads them
+    Lw.Q = Tc.wq; Lw.K = Tc.wk; Lw.V = Tc.wv; Lw.O = Tc.wa;
+    Run rw{d, s, tcm, Lw};
+    TRY(run_window(rw, wg0, wsa, flags, z1, zh, nullptr, 0.f, false));
+    Ws Ls{};  // and SWSA's
+    Ls.Q = T.sq; Ls.K = T.sk; Ls.V = T.sv; Ls.O = T.sa;
+    Run rs{d, s, base, Ls};
+    return run_window(rs, wg1, swsa, flags, zh, z_out, nullptr, 0.f, false);
+}
+
+int ptdit_block_attn_bwd_saved(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                               const int shift[3], const ptdit_attn_w *psa,
+                               const ptdit_attn_w *cross, const ptdit_attn_w *wsa,
+                               const ptdit_attn_w *swsa, unsigned flags, const void *z_in,
+                               const void *dz_out, void *dz_in, const ptdit_attn_wgrad *dw_psa,
+                               const ptdit_attn_wgrad *dw_cross, const ptdit_attn_wgrad *dw_wsa,
+                               const ptdit_attn_wgrad *dw_swsa, void *ws, size_t ws_bytes,
+                               ptdit_stream_t stream) {
+    Dims d;
+    ProxyGeom pg;
+    WinGeom wg0, wg1;
+    TRY(path_geometry(shape, ratio, window, shift, &d, &pg, &wg0, &wg1));
+    const ptdit_attn_w *W[4] = {psa, cross, wsa, swsa};
+    const ptdit_attn_wgrad *G[4] = {dw_psa, dw_cross, dw_wsa, dw_swsa};
+    TRY(check_path_grads(d, W, G, z_in, dz_out, dz_in, ws, ws_bytes));
+    const TrainLayout T = train_layout(d, pg.M);
+    TRY(check_bwd_ws(ws, ws_bytes, T.total));
+    const cudaStream_t s = (cudaStream_t)stream;
+    char *base = static_cast<char *>(ws), *tcm = base + T.b.tcm;
+    void *z1 = base + T.b.z1, *dz1 = base + T.b.dz1;
+    const TcmBwd Tc = tcm_bwd_layout(d);
+    void *zh = tcm + Tc.zh, *dzh = tcm + Tc.dzh;
+    const Ws none{};
+    Run r{d, s, tcm, none};
+    WsBwd Ls = Tc.bwd;  // SWSA's kept forward, outside TCM's area
+    Ls.Q = T.sq - T.b.tcm; Ls.K = T.sk - T.b.tcm; Ls.V = T.sv - T.b.tcm; Ls.A = T.sa - T.b.tcm;
+    TRY(run_window_bwd(r, Ls, wg1, swsa, flags, zh, dz_out, dzh, dw_swsa, false));
+    WsBwd Lw = Tc.bwd;
+    Lw.Q = Tc.wq; Lw.K = Tc.wk; Lw.V = Tc.wv; Lw.A = Tc.wa;
+    TRY(run_window_bwd(r, Lw, wg0, wsa, flags, z1, dzh, dz1, dw_wsa, false));
+    const WsGB Lg = ws_layout_giim_bwd(d, pg.M);
+    Run rg{d, s, base + T.b.giim, none};
     return giim_backward(rg, Lg, pg, psa, cross, flags, z_in, dz1, dz_in, dw_psa, dw_cross);
 }
 

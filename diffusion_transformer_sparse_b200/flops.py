@@ -114,3 +114,22 @@ def block_bwd_flops(N: int, M: int, n: int, D: int) -> dict:
     f["window_core_bwd"] = 2 * w["core_bwd"]
     f["rows_core_bwd"] = g["rows_core_bwd"]
     return f
+
+
+def train_step_flops(N: int, M: int, n: int, D: int) -> dict:
+    """A training step of the block-attention path as ptdit_block_attn_fwd_train plus
+    ptdit_block_attn_bwd_saved run it, per batch item: the forward (block_flops) and the
+    backward without any recomputation (both window branches' and GIIM's backward
+    proper)."""
+    fwd = block_flops(N, M, n, D)
+    w = window_bwd_flops(N, n, D)
+    g = giim_bwd_flops(N, M, D)
+    f = {
+        "forward": fwd["total"],
+        "tcm_bwd": 2 * (w["total"] - w["recompute_proj"] - w["recompute_core"]),
+        "giim_bwd": g["total"] - g["recompute"],
+    }
+    f["total"] = sum(f.values())
+    f["window_core_bwd"] = 2 * w["core_bwd"]
+    f["rows_core_bwd"] = g["rows_core_bwd"]
+    return f

@@ -276,6 +276,35 @@ int ptdit_block_attn_bwd(const ptdit_shape *shape, const int ratio[3], const int
                          size_t ws_bytes, ptdit_stream_t stream);
 
 /*
+ * The training pair: ptdit_block_attn_fwd_train runs the block-attention path's
+ *   forward (z_out as ptdit_block_attn, up to rounding order) and keeps what the
+ *   backward reads in the workspace (GIIM's intermediates with each query row's
+ *   log-sum-exp, z1, z^, both window branches' Q, K, V window tiles and attention
+ *   outputs); ptdit_block_attn_bwd_saved then computes what ptdit_block_attn_bwd
+ *   computes without recomputing the forward.  The second call must get the same
+ *   shape, ratio, window, shift, weights, flags, z_in and workspace, with nothing
+ *   written to the workspace in between.  Workspace:
+ *   ptdit_block_attn_train_workspace_bytes(shape, ratio, window).  Restrictions
+ *   and errors: those of ptdit_block_attn_bwd (fwd_train checks z_out as
+ *   ptdit_block_attn does).
+ */
+size_t ptdit_block_attn_train_workspace_bytes(const ptdit_shape *shape, const int ratio[3],
+                                              const int window[3]);
+int ptdit_block_attn_fwd_train(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                               const int shift[3], const ptdit_attn_w *psa,
+                               const ptdit_attn_w *cross, const ptdit_attn_w *wsa,
+                               const ptdit_attn_w *swsa, unsigned flags, const void *z_in,
+                               void *z_out, void *ws, size_t ws_bytes, ptdit_stream_t stream);
+int ptdit_block_attn_bwd_saved(const ptdit_shape *shape, const int ratio[3], const int window[3],
+                               const int shift[3], const ptdit_attn_w *psa,
+                               const ptdit_attn_w *cross, const ptdit_attn_w *wsa,
+                               const ptdit_attn_w *swsa, unsigned flags, const void *z_in,
+                               const void *dz_out, void *dz_in, const ptdit_attn_wgrad *dw_psa,
+                               const ptdit_attn_wgrad *dw_cross, const ptdit_attn_wgrad *dw_wsa,
+                               const ptdit_attn_wgrad *dw_swsa, void *ws, size_t ws_bytes,
+                               ptdit_stream_t stream);
+
+/*
  * ptdit_tcm -- Eq. TCM: WSA with weights wsa, then SWSA with weights swsa
  *   and the given shift, each with its residual (unless PTDIT_NO_RESIDUAL).
  */

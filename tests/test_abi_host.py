@@ -378,3 +378,24 @@ def test_block_attn_bwd_rejects(L):
     clash = [g[0], g[1], g[2], _wg(FAKE * 40 + 0x200000)]  # dw_swsa.dwq is dw_psa.dwv
     assert call(grads=clash) == 8
     assert b"dw_swsa and dw_psa overlap" in L.ptdit_last_error()
+
+
+def test_training_pair_workspace_and_refusals(L):
+    """The training pair's workspace adds SWSA's kept Q, K, V tiles and attention output to
+    the whole-path backward's; both calls validate on the host first."""
+    s = _bshape(B=4, H=64, W=64, D=1152, heads=16)
+    b = L.ptdit_block_attn_bwd_workspace_bytes(ctypes.byref(s), pt._i3((1, 4, 4)), pt._i3((1, 8, 8)))
+    t = L.ptdit_block_attn_train_workspace_bytes(ctypes.byref(s), pt._i3((1, 4, 4)), pt._i3((1, 8, 8)))
+    tq = 4 * 32 * 16 * 20480  # window tiles of 72 columns padded to 80, 32 tiles per item
+    assert t == b + 3 * tq + 4 * 4096 * 1152 * 2
+    small = _bshape()
+    args = (ctypes.byref(small), pt._i3((1, 2, 2)), pt._i3((1, 8, 8)), pt._i3((0, 4, 4)),
+            *[ctypes.byref(_w(FAKE * (2 + i))) for i in range(4)], 0)
+    assert L.ptdit_block_attn_fwd_train(*args, FAKE * 20, FAKE * 21, FAKE * 128, 4096, None) == 4
+    assert L.ptdit_block_attn_fwd_train(*args, FAKE * 20, FAKE * 20, FAKE * 128, 1 << 40, None) == 8
+    g = [_wg(FAKE * (40 + 8 * i)) for i in range(4)]
+    assert L.ptdit_block_attn_bwd_saved(*args, FAKE * 20, FAKE * 21, FAKE * 22,
+                                        *[ctypes.byref(x) for x in g], FAKE * 128, 4096, None) == 4
+    f32 = _bshape(dtype=pt.PTDIT_F32)
+    assert L.ptdit_block_attn_fwd_train(ctypes.byref(f32), *args[1:], FAKE * 20, FAKE * 21,
+                                        FAKE * 128, 1 << 40, None) == 3

@@ -192,19 +192,8 @@ def test_giim_bwd_full_size_1024px():
 
 # ---------------------------------------------------------------- the whole path
 
-@pytest.mark.parametrize("grid,D,heads,ratio,window,shift,B", [
-    ((2, 16, 32), 1152, 16, (1, 2, 2), (2, 8, 8), (1, 4, 4), 1),
-    # t2i 1024 px (two of its four items): 64 x 64 latents, 256 proxies, 8 x 8 windows
-    ((1, 64, 64), 1152, 16, (1, 4, 4), (1, 8, 8), (0, 4, 4), 2),
-    # t2v in full: 16 x 32 x 48 latents, 1536 proxies (12 key tiles summed), 3D windows
-    ((16, 32, 48), 1152, 16, (1, 4, 4), (2, 8, 8), (1, 4, 4), 1),
-])
-def test_block_attn_bwd(grid, D, heads, ratio, window, shift, B):
-    """GIIM then TCM: dL/dz and the four modules' weight gradients."""
-    c = Case(B, grid, D, heads, "bf16")
-    dout_cpu = _dout(c.B, c.N, c.D)
-    dz, *dw = pt.ptdit_block_attn_bwd(c.z, dout_cpu.cuda(), c.grid, ratio, window, shift,
-                                      c.w["psa"], c.w["cross"], c.w["wsa"], c.w["swsa"], c.heads)
+def _check_path(c, ratio, window, shift, dout_cpu, dz, dw):
+    """dz and the four modules' weight gradients of the whole path against the oracle."""
     dz = c.out64(dz)
     g64 = synth.as_f64(dout_cpu)
     mods = ("psa", "cross", "wsa", "swsa")
@@ -223,3 +212,47 @@ def test_block_attn_bwd(grid, D, heads, ratio, window, shift, B):
         for i in range(4):
             tol = tol_qk if (name == "cross" and i < 2) else TOL["bf16"]
             assert rel_err(c.out64(dw[m][i]), want[m][i]) <= tol, (name, i, kappa)
+
+
+@pytest.mark.parametrize("grid,D,heads,ratio,window,shift,B", [
+    ((2, 16, 32), 1152, 16, (1, 2, 2), (2, 8, 8), (1, 4, 4), 1),
+    # t2i 1024 px (two of its four items): 64 x 64 latents, 256 proxies, 8 x 8 windows
+    ((1, 64, 64), 1152, 16, (1, 4, 4), (1, 8, 8), (0, 4, 4), 2),
+    # t2v in full: 16 x 32 x 48 latents, 1536 proxies (12 key tiles summed), 3D windows
+    ((16, 32, 48), 1152, 16, (1, 4, 4), (2, 8, 8), (1, 4, 4), 1),
+])
+def test_block_attn_bwd(grid, D, heads, ratio, window, shift, B):
+    """GIIM then TCM: dL/dz and the four modules' weight gradients."""
+    c = Case(B, grid, D, heads, "bf16")
+    dout_cpu = _dout(c.B, c.N, c.D)
+    dz, *dw = pt.ptdit_block_attn_bwd(c.z, dout_cpu.cuda(), c.grid, ratio, window, shift,
+                                      c.w["psa"], c.w["cross"], c.w["wsa"], c.w["swsa"], c.heads)
+    _check_path(c, ratio, window, shift, dout_cpu, dz, dw)
+
+
+@pytest.mark.parametrize("grid,D,heads,ratio,window,shift,B", [
+    ((2, 16, 32), 1152, 16, (1, 2, 2), (2, 8, 8), (1, 4, 4), 1),
+    ((1, 64, 64), 1152, 16, (1, 4, 4), (1, 8, 8), (0, 4, 4), 2),
+])
+def test_block_attn_train_pair(grid, D, heads, ratio, window, shift, B):
+    """The forward that keeps its activations, then the backward from them: the forward's
+    output and every gradient against the oracle, and the gradients against the backward
+    that recomputes the forward (same kernels; only the order of the fp32 reductions of
+    dK, dV and the weight gradients differs)."""
+    c = Case(B, grid, D, heads, "bf16")
+    mods = ("psa", "cross", "wsa", "swsa")
+    W = [c.w[m] for m in mods]
+    ws = pt.train_workspace(c.z, grid, ratio, window, heads)
+    out = c.out64(pt.ptdit_block_attn_fwd_train(c.z, grid, ratio, window, shift, *W, heads, ws))
+    for b in range(B):
+        want = O.block_attn(c.z64[b], grid, ratio, window, shift, *[c.w64[m] for m in mods], heads)
+        assert rel_err(out[b], want) <= TOL["bf16"], ("forward", b)
+    dout_cpu = _dout(c.B, c.N, c.D)
+    dz, *dw = pt.ptdit_block_attn_bwd_saved(c.z, dout_cpu.cuda(), grid, ratio, window, shift, *W,
+                                            heads, ws)
+    _check_path(c, ratio, window, shift, dout_cpu, dz, dw)
+    dz2, *dw2 = pt.ptdit_block_attn_bwd(c.z, dout_cpu.cuda(), grid, ratio, window, shift, *W, heads)
+    assert rel_err(c.out64(dz), c.out64(dz2)) <= 1e-2
+    for m in range(4):
+        for i in range(4):
+            assert rel_err(c.out64(dw[m][i]), c.out64(dw2[m][i])) <= 1e-2, (mods[m], i)
