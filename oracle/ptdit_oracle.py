@@ -226,7 +226,8 @@ def multihead_attention(x_q, x_kv, W, heads, allow=None) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# GIIM  [T2X §3 Eq. GIIM: z_s = CS(z_s, SA(Averaging(z_s))); code listing steps 1-2]
+# GIIM  [T2X §3 Eq. GIIM: z_s = CS(z_s, SA(Averaging(z_s))); the code listing's proxy
+#        self-attention and cross-attention]
 # --------------------------------------------------------------------------
 
 def proxy_self_attention(z, grid, ratio, W_psa, heads, proxy_residual=False, proxy_mode="mean",
@@ -479,7 +480,8 @@ def tcm(z, grid, window, shift, W_wsa, W_swsa, heads, *, residual=True) -> np.nd
 
 def block_attn(z, grid, ratio, window, shift, W_psa, W_cross, W_wsa, W_swsa, heads, *,
                proxy_residual=False, residual=True) -> np.ndarray:
-    """GIIM then TCM on one batch item  [T2X code listing: ProxyTokensTransformerBlock.forward 1-4]."""
+    """GIIM then TCM on one batch item  [T2X code listing: ProxyTokensTransformerBlock.forward,
+    its GIIM and TCM attentions]."""
     z1 = giim(z, grid, ratio, W_psa, W_cross, heads, proxy_residual=proxy_residual,
               residual=residual)
     return tcm(z1, grid, window, shift, W_wsa, W_swsa, heads, residual=residual)
@@ -564,13 +566,13 @@ def masked_self_attention(z, W, heads, allow, *, residual=True) -> np.ndarray:
 # --------------------------------------------------------------------------
 # The complete PT-Block  [T2X §3 Method: "PT-Block (GIIM + TCM + text
 # cross-attn + MLP)", the block diagram; code-comparison section,
-# ProxyTokensTransformerBlock.forward steps 1-4]
+# ProxyTokensTransformerBlock.forward]
 #
 # Readings (the pages name the sub-layers and their order but not the norms'
 # form, the MLP's width or activation, nor where each norm sits):
 #   * every sub-layer is pre-norm with a residual: x <- x + F(LN(x)); the proxy
 #     self-attention normalises the proxies (proxy_norm1) and adds them back,
-#     as the listing's step 1 does;
+#     as the listing's proxy self-attention does;
 #   * LN is a LayerNorm over D with a per-channel scale and shift and
 #     epsilon eps; its variance is the population (biased) variance;
 #   * the text cross-attention takes the normalised latents as queries and the

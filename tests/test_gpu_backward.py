@@ -192,21 +192,24 @@ def test_giim_bwd_full_size_1024px():
 
 # ---------------------------------------------------------------- the whole path
 
-def _check_path(c, ratio, window, shift, dout_cpu, dz, dw):
+def _check_path(c, ratio, window, shift, dout_cpu, dz, dw, flags=0):
     """dz and the four modules' weight gradients of the whole path against the oracle."""
     dz = c.out64(dz)
     g64 = synth.as_f64(dout_cpu)
     mods = ("psa", "cross", "wsa", "swsa")
     want = [[np.zeros((c.D, c.D)) for _ in range(4)] for _ in mods]
     kappa = 0.0
+    pres = bool(flags & pt.PTDIT_PROXY_RESIDUAL)
     for b in range(c.B):
         wdz, *ww = O.block_attn_bwd(c.z64[b], c.grid, ratio, window, shift,
-                                    *[c.w64[m] for m in mods], c.heads, g64[b])
+                                    *[c.w64[m] for m in mods], c.heads, g64[b],
+                                    proxy_residual=pres,
+                                    residual=not flags & pt.PTDIT_NO_RESIDUAL)
         assert rel_err(dz[b], wdz) <= TOL["bf16"], ("dz", b)
         for m in range(4):
             for i in range(4):
                 want[m][i] += ww[m][i]
-        kappa = max(kappa, _proxy_kappa(c.z64[b], c.grid, ratio, c.w64["psa"], c.heads, False))
+        kappa = max(kappa, _proxy_kappa(c.z64[b], c.grid, ratio, c.w64["psa"], c.heads, pres))
     tol_qk = TOL["bf16"] + 2 * 2.0 ** -8 * kappa
     for m, name in enumerate(mods):
         for i in range(4):
@@ -256,3 +259,27 @@ def test_block_attn_train_pair(grid, D, heads, ratio, window, shift, B):
     for m in range(4):
         for i in range(4):
             assert rel_err(c.out64(dw[m][i]), c.out64(dw2[m][i])) <= 1e-2, (mods[m], i)
+
+
+@pytest.mark.parametrize("flags", ["proxy_residual", "no_residual"])
+def test_block_attn_bwd_flags(flags):
+    """The whole path with the proxy residual and without the latent residuals, through
+    both the recomputing backward and the training pair."""
+    f = pt.PTDIT_PROXY_RESIDUAL if flags == "proxy_residual" else pt.PTDIT_NO_RESIDUAL
+    grid, ratio, window, shift = (2, 16, 32), (1, 2, 2), (2, 8, 8), (1, 4, 4)
+    c = Case(1, grid, 1152, 16, "bf16")
+    W = [c.w[m] for m in ("psa", "cross", "wsa", "swsa")]
+    dout_cpu = _dout(c.B, c.N, c.D)
+    dz, *dw = pt.ptdit_block_attn_bwd(c.z, dout_cpu.cuda(), grid, ratio, window, shift, *W,
+                                      c.heads, f)
+    _check_path(c, ratio, window, shift, dout_cpu, dz, dw, f)
+    ws = pt.train_workspace(c.z, grid, ratio, window, c.heads)
+    out = c.out64(pt.ptdit_block_attn_fwd_train(c.z, grid, ratio, window, shift, *W, c.heads, ws, f))
+    want = O.block_attn(c.z64[0], grid, ratio, window, shift,
+                        *[c.w64[m] for m in ("psa", "cross", "wsa", "swsa")], c.heads,
+                        proxy_residual=bool(f & pt.PTDIT_PROXY_RESIDUAL),
+                        residual=not f & pt.PTDIT_NO_RESIDUAL)
+    assert rel_err(out[0], want) <= TOL["bf16"]
+    dz, *dw = pt.ptdit_block_attn_bwd_saved(c.z, dout_cpu.cuda(), grid, ratio, window, shift, *W,
+                                            c.heads, ws, f)
+    _check_path(c, ratio, window, shift, dout_cpu, dz, dw, f)
