@@ -212,9 +212,17 @@ def _check_path(c, ratio, window, shift, dout_cpu, dz, dw, flags=0):
         kappa = max(kappa, _proxy_kappa(c.z64[b], c.grid, ratio, c.w64["psa"], c.heads, pres))
     tol_qk = TOL["bf16"] + 2 * 2.0 ** -8 * kappa
     for m, name in enumerate(mods):
+        # without the residual stream z1 is the cross-attention output alone, nearly the
+        # same row for every token, so the window modules' scores are nearly equal across
+        # keys and their dWq, dWk nearly vanish: there each gradient's error is measured
+        # against its module's gradient scale (the largest entry of its four matrices)
+        scale = max(np.abs(x).max() for x in want[m]) if flags & pt.PTDIT_NO_RESIDUAL else None
         for i in range(4):
             tol = tol_qk if (name == "cross" and i < 2) else TOL["bf16"]
-            assert rel_err(c.out64(dw[m][i]), want[m][i]) <= tol, (name, i, kappa)
+            got = c.out64(dw[m][i])
+            err = (rel_err(got, want[m][i]) if scale is None
+                   else float(np.abs(got - want[m][i]).max() / scale))
+            assert err <= tol, (name, i, kappa, err)
 
 
 @pytest.mark.parametrize("grid,D,heads,ratio,window,shift,B", [
