@@ -6,6 +6,8 @@ head widths 72 (two swizzle atoms), 64 and 32, several batch items, a grid whose
 windows leave one CTA with more units than another, and the T2V workload in full.
 Both forms must also agree with each other closely (same operands, different
 rounding order in the softmax)."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -86,3 +88,35 @@ def test_fused_setting_reads_and_restores():
     assert L.ptdit_window_fused(-1) == 0
     assert L.ptdit_window_fused(prev) == 0
     assert L.ptdit_window_fused(7) == prev  # any other value only reads
+
+
+def test_fused_in_the_complete_block():
+    """The complete PT-Block with the fused window kernel: its window branches read the
+    LayerNorm output and add the residual stream."""
+    from tests.test_gpu_block import _run_block
+    c = Case(2, (2, 16, 16), 1152, 16, "bf16")
+    prev = pt.lib().ptdit_window_fused(1)
+    try:
+        _run_block(c, (1, 4, 4), (2, 8, 8), (1, 4, 4), 120, 4608)
+    finally:
+        pt.lib().ptdit_window_fused(prev)
+
+
+def test_fused_needs_its_workspace():
+    """A workspace that holds everything but the repacked weight rows runs the two-kernel
+    form: same result as a full workspace with the fused kernel off."""
+    c = Case(1, (2, 16, 16), 1152, 16, "bf16")
+    window, shift = (2, 8, 8), (1, 4, 4)
+    shape = pt.make_shape(c.z, c.grid, c.heads)
+    full = pt.lib().ptdit_workspace_bytes(ctypes.byref(shape), None, pt._i3(window))
+    small = full - 16 * 224 * 1152 * 2  # less the repacked weight rows
+    ws = torch.empty(small, dtype=torch.uint8, device="cuda")
+    prev = pt.lib().ptdit_window_fused(1)
+    try:
+        got = pt.ptdit_window_attn(c.z, c.grid, window, shift, c.w["swsa"], c.heads, ws=ws)
+    finally:
+        pt.lib().ptdit_window_fused(prev)
+    pt.lib().ptdit_window_fused(0)
+    want = pt.ptdit_window_attn(c.z, c.grid, window, shift, c.w["swsa"], c.heads)
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
