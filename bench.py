@@ -62,9 +62,9 @@ def l2_policy(w):
 TRAFFIC = {
     # profiles/gemm_tc2_t2i_2048px_qkv_and_oproj.md: nine launches measured
     "t2i_2048px_128x128": 59.4e6,
-    # the same capture scaled by rows to the long video (a lower bound: at 16384 rows
-    # part of every output is still in L2 when the kernel ends)
-    "video_32x64x64": 461e6,
+    # profiles/gemm_tc2_dram_traffic_video_32x64x64.md: one step's nine launches
+    # captured on the long video itself, per launch
+    "video_32x64x64": 641.3e6,
 }
 
 
