@@ -52,34 +52,38 @@ __global__ void row_delta_kernel(const uint8_t *__restrict__ dO, const __nv_bflo
     delta[(b * heads + h) * nq + q] = s;
 }
 
-// One thread per 8 columns of one token: dz = (dout +) dPa[proxy of the token] / P.
+// One warp per token row: dz = (dout +) dPa[proxy of the token] / P, the proxy index
+// computed once per row, the lanes on consecutive 16-byte pieces.
 __global__ void proxy_broadcast_kernel(ProxyGeom g, int B, int D, const __nv_bfloat16 *__restrict__ dPa,
                                        const __nv_bfloat16 *__restrict__ dout,
                                        __nv_bfloat16 *__restrict__ dz) {
     pdl_wait();
     pdl_trigger();
-    const int pieces = D / 8;
+    const int pieces = D / 8, lane = threadIdx.x % 32;
     const long N = (long)g.f * g.h * g.w;
-    const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (long)B * N * pieces) return;
-    const long tok = idx / pieces;
-    const int c = static_cast<int>(idx - tok * pieces) * 8;
+    const long tok = ((long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    if (tok >= (long)B * N) return;
     const long b = tok / N;
     const int m = proxy_of_token(g, static_cast<int>(tok - b * N));
     const float inv = 1.f / static_cast<float>(g.P);
-    const uint4 vp = *reinterpret_cast<const uint4 *>(dPa + ((long)b * g.M + m) * D + c);
-    uint4 vr = make_uint4(0, 0, 0, 0);
-    if (dout) vr = *reinterpret_cast<const uint4 *>(dout + tok * D + c);
-    const uint32_t wp[4] = {vp.x, vp.y, vp.z, vp.w}, wr[4] = {vr.x, vr.y, vr.z, vr.w};
-    uint32_t o[4];
+    const __nv_bfloat16 *prow = dPa + ((long)b * g.M + m) * D;
+    const __nv_bfloat16 *rrow = dout ? dout + tok * D : nullptr;
+    __nv_bfloat16 *orow = dz + tok * D;
+    for (int pc = lane; pc < pieces; pc += 32) {
+        const uint4 vp = *reinterpret_cast<const uint4 *>(prow + 8 * pc);
+        uint4 vr = make_uint4(0, 0, 0, 0);
+        if (rrow) vr = *reinterpret_cast<const uint4 *>(rrow + 8 * pc);
+        const uint32_t wp[4] = {vp.x, vp.y, vp.z, vp.w}, wr[4] = {vr.x, vr.y, vr.z, vr.w};
+        uint32_t o[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const float2 fp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wp[t]));
-        const float2 fr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[t]));
-        const __nv_bfloat162 v = __floats2bfloat162_rn(fmaf(fp.x, inv, fr.x), fmaf(fp.y, inv, fr.y));
-        o[t] = *reinterpret_cast<const uint32_t *>(&v);
+        for (int t = 0; t < 4; ++t) {
+            const float2 fp = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wp[t]));
+            const float2 fr = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[t]));
+            const __nv_bfloat162 v = __floats2bfloat162_rn(fmaf(fp.x, inv, fr.x), fmaf(fp.y, inv, fr.y));
+            o[t] = *reinterpret_cast<const uint32_t *>(&v);
+        }
+        *reinterpret_cast<uint4 *>(orow + 8 * pc) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    *reinterpret_cast<uint4 *>(dz + tok * D + c) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __global__ void to_bf16_kernel(const float *__restrict__ src, long rows, int cols,
@@ -271,7 +275,7 @@ cudaError_t launch_row_delta(const void *dO_tiles, const void *O, int B, int nq,
 cudaError_t launch_proxy_broadcast(const ProxyGeom &g, int B, int D, const void *dPa,
                                    const void *dout, void *dz, cudaStream_t s) {
     if (D % 8) return cudaErrorInvalidValue;
-    const long n = (long)B * g.f * g.h * g.w * (D / 8);
+    const long n = (long)B * g.f * g.h * g.w * 32;  // one warp per token
     const int threads = 256;
     return launch_pdl(proxy_broadcast_kernel, dim3((unsigned)((n + threads - 1) / threads)),
                       dim3(threads), 0, s, g, B, D, static_cast<const __nv_bfloat16 *>(dPa),
