@@ -399,3 +399,19 @@ def test_training_pair_workspace_and_refusals(L):
     f32 = _bshape(dtype=pt.PTDIT_F32)
     assert L.ptdit_block_attn_fwd_train(ctypes.byref(f32), *args[1:], FAKE * 20, FAKE * 21,
                                         FAKE * 128, 1 << 40, None) == 3
+
+
+def test_window_fused_setting_is_per_thread(L):
+    """ptdit_window_fused: off by default, 0/1 set it, anything else only reads it, and
+    the setting belongs to the calling host thread."""
+    import threading
+    assert L.ptdit_window_fused(-1) == 0
+    assert L.ptdit_window_fused(1) == 0
+    assert L.ptdit_window_fused(2) == 1  # reads only
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(L.ptdit_window_fused(-1)))
+    t.start()
+    t.join()
+    assert seen == [0]  # another thread still has the default
+    assert L.ptdit_window_fused(0) == 1
+    assert L.ptdit_window_fused(-1) == 0
