@@ -309,10 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_wait();
                 const uint32_t w0 = allow[0], w1 = allow[1];
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if ((w0 & w1) != 0xffffffffu) {  // some key masked (a window the roll wrapped)
 #pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const bool ok = ((e < 32 ? w0 : w1) >> (e & 31)) & 1u;
-                    if (!ok) sv[e] = __float_as_uint(-INFINITY);
+                    for (int e = 0; e < 64; ++e) {
+                        const bool ok = ((e < 32 ? w0 : w1) >> (e & 31)) & 1u;
+                        if (!ok) sv[e] = __float_as_uint(-INFINITY);
+                    }
                 }
 #pragma unroll
                 for (int e = 0; e < 64; e += 8)
@@ -345,9 +347,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(t_s + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * q));
                 tmem_ld_wait();
                 float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if ((allow[0] & allow[1] & allow[2] & allow[3]) != 0xffffffffu) {  // some key masked
 #pragma unroll
-                for (int e = 0; e < 128; ++e)
-                    if (!((allow[e >> 5] >> (e & 31)) & 1u)) sv[e] = __float_as_uint(-INFINITY);
+                    for (int e = 0; e < 128; ++e)
+                        if (!((allow[e >> 5] >> (e & 31)) & 1u)) sv[e] = __float_as_uint(-INFINITY);
+                }
 #pragma unroll
                 for (int e = 0; e < 128; e += 8)
 #pragma unroll
