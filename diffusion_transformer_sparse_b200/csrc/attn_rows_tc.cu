@@ -6,16 +6,20 @@
 //
 // FlashAttention-style warp specialisation, one persistent CTA per SM:
 //   warp 0       loader: two 128-row query tiles per unit (double buffered
-//                across units) and K and V tiles into a two-stage ring, each
-//                one contiguous bulk copy: the projections wrote Q, K and V in
-//                tiled head layout (thl.cuh), so a (tile, head) block already
+//                across units), K tiles and V tiles into two-stage rings of
+//                their own (a K stage is released after both score MMAs, a V
+//                stage after both P V MMAs), each one contiguous bulk copy:
+//                the projections wrote Q, K and V in tiled head layout
+//                (thl.cuh), so a (tile, head) block already
 //                is the swizzled shared-memory tile (columns 0..63 with the
 //                128-byte swizzle, 64..79 with the 32-byte swizzle, zeros past
 //                the head; V padded to 128 columns).
-//   warp 1       MMA issuer: S_g = Q_g K^T (K-major operands) into TMEM, and
+//   warp 1       MMA issuer (the whole warp runs the loop, lane 0 issues):
+//                S_g = Q_g K^T (K-major operands) into TMEM, and
 //                once softmax g has written P_g, P_g V with P_g read straight
 //                from TMEM and V as an MN-major operand (no transpose),
 //                accumulating into O_g in TMEM.
+//   warp 2       output stores: one tensor store per staged 128-row output tile.
 //   warps 4-7 and 8-11   two softmax warpgroups, one per query tile: thread r
 //                owns row r (its TMEM lane), reads its 128 scores with one
 //                wait, runs the fp32 online softmax and writes P (bf16, two per
@@ -46,7 +50,7 @@ constexpr int BQ = 128, BKV = 128;
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;  // S0, S1, O0, O1: 128 columns each
 
-constexpr int NSTAGE = 2;  // K/V ring depth
+constexpr int NSTAGE = 2;  // depth of the K ring and of the V ring
 
 template <int DPAD>
 struct RowsLayout {
@@ -67,9 +71,10 @@ struct RowsLayout {
     static constexpr int STG = BQ * 160;
     static constexpr int OFF_STG = OFF_V + NSTAGE * VTILE;
     static constexpr int OFF_BAR = OFF_STG + 2 * STG;
-    // kv_full[NSTAGE], kv_empty[NSTAGE], q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2],
+    // k_full[NSTAGE], k_empty[NSTAGE], v_full[NSTAGE], v_empty[NSTAGE], q_full[2], q_empty[2],
+    // s_full[2], p_full[2], o_full[2],
     // drain, stage_full[2], stage_free[2]
-    static constexpr int NBARS = 2 * NSTAGE + 15;
+    static constexpr int NBARS = 4 * NSTAGE + 15;
     static constexpr int BYTES = OFF_BAR + NBARS * 8 + 16 + 1024;  // + base alignment slack
     static_assert(TILE % 1024 == 0 && TILE_A % 1024 == 0, "swizzled tiles stay 1 KB aligned");
     static_assert(BYTES <= 232448, "shared memory budget");
@@ -91,15 +96,17 @@ __device__ __forceinline__ void decode(const AttnArgs &a, const RowsSched &sc, i
 
 template <int DPAD, bool SUMV>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_rows_kernel(const __grid_constant__ AttnArgs a, RowsSched sc, int *status) {
+    attn_rows_kernel(const __grid_constant__ AttnArgs a, RowsSched sc,
+                     const __grid_constant__ CUtensorMap omap, int *status) {
     using L = RowsLayout<DPAD>;
     extern __shared__ uint8_t sm_raw[];
     // TMA destinations: align the base to 1 KB (tile offsets are multiples of 1 KB)
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
-    uint64_t *kv_full = bars, *kv_empty = bars + NSTAGE;
-    uint64_t *q_full = bars + 2 * NSTAGE, *q_empty = q_full + 2, *s_full = q_full + 4;
+    uint64_t *k_full = bars, *k_empty = bars + NSTAGE;
+    uint64_t *v_full = bars + 2 * NSTAGE, *v_empty = bars + 3 * NSTAGE;
+    uint64_t *q_full = bars + 4 * NSTAGE, *q_empty = q_full + 2, *s_full = q_full + 4;
     uint64_t *p_full = q_full + 6, *o_full = q_full + 8, *drain = q_full + 10;
     uint64_t *stage_full = q_full + 11, *stage_free = q_full + 13;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::NBARS);
@@ -110,8 +117,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
@@ -123,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(drain, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&stage_full[s], BQ);
-            mbar_init(&stage_free[s], BQ);
+            mbar_init(&stage_free[s], 1);
         }
         *abort = 0;
         fence_mbar_init();
@@ -150,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              uint32_t bytes) {
                 return base + (((long)b * t.tiles + tile) * a.heads + h) * (long)bytes;
             };
-            int item = 0, last_q_unit = -1;
+            int item = 0, k_issued = 0, v_issued = 0, last_q_unit = -1;
             bool ok = true;
             for (int u = u0; u < u1 && ok; ++u) {
                 int b, h, qp;
@@ -171,18 +180,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       L::TILE, &q_full[qb]);
                         last_q_unit = un;
                     }
-                    if (!mbar_wait(&kv_empty[st], ((item / NSTAGE) & 1) ^ 1, abort, status)) { ok = false; break; }
-                    mbar_expect_tx(&kv_full[st], L::TILE + L::VTILE);
+                    // K and V have rings of their own: a K stage is free once both
+                    // score MMAs of its item have read it, a V stage only after both
+                    // P V MMAs, so the next K tile is on its way a P V earlier
+                    const uint32_t par = ((item / NSTAGE) & 1) ^ 1;
+                    if (!mbar_wait(&k_empty[st], par, abort, status)) { ok = false; break; }
+                    mbar_expect_tx(&k_full[st], L::TILE);
                     bulk_load(sm + L::OFF_K + st * L::TILE, block(kg, a.tk, b, j, h, L::TILE), L::TILE,
-                              &kv_full[st]);
+                              &k_full[st]);
+                    ++k_issued;
+                    if (!mbar_wait(&v_empty[st], par, abort, status)) { ok = false; break; }
+                    mbar_expect_tx(&v_full[st], L::VTILE);
                     bulk_load(sm + L::OFF_V + st * L::VTILE, block(vg, a.tv, b, j, h, L::VTILE),
-                              L::VTILE, &kv_full[st]);
+                              L::VTILE, &v_full[st]);
+                    ++v_issued;
                 }
             }
             if (!ok) {  // let copies still in flight land before the CTA exits
                 volatile int never = 0;
-                for (int i = item - NSTAGE; i < item; ++i)
-                    if (i >= 0) mbar_wait(&kv_full[i % NSTAGE], (i / NSTAGE) & 1, &never, status);
+                for (int i = k_issued - NSTAGE; i < k_issued; ++i)
+                    if (i >= 0) mbar_wait(&k_full[i % NSTAGE], (i / NSTAGE) & 1, &never, status);
+                for (int i = v_issued - NSTAGE; i < v_issued; ++i)
+                    if (i >= 0) mbar_wait(&v_full[i % NSTAGE], (i / NSTAGE) & 1, &never, status);
                 if (last_q_unit >= 0)
                     mbar_wait(&q_full[last_q_unit & 1], (last_q_unit >> 1) & 1, &never, status);
             }
@@ -191,58 +210,103 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA issuer
         // Order per item i: PV0(i), S0(i+1), PV1(i), S1(i+1), so each softmax
         // warpgroup gets its next S right after handing over its P, while the
-        // other warpgroup is still busy.
-        if (lane == 0) {
+        // other warpgroup is still busy.  The whole warp runs this loop (its
+        // operands stay warp-uniform) and lane 0 issues each MMA and commit; the
+        // waits are taken by the whole warp.
+        {
             constexpr uint32_t idesc_s = idesc_bf16(BQ, BKV);
             constexpr uint32_t idesc_o = idesc_bf16(BQ, L::NPV, true);
             const int n_items = (u1 - u0) * sc.kt;
             bool ok = true, any = false;
-            // S_g(i) = Q_g K(i)^T; waits for the K tile (and, at a unit's first
-            // tile, for the unit's Q tiles) when g == 0
+            // the operands of S(i): the K tile and, at a unit's first tile, the
+            // unit's Q tiles
+            auto wait_s_operands = [&](int i) {
+                const int st = i % NSTAGE, j = i % sc.kt, un = i / sc.kt, qb = un & 1;
+                if (!mbar_wait_warp(&k_full[st], (i / NSTAGE) & 1, abort, status)) return false;
+                if (j == 0 && !mbar_wait_warp(&q_full[qb], (un >> 1) & 1, abort, status)) return false;
+                return true;
+            };
+            // S_g(i) = Q_g K(i)^T (its operands waited for)
             auto issue_s = [&](int i, int g) {
                 const int st = i % NSTAGE, j = i % sc.kt, un = i / sc.kt, qb = un & 1;
-                if (g == 0) {
-                    if (!mbar_wait(&kv_full[st], (i / NSTAGE) & 1, abort, status)) return false;
-                    if (j == 0 && !mbar_wait(&q_full[qb], (un >> 1) & 1, abort, status)) return false;
-                    fence_after_sync();
-                }
                 const uint32_t aK = smem_u32(sm + L::OFF_K + st * L::TILE);
                 const uint32_t aQ = smem_u32(sm + L::OFF_Q + (qb * 2 + g) * L::TILE);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + g * BKV, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
-                             idesc_s, kk > 0);
+                    warp_mma_bf16(tmem + g * BKV, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
+                                  idesc_s, kk > 0);
                 if (L::HAS_B)
-                    mma_bf16(tmem + g * BKV, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
-                             idesc_s, 1);
-                mma_commit(&s_full[g]);
-                if (g == 1 && j == sc.kt - 1) mma_commit(&q_empty[qb]);  // the unit's Q tiles are read
+                    warp_mma_bf16(tmem + g * BKV, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
+                                  idesc_s, 1);
+                warp_mma_commit(&s_full[g]);
+                if (g == 1) {
+                    warp_mma_commit(&k_empty[st]);  // both S of item i have read K(i)
+                    if (j == sc.kt - 1) warp_mma_commit(&q_empty[qb]);  // the unit's Q tiles are read
+                }
                 any = true;
-                return true;
             };
-            if (n_items > 0) ok = issue_s(0, 0) && issue_s(0, 1);
+            if (n_items > 0) {
+                ok = wait_s_operands(0);
+                fence_after_sync();
+                if (ok) {
+                    issue_s(0, 0);
+                    issue_s(0, 1);
+                }
+            }
             for (int i = 0; i < n_items && ok; ++i) {
                 const int st = i % NSTAGE, j = i % sc.kt;
                 const uint32_t aV = smem_u32(sm + L::OFF_V + st * L::VTILE);
+                // V(i) and the operands of S(i+1) are waited for here, while the
+                // softmax still works on S(i): both landed long ago (their stages
+                // were released an item earlier), and no wait then sits between
+                // P_g(i) and the MMAs that follow it.  A wait issued right behind
+                // a burst of MMAs only answers once they have run.
+                if (!mbar_wait_warp(&v_full[st], (i / NSTAGE) & 1, abort, status) ||
+                    (i + 1 < n_items && !wait_s_operands(i + 1))) { ok = false; break; }
                 for (int g = 0; g < 2 && ok; ++g) {
-                    if (!mbar_wait(&p_full[g], i & 1, abort, status)) { ok = false; break; }
+                    if (!mbar_wait_warp(&p_full[g], i & 1, abort, status)) { ok = false; break; }
                     fence_after_sync();
                     const uint32_t tP = tmem + g * BKV;  // P_g over the first 64 columns of S_g
                     const uint32_t tO = tmem + 256 + g * 128;
 #pragma unroll
                     for (int ks = 0; ks < BKV / 16; ++ks)
-                        mma_bf16_ts(tO, tP + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
-                                    idesc_o, (j | ks) > 0);
-                    mma_commit(&o_full[g]);
-                    if (g == 1) mma_commit(&kv_empty[st]);  // both S and both P V of item i
-                    if (i + 1 < n_items) ok = issue_s(i + 1, g);
+                        warp_mma_bf16_ts(tO, tP + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
+                                         idesc_o, (j | ks) > 0);
+                    warp_mma_commit(&o_full[g]);
+                    if (g == 1) warp_mma_commit(&v_empty[st]);  // both P V of item i have read V(i)
+                    if (i + 1 < n_items) issue_s(i + 1, g);
                 }
             }
             if (any) {  // every issued MMA has finished before TMEM is released
-                mma_commit(drain);
+                warp_mma_commit(drain);
                 volatile int never = 0;
-                mbar_wait(drain, 0, &never, status);
+                mbar_wait_warp(drain, 0, &never, status);
             }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ output stores
+        // Each softmax warpgroup stages its unit's 128 normalised output rows
+        // in shared memory and moves on; lane 0 here writes them out with one
+        // tensor store per query tile (rows past nq are not written).
+        if (lane == 0) {
+            prefetch_tensormap(&omap);
+            int un_count = 0;
+            bool ok = true;
+            for (int u = u0; u < u1 && ok; ++u, ++un_count) {
+                int b, h, qp;
+                decode(a, sc, u, b, h, qp);
+                for (int g = 0; g < 2; ++g) {
+                    if (!mbar_wait(&stage_full[g], un_count & 1, abort, status)) { ok = false; break; }
+                    const int q0 = qp * 2 * BQ + g * BQ;  // query index of staging row 0
+                    if (q0 < a.nq) {
+                        tma_store_3d(&omap, sm + L::OFF_STG + g * L::STG, h * d, q0, b);
+                        bulk_commit();
+                    }
+                    bulk_wait_read_all();  // the staging rows have been read
+                    mbar_arrive(&stage_free[g]);
+                }
+            }
+            bulk_wait_all();  // the output is in global memory before the CTA exits
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax warpgroups
@@ -263,9 +327,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_s = tmem + lane_base + g * BKV;
         const uint32_t t_o = tmem + lane_base + 256 + g * 128;
         const float sl2 = a.scale * 1.4426950408889634f;
-        __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.o);
-        // staging row pitch: an odd number of 16-byte units where that fits
-        const int pitch = nch * 16 + (nch % 8 == 0 ? 16 : 0);
+        // staging rows as the tensor store reads them: packed at nch * 16 bytes,
+        // or, for nch == 8, 128 bytes with the 128-byte swizzle (16-byte piece u
+        // of row r at (u ^ (r & 7)) * 16), so that no two lanes of a store
+        // phase hit the same banks
+        const bool sw128 = nch == 8;
         int item = 0, un_count = 0;
         bool ok = true;
         for (int u = u0; u < u1 && ok; ++u) {
@@ -355,9 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&p_full[g]);
             }
             if (!ok) break;
-            // the unit's last P V, then O / l to global memory through the staging
-            // rows, so that consecutive lanes store consecutive 16-byte pieces of
-            // a row (a few rows per store instruction instead of 32)
+            // the unit's last P V, then O / l into the staging rows (once the
+            // store warp has read the previous unit's); warp 2 writes them out
             if (!wait_all(&o_full[g], (item - 1) & 1)) { ok = false; break; }
             if (!wait_all(&stage_free[g], (un_count & 1) ^ 1)) { ok = false; break; }
             fence_after_sync();
@@ -384,23 +449,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         v.y = pack_bf16(__uint_as_float(ov[8 * u + 2]) * inv, __uint_as_float(ov[8 * u + 3]) * inv);
                         v.z = pack_bf16(__uint_as_float(ov[8 * u + 4]) * inv, __uint_as_float(ov[8 * u + 5]) * inv);
                         v.w = pack_bf16(__uint_as_float(ov[8 * u + 6]) * inv, __uint_as_float(ov[8 * u + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(stg + r * pitch + u * 16) = v;
+                        const int piece = sw128 ? (u ^ (r & 7)) : u;
+                        *reinterpret_cast<uint4 *>(stg + r * nch * 16 + piece * 16) = v;
                     }
             }
             fence_before_sync();  // O is read before the next unit's first P V overwrites it
+            fence_async_smem();   // the staging rows are visible to the tensor store
             mbar_arrive(&stage_full[g]);
-            if (!wait_all(&stage_full[g], un_count & 1)) { ok = false; break; }
-            {
-                const int q0 = qp * 2 * BQ + g * BQ;  // query index of staging row 0
-                __nv_bfloat16 *obase = og + (long)b * a.q_bstride * a.ldo + (long)h * d;
-                for (int i = r; i < BQ * nch; i += BQ) {
-                    const int row = i / nch, u = i - row * nch;
-                    if (q0 + row < a.nq)
-                        *reinterpret_cast<uint4 *>(obase + (long)(q0 + row) * a.ldo + u * 8) =
-                            *reinterpret_cast<const uint4 *>(stg + row * pitch + u * 16);
-                }
-            }
-            mbar_arrive(&stage_free[g]);
             ++un_count;
         }
     }
@@ -422,6 +477,13 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
         a.tq.vpad || a.tk.vpad || !a.tv.vpad || L::TILE != (int)thl_block_bytes(a.d, 0) ||
         L::VTILE != (int)thl_block_bytes(a.d, 1))
         return cudaErrorInvalidValue;
+    // the output tiles go out as tensor stores of (d columns, 128 rows) boxes
+    CUtensorMap omap;
+    if (reinterpret_cast<uintptr_t>(a.o) % 16 || a.ldo % 8 ||
+        !encode_map_out_rows_bf16(&omap, a.o, (uint64_t)a.heads * a.d, (uint64_t)a.nq,
+                                  (uint64_t)a.B, (uint64_t)a.ldo * 2,
+                                  (uint64_t)a.q_bstride * a.ldo * 2, (uint32_t)a.d, BQ, a.d == 64))
+        return cudaErrorInvalidValue;
     RowsSched sc;
     sc.qp = (a.nq + 2 * BQ - 1) / (2 * BQ);
     sc.kt = (a.nk + BKV - 1) / BKV;
@@ -432,7 +494,7 @@ cudaError_t launch_rows(const AttnArgs &a, cudaStream_t s) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
     return launch_pdl(attn_rows_kernel<DPAD, SUMV>, dim3(grid), dim3(kThreads), L::BYTES, s, a, sc,
-                      status);
+                      omap, status);
 }
 
 }  // namespace

@@ -92,6 +92,23 @@ bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows
     return r == CUDA_SUCCESS;
 }
 
+bool encode_map_out_rows_bf16(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                              uint64_t batches, uint64_t row_pitch_bytes,
+                              uint64_t batch_pitch_bytes, uint32_t box_cols, uint32_t box_rows,
+                              bool swizzle128) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cols, rows, batches};
+    cuuint64_t strides[2] = {row_pitch_bytes, batch_pitch_bytes};
+    cuuint32_t box[3] = {box_cols, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool encode_map_grid_bf16(CUtensorMap *map, const void *base, int B, int F, int H, int W, int D,
                           uint32_t box_c, uint32_t box_x, uint32_t box_y, uint32_t box_t) {
     EncodeTiledFn fn = encode_fn();

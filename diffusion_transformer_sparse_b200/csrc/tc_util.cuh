@@ -196,6 +196,15 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
         : "memory");
 }
 
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int x, int y,
+                                             int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -270,6 +279,43 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// The same three instructions for an issuer that runs as a whole converged warp:
+// every lane computes the (warp-uniform) operands and lane 0 alone issues, under a
+// predicate inside the instruction sequence rather than a branch around it.
+__device__ __forceinline__ void warp_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .u32 l;\n\t"
+        "mov.u32 l, %%laneid;\n\t"
+        "setp.eq.u32 e, l, 0;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void warp_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .u32 l;\n\t"
+        "mov.u32 l, %%laneid;\n\t"
+        "setp.eq.u32 e, l, 0;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void warp_mma_commit(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"
+        "mov.u32 l, %%laneid;\n\t"
+        "setp.eq.u32 e, l, 0;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
             smem_u32(bar))
         : "memory");
 }
@@ -485,6 +531,15 @@ bool encode_map_rows_heads_bf16(CUtensorMap *map, const void *base, uint64_t row
 bool encode_map_head_tile_bf16(CUtensorMap *map, const void *base, uint64_t rows,
                                uint64_t row_pitch_bytes, int heads, int d, uint32_t box_elems,
                                uint32_t box_rows, int swizzle_bytes);
+
+// Host: a 3-D map over a bf16 output of `batches` items of `rows` rows each, dims
+// (cols, rows, batches), strides (row pitch, batch pitch); box (box_cols, box_rows,
+// 1), unswizzled (rows packed at box_cols * 2 bytes in shared memory) or with the
+// 128-byte swizzle (box_cols * 2 == 128).  A store writes nothing past the extents.
+bool encode_map_out_rows_bf16(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                              uint64_t batches, uint64_t row_pitch_bytes,
+                              uint64_t batch_pitch_bytes, uint32_t box_cols, uint32_t box_rows,
+                              bool swizzle128);
 
 // Host: a 5-D map over a [B, F, H, W, D] bf16 token grid, dims (D, W, H, F, B), with the
 // 128-byte swizzle; box (box_c channels, box_x, box_y, box_t tokens, 1 item): a box of
