@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (the whole warp runs the loop with warp-uniform operands; lane 0 issues)
+        {
             constexpr uint32_t id_s = idesc_bf16(BQ, BQ);
             constexpr uint32_t id_mm64 = idesc_bf16(BQ, 64, true, true);
             constexpr uint32_t id_mm16 = idesc_bf16(BQ, 16, true, true);
@@ -204,18 +205,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto scores = [&](uint32_t d_col, uint32_t aX, uint32_t aY) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + d_col, sdesc_sw128(aX + kk * 32), sdesc_sw128(aY + kk * 32), id_s,
+                    warp_mma_bf16(tmem + d_col, sdesc_sw128(aX + kk * 32), sdesc_sw128(aY + kk * 32), id_s,
                              kk > 0);
                 if (L::HAS_B)
-                    mma_bf16(tmem + d_col, sdesc_sw32(aX + L::TILE_A), sdesc_sw32(aY + L::TILE_A),
+                    warp_mma_bf16(tmem + d_col, sdesc_sw32(aX + L::TILE_A), sdesc_sw32(aY + L::TILE_A),
                              id_s, 1);
             };
             auto grad = [&](uint32_t d_col, uint64_t a_desc, uint32_t aB, int ks, bool a_mn,
                             bool acc) {
-                mma_bf16(tmem + d_col, a_desc, sdesc_sw128_mn(aB + ks * 2048, L::TILE_A),
+                warp_mma_bf16(tmem + d_col, a_desc, sdesc_sw128_mn(aB + ks * 2048, L::TILE_A),
                          a_mn ? id_mm64 : id_km64, acc);
                 if (L::HAS_B)
-                    mma_bf16(tmem + d_col + 64, a_desc, sdesc_sw32_mn(aB + L::TILE_A + ks * 512),
+                    warp_mma_bf16(tmem + d_col + 64, a_desc, sdesc_sw32_mn(aB + L::TILE_A + ks * 512),
                              a_mn ? id_mm16 : id_km16, acc);
             };
             // the CTA's query tiles in order, with their item's ordinal and position
@@ -233,20 +234,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             // S(t) into columns 0-127 (K of item nix when t opens it)
             auto issue_s = [&](int t, bool new_item, int nix) {
-                if (new_item && !mbar_wait(kv_full, nix & 1, abort, status)) return false;
-                if (!mbar_wait(&q_full[t % NQB], (t / NQB) & 1, abort, status)) return false;
+                if (new_item && !mbar_wait_warp(kv_full, nix & 1, abort, status)) return false;
+                if (!mbar_wait_warp(&q_full[t % NQB], (t / NQB) & 1, abort, status)) return false;
                 fence_after_sync();
                 scores(T_S, qbuf(t), aK);
-                mma_commit(s_full);
+                warp_mma_commit(s_full);
                 any = true;
                 return true;
             };
             // dP(t) into the same columns once the warpgroups have read S(t)
             auto issue_dp = [&](int t) {
-                if (!mbar_wait(s_read, t & 1, abort, status)) return false;
+                if (!mbar_wait_warp(s_read, t & 1, abort, status)) return false;
                 fence_after_sync();
                 scores(T_DP, qbuf(t) + L::TILE, aV);
-                mma_commit(dp_full);
+                warp_mma_commit(dp_full);
                 return true;
             };
             // dV += P^T dO, then dK += dS^T Q of tile t (the item's first tile overwrites)
@@ -256,22 +257,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int ks = 0; ks < BQ / 16; ++ks)
                     grad(T_DV, sdesc_sw128_mn(aP + ks * 2048, L::TILE_A), aO, ks, true,
                          !first || ks > 0);
-                mma_commit(p_free);  // P is read
+                warp_mma_commit(p_free);  // P is read
 #pragma unroll
                 for (int ks = 0; ks < BQ / 16; ++ks)
                     grad(T_DK, sdesc_sw128_mn(aDS + ks * 2048, L::TILE_A), aQ, ks, true,
                          !first || ks > 0);
-                mma_commit(&q_free[t % NQB]);  // Q and dO are read
+                warp_mma_commit(&q_free[t % NQB]);  // Q and dO are read
             };
             // dQ = dS K of tile t in its own columns, once the previous dQ is read
             auto issue_dq = [&](int t) {
-                if (t > 0 && !mbar_wait(dq_free, (t - 1) & 1, abort, status)) return false;
+                if (t > 0 && !mbar_wait_warp(dq_free, (t - 1) & 1, abort, status)) return false;
                 fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < BQ / 16; ++ks)
                     grad(T_DQ, sdesc_sw128(aDS + (ks >> 2) * L::TILE_A + (ks & 3) * 32), aK, ks,
                          false, ks > 0);
-                mma_commit(dq_full);  // dQ is in TMEM and dS is read
+                warp_mma_commit(dq_full);  // dQ is in TMEM and dS is read
                 return true;
             };
             if (T > 0) ok = issue_s(0, true, 0) && issue_dp(0);
@@ -280,8 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int it2 = it, n2 = n_item, pos2 = pos;
                 advance(it2, n2, pos2);  // tile t + 1
                 // P(t) and dS(t) written, dP(t) read (S's columns are free)
-                if (!mbar_wait(pds_full, t & 1, abort, status)) break;
-                if (first && n_item > 0 && !mbar_wait(kvacc_free, (n_item - 1) & 1, abort, status))
+                if (!mbar_wait_warp(pds_full, t & 1, abort, status)) break;
+                if (first && n_item > 0 && !mbar_wait_warp(kvacc_free, (n_item - 1) & 1, abort, status))
                     break;
                 fence_after_sync();
                 if (!last) {
@@ -295,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // load only once dQ has read K)
                     issue_dvdk(t, first);
                     if (!issue_dq(t)) break;
-                    mma_commit(kvacc_full);
-                    mma_commit(kv_free);
+                    warp_mma_commit(kvacc_full);
+                    warp_mma_commit(kv_free);
                     if (t + 1 < T) ok = issue_s(t + 1, true, n2) && issue_dp(t + 1);
                 }
                 it = it2;
@@ -304,9 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pos = pos2;
             }
             if (any) {
-                mma_commit(drain);
+                warp_mma_commit(drain);
                 volatile int never = 0;
-                mbar_wait(drain, 0, &never, status);
+                mbar_wait_warp(drain, 0, &never, status);
             }
         }
     } else if (warp < 8) {

@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (the whole warp runs the loop with warp-uniform operands; lane 0 issues)
+        {
             constexpr uint32_t id_s = idesc_bf16(BQ, BQ);                 // K-major A and B
             constexpr uint32_t id_mm64 = idesc_bf16(BQ, 64, true, true);  // MN-major A and B
             constexpr uint32_t id_mm16 = idesc_bf16(BQ, 16, true, true);
@@ -204,20 +205,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto scores = [&](uint32_t d_col, uint32_t aX, uint32_t aY) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + d_col, sdesc_sw128(aX + kk * 32), sdesc_sw128(aY + kk * 32), id_s,
+                    warp_mma_bf16(tmem + d_col, sdesc_sw128(aX + kk * 32), sdesc_sw128(aY + kk * 32), id_s,
                              kk > 0);
                 if (L::HAS_B)
-                    mma_bf16(tmem + d_col, sdesc_sw32(aX + L::TILE_A), sdesc_sw32(aY + L::TILE_A),
+                    warp_mma_bf16(tmem + d_col, sdesc_sw32(aX + L::TILE_A), sdesc_sw32(aY + L::TILE_A),
                              id_s, 1);
             };
             // S = Q K^T of unit k (waits for its blocks)
             auto issue_s = [&](int k) {
                 const int bf = k % NBUF;
-                if (!mbar_wait(&ld_full[bf], (k / NBUF) & 1, abort, status)) return false;
+                if (!mbar_wait_warp(&ld_full[bf], (k / NBUF) & 1, abort, status)) return false;
                 fence_after_sync();
                 const uint32_t aQ = smem_u32(sm + bf * L::BUF);
                 scores(T_S, aQ, aQ + L::TILE);
-                mma_commit(s_full);
+                warp_mma_commit(s_full);
                 any = true;
                 return true;
             };
@@ -225,21 +226,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto issue_dp = [&](int k) {
                 const uint32_t aQ = smem_u32(sm + (k % NBUF) * L::BUF);
                 scores(T_DP, aQ + 3 * L::TILE, aQ + 2 * L::TILE);
-                mma_commit(dp_full);
+                warp_mma_commit(dp_full);
             };
             // D (rows of the reduction: K steps of 16) += A^T-or-A times the head
             // columns of the MN-major B operand at aB (N = 64, then N = 16)
             auto grad = [&](uint32_t d_col, uint64_t a_desc, uint32_t aB, int ks, bool a_mn) {
-                mma_bf16(tmem + d_col, a_desc, sdesc_sw128_mn(aB + ks * 2048, L::TILE_A),
+                warp_mma_bf16(tmem + d_col, a_desc, sdesc_sw128_mn(aB + ks * 2048, L::TILE_A),
                          a_mn ? id_mm64 : id_km64, ks > 0);
                 if (L::HAS_B)
-                    mma_bf16(tmem + d_col + 64, a_desc, sdesc_sw32_mn(aB + L::TILE_A + ks * 512),
+                    warp_mma_bf16(tmem + d_col + 64, a_desc, sdesc_sw32_mn(aB + L::TILE_A + ks * 512),
                              a_mn ? id_mm16 : id_km16, ks > 0);
             };
             auto issue_grads = [&](int k) {
                 const int bf = k % NBUF;
-                if (!mbar_wait(pds_full, k & 1, abort, status)) return false;
-                if (k > 0 && !mbar_wait(acc_free, (k - 1) & 1, abort, status)) return false;
+                if (!mbar_wait_warp(pds_full, k & 1, abort, status)) return false;
+                if (k > 0 && !mbar_wait_warp(acc_free, (k - 1) & 1, abort, status)) return false;
                 fence_after_sync();
                 const uint32_t aQ = smem_u32(sm + bf * L::BUF), aK = aQ + L::TILE,
                                aO = aQ + 3 * L::TILE;
@@ -254,9 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     grad(T_DK, sT, aQ, ks, true);   // dK += dS^T Q
                     grad(T_DQ, sK, aK, ks, false);  // dQ += dS K
                 }
-                mma_commit(acc_full);
-                mma_commit(pds_free);
-                mma_commit(&buf_free[bf]);
+                warp_mma_commit(acc_full);
+                warp_mma_commit(pds_free);
+                warp_mma_commit(&buf_free[bf]);
                 return true;
             };
             if (nunits > 0) {
@@ -266,20 +267,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < nunits && ok; ++k) {
                 // the softmax has read this unit's S and dP: the next S may overwrite S,
                 // and the gradients (dQ in dP's columns) may start
-                if (!mbar_wait(sp_free, k & 1, abort, status)) break;
+                if (!mbar_wait_warp(sp_free, k & 1, abort, status)) break;
                 if (k + 1 < nunits) ok = issue_s(k + 1);
                 if (ok) ok = issue_grads(k);
                 if (ok && k + 1 < nunits) {
                     // the epilogue has read dQ(k) out of dP's columns
-                    if (!mbar_wait(dq_free, k & 1, abort, status)) break;
+                    if (!mbar_wait_warp(dq_free, k & 1, abort, status)) break;
                     fence_after_sync();
                     issue_dp(k + 1);
                 }
             }
             if (any) {  // every issued MMA has finished before TMEM is released
-                mma_commit(drain);
+                warp_mma_commit(drain);
                 volatile int never = 0;
-                mbar_wait(drain, 0, &never, status);
+                mbar_wait_warp(drain, 0, &never, status);
             }
         }
     } else if (warp < 8) {

@@ -159,6 +159,38 @@ __device__ __forceinline__ void mma_commit_pair_local(uint64_t *bar) {
             smem_u32(bar))
         : "memory");
 }
+// The issuer runs as a whole converged warp (warp-uniform operands); lane 0
+// alone issues, under a predicate inside each instruction sequence.
+__device__ __forceinline__ void warp_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                   uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .u32 l;\n\t"
+        "mov.u32 l, %%laneid;\n\t"
+        "setp.eq.u32 e, l, 0;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void warp_mma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"
+        "mov.u32 l, %%laneid;\n\t"
+        "setp.eq.u32 e, l, 0;\n\t"
+        "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+__device__ __forceinline__ void warp_mma_commit_pair_local(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"
+        "mov.u32 l, %%laneid;\n\t"
+        "setp.eq.u32 e, l, 0;\n\t"
+        "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
@@ -275,7 +307,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        if (leader && lane == 0) {
+        // the MMA issuer: the whole warp of the pair's leader CTA runs the loop,
+        // lane 0 issues
+        if (leader) {
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, any = false;
@@ -283,11 +317,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 int m_tile, seg, n_tile;
                 decode_tile2(p, t, m_tile, seg, n_tile);
                 const uint32_t idesc = idesc_bf16(2 * BMC, tile_width<BN>(p, n_tile));
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort, p.status)) break;
+                if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1, abort, p.status)) break;
                 fence_after_sync();
                 const uint32_t d = tmem + acc * L::ACC_STRIDE;
                 for (int kb = 0; kb < p.kblocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, abort, p.status)) {
+                    if (!mbar_wait_warp(&full[stage], phase, abort, p.status)) {
                         ok = false;
                         break;
                     }
@@ -296,24 +330,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t sb = sa + L::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_bf16_pair(d, sdesc_sw128(sa + kk * 32), sdesc_sw128(sb + kk * 32), idesc,
-                                      (kb | kk) != 0);
+                        warp_mma_bf16_pair(d, sdesc_sw128(sa + kk * 32), sdesc_sw128(sb + kk * 32),
+                                           idesc, (kb | kk) != 0);
                     any = true;
-                    mma_commit_pair(&empty[stage]);
+                    warp_mma_commit_pair(&empty[stage]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
                 if (!ok) break;
-                mma_commit_pair(&tfull[acc]);
+                warp_mma_commit_pair(&tfull[acc]);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
             if (any) {  // every issued MMA has finished before TMEM is released
-                mma_commit_pair_local(drain);
+                warp_mma_commit_pair_local(drain);
                 volatile int never = 0;
-                mbar_wait(drain, 0, &never, p.status);
+                mbar_wait_warp(drain, 0, &never, p.status);
             }
         }
     } else {

@@ -147,40 +147,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (the whole warp runs the loop with warp-uniform operands; lane 0 issues)
+        {
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true, any = false;
             for (int t = blockIdx.x; ok && t < p.items; t += gridDim.x) {
                 const Item it = decode_item(p, t);
                 const uint32_t idesc = idesc_bf16(WM, it.width, true, true);
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort, p.status)) break;
+                if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1, abort, p.status)) break;
                 fence_after_sync();
                 const uint32_t d = tmem + acc * WN;
                 for (int kb = it.kb0; kb < it.kb1; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, abort, p.status)) { ok = false; break; }
+                    if (!mbar_wait_warp(&full[stage], phase, abort, p.status)) { ok = false; break; }
                     fence_after_sync();
                     const uint32_t sa = smem_u32(sm + stage * L::STAGE), sb = sa + L::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < WK / 16; ++kk)
-                        mma_bf16(d, sdesc_sw128_mn(sa + kk * 2048, BOX),
+                        warp_mma_bf16(d, sdesc_sw128_mn(sa + kk * 2048, BOX),
                                  sdesc_sw128_mn(sb + kk * 2048, BOX), idesc, (kb > it.kb0) | kk);
                     any = true;
-                    mma_commit(&empty[stage]);
+                    warp_mma_commit(&empty[stage]);
                     if (++stage == WSTAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
                 if (!ok) break;
-                mma_commit(&tfull[acc]);
+                warp_mma_commit(&tfull[acc]);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
             if (any) {  // every issued MMA has finished before TMEM is released
-                mma_commit(drain);
+                warp_mma_commit(drain);
                 volatile int never = 0;
-                mbar_wait(drain, 0, &never, p.status);
+                mbar_wait_warp(drain, 0, &never, p.status);
             }
         }
     } else {
