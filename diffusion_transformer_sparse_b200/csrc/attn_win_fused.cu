@@ -189,7 +189,8 @@ __global__ void __maxnreg__(168)
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (the whole warp runs the loop with warp-uniform operands; lane 0 issues)
+        {
             constexpr uint32_t id_s = idesc_bf16(BQ, BQ);
             constexpr uint32_t id_o = idesc_bf16(BQ, 64, true);   // V columns 0..63
             constexpr uint32_t id_ob = idesc_bf16(BQ, 16, true);  // V columns 64..79
@@ -198,16 +199,16 @@ __global__ void __maxnreg__(168)
             bool ok = true, any = false;
             // S(j) = Q K^T, once O(j - 1) has been read out of the same columns
             auto issue_s = [&](int j) {
-                if (j >= 1 && !mbar_wait(o_free, (j - 1) & 1, abort, status, wns)) return false;
+                if (j >= 1 && !mbar_wait_warp(o_free, (j - 1) & 1, abort, status, wns)) return false;
                 fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + T_SO, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32), id_s,
+                    warp_mma_bf16(tmem + T_SO, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32), id_s,
                              kk > 0);
                 if (L::HAS_B)
-                    mma_bf16(tmem + T_SO, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
+                    warp_mma_bf16(tmem + T_SO, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
                              id_s, 1);
-                mma_commit(s_full);
+                warp_mma_commit(s_full);
                 return true;
             };
             // O(j) = P(j) V into S's columns (P from TMEM, written by the softmax)
@@ -215,25 +216,25 @@ __global__ void __maxnreg__(168)
                 fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < BQ / 16; ++ks) {
-                    mma_bf16_ts(tmem + T_SO, tmem + T_P + ks * 8,
+                    warp_mma_bf16_ts(tmem + T_SO, tmem + T_P + ks * 8,
                                 sdesc_sw128_mn(aV + ks * 2048, L::TILE_A), id_o, ks > 0);
                     if (L::HAS_B)
-                        mma_bf16_ts(tmem + T_SO + 64, tmem + T_P + ks * 8,
+                        warp_mma_bf16_ts(tmem + T_SO + 64, tmem + T_P + ks * 8,
                                     sdesc_sw32_mn(aV + L::TILE_A + ks * 512), id_ob, ks > 0);
                 }
-                mma_commit(o_full);
-                mma_commit(qkv_free);  // S and P V have read Q, K and V
+                warp_mma_commit(o_full);
+                warp_mma_commit(qkv_free);  // S and P V have read Q, K and V
             };
             int c = 0;
             for (int j = 0; j < J && ok; ++j) {
                 bool pv_done = j == 0;
                 if (j >= 1) {
                     // job j-1's projection is out of TMEM (its Q, K, V in shared memory)
-                    if (!mbar_wait(drained, (j - 1) & 1, abort, status, wns) || !issue_s(j - 1)) break;
+                    if (!mbar_wait_warp(drained, (j - 1) & 1, abort, status, wns) || !issue_s(j - 1)) break;
                 }
                 for (int kb = 0; kb < KT; ++kb, ++c) {
                     const int s = c % NST;
-                    if (!mbar_wait(&full[s], (c / NST) & 1, abort, status, wns)) {
+                    if (!mbar_wait_warp(&full[s], (c / NST) & 1, abort, status, wns)) {
                         ok = false;
                         break;
                     }
@@ -241,31 +242,33 @@ __global__ void __maxnreg__(168)
                     const uint32_t aA = smem_u32(sm + s * L::STAGE), aB = aA + L::A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + T_ACC, sdesc_sw128(aA + kk * 32), sdesc_sw128(aB + kk * 32),
+                        warp_mma_bf16(tmem + T_ACC, sdesc_sw128(aA + kk * 32), sdesc_sw128(aB + kk * 32),
                                  id_acc, kb > 0 || kk > 0);
-                    mma_commit(&empty[s]);
+                    warp_mma_commit(&empty[s]);
                     any = true;
-                    // job j-1's P V as soon as its softmax is done
-                    if (!pv_done && mbar_test_wait(p_full, (j - 1) & 1)) {
+                    // job j-1's P V as soon as its softmax is done (lane 0's answer
+                    // for the whole warp, so that the warp stays converged)
+                    if (!pv_done &&
+                        __shfl_sync(0xffffffffu, (int)mbar_test_wait(p_full, (j - 1) & 1), 0)) {
                         issue_pv();
                         pv_done = true;
                     }
                 }
                 if (!ok) break;
-                mma_commit(acc_full);
+                warp_mma_commit(acc_full);
                 if (!pv_done) {
-                    if (!mbar_wait(p_full, (j - 1) & 1, abort, status, wns)) break;
+                    if (!mbar_wait_warp(p_full, (j - 1) & 1, abort, status, wns)) break;
                     issue_pv();
                 }
             }
             // the last job's attention
-            if (ok && J > 0 && mbar_wait(drained, (J - 1) & 1, abort, status, wns) && issue_s(J - 1) &&
-                mbar_wait(p_full, (J - 1) & 1, abort, status, wns))
+            if (ok && J > 0 && mbar_wait_warp(drained, (J - 1) & 1, abort, status, wns) && issue_s(J - 1) &&
+                mbar_wait_warp(p_full, (J - 1) & 1, abort, status, wns))
                 issue_pv();
             if (any) {  // every issued MMA has finished before TMEM is released
-                mma_commit(drain);
+                warp_mma_commit(drain);
                 volatile int never = 0;
-                mbar_wait(drain, 0, &never, status);
+                mbar_wait_warp(drain, 0, &never, status);
             }
         }
     } else {

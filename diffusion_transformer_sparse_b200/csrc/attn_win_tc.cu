@@ -199,7 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (the whole warp runs the loop with warp-uniform operands; lane 0 issues)
+        {
             constexpr uint32_t idesc_s = idesc_bf16(BQ, BQ);
             constexpr uint32_t idesc_o = idesc_bf16(BQ, 64, true);   // V columns 0..63
             constexpr uint32_t idesc_ob = idesc_bf16(BQ, 16, true);  // V columns 64..79
@@ -207,18 +208,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             // S(k) into TMEM slot k % 2 (after P V(k - 2), issued earlier, has read P(k - 2))
             auto issue_s = [&](int k) {
                 const int bf = k % NBUF, g = k & 1;
-                if (!mbar_wait(&qk_full[bf], (k / NBUF) & 1, abort, status, sc.wait_ns)) return false;
+                if (!mbar_wait_warp(&qk_full[bf], (k / NBUF) & 1, abort, status, sc.wait_ns)) return false;
                 fence_after_sync();
                 const uint32_t aQ = smem_u32(sm + bf * L::BUF);
                 const uint32_t aK = aQ + L::TILE;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(tmem + g * 256, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
+                    warp_mma_bf16(tmem + g * 256, sdesc_sw128(aQ + kk * 32), sdesc_sw128(aK + kk * 32),
                              idesc_s, kk > 0);
                 if (L::HAS_B)
-                    mma_bf16(tmem + g * 256, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
+                    warp_mma_bf16(tmem + g * 256, sdesc_sw32(aQ + L::TILE_A), sdesc_sw32(aK + L::TILE_A),
                              idesc_s, 1);
-                mma_commit(&s_full[g]);
+                warp_mma_commit(&s_full[g]);
                 any = true;
                 return true;
             };
@@ -226,23 +227,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             // unit k - 2 has been read out of the slot's O columns
             auto issue_pv = [&](int k) {
                 const int bf = k % NBUF, g = k & 1;
-                if (!mbar_wait(&p_full[g], (k >> 1) & 1, abort, status, sc.wait_ns)) return false;
-                if (!mbar_wait(&o_free[g], ((k >> 1) & 1) ^ 1, abort, status, sc.wait_ns))
+                if (!mbar_wait_warp(&p_full[g], (k >> 1) & 1, abort, status, sc.wait_ns)) return false;
+                if (!mbar_wait_warp(&o_free[g], ((k >> 1) & 1) ^ 1, abort, status, sc.wait_ns))
                     return false;
-                if (!mbar_wait(&v_full[bf], (k / NBUF) & 1, abort, status, sc.wait_ns)) return false;
+                if (!mbar_wait_warp(&v_full[bf], (k / NBUF) & 1, abort, status, sc.wait_ns)) return false;
                 fence_after_sync();
                 const uint32_t aV = smem_u32(sm + bf * L::BUF + 2 * L::TILE);
                 const uint32_t tO = tmem + g * 256 + 128;
 #pragma unroll
                 for (int ks = 0; ks < BQ / 16; ++ks) {
-                    mma_bf16_ts(tO, tmem + g * 256 + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
+                    warp_mma_bf16_ts(tO, tmem + g * 256 + ks * 8, sdesc_sw128_mn(aV + ks * 2048, L::TILE_A),
                                 idesc_o, ks > 0);
                     if (L::HAS_B)
-                        mma_bf16_ts(tO + 64, tmem + g * 256 + ks * 8,
+                        warp_mma_bf16_ts(tO + 64, tmem + g * 256 + ks * 8,
                                     sdesc_sw32_mn(aV + L::TILE_A + ks * 512), idesc_ob, ks > 0);
                 }
-                mma_commit(&o_full[g]);
-                mma_commit(&buf_free[bf]);  // S and P V have read the unit's Q, K and V
+                warp_mma_commit(&o_full[g]);
+                warp_mma_commit(&buf_free[bf]);  // S and P V have read the unit's Q, K and V
                 return true;
             };
             if (nunits > 0) ok = issue_s(0);
@@ -252,9 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok && k + 2 < nunits) ok = issue_s(k + 2);
             }
             if (any) {  // every issued MMA has finished before TMEM is released
-                mma_commit(drain);
+                warp_mma_commit(drain);
                 volatile int never = 0;
-                mbar_wait(drain, 0, &never, status);
+                mbar_wait_warp(drain, 0, &never, status);
             }
         }
     } else if (warp >= 4) {
