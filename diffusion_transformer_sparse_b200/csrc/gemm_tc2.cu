@@ -134,33 +134,11 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
         : "memory");
 }
 
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                              uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrives once on `bar` in both CTAs of the pair when the pair's MMAs so far have completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(smem_u32(bar)),
-        "h"(static_cast<uint16_t>(3))
-        : "memory");
-}
-
-__device__ __forceinline__ void mma_commit_pair_local(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
 // The issuer runs as a whole converged warp (warp-uniform operands); lane 0
 // alone issues, under a predicate inside each instruction sequence.
+//
+// D (+)= A B^T on the CTA pair: M = 256, each CTA holding its 128 rows of A and
+// half of B's rows, the accumulator in each CTA's TMEM.
 __device__ __forceinline__ void warp_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                    uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -172,6 +150,7 @@ __device__ __forceinline__ void warp_mma_bf16_pair(uint32_t d_tmem, uint64_t a_d
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Arrives on `bar` in both CTAs of the pair once the pair's MMAs so far have completed.
 __device__ __forceinline__ void warp_mma_commit_pair(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"
@@ -182,6 +161,7 @@ __device__ __forceinline__ void warp_mma_commit_pair(uint64_t *bar) {
         "h"(static_cast<uint16_t>(3))
         : "memory");
 }
+// The same, arriving on this CTA's `bar` only.
 __device__ __forceinline__ void warp_mma_commit_pair_local(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"

@@ -252,40 +252,12 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// MMA issue for an issuer that runs as a whole converged warp: every lane computes
+// the (warp-uniform) operands and lane 0 alone issues, under a predicate inside the
+// instruction sequence rather than a branch around it (a loop run by one lane
+// issued far slower than the tensor core ran it).
+//
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate, one CTA.
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                         uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem]^T: A (bf16, K-major) read from tensor memory,
-// lane m = row m, two K elements per 32-bit column (even element in the low half).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrives once on `bar` when every tcgen05.mma this thread issued so far has completed.
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
-// The same three instructions for an issuer that runs as a whole converged warp:
-// every lane computes the (warp-uniform) operands and lane 0 alone issues, under a
-// predicate inside the instruction sequence rather than a branch around it.
 __device__ __forceinline__ void warp_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                               uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -298,6 +270,8 @@ __device__ __forceinline__ void warp_mma_bf16(uint32_t d_tmem, uint64_t a_desc, 
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (bf16, K-major) read from tensor memory,
+// lane m = row m, two K elements per 32-bit column (even element in the low half).
 __device__ __forceinline__ void warp_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                                  uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -310,6 +284,7 @@ __device__ __forceinline__ void warp_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tme
         : "memory");
 }
 
+// Arrives once on `bar` when every tcgen05.mma lane 0 issued so far has completed.
 __device__ __forceinline__ void warp_mma_commit(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"
