@@ -63,7 +63,10 @@ def l2_policy(w):
 # launch on the long video) and profiles/gemm_tc2_t2i_2048px_qkv_and_oproj.md
 # (59.4 MB at 2048 px) predate the whole-warp MMA issuer of gemm_tc2, so they are
 # not used here.
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/gemm_tc2_dram_traffic_t2i_1024px.md: one step's nine launches, per launch
+    "t2i_1024px_64x64_b4": 59.7e6,
+}
 
 
 def load_peaks():
